@@ -1,0 +1,676 @@
+"""Pins of the fp64 oracle against what the pages and the mathematics fix.
+
+Each test checks the oracle against something other than itself: values the
+pages print for their worked examples (tests/golden/), closed forms, brute
+force over tiny inputs, library routines (numpy, torch SDPA, cuRAND's host
+Philox generator) and statistical laws (chi-square, the expected acceptance
+length).  None of these needs a GPU.
+"""
+import ctypes
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from conftest import read_golden
+from medusa_tree_speculative_heads_b200 import inputs as I
+
+
+# ----------------------------------------------------------------------------
+# tree structure and mask
+# ----------------------------------------------------------------------------
+
+def _ints(s):
+    return [int(x) for x in s.split()]
+
+
+def test_mask_guide_5_candidates(orc):
+    g = read_golden("guide_tree_mask_5.txt")
+    par = _ints(g["parents"])
+    expect = np.array([[0 if x == "0" else 1 for x in row.split()] for row in g["mask"]])
+    allowed = orc.tree_mask(par)
+    # the page prints the additive form: 0 = visible, -inf = blocked
+    assert np.array_equal(allowed, (expect == 0).astype(np.uint8))
+
+
+def test_mask_guide_paths_demo(orc):
+    g = read_golden("guide_paths_demo.txt")
+    paths = [[int(t) for t in p.split(",")] for p in g["paths"].split("|")]
+    nodes = _ints(g["nodes"])
+    par = _ints(g["parents"])
+    expect = np.array([_ints(r) for r in g["mask"]], dtype=np.uint8)
+    # the page's construction: unique nodes in first-appearance order; each
+    # path position sees that path's prefix up to itself
+    order = []
+    for p in paths:
+        for n in p:
+            if n not in order:
+                order.append(n)
+    assert order == nodes
+    via_paths = np.zeros((len(order), len(order)), np.uint8)
+    for p in paths:
+        for i, n in enumerate(p):
+            for a in p[: i + 1]:
+                via_paths[order.index(n), order.index(a)] = 1
+    assert np.array_equal(via_paths, expect)
+    assert np.array_equal(orc.tree_mask(par), expect)
+
+
+def test_mask_mtp_parent_array_forest(orc):
+    g = read_golden("mtp_parent_array.txt")
+    par = _ints(g["parents"])
+    m = orc.tree_mask(par)
+    for row in g["attends"]:
+        i, rest = row.split(":")
+        assert sorted(np.nonzero(m[int(i)])[0].tolist()) == _ints(rest)
+    # a forest is not a single-rooted tree: the step's functions reject it
+    with pytest.raises(ValueError):
+        orc.tree_shape(par)
+
+
+def test_mask_rejects_bad_parents(orc):
+    for bad in ([-1, 1], [-1, 0, 5], [-1, -2]):
+        with pytest.raises(ValueError):
+            orc.tree_mask(bad)
+    for bad in ([0], [-1, 0, -1], [-1, 2, 0]):
+        with pytest.raises(ValueError):
+            orc.tree_shape(bad)
+
+
+def test_tree_shape_hand_example(orc):
+    # root 0; children 1,2,3; 4 under 2; 5, 6 under 1 (index order != BFS of
+    # a product tree, still topologically ordered)
+    par = [-1, 0, 0, 0, 2, 1, 1]
+    depth, rank = orc.tree_shape(par)
+    assert depth.tolist() == [1, 2, 2, 2, 3, 3, 3]
+    assert rank.tolist() == [0, 0, 1, 2, 0, 0, 1]
+
+
+@pytest.mark.parametrize("s,nodes,leaves", [((2, 2), 7, 4), ((4, 2, 2), 29, 16), ((4, 4, 2, 2), 117, 64)])
+def test_product_tree_counts(orc, s, nodes, leaves):
+    # [MTP] "Tree-Structured Attention Verification": depth 4 with branching
+    # (4,2,2) gives 16 candidate trajectories; the 117-node tree of the
+    # workloads is 1 + 4 + 16 + 32 + 64 with 64 leaf paths
+    par = orc.product_tree(s)
+    assert len(par) == nodes
+    has_child = set(par[1:].tolist())
+    assert sum(1 for i in range(nodes) if i not in has_child) == leaves
+    assert par.tolist() == I.product_tree_parents(s)
+    depth, rank = orc.tree_shape(par)
+    assert depth.max() == len(s) + 1
+    for k, sk in enumerate(s):
+        assert rank[depth == k + 2].max() == sk - 1
+
+
+def test_product_tree_matches_path_enumeration(orc):
+    # brute force: enumerate the Cartesian product of rank tuples; every path
+    # prefix is a node; compare parent relations as sets of prefixes
+    s = (3, 2, 2)
+    import itertools
+    par = orc.product_tree(s)
+    depth, rank = orc.tree_shape(par)
+
+    def prefix_of(i):
+        out = []
+        while par[i] != -1:
+            out.append(int(rank[i]))
+            i = par[i]
+        return tuple(reversed(out))
+
+    got = sorted(prefix_of(i) for i in range(len(par)))
+    want = sorted(set(p[:k] for p in itertools.product(*[range(x) for x in s]) for k in range(len(s) + 1)))
+    assert got == want
+
+
+def test_random_tree_generator_is_valid(orc):
+    w = I.WORKLOADS["stoch_b64"]
+    par = I.workload_tree(w)
+    assert len(par) == 32
+    depth, rank = orc.tree_shape(par)
+    assert depth.max() <= 4
+    assert max(np.bincount(np.array(par[1:]), minlength=32)) <= 6
+    assert all(par[i] <= par[i + 1] for i in range(1, 31))   # breadth-first numbering
+
+
+# ----------------------------------------------------------------------------
+# Medusa heads
+# ----------------------------------------------------------------------------
+
+def _floats(s):
+    return [float(x) for x in s.split()]
+
+
+def _mat(s):
+    return [[float(x) for x in row.split()] for row in s.split("|")]
+
+
+def test_heads_hand_d4_case_a(orc):
+    g = read_golden("guide_head_d4.txt")
+    h = torch.tensor([_floats(g["h"])], dtype=torch.float32)
+    W_res = torch.zeros((1, 4, 4), dtype=torch.float32)
+    W_head = torch.tensor([_mat(g["W_head"])], dtype=torch.float32)
+    r = orc.heads(h, W_res, W_head)
+    np.testing.assert_array_equal(r["hk"][0, 0], _floats(g["A_hk"]))
+    np.testing.assert_array_equal(r["logits"][0, 0], _floats(g["A_logits"]))
+    np.testing.assert_allclose(r["probs"][0, 0], _floats(g["A_probs"]), rtol=0, atol=1e-15)
+    assert orc.topk(r["logits"][0, 0], 2).tolist() == _ints(g["A_top2"])
+
+
+def test_heads_hand_d4_case_b_silu_ln3(orc):
+    g = read_golden("guide_head_d4.txt")
+    h = torch.tensor([_floats(g["h"])], dtype=torch.float32)
+    W_res = torch.zeros((1, 4, 4), dtype=torch.float32)
+    W_res[0, 0, 0] = math.log(3.0)          # z = (ln 3, 0, 0, 0) up to fp32 rounding of ln 3
+    W_head = torch.tensor([_mat(g["W_head"])], dtype=torch.float32)
+    r = orc.heads(h, W_res, W_head)
+    # fp32(ln 3) differs from ln 3 by < 6e-8; dSiLU/dz < 1 there
+    np.testing.assert_allclose(r["hk"][0, 0], _floats(g["B_hk"]), rtol=0, atol=1e-7)
+    np.testing.assert_allclose(r["logits"][0, 0], _floats(g["B_logits"]), rtol=0, atol=1e-7)
+
+
+def test_heads_silu_limits(orc):
+    # SiLU(z) -> z for z >> 0 and -> 0 for z << 0
+    h = torch.tensor([[1.0, 0.0]], dtype=torch.float32)
+    W_res = torch.tensor([[[1000.0, 0.0], [-1000.0, 0.0]]], dtype=torch.float32)
+    W_head = torch.eye(2, dtype=torch.float32)[None]
+    r = orc.heads(h, W_res, W_head)
+    assert r["hk"][0, 0].tolist() == [1001.0, 0.0]
+
+
+def test_heads_vs_numpy_matmul_and_softmax_sum(orc):
+    # random small case against numpy's fp64 matmul (a library routine) with
+    # the head formula; softmax rows sum to 1
+    g = torch.Generator().manual_seed(11)
+    B, d, V, K = 3, 16, 50, 2
+    h = torch.randn((B, d), generator=g)
+    W_res = torch.randn((K, d, d), generator=g) / 4
+    W_head = torch.randn((K, V, d), generator=g) / 4
+    r = orc.heads(h, W_res, W_head)
+    hn, Wr, Wh = h.double().numpy(), W_res.double().numpy(), W_head.double().numpy()
+    for k in range(K):
+        z = hn @ Wr[k].T
+        hk = z / (1 + np.exp(-z)) + hn
+        lg = hk @ Wh[k].T
+        np.testing.assert_allclose(r["hk"][:, k], hk, rtol=1e-13, atol=1e-13)
+        np.testing.assert_allclose(r["logits"][:, k], lg, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(r["probs"].sum(-1), 1.0, rtol=0, atol=1e-12)
+    # bf16 inputs are widened exactly: same result as the fp32 copy of them
+    rb = orc.heads(h.bfloat16(), W_res.bfloat16(), W_head.bfloat16())
+    rf = orc.heads(h.bfloat16().float(), W_res.bfloat16().float(), W_head.bfloat16().float())
+    np.testing.assert_array_equal(rb["logits"], rf["logits"])
+
+
+def test_heads_subset_selection(orc):
+    g = torch.Generator().manual_seed(12)
+    B, d, V, K = 2, 8, 20, 3
+    h = torch.randn((B, d), generator=g)
+    W_res = torch.randn((K, d, d), generator=g)
+    W_head = torch.randn((K, V, d), generator=g)
+    full = orc.heads(h, W_res, W_head)
+    one = orc.heads(h, W_res, W_head, b_only=1, k_only=2)
+    np.testing.assert_array_equal(one["logits"][1, 2], full["logits"][1, 2])
+    assert np.isnan(one["logits"][0]).all() and np.isnan(one["logits"][1, :2]).all()
+
+
+def test_topk_equals_stable_sort(orc):
+    rng = np.random.default_rng(5)
+    for trial in range(200):
+        n = int(rng.integers(1, 40))
+        x = rng.integers(-3, 4, size=n).astype(np.float64)   # many ties
+        if trial % 5 == 0:
+            x[rng.integers(0, n)] = np.nan
+        s = int(rng.integers(1, 9))
+        got = orc.topk(x, s)
+        keys = np.where(np.isnan(x), np.inf, -x)
+        want = np.argsort(keys, kind="stable")
+        want = [int(i) for i in want if not np.isnan(x[i])][:s]
+        want += [-1] * (s - len(want))
+        assert got.tolist() == want
+
+
+def test_tree_fill_product_tree(orc):
+    par = orc.product_tree((2, 3))
+    B, K, S = 2, 2, 8
+    ti = np.arange(B * K * S, dtype=np.int32).reshape(B, K, S) + 1000
+    tp = np.random.default_rng(0).random((B, K, S))
+    tok, nq = orc.tree_fill(par, [7, 9], ti, tp)
+    # root, then head-1 entries 0..1, then for each depth-2 node head-2 entries 0..2
+    assert tok[0].tolist() == [7, 1000, 1001] + [1008, 1009, 1010] * 2
+    assert tok[1].tolist() == [9, 1016, 1017] + [1024, 1025, 1026] * 2
+    assert nq[0, 0] == 1.0 and nq[1, 4] == tp[1, 1, 1]
+    with pytest.raises(ValueError):
+        orc.tree_fill(orc.product_tree((2, 2, 2)), [1, 1], ti, tp)   # deeper than K+1
+
+
+# ----------------------------------------------------------------------------
+# tree attention
+# ----------------------------------------------------------------------------
+
+def _sdpa_reference(q, kt, vt, kc, vc, pl, allowed_tree, scale=None):
+    """torch SDPA in fp64 (a library routine) with an explicit dense boolean
+    mask over [prefix ; tree] keys; kv heads repeated for GQA."""
+    B, T, Hq, D = q.shape
+    Hkv = kt.shape[2]
+    G = Hq // Hkv
+    outs = []
+    for b in range(B):
+        S = int(pl[b])
+        K_ = torch.cat([kc[b, :, :S].double(), kt[b].double().permute(1, 0, 2)], dim=1)  # [Hkv, S+T, D]
+        V_ = torch.cat([vc[b, :, :S].double(), vt[b].double().permute(1, 0, 2)], dim=1)
+        K_ = K_.repeat_interleave(G, dim=0)
+        V_ = V_.repeat_interleave(G, dim=0)
+        Q_ = q[b].double().permute(1, 0, 2)                                              # [Hq, T, D]
+        mask = torch.cat([torch.ones((T, S), dtype=torch.bool), torch.as_tensor(allowed_tree, dtype=torch.bool)],
+                         dim=1)
+        o = torch.nn.functional.scaled_dot_product_attention(Q_, K_, V_, attn_mask=mask, scale=scale)
+        outs.append(o.permute(1, 0, 2))                                                  # [T, Hq, D]
+    return torch.stack(outs).numpy()
+
+
+def _attn_case(B, T, Hq, Hkv, D, S_max, pl, seed):
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn((B, T, Hq, D), generator=g)
+    kt = torch.randn((B, T, Hkv, D), generator=g)
+    vt = torch.randn((B, T, Hkv, D), generator=g)
+    kc = torch.randn((B, Hkv, S_max, D), generator=g)
+    vc = torch.randn((B, Hkv, S_max, D), generator=g)
+    return q, kt, vt, kc, vc, torch.tensor(pl, dtype=torch.int32)
+
+
+def test_attention_chain_tree_is_causal_attention(orc):
+    # a chain tree (parent i-1) must equal plain causal attention over
+    # prefix + chain, written here with numpy from the softmax definition
+    B, T, Hq, Hkv, D, S_max = 2, 5, 4, 2, 8, 12
+    q, kt, vt, kc, vc, pl = _attn_case(B, T, Hq, Hkv, D, S_max, [7, 0], 1)
+    par = [-1] + list(range(T - 1))
+    out, lse = orc.tree_attention(q, kt, vt, kc, vc, pl, par)
+    out = out.reshape(B, T, Hq, D)
+    for b in range(B):
+        S = int(pl[b])
+        for h in range(Hq):
+            g_ = h // (Hq // Hkv)
+            keys = np.concatenate([kc[b, g_, :S].double().numpy(), kt[b, :, g_].double().numpy()])
+            vals = np.concatenate([vc[b, g_, :S].double().numpy(), vt[b, :, g_].double().numpy()])
+            for i in range(T):
+                n = S + i + 1                                   # causal: prefix and chain up to i
+                sc = keys[:n] @ q[b, i, h].double().numpy() / math.sqrt(D)
+                w = np.exp(sc - sc.max())
+                np.testing.assert_allclose(out[b, i, h], (w / w.sum()) @ vals[:n], rtol=1e-12, atol=1e-12)
+                np.testing.assert_allclose(lse.reshape(B, T, Hq)[b, i, h], sc.max() + np.log(w.sum()),
+                                           rtol=1e-12, atol=1e-12)
+
+
+def test_attention_single_node_is_decode_attention(orc):
+    B, T, Hq, Hkv, D, S_max = 1, 1, 2, 1, 16, 40
+    q, kt, vt, kc, vc, pl = _attn_case(B, T, Hq, Hkv, D, S_max, [33], 2)
+    out, _ = orc.tree_attention(q, kt, vt, kc, vc, pl, [-1])
+    ref = _sdpa_reference(q, kt, vt, kc, vc, pl, np.ones((1, 1)))
+    np.testing.assert_allclose(out.reshape(ref.shape), ref, rtol=1e-12, atol=1e-12)
+
+
+def test_attention_product_tree_vs_sdpa_with_path_mask(orc):
+    # mask built from the candidate paths (prefixes of rank tuples), not from
+    # parent pointers; GQA with 3 q-heads per kv-head; custom scale
+    s = (3, 2)
+    par = orc.product_tree(s)
+    T = len(par)
+    depth, rank = orc.tree_shape(par)
+    B, Hq, Hkv, D, S_max = 2, 6, 2, 8, 20
+    q, kt, vt, kc, vc, pl = _attn_case(B, T, Hq, Hkv, D, S_max, [20, 3], 3)
+
+    def tuple_of(i):
+        t = []
+        while par[i] != -1:
+            t.append(int(rank[i]))
+            i = par[i]
+        return tuple(reversed(t))
+
+    tuples = [tuple_of(i) for i in range(T)]
+    allowed = np.array([[1 if tuples[i][: len(tuples[j])] == tuples[j] else 0 for j in range(T)] for i in range(T)])
+    out, _ = orc.tree_attention(q, kt, vt, kc, vc, pl, par, scale=0.3)
+    ref = _sdpa_reference(q, kt, vt, kc, vc, pl, allowed, scale=0.3)
+    np.testing.assert_allclose(out.reshape(ref.shape), ref, rtol=1e-12, atol=1e-12)
+
+
+def test_attention_row_subset_matches_full(orc):
+    par = orc.product_tree((2, 2))
+    B, T, Hq, Hkv, D, S_max = 2, 7, 4, 4, 8, 10
+    q, kt, vt, kc, vc, pl = _attn_case(B, T, Hq, Hkv, D, S_max, [10, 5], 4)
+    full, lse = orc.tree_attention(q, kt, vt, kc, vc, pl, par)
+    rows = np.array([[1, 6, 3], [0, 0, 0], [1, 2, 1]])
+    sub, lsub = orc.tree_attention(q, kt, vt, kc, vc, pl, par, rows=rows)
+    for r, (b, i, h) in enumerate(rows):
+        n = (b * T + i) * Hq + h
+        np.testing.assert_array_equal(sub[r], full[n])
+        assert lsub[r] == lse[n]
+
+
+# ----------------------------------------------------------------------------
+# greedy verification
+# ----------------------------------------------------------------------------
+
+def _brute_force_greedy(logits, tok, par):
+    """Every root-to-leaf path in leaf order; the longest matched prefix wins,
+    a strictly longer one replacing it (first found wins ties)."""
+    T = len(par)
+    pred = [int(np.argmax(logits[u])) for u in range(T)]   # numpy: first maximum
+    children = I.tree_children(par)
+    leaves = [i for i in range(T) if not children[i]]
+    best = [0]
+    for leaf in leaves:
+        path = []
+        cur = leaf
+        while cur != -1:
+            path.append(cur)
+            cur = par[cur]
+        path.reverse()
+        ok = [0]
+        for a, c in zip(path[:-1], path[1:]):
+            if tok[c] != pred[a]:
+                break
+            ok.append(c)
+        if len(ok) > len(best):
+            best = ok
+    return best, pred[best[-1]]
+
+
+def test_greedy_vs_brute_force(orc):
+    rng = np.random.default_rng(7)
+    par = orc.product_tree((3, 2, 2))
+    T, V = len(par), 12
+    children = I.tree_children(par.tolist())
+    for trial in range(300):
+        logits = rng.standard_normal((1, T, V)).astype(np.float32)
+        tok = np.zeros((1, T), np.int32)
+        for u in range(T):
+            if children[u]:
+                picks = rng.choice(V, size=len(children[u]), replace=False)
+                tok[0, children[u]] = picks
+        # force many matches
+        for u in range(T):
+            if children[u] and rng.random() < 0.7:
+                c = children[u][rng.integers(len(children[u]))]
+                logits[0, u, tok[0, c]] = 10.0
+        path, ln, bonus = orc.verify_greedy(torch.from_numpy(logits), tok, par, max_path=4)
+        want, wb = _brute_force_greedy(logits[0], tok[0], par.tolist())
+        assert path[0, : ln[0]].tolist() == want
+        assert bonus[0] == wb
+        assert (path[0, ln[0]:] == -1).all()
+
+
+def test_greedy_draft_equals_target(orc):
+    # every node's first child carries the target's prediction at its parent:
+    # the whole first-child chain is accepted, bonus = prediction at its end
+    par = orc.product_tree((4, 4, 2, 2))
+    T, V = len(par), 64
+    children = I.tree_children(par.tolist())
+    rng = np.random.default_rng(8)
+    logits = rng.standard_normal((2, T, V)).astype(np.float32)
+    tok = np.zeros((2, T), np.int32)
+    for b in range(2):
+        for u in range(T):
+            if children[u]:
+                am = int(np.argmax(logits[b, u]))
+                others = [x for x in range(V) if x != am]
+                tok[b, children[u]] = [am] + list(rng.choice(others, len(children[u]) - 1, replace=False))
+    path, ln, bonus = orc.verify_greedy(torch.from_numpy(logits), tok, par, max_path=5)
+    chain = [0]
+    while children[chain[-1]]:
+        chain.append(children[chain[-1]][0])
+    for b in range(2):
+        assert ln[b] == 5 and path[b].tolist() == chain
+        assert bonus[b] == int(np.argmax(logits[b, chain[-1]]))
+
+
+def test_greedy_argmax_ties_lowest_index(orc):
+    logits = torch.zeros((1, 3, 8), dtype=torch.bfloat16)
+    logits[0, 0, 5] = 2.0
+    logits[0, 0, 3] = 2.0       # tie: index 3 wins
+    logits[0, 1, :] = float("nan")
+    logits[0, 1, 6] = 1.0       # NaN never wins
+    par = [-1, 0, 1]
+    path, ln, bonus = orc.verify_greedy(logits, [[0, 3, 6]], par, max_path=3)
+    assert ln[0] == 3 and path[0].tolist() == [0, 1, 2] and bonus[0] == 0   # row 2 all zero -> index 0
+    path, ln, bonus = orc.verify_greedy(logits, [[0, 5, 6]], par, max_path=3)
+    assert ln[0] == 1 and bonus[0] == 3
+
+
+def test_greedy_mtp_engine_demo_longest_path(orc):
+    # The page's engine uses a fixed score threshold as its acceptance test;
+    # reproduce the same accepted set with the greedy rule (a matching child
+    # token for every passing node, under a virtual root joining the two
+    # roots) and check the committed path and count the page prints.
+    g = read_golden("mtp_engine_demo.txt")
+    par0 = _ints(g["parents"])
+    scores = _floats(g["scores"])
+    thr = float(g["threshold"])
+    n = len(par0)
+    par = [-1] + [p + 1 for p in par0]          # node i -> i+1; roots hang under 0
+    T, V = n + 1, 32
+    tok = np.zeros((1, T), np.int32)
+    logits = torch.zeros((1, T, V))
+    children = I.tree_children(par)
+    for u in range(T):
+        kids = children[u]
+        passing = [c for c in kids if scores[c - 1] >= thr]
+        # passing siblings share the parent's predicted token; failing ones differ
+        pred = 1 + u
+        logits[0, u, pred] = 5.0
+        for j, c in enumerate(kids):
+            tok[0, c] = pred if c in passing else 20 + j
+    path, ln, bonus = orc.verify_greedy(logits, tok, par, max_path=T)
+    committed = [int(x) - 1 for x in path[0, 1: ln[0]]]
+    assert committed == _ints(g["committed_nodes"])
+    words = g["tokens"].split()
+    assert " ".join(words[i] for i in committed) == g["committed_tokens"]
+    assert len(committed) == int(g["count"])
+    assert round((len(committed) + 1) / (1 + float(g["overhead"])), 2) == float(g["speedup"])
+
+
+@pytest.mark.parametrize("branching,pi,V,n_steps", [((2, 2), 0.6, 1024, 20000), ((4, 4, 2, 2), 0.6, 256, 6000),
+                                                    ((4, 4, 2, 2), 0.7, 256, 6000)])
+def test_greedy_expected_acceptance_length(orc, branching, pi, V, n_steps):
+    # [MTP] "Expected Acceptance Length": tau = 1 + sum_k prod_{j<=k} alpha_j.
+    # Boost model: at an accepted node with s children, with probability pi
+    # one child's token gets +10 on the node's row (so it is the argmax);
+    # otherwise the argmax of i.i.d. N(0,1) logits is uniform over V and hits
+    # one of the s distinct child tokens with probability s/V.  So depth j is
+    # accepted with alpha_j = pi + (1 - pi) s_j / V.
+    par = orc.product_tree(branching)
+    T, K = len(par), len(branching)
+    children = I.tree_children(par.tolist())
+    rng = np.random.default_rng(99)
+    lens = []
+    chunk = 1000
+    for c0 in range(0, n_steps, chunk):
+        B = min(chunk, n_steps - c0)
+        logits = rng.standard_normal((B, T, V)).astype(np.float32)
+        tok = np.zeros((B, T), np.int32)
+        for u in range(T):
+            if children[u]:
+                m = len(children[u])
+                start = rng.integers(0, V - m + 1, size=B)
+                tok[:, children[u]] = start[:, None] + np.arange(m)[None, :]
+                hit = rng.random(B) < pi
+                which = rng.integers(0, m, size=B)
+                bb = np.nonzero(hit)[0]
+                logits[bb, u, tok[bb, np.array(children[u])[which[bb]]]] += 10.0
+        _, ln, _ = orc.verify_greedy(torch.from_numpy(logits), tok, par, max_path=K + 1)
+        lens.append(ln)
+    lens = np.concatenate(lens).astype(np.float64)
+    alpha = [pi + (1 - pi) * s / V for s in branching]
+    tau = 1 + sum(float(np.prod(alpha[:k])) for k in range(1, K + 1))
+    se = lens.std() / math.sqrt(len(lens))
+    assert abs(lens.mean() - tau) < 4 * se, (lens.mean(), tau, se)
+
+
+# ----------------------------------------------------------------------------
+# Philox and stochastic verification
+# ----------------------------------------------------------------------------
+
+def test_philox_known_answers(orc):
+    g = read_golden("philox4x32_10_kat.txt")
+    for row in g["_rows"]:
+        lhs, rhs = row.split("->")
+        w = [int(x, 16) for x in lhs.split()]
+        want = [int(x, 16) for x in rhs.split()]
+        assert orc.philox4x32_10(w[:4], w[4:6]).tolist() == want
+
+
+def test_philox_vs_curand_host_generator(orc):
+    # cuRAND's host Philox4x32-10 generator with seed s emits, as its n-th
+    # 4-word block, the block of counter (0, 0, n, 0) under key
+    # (s low word, s high word)
+    import os
+    path = "/usr/local/cuda/lib64/libcurand.so"
+    if not os.path.exists(path):
+        pytest.skip("libcurand not installed")
+    lib = ctypes.CDLL(path)
+    for seed in (0, 0x0123456789ABCDEF, 2**64 - 1):
+        gen = ctypes.c_void_p()
+        assert lib.curandCreateGeneratorHost(ctypes.byref(gen), 161) == 0
+        assert lib.curandSetPseudoRandomGeneratorSeed(gen, ctypes.c_ulonglong(seed)) == 0
+        n = 4 * 40
+        buf = (ctypes.c_uint32 * n)()
+        assert lib.curandGenerate(gen, buf, ctypes.c_size_t(n)) == 0
+        lib.curandDestroyGenerator(gen)
+        got = np.array(buf[:], dtype=np.uint32).reshape(-1, 4)
+        key = [seed & 0xFFFFFFFF, seed >> 32]
+        for c in range(got.shape[0]):
+            assert orc.philox4x32_10([0, 0, c, 0], key).tolist() == got[c].tolist()
+
+
+def test_residual_normalises_and_closed_form(orc):
+    rng = np.random.default_rng(3)
+    for _ in range(50):
+        V = int(rng.integers(2, 300))
+        P = rng.dirichlet(np.ones(V))
+        Q = rng.dirichlet(np.ones(V)).astype(np.float32)
+        out, W, S = orc.residual(P, Q)
+        assert S == int(W.sum()) and S > 0
+        assert abs(out.sum() - 1.0) < 1e-12
+        r = np.maximum(0.0, P - Q.astype(np.float64))
+        np.testing.assert_allclose(out, r / r.sum(), rtol=0, atol=V * 2.0 ** -31)
+    # P <= Q everywhere: the residual is empty and P is kept
+    P = np.array([0.25, 0.25, 0.5])
+    out, W, S = orc.residual(P, np.array([0.25, 0.25, 0.5], np.float32))
+    assert S == 0 and out.tolist() == P.tolist()
+
+
+def _chi2_pvalue(counts, probs):
+    from scipy.stats import chisquare
+    n = counts.sum()
+    probs = np.asarray(probs, np.float64)
+    assert (counts[probs == 0] == 0).all()          # impossible outcomes never occur
+    keep = probs > 0
+    return chisquare(counts[keep], probs[keep] / probs[keep].sum() * n).pvalue
+
+
+P8 = np.array([0.30, 0.05, 0.15, 0.02, 0.18, 0.10, 0.12, 0.08], np.float32)
+Q8 = np.array([0.10, 0.25, 0.05, 0.20, 0.10, 0.05, 0.15, 0.10], np.float32)
+
+
+@pytest.mark.parametrize("n_children", [1, 3])
+def test_stochastic_first_token_follows_target(orc, n_children):
+    # [SPEC] "The Acceptance Sampling Rule (Zero Distributional Drift)": the
+    # emitted token follows P_target.  Children are drawn i.i.d. from the
+    # draft; over 10^6 trials the first emitted token must match p (root row)
+    # and, when the first child was accepted, the second must match that
+    # child's row.
+    N = 1_000_000
+    T, V = 1 + n_children, 8
+    par = [-1] + [0] * n_children
+    rng = np.random.default_rng(100 + n_children)
+    p_child = np.array([0.05, 0.4, 0.05, 0.1, 0.1, 0.1, 0.1, 0.1], np.float32)
+    p = np.empty((N, T, V), np.float32)
+    p[:, 0] = P8
+    p[:, 1:] = p_child
+    q = np.empty((N, T, V), np.float32)
+    q[:, :] = Q8
+    tok = np.zeros((N, T), np.int32)
+    tok[:, 1:] = rng.choice(V, size=(N, n_children), p=Q8.astype(np.float64) / Q8.sum())
+    path, ln, bonus, st = orc.verify_stochastic(p, q, tok, par, seed=1234, step=7, max_path=2)
+    assert st == 0
+    first = np.where(ln >= 2, tok[np.arange(N), np.maximum(path[:, 1], 0)], bonus)
+    assert _chi2_pvalue(np.bincount(first, minlength=V), P8.astype(np.float64)) > 1e-3
+    acc = ln >= 2
+    second = bonus[acc]                     # the child is a leaf: bonus from its row
+    assert _chi2_pvalue(np.bincount(second, minlength=V), p_child.astype(np.float64)) > 1e-3
+
+
+def test_stochastic_one_hot_draft_closed_form(orc):
+    # draft q = one-hot at x: P(accept) = p(x); on rejection the bonus follows
+    # p with x removed and renormalised
+    N, V, x = 400_000, 8, 2
+    par = [-1, 0]
+    p = np.broadcast_to(P8, (N, 2, V)).copy()
+    q = np.zeros((N, 2, V), np.float32)
+    q[:, :, x] = 1.0
+    tok = np.full((N, 2), x, np.int32)
+    path, ln, bonus, _ = orc.verify_stochastic(p, q, tok, par, seed=77, step=0, max_path=2)
+    acc = (ln == 2).mean()
+    assert abs(acc - P8[x]) < 4 * math.sqrt(P8[x] * (1 - P8[x]) / N)
+    rej = bonus[ln == 1]
+    assert (rej != x).all()
+    want = P8.astype(np.float64).copy()
+    want[x] = 0
+    want /= want.sum()
+    assert _chi2_pvalue(np.bincount(rej, minlength=V), want) > 1e-3
+
+
+def test_stochastic_draft_equals_target_accepts_all(orc):
+    # q = p: u * q(x) < p(x) whenever p(x) > 0, so every first child is taken
+    w = I.scaled(I.WORKLOADS["stoch_b64"], B=3, V=500)
+    par = I.workload_tree(w)
+    d = I.stochastic_inputs(w, par)
+    children = I.tree_children(par)
+    path, ln, bonus, _ = orc.verify_stochastic(d["p"], d["p"], d["node_tokens"], par, seed=5, step=1,
+                                               max_path=4)
+    chain = [0]
+    while children[chain[-1]]:
+        chain.append(children[chain[-1]][0])
+    for b in range(3):
+        ok = all(float(d["p"][b, a, int(d["node_tokens"][b, c])]) > 0 for a, c in zip(chain, chain[1:]))
+        assert ok
+        assert path[b, : ln[b]].tolist() == chain
+
+
+def test_stochastic_q_row_mapping(orc):
+    # q_row maps each node to a shared draft row (Medusa: one row per head)
+    w = I.scaled(I.WORKLOADS["stoch_b64"], B=2, V=300)
+    par = I.workload_tree(w)
+    d = I.stochastic_inputs(w, par)
+    depth, _ = orc.tree_shape(par)
+    K = int(depth.max())
+    q_rows = d["q"][:, :K].clone()
+    q_row = (depth - 1).astype(np.int32)
+    q_full = torch.stack([q_rows[:, int(r)] for r in q_row], dim=1)
+    a = orc.verify_stochastic(d["p"], q_rows, d["node_tokens"], par, 9, 3, 4, q_row=q_row)
+    b = orc.verify_stochastic(d["p"], q_full, d["node_tokens"], par, 9, 3, 4)
+    for x, y in zip(a[:3], b[:3]):
+        assert np.array_equal(x, y)
+
+
+# ----------------------------------------------------------------------------
+# commit
+# ----------------------------------------------------------------------------
+
+def test_kv_commit_exact_and_canaries(orc):
+    g = torch.Generator().manual_seed(21)
+    B, Hkv, S_max, D, T = 3, 2, 16, 4, 7
+    kc = torch.full((B, Hkv, S_max, D), -777.0).bfloat16()
+    vc = torch.full((B, Hkv, S_max, D), 555.0).bfloat16()
+    kt = torch.randn((B, T, Hkv, D), generator=g).bfloat16()
+    vt = torch.randn((B, T, Hkv, D), generator=g).bfloat16()
+    path = np.array([[0, 2, 5], [0, -1, -1], [0, 1, 4]], np.int32)
+    ln = np.array([3, 1, 3], np.int32)
+    pl = np.array([4, 0, 14], np.int32)          # sequence 2 would overflow
+    k2, v2, npl, st = orc.kv_commit(kc, vc, kt, vt, path, ln, pl)
+    assert npl.tolist() == [7, 1, 14] and st == 1
+    ek, ev = kc.clone(), vc.clone()
+    for b in range(2):
+        for t in range(ln[b]):
+            ek[b, :, pl[b] + t] = kt[b, path[b, t]]
+            ev[b, :, pl[b] + t] = vt[b, path[b, t]]
+    assert torch.equal(k2, ek) and torch.equal(v2, ev)
