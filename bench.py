@@ -1,0 +1,399 @@
+#!/usr/bin/env python
+"""Benchmark of one Medusa speculative decode step on B200.
+
+A step is the whole hot path over one batch: medusa_heads (residual block,
+LM-head projection, softmax statistics, top-8, tree fill) -> tree_attention
+(one layer) -> tree_verify (greedy) -> kv_commit, on the 8B-shaped workload
+(B=1, d=4096, V=128256, K=4 heads, top-s (4,4,2,2) = 117 nodes, 32/8 heads,
+head_dim 128, prefix 2048), bf16 with fp32 accumulation, synthetic seeded
+inputs and random weights.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mine|reference]
+
+Prints one JSON line (rank 0).  Multi-GPU runs (torchrun) are independent
+replicas, one per GPU: the step has no cross-sequence exchange.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = "Medusa verify steps/s (8B shape, 117-node tree); tree-attn HBM GB/s vs peak"
+UNIT = "steps/s"
+WORKLOAD = "llama8b"
+# DRAM bytes per launch of the heads stage from an ncu capture (sum over its
+# kernels); None until a capture of the current kernels exists.
+HEADS_DRAM_BYTES = None
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[j] for r in rows for j in range(4) if r[5 + j].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------
+# oracle timing (the CPU baseline / reference arm)
+# ----------------------------------------------------------------------------
+
+class OracleSample:
+    """A bounded sample of the step, run by the fp64 oracle on the host: the
+    residual block of every head, the LM-head rows of a `fraction` slice of
+    the vocabulary, the attention of a `fraction` of the query rows, greedy
+    verification over the full tree and the commit.  Inputs are drawn once
+    (not timed); run() returns (seconds, fraction of a full step's work)."""
+
+    def __init__(self, w, fraction: float, seed: int = 0):
+        import numpy as np
+
+        from medusa_tree_speculative_heads_b200 import inputs as I
+        self.w = w
+        self.parents = I.workload_tree(w)
+        T = len(self.parents)
+        self.Vs = max(8, int(round(w.V * fraction)))
+        self.ws = I.scaled(w, V=self.Vs)
+        self.hin = I.head_inputs(self.ws)
+        self.ain = I.attention_inputs(w, T)
+        n_rows = w.B * T * w.Hq
+        nr = max(1, int(round(n_rows * fraction)))
+        g = np.random.default_rng(seed)
+        rid = g.choice(n_rows, size=nr, replace=False)
+        self.rows = np.stack([rid // (T * w.Hq), (rid // w.Hq) % T, rid % w.Hq], axis=1)
+        # the residual block and verification/commit run whole; the LM head
+        # and attention (all but ~2% of the work) are sampled at `fraction`
+        lm = w.K * w.V * w.d
+        att = n_rows * (w.prefix + 5) * w.D * 2
+        res = w.K * w.d * w.d
+        self.frac = (res + lm * self.Vs / w.V + att * nr / n_rows) / (res + lm + att)
+        self.logits = None
+
+    def run(self):
+        import numpy as np
+
+        import oracle
+        from medusa_tree_speculative_heads_b200 import inputs as I
+        w, parents, hin, ain = self.w, self.parents, self.hin, self.ain
+        t0 = time.perf_counter()
+        ref = oracle.heads(hin["h"], hin["W_res"], hin["W_head"], want_hk=False)
+        otop = np.stack([np.stack([oracle.topk(ref["logits"][b, k], 8) for k in range(w.K)]) for b in range(w.B)])
+        otok, _ = oracle.tree_fill(parents, hin["root_token"], otop,
+                                   np.take_along_axis(ref["probs"], otop, axis=-1))
+        t1 = time.perf_counter()
+        if self.logits is None:   # the target model's logits: input generation, not timed
+            self.logits = I.boosted_target_logits(self.ws, parents, torch.from_numpy(otok))
+        t2 = time.perf_counter()
+        oracle.tree_attention(ain["q"], ain["k_tree"], ain["v_tree"], ain["k_cache"], ain["v_cache"],
+                              ain["prefix_len"], parents, rows=self.rows)
+        maxd = int(max(oracle.tree_shape(parents)[0]))
+        path, ln, _ = oracle.verify_greedy(self.logits, otok, parents, maxd)
+        oracle.kv_commit(ain["k_cache"], ain["v_cache"], ain["k_tree"], ain["v_tree"], path, ln, ain["prefix_len"])
+        t3 = time.perf_counter()
+        return (t1 - t0) + (t3 - t2), self.frac
+
+
+def run_reference(args, rank, world):
+    from medusa_tree_speculative_heads_b200 import inputs as I
+    if rank != 0:
+        return
+    w = I.WORKLOADS[args.workload]
+    import oracle
+    oracle.build()
+    sample = OracleSample(w, 1.0 / 64, seed=1)
+    for _ in range(args.warmup):
+        sample.run()
+    tot_t, tot_f = 0.0, 0.0
+    for _ in range(args.steps):
+        t, f = sample.run()
+        tot_t += t
+        tot_f += f
+    value = tot_f / tot_t
+    sample = (f"per step: fp64 oracle on the host, residual block of all {w.K} heads, LM-head rows of a 1/64 "
+              f"vocabulary slice, attention of 1/64 of the query rows, full greedy verify and commit; "
+              f"steps/s scaled by the sampled fraction of the step's work")
+    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 / value, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": config_dict(w, world),
+           "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+           "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+# ----------------------------------------------------------------------------
+# the CUDA path
+# ----------------------------------------------------------------------------
+
+def config_dict(w, world):
+    return {"workload": (f"{w.name}: B={w.B} d={w.d} V={w.V} K={w.K} heads, top-s {w.topk} -> 117-node tree, "
+                         f"{w.Hq}/{w.Hkv} heads head_dim {w.D}, prefix {w.prefix}, greedy verify, "
+                         f"match prob {w.match_prob}, one attention layer"),
+            "global_batch": w.B * world, "seq_len": w.prefix, "parallelism": f"replicas x{world}",
+            "l2": "inputs larger than L2: each step streams 4.34 GB of head weights through the 126 MB L2"}
+
+
+def launches_per_step(w, mode_greedy=True):
+    groups = (w.B + 7) // 8
+    heads = 1 + 2 * groups
+    attn = 2 if w.dtype == "bf16" else 1
+    verify = 2 if mode_greedy else 1
+    return heads + attn + verify + 1
+
+
+def run_mine(args, rank, world, local_rank):
+    import torch.distributed as dist
+
+    from medusa_tree_speculative_heads_b200 import build as build_mod
+    from medusa_tree_speculative_heads_b200 import inputs as I
+    from medusa_tree_speculative_heads_b200.api import MedusaStep
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    if rank == 0:
+        build_mod.build()
+    if world > 1:
+        dist.barrier()
+
+    w = I.WORKLOADS[args.workload]
+    parents = I.workload_tree(w)
+    T = len(parents)
+    hin = I.head_inputs(w, device="cuda")
+    ain = I.attention_inputs(w, T, device="cuda")
+    step = MedusaStep(B=w.B, d=w.d, V=w.V, K=w.K, Hq=w.Hq, Hkv=w.Hkv, D=w.D, S_max=w.S_max, parents=parents,
+                      dtype=w.torch_dtype, max_prefix=w.max_prefix, device=dev)
+    # the target model's logits (outside this path) are synthesised once from
+    # the tree the heads propose, with the workload's match probability
+    step.heads(hin["h"], hin["W_res"], hin["W_head"], hin["root_token"])
+    torch.cuda.synchronize()
+    logits = I.boosted_target_logits(w, parents, step.node_tokens.cpu(), device="cuda")
+    new_pl = torch.empty_like(ain["prefix_len"])
+
+    def run_step():
+        step.run(h=hin["h"], W_res=hin["W_res"], W_head=hin["W_head"], root_token=hin["root_token"], q=ain["q"],
+                 k_tree=ain["k_tree"], v_tree=ain["v_tree"], k_cache=ain["k_cache"], v_cache=ain["v_cache"],
+                 prefix_len=ain["prefix_len"], new_prefix_len=new_pl, target=logits)
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(max(args.warmup, 3)):
+        run_step()
+    torch.cuda.synchronize()
+
+    # ---- device-timed steps, with per-stage events ----
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record()
+    for i in range(K):
+        ev[i][0].record()
+        step.heads(hin["h"], hin["W_res"], hin["W_head"], hin["root_token"])
+        ev[i][1].record()
+        step.attention(ain["q"], ain["k_tree"], ain["v_tree"], ain["k_cache"], ain["v_cache"], ain["prefix_len"])
+        ev[i][2].record()
+        step.verify(logits)
+        ev[i][3].record()
+        step.commit(ain["k_cache"], ain["v_cache"], ain["k_tree"], ain["v_tree"], ain["prefix_len"], new_pl)
+        ev[i][4].record()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    t_local = e0.elapsed_time(e1) / 1000.0
+    t = max_over_ranks(t_local)
+    value = world * K / t
+    stage = [statistics.mean(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K)) / 1000.0 for j in range(4)]
+    assert int(step.status.item()) == 0, "device status set during the benchmark"
+    mean_len = float(step.accept_len.float().mean().item())
+
+    # ---- end to end through the public API with host buffers ----
+    names_in = ["h", "root_token", "q", "k_tree", "v_tree"]
+    host_in = {n: (hin if n in hin else ain)[n].cpu().pin_memory() for n in names_in}
+    host_in["target"] = logits.cpu().pin_memory()
+    dev_in = {n: torch.empty_like(host_in[n], device=dev) for n in host_in}
+    outs = [step.accept_path, step.accept_len, step.bonus, step.node_tokens]
+    host_out = [torch.empty_like(o, device="cpu").pin_memory() for o in outs]
+    h2d = sum(x.numel() * x.element_size() for x in host_in.values())
+    d2h = sum(x.numel() * x.element_size() for x in host_out)
+
+    def e2e_step():
+        for n in host_in:
+            dev_in[n].copy_(host_in[n], non_blocking=True)
+        step.run(h=dev_in["h"], W_res=hin["W_res"], W_head=hin["W_head"], root_token=dev_in["root_token"],
+                 q=dev_in["q"], k_tree=dev_in["k_tree"], v_tree=dev_in["v_tree"], k_cache=ain["k_cache"],
+                 v_cache=ain["v_cache"], prefix_len=ain["prefix_len"], new_prefix_len=new_pl,
+                 target=dev_in["target"])
+        for o, ho in zip(outs, host_out):
+            ho.copy_(o, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(K):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier()
+    t_e2e = max_over_ranks(e0.elapsed_time(e1) / 1000.0)
+    value_e2e = world * K / t_e2e
+
+    # ---- roofline of the dominant stage (the heads) and of tree attention ----
+    pk = peaks()
+    elt = 2
+    heads_bytes = (w.K * w.d * w.d + w.K * w.V * w.d) * elt + w.B * w.d * elt
+    heads_gbs = heads_bytes / stage[0] / 1e9
+    S = w.prefix
+    attn_bytes = (2 * w.B * w.Hkv * S * w.D + 2 * w.B * T * w.Hq * w.D + 2 * w.B * T * w.Hkv * w.D) * elt
+    attn_gbs = attn_bytes / stage[1] / 1e9
+    anc_pairs = sum(bin(sum(1 << j for j in range(T) if _is_anc(parents, i, j))).count("1") for i in range(T))
+    attn_flops = 4 * w.D * w.Hq * (T * S * w.B + anc_pairs * w.B)
+    attn_tflops = attn_flops / stage[1] / 1e12
+
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * t / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded random weights and activations; target logits synthesised "
+                                   "from the proposed tree with match probability 0.6)",
+        "config": config_dict(w, world),
+        "roofline": {"kernel": "medusa_heads (residual GEMV + LM-head GEMV with softmax/top-8 + merge)",
+                     "bound": "hbm", "achieved": heads_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "frac": heads_gbs / pk["hbm_gbs"], "peak_source": pk["source"],
+                     "algorithmic_bytes": heads_bytes, "traffic": HEADS_DRAM_BYTES},
+        "tree_attention": {"us": stage[1] * 1e6, "algorithmic_bytes": attn_bytes, "hbm_gbs": attn_gbs,
+                           "hbm_frac": attn_gbs / pk["hbm_gbs"], "hbm_frac_nominal_8tbs": attn_gbs / 8000.0,
+                           "tflops": attn_tflops, "tc_frac": attn_tflops * 1000.0 / pk["bf16_tflops"]},
+        "stage_us": {"medusa_heads": stage[0] * 1e6, "tree_attention": stage[1] * 1e6,
+                     "tree_verify": stage[2] * 1e6, "kv_commit": stage[3] * 1e6},
+        "mean_accept_len": mean_len,
+        "tokens_per_s": value * w.B * (mean_len + 1),
+        "e2e": {"value": value_e2e, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": K * launches_per_step(w),
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        sample = OracleSample(w, 1.0)
+        tt, ff = 0.0, 0.0
+        while tt < 10.0 and ff < 3.0:
+            t1, f1 = sample.run()
+            tt += t1
+            ff += f1
+        out["cpu_baseline"] = {"value": ff / tt, "unit": UNIT, "cores": 1, "kind": "oracle",
+                               "sample": f"{ff:.2f} whole steps of the same workload run by the single-threaded fp64 "
+                                         f"oracle on the host ({tt:.1f} s)"}
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def _is_anc(parents, i, j):
+    while i != -1:
+        if i == j:
+            return True
+        i = parents[i]
+    return False
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="mine", choices=["mine", "reference"])
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_mine(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

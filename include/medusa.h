@@ -1,0 +1,255 @@
+/*
+ * medusa.h -- C ABI of libmedusa.so: one Medusa speculative decode step on an
+ * NVIDIA B200 (sm_100a).
+ *
+ * The step has four calls, run in this order on one CUDA stream:
+ *   medusa_heads    Medusa heads, top-s per head, candidate-tree tokens
+ *   tree_attention  attention of every tree node over the prefix KV cache and
+ *                   its tree ancestors (one attention layer)
+ *   tree_verify     greedy or stochastic verification: longest accepted
+ *                   root-to-node path plus one bonus token
+ *   kv_commit       append the accepted path's K/V to the cache
+ *
+ * Sources of the operations (public web pages on Medusa):
+ *   [SPEC]  "Speculative Decoding & Medusa Tree Attention: Accelerating LLM
+ *           Inference by 3x Without Accuracy Loss", section 2 "The
+ *           Mathematical Foundation of Speculative Sampling".
+ *   [GUIDE] "Medusa Explained: Multi-Head Speculative Decoding Guide",
+ *           sections "The Architectural Blueprint", "1. Combinatorial Tree
+ *           Construction", "2. Single-Pass Tree Attention Verification".
+ *   [MTP]   "Multi-Token Prediction & Draft-Model-Free Speculative Decoding",
+ *           sections "The 2D Tree Attention Mask" and "Production Deployment
+ *           Guidelines".
+ *
+ * Conventions shared by every call
+ *   - Every function returns MEDUSA_OK (0) or a negative MEDUSA_ERR_* code;
+ *     medusa_last_error() then gives a message (thread-local).
+ *   - Tensor pointers are caller-owned DEVICE memory on the current device,
+ *     row-major and contiguous in the layout stated, 16-byte aligned.  The
+ *     library never frees or retains them.
+ *   - Compute calls are asynchronous on `stream` (a cudaStream_t; NULL is the
+ *     legacy default stream).  They do not synchronise and do not allocate:
+ *     scratch memory is the caller's `workspace` of at least the size the
+ *     matching *_workspace_size() query returns.
+ *   - Host-side argument errors (null pointer, bad shape, misalignment, too
+ *     small a workspace) are reported by the return code before anything is
+ *     launched.  Errors that only the data shows (a token id >= V, a cache
+ *     overflow, a prefix length out of range, a distribution with no mass)
+ *     are OR-ed as MEDUSA_STATUS_* bits into the caller's device int32
+ *     `status` (nullable; never cleared by the library) and never trap.
+ *   - dtype MEDUSA_F32 computes in fp32 throughout; MEDUSA_BF16 takes bf16
+ *     inputs, accumulates in fp32 and stores bf16 activations.
+ */
+#ifndef MEDUSA_H
+#define MEDUSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* medusa_stream_t; /* same type as cudaStream_t */
+
+enum {
+    MEDUSA_OK = 0,
+    MEDUSA_ERR_INVALID_ARG = -1, /* null pointer, bad size, misaligned pointer, bad tree */
+    MEDUSA_ERR_UNSUPPORTED = -2, /* T > 128, head_dim not 64/128, unsupported dtype */
+    MEDUSA_ERR_WORKSPACE = -3,   /* workspace smaller than the query says */
+    MEDUSA_ERR_CUDA = -4         /* a CUDA launch or runtime call failed */
+};
+
+/* device-side status bits (OR-ed into *status) */
+enum {
+    MEDUSA_STATUS_BAD_TOKEN = 1,      /* a token / node id outside its range */
+    MEDUSA_STATUS_CACHE_OVERFLOW = 2, /* kv_commit: prefix_len + len > S_max */
+    MEDUSA_STATUS_BAD_PREFIX = 4,     /* prefix_len outside [0, max_prefix] */
+    MEDUSA_STATUS_NO_MASS = 8         /* stochastic bonus drawn from an all-zero distribution */
+};
+
+typedef enum { MEDUSA_F32 = 0, MEDUSA_BF16 = 1 } medusa_dtype;
+typedef enum { MEDUSA_VERIFY_GREEDY = 0, MEDUSA_VERIFY_STOCHASTIC = 1 } medusa_verify_mode;
+
+/* largest top-s list per head and largest tree */
+#define MEDUSA_TOPK 8
+#define MEDUSA_MAX_TREE 128
+
+/* Message of the last failed call on this thread ("" if none). */
+const char* medusa_last_error(void);
+
+/* ABI version (major * 100 + minor). */
+int medusa_version(void);
+
+/* ------------------------------------------------------------------------ */
+/* Candidate tree                                                            */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Opaque, immutable description of a candidate tree ([GUIDE] "1. Combinatorial
+ * Tree Construction": the tree is flattened into one packed sequence of T
+ * nodes; [MTP] "The 2D Tree Attention Mask": node i may attend to node j when
+ * j is an ancestor of i or j = i).
+ *
+ * parent_host: HOST array of T int32.  Node 0 is the single root
+ *   (parent -1); for i > 0, 0 <= parent[i] < i.  Siblings are ordered by
+ *   index.  A node's depth counts the root as 1; a node at depth k >= 2 with
+ *   sibling rank r (number of earlier siblings) holds entry r of Medusa head
+ *   k-1's top-s list.
+ * T: 1 <= T <= MEDUSA_MAX_TREE.
+ * out: receives the handle.  The call allocates a few KB of device memory on
+ *   the current device (set-up time, not on the step) and synchronises; the
+ *   handle is valid on that device only.
+ * Errors: MEDUSA_ERR_INVALID_ARG (bad parent array), MEDUSA_ERR_UNSUPPORTED
+ *   (T > 128), MEDUSA_ERR_CUDA.
+ */
+typedef struct medusa_tree medusa_tree;
+int medusa_tree_create(const int32_t* parent_host, int T, medusa_tree** out);
+
+/* Frees the handle (synchronises the device first).  NULL is a no-op. */
+int medusa_tree_destroy(medusa_tree* tree);
+
+/* Node count, maximum depth (root = 1) and the largest child count. */
+int medusa_tree_info(const medusa_tree* tree, int* T, int* max_depth, int* max_children);
+
+/* ------------------------------------------------------------------------ */
+/* Medusa heads                                                              */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * [GUIDE] "The Architectural Blueprint": for every sequence b and Medusa head
+ * k = 1..K (array index k-1),
+ *     h^(k) = SiLU(W_res^(k) h) + h,    p^(k) = softmax(W_head^(k) h^(k)),
+ * no bias.  Then ([GUIDE] "1. Combinatorial Tree Construction") each head's
+ * top-MEDUSA_TOPK tokens (logit descending, lower token id first among equal
+ * logits) with their probabilities, and, if `tree` is given, the tree's node
+ * tokens: node 0 gets root_token[b] (w_{t+1}, the base model's own next
+ * token); a node at depth k+1 with sibling rank r gets topk_idx[b,k-1,r].
+ *
+ * h        [B, d]         dtype dt
+ * W_res    [K, d, d]      dtype dt, row = output feature, column = input
+ * W_head   [K, V, d]      dtype dt
+ * root_token [B] int32    (read only when tree != NULL)
+ * topk_idx [B, K, 8] int32 out   (-1 where V < 8)
+ * topk_prob [B, K, 8] f32 out    softmax probability of each entry
+ * node_tokens [B, T] int32 out  (tree != NULL)
+ * node_q   [B, T] f32 out, nullable: probability of each node's token under
+ *          the head that proposed it (1 at the root)
+ * h_res_out [B, K, d] dtype dt, nullable: h^(k) (bf16-rounded for BF16)
+ * logits_out [B, K, V] f32, nullable;  probs_out [B, K, V] f32, nullable
+ * Limits: d % 8 == 0 (BF16) or d % 4 == 0 (F32); d <= 16384; 1 <= V;
+ *   1 <= K <= 16; tree max depth <= K + 1 and every sibling rank < 8.
+ * Workspace: medusa_heads_workspace_size(B, d, V, K, dt) bytes.
+ */
+size_t medusa_heads_workspace_size(int B, int d, int V, int K, medusa_dtype dt);
+int medusa_heads(const void* h, const void* W_res, const void* W_head, int B, int d, int V, int K,
+                 medusa_dtype dt, const medusa_tree* tree, const int32_t* root_token, int32_t* topk_idx,
+                 float* topk_prob, int32_t* node_tokens, float* node_q, void* h_res_out, float* logits_out,
+                 float* probs_out, void* workspace, size_t workspace_bytes, int32_t* status,
+                 medusa_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Tree attention                                                            */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * [GUIDE] "2. Single-Pass Tree Attention Verification" and [MTP] "The 2D Tree
+ * Attention Mask": every tree node i attends to the whole cached prefix and
+ * to the tree nodes j that are its ancestors or itself.  For query head h
+ * (kv-head g = h / (Hq/Hkv)):
+ *     O[b,i,h,:] = sum_j softmax_j(scale * <q[b,i,h,:], k_j>) v_j
+ * over j in cache positions [0, prefix_len[b]) of kv-head g and the visible
+ * tree nodes.  RoPE and all projections are the caller's (Q/K/V arrive ready).
+ *
+ * q        [B, T, Hq, D]       dtype dt
+ * k_tree, v_tree [B, T, Hkv, D] dtype dt (this step's tree K/V)
+ * k_cache, v_cache [B, Hkv, S_max, D] dtype dt (only [0, prefix_len[b]) read)
+ * prefix_len [B] int32, device; each in [0, max_prefix]
+ * max_prefix: upper bound of prefix_len the grid is sized for (0 = S_max)
+ * scale: softmax scale; <= 0 means 1/sqrt(D)
+ * out      [B, T, Hq, D]       dtype dt
+ * lse      [B, T, Hq] f32, nullable: natural-log sum of exp of the scaled scores
+ * Limits: D in {64, 128}; Hq % Hkv == 0; T = tree node count (<= 128).
+ * A prefix_len outside [0, max_prefix] sets MEDUSA_STATUS_BAD_PREFIX and the
+ * sequence's rows are computed over the clamped prefix.
+ * Workspace: tree_attention_workspace_size(...) bytes.
+ */
+size_t tree_attention_workspace_size(int B, int Hq, int Hkv, int D, int S_max, int max_prefix,
+                                     const medusa_tree* tree, medusa_dtype dt);
+int tree_attention(const void* q, const void* k_tree, const void* v_tree, const void* k_cache,
+                   const void* v_cache, const int32_t* prefix_len, int B, int Hq, int Hkv, int D, int S_max,
+                   int max_prefix, float scale, medusa_dtype dt, const medusa_tree* tree, void* out, float* lse,
+                   void* workspace, size_t workspace_bytes, int32_t* status, medusa_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Verification                                                              */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * GREEDY ([GUIDE] "2. Single-Pass Tree Attention Verification", steps 2-4;
+ * [MTP] "The 2D Tree Attention Mask": the longest accepted path plus one
+ * bonus token from the target): the target's prediction after node u is
+ * argmax(target[b,u,:]) (largest logit, lowest id among equal ones, NaN never
+ * wins).  The root is accepted; node c is accepted when its parent is and
+ * node_tokens[b,c] equals the parent's prediction.  The path ends at the
+ * deepest accepted node (lowest index among equally deep ones); the bonus is
+ * that node's prediction.
+ *   target: logits [B, T, V], dtype target_dt (F32 or BF16).
+ *
+ * STOCHASTIC ([SPEC] section 2: accept x with probability
+ * min(1, P_target(x)/P_draft(x)); on rejection resample from
+ * normalize(max(0, P_target - P_draft))), walked over the tree: at the
+ * current node u, with current distribution P (first p[b,u,:]) and draft
+ * Q = q[b, q_row[u], :], children are tried in index order.  Child c with
+ * token x is accepted iff u_c * Q(x) < P(x); the walk then moves to c with
+ * P = p[b,c,:].  On rejection P becomes the residual W/S with
+ * W(y) = floor(max(0, P(y) - Q(y)) * 2^32), S = sum W (P kept when S = 0).
+ * When no child is left the bonus is the smallest y whose inclusive prefix
+ * sum of floor(P(y) * 2^32) exceeds floor(U * S / 2^32).  Uniforms come from
+ * Philox4x32-10 (Salmon et al., SC'11) with key (seed low word, seed high
+ * word) and counter (b, node, step, 0): u_c = (word0 >> 8) * 2^-24 of child
+ * c's block, U = word1 of the block of the node where the walk ends.  All
+ * arithmetic is integer or correctly rounded fp64, so results are exact.
+ *   target: p [B, T, V] f32 (target_dt must be MEDUSA_F32);
+ *   q [B, q_rows, V] f32; q_row [T] int32 device, nullable (identity, then
+ *   q_rows must equal T).  Medusa heads' probs_out [B, K, V] serves as q with
+ *   q_row[u] = depth(u) - 1.
+ *
+ * node_tokens [B, T] int32; accept_path [B, max_path] int32 out (node ids,
+ * root first, -1 padded); accept_len [B] int32 out (>= 1, counts the root);
+ * bonus [B] int32 out.  max_path >= the tree's max depth.
+ * Workspace: tree_verify_workspace_size(...) bytes.
+ */
+size_t tree_verify_workspace_size(medusa_verify_mode mode, int B, int V, const medusa_tree* tree);
+int tree_verify(medusa_verify_mode mode, const void* target, medusa_dtype target_dt, const float* q, int q_rows,
+                const int32_t* q_row, const int32_t* node_tokens, int B, int V, const medusa_tree* tree,
+                uint64_t seed, uint32_t step, int32_t* accept_path, int max_path, int32_t* accept_len,
+                int32_t* bonus, void* workspace, size_t workspace_bytes, int32_t* status,
+                medusa_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* KV commit                                                                 */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * [MTP] "The 2D Tree Attention Mask" (the engine commits the longest accepted
+ * path) and "Production Deployment Guidelines" (unselected branches are
+ * culled): for t < accept_len[b],
+ *     cache[b, g, prefix_len[b] + t, :] = tree[b, accept_path[b,t], g, :]
+ * for K and V and every kv-head g, bit for bit; then
+ *     new_prefix_len[b] = prefix_len[b] + accept_len[b].
+ * k_cache, v_cache [B, Hkv, S_max, D] (in place); k_tree, v_tree
+ * [B, T, Hkv, D]; accept_path [B, max_path]; accept_len [B];
+ * prefix_len [B] in; new_prefix_len [B] out (may alias prefix_len).
+ * A sequence whose commit would pass S_max, or whose path holds an id
+ * outside [0, T), is left untouched (new_prefix_len = prefix_len) and sets
+ * MEDUSA_STATUS_CACHE_OVERFLOW or MEDUSA_STATUS_BAD_TOKEN.
+ */
+int kv_commit(void* k_cache, void* v_cache, const void* k_tree, const void* v_tree, const int32_t* accept_path,
+              int max_path, const int32_t* accept_len, const int32_t* prefix_len, int32_t* new_prefix_len, int B,
+              int T, int Hkv, int D, int S_max, medusa_dtype dt, int32_t* status, medusa_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MEDUSA_H */

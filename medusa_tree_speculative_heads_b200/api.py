@@ -1,0 +1,177 @@
+"""Tensor-level API over the C ABI.
+
+The functions here allocate outputs and workspaces with torch and call the
+binding; every step of the computation runs in libmedusa's CUDA kernels.
+``MedusaStep`` preallocates everything for a fixed shape, so a decode step
+is four library calls with no allocation (and can be captured in a CUDA
+graph).
+"""
+from __future__ import annotations
+
+from typing import Dict, Optional, Sequence
+
+import torch
+
+from . import binding as _b
+from .binding import Tree
+
+
+def _ws(nbytes: int, device) -> torch.Tensor:
+    return torch.empty(max(int(nbytes), 16), dtype=torch.uint8, device=device)
+
+
+def _status(device) -> torch.Tensor:
+    return torch.zeros(1, dtype=torch.int32, device=device)
+
+
+def heads(h: torch.Tensor, W_res: torch.Tensor, W_head: torch.Tensor, tree: Optional[Tree] = None,
+          root_token: Optional[torch.Tensor] = None, want_logits: bool = False, want_probs: bool = False,
+          want_hres: bool = False) -> Dict[str, torch.Tensor]:
+    """Medusa heads: top-8 ids/probabilities per head and, with a tree, the
+    tree's node tokens.  h [B,d], W_res [K,d,d], W_head [K,V,d]."""
+    B, d = h.shape
+    K, V, _ = W_head.shape
+    dev = h.device
+    dt = _b.dtype_code(h.dtype)
+    out = {
+        "topk_idx": torch.empty((B, K, _b.TOPK), dtype=torch.int32, device=dev),
+        "topk_prob": torch.empty((B, K, _b.TOPK), dtype=torch.float32, device=dev),
+        "status": _status(dev),
+    }
+    if tree is not None:
+        out["node_tokens"] = torch.empty((B, tree.T), dtype=torch.int32, device=dev)
+        out["node_q"] = torch.empty((B, tree.T), dtype=torch.float32, device=dev)
+    if want_logits:
+        out["logits"] = torch.empty((B, K, V), dtype=torch.float32, device=dev)
+    if want_probs:
+        out["probs"] = torch.empty((B, K, V), dtype=torch.float32, device=dev)
+    if want_hres:
+        out["h_res"] = torch.empty((B, K, d), dtype=h.dtype, device=dev)
+    nb = _b.medusa_heads_workspace_size(B, d, V, K, dt)
+    ws = _ws(nb, dev)
+    _b.medusa_heads(h, W_res, W_head, B, d, V, K, dt, tree, root_token, out["topk_idx"], out["topk_prob"],
+                    out.get("node_tokens"), out.get("node_q"), out.get("h_res"), out.get("logits"),
+                    out.get("probs"), ws, nb, out["status"])
+    return out
+
+
+def tree_attention(q, k_tree, v_tree, k_cache, v_cache, prefix_len, tree: Tree, scale: float = 0.0,
+                   max_prefix: int = 0, want_lse: bool = False) -> Dict[str, torch.Tensor]:
+    """Tree attention; q [B,T,Hq,D], k/v_tree [B,T,Hkv,D], caches
+    [B,Hkv,S_max,D], prefix_len [B] int32."""
+    B, T, Hq, D = q.shape
+    Hkv = k_tree.shape[2]
+    S_max = k_cache.shape[2]
+    dev = q.device
+    dt = _b.dtype_code(q.dtype)
+    out = {"out": torch.empty_like(q), "status": _status(dev)}
+    if want_lse:
+        out["lse"] = torch.empty((B, T, Hq), dtype=torch.float32, device=dev)
+    nb = _b.tree_attention_workspace_size(B, Hq, Hkv, D, S_max, max_prefix, tree, dt)
+    ws = _ws(nb, dev)
+    _b.tree_attention(q, k_tree, v_tree, k_cache, v_cache, prefix_len, B, Hq, Hkv, D, S_max, max_prefix, scale, dt,
+                      tree, out["out"], out.get("lse"), ws, nb, out["status"])
+    return out
+
+
+def tree_verify(mode: int, target: torch.Tensor, node_tokens: torch.Tensor, tree: Tree,
+                q: Optional[torch.Tensor] = None, q_row: Optional[torch.Tensor] = None, seed: int = 0,
+                step: int = 0, max_path: Optional[int] = None) -> Dict[str, torch.Tensor]:
+    """Greedy (target = logits [B,T,V]) or stochastic (target = p [B,T,V]
+    fp32, q [B,q_rows,V] fp32, optional q_row [T]) verification."""
+    B, T, V = target.shape
+    dev = target.device
+    max_path = max_path or tree.max_depth
+    out = {
+        "accept_path": torch.empty((B, max_path), dtype=torch.int32, device=dev),
+        "accept_len": torch.empty((B,), dtype=torch.int32, device=dev),
+        "bonus": torch.empty((B,), dtype=torch.int32, device=dev),
+        "status": _status(dev),
+    }
+    nb = _b.tree_verify_workspace_size(mode, B, V, tree)
+    ws = _ws(nb, dev)
+    q_rows = q.shape[1] if q is not None else 0
+    _b.tree_verify(mode, target, _b.dtype_code(target.dtype), q, q_rows, q_row, node_tokens, B, V, tree, seed, step,
+                   out["accept_path"], max_path, out["accept_len"], out["bonus"], ws, nb, out["status"])
+    return out
+
+
+def kv_commit(k_cache, v_cache, k_tree, v_tree, accept_path, accept_len, prefix_len,
+              new_prefix_len: Optional[torch.Tensor] = None) -> Dict[str, torch.Tensor]:
+    """Append the accepted path's K/V in place; returns new_prefix_len (a new
+    tensor unless one is given, which may be prefix_len itself)."""
+    B, Hkv, S_max, D = k_cache.shape
+    T = k_tree.shape[1]
+    dev = k_cache.device
+    if new_prefix_len is None:
+        new_prefix_len = torch.empty_like(prefix_len)
+    st = _status(dev)
+    _b.kv_commit(k_cache, v_cache, k_tree, v_tree, accept_path, accept_path.shape[1], accept_len, prefix_len,
+                 new_prefix_len, B, T, Hkv, D, S_max, _b.dtype_code(k_cache.dtype), st)
+    return {"new_prefix_len": new_prefix_len, "status": st}
+
+
+class MedusaStep:
+    """All buffers of one decode step of a fixed shape, allocated once.
+
+    ``run`` issues the four library calls on the current stream:
+    medusa_heads -> tree_attention -> tree_verify -> kv_commit.  The new
+    prefix lengths go to ``new_prefix_len`` (pass the same tensor as
+    ``prefix_len`` to advance in place)."""
+
+    def __init__(self, *, B: int, d: int, V: int, K: int, Hq: int, Hkv: int, D: int, S_max: int,
+                 parents: Sequence[int], dtype: torch.dtype, mode: int = _b.GREEDY, max_prefix: int = 0,
+                 q_rows: int = 0, device=None):
+        dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+        self.B, self.d, self.V, self.K = B, d, V, K
+        self.Hq, self.Hkv, self.D, self.S_max, self.max_prefix = Hq, Hkv, D, S_max, max_prefix
+        self.dt = _b.dtype_code(dtype)
+        self.mode = mode
+        self.tree = Tree(parents)
+        T = self.T = self.tree.T
+        self.max_path = self.tree.max_depth
+        self.q_rows = q_rows
+        i32, f32 = torch.int32, torch.float32
+        self.topk_idx = torch.empty((B, K, _b.TOPK), dtype=i32, device=dev)
+        self.topk_prob = torch.empty((B, K, _b.TOPK), dtype=f32, device=dev)
+        self.node_tokens = torch.empty((B, T), dtype=i32, device=dev)
+        self.node_q = torch.empty((B, T), dtype=f32, device=dev)
+        self.attn_out = torch.empty((B, T, Hq, D), dtype=dtype, device=dev)
+        self.accept_path = torch.empty((B, self.max_path), dtype=i32, device=dev)
+        self.accept_len = torch.empty((B,), dtype=i32, device=dev)
+        self.bonus = torch.empty((B,), dtype=i32, device=dev)
+        self.status = torch.zeros(1, dtype=i32, device=dev)
+        self.ws_heads_n = _b.medusa_heads_workspace_size(B, d, V, K, self.dt)
+        self.ws_attn_n = _b.tree_attention_workspace_size(B, Hq, Hkv, D, S_max, max_prefix, self.tree, self.dt)
+        self.ws_verify_n = _b.tree_verify_workspace_size(mode, B, V, self.tree)
+        self.ws_heads = _ws(self.ws_heads_n, dev)
+        self.ws_attn = _ws(self.ws_attn_n, dev)
+        self.ws_verify = _ws(self.ws_verify_n, dev)
+
+    def heads(self, h, W_res, W_head, root_token, probs_out=None):
+        _b.medusa_heads(h, W_res, W_head, self.B, self.d, self.V, self.K, self.dt, self.tree, root_token,
+                        self.topk_idx, self.topk_prob, self.node_tokens, self.node_q, None, None, probs_out,
+                        self.ws_heads, self.ws_heads_n, self.status)
+
+    def attention(self, q, k_tree, v_tree, k_cache, v_cache, prefix_len):
+        _b.tree_attention(q, k_tree, v_tree, k_cache, v_cache, prefix_len, self.B, self.Hq, self.Hkv, self.D,
+                          self.S_max, self.max_prefix, 0.0, self.dt, self.tree, self.attn_out, None, self.ws_attn,
+                          self.ws_attn_n, self.status)
+
+    def verify(self, target, q=None, q_row=None, seed: int = 0, step: int = 0, node_tokens=None):
+        tgt_dt = _b.dtype_code(target.dtype)
+        _b.tree_verify(self.mode, target, tgt_dt, q, self.q_rows if q is not None else 0, q_row,
+                       self.node_tokens if node_tokens is None else node_tokens, self.B, self.V, self.tree, seed,
+                       step, self.accept_path, self.max_path, self.accept_len, self.bonus, self.ws_verify,
+                       self.ws_verify_n, self.status)
+
+    def commit(self, k_cache, v_cache, k_tree, v_tree, prefix_len, new_prefix_len):
+        _b.kv_commit(k_cache, v_cache, k_tree, v_tree, self.accept_path, self.max_path, self.accept_len, prefix_len,
+                     new_prefix_len, self.B, self.T, self.Hkv, self.D, self.S_max, self.dt, self.status)
+
+    def run(self, *, h, W_res, W_head, root_token, q, k_tree, v_tree, k_cache, v_cache, prefix_len, new_prefix_len,
+            target, q_draft=None, q_row=None, seed: int = 0, step: int = 0, node_tokens=None):
+        self.heads(h, W_res, W_head, root_token)
+        self.attention(q, k_tree, v_tree, k_cache, v_cache, prefix_len)
+        self.verify(target, q_draft, q_row, seed, step, node_tokens)
+        self.commit(k_cache, v_cache, k_tree, v_tree, prefix_len, new_prefix_len)

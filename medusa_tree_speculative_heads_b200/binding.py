@@ -1,0 +1,182 @@
+"""ctypes binding of libmedusa.so (argument marshalling only).
+
+Every function has the name and argument order of its C entry point in
+include/medusa.h.  Tensors are torch CUDA tensors (or None for nullable
+pointers); the current torch stream of the current device is used unless a
+``stream`` is given.  Non-zero return codes raise :class:`MedusaError` with
+the library's message.  There is no fallback: if the library was not built,
+the first call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmedusa.so")
+HEADER = os.path.join(os.path.dirname(_HERE), "include", "medusa.h")
+
+MEDUSA_OK = 0
+MEDUSA_ERR_INVALID_ARG = -1
+MEDUSA_ERR_UNSUPPORTED = -2
+MEDUSA_ERR_WORKSPACE = -3
+MEDUSA_ERR_CUDA = -4
+
+STATUS_BAD_TOKEN = 1
+STATUS_CACHE_OVERFLOW = 2
+STATUS_BAD_PREFIX = 4
+STATUS_NO_MASS = 8
+
+F32, BF16 = 0, 1
+GREEDY, STOCHASTIC = 0, 1
+TOPK = 8
+MAX_TREE = 128
+
+_lib = None
+
+
+class MedusaError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"[{code}] {msg}")
+        self.code = code
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmedusa.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libmedusa.so not built ({LIB_PATH}); run medusa_tree_speculative_heads_b200/build.py")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, u32, u64, sz, f32 = (ctypes.c_void_p, ctypes.c_int, ctypes.c_uint32, ctypes.c_uint64, ctypes.c_size_t,
+                                      ctypes.c_float)
+        L.medusa_last_error.restype = ctypes.c_char_p
+        L.medusa_last_error.argtypes = []
+        L.medusa_version.restype = i32
+        L.medusa_tree_create.argtypes = [vp, i32, ctypes.POINTER(vp)]
+        L.medusa_tree_destroy.argtypes = [vp]
+        L.medusa_tree_info.argtypes = [vp, vp, vp, vp]
+        L.medusa_heads_workspace_size.argtypes = [i32, i32, i32, i32, i32]
+        L.medusa_heads_workspace_size.restype = sz
+        L.medusa_heads.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
+                                   vp, vp]
+        L.tree_attention_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32, vp, i32]
+        L.tree_attention_workspace_size.restype = sz
+        L.tree_attention.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, i32, vp, vp, vp, vp,
+                                     sz, vp, vp]
+        L.tree_verify_workspace_size.argtypes = [i32, i32, i32, vp]
+        L.tree_verify_workspace_size.restype = sz
+        L.tree_verify.argtypes = [i32, vp, i32, vp, i32, vp, vp, i32, i32, vp, u64, u32, vp, i32, vp, vp, vp, sz, vp,
+                                  vp]
+        L.kv_commit.argtypes = [vp, vp, vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp]
+        _lib = L
+    return _lib
+
+
+def declared_functions() -> list:
+    """Names of the functions include/medusa.h declares."""
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*([a-z_][a-z0-9_]*)\s*\(", src,
+                                 flags=re.M)))
+
+
+def _check(rc: int):
+    if rc != MEDUSA_OK:
+        raise MedusaError(rc, lib().medusa_last_error().decode())
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        stream = stream.cuda_stream
+    return ctypes.c_void_p(int(stream))
+
+
+def dtype_code(t: torch.dtype) -> int:
+    if t == torch.float32:
+        return F32
+    if t == torch.bfloat16:
+        return BF16
+    raise TypeError(f"unsupported dtype {t}")
+
+
+def version() -> int:
+    return lib().medusa_version()
+
+
+class Tree:
+    """Owner of a medusa_tree handle (created on the current device)."""
+
+    def __init__(self, parents: Sequence[int]):
+        arr = (ctypes.c_int32 * len(parents))(*[int(x) for x in parents])
+        h = ctypes.c_void_p()
+        _check(lib().medusa_tree_create(arr, len(parents), ctypes.byref(h)))
+        self.handle = h
+        self.parents = [int(x) for x in parents]
+        T, dep, mc = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+        _check(lib().medusa_tree_info(h, ctypes.byref(T), ctypes.byref(dep), ctypes.byref(mc)))
+        self.T, self.max_depth, self.max_children = T.value, dep.value, mc.value
+
+    def close(self):
+        if self.handle:
+            _check(lib().medusa_tree_destroy(self.handle))
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def medusa_heads_workspace_size(B: int, d: int, V: int, K: int, dt: int) -> int:
+    return lib().medusa_heads_workspace_size(B, d, V, K, dt)
+
+
+def medusa_heads(h, W_res, W_head, B, d, V, K, dt, tree: Optional[Tree], root_token, topk_idx, topk_prob,
+                 node_tokens, node_q, h_res_out, logits_out, probs_out, workspace, workspace_bytes, status,
+                 stream=None):
+    _check(lib().medusa_heads(_p(h), _p(W_res), _p(W_head), B, d, V, K, dt, tree.handle if tree else None,
+                              _p(root_token), _p(topk_idx), _p(topk_prob), _p(node_tokens), _p(node_q),
+                              _p(h_res_out), _p(logits_out), _p(probs_out), _p(workspace), workspace_bytes,
+                              _p(status), _stream(stream)))
+
+
+def tree_attention_workspace_size(B, Hq, Hkv, D, S_max, max_prefix, tree: Tree, dt) -> int:
+    return lib().tree_attention_workspace_size(B, Hq, Hkv, D, S_max, max_prefix, tree.handle, dt)
+
+
+def tree_attention(q, k_tree, v_tree, k_cache, v_cache, prefix_len, B, Hq, Hkv, D, S_max, max_prefix, scale, dt,
+                   tree: Tree, out, lse, workspace, workspace_bytes, status, stream=None):
+    _check(lib().tree_attention(_p(q), _p(k_tree), _p(v_tree), _p(k_cache), _p(v_cache), _p(prefix_len), B, Hq,
+                                Hkv, D, S_max, max_prefix, float(scale), dt, tree.handle, _p(out), _p(lse),
+                                _p(workspace), workspace_bytes, _p(status), _stream(stream)))
+
+
+def tree_verify_workspace_size(mode, B, V, tree: Tree) -> int:
+    return lib().tree_verify_workspace_size(mode, B, V, tree.handle)
+
+
+def tree_verify(mode, target, target_dt, q, q_rows, q_row, node_tokens, B, V, tree: Tree, seed, step, accept_path,
+                max_path, accept_len, bonus, workspace, workspace_bytes, status, stream=None):
+    _check(lib().tree_verify(mode, _p(target), target_dt, _p(q), q_rows, _p(q_row), _p(node_tokens), B, V,
+                             tree.handle, ctypes.c_uint64(seed & (2**64 - 1)), ctypes.c_uint32(step & 0xFFFFFFFF),
+                             _p(accept_path), max_path, _p(accept_len), _p(bonus), _p(workspace), workspace_bytes,
+                             _p(status), _stream(stream)))
+
+
+def kv_commit(k_cache, v_cache, k_tree, v_tree, accept_path, max_path, accept_len, prefix_len, new_prefix_len, B, T,
+              Hkv, D, S_max, dt, status, stream=None):
+    _check(lib().kv_commit(_p(k_cache), _p(v_cache), _p(k_tree), _p(v_tree), _p(accept_path), max_path,
+                           _p(accept_len), _p(prefix_len), _p(new_prefix_len), B, T, Hkv, D, S_max, dt, _p(status),
+                           _stream(stream)))

@@ -1,0 +1,384 @@
+// C ABI of libmedusa: argument validation, the candidate-tree handle,
+// workspace queries and launches.  See include/medusa.h for the contract of
+// every entry point.
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <string>
+
+#include "kernels.h"
+
+struct medusa_tree {
+    medusa::TreeDev host;
+    medusa::TreeDev* dev;
+    int device;
+};
+
+namespace medusa {
+
+namespace {
+thread_local std::string g_err;
+
+int fail(int code, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return code;
+}
+
+int ok() {
+    g_err.clear();
+    return MEDUSA_OK;
+}
+
+bool al16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+int cuda_fail(cudaError_t e, const char* what) {
+    return fail(MEDUSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+int check_tree(const medusa_tree* t) {
+    if (!t) return fail(MEDUSA_ERR_INVALID_ARG, "tree is NULL");
+    int dev = -1;
+    cudaGetDevice(&dev);
+    if (dev != t->device)
+        return fail(MEDUSA_ERR_INVALID_ARG, "tree was created on device %d, current device is %d", t->device, dev);
+    return MEDUSA_OK;
+}
+}  // namespace
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+int num_sms() {
+    static int cache[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) dev = 0;
+    if (!cache[dev]) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        cache[dev] = n > 0 ? n : 1;
+    }
+    return cache[dev];
+}
+
+}  // namespace medusa
+
+using namespace medusa;
+
+extern "C" const char* medusa_last_error(void) { return g_err.c_str(); }
+
+extern "C" int medusa_version(void) { return 100; }
+
+// ---------------------------------------------------------------------------
+// tree handle
+// ---------------------------------------------------------------------------
+
+extern "C" int medusa_tree_create(const int32_t* parent, int T, medusa_tree** out) {
+    if (!parent || !out) return fail(MEDUSA_ERR_INVALID_ARG, "medusa_tree_create: NULL argument");
+    if (T < 1) return fail(MEDUSA_ERR_INVALID_ARG, "medusa_tree_create: T = %d < 1", T);
+    if (T > kMaxTree) return fail(MEDUSA_ERR_UNSUPPORTED, "medusa_tree_create: T = %d > %d", T, kMaxTree);
+    if (parent[0] != -1) return fail(MEDUSA_ERR_INVALID_ARG, "medusa_tree_create: node 0 must be the root (parent -1)");
+    for (int i = 1; i < T; ++i)
+        if (parent[i] < 0 || parent[i] >= i)
+            return fail(MEDUSA_ERR_INVALID_ARG,
+                        "medusa_tree_create: parent[%d] = %d; need 0 <= parent[i] < i (one root, topological order)",
+                        i, parent[i]);
+    medusa_tree* t = new medusa_tree();
+    TreeDev& h = t->host;
+    memset(&h, 0, sizeof h);
+    h.T = T;
+    int cnt[kMaxTree] = {0};
+    h.parent[0] = -1;
+    h.depth[0] = 1;
+    h.anc[0][0] = 1u;
+    h.max_depth = 1;
+    for (int i = 1; i < T; ++i) {
+        const int p = parent[i];
+        h.parent[i] = (int16_t)p;
+        h.depth[i] = (uint8_t)(h.depth[p] + 1);
+        h.rank[i] = (uint8_t)cnt[p]++;
+        for (int w = 0; w < 4; ++w) h.anc[i][w] = h.anc[p][w];
+        h.anc[i][i >> 5] |= 1u << (i & 31);
+        if (h.depth[i] > h.max_depth) h.max_depth = h.depth[i];
+    }
+    int off = 0;
+    for (int u = 0; u < T; ++u) {
+        h.child_off[u] = (uint8_t)off;
+        off += cnt[u];
+        if (cnt[u] > h.max_children) h.max_children = cnt[u];
+    }
+    h.child_off[T] = (uint8_t)off;
+    int fill[kMaxTree] = {0};
+    for (int c = 1; c < T; ++c) {
+        const int p = parent[c];
+        h.child_idx[h.child_off[p] + fill[p]++] = (uint8_t)c;
+    }
+    cudaGetDevice(&t->device);
+    cudaError_t e = cudaMalloc((void**)&t->dev, sizeof(TreeDev));
+    if (e == cudaSuccess) e = cudaMemcpy(t->dev, &h, sizeof(TreeDev), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) {
+        if (t->dev) cudaFree(t->dev);
+        delete t;
+        return cuda_fail(e, "medusa_tree_create");
+    }
+    *out = t;
+    return ok();
+}
+
+extern "C" int medusa_tree_destroy(medusa_tree* t) {
+    if (!t) return ok();
+    cudaDeviceSynchronize();
+    cudaError_t e = cudaFree(t->dev);
+    delete t;
+    if (e != cudaSuccess) return cuda_fail(e, "medusa_tree_destroy");
+    return ok();
+}
+
+extern "C" int medusa_tree_info(const medusa_tree* t, int* T, int* max_depth, int* max_children) {
+    if (!t) return fail(MEDUSA_ERR_INVALID_ARG, "medusa_tree_info: tree is NULL");
+    if (T) *T = t->host.T;
+    if (max_depth) *max_depth = t->host.max_depth;
+    if (max_children) *max_children = t->host.max_children;
+    return ok();
+}
+
+// ---------------------------------------------------------------------------
+// medusa_heads
+// ---------------------------------------------------------------------------
+
+extern "C" size_t medusa_heads_workspace_size(int B, int d, int V, int K, medusa_dtype dt) {
+    if (B < 1 || d < 1 || V < 1 || K < 1) return 0;
+    return heads_workspace_size(B, d, V, K, dt);
+}
+
+extern "C" int medusa_heads(const void* h, const void* W_res, const void* W_head, int B, int d, int V, int K,
+                            medusa_dtype dt, const medusa_tree* tree, const int32_t* root_token, int32_t* topk_idx,
+                            float* topk_prob, int32_t* node_tokens, float* node_q, void* h_res_out,
+                            float* logits_out, float* probs_out, void* workspace, size_t workspace_bytes,
+                            int32_t* status, medusa_stream_t stream) {
+    if (dt != MEDUSA_F32 && dt != MEDUSA_BF16) return fail(MEDUSA_ERR_UNSUPPORTED, "medusa_heads: unknown dtype");
+    if (!h || !W_res || !W_head || !topk_idx || !topk_prob || !workspace)
+        return fail(MEDUSA_ERR_INVALID_ARG, "medusa_heads: NULL tensor argument");
+    if (B < 1 || d < 1 || V < 1 || K < 1 || K > 16 || d > 16384)
+        return fail(MEDUSA_ERR_INVALID_ARG, "medusa_heads: bad sizes B=%d d=%d V=%d K=%d", B, d, V, K);
+    const int vec = dt == MEDUSA_BF16 ? 8 : 4;
+    if (d % vec) return fail(MEDUSA_ERR_INVALID_ARG, "medusa_heads: d=%d must be a multiple of %d", d, vec);
+    if (!al16(h) || !al16(W_res) || !al16(W_head) || !al16(h_res_out))
+        return fail(MEDUSA_ERR_INVALID_ARG, "medusa_heads: h, W_res, W_head, h_res_out must be 16-byte aligned");
+    if (workspace_bytes < heads_workspace_size(B, d, V, K, dt) || !al16(workspace))
+        return fail(MEDUSA_ERR_WORKSPACE, "medusa_heads: workspace of %zu bytes, need %zu (16-byte aligned)",
+                    workspace_bytes, heads_workspace_size(B, d, V, K, dt));
+    int T = 0;
+    if (tree) {
+        int rc = check_tree(tree);
+        if (rc) return rc;
+        if (!node_tokens || !root_token)
+            return fail(MEDUSA_ERR_INVALID_ARG, "medusa_heads: a tree needs root_token and node_tokens");
+        const TreeDev& th = tree->host;
+        if (th.max_depth > K + 1)
+            return fail(MEDUSA_ERR_INVALID_ARG, "medusa_heads: tree depth %d needs more than K=%d heads",
+                        th.max_depth, K);
+        const int smax = V < kTopK ? V : kTopK;
+        for (int i = 1; i < th.T; ++i)
+            if (th.rank[i] >= smax)
+                return fail(MEDUSA_ERR_UNSUPPORTED, "medusa_heads: node %d has sibling rank %d >= %d", i, th.rank[i],
+                            smax);
+        T = th.T;
+    }
+    HeadsArgs a;
+    a.h = h;
+    a.W_res = W_res;
+    a.W_head = W_head;
+    a.B = B;
+    a.d = d;
+    a.V = V;
+    a.K = K;
+    a.dt = dt;
+    a.tree = tree ? tree->dev : nullptr;
+    a.T = T;
+    a.root_token = root_token;
+    a.topk_idx = topk_idx;
+    a.topk_prob = topk_prob;
+    a.node_tokens = node_tokens;
+    a.node_q = node_q;
+    a.h_res_out = h_res_out;
+    a.logits_out = logits_out;
+    a.probs_out = probs_out;
+    a.ws = workspace;
+    a.ws_bytes = workspace_bytes;
+    a.status = status;
+    cudaError_t e = heads_launch(a, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "medusa_heads launch");
+    return ok();
+}
+
+// ---------------------------------------------------------------------------
+// tree_attention
+// ---------------------------------------------------------------------------
+
+extern "C" size_t tree_attention_workspace_size(int B, int Hq, int Hkv, int D, int S_max, int max_prefix,
+                                                const medusa_tree* tree, medusa_dtype dt) {
+    if (!tree || B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || (D != 64 && D != 128)) return 0;
+    if (max_prefix <= 0) max_prefix = S_max;
+    return attn_workspace_size(B, tree->host.T, Hq, Hkv, D, max_prefix, dt);
+}
+
+extern "C" int tree_attention(const void* q, const void* k_tree, const void* v_tree, const void* k_cache,
+                              const void* v_cache, const int32_t* prefix_len, int B, int Hq, int Hkv, int D,
+                              int S_max, int max_prefix, float scale, medusa_dtype dt, const medusa_tree* tree,
+                              void* out, float* lse, void* workspace, size_t workspace_bytes, int32_t* status,
+                              medusa_stream_t stream) {
+    if (dt != MEDUSA_F32 && dt != MEDUSA_BF16) return fail(MEDUSA_ERR_UNSUPPORTED, "tree_attention: unknown dtype");
+    if (!q || !k_tree || !v_tree || !k_cache || !v_cache || !prefix_len || !out)
+        return fail(MEDUSA_ERR_INVALID_ARG, "tree_attention: NULL tensor argument");
+    int rc = check_tree(tree);
+    if (rc) return rc;
+    if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || S_max < 0)
+        return fail(MEDUSA_ERR_INVALID_ARG, "tree_attention: bad sizes B=%d Hq=%d Hkv=%d S_max=%d", B, Hq, Hkv, S_max);
+    if (D != 64 && D != 128) return fail(MEDUSA_ERR_UNSUPPORTED, "tree_attention: head_dim %d (64 or 128)", D);
+    if (max_prefix <= 0) max_prefix = S_max;
+    if (max_prefix > S_max)
+        return fail(MEDUSA_ERR_INVALID_ARG, "tree_attention: max_prefix %d > S_max %d", max_prefix, S_max);
+    if (!al16(q) || !al16(k_tree) || !al16(v_tree) || !al16(k_cache) || !al16(v_cache) || !al16(out))
+        return fail(MEDUSA_ERR_INVALID_ARG, "tree_attention: tensors must be 16-byte aligned");
+    const size_t need = attn_workspace_size(B, tree->host.T, Hq, Hkv, D, max_prefix, dt);
+    if (need && (!workspace || workspace_bytes < need || !al16(workspace)))
+        return fail(MEDUSA_ERR_WORKSPACE, "tree_attention: workspace of %zu bytes, need %zu (16-byte aligned)",
+                    workspace_bytes, need);
+    AttnArgs a;
+    a.q = q;
+    a.k_tree = k_tree;
+    a.v_tree = v_tree;
+    a.k_cache = k_cache;
+    a.v_cache = v_cache;
+    a.prefix_len = prefix_len;
+    a.B = B;
+    a.T = tree->host.T;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.D = D;
+    a.S_max = S_max;
+    a.max_prefix = max_prefix;
+    a.scale = scale;
+    a.dt = dt;
+    a.tree = tree->dev;
+    a.out = out;
+    a.lse = lse;
+    a.ws = workspace;
+    a.ws_bytes = workspace_bytes;
+    a.status = status;
+    cudaError_t e = attn_launch(a, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "tree_attention launch");
+    return ok();
+}
+
+// ---------------------------------------------------------------------------
+// tree_verify
+// ---------------------------------------------------------------------------
+
+extern "C" size_t tree_verify_workspace_size(medusa_verify_mode mode, int B, int V, const medusa_tree* tree) {
+    if (!tree || B < 1 || V < 1) return 0;
+    return verify_workspace_size(mode, B, V, tree->host.T);
+}
+
+extern "C" int tree_verify(medusa_verify_mode mode, const void* target, medusa_dtype target_dt, const float* q,
+                           int q_rows, const int32_t* q_row, const int32_t* node_tokens, int B, int V,
+                           const medusa_tree* tree, uint64_t seed, uint32_t step, int32_t* accept_path, int max_path,
+                           int32_t* accept_len, int32_t* bonus, void* workspace, size_t workspace_bytes,
+                           int32_t* status, medusa_stream_t stream) {
+    if (mode != MEDUSA_VERIFY_GREEDY && mode != MEDUSA_VERIFY_STOCHASTIC)
+        return fail(MEDUSA_ERR_INVALID_ARG, "tree_verify: unknown mode");
+    if (!target || !node_tokens || !accept_path || !accept_len || !bonus)
+        return fail(MEDUSA_ERR_INVALID_ARG, "tree_verify: NULL tensor argument");
+    int rc = check_tree(tree);
+    if (rc) return rc;
+    const int T = tree->host.T;
+    if (B < 1 || V < 1) return fail(MEDUSA_ERR_INVALID_ARG, "tree_verify: bad sizes B=%d V=%d", B, V);
+    if (max_path < tree->host.max_depth || max_path > kMaxTree)
+        return fail(MEDUSA_ERR_INVALID_ARG, "tree_verify: max_path %d outside [tree depth %d, %d]", max_path,
+                    tree->host.max_depth, kMaxTree);
+    if (mode == MEDUSA_VERIFY_GREEDY) {
+        if (target_dt != MEDUSA_F32 && target_dt != MEDUSA_BF16)
+            return fail(MEDUSA_ERR_UNSUPPORTED, "tree_verify: greedy target dtype");
+        const size_t need = verify_workspace_size(mode, B, V, T);
+        if (!workspace || workspace_bytes < need || !al16(workspace))
+            return fail(MEDUSA_ERR_WORKSPACE, "tree_verify: workspace of %zu bytes, need %zu", workspace_bytes, need);
+    } else {
+        if (target_dt != MEDUSA_F32)
+            return fail(MEDUSA_ERR_UNSUPPORTED, "tree_verify: stochastic target p must be MEDUSA_F32");
+        if (!q) return fail(MEDUSA_ERR_INVALID_ARG, "tree_verify: stochastic mode needs q");
+        if (q_rows < 1 || (!q_row && q_rows != T))
+            return fail(MEDUSA_ERR_INVALID_ARG, "tree_verify: q_rows=%d (must equal T=%d without q_row)", q_rows, T);
+    }
+    VerifyArgs a;
+    a.mode = mode;
+    a.target = target;
+    a.target_dt = target_dt;
+    a.q = q;
+    a.q_rows = q_rows;
+    a.q_row = q_row;
+    a.node_tokens = node_tokens;
+    a.B = B;
+    a.V = V;
+    a.T = T;
+    a.tree = tree->dev;
+    a.seed = seed;
+    a.step = step;
+    a.accept_path = accept_path;
+    a.max_path = max_path;
+    a.accept_len = accept_len;
+    a.bonus = bonus;
+    a.ws = workspace;
+    a.ws_bytes = workspace_bytes;
+    a.status = status;
+    cudaError_t e = verify_launch(a, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "tree_verify launch");
+    return ok();
+}
+
+// ---------------------------------------------------------------------------
+// kv_commit
+// ---------------------------------------------------------------------------
+
+extern "C" int kv_commit(void* k_cache, void* v_cache, const void* k_tree, const void* v_tree,
+                         const int32_t* accept_path, int max_path, const int32_t* accept_len,
+                         const int32_t* prefix_len, int32_t* new_prefix_len, int B, int T, int Hkv, int D, int S_max,
+                         medusa_dtype dt, int32_t* status, medusa_stream_t stream) {
+    if (dt != MEDUSA_F32 && dt != MEDUSA_BF16) return fail(MEDUSA_ERR_UNSUPPORTED, "kv_commit: unknown dtype");
+    if (!k_cache || !v_cache || !k_tree || !v_tree || !accept_path || !accept_len || !prefix_len || !new_prefix_len)
+        return fail(MEDUSA_ERR_INVALID_ARG, "kv_commit: NULL tensor argument");
+    const int esize = dt == MEDUSA_BF16 ? 2 : 4;
+    if (B < 1 || T < 1 || T > kMaxTree || Hkv < 1 || D < 1 || S_max < 0 || max_path < 1 || max_path > kMaxTree)
+        return fail(MEDUSA_ERR_INVALID_ARG, "kv_commit: bad sizes B=%d T=%d Hkv=%d D=%d S_max=%d max_path=%d", B, T,
+                    Hkv, D, S_max, max_path);
+    if ((D * esize) % 16)
+        return fail(MEDUSA_ERR_INVALID_ARG, "kv_commit: a K/V row (%d bytes) must be a multiple of 16 bytes",
+                    D * esize);
+    if (!al16(k_cache) || !al16(v_cache) || !al16(k_tree) || !al16(v_tree))
+        return fail(MEDUSA_ERR_INVALID_ARG, "kv_commit: tensors must be 16-byte aligned");
+    CommitArgs a;
+    a.k_cache = k_cache;
+    a.v_cache = v_cache;
+    a.k_tree = k_tree;
+    a.v_tree = v_tree;
+    a.accept_path = accept_path;
+    a.max_path = max_path;
+    a.accept_len = accept_len;
+    a.prefix_len = prefix_len;
+    a.new_prefix_len = new_prefix_len;
+    a.B = B;
+    a.T = T;
+    a.Hkv = Hkv;
+    a.D = D;
+    a.S_max = S_max;
+    a.esize = esize;
+    a.status = status;
+    cudaError_t e = commit_launch(a, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "kv_commit launch");
+    return ok();
+}

@@ -1,0 +1,71 @@
+// KV commit on B200 ("Multi-Token Prediction & Draft-Model-Free Speculative
+// Decoding", sections "The 2D Tree Attention Mask" -- the longest accepted
+// path is committed -- and "Production Deployment Guidelines" -- unselected
+// branches are culled): the accepted path's K/V rows are appended to each
+// sequence's cache after its prefix.  One CTA per sequence; 16-byte copies.
+#include "kernels.h"
+
+namespace medusa {
+
+namespace {
+
+__global__ void __launch_bounds__(256) kv_commit_kernel(uint8_t* __restrict__ kc, uint8_t* __restrict__ vc,
+                                                        const uint8_t* __restrict__ kt, const uint8_t* __restrict__ vt,
+                                                        const int32_t* __restrict__ path, int max_path,
+                                                        const int32_t* __restrict__ len, const int32_t* prefix_len,
+                                                        int32_t* new_prefix_len, int T, int Hkv, int S_max,
+                                                        int row_bytes, int32_t* status) {
+    __shared__ int s_ok, s_S, s_L;
+    __shared__ int s_node[MEDUSA_MAX_TREE];
+    const int b = blockIdx.x, tid = threadIdx.x;
+    if (tid == 0) {
+        // read prefix_len before anything is written: new_prefix_len may alias it
+        const int S = prefix_len[b], L = len[b];
+        int ok = 1;
+        if (L < 0 || L > max_path || L > MEDUSA_MAX_TREE || S < 0) {
+            ok = 0;
+            set_status(status, MEDUSA_STATUS_BAD_TOKEN);
+        } else if (S + L > S_max) {
+            ok = 0;
+            set_status(status, MEDUSA_STATUS_CACHE_OVERFLOW);
+        }
+        for (int t = 0; ok && t < L; ++t) {
+            const int n = path[(long)b * max_path + t];
+            if (n < 0 || n >= T) {
+                ok = 0;
+                set_status(status, MEDUSA_STATUS_BAD_TOKEN);
+            }
+            s_node[t] = n;
+        }
+        s_ok = ok;
+        s_S = S;
+        s_L = L;
+    }
+    __syncthreads();
+    if (s_ok) {
+        const int vecs = row_bytes / 16;
+        const int per_t = Hkv * vecs;
+        for (int e = tid; e < s_L * per_t; e += blockDim.x) {
+            const int t = e / per_t, rem = e % per_t;
+            const int g = rem / vecs, c = rem % vecs;
+            const long src = (((long)b * T + s_node[t]) * Hkv + g) * row_bytes + c * 16;
+            const long dst = (((long)b * Hkv + g) * S_max + s_S + t) * row_bytes + c * 16;
+            *reinterpret_cast<uint4*>(kc + dst) = *reinterpret_cast<const uint4*>(kt + src);
+            *reinterpret_cast<uint4*>(vc + dst) = *reinterpret_cast<const uint4*>(vt + src);
+        }
+    }
+    __syncthreads();
+    if (tid == 0) new_prefix_len[b] = s_ok ? s_S + s_L : s_S;
+}
+
+}  // namespace
+
+cudaError_t commit_launch(const CommitArgs& a, cudaStream_t st) {
+    kv_commit_kernel<<<a.B, 256, 0, st>>>((uint8_t*)a.k_cache, (uint8_t*)a.v_cache, (const uint8_t*)a.k_tree,
+                                          (const uint8_t*)a.v_tree, a.accept_path, a.max_path, a.accept_len,
+                                          a.prefix_len, a.new_prefix_len, a.T, a.Hkv, a.S_max, a.D * a.esize,
+                                          a.status);
+    return cudaGetLastError();
+}
+
+}  // namespace medusa

@@ -1,0 +1,103 @@
+// Shared device-side definitions of libmedusa (B200, sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "medusa.h"
+
+namespace medusa {
+
+constexpr int kMaxTree = MEDUSA_MAX_TREE;  // nodes per tree
+constexpr int kTopK = MEDUSA_TOPK;         // entries kept per head
+constexpr unsigned kFull = 0xffffffffu;
+
+// Candidate tree as the kernels read it (device memory, built once by
+// medusa_tree_create).  Children of a node are child_idx[child_off[u] ..
+// child_off[u+1]) in increasing index order.  anc[i] has bit j set when node j
+// is node i or one of its ancestors (the tree attention mask row of node i).
+struct TreeDev {
+    int T;
+    int max_depth;
+    int max_children;
+    int pad;
+    int16_t parent[kMaxTree];
+    uint8_t depth[kMaxTree];
+    uint8_t rank[kMaxTree];
+    uint8_t child_off[kMaxTree + 4];
+    uint8_t child_idx[kMaxTree];
+    uint32_t anc[kMaxTree][4];
+};
+
+// ---------------------------------------------------------------------------
+// small helpers
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(kFull, x, o);
+    return x;
+}
+
+// 16-byte streaming load of read-only data that is used once (weights):
+// bypasses L1 allocation and asks L2 for 256-byte sectors.
+__device__ __forceinline__ uint4 ld_stream(const void* p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+// 16-byte read-only load that may stay in L1 (small vectors reused by a CTA).
+__device__ __forceinline__ uint4 ld_nc(const void* p) {
+    uint4 r;
+    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// Element-type traits: number of elements in 16 bytes and conversions.
+template <typename T>
+struct Elt;
+template <>
+struct Elt<float> {
+    static constexpr int kVec = 4;
+    __device__ __forceinline__ static void unpack(const uint4& v, float* f) {
+        f[0] = __uint_as_float(v.x);
+        f[1] = __uint_as_float(v.y);
+        f[2] = __uint_as_float(v.z);
+        f[3] = __uint_as_float(v.w);
+    }
+    __device__ __forceinline__ static float to_float(float x) { return x; }
+    __device__ __forceinline__ static float from_float(float x) { return x; }
+};
+template <>
+struct Elt<__nv_bfloat16> {
+    static constexpr int kVec = 8;
+    __device__ __forceinline__ static void unpack(const uint4& v, float* f) {
+        f[0] = bf16lo(v.x);
+        f[1] = bf16hi(v.x);
+        f[2] = bf16lo(v.y);
+        f[3] = bf16hi(v.y);
+        f[4] = bf16lo(v.z);
+        f[5] = bf16hi(v.z);
+        f[6] = bf16lo(v.w);
+        f[7] = bf16hi(v.w);
+    }
+    __device__ __forceinline__ static float to_float(__nv_bfloat16 x) { return __bfloat162float(x); }
+    __device__ __forceinline__ static __nv_bfloat16 from_float(float x) { return __float2bfloat16_rn(x); }
+};
+
+__device__ __forceinline__ void set_status(int32_t* status, int bits) {
+    if (status) atomicOr(status, bits);
+}
+
+// Total order of (value, index) candidates used by top-s and argmax: a larger
+// value wins; among equal values the lower index wins; NaN never wins.
+__device__ __forceinline__ bool beats(float v, int i, float w, int j) { return v > w || (v == w && i < j); }
+
+}  // namespace medusa

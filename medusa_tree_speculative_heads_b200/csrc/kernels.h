@@ -1,0 +1,101 @@
+// Internal launch interface between the C ABI (abi.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace medusa {
+
+// ------------------------------- heads -------------------------------------
+struct HeadsArgs {
+    const void* h;
+    const void* W_res;
+    const void* W_head;
+    int B, d, V, K;
+    medusa_dtype dt;
+    const TreeDev* tree;  // device, nullable
+    int T;
+    const int32_t* root_token;
+    int32_t* topk_idx;
+    float* topk_prob;
+    int32_t* node_tokens;
+    float* node_q;
+    void* h_res_out;
+    float* logits_out;
+    float* probs_out;
+    void* ws;
+    size_t ws_bytes;
+    int32_t* status;
+};
+size_t heads_workspace_size(int B, int d, int V, int K, medusa_dtype dt);
+cudaError_t heads_launch(const HeadsArgs& a, cudaStream_t st);
+
+// ------------------------------ attention ----------------------------------
+struct AttnArgs {
+    const void* q;
+    const void* k_tree;
+    const void* v_tree;
+    const void* k_cache;
+    const void* v_cache;
+    const int32_t* prefix_len;
+    int B, T, Hq, Hkv, D, S_max, max_prefix;
+    float scale;
+    medusa_dtype dt;
+    const TreeDev* tree;
+    void* out;
+    float* lse;
+    void* ws;
+    size_t ws_bytes;
+    int32_t* status;
+};
+size_t attn_workspace_size(int B, int T, int Hq, int Hkv, int D, int max_prefix, medusa_dtype dt);
+cudaError_t attn_launch(const AttnArgs& a, cudaStream_t st);
+
+// ------------------------------- verify ------------------------------------
+struct VerifyArgs {
+    medusa_verify_mode mode;
+    const void* target;
+    medusa_dtype target_dt;
+    const float* q;
+    int q_rows;
+    const int32_t* q_row;
+    const int32_t* node_tokens;
+    int B, V, T;
+    const TreeDev* tree;
+    uint64_t seed;
+    uint32_t step;
+    int32_t* accept_path;
+    int max_path;
+    int32_t* accept_len;
+    int32_t* bonus;
+    void* ws;
+    size_t ws_bytes;
+    int32_t* status;
+};
+size_t verify_workspace_size(medusa_verify_mode mode, int B, int V, int T);
+cudaError_t verify_launch(const VerifyArgs& a, cudaStream_t st);
+
+// ------------------------------- commit ------------------------------------
+struct CommitArgs {
+    void* k_cache;
+    void* v_cache;
+    const void* k_tree;
+    const void* v_tree;
+    const int32_t* accept_path;
+    int max_path;
+    const int32_t* accept_len;
+    const int32_t* prefix_len;
+    int32_t* new_prefix_len;
+    int B, T, Hkv, D, S_max, esize;
+    int32_t* status;
+};
+cudaError_t commit_launch(const CommitArgs& a, cudaStream_t st);
+
+// device properties, cached per device
+int num_sms();
+size_t align256(size_t x);
+
+}  // namespace medusa

@@ -1,0 +1,73 @@
+"""Host-side checks of the C ABI that need no GPU: the library builds, loads
+and exports every function include/medusa.h declares, and argument errors
+are reported by return code before anything reaches the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from medusa_tree_speculative_heads_b200 import binding as B
+from medusa_tree_speculative_heads_b200 import build as build_mod
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_mod.build()
+    return B.lib()
+
+
+def test_header_declares_the_four_step_calls():
+    names = B.declared_functions()
+    for n in ("medusa_heads", "tree_attention", "tree_verify", "kv_commit", "medusa_tree_create",
+              "medusa_tree_destroy", "medusa_last_error"):
+        assert n in names, n
+
+
+def test_library_exports_every_declared_symbol(lib):
+    missing = [n for n in B.declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+    assert lib.medusa_version() == 100
+
+
+def test_sm100a_only():
+    src = open(build_mod.__file__).read()
+    assert "arch=compute_100a,code=sm_100a" in src
+
+
+def test_tree_create_rejects_bad_parents(lib):
+    h = ctypes.c_void_p()
+    for parents, code in (([0, 0], B.MEDUSA_ERR_INVALID_ARG), ([-1, 1], B.MEDUSA_ERR_INVALID_ARG),
+                          ([-1, 0, -1], B.MEDUSA_ERR_INVALID_ARG), ([-1, 0, 5], B.MEDUSA_ERR_INVALID_ARG),
+                          ([-1] + list(range(128)), B.MEDUSA_ERR_UNSUPPORTED)):
+        arr = (ctypes.c_int32 * len(parents))(*parents)
+        assert lib.medusa_tree_create(arr, len(parents), ctypes.byref(h)) == code
+        assert lib.medusa_last_error()
+    assert lib.medusa_tree_create(None, 3, ctypes.byref(h)) == B.MEDUSA_ERR_INVALID_ARG
+
+
+def test_null_and_size_errors_before_launch(lib):
+    # no tensor touches the device: every one of these fails validation first
+    assert lib.medusa_heads(None, None, None, 1, 8, 8, 1, 1, None, None, None, None, None, None, None, None, None,
+                            None, 0, None, None) == B.MEDUSA_ERR_INVALID_ARG
+    assert b"NULL" in lib.medusa_last_error()
+    fake = ctypes.c_void_p(0x1000)
+    assert lib.medusa_heads(fake, fake, fake, 1, 12, 8, 1, 1, None, None, fake, fake, None, None, None, None, None,
+                            fake, 1 << 30, None, None) == B.MEDUSA_ERR_INVALID_ARG  # d % 8 != 0 for bf16
+    assert lib.medusa_heads(fake, fake, fake, 1, 16, 8, 1, 7, None, None, fake, fake, None, None, None, None, None,
+                            fake, 1 << 30, None, None) == B.MEDUSA_ERR_UNSUPPORTED  # unknown dtype
+    assert lib.medusa_heads(fake, fake, fake, 1, 16, 8, 1, 1, None, None, fake, fake, None, None, None, None, None,
+                            fake, 16, None, None) == B.MEDUSA_ERR_WORKSPACE
+    assert lib.tree_attention(None, None, None, None, None, None, 1, 4, 4, 64, 64, 0, 0.0, 1, None, None, None, None,
+                              0, None, None) == B.MEDUSA_ERR_INVALID_ARG
+    assert lib.tree_verify(0, None, 1, None, 0, None, None, 1, 8, None, 0, 0, None, 1, None, None, None, 0, None,
+                           None) == B.MEDUSA_ERR_INVALID_ARG
+    assert lib.kv_commit(fake, fake, fake, fake, fake, 1, fake, fake, fake, 1, 7, 2, 12, 16, 1, None,
+                         None) == B.MEDUSA_ERR_INVALID_ARG  # a 24-byte row is not a multiple of 16
+
+
+def test_workspace_queries_are_pure(lib):
+    a = lib.medusa_heads_workspace_size(1, 4096, 128256, 4, 1)
+    b = lib.medusa_heads_workspace_size(1, 4096, 128256, 4, 1)
+    assert a == b and a > 0
+    assert lib.medusa_heads_workspace_size(0, 4096, 128256, 4, 1) == 0

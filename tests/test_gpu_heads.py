@@ -1,0 +1,110 @@
+"""medusa_heads on the GPU against the fp64 oracle (same seeded inputs)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from helpers import assert_float_parity, check_topk, float_tol
+from medusa_tree_speculative_heads_b200 import api
+from medusa_tree_speculative_heads_b200 import inputs as I
+from medusa_tree_speculative_heads_b200.binding import Tree
+
+pytestmark = pytest.mark.gpu
+
+
+def run_case(w, parents):
+    inp = I.head_inputs(w)
+    ref = oracle.heads(inp["h"], inp["W_res"], inp["W_head"])
+    dev = {k: v.cuda() for k, v in inp.items()}
+    tree = Tree(parents) if parents is not None else None
+    out = api.heads(dev["h"], dev["W_res"], dev["W_head"], tree, dev["root_token"], want_logits=True,
+                    want_probs=True, want_hres=True)
+    # the same call without the optional outputs must give the same discrete results
+    out2 = api.heads(dev["h"], dev["W_res"], dev["W_head"], tree, dev["root_token"])
+    torch.cuda.synchronize()
+    return inp, ref, out, out2
+
+
+def check(w, parents, inp, ref, out, out2):
+    dt = w.torch_dtype
+    tol = float_tol(dt)
+    assert int(out["status"].item()) == 0
+    assert_float_parity(out["logits"], ref["logits"], dt, "logits")
+    assert_float_parity(out["probs"], ref["probs"], dt, "probs")
+    # h^(k): fp32, or bf16 storage (round to nearest: |err| <= 2^-8 |x|)
+    hres = out["h_res"].float().cpu().numpy()
+    if dt == torch.float32:
+        assert np.abs(hres - ref["hk"]).max() <= tol
+    else:
+        assert (np.abs(hres - ref["hk"]) <= 2.0 ** -8 * np.abs(ref["hk"]) + 1e-4).all()
+    ti = out["topk_idx"].cpu().numpy()
+    tp = out["topk_prob"].cpu().numpy()
+    B, K = ti.shape[:2]
+    s = min(8, w.V)
+    mismatches = 0
+    for b in range(B):
+        for k in range(K):
+            mismatches += check_topk(ti[b, k, :s], ref["logits"][b, k], tol)
+            assert (ti[b, k, s:] == -1).all()
+            np.testing.assert_allclose(tp[b, k, :s], ref["probs"][b, k, ti[b, k, :s]], rtol=0, atol=tol)
+    # decisions in the kernel's own precision: the list is the stable sort of
+    # the kernel's own fp32 logits (largest first, lower id on ties)
+    order = torch.sort(-out["logits"], dim=-1, stable=True).indices[..., :s].to(torch.int32)
+    assert torch.equal(order, out["topk_idx"][..., :s])
+    assert torch.equal(out["topk_idx"], out2["topk_idx"])
+    assert torch.equal(out["topk_prob"], out2["topk_prob"])
+    if parents is not None:
+        nt = out["node_tokens"].cpu().numpy()
+        assert torch.equal(out["node_tokens"], out2["node_tokens"])
+        depth, rank = oracle.tree_shape(parents)
+        for b in range(B):
+            assert nt[b, 0] == int(inp["root_token"][b])
+            for i in range(1, len(parents)):
+                assert nt[b, i] == ti[b, depth[i] - 2, rank[i]]
+        if mismatches == 0:
+            otop = np.stack([np.stack([oracle.topk(ref["logits"][b, k], 8) for k in range(K)]) for b in range(B)])
+            otok, oq = oracle.tree_fill(parents, inp["root_token"], otop,
+                                        np.take_along_axis(ref["probs"], np.maximum(otop, 0), axis=-1))
+            assert np.array_equal(nt, otok)
+            np.testing.assert_allclose(out["node_q"].cpu().numpy(), oq, rtol=0, atol=tol)
+    return mismatches
+
+
+@pytest.mark.parametrize("name,kw,tree", [
+    ("tiny", {}, "workload"),                                           # fp32, d=256, V=1024, (2,2)
+    ("tiny", dict(d=1024, V=5003, K=3), (3, 2, 1)),                     # fp32, ragged V
+    ("llama8b", dict(d=512, V=3001, K=3), (3, 2, 1)),                   # bf16 register path, ragged V
+    ("llama8b", dict(B=3, d=256, V=2000, K=2), (4, 2)),                 # bf16, several sequences
+    ("llama8b", dict(B=10, d=128, V=700, K=2), (2, 2)),                 # two sequence groups (8 + 2)
+    ("llama8b", dict(d=8192, V=1500, K=1), (4,)),                       # d too wide for registers
+    ("llama8b", dict(d=64, V=5, K=2), (3, 2)),                          # V < 8: missing entries are -1
+])
+def test_heads_parity(name, kw, tree):
+    w = I.scaled(I.WORKLOADS[name], **kw)
+    parents = I.workload_tree(w) if tree == "workload" else I.product_tree_parents(tree)
+    inp, ref, out, out2 = run_case(w, parents)
+    check(w, parents, inp, ref, out, out2)
+
+
+def test_heads_parity_llama8b_full_size():
+    # the 8B-shaped workload at full size: d=4096, V=128256, K=4, 117 nodes
+    w = I.WORKLOADS["llama8b"]
+    parents = I.workload_tree(w)
+    inp, ref, out, out2 = run_case(w, parents)
+    mism = check(w, parents, inp, ref, out, out2)
+    assert mism <= 2
+
+
+def test_heads_without_tree():
+    w = I.scaled(I.WORKLOADS["llama8b"], d=256, V=999, K=2)
+    inp, ref, out, out2 = run_case(w, None)
+    check(w, None, inp, ref, out, out2)
+
+
+def test_heads_rejects_deep_tree():
+    w = I.scaled(I.WORKLOADS["tiny"], d=64, V=64, K=1)
+    inp = {k: v.cuda() for k, v in I.head_inputs(w).items()}
+    tree = Tree(I.product_tree_parents((2, 2)))
+    from medusa_tree_speculative_heads_b200.binding import MedusaError
+    with pytest.raises(MedusaError):
+        api.heads(inp["h"], inp["W_res"], inp["W_head"], tree, inp["root_token"])

@@ -1,0 +1,54 @@
+"""One whole decode step (heads -> tree -> attention -> verify -> commit) on
+the GPU against the same step run by the oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from helpers import assert_float_parity, check_topk, float_tol
+from medusa_tree_speculative_heads_b200 import inputs as I
+from medusa_tree_speculative_heads_b200.api import MedusaStep
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("name", ["tiny", "llama8b"])
+def test_whole_step_matches_oracle(name):
+    w = I.WORKLOADS[name]
+    parents = I.workload_tree(w)
+    T = len(parents)
+    hin = I.head_inputs(w)
+    ain = I.attention_inputs(w, T)
+    # ---- oracle step ----
+    ref = oracle.heads(hin["h"], hin["W_res"], hin["W_head"], want_hk=False)
+    otop = np.stack([np.stack([oracle.topk(ref["logits"][b, k], 8) for k in range(w.K)]) for b in range(w.B)])
+    otok, _ = oracle.tree_fill(parents, hin["root_token"], otop,
+                               np.take_along_axis(ref["probs"], otop, axis=-1))
+    logits = I.boosted_target_logits(w, parents, torch.from_numpy(otok))
+    o_att, _ = oracle.tree_attention(ain["q"], ain["k_tree"], ain["v_tree"], ain["k_cache"], ain["v_cache"],
+                                     ain["prefix_len"], parents)
+    maxd = int(max(oracle.tree_shape(parents)[0]))
+    opath, olen, obonus = oracle.verify_greedy(logits, otok, parents, maxd)
+    okc, ovc, onpl, ost = oracle.kv_commit(ain["k_cache"], ain["v_cache"], ain["k_tree"], ain["v_tree"], opath, olen,
+                                           ain["prefix_len"])
+    # ---- GPU step ----
+    d = {k: v.cuda() for k, v in {**hin, **ain}.items()}
+    st = MedusaStep(B=w.B, d=w.d, V=w.V, K=w.K, Hq=w.Hq, Hkv=w.Hkv, D=w.D, S_max=w.S_max, parents=parents,
+                    dtype=w.torch_dtype, max_prefix=w.max_prefix)
+    new_pl = torch.empty_like(d["prefix_len"])
+    st.run(h=d["h"], W_res=d["W_res"], W_head=d["W_head"], root_token=d["root_token"], q=d["q"], k_tree=d["k_tree"],
+           v_tree=d["v_tree"], k_cache=d["k_cache"], v_cache=d["v_cache"], prefix_len=d["prefix_len"],
+           new_prefix_len=new_pl, target=logits.cuda())
+    torch.cuda.synchronize()
+    assert int(st.status.item()) == 0
+    ti = st.topk_idx.cpu().numpy()
+    mism = sum(check_topk(ti[b, k], ref["logits"][b, k], float_tol(w.torch_dtype)) for b in range(w.B)
+               for k in range(w.K))
+    assert_float_parity(st.attn_out.float().cpu().reshape(-1, w.D), o_att, w.torch_dtype, "attention")
+    if mism == 0:
+        assert np.array_equal(st.node_tokens.cpu().numpy(), otok)
+        assert np.array_equal(st.accept_path.cpu().numpy(), opath)
+        assert np.array_equal(st.accept_len.cpu().numpy(), olen)
+        assert np.array_equal(st.bonus.cpu().numpy(), obonus)
+        assert np.array_equal(new_pl.cpu().numpy(), onpl)
+        assert torch.equal(d["k_cache"].cpu(), okc) and torch.equal(d["v_cache"].cpu(), ovc)

@@ -1,0 +1,138 @@
+"""tree_verify on the GPU against the oracle: bit-exact paths, lengths and
+bonus tokens on identical logits / probabilities and Philox counters."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from medusa_tree_speculative_heads_b200 import api
+from medusa_tree_speculative_heads_b200 import binding as B
+from medusa_tree_speculative_heads_b200 import inputs as I
+from medusa_tree_speculative_heads_b200.binding import Tree
+
+pytestmark = pytest.mark.gpu
+
+
+def greedy_case(w, parents, seed_offset=0):
+    tok = I.random_node_tokens(w, parents, seed_offset)
+    logits = I.boosted_target_logits(w, parents, tok, seed_offset=seed_offset)
+    return tok, logits
+
+
+def run_greedy(parents, tok, logits):
+    tree = Tree(parents)
+    out = api.tree_verify(B.GREEDY, logits.cuda(), tok.cuda(), tree)
+    torch.cuda.synchronize()
+    return out
+
+
+def assert_same(out, ref):
+    path, ln, bonus = ref[:3]
+    assert np.array_equal(out["accept_len"].cpu().numpy(), ln)
+    assert np.array_equal(out["accept_path"].cpu().numpy(), path)
+    assert np.array_equal(out["bonus"].cpu().numpy(), bonus)
+
+
+@pytest.mark.parametrize("name,kw,tree", [
+    ("tiny", {}, "workload"),
+    ("llama8b", dict(B=4, V=1001), (4, 4, 2, 2)),      # rows not 16-byte aligned: scalar path
+    ("llama8b", dict(B=2), (4, 4, 2, 2)),              # full vocabulary, 117 nodes
+    ("llama70b_b8", dict(V=20000), (4, 4, 2, 2)),       # 8 sequences, match prob 0.7
+    ("stoch_b64", dict(B=6, V=5000), "workload"),       # random sparse tree
+])
+def test_greedy_parity(name, kw, tree):
+    w = I.scaled(I.WORKLOADS[name], **kw)
+    parents = I.workload_tree(w) if tree == "workload" else I.product_tree_parents(tree)
+    for off in range(3):
+        tok, logits = greedy_case(w, parents, off)
+        out = run_greedy(parents, tok, logits)
+        ref = oracle.verify_greedy(logits, tok, parents, max_path=max(oracle.tree_shape(parents)[0]))
+        assert_same(out, ref)
+
+
+def test_greedy_ties_nan_and_float32():
+    parents = [-1, 0, 0, 1]
+    V = 40
+    logits = torch.zeros((2, 4, V))
+    logits[0, 0, 7] = 3.0
+    logits[0, 0, 5] = 3.0                # tie: 5 wins
+    logits[0, 1, :] = float("nan")
+    logits[0, 1, 9] = 1.0                # NaN never wins
+    logits[1, :, :] = float("nan")       # all NaN: index 0
+    tok = torch.tensor([[1, 5, 7, 9], [1, 0, 0, 0]], dtype=torch.int32)
+    for dt in (torch.float32, torch.bfloat16):
+        out = run_greedy(parents, tok, logits.to(dt))
+        ref = oracle.verify_greedy(logits.to(dt), tok, parents, max_path=3)
+        assert_same(out, ref)
+        assert out["accept_len"].tolist() == [3, 3]
+
+
+def test_greedy_draft_equals_target_full_vocab():
+    w = I.scaled(I.WORKLOADS["llama8b"], B=2)
+    parents = I.workload_tree(w)
+    tok, logits = greedy_case(w, parents)
+    ch = I.tree_children(parents)
+    am = logits.float().argmax(-1)
+    for b in range(w.B):
+        for u in range(len(parents)):
+            if ch[u]:
+                tok[b, ch[u][0]] = am[b, u]
+    out = run_greedy(parents, tok, logits)
+    assert out["accept_len"].tolist() == [5, 5]
+    assert_same(out, oracle.verify_greedy(logits, tok, parents, max_path=5))
+
+
+def stoch_case(w, parents):
+    d = I.stochastic_inputs(w, parents)
+    return d["p"], d["q"], d["node_tokens"]
+
+
+def run_stoch(parents, p, q, tok, seed, step, q_row=None):
+    tree = Tree(parents)
+    out = api.tree_verify(B.STOCHASTIC, p.cuda(), tok.cuda(), tree, q=q.cuda(),
+                          q_row=None if q_row is None else torch.as_tensor(q_row, dtype=torch.int32).cuda(),
+                          seed=seed, step=step)
+    torch.cuda.synchronize()
+    return out
+
+
+@pytest.mark.parametrize("kw", [dict(B=8), dict(B=3, V=777), dict()])
+def test_stochastic_parity(kw):
+    w = I.scaled(I.WORKLOADS["stoch_b64"], **kw)
+    parents = I.workload_tree(w)
+    p, q, tok = stoch_case(w, parents)
+    maxd = int(max(oracle.tree_shape(parents)[0]))
+    for seed, step in ((0, 0), (0x123456789ABCDEF0, 17), (2**64 - 1, 2**32 - 1)):
+        out = run_stoch(parents, p, q, tok, seed, step)
+        ref = oracle.verify_stochastic(p, q, tok, parents, seed, step, maxd)
+        assert_same(out, ref)
+        assert int(out["status"].item()) == 0
+
+
+def test_stochastic_many_siblings_and_q_row():
+    # a wide product tree (many rejections per node), Medusa-style shared
+    # draft rows: q [B, K, V] with q_row[u] = depth(u) - 1
+    w = I.scaled(I.WORKLOADS["stoch_b64"], B=5, V=600)
+    parents = I.product_tree_parents((6, 3, 2))
+    p, q, tok = stoch_case(w, parents)
+    depth, _ = oracle.tree_shape(parents)
+    K = int(depth.max())
+    q_rows = q[:, :K].contiguous()
+    q_row = (depth - 1).astype(np.int32)
+    for step in range(4):
+        out = run_stoch(parents, p, q_rows, tok, 99, step, q_row=q_row)
+        ref = oracle.verify_stochastic(p, q_rows, tok, parents, 99, step, K, q_row=q_row)
+        assert_same(out, ref)
+
+
+def test_stochastic_draft_equals_target_accepts_first_children():
+    w = I.scaled(I.WORKLOADS["stoch_b64"], B=4)
+    parents = I.workload_tree(w)
+    p, q, tok = stoch_case(w, parents)
+    out = run_stoch(parents, p, p, tok, 3, 1)
+    ch = I.tree_children(parents)
+    chain = [0]
+    while ch[chain[-1]]:
+        chain.append(ch[chain[-1]][0])
+    for b in range(w.B):
+        assert out["accept_path"][b, : len(chain)].tolist() == chain
