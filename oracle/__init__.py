@@ -63,6 +63,8 @@ def lib():
         L.orc_kv_commit.restype = None
         L.orc_residual.argtypes = [vp, vp, i32, vp, vp]
         L.orc_residual.restype = u64
+        L.orc_round_bf16.argtypes = [dbl]
+        L.orc_round_bf16.restype = dbl
         _lib = L
     return _lib
 
@@ -152,6 +154,10 @@ def heads(h, W_res, W_head, b_only: int = -1, k_only: int = -1, want_hk=True, wa
     probs = np.full((B, K, V), np.nan) if want_probs else None
     lib().orc_heads(_p(hr), _p(wr), _p(wh), dt, B, d, V, K, b_only, k_only, _p(hk), _p(logits), _p(probs))
     return {"hk": hk, "logits": logits, "probs": probs}
+
+
+def round_bf16(x: float) -> float:
+    return lib().orc_round_bf16(float(x))
 
 
 def topk(x: np.ndarray, s: int) -> np.ndarray:

@@ -107,6 +107,23 @@ int orc_product_tree(const int32_t* s, int K, int32_t* parent, int cap) {
     return n;
 }
 
+/*
+ * Round a double to the nearest bf16 value (8 significant bits, ties to
+ * even), directly from the double so no intermediate rounding occurs.  Used
+ * for the bf16 storage of the residual block's output (see orc_heads).
+ */
+double orc_round_bf16(double x) {
+    if (x == 0.0 || x != x || isinf(x)) return x;
+    int e;
+    frexp(fabs(x), &e);              /* |x| = m 2^e, m in [0.5, 1) */
+    int qe = e - 8;                  /* quantum of 8 significant bits */
+    if (qe < -133) qe = -133;        /* bf16 subnormal spacing */
+    double q = ldexp(1.0, qe);
+    double r = nearbyint(x / q) * q; /* default rounding: to nearest, ties to even */
+    if (fabs(r) > 3.3895313892515355e38) r = x > 0 ? INFINITY : -INFINITY;
+    return r;
+}
+
 /* ------------------------------------------------------------------------ */
 /* Medusa heads                                                              */
 /* ------------------------------------------------------------------------ */
@@ -115,7 +132,11 @@ int orc_product_tree(const int32_t* s, int K, int32_t* parent, int cap) {
  * [GUIDE] "The Architectural Blueprint": for head k,
  *     h^(k) = SiLU(W_res^(k) h) + h,     p^(k) = softmax(W_head^(k) h^(k)),
  * with SiLU(z) = z * sigma(z), sigma(z) = 1 / (1 + e^-z).  No bias (the
- * formula has none).  Layouts: h [B,d]; W_res [K,d,d] (output row, input
+ * formula has none).  Reading on precision (the pages fix none): h^(k) is an
+ * activation of the model's dtype, so for bf16 inputs it is stored rounded
+ * to bf16 (from the exact fp64 value) before the vocabulary projection; the
+ * top-s decision is then taken on the same operand precision as a bf16
+ * kernel's.  Layouts: h [B,d]; W_res [K,d,d] (output row, input
  * column); W_head [K,V,d].  Outputs (each nullable): hk [B,K,d],
  * logits [B,K,V], probs [B,K,V].  Only sequence b_only / head k_only is
  * computed when those are >= 0 (others untouched).
@@ -136,6 +157,7 @@ void orc_heads(const void* h, const void* W_res, const void* W_head, int dtype,
                     z += load(W_res, dtype, ((size_t)k * d + o) * d + i) * load(h, dtype, (size_t)b * d + i);
                 double sig = 1.0 / (1.0 + exp(-z));
                 hk[o] = z * sig + load(h, dtype, (size_t)b * d + o);
+                if (dtype == ORC_BF16) hk[o] = orc_round_bf16(hk[o]);
             }
             /* projection to the vocabulary */
             for (int v = 0; v < V; ++v) {

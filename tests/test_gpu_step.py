@@ -42,13 +42,27 @@ def test_whole_step_matches_oracle(name):
     torch.cuda.synchronize()
     assert int(st.status.item()) == 0
     ti = st.topk_idx.cpu().numpy()
+    chain = dict(path=st.accept_path.cpu().numpy(), len=st.accept_len.cpu().numpy(), bonus=st.bonus.cpu().numpy(),
+                 npl=new_pl.cpu().numpy(), kc=d["k_cache"].cpu(), vc=d["v_cache"].cpu())
     mism = sum(check_topk(ti[b, k], ref["logits"][b, k], float_tol(w.torch_dtype)) for b in range(w.B)
                for k in range(w.K))
     assert_float_parity(st.attn_out.float().cpu().reshape(-1, w.D), o_att, w.torch_dtype, "attention")
+    # verify and commit on identical inputs: the oracle's node tokens
+    kc2, vc2 = ain["k_cache"].cuda(), ain["v_cache"].cuda()
+    pl2 = torch.empty_like(d["prefix_len"])
+    st.verify(logits.cuda(), node_tokens=torch.from_numpy(otok).cuda())
+    st.commit(kc2, vc2, d["k_tree"], d["v_tree"], d["prefix_len"], pl2)
+    torch.cuda.synchronize()
+    assert np.array_equal(st.accept_path.cpu().numpy(), opath)
+    assert np.array_equal(st.accept_len.cpu().numpy(), olen)
+    assert np.array_equal(st.bonus.cpu().numpy(), obonus)
+    assert np.array_equal(pl2.cpu().numpy(), onpl)
+    assert torch.equal(kc2.cpu(), okc) and torch.equal(vc2.cpu(), ovc)
+    # the GPU's own chain, when every top-s decision matched the oracle's
     if mism == 0:
         assert np.array_equal(st.node_tokens.cpu().numpy(), otok)
-        assert np.array_equal(st.accept_path.cpu().numpy(), opath)
-        assert np.array_equal(st.accept_len.cpu().numpy(), olen)
-        assert np.array_equal(st.bonus.cpu().numpy(), obonus)
-        assert np.array_equal(new_pl.cpu().numpy(), onpl)
-        assert torch.equal(d["k_cache"].cpu(), okc) and torch.equal(d["v_cache"].cpu(), ovc)
+        assert np.array_equal(chain["path"], opath)
+        assert np.array_equal(chain["len"], olen)
+        assert np.array_equal(chain["bonus"], obonus)
+        assert np.array_equal(chain["npl"], onpl)
+        assert torch.equal(chain["kc"], okc) and torch.equal(chain["vc"], ovc)

@@ -195,10 +195,48 @@ def test_heads_vs_numpy_matmul_and_softmax_sum(orc):
         np.testing.assert_allclose(r["hk"][:, k], hk, rtol=1e-13, atol=1e-13)
         np.testing.assert_allclose(r["logits"][:, k], lg, rtol=1e-12, atol=1e-12)
     np.testing.assert_allclose(r["probs"].sum(-1), 1.0, rtol=0, atol=1e-12)
-    # bf16 inputs are widened exactly: same result as the fp32 copy of them
-    rb = orc.heads(h.bfloat16(), W_res.bfloat16(), W_head.bfloat16())
-    rf = orc.heads(h.bfloat16().float(), W_res.bfloat16().float(), W_head.bfloat16().float())
+    # bf16 inputs are widened exactly: with W_res = 0, h^(k) = h is already a
+    # bf16 value, so the bf16 and fp32 copies give identical results
+    Z = torch.zeros_like(W_res)
+    rb = orc.heads(h.bfloat16(), Z.bfloat16(), W_head.bfloat16())
+    rf = orc.heads(h.bfloat16().float(), Z, W_head.bfloat16().float())
     np.testing.assert_array_equal(rb["logits"], rf["logits"])
+
+
+def test_round_bf16_ties_and_library(orc):
+    # 8 significant bits, ties to even: 1 + 2^-8 lies halfway between 1 and
+    # 1 + 2^-7 (odd mantissa) -> 1; 1 + 3 * 2^-8 lies between 1 + 2^-7 (odd)
+    # and 1 + 2^-6 (even) -> 1 + 2^-6
+    assert orc.round_bf16(1 + 2 ** -8) == 1.0
+    assert orc.round_bf16(1 + 3 * 2 ** -8) == 1 + 2 ** -6
+    assert orc.round_bf16(-(1 + 3 * 2 ** -8)) == -(1 + 2 ** -6)
+    assert orc.round_bf16(1 + 2 ** -8 + 2 ** -30) == 1 + 2 ** -7   # just above halfway
+    assert orc.round_bf16(0.0) == 0.0
+    # against torch's fp32 -> bf16 conversion (round to nearest even) on
+    # values exactly representable in fp32
+    x = torch.randn(20000, generator=torch.Generator().manual_seed(4)) * torch.logspace(-30, 30, 20000)
+    want = x.bfloat16().double().numpy()
+    got = np.array([orc.round_bf16(float(v)) for v in x.double().numpy()])
+    assert np.array_equal(got, want)
+
+
+def test_heads_bf16_stores_hk_as_bf16(orc):
+    # for bf16 inputs h^(k) is the bf16 rounding of the exact value, and the
+    # logits are the exact products with that rounded activation
+    g = torch.Generator().manual_seed(13)
+    B, d, V, K = 2, 32, 40, 2
+    h = torch.randn((B, d), generator=g).bfloat16()
+    W_res = (torch.randn((K, d, d), generator=g) / 4).bfloat16()
+    W_head = (torch.randn((K, V, d), generator=g) / 4).bfloat16()
+    r = orc.heads(h, W_res, W_head)
+    hn, Wr, Wh = h.double().numpy(), W_res.double().numpy(), W_head.double().numpy()
+    for k in range(K):
+        z = hn @ Wr[k].T
+        exact = z / (1 + np.exp(-z)) + hn
+        rounded = torch.from_numpy(exact).float().bfloat16().double().numpy()   # fp32 first: tiny double-rounding risk
+        assert (r["hk"][:, k] == rounded).mean() > 0.999
+        assert (np.abs(r["hk"][:, k] - exact) <= 2.0 ** -8 * np.abs(exact)).all()   # half an ulp of 8 bits
+        np.testing.assert_allclose(r["logits"][:, k], r["hk"][:, k] @ Wh[k].T, rtol=1e-12, atol=1e-12)
 
 
 def test_heads_subset_selection(orc):
