@@ -385,7 +385,13 @@ def main():
     ap.add_argument("--impl", default="mine", choices=["mine", "reference"])
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--override", action="append", default=[],
+                    help="replace a workload size, e.g. --override V=32000 (profiling a smaller case)")
     args = ap.parse_args()
+    from medusa_tree_speculative_heads_b200 import inputs as I
+    for ov in args.override:
+        key, val = ov.split("=")
+        I.WORKLOADS[args.workload] = I.scaled(I.WORKLOADS[args.workload], **{key: int(val)})
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
