@@ -148,6 +148,31 @@ int medusa_heads(const void* h, const void* W_res, const void* W_head, int B, in
                  float* probs_out, void* workspace, size_t workspace_bytes, int32_t* status,
                  medusa_stream_t stream);
 
+/*
+ * medusa_heads without a workspace argument (the pages have no counterpart:
+ * this is a library convenience, not part of the method).  For callers that
+ * cannot allocate device memory -- a plug-in inside a framework that owns all
+ * of the GPU's memory and offers it no allocator, or a loop that must never
+ * call cudaMalloc/cudaFree because they synchronise the device.  Same
+ * arguments and results as medusa_heads, minus workspace/workspace_bytes.
+ *   - Scratch is a fixed 32 MiB array inside the library's device code; every
+ *     GPU that loads the library holds it until the process exits.  Sizes
+ *     whose medusa_heads_workspace_size exceeds 32 MiB are rejected with
+ *     MEDUSA_ERR_UNSUPPORTED and a message; nothing is launched.
+ *   - The first call on each device looks up the array's device address (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture begins.
+ *   - The call itself allocates nothing (no cudaMalloc/cudaFree).
+ *   - Every call on a device shares the one array: calls whose work overlaps
+ *     on the GPU (different streams, or different host threads) race and
+ *     corrupt each other's results; serialise them.  No part of the scratch
+ *     needs to start at zero: each call writes every byte it later reads.
+ */
+int medusa_heads_noalloc(const void* h, const void* W_res, const void* W_head, int B, int d, int V, int K,
+                         medusa_dtype dt, const medusa_tree* tree, const int32_t* root_token, int32_t* topk_idx,
+                         float* topk_prob, int32_t* node_tokens, float* node_q, void* h_res_out, float* logits_out,
+                         float* probs_out, int32_t* status, medusa_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* Tree attention                                                            */
 /* ------------------------------------------------------------------------ */

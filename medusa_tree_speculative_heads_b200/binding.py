@@ -64,6 +64,8 @@ def lib() -> ctypes.CDLL:
         L.medusa_heads_workspace_size.restype = sz
         L.medusa_heads.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
                                    vp, vp]
+        L.medusa_heads_noalloc.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp,
+                                           vp, vp, vp]
         L.tree_attention_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32, vp, i32]
         L.tree_attention_workspace_size.restype = sz
         L.tree_attention.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, i32, vp, vp, vp, vp,
@@ -150,6 +152,15 @@ def medusa_heads(h, W_res, W_head, B, d, V, K, dt, tree: Optional[Tree], root_to
                               _p(root_token), _p(topk_idx), _p(topk_prob), _p(node_tokens), _p(node_q),
                               _p(h_res_out), _p(logits_out), _p(probs_out), _p(workspace), workspace_bytes,
                               _p(status), _stream(stream)))
+
+
+def medusa_heads_noalloc(h, W_res, W_head, B, d, V, K, dt, tree: Optional[Tree], root_token, topk_idx, topk_prob,
+                         node_tokens, node_q, h_res_out, logits_out, probs_out, status, stream=None):
+    """medusa_heads for callers that cannot allocate device memory: the
+    scratch is a fixed array inside the library (see include/medusa.h)."""
+    _check(lib().medusa_heads_noalloc(_p(h), _p(W_res), _p(W_head), B, d, V, K, dt, tree.handle if tree else None,
+                                      _p(root_token), _p(topk_idx), _p(topk_prob), _p(node_tokens), _p(node_q),
+                                      _p(h_res_out), _p(logits_out), _p(probs_out), _p(status), _stream(stream)))
 
 
 def tree_attention_workspace_size(B, Hq, Hkv, D, S_max, max_prefix, tree: Tree, dt) -> int:

@@ -53,6 +53,9 @@ int check_tree(const medusa_tree* t) {
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
+// lets other translation units set this thread's last-error message
+int report_error(int code, const char* msg) { return fail(code, "%s", msg); }
+
 int num_sms() {
     static int cache[64] = {0};
     int dev = 0;
