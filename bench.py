@@ -196,8 +196,15 @@ def config_dict(w, world):
 
 
 def launches_per_step(w, mode_greedy=True):
-    groups = (w.B + 7) // 8
-    heads = 1 + 2 * groups
+    """Library kernels per step: medusa_heads is one cooperative kernel on the
+    bf16 tensor-core path (B <= 64); otherwise residual + per-8-sequence LM
+    and merge kernels."""
+    if w.dtype == "bf16" and w.B <= 64 and w.d % 8 == 0:
+        heads = 1
+    elif w.B == 1:
+        heads = 1
+    else:
+        heads = 1 + 2 * ((w.B + 7) // 8)
     attn = 2 if w.dtype == "bf16" else 1
     verify = 2 if mode_greedy else 1
     return heads + attn + verify + 1

@@ -65,7 +65,8 @@ enum {
     MEDUSA_STATUS_BAD_TOKEN = 1,      /* a token / node id outside its range */
     MEDUSA_STATUS_CACHE_OVERFLOW = 2, /* kv_commit: prefix_len + len > S_max */
     MEDUSA_STATUS_BAD_PREFIX = 4,     /* prefix_len outside [0, max_prefix] */
-    MEDUSA_STATUS_NO_MASS = 8         /* stochastic bonus drawn from an all-zero distribution */
+    MEDUSA_STATUS_NO_MASS = 8,        /* stochastic bonus drawn from an all-zero distribution */
+    MEDUSA_STATUS_TIMEOUT = 16        /* an internal pipeline wait gave up after ~2 s (a library bug) */
 };
 
 typedef enum { MEDUSA_F32 = 0, MEDUSA_BF16 = 1 } medusa_dtype;

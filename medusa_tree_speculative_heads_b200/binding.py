@@ -30,6 +30,7 @@ STATUS_BAD_TOKEN = 1
 STATUS_CACHE_OVERFLOW = 2
 STATUS_BAD_PREFIX = 4
 STATUS_NO_MASS = 8
+STATUS_TIMEOUT = 16
 
 F32, BF16 = 0, 1
 GREEDY, STOCHASTIC = 0, 1

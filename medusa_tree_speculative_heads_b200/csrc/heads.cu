@@ -15,6 +15,7 @@
 #include <float.h>
 #include <limits.h>
 
+#include "heads_common.cuh"
 #include "kernels.h"
 
 namespace medusa {
@@ -25,95 +26,6 @@ constexpr int kResWarps = 8;   // warps per block of the residual kernel
 constexpr int kLmWarps = 8;    // warps per block of the LM-head kernel
 constexpr int kBG = 8;         // sequences handled per LM-head launch
 constexpr int kUnroll = 8;     // 16-byte loads issued back to back per lane
-
-// Running softmax statistics and top-8 list of one (sequence, head) over a
-// set of vocabulary rows: m = max logit, l = sum exp(logit - m).
-struct HeadState {
-    float m, l;
-    float val[kTopK];
-    int idx[kTopK];
-};
-
-__device__ __forceinline__ HeadState empty_state() {
-    HeadState s;
-    s.m = -INFINITY;
-    s.l = 0.f;
-#pragma unroll
-    for (int j = 0; j < kTopK; ++j) {
-        s.val[j] = -INFINITY;
-        s.idx[j] = INT_MAX;
-    }
-    return s;
-}
-
-// merge softmax statistics (m2, l2) into (m, l)
-__device__ __forceinline__ void merge_ml(float& m, float& l, float m2, float l2) {
-    if (m2 == -INFINITY) return;
-    if (m == -INFINITY) {
-        m = m2;
-        l = l2;
-        return;
-    }
-    float mn = fmaxf(m, m2);
-    l = l * expf(m - mn) + l2 * expf(m2 - mn);
-    m = mn;
-}
-
-// Insert (v, i) into a register-resident list sorted best-first.
-__device__ __forceinline__ void list_insert(float (&lv)[kTopK], int (&li)[kTopK], float v, int i) {
-    if (!beats(v, i, lv[kTopK - 1], li[kTopK - 1])) return;
-    lv[kTopK - 1] = v;
-    li[kTopK - 1] = i;
-#pragma unroll
-    for (int j = kTopK - 1; j > 0; --j) {
-        if (beats(lv[j], li[j], lv[j - 1], li[j - 1])) {
-            float tv = lv[j];
-            lv[j] = lv[j - 1];
-            lv[j - 1] = tv;
-            int ti = li[j];
-            li[j] = li[j - 1];
-            li[j - 1] = ti;
-        }
-    }
-}
-
-// Warp-wide selection of the best kTopK candidates from per-lane sorted
-// lists.  Lane j < kTopK receives the j-th best in (out_v, out_i).
-__device__ __forceinline__ void warp_select(float (&lv)[kTopK], int (&li)[kTopK], float& out_v, int& out_i) {
-    const int lane = threadIdx.x & 31;
-    out_v = -INFINITY;
-    out_i = INT_MAX;
-#pragma unroll 1
-    for (int r = 0; r < kTopK; ++r) {
-        float wv = lv[0];
-        int wi = li[0];
-        int wl = lane;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            float ov = __shfl_xor_sync(kFull, wv, o);
-            int oi = __shfl_xor_sync(kFull, wi, o);
-            int ol = __shfl_xor_sync(kFull, wl, o);
-            if (beats(ov, oi, wv, wi) || (ov == wv && oi == wi && ol < wl)) {
-                wv = ov;
-                wi = oi;
-                wl = ol;
-            }
-        }
-        if (lane == r) {
-            out_v = wv;
-            out_i = wi;
-        }
-        if (lane == wl) {  // pop the head of the winning lane's list
-#pragma unroll
-            for (int j = 0; j < kTopK - 1; ++j) {
-                lv[j] = lv[j + 1];
-                li[j] = li[j + 1];
-            }
-            lv[kTopK - 1] = -INFINITY;
-            li[kTopK - 1] = INT_MAX;
-        }
-    }
-}
 
 // ---------------------------------------------------------------------------
 // K1: residual block.  One warp per output feature (k, o); the W_res row is
@@ -371,10 +283,331 @@ __global__ void __launch_bounds__(kLmWarps * 32) heads_lm_kernel(const T* __rest
 }
 
 // ---------------------------------------------------------------------------
-// K3: merge the CTAs' partials of one (sequence, head) in a fixed order,
-// write the top-8 entries with their probabilities and the head's softmax
-// statistics, and fill the tree nodes this head proposes.
+// Fused heads for one sequence (rows of <= 8 KB): a persistent cooperative
+// kernel, one CTA per SM, that runs the whole medusa_heads call.
+//   - A producer thread streams contiguous chunks of weight rows into a ring
+//     of kFStages shared-memory stages with bulk asynchronous copies (192 KB
+//     in flight per SM, independent of register pressure): first the CTA's
+//     slice of W_res rows, then, without a break, its slice of W_head rows.
+//   - kFC consumer warps dot each row with the vector held in registers:
+//     phase 1 writes h^(k) = SiLU(W_res h) + h; after a grid-wide barrier
+//     (all of h^(k) written; the producer keeps prefetching W_head meanwhile)
+//     phase 2 computes logits and keeps running softmax statistics and a
+//     top-8 list per head.
+//   - Each CTA merges its warps into one partial per head; the last CTA to
+//     finish merges all partials (in CTA order) and fills the tree.
+// Every wait -- ring barriers and the grid barrier -- gives up after ~2 s and
+// sets MEDUSA_STATUS_TIMEOUT instead of hanging.
 // ---------------------------------------------------------------------------
+#ifndef MEDUSA_FC
+#define MEDUSA_FC 6
+#endif
+#ifndef MEDUSA_FSTAGES
+#define MEDUSA_FSTAGES 4
+#endif
+constexpr int kFC = MEDUSA_FC;           // consumer warps (+1 producer warp)
+constexpr int kFStages = MEDUSA_FSTAGES; // ring depth
+constexpr int kRowCap = 8192;    // largest weight row (bytes) the fused kernel takes
+
+struct FusedArgs {
+    const void* h;
+    const void* W_res;
+    const void* W_head;
+    int d, V, K;
+    void* hk;
+    void* hk_out;
+    float* logits;
+    HeadState* part;     // [grid][K][kBG]
+    unsigned int* ctr;   // [2], zero at launch: grid-barrier arrivals, CTAs done
+    const TreeDev* tree;
+    const int32_t* root_token;
+    int32_t* topk_idx;
+    float* topk_prob;
+    int32_t* node_tokens;
+    float* node_q;
+    float2* stats;
+    int32_t* status;
+};
+
+size_t fused_smem_bytes(int row_bytes, int K) {
+    const int rpw = kRowCap / row_bytes;
+    return (size_t)kFStages * kFC * rpw * row_bytes + 2 * kFStages * sizeof(uint64_t) +
+           (size_t)kFC * K * sizeof(HeadState) + 16;
+}
+
+__device__ __forceinline__ uint4 ld_cg(const void* p) {
+    uint4 r;
+    asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ void consumers_sync() { asm volatile("bar.sync 1, %0;" ::"r"(kFC * 32) : "memory"); }
+
+template <typename T>
+__global__ void __launch_bounds__((kFC + 1) * 32, 1) heads_fused_kernel(const __grid_constant__ FusedArgs a) {
+    constexpr int VEC = Elt<T>::kVec;
+    constexpr int NXV = kRowCap / 16 / 32;  // 16-byte pieces of a row per lane
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ int s_flag;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int row_bytes = a.d * (int)sizeof(T);
+    const int nvec = a.d / VEC;
+    const int rpw = kRowCap / row_bytes;
+    const int srows = kFC * rpw;
+    const int stage_bytes = srows * row_bytes;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kFStages * stage_bytes);
+    uint64_t* empty = full + kFStages;
+    HeadState* sstate = reinterpret_cast<HeadState*>(empty + kFStages);  // [kFC][K]
+    const long R1 = (long)a.K * a.d, R2 = (long)a.K * a.V;
+    const long a0 = R1 * blockIdx.x / gridDim.x, a1 = R1 * (blockIdx.x + 1) / gridDim.x;
+    const long b0 = R2 * blockIdx.x / gridDim.x, b1 = R2 * (blockIdx.x + 1) / gridDim.x;
+    const int n1 = (int)((a1 - a0 + srows - 1) / srows);
+    const int n2 = (int)((b1 - b0 + srows - 1) / srows);
+
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < kFStages; ++st) {
+            mbar_init(&full[st], 1);
+            mbar_init(&empty[st], kFC);
+        }
+        mbar_fence_init();
+        s_flag = 0;
+    }
+    for (int t = threadIdx.x; t < kFC * a.K; t += blockDim.x) sstate[t] = empty_state();
+    __syncthreads();
+
+    if (warp == kFC) {
+        // ---------------- producer ----------------
+        if (lane == 0) {
+            int issued = 0;
+            for (int it = 0; it < n1 + n2; ++it) {
+                const int st = it % kFStages;
+                if (it >= kFStages && !mbar_wait(&empty[st], ((it / kFStages) - 1) & 1)) {
+                    set_status(a.status, MEDUSA_STATUS_TIMEOUT);
+                    break;
+                }
+                long row0, nr;
+                const uint8_t* src;
+                if (it < n1) {
+                    row0 = a0 + (long)it * srows;
+                    nr = min((long)srows, a1 - row0);
+                    src = (const uint8_t*)a.W_res;
+                } else {
+                    row0 = b0 + (long)(it - n1) * srows;
+                    nr = min((long)srows, b1 - row0);
+                    src = (const uint8_t*)a.W_head;
+                }
+                const uint32_t bytes = (uint32_t)(nr * row_bytes);
+                mbar_arrive_expect_tx(&full[st], bytes);
+                bulk_g2s(smem + st * stage_bytes, src + row0 * row_bytes, bytes, &full[st]);
+                ++issued;
+            }
+            for (int st = 0; st < kFStages && st < issued; ++st) {  // drain before exit
+                const int last = st + ((issued - 1 - st) / kFStages) * kFStages;
+                mbar_wait(&full[st], (last / kFStages) & 1);
+            }
+        }
+    } else {
+        // ---------------- consumers ----------------
+        uint4 xr[NXV];
+        auto load_x = [&](const T* src, bool written_here) {
+#pragma unroll
+            for (int j = 0; j < NXV; ++j) {
+                const int c = j * 32 + lane;
+                xr[j] = c >= nvec ? make_uint4(0, 0, 0, 0) : written_here ? ld_cg(src + (long)c * VEC)
+                                                                           : ld_nc(src + (long)c * VEC);
+            }
+        };
+        auto dot = [&](const uint8_t* rowp) {
+            const uint4* row = reinterpret_cast<const uint4*>(rowp);
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int j = 0; j < NXV; ++j) {
+                const int c = j * 32 + lane;
+                if (c < nvec) {
+                    float wf[VEC], xf[VEC];
+                    Elt<T>::unpack(row[c], wf);
+                    Elt<T>::unpack(xr[j], xf);
+#pragma unroll
+                    for (int e = 0; e < VEC; ++e) acc[j & 3] = fmaf(wf[e], xf[e], acc[j & 3]);
+                }
+            }
+            return warp_sum((acc[0] + acc[1]) + (acc[2] + acc[3]));
+        };
+        // ok: results are valid so far; dead: a ring wait expired, so this warp
+        // stops consuming (and releasing) stages -- the producer's own bounded
+        // wait then ends the stream and it drains its copies.
+        bool ok = true, dead = false;
+        // phase 1: h^(k) rows
+        load_x((const T*)a.h, false);
+        int it = 0;
+        for (; it < n1 && !dead; ++it) {
+            const int st = it % kFStages;
+            if (!mbar_wait(&full[st], (it / kFStages) & 1)) {
+                if (lane == 0) set_status(a.status, MEDUSA_STATUS_TIMEOUT);
+                ok = false;
+                dead = true;
+                break;
+            }
+            {
+                const uint8_t* stage = smem + st * stage_bytes;
+                for (int j = 0; j < rpw; ++j) {
+                    const int lr = j * kFC + warp;
+                    const long r = a0 + (long)it * srows + lr;
+                    if (r >= a1) break;
+                    const int o = (int)(r % a.d);
+                    const float hres = Elt<T>::to_float(((const T*)a.h)[o]);
+                    const float z = dot(stage + lr * row_bytes);
+                    if (lane == 0) {
+                        const T y = Elt<T>::from_float(z / (1.f + expf(-z)) + hres);
+                        ((T*)a.hk)[r] = y;
+                        if (a.hk_out) ((T*)a.hk_out)[r] = y;
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[st]);
+        }
+        // grid barrier: every CTA's h^(k) rows are written before any is read
+        consumers_sync();
+        if (warp == 0 && lane == 0) {
+            __threadfence();
+            atomicAdd(&a.ctr[0], 1u);
+            const uint64_t t0 = global_ns();
+            while (ld_acquire_u32(&a.ctr[0]) < gridDim.x) {
+                if (global_ns() - t0 > 2000000000ull) {
+                    set_status(a.status, MEDUSA_STATUS_TIMEOUT);
+                    s_flag = 1;
+                    break;
+                }
+                __nanosleep(64);
+            }
+            __threadfence();
+        }
+        consumers_sync();
+        if (s_flag) ok = false;
+        // phase 2: logits, softmax statistics and top-8 per head
+        float m = -INFINITY, l = 0.f, tv = -INFINITY;
+        int ti = INT_MAX, cur_k = -1;
+        auto flush = [&](int kk) {
+            HeadState* sp = &sstate[warp * a.K + kk];
+            if (lane < kTopK) {
+                sp->val[lane] = tv;
+                sp->idx[lane] = ti;
+            }
+            if (lane == 0) {
+                sp->m = m;
+                sp->l = l;
+            }
+            m = -INFINITY;
+            l = 0.f;
+            tv = -INFINITY;
+            ti = INT_MAX;
+        };
+        for (it = n1; it < n1 + n2 && !dead; ++it) {
+            const int st = it % kFStages;
+            if (!mbar_wait(&full[st], (it / kFStages) & 1)) {
+                if (lane == 0) set_status(a.status, MEDUSA_STATUS_TIMEOUT);
+                ok = false;
+                dead = true;
+                break;
+            }
+            if (ok) {
+                const uint8_t* stage = smem + st * stage_bytes;
+                for (int j = 0; j < rpw; ++j) {
+                    const int lr = j * kFC + warp;
+                    const long r = b0 + (long)(it - n1) * srows + lr;
+                    if (r >= b1) break;
+                    const int k = (int)(r / a.V);
+                    const int v = (int)(r - (long)k * a.V);
+                    if (k != cur_k) {
+                        if (cur_k >= 0) flush(cur_k);
+                        cur_k = k;
+                        load_x((const T*)a.hk + (long)k * a.d, true);
+                    }
+                    const float z = dot(stage + lr * row_bytes);
+                    if (a.logits && lane == 0) a.logits[r] = z;
+                    if (z > -INFINITY || z != z) {
+                        const float mn = fmaxf(m, z);
+                        l = (m == -INFINITY ? 0.f : l * expf(m - mn)) + expf(z - mn);
+                        m = mn;
+                    }
+                    const unsigned mask = __ballot_sync(kFull, lane < kTopK && beats(z, v, tv, ti));
+                    if (mask) {
+                        const int pos = __ffs(mask) - 1;
+                        const float pv = __shfl_up_sync(kFull, tv, 1);
+                        const int pi = __shfl_up_sync(kFull, ti, 1);
+                        if (lane == pos) {
+                            tv = z;
+                            ti = v;
+                        } else if (lane > pos && lane < kTopK) {
+                            tv = pv;
+                            ti = pi;
+                        }
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[st]);
+        }
+        if (cur_k >= 0) flush(cur_k);
+    }
+    __syncthreads();
+
+    // this CTA's partial per head it covered
+    if (warp < kFC && b1 > b0) {
+        const int k_lo = (int)(b0 / a.V), k_hi = (int)((b1 - 1) / a.V);
+        for (int k = k_lo + warp; k <= k_hi; k += kFC) {
+            float mm = -INFINITY, ll = 0.f;
+            if (lane < kFC) {
+                mm = sstate[lane * a.K + k].m;
+                ll = sstate[lane * a.K + k].l;
+            }
+#pragma unroll
+            for (int o = 1; o < 8; o <<= 1) {
+                const float m2 = __shfl_xor_sync(kFull, mm, o);
+                const float l2 = __shfl_xor_sync(kFull, ll, o);
+                merge_ml(mm, ll, m2, l2);
+            }
+            float lv[kTopK];
+            int li[kTopK];
+#pragma unroll
+            for (int j = 0; j < kTopK; ++j) {
+                lv[j] = -INFINITY;
+                li[j] = INT_MAX;
+            }
+            if ((lane >> 2) < kFC) {  // lane j takes entries 2(j%4), 2(j%4)+1 of warp j/4
+                const HeadState* sp = &sstate[(lane >> 2) * a.K + k];
+                const int e = (lane & 3) * 2;
+                list_insert(lv, li, sp->val[e], sp->idx[e]);
+                list_insert(lv, li, sp->val[e + 1], sp->idx[e + 1]);
+            }
+            float ov;
+            int oi;
+            warp_select(lv, li, ov, oi);
+            HeadState* dst = &a.part[((long)blockIdx.x * a.K + k) * kBG];
+            if (lane < kTopK) {
+                dst->val[lane] = ov;
+                dst->idx[lane] = oi;
+            }
+            if (lane == 0) {
+                dst->m = mm;
+                dst->l = ll;
+            }
+        }
+    }
+    // the last CTA to finish merges every head
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_flag = atomicAdd(&a.ctr[1], 1u) == gridDim.x - 1;
+    __syncthreads();
+    if (!s_flag) return;
+    __threadfence();
+    for (int k = warp; k < a.K; k += kFC + 1)
+        merge_head(a.part, gridDim.x, a.V, kBG, 0, 0, a.V, a.K, k, a.tree, a.root_token, a.topk_idx, a.topk_prob,
+                   a.node_tokens, a.node_q, a.stats, a.status);
+}
+
+// K3 of the general path: one warp per (sequence, head).
 __global__ void __launch_bounds__(32) heads_merge_kernel(const HeadState* __restrict__ part, int nparts, int b0,
                                                          int nb, int V, int K, const TreeDev* __restrict__ tree,
                                                          const int32_t* __restrict__ root_token,
@@ -383,62 +616,9 @@ __global__ void __launch_bounds__(32) heads_merge_kernel(const HeadState* __rest
                                                          int32_t* __restrict__ node_tokens,
                                                          float* __restrict__ node_q, float2* __restrict__ stats,
                                                          int32_t* status) {
-    const int lane = threadIdx.x;
     const int bb = blockIdx.x % nb, k = blockIdx.x / nb;
-    const int b = b0 + bb;
-    const long R = (long)K * V;
-    float mm = -INFINITY, ll = 0.f;
-    float lv[kTopK];
-    int li[kTopK];
-#pragma unroll
-    for (int j = 0; j < kTopK; ++j) {
-        lv[j] = -INFINITY;
-        li[j] = INT_MAX;
-    }
-    for (int c = lane; c < nparts; c += 32) {
-        const long r0 = R * c / nparts, r1 = R * (c + 1) / nparts;
-        if (r1 <= r0 || (long)(k + 1) * V <= r0 || r1 <= (long)k * V) continue;  // CTA c did not cover head k
-        const HeadState* s = &part[((long)c * K + k) * kBG + bb];
-        merge_ml(mm, ll, s->m, s->l);
-#pragma unroll
-        for (int j = 0; j < kTopK; ++j) list_insert(lv, li, s->val[j], s->idx[j]);
-    }
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        float m2 = __shfl_xor_sync(kFull, mm, o);
-        float l2 = __shfl_xor_sync(kFull, ll, o);
-        merge_ml(mm, ll, m2, l2);
-    }
-    float ov;
-    int oi;
-    warp_select(lv, li, ov, oi);
-    const bool valid = oi != INT_MAX;
-    const float prob = valid ? expf(ov - mm) / ll : 0.f;
-    if (lane < kTopK) {
-        topk_idx[((long)b * K + k) * kTopK + lane] = valid ? oi : -1;
-        topk_prob[((long)b * K + k) * kTopK + lane] = prob;
-    }
-    if (lane == 0 && stats) stats[(long)b * K + k] = make_float2(mm, ll);
-    if (tree) {
-        const int T = tree->T;
-        for (int i0 = 0; i0 < T; i0 += 32) {
-            int i = i0 + lane;
-            int rk = i < T ? tree->rank[i] : 0;
-            int tok = __shfl_sync(kFull, valid ? oi : -1, rk & (kTopK - 1));
-            float pq = __shfl_sync(kFull, prob, rk & (kTopK - 1));
-            if (i < T && i > 0 && tree->depth[i] == k + 2) {
-                node_tokens[(long)b * T + i] = tok;
-                if (node_q) node_q[(long)b * T + i] = pq;
-                if (tok < 0) set_status(status, MEDUSA_STATUS_BAD_TOKEN);
-            }
-        }
-        if (k == 0 && lane == 0) {
-            int rt = root_token[b];
-            node_tokens[(long)b * T] = rt;
-            if (node_q) node_q[(long)b * T] = 1.f;
-            if (rt < 0 || rt >= V) set_status(status, MEDUSA_STATUS_BAD_TOKEN);
-        }
-    }
+    merge_head(part, nparts, V, kBG, bb, b0 + bb, V, K, k, tree, root_token, topk_idx, topk_prob, node_tokens, node_q,
+               stats, status);
 }
 
 // probs[b,k,v] = exp(logit - m) / l
@@ -474,7 +654,7 @@ LmConfig lm_config(int K) {
 int lm_grid_bound() { return num_sms() * (2048 / (kLmWarps * 32)); }
 
 struct HeadsWs {
-    size_t hk, part, stats, logits, total;
+    size_t hk, part, stats, ctr, logits, total;
 };
 
 HeadsWs heads_ws_layout(int B, int d, int V, int K, medusa_dtype dt) {
@@ -482,8 +662,10 @@ HeadsWs heads_ws_layout(int B, int d, int V, int K, medusa_dtype dt) {
     size_t esz = dt == MEDUSA_BF16 ? 2 : 4;
     w.hk = 0;
     w.part = w.hk + align256((size_t)B * K * d * esz);
-    w.stats = w.part + align256((size_t)lm_grid_bound() * K * kBG * sizeof(HeadState));
-    w.logits = w.stats + align256((size_t)B * K * sizeof(float2));
+    const int bstride = B > kBG ? (B < 64 ? B : 64) : kBG;  // tensor-core path keeps one partial per sequence
+    w.stats = w.part + align256((size_t)lm_grid_bound() * K * bstride * sizeof(HeadState));
+    w.ctr = w.stats + align256((size_t)B * K * sizeof(float2));
+    w.logits = w.ctr + 256;
     w.total = w.logits + align256((size_t)B * K * V * sizeof(float));
     return w;
 }
@@ -498,10 +680,77 @@ cudaError_t heads_launch_t(const HeadsArgs& a, cudaStream_t st) {
     float2* stats = (float2*)(ws + w.stats);
     float* logits = a.logits_out ? a.logits_out : (a.probs_out ? (float*)(ws + w.logits) : nullptr);
 
+    const int row_bytes = a.d * (int)sizeof(T);
+    cudaError_t e;
+    if (heads_tc_supported(a.B, a.d, a.dt)) {
+        // bf16: weight streaming on the tensor cores (one cooperative kernel)
+        e = heads_tc_launch(a, hk, part, (unsigned int*)(ws + w.ctr), stats, logits, st);
+        if (e != cudaSuccess) return e;
+        if (a.probs_out) {
+            const long n = (long)a.B * a.K * a.V;
+            int pg = (int)((n + 255) / 256);
+            if (pg > num_sms() * 8) pg = num_sms() * 8;
+            heads_probs_kernel<<<pg, 256, 0, st>>>(logits, stats, a.B, a.K, a.V, a.probs_out);
+            e = cudaGetLastError();
+        }
+        return e;
+    }
+    if (a.B == 1 && row_bytes <= kRowCap && row_bytes % 16 == 0) {
+        // one sequence: the whole call is one cooperative persistent kernel
+        const size_t smem = fused_smem_bytes(row_bytes, a.K);
+        auto kern = heads_fused_kernel<T>;
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        int occ = 0;
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, (kFC + 1) * 32, smem);
+        if (occ >= 1) {
+            unsigned int* ctr = (unsigned int*)(ws + w.ctr);
+            if ((e = cudaMemsetAsync(ctr, 0, 2 * sizeof(unsigned int), st)) != cudaSuccess) return e;
+            FusedArgs fa;
+            fa.h = a.h;
+            fa.W_res = a.W_res;
+            fa.W_head = a.W_head;
+            fa.d = a.d;
+            fa.V = a.V;
+            fa.K = a.K;
+            fa.hk = hk;
+            fa.hk_out = a.h_res_out;
+            fa.logits = logits;
+            fa.part = part;
+            fa.ctr = ctr;
+            fa.tree = a.tree;
+            fa.root_token = a.root_token;
+            fa.topk_idx = a.topk_idx;
+            fa.topk_prob = a.topk_prob;
+            fa.node_tokens = a.node_tokens;
+            fa.node_q = a.node_q;
+            fa.stats = stats;
+            fa.status = a.status;
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(num_sms());  // one CTA per SM, all resident (cooperative)
+            cfg.blockDim = dim3((kFC + 1) * 32);
+            cfg.dynamicSmemBytes = smem;
+            cfg.stream = st;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeCooperative;
+            attr[0].val.cooperative = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            if ((e = cudaLaunchKernelEx(&cfg, kern, fa)) != cudaSuccess) return e;
+            if (a.probs_out) {
+                const long n = (long)a.K * a.V;
+                int pg = (int)((n + 255) / 256);
+                if (pg > num_sms() * 8) pg = num_sms() * 8;
+                heads_probs_kernel<<<pg, 256, 0, st>>>(logits, stats, 1, a.K, a.V, a.probs_out);
+                e = cudaGetLastError();
+            }
+            return e;
+        }
+    }
+
     const long rows = (long)a.K * a.d;
     heads_res_kernel<T><<<(unsigned)((rows + kResWarps - 1) / kResWarps), kResWarps * 32, 0, st>>>(
         (const T*)a.h, (const T*)a.W_res, a.B, a.d, a.K, hk, (T*)a.h_res_out);
-    cudaError_t e = cudaGetLastError();
+    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
 
     const bool hreg = a.B == 1 && a.d / VEC <= 32 * 2 * kUnroll;

@@ -1,0 +1,181 @@
+// Device helpers shared by the heads kernels: running softmax statistics and
+// top-8 lists per (sequence, head), their merges, and the final per-head
+// merge that writes top-8 entries and fills the candidate tree.
+#pragma once
+
+#include <limits.h>
+
+#include "common.cuh"
+
+namespace medusa {
+
+// Running softmax statistics and top-8 list of one (sequence, head) over a
+// set of vocabulary rows: m = max logit, l = sum exp(logit - m).
+struct HeadState {
+    float m, l;
+    float val[kTopK];
+    int idx[kTopK];
+};
+
+__device__ __forceinline__ HeadState empty_state() {
+    HeadState s;
+    s.m = -INFINITY;
+    s.l = 0.f;
+#pragma unroll
+    for (int j = 0; j < kTopK; ++j) {
+        s.val[j] = -INFINITY;
+        s.idx[j] = INT_MAX;
+    }
+    return s;
+}
+
+// merge softmax statistics (m2, l2) into (m, l)
+__device__ __forceinline__ void merge_ml(float& m, float& l, float m2, float l2) {
+    if (m2 == -INFINITY) return;
+    if (m == -INFINITY) {
+        m = m2;
+        l = l2;
+        return;
+    }
+    float mn = fmaxf(m, m2);
+    l = l * expf(m - mn) + l2 * expf(m2 - mn);
+    m = mn;
+}
+
+// Insert (v, i) into a register-resident list sorted best-first.
+__device__ __forceinline__ void list_insert(float (&lv)[kTopK], int (&li)[kTopK], float v, int i) {
+    if (!beats(v, i, lv[kTopK - 1], li[kTopK - 1])) return;
+    lv[kTopK - 1] = v;
+    li[kTopK - 1] = i;
+#pragma unroll
+    for (int j = kTopK - 1; j > 0; --j) {
+        if (beats(lv[j], li[j], lv[j - 1], li[j - 1])) {
+            float tv = lv[j];
+            lv[j] = lv[j - 1];
+            lv[j - 1] = tv;
+            int ti = li[j];
+            li[j] = li[j - 1];
+            li[j - 1] = ti;
+        }
+    }
+}
+
+// Warp-wide selection of the best kTopK candidates from per-lane sorted
+// lists.  Lane j < kTopK receives the j-th best in (out_v, out_i).
+__device__ __forceinline__ void warp_select(float (&lv)[kTopK], int (&li)[kTopK], float& out_v, int& out_i) {
+    const int lane = threadIdx.x & 31;
+    out_v = -INFINITY;
+    out_i = INT_MAX;
+#pragma unroll 1
+    for (int r = 0; r < kTopK; ++r) {
+        float wv = lv[0];
+        int wi = li[0];
+        int wl = lane;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            float ov = __shfl_xor_sync(kFull, wv, o);
+            int oi = __shfl_xor_sync(kFull, wi, o);
+            int ol = __shfl_xor_sync(kFull, wl, o);
+            if (beats(ov, oi, wv, wi) || (ov == wv && oi == wi && ol < wl)) {
+                wv = ov;
+                wi = oi;
+                wl = ol;
+            }
+        }
+        if (lane == r) {
+            out_v = wv;
+            out_i = wi;
+        }
+        if (lane == wl) {  // pop the head of the winning lane's list
+#pragma unroll
+            for (int j = 0; j < kTopK - 1; ++j) {
+                lv[j] = lv[j + 1];
+                li[j] = li[j + 1];
+            }
+            lv[kTopK - 1] = -INFINITY;
+            li[kTopK - 1] = INT_MAX;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Merge of one (sequence, head): the partials of the CTAs that covered the
+// head, in CTA order (the CTAs split K*uph units evenly, head k owning units
+// [k*uph, (k+1)*uph); partial (c, k, b) sits at part[(c*K + k)*bstride + b]) (so the result does not depend on which CTA runs
+// the merge); writes the top-8 entries with their probabilities, the head's
+// softmax statistics, and fills the tree nodes this head proposes.  One warp.
+// Partials are read through L2 (they may have been written by other CTAs of
+// the same kernel).
+// ---------------------------------------------------------------------------
+static __device__ __noinline__ void merge_head(const HeadState* __restrict__ part, int nparts, long uph, int bstride, int bb,
+                                       int b, int V, int K, int k,
+                           const TreeDev* __restrict__ tree, const int32_t* __restrict__ root_token,
+                           int32_t* __restrict__ topk_idx, float* __restrict__ topk_prob,
+                           int32_t* __restrict__ node_tokens, float* __restrict__ node_q, float2* __restrict__ stats,
+                           int32_t* status) {
+    const int lane = threadIdx.x & 31;
+    const long R = (long)K * uph;
+    float mm = -INFINITY, ll = 0.f;
+    float lv[kTopK];
+    int li[kTopK];
+#pragma unroll
+    for (int j = 0; j < kTopK; ++j) {
+        lv[j] = -INFINITY;
+        li[j] = INT_MAX;
+    }
+    for (int c = lane; c < nparts; c += 32) {
+        const long r0 = R * c / nparts, r1 = R * (c + 1) / nparts;
+        if (r1 <= r0 || (long)(k + 1) * uph <= r0 || r1 <= (long)k * uph) continue;  // CTA c did not cover head k
+        const HeadState* s = &part[((long)c * K + k) * bstride + bb];
+        float pv[kTopK];
+        int pi[kTopK];
+#pragma unroll
+        for (int j = 0; j < kTopK; ++j) {  // issue every load before using any
+            pv[j] = __ldcg(&s->val[j]);
+            pi[j] = __ldcg(&s->idx[j]);
+        }
+        const float sm = __ldcg(&s->m), sl = __ldcg(&s->l);
+        merge_ml(mm, ll, sm, sl);
+#pragma unroll
+        for (int j = 0; j < kTopK; ++j) list_insert(lv, li, pv[j], pi[j]);
+    }
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float m2 = __shfl_xor_sync(kFull, mm, o);
+        const float l2 = __shfl_xor_sync(kFull, ll, o);
+        merge_ml(mm, ll, m2, l2);
+    }
+    float ov;
+    int oi;
+    warp_select(lv, li, ov, oi);
+    const bool valid = oi != INT_MAX;
+    const float prob = valid ? expf(ov - mm) / ll : 0.f;
+    if (lane < kTopK) {
+        topk_idx[((long)b * K + k) * kTopK + lane] = valid ? oi : -1;
+        topk_prob[((long)b * K + k) * kTopK + lane] = prob;
+    }
+    if (lane == 0 && stats) stats[(long)b * K + k] = make_float2(mm, ll);
+    if (tree) {
+        const int T = tree->T;
+        for (int i0 = 0; i0 < T; i0 += 32) {
+            const int i = i0 + lane;
+            const int rk = i < T ? tree->rank[i] : 0;
+            const int dp = i < T ? tree->depth[i] : 0;
+            const int tok = __shfl_sync(kFull, valid ? oi : -1, rk & (kTopK - 1));
+            const float pq = __shfl_sync(kFull, prob, rk & (kTopK - 1));
+            if (i < T && i > 0 && dp == k + 2) {
+                node_tokens[(long)b * T + i] = tok;
+                if (node_q) node_q[(long)b * T + i] = pq;
+                if (tok < 0) set_status(status, MEDUSA_STATUS_BAD_TOKEN);
+            }
+        }
+        if (k == 0 && lane == 0) {
+            const int rt = root_token[b];
+            node_tokens[(long)b * T] = rt;
+            if (node_q) node_q[(long)b * T] = 1.f;
+            if (rt < 0 || rt >= V) set_status(status, MEDUSA_STATUS_BAD_TOKEN);
+        }
+    }
+}
+
+}  // namespace medusa

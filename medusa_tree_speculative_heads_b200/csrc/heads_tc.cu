@@ -1,0 +1,471 @@
+// Medusa heads on the 5th-generation tensor cores (bf16, batch <= 64).
+//
+// Operation ("Medusa Explained: Multi-Head Speculative Decoding Guide",
+// section "The Architectural Blueprint"): h^(k) = SiLU(W_res^(k) h) + h,
+// p^(k) = softmax(W_head^(k) h^(k)), then each head's top-8 fills the
+// candidate tree ("1. Combinatorial Tree Construction").
+//
+// Both products read every weight once, with only B (1..64) columns on the
+// other side: weight streaming is the cost, so the kernel is built around
+// keeping HBM busy and the SMs' ALUs idle.  Each weight tile of 128 rows x 64
+// k-elements (16 KB) is a tcgen05 MMA A operand (M = 128), the batch vectors
+// are the B operand (N = batch rounded up to 16; TMA zero-fills the padding
+// rows), and the fp32 accumulator lives in TMEM.  One cooperative persistent
+// kernel per call, one CTA per SM, 7 warps:
+//   warp 0   TMA producer of weight tiles (a ring of shared-memory stages)
+//   warp 1   TMEM allocation; one thread issues the MMAs (double-buffered
+//            accumulator, commits release ring stages and hand tiles over)
+//   warp 2   TMA producer of the batch-vector tiles; before the first
+//            vocabulary tile it waits at the grid barrier (all of h^(k) must
+//            be written by every CTA)
+//   warps 3-6 epilogue, one TMEM lane (= weight row) per thread: residual
+//            tiles write h^(k) = SiLU(z) + h (bf16); vocabulary tiles update
+//            per-(head, sequence) running softmax statistics and top-8 lists.
+// The residual tiles of every head come first, then the vocabulary tiles;
+// the weight producer keeps prefetching across the grid barrier.  The last
+// CTA to finish merges all CTAs' partials in CTA order and fills the tree.
+// Every wait is bounded (~2 s) and sets MEDUSA_STATUS_TIMEOUT on expiry.
+#include <limits.h>
+
+#include "heads_common.cuh"
+#include "kernels.h"
+#include "tc.cuh"
+#include "tma.h"
+
+namespace medusa {
+
+namespace {
+
+constexpr int kTcWarps = 7;
+constexpr int kTM = 128;                 // weight rows per tile (MMA M)
+constexpr int kTK = 64;                  // k-elements per stage (128 bytes, one swizzle row)
+constexpr int kABytes = kTM * kTK * 2;   // 16 KB
+constexpr int kEpiWarp0 = 3;             // first epilogue warp
+constexpr int kSmemBudget = 227 * 1024;
+
+struct TcHeadsArgs {
+    CUtensorMap mW_res;   // W_res  as (d_in, d_out, K), box (64, 128, 1)
+    CUtensorMap mW_head;  // W_head as (d, V, K),        box (64, 128, 1)
+    CUtensorMap mh;       // h      as (d, B),           box (64, N)
+    CUtensorMap mhk;      // h^(k)  as (d, K, B),        box (64, 1, N)
+    const __nv_bfloat16* h;
+    __nv_bfloat16* hk;      // [B][K][d] (workspace)
+    __nv_bfloat16* hk_out;  // nullable copy for the caller
+    float* logits;          // [B][K][V], nullable
+    HeadState* part;        // [grid][K][B]
+    unsigned int* ctr;      // [2], zero at launch
+    const TreeDev* tree;
+    const int32_t* root_token;
+    int32_t* topk_idx;
+    float* topk_prob;
+    int32_t* node_tokens;
+    float* node_q;
+    float2* stats;
+    int32_t* status;
+    int B, d, V, K;
+    int stages;
+};
+
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(kFull, x, o));
+    return x;
+}
+
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
+
+// sorted insert into a shared-memory top-8 list (one thread)
+__device__ __forceinline__ void smem_list_insert(HeadState* s, float v, int i) {
+    if (!beats(v, i, s->val[kTopK - 1], s->idx[kTopK - 1])) return;
+    int j = kTopK - 1;
+    while (j > 0 && beats(v, i, s->val[j - 1], s->idx[j - 1])) {
+        s->val[j] = s->val[j - 1];
+        s->idx[j] = s->idx[j - 1];
+        --j;
+    }
+    s->val[j] = v;
+    s->idx[j] = i;
+}
+
+template <int N>
+__global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid_constant__ TcHeadsArgs a) {
+    constexpr int kBBytes = N * kTK * 2;  // batch tile per stage (multiple of 1024)
+    constexpr int kTmemCols = N * 2 <= 32 ? 32 : N * 2 <= 64 ? 64 : 128;
+    constexpr uint32_t kIdesc = idesc_bf16_f32(kTM, N);
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const int S = a.stages;
+    uint8_t* sA = smem;
+    uint8_t* sB = sA + (size_t)S * kABytes;
+    uint64_t* full = reinterpret_cast<uint64_t*>(sB + (size_t)S * kBBytes);
+    uint64_t* empty = full + S;
+    uint64_t* acc_full = empty + S;    // [2]
+    uint64_t* acc_empty = acc_full + 2;  // [2]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+    int* flag = reinterpret_cast<int*>(tmem_slot + 1);
+    HeadState* st = reinterpret_cast<HeadState*>(tmem_slot + 4);  // [4][N]
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int K = a.K, B = a.B;
+    const int tph_r = (a.d + kTM - 1) / kTM;   // residual tiles per head
+    const int tph_l = (a.V + kTM - 1) / kTM;   // vocabulary tiles per head
+    const int nkb = (a.d + kTK - 1) / kTK;
+    const long T1 = (long)K * tph_r, T2 = (long)K * tph_l;
+    const long t1a = T1 * blockIdx.x / gridDim.x, t1b = T1 * (blockIdx.x + 1) / gridDim.x;
+    const long t2a = T2 * blockIdx.x / gridDim.x, t2b = T2 * (blockIdx.x + 1) / gridDim.x;
+    const int n1 = (int)(t1b - t1a), n2 = (int)(t2b - t2a);
+    const int ntiles = n1 + n2;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 2);  // the weight and the batch producer each arrive with their bytes
+            mbar_init(&empty[s], 1);
+        }
+        for (int j = 0; j < 2; ++j) {
+            mbar_init(&acc_full[j], 1);
+            mbar_init(&acc_empty[j], 4);
+        }
+        mbar_fence_init();
+        *flag = 0;
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&a.mW_res);
+        tma_prefetch_desc(&a.mW_head);
+        tma_prefetch_desc(&a.mh);
+        tma_prefetch_desc(&a.mhk);
+    }
+    for (int t = threadIdx.x; t < 4 * N; t += blockDim.x) st[t] = empty_state();
+    if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0 || warp == 2) {
+        // ---------------- producers ----------------
+        if (lane == 0) {
+            const bool weights = warp == 0;
+            const uint32_t bytes = weights ? kABytes : kBBytes;
+            int issued = 0;
+            bool ok = true;
+            for (int li = 0; li < ntiles && ok; ++li) {
+                const bool res = li < n1;
+                const long t = res ? t1a + li : t2a + (li - n1);
+                const int k = (int)(res ? t / tph_r : t / tph_l);
+                const int row0 = (int)(res ? t % tph_r : t % tph_l) * kTM;
+                if (!weights && li == n1) {
+                    // vocabulary tiles read h^(k): wait until every CTA wrote its rows
+                    const uint64_t t0 = global_ns();
+                    while (ld_acquire_u32(&a.ctr[0]) < gridDim.x) {
+                        if (global_ns() - t0 > 2000000000ull) {
+                            set_status(a.status, MEDUSA_STATUS_TIMEOUT);
+                            ok = false;
+                            break;
+                        }
+                        __nanosleep(100);
+                    }
+                    fence_proxy_async_global();
+                    if (!ok) break;
+                }
+                for (int kb = 0; kb < nkb; ++kb) {
+                    const int it = li * nkb + kb;
+                    const int s = it % S;
+                    if (it >= S && !mbar_wait(&empty[s], ((it / S) - 1) & 1)) {
+                        set_status(a.status, MEDUSA_STATUS_TIMEOUT);
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&full[s], bytes);
+                    if (weights)
+                        tma_load_3d(sA + (size_t)s * kABytes, res ? &a.mW_res : &a.mW_head, kb * kTK, row0, k,
+                                    &full[s]);
+                    else if (res)
+                        tma_load_2d(sB + (size_t)s * kBBytes, &a.mh, kb * kTK, 0, &full[s]);
+                    else
+                        tma_load_3d(sB + (size_t)s * kBBytes, &a.mhk, kb * kTK, k, 0, &full[s]);
+                    ++issued;
+                }
+            }
+            // drain: no copy may still be landing when the CTA exits
+            for (int s = 0; s < S && s < issued; ++s) {
+                const int last = s + ((issued - 1 - s) / S) * S;
+                mbar_wait(&full[s], (last / S) & 1);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            bool ok = true;
+            for (int li = 0; li < ntiles && ok; ++li) {
+                const int buf = li & 1;
+                if (li >= 2 && !mbar_wait(&acc_empty[buf], ((li >> 1) - 1) & 1)) {
+                    set_status(a.status, MEDUSA_STATUS_TIMEOUT);
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + buf * N;
+                for (int kb = 0; kb < nkb; ++kb) {
+                    const int it = li * nkb + kb;
+                    const int s = it % S;
+                    if (!mbar_wait(&full[s], (it / S) & 1)) {
+                        set_status(a.status, MEDUSA_STATUS_TIMEOUT);
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t adesc = sw128_kmajor_desc(smem_addr(sA + (size_t)s * kABytes));
+                    const uint64_t bdesc = sw128_kmajor_desc(smem_addr(sB + (size_t)s * kBBytes));
+#pragma unroll
+                    for (int ks = 0; ks < kTK / 16; ++ks)  // 16 k-elements = 32 bytes per MMA
+                        tc_mma_bf16(d_tmem, adesc + 2 * ks, bdesc + 2 * ks, kIdesc, (kb | ks) != 0);
+                    tc_commit(&empty[s]);
+                }
+                tc_commit(&acc_full[buf]);
+            }
+            // let every issued MMA finish before the accumulator is released
+            if (ntiles > 0) mbar_wait(&acc_full[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1);
+        }
+    } else {
+        // ---------------- epilogue ----------------
+        const int ew = warp - kEpiWarp0;     // 0..3
+        const int q = warp & 3;              // TMEM lane quarter this warp may access
+        const int row = q * 32 + lane;       // weight row of the tile held by this thread
+        HeadState* mine = st + ew * N;
+        int cur_k = -1;
+        bool ok = true;
+        auto flush = [&](int kk) {
+            epi_sync();
+            // warp ew merges columns b = ew, ew+4, ... over the 4 epilogue warps
+            for (int b = ew; b < B; b += 4) {
+                float mm = -INFINITY, ll = 0.f;
+                if (lane < 4) {
+                    mm = st[lane * N + b].m;
+                    ll = st[lane * N + b].l;
+                }
+#pragma unroll
+                for (int o = 1; o < 4; o <<= 1) {
+                    const float m2 = __shfl_xor_sync(kFull, mm, o);
+                    const float l2 = __shfl_xor_sync(kFull, ll, o);
+                    merge_ml(mm, ll, m2, l2);
+                }
+                float lv[kTopK];
+                int li2[kTopK];
+#pragma unroll
+                for (int j = 0; j < kTopK; ++j) {
+                    lv[j] = -INFINITY;
+                    li2[j] = INT_MAX;
+                }
+                lv[0] = st[(lane >> 3) * N + b].val[lane & 7];
+                li2[0] = st[(lane >> 3) * N + b].idx[lane & 7];
+                float ov;
+                int oi;
+                warp_select(lv, li2, ov, oi);
+                HeadState* dst = &a.part[((long)blockIdx.x * K + kk) * B + b];
+                if (lane < kTopK) {
+                    dst->val[lane] = ov;
+                    dst->idx[lane] = oi;
+                }
+                if (lane == 0) {
+                    dst->m = mm;
+                    dst->l = ll;
+                }
+            }
+            epi_sync();
+            for (int b = lane; b < B; b += 32) mine[b] = empty_state();
+            __syncwarp();
+        };
+        auto arrive_grid = [&]() {
+            // this CTA's h^(k) rows are written: publish them (also to the TMA proxy)
+            fence_proxy_async_global();
+            __threadfence();
+            epi_sync();
+            if (ew == 0 && lane == 0) atomicAdd(&a.ctr[0], 1u);
+        };
+        if (n1 == 0) arrive_grid();
+        for (int li = 0; li < ntiles; ++li) {
+            const int buf = li & 1;
+            if (ok && !mbar_wait(&acc_full[buf], (li >> 1) & 1)) {
+                if (lane == 0) set_status(a.status, MEDUSA_STATUS_TIMEOUT);
+                ok = false;
+            }
+            float v[N];
+#pragma unroll
+            for (int e = 0; e < N; ++e) v[e] = 0.f;
+            if (ok) {
+                tc_fence_after();
+#pragma unroll
+                for (int c = 0; c < N / 16; ++c) {
+                    float t16[16];
+                    tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + buf * N + c * 16, t16);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) v[c * 16 + e] = t16[e];
+                }
+                tc_fence_before();
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[buf]);
+            if (li < n1) {
+                // residual tile: h^(k)[b, o] = SiLU(z) + h[b, o]
+                const long t = t1a + li;
+                const int k = (int)(t / tph_r);
+                const int o = (int)(t % tph_r) * kTM + row;
+                if (ok && o < a.d) {
+                    for (int b = 0; b < B; ++b) {
+                        const float z = v[b];
+                        const float y = z / (1.f + expf(-z)) + __bfloat162float(a.h[(long)b * a.d + o]);
+                        const __nv_bfloat16 yb = __float2bfloat16_rn(y);
+                        a.hk[((long)b * K + k) * a.d + o] = yb;
+                        if (a.hk_out) a.hk_out[((long)b * K + k) * a.d + o] = yb;
+                    }
+                }
+                if (li == n1 - 1) arrive_grid();
+                continue;
+            }
+            // vocabulary tile
+            const long t = t2a + (li - n1);
+            const int k = (int)(t / tph_l);
+            const int vrow = (int)(t % tph_l) * kTM + row;
+            const bool valid = ok && vrow < a.V;
+            if (k != cur_k) {
+                if (cur_k >= 0) flush(cur_k);
+                cur_k = k;
+            }
+            for (int b = 0; b < B; ++b) {
+                const float x = v[b];
+                if (a.logits && valid) a.logits[((long)b * K + k) * a.V + vrow] = x;
+                // softmax statistics of the tile's 32 rows of this warp
+                const float tm = warp_max(valid ? x : -INFINITY);
+                if (tm > -INFINITY) {
+                    const float tl = warp_sum(valid ? expf(x - tm) : 0.f);
+                    if (lane == 0) merge_ml(mine[b].m, mine[b].l, tm, tl);
+                }
+                // top-8: the rows that beat the current 8th entry
+                const float thr_v = mine[b].val[kTopK - 1];
+                const int thr_i = mine[b].idx[kTopK - 1];
+                unsigned mask = __ballot_sync(kFull, valid && beats(x, vrow, thr_v, thr_i));
+                while (mask) {
+                    const int j = __ffs(mask) - 1;
+                    const float xv = __shfl_sync(kFull, x, j);
+                    const int xi = __shfl_sync(kFull, vrow, j);
+                    if (lane == 0) smem_list_insert(&mine[b], xv, xi);
+                    mask &= mask - 1;
+                }
+                __syncwarp();
+            }
+        }
+        if (cur_k >= 0) flush(cur_k);
+    }
+
+    // ---------------- teardown ----------------
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+    // the last CTA to finish merges every (sequence, head)
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) *flag = atomicAdd(&a.ctr[1], 1u) == gridDim.x - 1;
+    __syncthreads();
+    if (!*flag) return;
+    __threadfence();
+    for (int p = warp; p < B * K; p += kTcWarps) {
+        const int b = p % B, k = p / B;
+        merge_head(a.part, gridDim.x, tph_l, B, b, b, a.V, K, k, a.tree, a.root_token, a.topk_idx, a.topk_prob,
+                   a.node_tokens, a.node_q, a.stats, a.status);
+    }
+}
+
+template <int N>
+size_t tc_smem_bytes(int stages) {
+    return 1024 + (size_t)stages * (kABytes + N * kTK * 2) + (2 * (size_t)stages + 4) * 8 + 16 +
+           4 * (size_t)N * sizeof(HeadState);
+}
+
+template <int N>
+int tc_stages() {
+    int s = 12;
+    while (s > 2 && tc_smem_bytes<N>(s) > (size_t)kSmemBudget) --s;
+    return s;
+}
+
+template <int N>
+cudaError_t launch_n(const TcHeadsArgs& args, cudaStream_t st) {
+    TcHeadsArgs a = args;
+    a.stages = tc_stages<N>();
+    const size_t smem = tc_smem_bytes<N>(a.stages);
+    auto kern = heads_tc_kernel<N>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(num_sms());
+    cfg.blockDim = dim3(kTcWarps * 32);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
+}  // namespace
+
+bool heads_tc_supported(int B, int d, medusa_dtype dt) { return dt == MEDUSA_BF16 && B >= 1 && B <= 64 && d % 8 == 0; }
+
+cudaError_t heads_tc_launch(const HeadsArgs& x, void* hk, void* part, unsigned int* ctr, float2* stats, float* logits,
+                            cudaStream_t st) {
+    TcHeadsArgs a;
+    const uint64_t d = x.d, V = x.V, K = x.K, B = x.B;
+    const int N = (x.B + 15) / 16 * 16;
+    {
+        const uint64_t dims[3] = {d, d, K}, strides[2] = {d * 2, d * d * 2};
+        const uint32_t box[3] = {kTK, kTM, 1};
+        if (!make_tmap_bf16(&a.mW_res, x.W_res, 3, dims, strides, box)) return cudaErrorInvalidValue;
+    }
+    {
+        const uint64_t dims[3] = {d, V, K}, strides[2] = {d * 2, V * d * 2};
+        const uint32_t box[3] = {kTK, kTM, 1};
+        if (!make_tmap_bf16(&a.mW_head, x.W_head, 3, dims, strides, box)) return cudaErrorInvalidValue;
+    }
+    {
+        const uint64_t dims[2] = {d, B}, strides[1] = {d * 2};
+        const uint32_t box[2] = {kTK, (uint32_t)N};
+        if (!make_tmap_bf16(&a.mh, x.h, 2, dims, strides, box)) return cudaErrorInvalidValue;
+    }
+    {
+        const uint64_t dims[3] = {d, K, B}, strides[2] = {d * 2, K * d * 2};
+        const uint32_t box[3] = {kTK, 1, (uint32_t)N};
+        if (!make_tmap_bf16(&a.mhk, hk, 3, dims, strides, box)) return cudaErrorInvalidValue;
+    }
+    a.h = (const __nv_bfloat16*)x.h;
+    a.hk = (__nv_bfloat16*)hk;
+    a.hk_out = (__nv_bfloat16*)x.h_res_out;
+    a.logits = logits;
+    a.part = (HeadState*)part;
+    a.ctr = ctr;
+    a.tree = x.tree;
+    a.root_token = x.root_token;
+    a.topk_idx = x.topk_idx;
+    a.topk_prob = x.topk_prob;
+    a.node_tokens = x.node_tokens;
+    a.node_q = x.node_q;
+    a.stats = stats;
+    a.status = x.status;
+    a.B = x.B;
+    a.d = x.d;
+    a.V = x.V;
+    a.K = x.K;
+    cudaError_t e = cudaMemsetAsync(ctr, 0, 2 * sizeof(unsigned int), st);
+    if (e != cudaSuccess) return e;
+    switch (N) {
+        case 16: return launch_n<16>(a, st);
+        case 32: return launch_n<32>(a, st);
+        case 48: return launch_n<48>(a, st);
+        default: return launch_n<64>(a, st);
+    }
+}
+
+}  // namespace medusa

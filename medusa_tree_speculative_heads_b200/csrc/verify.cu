@@ -52,11 +52,24 @@ __global__ void __launch_bounds__(kArgmaxThreads) row_argmax_kernel(const T* __r
         int va = v0;
         if ((((uintptr_t)(rp + v0)) & 15) == 0) {
             const int nvec = (v1 - v0) / VEC;
-            for (int c = threadIdx.x; c < nvec; c += kArgmaxThreads) {
-                float f[VEC];
-                Elt<T>::unpack(ld_stream(rp + v0 + (long)c * VEC), f);
+            constexpr int U = 4;  // independent 16-byte loads in flight per thread
+            for (int c0 = threadIdx.x; c0 < nvec; c0 += U * kArgmaxThreads) {
+                uint4 raw[U];
 #pragma unroll
-                for (int e = 0; e < VEC; ++e) argmax_merge(bv, bi, f[e], v0 + c * VEC + e);
+                for (int u = 0; u < U; ++u) {
+                    const int c = c0 + u * kArgmaxThreads;
+                    raw[u] = c < nvec ? ld_stream(rp + v0 + (long)c * VEC) : make_uint4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int c = c0 + u * kArgmaxThreads;
+                    if (c < nvec) {
+                        float f[VEC];
+                        Elt<T>::unpack(raw[u], f);
+#pragma unroll
+                        for (int e = 0; e < VEC; ++e) argmax_merge(bv, bi, f[e], v0 + c * VEC + e);
+                    }
+                }
             }
             va = v0 + nvec * VEC;
         }
@@ -98,7 +111,7 @@ __global__ void __launch_bounds__(32) greedy_walk_kernel(const float* __restrict
                                                          int splits, const int32_t* __restrict__ node_tokens,
                                                          const TreeDev* __restrict__ tree, int32_t* accept_path,
                                                          int max_path, int32_t* accept_len, int32_t* bonus) {
-    __shared__ int pred[kMaxTree];
+    __shared__ int pred[kMaxTree], tok[kMaxTree], par[kMaxTree], dep[kMaxTree];
     __shared__ uint8_t acc[kMaxTree];
     const int b = blockIdx.x, lane = threadIdx.x;
     const int T = tree->T;
@@ -108,21 +121,24 @@ __global__ void __launch_bounds__(32) greedy_walk_kernel(const float* __restrict
         int bi = INT_MAX;
         for (int s = 0; s < splits; ++s) argmax_merge(bv, bi, pval[base + s], pidx[base + s]);
         pred[u] = bi;
+        tok[u] = node_tokens[(long)b * T + u];
+        par[u] = tree->parent[u];
+        dep[u] = tree->depth[u];
     }
     __syncwarp();
     if (lane == 0) {
         acc[0] = 1;
         int best = 0;
         for (int c = 1; c < T; ++c) {
-            const int p = tree->parent[c];
-            acc[c] = acc[p] && node_tokens[(long)b * T + c] == pred[p];
-            if (acc[c] && tree->depth[c] > tree->depth[best]) best = c;
+            const int p = par[c];
+            acc[c] = acc[p] && tok[c] == pred[p];
+            if (acc[c] && dep[c] > dep[best]) best = c;
         }
-        const int L = tree->depth[best];
+        const int L = dep[best];
         int cur = best;
         for (int t = L - 1; t >= 0; --t) {
             accept_path[(long)b * max_path + t] = cur;
-            cur = tree->parent[cur];
+            cur = par[cur];
         }
         for (int t = L; t < max_path; ++t) accept_path[(long)b * max_path + t] = -1;
         accept_len[b] = L;

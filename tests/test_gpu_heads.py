@@ -32,13 +32,15 @@ def check(w, parents, inp, ref, out, out2):
     assert_float_parity(out["logits"], ref["logits"], dt, "logits")
     assert_float_parity(out["probs"], ref["probs"], dt, "probs")
     # h^(k): fp32; or bf16 on both sides, equal up to one bf16 step where the
-    # fp32 pre-activation sits on a rounding boundary (|step| <= 2^-7 |x|)
+    # fp32 pre-activation sits on a rounding boundary (|step| <= 2^-7 |x|),
+    # plus an absolute 1e-3 where SiLU(z) + h nearly cancels (there the fp32
+    # accumulation order of z, ~d * 2^-24 relative, moves a tiny value)
     hres = out["h_res"].float().cpu().numpy()
     if dt == torch.float32:
         assert np.abs(hres - ref["hk"]).max() <= tol
     else:
         diff = np.abs(hres - ref["hk"])
-        assert (diff <= 2.0 ** -7 * np.abs(ref["hk"]) + 1e-30).all()
+        assert (diff <= 2.0 ** -7 * np.abs(ref["hk"]) + 1e-3).all()
         assert (diff == 0).mean() > 0.99
     ti = out["topk_idx"].cpu().numpy()
     tp = out["topk_prob"].cpu().numpy()
