@@ -292,6 +292,8 @@ __global__ void __launch_bounds__(kThreads) tree_attn_mma_kernel(const __grid_co
 }
 
 // One warp per output row (b, node, q-head): log-sum-exp merge of the splits.
+// Lane s holds split s's log-sum-exp (32 splits at a time), so the row's
+// loads are independent of each other.
 template <int D>
 __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restrict__ part_o,
                                                            const float* __restrict__ part_lse, int B, int T, int Hq,
@@ -306,21 +308,43 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restri
     const int G = Hq / Hkv, g = h / G, hh = h % G;
     const int R = T * G, r = i * G + hh;
     const long BH = (long)B * Hkv, bg = (long)b * Hkv + g;
-    float M = -INFINITY;
-    for (int s = 0; s < n_splits; ++s) M = fmaxf(M, part_lse[((long)s * BH + bg) * R + r]);
     constexpr int PL = D / 32;
     float acc[PL];
 #pragma unroll
     for (int e = 0; e < PL; ++e) acc[e] = 0.f;
-    float wsum = 0.f;
-    if (M > -INFINITY) {
-        for (int s = 0; s < n_splits; ++s) {
-            const float ls = part_lse[((long)s * BH + bg) * R + r];
-            const float w = exp2f(ls - M);
-            wsum += w;
-            const float* src = part_o + (((long)s * BH + bg) * R + r) * D + lane * PL;
+    float M = -INFINITY, wsum = 0.f;
+    for (int s0 = 0; s0 < n_splits; s0 += 32) {
+        const int s = s0 + lane;
+        const float ls = s < n_splits ? __ldg(&part_lse[((long)s * BH + bg) * R + r]) : -INFINITY;
+        float m2 = ls;
 #pragma unroll
-            for (int e = 0; e < PL; ++e) acc[e] += w * src[e];
+        for (int o = 16; o > 0; o >>= 1) m2 = fmaxf(m2, __shfl_xor_sync(kFull, m2, o));
+        if (m2 == -INFINITY) continue;
+        const float Mn = fmaxf(M, m2);
+        const float rescale = M == -INFINITY ? 0.f : exp2f(M - Mn);
+        wsum *= rescale;
+#pragma unroll
+        for (int e = 0; e < PL; ++e) acc[e] *= rescale;
+        M = Mn;
+        const float w = ls == -INFINITY ? 0.f : exp2f(ls - M);
+        const int cnt = min(32, n_splits - s0);
+        for (int t0 = 0; t0 < cnt; t0 += 8) {  // 8 splits' loads in flight at once
+            float vals[8][PL];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const float* src = part_o + (((long)(s0 + t0 + u) * BH + bg) * R + r) * D + lane * PL;
+#pragma unroll
+                for (int e = 0; e < PL; ++e) vals[u][e] = t0 + u < cnt ? __ldg(&src[e]) : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const float wt = __shfl_sync(kFull, w, (t0 + u) & 31);
+                if (t0 + u < cnt) {
+                    wsum += wt;
+#pragma unroll
+                    for (int e = 0; e < PL; ++e) acc[e] += wt * vals[u][e];
+                }
+            }
         }
     }
     const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
@@ -388,12 +412,14 @@ struct SplitPlan {
     int m_tiles, n_splits, split_len;
 };
 
-SplitPlan plan_splits(int B, int T, int Hq, int Hkv, int max_prefix) {
+// Key splits so that the grid fills the GPU: tile_rows query rows per CTA,
+// `waves` CTAs per SM targeted.
+SplitPlan plan_splits(int B, int T, int Hq, int Hkv, int max_prefix, int tile_rows = kBM, int waves = 2) {
     SplitPlan sp;
     const int R = T * (Hq / Hkv);
-    sp.m_tiles = (R + kBM - 1) / kBM;
+    sp.m_tiles = (R + tile_rows - 1) / tile_rows;
     const long per_split = (long)sp.m_tiles * B * Hkv;
-    const long target = 2L * num_sms();
+    const long target = (long)waves * num_sms();
     int nps = 0;
     sp.split_len = kBN;
     if (max_prefix > 0) {
@@ -410,9 +436,15 @@ SplitPlan plan_splits(int B, int T, int Hq, int Hkv, int max_prefix) {
     return sp;
 }
 
+SplitPlan plan_bf16(int B, int T, int Hq, int Hkv, int D, int max_prefix) {
+    // tensor-core kernel: 128-row tiles, two CTAs per SM
+    if (attn_tc_supported(Hq, Hkv, D, T, MEDUSA_BF16)) return plan_splits(B, T, Hq, Hkv, max_prefix, 128, 2);
+    return plan_splits(B, T, Hq, Hkv, max_prefix);
+}
+
 template <int D>
 cudaError_t attn_launch_bf16(const AttnArgs& a, cudaStream_t st) {
-    SplitPlan sp = plan_splits(a.B, a.T, a.Hq, a.Hkv, a.max_prefix);
+    SplitPlan sp = plan_bf16(a.B, a.T, a.Hq, a.Hkv, D, a.max_prefix);
     AttnParams p;
     p.q = (const __nv_bfloat16*)a.q;
     p.k_tree = (const __nv_bfloat16*)a.k_tree;
@@ -437,11 +469,16 @@ cudaError_t attn_launch_bf16(const AttnArgs& a, cudaStream_t st) {
     p.part_o = (float*)a.ws;
     p.part_lse = (float*)((char*)a.ws + align256((size_t)sp.n_splits * BH * p.R * D * sizeof(float)));
     p.status = a.status;
-    const size_t smem = (size_t)kBM * D * 2 + 4 * (size_t)kBN * D * 2 + kBM * 4 * sizeof(uint32_t);
-    cudaFuncSetAttribute(tree_attn_mma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    dim3 grid(sp.m_tiles, (unsigned)BH, sp.n_splits);
-    tree_attn_mma_kernel<D><<<grid, kThreads, smem, st>>>(p);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e;
+    if (attn_tc_supported(a.Hq, a.Hkv, D, a.T, a.dt)) {
+        e = attn_tc_launch(a, sp.m_tiles, sp.n_splits, sp.split_len, p.scale_log2, p.part_o, p.part_lse, st);
+    } else {
+        const size_t smem = (size_t)kBM * D * 2 + 4 * (size_t)kBN * D * 2 + kBM * 4 * sizeof(uint32_t);
+        cudaFuncSetAttribute(tree_attn_mma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        dim3 grid(sp.m_tiles, (unsigned)BH, sp.n_splits);
+        tree_attn_mma_kernel<D><<<grid, kThreads, smem, st>>>(p);
+        e = cudaGetLastError();
+    }
     if (e != cudaSuccess) return e;
     const long rows = (long)a.B * a.T * a.Hq;
     attn_combine_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(p.part_o, p.part_lse, a.B, a.T, a.Hq, a.Hkv,
@@ -464,7 +501,7 @@ cudaError_t attn_launch_f32(const AttnArgs& a, cudaStream_t st) {
 
 size_t attn_workspace_size(int B, int T, int Hq, int Hkv, int D, int max_prefix, medusa_dtype dt) {
     if (dt != MEDUSA_BF16) return 0;
-    SplitPlan sp = plan_splits(B, T, Hq, Hkv, max_prefix);
+    SplitPlan sp = plan_bf16(B, T, Hq, Hkv, D, max_prefix);
     const size_t R = (size_t)T * (Hq / Hkv);
     const size_t BH = (size_t)B * Hkv;
     return align256(sp.n_splits * BH * R * D * sizeof(float)) + align256(sp.n_splits * BH * R * sizeof(float));

@@ -1,0 +1,436 @@
+// Tree attention on the 5th-generation tensor cores (bf16, head_dim 64/128,
+// a power-of-two number of q-heads per kv-head).
+//
+// Operation ("Medusa Explained: Multi-Head Speculative Decoding Guide",
+// section "2. Single-Pass Tree Attention Verification"; "Multi-Token
+// Prediction & Draft-Model-Free Speculative Decoding", section "The 2D Tree
+// Attention Mask"): every tree node attends to the cached prefix and to its
+// ancestors and itself.
+//
+// One CTA takes 128 query rows of one (sequence, kv-head) -- rows are
+// node-major, row = node * G + (q-head within the group), so the G q-heads
+// of a node share every K/V element -- and one range of keys (a prefix split
+// or the tree itself).  Per 64-key chunk:
+//   S   = Q K^T      tcgen05.mma M=128, N=64,  K=D   (both operands K-major)
+//   P   = exp2(S * scale * log2 e - m), masked; bf16 into shared memory
+//   O  += P V        tcgen05.mma M=128, N=D,   K=64  (V read MN-major)
+// with fp32 accumulators in TMEM (S double-buffered, O accumulated across
+// chunks).  When a row's running max rises, its softmax thread rescales the
+// row of O in TMEM by alpha = exp2(m_old - m_new) before the next PV (rows
+// whose max did not change are left alone: alpha would be 1).
+// Warps: 0 TMA producer (Q once, K/V chunks in a 2-stage ring), 1 TMEM
+// allocation + MMA issue (QK of chunk j+1 overlaps the softmax of chunk j),
+// 2-5 softmax / output.  Prefix chunks are laid out backwards from the
+// sequence's prefix end, so no cache slot at or past prefix_len is ever read
+// (the first chunk may reach before the split's start: those keys are
+// finite cache entries or zero-filled, and masked).  Tree keys are masked
+// with each row's ancestor bitmask.  Each CTA writes its normalised partial
+// output and log-sum-exp; a combine kernel merges the splits.  Every wait
+// is bounded (~2 s) and sets MEDUSA_STATUS_TIMEOUT on expiry.
+#include <limits.h>
+
+#include "kernels.h"
+#include "tc.cuh"
+#include "tma.h"
+
+namespace medusa {
+
+namespace {
+
+constexpr int kAW = 6;       // 0 producer, 1 MMA, 2-5 softmax
+constexpr int kAM = 128;     // query rows per CTA (MMA M)
+constexpr int kCh = 64;      // keys per chunk
+constexpr int kKVStages = 2;  // with one P buffer: ~112 KB, two CTAs per SM
+
+struct TcAttnArgs {
+    CUtensorMap mq;    // q as (D, Hq, B*T), box (64, G, 128/G)
+    CUtensorMap mkc;   // k_cache as (D, S_max, B*Hkv), box (64, 64, 1)
+    CUtensorMap mvc;
+    CUtensorMap mkt;   // k_tree as (D, Hkv, B*T), box (64, 1, 64)
+    CUtensorMap mvt;
+    const int32_t* prefix_len;
+    const TreeDev* tree;
+    float* part_o;     // [n_splits][B*Hkv][R][D]
+    float* part_lse;   // [n_splits][B*Hkv][R], log2 units
+    int32_t* status;
+    int B, T, Hq, Hkv, G, S_max, max_prefix, R, n_splits, split_len;
+    float scale_log2;
+};
+
+// descriptor of an MN-major operand stored as TMA writes a (64 MN x rows K)
+// box with a 128-byte swizzle: 8 K-rows of 128 bytes per 1024-byte group;
+// `lbo` = byte distance to the next 64-element MN block
+__device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t smem_byte_addr, uint32_t lbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((smem_byte_addr & 0x3FFFFu) >> 4);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)(1024u >> 4) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+template <int D>
+__global__ void __launch_bounds__(kAW * 32, 2) tree_attn_tc_kernel(const __grid_constant__ TcAttnArgs a) {
+    constexpr int NSUB = D / 64;              // 64-element blocks along D
+    constexpr int kQBytes = kAM * D * 2;
+    constexpr int kSub = kCh * 128;           // [64 keys x 64 D] block = 8 KB
+    constexpr int kKVBytes = kCh * D * 2;
+    constexpr int kPBytes = kAM * kCh * 2;    // 16 KB
+    constexpr uint32_t kIdescQK = idesc_bf16_f32(kAM, kCh);
+    constexpr uint32_t kIdescPV = idesc_bf16_f32(kAM, D) | (1u << 16);  // B operand (V) MN-major
+    constexpr uint32_t kTmemCols = 256;       // S: 2 x 64 columns, O: D columns at 128
+    // Dynamic shared memory starts on a 1024-byte boundary when the kernel has
+    // no static shared memory; the tiles below rely on it (checked at entry,
+    // so two CTAs fit per SM without alignment padding).
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint8_t* sQ = smem;
+    uint8_t* sK = sQ + kQBytes;
+    uint8_t* sV = sK + kKVStages * kKVBytes;
+    uint8_t* sP = sV + kKVStages * kKVBytes;  // one P tile: the softmax writes chunk j+1 after PV(j) completed
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sP + kPBytes);
+    uint64_t* q_full = bars;
+    uint64_t* kv_full = bars + 1;
+    uint64_t* kv_empty = bars + 1 + kKVStages;
+    uint64_t* s_full = bars + 1 + 2 * kKVStages;
+    uint64_t* s_free = s_full + 2;
+    uint64_t* p_full = s_free + 2;
+    uint64_t* o_full = p_full + 2;
+    uint64_t* o_free = o_full + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_free + 1);
+
+    const int mt = blockIdx.x, bg = blockIdx.y, split = blockIdx.z;
+    const int b = bg / a.Hkv, g = bg % a.Hkv;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const bool tree_split = split == a.n_splits - 1;
+    if (smem_addr(smem) & 1023u) {  // never expected; refuse rather than misread swizzled tiles
+        if (threadIdx.x == 0) set_status(a.status, MEDUSA_STATUS_TIMEOUT);
+        return;
+    }
+    const int NB = kAM / a.G;  // nodes per tile
+
+    int S = a.prefix_len[b];
+    if (S < 0 || S > a.max_prefix) {
+        if (threadIdx.x == 0 && split == 0 && mt == 0 && g == 0) set_status(a.status, MEDUSA_STATUS_BAD_PREFIX);
+        S = S < 0 ? 0 : a.max_prefix;
+    }
+    int k_begin, k_end, nc;
+    if (tree_split) {
+        k_begin = 0;
+        k_end = a.T;
+        nc = (a.T + kCh - 1) / kCh;
+    } else {
+        k_begin = split * a.split_len;
+        k_end = min(S, k_begin + a.split_len);
+        nc = k_end > k_begin ? (k_end - k_begin + kCh - 1) / kCh : 0;
+    }
+    // first key of chunk j (prefix chunks end exactly at k_end)
+    auto chunk_start = [&](int j) { return tree_split ? j * kCh : k_end - (nc - j) * kCh; };
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        for (int s = 0; s < kKVStages; ++s) {
+            mbar_init(&kv_full[s], 1);
+            mbar_init(&kv_empty[s], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s_full[i], 1);
+            mbar_init(&s_free[i], 4);
+            mbar_init(&p_full[i], 4);
+        }
+        mbar_init(o_full, 1);
+        mbar_init(o_free, 4);  // unused
+        mbar_fence_init();
+    }
+    if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ---------------- producer ----------------
+        if (lane == 0 && nc > 0) {
+            int issued = 0;
+            mbar_arrive_expect_tx(q_full, kQBytes);
+#pragma unroll
+            for (int sub = 0; sub < NSUB; ++sub)
+                tma_load_3d(sQ + sub * (kAM * 128), &a.mq, sub * 64, g * a.G, b * a.T + mt * NB, q_full);
+            for (int j = 0; j < nc; ++j) {
+                const int s = j % kKVStages;
+                if (j >= kKVStages && !mbar_wait(&kv_empty[s], ((j / kKVStages) - 1) & 1)) {
+                    set_status(a.status, MEDUSA_STATUS_TIMEOUT);
+                    break;
+                }
+                const int cs = chunk_start(j);
+                mbar_arrive_expect_tx(&kv_full[s], 2 * kKVBytes);
+#pragma unroll
+                for (int sub = 0; sub < NSUB; ++sub) {
+                    uint8_t* dk = sK + s * kKVBytes + sub * kSub;
+                    uint8_t* dv = sV + s * kKVBytes + sub * kSub;
+                    if (tree_split) {
+                        tma_load_3d(dk, &a.mkt, sub * 64, g, b * a.T + cs, &kv_full[s]);
+                        tma_load_3d(dv, &a.mvt, sub * 64, g, b * a.T + cs, &kv_full[s]);
+                    } else {
+                        tma_load_3d(dk, &a.mkc, sub * 64, cs, bg, &kv_full[s]);
+                        tma_load_3d(dv, &a.mvc, sub * 64, cs, bg, &kv_full[s]);
+                    }
+                }
+                ++issued;
+            }
+            mbar_wait(q_full, 0);
+            for (int s = 0; s < kKVStages && s < issued; ++s) {  // drain before exit
+                const int last = s + ((issued - 1 - s) / kKVStages) * kKVStages;
+                mbar_wait(&kv_full[s], (last / kKVStages) & 1);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0 && nc > 0) {
+            bool ok = mbar_wait(q_full, 0);
+            auto issue_qk = [&](int j) -> bool {
+                const int s = j % kKVStages, sb = j & 1;
+                if (!mbar_wait(&kv_full[s], (j / kKVStages) & 1)) return false;
+                if (j >= 2 && !mbar_wait(&s_free[sb], ((j >> 1) - 1) & 1)) return false;
+                tc_fence_after();
+#pragma unroll
+                for (int sub = 0; sub < NSUB; ++sub) {
+                    const uint64_t ad = sw128_kmajor_desc(smem_addr(sQ + sub * (kAM * 128)));
+                    const uint64_t bd = sw128_kmajor_desc(smem_addr(sK + s * kKVBytes + sub * kSub));
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        tc_mma_bf16(tmem + sb * kCh, ad + 2 * ks, bd + 2 * ks, kIdescQK, (sub | ks) != 0);
+                }
+                tc_commit(&s_full[sb]);
+                return true;
+            };
+            if (ok) ok = issue_qk(0);
+            for (int j = 0; j < nc && ok; ++j) {
+                if (j + 1 < nc && !(ok = issue_qk(j + 1))) break;
+                if (!mbar_wait(&p_full[j & 1], (j >> 1) & 1)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const int s = j % kKVStages;
+                const uint64_t ad = sw128_kmajor_desc(smem_addr(sP));
+                const uint64_t bd = sw128_mnmajor_desc(smem_addr(sV + s * kKVBytes), kSub);
+#pragma unroll
+                for (int ks = 0; ks < kCh / 16; ++ks)  // 16 keys: +32 B in P, +2 K-groups (2048 B) in V
+                    tc_mma_bf16(tmem + 128, ad + 2 * ks, bd + (uint64_t)(2048 >> 4) * ks, kIdescPV, (j | ks) != 0);
+                tc_commit(o_full);
+                tc_commit(&kv_empty[s]);
+            }
+            if (!ok) set_status(a.status, MEDUSA_STATUS_TIMEOUT);
+            else mbar_wait(o_full, (nc - 1) & 1);  // every MMA done before TMEM is released
+        }
+    } else {
+        // ---------------- softmax / output ----------------
+        const int q = warp & 3;
+        const int lr = q * 32 + lane;
+        const int r = mt * kAM + lr;
+        const bool row_ok = r < a.R;
+        const int node = row_ok ? r / a.G : 0;
+        uint32_t anc[4] = {0u, 0u, 0u, 0u};
+        if (tree_split && row_ok)
+#pragma unroll
+            for (int w = 0; w < 4; ++w) anc[w] = a.tree->anc[node][w];
+        float m = -INFINITY, l = 0.f;
+        bool ok = true;
+        const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
+        for (int j = 0; j < nc && ok; ++j) {
+            if (!mbar_wait(&s_full[j & 1], (j >> 1) & 1)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            float sv[kCh];
+            {
+                uint32_t raw[kCh / 16][16];
+#pragma unroll
+                for (int c = 0; c < kCh / 16; ++c) tmem_ld16_async(lane_base + (j & 1) * kCh + c * 16, raw[c]);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < kCh / 16; ++c)
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) sv[c * 16 + e] = __uint_as_float(raw[c][e]);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_free[j & 1]);
+            // mask and online softmax (log2 domain)
+            const int key0 = chunk_start(j);
+            float mx = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < kCh; ++c) {
+                const int key = key0 + c;
+                bool vis;
+                if (tree_split) vis = key < a.T && ((anc[(key >> 5) & 3] >> (key & 31)) & 1u);
+                else vis = key >= k_begin;
+                sv[c] = vis ? sv[c] * a.scale_log2 : -INFINITY;
+                mx = fmaxf(mx, sv[c]);
+            }
+            const float mn = fmaxf(m, mx);
+            const float mu = mn == -INFINITY ? 0.f : mn;
+            const float alpha = exp2f(m - mu);
+            float rs = 0.f;
+            uint8_t* prow = sP + lr * 128;
+            // the previous PV still reads P and accumulates into O: wait for it
+            if (j >= 1 && !mbar_wait(o_full, (j - 1) & 1)) {
+                ok = false;
+                break;
+            }
+#pragma unroll
+            for (int cc = 0; cc < kCh / 8; ++cc) {
+                uint32_t w4[4];
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    const float p0 = exp2f(sv[cc * 8 + 2 * h] - mu);
+                    const float p1 = exp2f(sv[cc * 8 + 2 * h + 1] - mu);
+                    rs += p0 + p1;
+                    __nv_bfloat162 pk = __floats2bfloat162_rn(p0, p1);
+                    w4[h] = *reinterpret_cast<uint32_t*>(&pk);
+                }
+                *reinterpret_cast<uint4*>(prow + ((cc ^ (lr & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+            }
+            l = l * alpha + rs;
+            // rescale this warp's rows of O when some row's max rose
+            if (j >= 1 && __any_sync(kFull, mn > m)) {
+                tc_fence_after();
+                const float f = mn > m ? alpha : 1.f;
+#pragma unroll
+                for (int c0 = 0; c0 < D / 16; c0 += 4) {
+                    uint32_t raw[4][16];
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        if (c0 + c < D / 16) tmem_ld16_async(lane_base + 128 + (c0 + c) * 16, raw[c]);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        if (c0 + c < D / 16) {
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) raw[c][e] = __float_as_uint(__uint_as_float(raw[c][e]) * f);
+                            tmem_st16(lane_base + 128 + (c0 + c) * 16, raw[c]);
+                        }
+                }
+                tmem_wait_st();
+            }
+            m = mn;
+            fence_proxy_async_smem();  // P is read by the tensor core (async proxy)
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_full[j & 1]);
+        }
+        // final O (after the last PV) for this row
+        float o[D];
+        if (ok && nc > 0) {
+            if (!mbar_wait(o_full, (nc - 1) & 1)) ok = false;
+        }
+        if (ok && nc > 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int c0 = 0; c0 < D / 16; c0 += 4) {
+                uint32_t raw[4][16];
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    if (c0 + c < D / 16) tmem_ld16_async(lane_base + 128 + (c0 + c) * 16, raw[c]);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    if (c0 + c < D / 16)
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) o[(c0 + c) * 16 + e] = __uint_as_float(raw[c][e]);
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < D; ++e) o[e] = 0.f;
+        }
+        if (!ok && lane == 0) set_status(a.status, MEDUSA_STATUS_TIMEOUT);
+        if (row_ok) {
+            const long BH = (long)a.B * a.Hkv;
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            float* dst = a.part_o + (((long)split * BH + bg) * a.R + r) * D;
+#pragma unroll
+            for (int e = 0; e < D; e += 4)
+                *reinterpret_cast<float4*>(dst + e) = make_float4(o[e] * inv, o[e + 1] * inv, o[e + 2] * inv, o[e + 3] * inv);
+            a.part_lse[((long)split * BH + bg) * a.R + r] = l > 0.f ? m + log2f(l) : -INFINITY;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+template <int D>
+size_t tc_attn_smem() {
+    return (size_t)kAM * D * 2 + 2 * (size_t)kKVStages * kCh * D * 2 + (size_t)kAM * kCh * 2 + 16 * 8 + 16;
+}
+
+}  // namespace
+
+bool attn_tc_supported(int Hq, int Hkv, int D, int T, medusa_dtype dt) {
+    const int G = Hkv > 0 ? Hq / Hkv : 0;
+    return dt == MEDUSA_BF16 && (D == 64 || D == 128) && G >= 1 && G <= 16 && (G & (G - 1)) == 0 && T <= kMaxTree;
+}
+
+// launch the tensor-core split kernel; the caller provides the split plan and
+// the partial buffers (same layout as the other bf16 path) and runs the combine
+cudaError_t attn_tc_launch(const AttnArgs& x, int m_tiles, int n_splits, int split_len, float scale_log2,
+                           float* part_o, float* part_lse, cudaStream_t st) {
+    TcAttnArgs a;
+    const uint64_t D = x.D, Hq = x.Hq, Hkv = x.Hkv, BT = (uint64_t)x.B * x.T, Smax = x.S_max, BH = (uint64_t)x.B * x.Hkv;
+    const int G = x.Hq / x.Hkv;
+    {
+        const uint64_t dims[3] = {D, Hq, BT}, strides[2] = {D * 2, Hq * D * 2};
+        const uint32_t box[3] = {64, (uint32_t)G, (uint32_t)(kAM / G)};
+        if (!make_tmap_bf16(&a.mq, x.q, 3, dims, strides, box)) return cudaErrorInvalidValue;
+    }
+    {
+        const uint64_t dims[3] = {D, Smax, BH}, strides[2] = {D * 2, Smax * D * 2};
+        const uint32_t box[3] = {64, (uint32_t)kCh, 1};
+        if (!make_tmap_bf16(&a.mkc, x.k_cache, 3, dims, strides, box)) return cudaErrorInvalidValue;
+        if (!make_tmap_bf16(&a.mvc, x.v_cache, 3, dims, strides, box)) return cudaErrorInvalidValue;
+    }
+    {
+        const uint64_t dims[3] = {D, Hkv, BT}, strides[2] = {D * 2, Hkv * D * 2};
+        const uint32_t box[3] = {64, 1, (uint32_t)kCh};
+        if (!make_tmap_bf16(&a.mkt, x.k_tree, 3, dims, strides, box)) return cudaErrorInvalidValue;
+        if (!make_tmap_bf16(&a.mvt, x.v_tree, 3, dims, strides, box)) return cudaErrorInvalidValue;
+    }
+    a.prefix_len = x.prefix_len;
+    a.tree = x.tree;
+    a.part_o = part_o;
+    a.part_lse = part_lse;
+    a.status = x.status;
+    a.B = x.B;
+    a.T = x.T;
+    a.Hq = x.Hq;
+    a.Hkv = x.Hkv;
+    a.G = G;
+    a.S_max = x.S_max;
+    a.max_prefix = x.max_prefix;
+    a.R = x.T * G;
+    a.n_splits = n_splits;
+    a.split_len = split_len;
+    a.scale_log2 = scale_log2;
+    const dim3 grid(m_tiles, (unsigned)BH, n_splits);
+    if (x.D == 128) {
+        const size_t smem = tc_attn_smem<128>();
+        cudaFuncSetAttribute(tree_attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        tree_attn_tc_kernel<128><<<grid, kAW * 32, smem, st>>>(a);
+    } else {
+        const size_t smem = tc_attn_smem<64>();
+        cudaFuncSetAttribute(tree_attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        tree_attn_tc_kernel<64><<<grid, kAW * 32, smem, st>>>(a);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace medusa

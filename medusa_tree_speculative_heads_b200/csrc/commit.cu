@@ -18,24 +18,24 @@ __global__ void __launch_bounds__(256) kv_commit_kernel(uint8_t* __restrict__ kc
     __shared__ int s_ok, s_S, s_L;
     __shared__ int s_node[MEDUSA_MAX_TREE];
     const int b = blockIdx.x, tid = threadIdx.x;
+    // read prefix_len before anything is written: new_prefix_len may alias it
+    const int S = prefix_len[b], L = len[b];
+    const bool len_ok = L >= 0 && L <= max_path && L <= MEDUSA_MAX_TREE && S >= 0;
+    bool node_ok = true;
+    if (len_ok && tid < L) {  // every path entry loaded at once
+        const int n = path[(long)b * max_path + tid];
+        node_ok = n >= 0 && n < T;
+        s_node[tid] = n;
+    }
+    const bool all_nodes_ok = __syncthreads_and(node_ok);
     if (tid == 0) {
-        // read prefix_len before anything is written: new_prefix_len may alias it
-        const int S = prefix_len[b], L = len[b];
         int ok = 1;
-        if (L < 0 || L > max_path || L > MEDUSA_MAX_TREE || S < 0) {
+        if (!len_ok || !all_nodes_ok) {
             ok = 0;
             set_status(status, MEDUSA_STATUS_BAD_TOKEN);
         } else if (S + L > S_max) {
             ok = 0;
             set_status(status, MEDUSA_STATUS_CACHE_OVERFLOW);
-        }
-        for (int t = 0; ok && t < L; ++t) {
-            const int n = path[(long)b * max_path + t];
-            if (n < 0 || n >= T) {
-                ok = 0;
-                set_status(status, MEDUSA_STATUS_BAD_TOKEN);
-            }
-            s_node[t] = n;
         }
         s_ok = ok;
         s_S = S;

@@ -24,7 +24,7 @@ namespace medusa {
 
 namespace {
 
-constexpr int kArgmaxThreads = 256;
+constexpr int kArgmaxThreads = 512;
 constexpr int kStochThreads = 512;
 
 // ------------------------------- greedy ------------------------------------
@@ -36,23 +36,27 @@ __device__ __forceinline__ void argmax_merge(float& bv, int& bi, float v, int i)
     }
 }
 
-template <typename T>
-__global__ void __launch_bounds__(kArgmaxThreads) row_argmax_kernel(const T* __restrict__ x, int V, int splits,
+// Row argmax partials over vocabulary chunks, one block per (row, chunk),
+// 8 independent 16-byte loads in flight per thread.
+template <typename E>
+__global__ void __launch_bounds__(kArgmaxThreads, 2) row_argmax_kernel(const E* __restrict__ x, int V, int splits,
                                                                     int chunk, float* __restrict__ pval,
                                                                     int* __restrict__ pidx) {
-    constexpr int VEC = Elt<T>::kVec;
+    constexpr int VEC = Elt<E>::kVec;
+    constexpr int NW = kArgmaxThreads / 32;
+    constexpr int U = 8;
     const long row = blockIdx.x;
     const int s = blockIdx.y;
     const int v0 = s * chunk;
     const int v1 = min(V, v0 + chunk);
-    const T* rp = x + row * (long)V;
+    const E* rp = x + row * (long)V;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     float bv = -INFINITY;
     int bi = v0;  // lowest index of the chunk: the answer when nothing beats -inf
     if (v0 < v1) {
         int va = v0;
         if ((((uintptr_t)(rp + v0)) & 15) == 0) {
             const int nvec = (v1 - v0) / VEC;
-            constexpr int U = 4;  // independent 16-byte loads in flight per thread
             for (int c0 = threadIdx.x; c0 < nvec; c0 += U * kArgmaxThreads) {
                 uint4 raw[U];
 #pragma unroll
@@ -65,7 +69,7 @@ __global__ void __launch_bounds__(kArgmaxThreads) row_argmax_kernel(const T* __r
                     const int c = c0 + u * kArgmaxThreads;
                     if (c < nvec) {
                         float f[VEC];
-                        Elt<T>::unpack(raw[u], f);
+                        Elt<E>::unpack(raw[u], f);
 #pragma unroll
                         for (int e = 0; e < VEC; ++e) argmax_merge(bv, bi, f[e], v0 + c * VEC + e);
                     }
@@ -73,74 +77,94 @@ __global__ void __launch_bounds__(kArgmaxThreads) row_argmax_kernel(const T* __r
             }
             va = v0 + nvec * VEC;
         }
-        for (int v = va + threadIdx.x; v < v1; v += kArgmaxThreads) argmax_merge(bv, bi, Elt<T>::to_float(rp[v]), v);
+        for (int v = va + threadIdx.x; v < v1; v += kArgmaxThreads) argmax_merge(bv, bi, Elt<E>::to_float(rp[v]), v);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
-        float ov = __shfl_xor_sync(kFull, bv, o);
-        int oi = __shfl_xor_sync(kFull, bi, o);
+        const float ov = __shfl_xor_sync(kFull, bv, o);
+        const int oi = __shfl_xor_sync(kFull, bi, o);
         argmax_merge(bv, bi, ov, oi);
     }
-    __shared__ float sv[kArgmaxThreads / 32];
-    __shared__ int si[kArgmaxThreads / 32];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    __shared__ float sv[NW];
+    __shared__ int si[NW];
     if (lane == 0) {
         sv[warp] = bv;
         si[warp] = bi;
     }
     __syncthreads();
-    if (warp == 0) {
-        bv = lane < kArgmaxThreads / 32 ? sv[lane] : -INFINITY;
-        bi = lane < kArgmaxThreads / 32 ? si[lane] : INT_MAX;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            float ov = __shfl_xor_sync(kFull, bv, o);
-            int oi = __shfl_xor_sync(kFull, bi, o);
-            argmax_merge(bv, bi, ov, oi);
-        }
-        if (lane == 0) {
-            pval[row * splits + s] = bv;
-            pidx[row * splits + s] = bi;
-        }
+    if (threadIdx.x == 0) {
+        for (int w = 1; w < NW; ++w) argmax_merge(bv, bi, sv[w], si[w]);
+        pval[row * splits + s] = bv;
+        pidx[row * splits + s] = bi;
     }
 }
 
-// One warp per sequence: predictions of all nodes, then the accepted set in
-// index order (a parent precedes its children) and the deepest accepted node.
-__global__ void __launch_bounds__(32) greedy_walk_kernel(const float* __restrict__ pval, const int* __restrict__ pidx,
-                                                         int splits, const int32_t* __restrict__ node_tokens,
-                                                         const TreeDev* __restrict__ tree, int32_t* accept_path,
-                                                         int max_path, int32_t* accept_len, int32_t* bonus) {
-    __shared__ int pred[kMaxTree], tok[kMaxTree], par[kMaxTree], dep[kMaxTree];
-    __shared__ uint8_t acc[kMaxTree];
-    const int b = blockIdx.x, lane = threadIdx.x;
+// One block of 128 threads per sequence, one thread per node: node u's
+// prediction is the merge of its partials (split order); node c "matches"
+// when its token equals its parent's prediction (the root always does).  A
+// node is accepted iff every node on its root path matches, i.e. iff its
+// ancestor bitmask has no bit outside the match mask.  The deepest accepted
+// node (lowest index among equally deep ones) ends the path, whose nodes are
+// the set bits of its ancestor mask in increasing index order (a parent's
+// index is below its child's).
+constexpr int kWalkThreads = kMaxTree;
+constexpr int kMaxSplits = 16;
+__global__ void __launch_bounds__(kWalkThreads) greedy_walk_kernel(const float* __restrict__ pval,
+                                                                   const int* __restrict__ pidx, int splits,
+                                                                   const int32_t* __restrict__ node_tokens,
+                                                                   const TreeDev* __restrict__ tree,
+                                                                   int32_t* accept_path, int max_path,
+                                                                   int32_t* accept_len, int32_t* bonus) {
+    __shared__ int pred[kMaxTree];
+    __shared__ uint32_t match[kMaxTree / 32];
+    __shared__ int best_key[kMaxTree / 32];
+    const int b = blockIdx.x, u = threadIdx.x, lane = u & 31, w = u >> 5;
     const int T = tree->T;
-    for (int u = lane; u < T; u += 32) {
+    float bv = -INFINITY;
+    int bi = INT_MAX;
+    int tok = 0, par = -1, dep = 0;
+    if (u < T) {
         const long base = ((long)b * T + u) * splits;
-        float bv = -INFINITY;
-        int bi = INT_MAX;
-        for (int s = 0; s < splits; ++s) argmax_merge(bv, bi, pval[base + s], pidx[base + s]);
+        float lv[kMaxSplits];
+        int li[kMaxSplits];
+#pragma unroll
+        for (int s = 0; s < kMaxSplits; ++s) {  // every load issued before any is used
+            lv[s] = s < splits ? pval[base + s] : -INFINITY;
+            li[s] = s < splits ? pidx[base + s] : INT_MAX;
+        }
+        tok = node_tokens[(long)b * T + u];
+        par = tree->parent[u];
+        dep = tree->depth[u];
+#pragma unroll
+        for (int s = 0; s < kMaxSplits; ++s) argmax_merge(bv, bi, lv[s], li[s]);
         pred[u] = bi;
-        tok[u] = node_tokens[(long)b * T + u];
-        par[u] = tree->parent[u];
-        dep[u] = tree->depth[u];
     }
-    __syncwarp();
-    if (lane == 0) {
-        acc[0] = 1;
-        int best = 0;
-        for (int c = 1; c < T; ++c) {
-            const int p = par[c];
-            acc[c] = acc[p] && tok[c] == pred[p];
-            if (acc[c] && dep[c] > dep[best]) best = c;
-        }
-        const int L = dep[best];
-        int cur = best;
-        for (int t = L - 1; t >= 0; --t) {
-            accept_path[(long)b * max_path + t] = cur;
-            cur = par[cur];
-        }
-        for (int t = L; t < max_path; ++t) accept_path[(long)b * max_path + t] = -1;
+    __syncthreads();
+    const bool m = u < T && (u == 0 || tok == pred[par]);
+    const uint32_t mb = __ballot_sync(kFull, m);
+    if (lane == 0) match[w] = mb;
+    __syncthreads();
+    bool accepted = false;
+    if (u < T) {
+        accepted = true;
+#pragma unroll
+        for (int k = 0; k < kMaxTree / 32; ++k) accepted &= (tree->anc[u][k] & ~match[k]) == 0u;
+    }
+    // deepest accepted node, lowest index among equally deep: maximise depth*256 + (255 - index)
+    int key = accepted ? dep * 256 + (255 - u) : -1;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) key = max(key, __shfl_xor_sync(kFull, key, o));
+    if (lane == 0) best_key[w] = key;
+    __syncthreads();
+    if (u == 0) {
+        int k = best_key[0];
+        for (int i = 1; i < kMaxTree / 32; ++i) k = max(k, best_key[i]);
+        const int best = 255 - (k & 255);
+        const int L = k >> 8;
+        int t = 0;
+        for (int j = 0; j <= best; ++j)
+            if ((tree->anc[best][j >> 5] >> (j & 31)) & 1u) accept_path[(long)b * max_path + t++] = j;
+        for (int j = L; j < max_path; ++j) accept_path[(long)b * max_path + j] = -1;
         accept_len[b] = L;
         bonus[b] = pred[best];
     }
@@ -312,10 +336,11 @@ __global__ void __launch_bounds__(kStochThreads) verify_stochastic_kernel(
 }
 
 int argmax_splits(int rows, int V) {
-    int target = 4 * num_sms();
-    int s = (target + rows - 1) / rows;
+    int target = 2 * num_sms();  // two 512-thread blocks per SM: one wave
+    int s = target / rows;
     int max_s = (V + 2047) / 2048;
     if (s > max_s) s = max_s;
+    if (s > kMaxSplits) s = kMaxSplits;
     if (s < 1) s = 1;
     return s;
 }
@@ -345,8 +370,8 @@ cudaError_t verify_launch(const VerifyArgs& a, cudaStream_t st) {
                                                                       pval, pidx);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
-        greedy_walk_kernel<<<a.B, 32, 0, st>>>(pval, pidx, splits, a.node_tokens, a.tree, a.accept_path,
-                                               a.max_path, a.accept_len, a.bonus);
+        greedy_walk_kernel<<<a.B, kWalkThreads, 0, st>>>(pval, pidx, splits, a.node_tokens, a.tree, a.accept_path,
+                                                         a.max_path, a.accept_len, a.bonus);
         return cudaGetLastError();
     }
     verify_stochastic_kernel<<<a.B, kStochThreads, 0, st>>>(
