@@ -292,33 +292,49 @@ def run_mine(args, rank, world, local_rank):
     mean_len = float(step.accept_len.float().mean().item())
 
     # ---- end to end through the public API with host buffers ----
+    # every step copies its own inputs from pinned host memory (h, root token,
+    # the tree's Q/K/V and the target logits) and reads its results back; the
+    # copies run on a second stream into two alternating device buffers, so the
+    # next step's 31 MB upload overlaps this step's compute, as a serving loop would
     names_in = ["h", "root_token", "q", "k_tree", "v_tree"]
     host_in = {n: (hin if n in hin else ain)[n].cpu().pin_memory() for n in names_in}
     host_in["target"] = logits.cpu().pin_memory()
-    dev_in = {n: torch.empty_like(host_in[n], device=dev) for n in host_in}
+    dev_in = [{n: torch.empty_like(host_in[n], device=dev) for n in host_in} for _ in range(2)]
     outs = [step.accept_path, step.accept_len, step.bonus, step.node_tokens]
     host_out = [torch.empty_like(o, device="cpu").pin_memory() for o in outs]
     h2d = sum(x.numel() * x.element_size() for x in host_in.values())
     d2h = sum(x.numel() * x.element_size() for x in host_out)
+    main_stream = torch.cuda.current_stream()
+    copy_stream = torch.cuda.Stream(device=dev)
+    copied = [torch.cuda.Event(), torch.cuda.Event()]
+    used = [torch.cuda.Event(), torch.cuda.Event()]
+    for ev in used:
+        ev.record(main_stream)
 
-    def e2e_step():
-        for n in host_in:
-            dev_in[n].copy_(host_in[n], non_blocking=True)
-        step.run(h=dev_in["h"], W_res=hin["W_res"], W_head=hin["W_head"], root_token=dev_in["root_token"],
-                 q=dev_in["q"], k_tree=dev_in["k_tree"], v_tree=dev_in["v_tree"], k_cache=ain["k_cache"],
-                 v_cache=ain["v_cache"], prefix_len=ain["prefix_len"], new_prefix_len=new_pl,
-                 target=dev_in["target"])
+    def e2e_step(i):
+        slot = i & 1
+        with torch.cuda.stream(copy_stream):
+            copy_stream.wait_event(used[slot])        # the step that last read this buffer is done
+            for n in host_in:
+                dev_in[slot][n].copy_(host_in[n], non_blocking=True)
+            copied[slot].record(copy_stream)
+        main_stream.wait_event(copied[slot])
+        d = dev_in[slot]
+        step.run(h=d["h"], W_res=hin["W_res"], W_head=hin["W_head"], root_token=d["root_token"], q=d["q"],
+                 k_tree=d["k_tree"], v_tree=d["v_tree"], k_cache=ain["k_cache"], v_cache=ain["v_cache"],
+                 prefix_len=ain["prefix_len"], new_prefix_len=new_pl, target=d["target"])
+        used[slot].record(main_stream)
         for o, ho in zip(outs, host_out):
             ho.copy_(o, non_blocking=True)
 
-    for _ in range(3):
-        e2e_step()
+    for i in range(3):
+        e2e_step(i)
     torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
     e0.record()
-    for _ in range(K):
-        e2e_step()
+    for i in range(K):
+        e2e_step(i)
     e1.record()
     torch.cuda.synchronize()
     barrier()

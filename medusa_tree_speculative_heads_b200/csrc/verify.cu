@@ -24,7 +24,7 @@ namespace medusa {
 
 namespace {
 
-constexpr int kArgmaxThreads = 512;
+constexpr int kArgmaxThreads = 256;
 constexpr int kStochThreads = 512;
 
 // ------------------------------- greedy ------------------------------------
@@ -39,7 +39,7 @@ __device__ __forceinline__ void argmax_merge(float& bv, int& bi, float v, int i)
 // Row argmax partials over vocabulary chunks, one block per (row, chunk),
 // 8 independent 16-byte loads in flight per thread.
 template <typename E>
-__global__ void __launch_bounds__(kArgmaxThreads, 2) row_argmax_kernel(const E* __restrict__ x, int V, int splits,
+__global__ void __launch_bounds__(kArgmaxThreads, 4) row_argmax_kernel(const E* __restrict__ x, int V, int splits,
                                                                     int chunk, float* __restrict__ pval,
                                                                     int* __restrict__ pidx) {
     constexpr int VEC = Elt<E>::kVec;
@@ -336,8 +336,8 @@ __global__ void __launch_bounds__(kStochThreads) verify_stochastic_kernel(
 }
 
 int argmax_splits(int rows, int V) {
-    int target = 2 * num_sms();  // two 512-thread blocks per SM: one wave
-    int s = target / rows;
+    int target = 4 * num_sms();  // four 256-thread blocks per SM: one balanced wave
+    int s = (target + rows / 2) / rows;
     int max_s = (V + 2047) / 2048;
     if (s > max_s) s = max_s;
     if (s > kMaxSplits) s = kMaxSplits;
