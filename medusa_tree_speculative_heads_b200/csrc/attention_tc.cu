@@ -12,12 +12,15 @@
 // of a node share every K/V element -- and one range of keys (a prefix split
 // or the tree itself).  Per 64-key chunk:
 //   S   = Q K^T      tcgen05.mma M=128, N=64,  K=D   (both operands K-major)
-//   P   = exp2(S * scale * log2 e - m), masked; bf16 into shared memory
-//   O  += P V        tcgen05.mma M=128, N=D,   K=64  (V read MN-major)
-// with fp32 accumulators in TMEM (S double-buffered, O accumulated across
-// chunks).  When a row's running max rises, its softmax thread rescales the
-// row of O in TMEM by alpha = exp2(m_old - m_new) before the next PV (rows
-// whose max did not change are left alone: alpha would be 1).
+//   P   = exp2(S * scale * log2 e - m), masked; bf16, written back into TMEM
+//         over S's own columns
+//   O  += P V        tcgen05.mma M=128, N=D,   K=64  (A = P from TMEM, V read
+//                    MN-major from shared memory)
+// with fp32 accumulators in TMEM (S/P double-buffered, O accumulated across
+// chunks).  The reference max m of a row is raised only when a chunk's max
+// exceeds it by more than 8 (log2 units), so P <= 2^8; when it is raised the
+// softmax thread rescales its row of O in TMEM by exp2(m_old - m_new) after
+// the previous PV completed.  The result is the same after the final 1/l.
 // Warps: 0 TMA producer (Q once, K/V chunks in a 2-stage ring), 1 TMEM
 // allocation + MMA issue (QK of chunk j+1 overlaps the softmax of chunk j),
 // 2-5 softmax / output.  Prefix chunks are laid out backwards from the
@@ -70,19 +73,14 @@ __device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t smem_byte_addr, 
     return d;
 }
 
-__device__ __forceinline__ void fence_proxy_async_smem() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 template <int D>
 __global__ void __launch_bounds__(kAW * 32, 2) tree_attn_tc_kernel(const __grid_constant__ TcAttnArgs a) {
     constexpr int NSUB = D / 64;              // 64-element blocks along D
     constexpr int kQBytes = kAM * D * 2;
     constexpr int kSub = kCh * 128;           // [64 keys x 64 D] block = 8 KB
     constexpr int kKVBytes = kCh * D * 2;
-    constexpr int kPBytes = kAM * kCh * 2;    // 16 KB
     constexpr uint32_t kIdescQK = idesc_bf16_f32(kAM, kCh);
-    constexpr uint32_t kIdescPV = idesc_bf16_f32(kAM, D) | (1u << 16);  // B operand (V) MN-major
+    constexpr uint32_t kIdescPV = idesc_bf16_f32(kAM, D) | (1u << 16);  // A (P) from TMEM, B (V) MN-major
     constexpr uint32_t kTmemCols = 256;       // S: 2 x 64 columns, O: D columns at 128
     // Dynamic shared memory starts on a 1024-byte boundary when the kernel has
     // no static shared memory; the tiles below rely on it (checked at entry,
@@ -91,17 +89,14 @@ __global__ void __launch_bounds__(kAW * 32, 2) tree_attn_tc_kernel(const __grid_
     uint8_t* sQ = smem;
     uint8_t* sK = sQ + kQBytes;
     uint8_t* sV = sK + kKVStages * kKVBytes;
-    uint8_t* sP = sV + kKVStages * kKVBytes;  // one P tile: the softmax writes chunk j+1 after PV(j) completed
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sP + kPBytes);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sV + kKVStages * kKVBytes);
     uint64_t* q_full = bars;
     uint64_t* kv_full = bars + 1;
     uint64_t* kv_empty = bars + 1 + kKVStages;
     uint64_t* s_full = bars + 1 + 2 * kKVStages;
-    uint64_t* s_free = s_full + 2;
-    uint64_t* p_full = s_free + 2;
+    uint64_t* p_full = s_full + 2;
     uint64_t* o_full = p_full + 2;
-    uint64_t* o_free = o_full + 1;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_free + 1);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_full + 1);
 
     const int mt = blockIdx.x, bg = blockIdx.y, split = blockIdx.z;
     const int b = bg / a.Hkv, g = bg % a.Hkv;
@@ -139,11 +134,9 @@ __global__ void __launch_bounds__(kAW * 32, 2) tree_attn_tc_kernel(const __grid_
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s_full[i], 1);
-            mbar_init(&s_free[i], 4);
             mbar_init(&p_full[i], 4);
         }
         mbar_init(o_full, 1);
-        mbar_init(o_free, 4);  // unused
         mbar_fence_init();
     }
     if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
@@ -192,10 +185,12 @@ __global__ void __launch_bounds__(kAW * 32, 2) tree_attn_tc_kernel(const __grid_
         // ---------------- MMA issuer ----------------
         if (lane == 0 && nc > 0) {
             bool ok = mbar_wait(q_full, 0);
+            // S_j goes to TMEM columns (j&1)*64; P_j is written over it, so the
+            // buffer is free for S_{j+2} once PV_j has completed (o_full phase j)
             auto issue_qk = [&](int j) -> bool {
                 const int s = j % kKVStages, sb = j & 1;
                 if (!mbar_wait(&kv_full[s], (j / kKVStages) & 1)) return false;
-                if (j >= 2 && !mbar_wait(&s_free[sb], ((j >> 1) - 1) & 1)) return false;
+                if (j >= 2 && !mbar_wait(o_full, (j - 2) & 1)) return false;
                 tc_fence_after();
 #pragma unroll
                 for (int sub = 0; sub < NSUB; ++sub) {
@@ -217,11 +212,11 @@ __global__ void __launch_bounds__(kAW * 32, 2) tree_attn_tc_kernel(const __grid_
                 }
                 tc_fence_after();
                 const int s = j % kKVStages;
-                const uint64_t ad = sw128_kmajor_desc(smem_addr(sP));
                 const uint64_t bd = sw128_mnmajor_desc(smem_addr(sV + s * kKVBytes), kSub);
 #pragma unroll
-                for (int ks = 0; ks < kCh / 16; ++ks)  // 16 keys: +32 B in P, +2 K-groups (2048 B) in V
-                    tc_mma_bf16(tmem + 128, ad + 2 * ks, bd + (uint64_t)(2048 >> 4) * ks, kIdescPV, (j | ks) != 0);
+                for (int ks = 0; ks < kCh / 16; ++ks)  // 16 keys: 8 P columns, +2 K-groups (2048 B) in V
+                    tc_mma_bf16_ts(tmem + 128, tmem + (j & 1) * kCh + ks * 8, bd + (uint64_t)(2048 >> 4) * ks,
+                                   kIdescPV, (j | ks) != 0);
                 tc_commit(o_full);
                 tc_commit(&kv_empty[s]);
             }
@@ -259,9 +254,6 @@ __global__ void __launch_bounds__(kAW * 32, 2) tree_attn_tc_kernel(const __grid_
 #pragma unroll
                     for (int e = 0; e < 16; ++e) sv[c * 16 + e] = __uint_as_float(raw[c][e]);
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s_free[j & 1]);
             // mask and online softmax (log2 domain)
             const int key0 = chunk_start(j);
             float mx = -INFINITY;
@@ -274,34 +266,36 @@ __global__ void __launch_bounds__(kAW * 32, 2) tree_attn_tc_kernel(const __grid_
                 sv[c] = vis ? sv[c] * a.scale_log2 : -INFINITY;
                 mx = fmaxf(mx, sv[c]);
             }
-            const float mn = fmaxf(m, mx);
+            // lazy reference max: raised only when the chunk's max exceeds it by > 8
+            const bool raise = mx > m + 8.f;
+            const float mn = raise ? mx : m;
             const float mu = mn == -INFINITY ? 0.f : mn;
-            const float alpha = exp2f(m - mu);
+            const float alpha = raise ? exp2f(m - mu) : 1.f;
             float rs = 0.f;
-            uint8_t* prow = sP + lr * 128;
-            // the previous PV still reads P and accumulates into O: wait for it
-            if (j >= 1 && !mbar_wait(o_full, (j - 1) & 1)) {
-                ok = false;
-                break;
-            }
+            {
+                uint32_t pk[2][16];  // P row: 64 keys as 32 bf16 pairs
 #pragma unroll
-            for (int cc = 0; cc < kCh / 8; ++cc) {
-                uint32_t w4[4];
-#pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    const float p0 = exp2f(sv[cc * 8 + 2 * h] - mu);
-                    const float p1 = exp2f(sv[cc * 8 + 2 * h + 1] - mu);
-                    rs += p0 + p1;
-                    __nv_bfloat162 pk = __floats2bfloat162_rn(p0, p1);
-                    w4[h] = *reinterpret_cast<uint32_t*>(&pk);
+                for (int c = 0; c < kCh / 2; ++c) {
+                    const float p0 = exp2f(sv[2 * c] - mu);
+                    const float p1 = exp2f(sv[2 * c + 1] - mu);
+                    __nv_bfloat162 v2 = __floats2bfloat162_rn(p0, p1);
+                    // the row sum uses the same bf16 weights PV multiplies by
+                    rs += __low2float(v2) + __high2float(v2);
+                    pk[c >> 4][c & 15] = *reinterpret_cast<uint32_t*>(&v2);
                 }
-                *reinterpret_cast<uint4*>(prow + ((cc ^ (lr & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                tmem_st16(lane_base + (j & 1) * kCh, pk[0]);
+                tmem_st16(lane_base + (j & 1) * kCh + 16, pk[1]);
             }
             l = l * alpha + rs;
-            // rescale this warp's rows of O when some row's max rose
-            if (j >= 1 && __any_sync(kFull, mn > m)) {
+            // rescale this warp's rows of O when some row's reference max rose
+            // (after the previous PV has completed)
+            if (j >= 1 && __any_sync(kFull, raise)) {
+                if (!mbar_wait(o_full, (j - 1) & 1)) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
-                const float f = mn > m ? alpha : 1.f;
+                const float f = alpha;
 #pragma unroll
                 for (int c0 = 0; c0 < D / 16; c0 += 4) {
                     uint32_t raw[4][16];
@@ -320,7 +314,7 @@ __global__ void __launch_bounds__(kAW * 32, 2) tree_attn_tc_kernel(const __grid_
                 tmem_wait_st();
             }
             m = mn;
-            fence_proxy_async_smem();  // P is read by the tensor core (async proxy)
+            tmem_wait_st();  // P (and any rescaled O) in TMEM before the MMA reads it
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&p_full[j & 1]);
@@ -370,7 +364,7 @@ __global__ void __launch_bounds__(kAW * 32, 2) tree_attn_tc_kernel(const __grid_
 
 template <int D>
 size_t tc_attn_smem() {
-    return (size_t)kAM * D * 2 + 2 * (size_t)kKVStages * kCh * D * 2 + (size_t)kAM * kCh * 2 + 16 * 8 + 16;
+    return (size_t)kAM * D * 2 + 2 * (size_t)kKVStages * kCh * D * 2 + 16 * 8 + 16;
 }
 
 }  // namespace
