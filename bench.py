@@ -187,12 +187,33 @@ def run_reference(args, rank, world):
 # the CUDA path
 # ----------------------------------------------------------------------------
 
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The slowest rank's value (timings are max-reduced across ranks)."""
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world: int, steps: int, seconds: float) -> float:
+    """Steps per second of the whole job: every rank ran `steps` steps of its
+    own replica; the job took as long as its slowest rank."""
+    return world * steps / seconds
+
+
 def config_dict(w, world):
-    return {"workload": (f"{w.name}: B={w.B} d={w.d} V={w.V} K={w.K} heads, top-s {w.topk} -> 117-node tree, "
-                         f"{w.Hq}/{w.Hkv} heads head_dim {w.D}, prefix {w.prefix}, greedy verify, "
-                         f"match prob {w.match_prob}, one attention layer"),
-            "global_batch": w.B * world, "seq_len": w.prefix, "parallelism": f"replicas x{world}",
-            "l2": "inputs larger than L2: each step streams 4.34 GB of head weights through the 126 MB L2"}
+    from medusa_tree_speculative_heads_b200 import inputs as I
+    T = len(I.workload_tree(w))
+    tree = f"top-s {w.topk}" if w.topk else f"random tree {w.random_tree}"
+    prefix = f"prefix U[{w.prefix_range[0]}, {w.prefix_range[1]}]" if w.prefix_range else f"prefix {w.prefix}"
+    verify = "stochastic verify" if w.stochastic else f"greedy verify, match prob {w.match_prob}"
+    head_gb = w.K * (w.d * w.d + w.V * w.d) * (2 if w.dtype == "bf16" else 4) / 1e9
+    return {"workload": (f"{w.name}: B={w.B} d={w.d} V={w.V} K={w.K} heads, {tree} -> {T}-node tree, "
+                         f"{w.Hq}/{w.Hkv} heads head_dim {w.D}, {prefix}, {verify}, one attention layer"),
+            "global_batch": w.B * world, "seq_len": w.max_prefix, "parallelism": f"replicas x{world}",
+            "l2": f"inputs larger than L2: each step streams {head_gb:.2f} GB of head weights through the 126 MB L2"}
 
 
 def launches_per_step(w, mode_greedy=True):
@@ -206,7 +227,7 @@ def launches_per_step(w, mode_greedy=True):
     else:
         heads = 1 + 2 * ((w.B + 7) // 8)
     attn = 2 if w.dtype == "bf16" else 1
-    verify = 2 if mode_greedy else 1
+    verify = 1 if w.stochastic else 2
     return heads + attn + verify + 1
 
 
@@ -231,26 +252,29 @@ def run_mine(args, rank, world, local_rank):
     T = len(parents)
     hin = I.head_inputs(w, device="cuda")
     ain = I.attention_inputs(w, T, device="cuda")
+    from medusa_tree_speculative_heads_b200 import binding as Bnd
+    mode = Bnd.STOCHASTIC if w.stochastic else Bnd.GREEDY
     step = MedusaStep(B=w.B, d=w.d, V=w.V, K=w.K, Hq=w.Hq, Hkv=w.Hkv, D=w.D, S_max=w.S_max, parents=parents,
-                      dtype=w.torch_dtype, max_prefix=w.max_prefix, device=dev)
-    # the target model's logits (outside this path) are synthesised once from
-    # the tree the heads propose, with the workload's match probability
-    step.heads(hin["h"], hin["W_res"], hin["W_head"], hin["root_token"])
-    torch.cuda.synchronize()
-    logits = I.boosted_target_logits(w, parents, step.node_tokens.cpu(), device="cuda")
+                      dtype=w.torch_dtype, max_prefix=w.max_prefix, device=dev, mode=mode, q_rows=T)
+    q_draft = vtok = None
+    if w.stochastic:
+        # the target's and the draft's distributions and the drafted tokens
+        # (children drawn from q at their parent) come from the harness
+        sd = I.stochastic_inputs(w, parents, device="cuda")
+        logits, q_draft, vtok = sd["p"], sd["q"], sd["node_tokens"]
+    else:
+        # the target model's logits (outside this path) are synthesised once
+        # from the tree the heads propose, with the workload's match probability
+        step.heads(hin["h"], hin["W_res"], hin["W_head"], hin["root_token"])
+        torch.cuda.synchronize()
+        logits = I.boosted_target_logits(w, parents, step.node_tokens.cpu(), device="cuda")
     new_pl = torch.empty_like(ain["prefix_len"])
 
     def run_step():
         step.run(h=hin["h"], W_res=hin["W_res"], W_head=hin["W_head"], root_token=hin["root_token"], q=ain["q"],
                  k_tree=ain["k_tree"], v_tree=ain["v_tree"], k_cache=ain["k_cache"], v_cache=ain["v_cache"],
-                 prefix_len=ain["prefix_len"], new_prefix_len=new_pl, target=logits)
-
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+                 prefix_len=ain["prefix_len"], new_prefix_len=new_pl, target=logits, q_draft=q_draft,
+                 node_tokens=vtok)
 
     def barrier():
         if world > 1:
@@ -276,7 +300,7 @@ def run_mine(args, rank, world, local_rank):
         ev[i][1].record()
         step.attention(ain["q"], ain["k_tree"], ain["v_tree"], ain["k_cache"], ain["v_cache"], ain["prefix_len"])
         ev[i][2].record()
-        step.verify(logits)
+        step.verify(logits, q_draft, None, 0, i, vtok)
         ev[i][3].record()
         step.commit(ain["k_cache"], ain["v_cache"], ain["k_tree"], ain["v_tree"], ain["prefix_len"], new_pl)
         ev[i][4].record()
@@ -285,8 +309,8 @@ def run_mine(args, rank, world, local_rank):
     barrier()
     clk = clocks.stop()
     t_local = e0.elapsed_time(e1) / 1000.0
-    t = max_over_ranks(t_local)
-    value = world * K / t
+    t = max_over_ranks(t_local, world, dev)
+    value = whole_job_rate(world, K, t)
     stage = [statistics.mean(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K)) / 1000.0 for j in range(4)]
     assert int(step.status.item()) == 0, "device status set during the benchmark"
     mean_len = float(step.accept_len.float().mean().item())
@@ -299,6 +323,9 @@ def run_mine(args, rank, world, local_rank):
     names_in = ["h", "root_token", "q", "k_tree", "v_tree"]
     host_in = {n: (hin if n in hin else ain)[n].cpu().pin_memory() for n in names_in}
     host_in["target"] = logits.cpu().pin_memory()
+    if w.stochastic:
+        host_in["q_draft"] = q_draft.cpu().pin_memory()
+        host_in["tokens"] = vtok.cpu().pin_memory()
     dev_in = [{n: torch.empty_like(host_in[n], device=dev) for n in host_in} for _ in range(2)]
     outs = [step.accept_path, step.accept_len, step.bonus, step.node_tokens]
     host_out = [torch.empty_like(o, device="cpu").pin_memory() for o in outs]
@@ -322,7 +349,8 @@ def run_mine(args, rank, world, local_rank):
         d = dev_in[slot]
         step.run(h=d["h"], W_res=hin["W_res"], W_head=hin["W_head"], root_token=d["root_token"], q=d["q"],
                  k_tree=d["k_tree"], v_tree=d["v_tree"], k_cache=ain["k_cache"], v_cache=ain["v_cache"],
-                 prefix_len=ain["prefix_len"], new_prefix_len=new_pl, target=d["target"])
+                 prefix_len=ain["prefix_len"], new_prefix_len=new_pl, target=d["target"],
+                 q_draft=d.get("q_draft"), node_tokens=d.get("tokens"))
         used[slot].record(main_stream)
         for o, ho in zip(outs, host_out):
             ho.copy_(o, non_blocking=True)
@@ -338,26 +366,28 @@ def run_mine(args, rank, world, local_rank):
     e1.record()
     torch.cuda.synchronize()
     barrier()
-    t_e2e = max_over_ranks(e0.elapsed_time(e1) / 1000.0)
-    value_e2e = world * K / t_e2e
+    t_e2e = max_over_ranks(e0.elapsed_time(e1) / 1000.0, world, dev)
+    value_e2e = whole_job_rate(world, K, t_e2e)
 
     # ---- roofline of the dominant stage (the heads) and of tree attention ----
     pk = peaks()
-    elt = 2
+    elt = 2 if w.dtype == "bf16" else 4
     heads_bytes = (w.K * w.d * w.d + w.K * w.V * w.d) * elt + w.B * w.d * elt
     heads_gbs = heads_bytes / stage[0] / 1e9
-    S = w.prefix
-    attn_bytes = (2 * w.B * w.Hkv * S * w.D + 2 * w.B * T * w.Hq * w.D + 2 * w.B * T * w.Hkv * w.D) * elt
+    sum_S = int(ain["prefix_len"].sum().item())
+    attn_bytes = (2 * w.Hkv * sum_S * w.D + 2 * w.B * T * w.Hq * w.D + 2 * w.B * T * w.Hkv * w.D) * elt
     attn_gbs = attn_bytes / stage[1] / 1e9
     anc_pairs = sum(bin(sum(1 << j for j in range(T) if _is_anc(parents, i, j))).count("1") for i in range(T))
-    attn_flops = 4 * w.D * w.Hq * (T * S * w.B + anc_pairs * w.B)
+    attn_flops = 4 * w.D * w.Hq * (T * sum_S + anc_pairs * w.B)
     attn_tflops = attn_flops / stage[1] / 1e12
 
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": 1000.0 * t / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16", "data": "synthetic (seeded random weights and activations; target logits synthesised "
-                                   "from the proposed tree with match probability 0.6)",
+        "dtype": w.dtype, "data": ("synthetic (seeded random weights and activations; stochastic verify on Zipf-"
+                                   "ranked target and draft distributions)" if w.stochastic else
+                                   "synthetic (seeded random weights and activations; target logits synthesised "
+                                   f"from the proposed tree with match probability {w.match_prob})"),
         "config": config_dict(w, world),
         "roofline": {"kernel": "medusa_heads (residual GEMV + LM-head GEMV with softmax/top-8 + merge)",
                      "bound": "hbm", "achieved": heads_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
@@ -374,7 +404,7 @@ def run_mine(args, rank, world, local_rank):
         "gpu_launches": K * launches_per_step(w),
         "clocks": clk,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not w.stochastic:
         import oracle
         oracle.build()
         sample = OracleSample(w, 1.0)
