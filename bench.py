@@ -381,6 +381,25 @@ def run_mine(args, rank, world, local_rank):
     attn_flops = 4 * w.D * w.Hq * (T * sum_S + anc_pairs * w.B)
     attn_tflops = attn_flops / stage[1] / 1e12
 
+    # the roofline object describes the step's dominant kernel: the heads
+    # kernel (HBM-bound weight stream) or, at long contexts, tree attention,
+    # bound by whichever of its HBM bytes and tensor-core FLOPs takes longer
+    attn_bound = "tensor" if attn_flops / (pk["bf16_tflops"] * 1e12) > attn_bytes / (pk["hbm_gbs"] * 1e9) else "hbm"
+    if stage[1] > stage[0]:
+        if attn_bound == "tensor":
+            roofline = {"kernel": "tree_attention (split-KV tcgen05 kernel + combine)", "bound": "tensor",
+                        "achieved": attn_tflops, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                        "frac": attn_tflops / pk["bf16_tflops"], "peak_source": pk["source"],
+                        "algorithmic_flops": attn_flops, "traffic": None}
+        else:
+            roofline = {"kernel": "tree_attention (split-KV tcgen05 kernel + combine)", "bound": "hbm",
+                        "achieved": attn_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": attn_gbs / pk["hbm_gbs"],
+                        "peak_source": pk["source"], "algorithmic_bytes": attn_bytes, "traffic": None}
+    else:
+        roofline = {"kernel": "medusa_heads (residual GEMV + LM-head GEMV with softmax/top-8 + merge)",
+                    "bound": "hbm", "achieved": heads_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                    "frac": heads_gbs / pk["hbm_gbs"], "peak_source": pk["source"],
+                    "algorithmic_bytes": heads_bytes, "traffic": HEADS_DRAM_BYTES}
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": 1000.0 * t / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -389,13 +408,10 @@ def run_mine(args, rank, world, local_rank):
                                    "synthetic (seeded random weights and activations; target logits synthesised "
                                    f"from the proposed tree with match probability {w.match_prob})"),
         "config": config_dict(w, world),
-        "roofline": {"kernel": "medusa_heads (residual GEMV + LM-head GEMV with softmax/top-8 + merge)",
-                     "bound": "hbm", "achieved": heads_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                     "frac": heads_gbs / pk["hbm_gbs"], "peak_source": pk["source"],
-                     "algorithmic_bytes": heads_bytes, "traffic": HEADS_DRAM_BYTES},
-        "tree_attention": {"us": stage[1] * 1e6, "algorithmic_bytes": attn_bytes, "hbm_gbs": attn_gbs,
-                           "hbm_frac": attn_gbs / pk["hbm_gbs"], "hbm_frac_nominal_8tbs": attn_gbs / 8000.0,
-                           "tflops": attn_tflops, "tc_frac": attn_tflops * 1000.0 / pk["bf16_tflops"]},
+        "roofline": roofline,
+        "tree_attention": {"us": stage[1] * 1e6, "algorithmic_bytes": attn_bytes, "algorithmic_flops": attn_flops,
+                           "hbm_gbs": attn_gbs, "hbm_frac": attn_gbs / pk["hbm_gbs"], "tflops": attn_tflops,
+                           "tc_frac": attn_tflops / pk["bf16_tflops"], "bound": attn_bound},
         "stage_us": {"medusa_heads": stage[0] * 1e6, "tree_attention": stage[1] * 1e6,
                      "tree_verify": stage[2] * 1e6, "kv_commit": stage[3] * 1e6},
         "mean_accept_len": mean_len,

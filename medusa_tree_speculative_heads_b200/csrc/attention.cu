@@ -438,7 +438,8 @@ SplitPlan plan_splits(int B, int T, int Hq, int Hkv, int max_prefix, int tile_ro
 
 SplitPlan plan_bf16(int B, int T, int Hq, int Hkv, int D, int max_prefix) {
     // tensor-core kernel: 128-row tiles, two CTAs per SM
-    if (attn_tc_supported(Hq, Hkv, D, T, MEDUSA_BF16)) return plan_splits(B, T, Hq, Hkv, max_prefix, 128, 2);
+    if (attn_tc_supported(Hq, Hkv, D, T, MEDUSA_BF16))
+        return plan_splits(B, T, Hq, Hkv, max_prefix, 128, attn_tc_ctas_per_sm());
     return plan_splits(B, T, Hq, Hkv, max_prefix);
 }
 

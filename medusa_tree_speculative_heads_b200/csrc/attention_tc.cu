@@ -43,7 +43,12 @@ namespace {
 constexpr int kAW = 6;       // 0 producer, 1 MMA, 2-5 softmax
 constexpr int kAM = 128;     // query rows per CTA (MMA M)
 constexpr int kCh = 64;      // keys per chunk
-constexpr int kKVStages = 2;  // with one P buffer: ~112 KB, two CTAs per SM
+#ifndef MEDUSA_ATTN_CTAS_PER_SM
+#define MEDUSA_ATTN_CTAS_PER_SM 2
+#endif
+constexpr int kCtasPerSm = MEDUSA_ATTN_CTAS_PER_SM;
+// K/V ring depth: two stages keep a CTA within half an SM's shared memory
+constexpr int kKVStages = kCtasPerSm == 2 ? 2 : 6;
 
 struct TcAttnArgs {
     CUtensorMap mq;    // q as (D, Hq, B*T), box (64, G, 128/G)
@@ -60,6 +65,14 @@ struct TcAttnArgs {
     float scale_log2;
 };
 
+// 2^x with the SFU's approximate exponential (relative error ~2^-22, far
+// below the bf16 rounding P goes through; 2^-inf = 0)
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // descriptor of an MN-major operand stored as TMA writes a (64 MN x rows K)
 // box with a 128-byte swizzle: 8 K-rows of 128 bytes per 1024-byte group;
 // `lbo` = byte distance to the next 64-element MN block
@@ -74,7 +87,7 @@ __device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t smem_byte_addr, 
 }
 
 template <int D>
-__global__ void __launch_bounds__(kAW * 32, 2) tree_attn_tc_kernel(const __grid_constant__ TcAttnArgs a) {
+__global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(const __grid_constant__ TcAttnArgs a) {
     constexpr int NSUB = D / 64;              // 64-element blocks along D
     constexpr int kQBytes = kAM * D * 2;
     constexpr int kSub = kCh * 128;           // [64 keys x 64 D] block = 8 KB
@@ -248,41 +261,57 @@ __global__ void __launch_bounds__(kAW * 32, 2) tree_attn_tc_kernel(const __grid_
                 uint32_t raw[kCh / 16][16];
 #pragma unroll
                 for (int c = 0; c < kCh / 16; ++c) tmem_ld16_async(lane_base + (j & 1) * kCh + c * 16, raw[c]);
-                tmem_wait_ld();
+                tmem_wait_ld(raw);
 #pragma unroll
                 for (int c = 0; c < kCh / 16; ++c)
 #pragma unroll
                     for (int e = 0; e < 16; ++e) sv[c * 16 + e] = __uint_as_float(raw[c][e]);
             }
-            // mask and online softmax (log2 domain)
+            // visible keys of this chunk for this row, bit c = key key0 + c
             const int key0 = chunk_start(j);
-            float mx = -INFINITY;
-#pragma unroll
-            for (int c = 0; c < kCh; ++c) {
-                const int key = key0 + c;
-                bool vis;
-                if (tree_split) vis = key < a.T && ((anc[(key >> 5) & 3] >> (key & 31)) & 1u);
-                else vis = key >= k_begin;
-                sv[c] = vis ? sv[c] * a.scale_log2 : -INFINITY;
-                mx = fmaxf(mx, sv[c]);
+            uint64_t vis;
+            if (tree_split) {
+                // ancestor bits (keys >= T have none); key0 is 0 or 64
+                vis = key0 == 0 ? ((uint64_t)anc[1] << 32 | anc[0]) : ((uint64_t)anc[3] << 32 | anc[2]);
+            } else {
+                vis = key0 >= k_begin ? ~0ull : ~0ull << (k_begin - key0);  // only a first chunk reaches back
             }
+            // online softmax in the log2 domain: p = 2^(s * scale * log2 e - mu)
+            float mx;
+            if (vis == ~0ull) {
+                float m4[4] = {sv[0], sv[1], sv[2], sv[3]};
+#pragma unroll
+                for (int c = 4; c < kCh; ++c) m4[c & 3] = fmaxf(m4[c & 3], sv[c]);
+                mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+            } else {
+                float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+                for (int c = 0; c < kCh; ++c) {
+                    sv[c] = (vis >> c) & 1ull ? sv[c] : -INFINITY;
+                    m4[c & 3] = fmaxf(m4[c & 3], sv[c]);
+                }
+                mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+            }
+            mx *= a.scale_log2;  // the scale is positive: the max commutes with it
             // lazy reference max: raised only when the chunk's max exceeds it by > 8
             const bool raise = mx > m + 8.f;
             const float mn = raise ? mx : m;
             const float mu = mn == -INFINITY ? 0.f : mn;
-            const float alpha = raise ? exp2f(m - mu) : 1.f;
-            float rs = 0.f;
+            const float alpha = raise ? fast_exp2(m - mu) : 1.f;
+            float rs;
             {
                 uint32_t pk[2][16];  // P row: 64 keys as 32 bf16 pairs
+                float r4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int c = 0; c < kCh / 2; ++c) {
-                    const float p0 = exp2f(sv[2 * c] - mu);
-                    const float p1 = exp2f(sv[2 * c + 1] - mu);
+                    const float p0 = fast_exp2(fmaf(sv[2 * c], a.scale_log2, -mu));
+                    const float p1 = fast_exp2(fmaf(sv[2 * c + 1], a.scale_log2, -mu));
                     __nv_bfloat162 v2 = __floats2bfloat162_rn(p0, p1);
                     // the row sum uses the same bf16 weights PV multiplies by
-                    rs += __low2float(v2) + __high2float(v2);
+                    r4[c & 3] += __low2float(v2) + __high2float(v2);
                     pk[c >> 4][c & 15] = *reinterpret_cast<uint32_t*>(&v2);
                 }
+                rs = (r4[0] + r4[1]) + (r4[2] + r4[3]);
                 tmem_st16(lane_base + (j & 1) * kCh, pk[0]);
                 tmem_st16(lane_base + (j & 1) * kCh + 16, pk[1]);
             }
@@ -302,7 +331,7 @@ __global__ void __launch_bounds__(kAW * 32, 2) tree_attn_tc_kernel(const __grid_
 #pragma unroll
                     for (int c = 0; c < 4; ++c)
                         if (c0 + c < D / 16) tmem_ld16_async(lane_base + 128 + (c0 + c) * 16, raw[c]);
-                    tmem_wait_ld();
+                    tmem_wait_ld(raw);
 #pragma unroll
                     for (int c = 0; c < 4; ++c)
                         if (c0 + c < D / 16) {
@@ -332,7 +361,7 @@ __global__ void __launch_bounds__(kAW * 32, 2) tree_attn_tc_kernel(const __grid_
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
                     if (c0 + c < D / 16) tmem_ld16_async(lane_base + 128 + (c0 + c) * 16, raw[c]);
-                tmem_wait_ld();
+                tmem_wait_ld(raw);
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
                     if (c0 + c < D / 16)
@@ -364,10 +393,13 @@ __global__ void __launch_bounds__(kAW * 32, 2) tree_attn_tc_kernel(const __grid_
 
 template <int D>
 size_t tc_attn_smem() {
-    return (size_t)kAM * D * 2 + 2 * (size_t)kKVStages * kCh * D * 2 + 16 * 8 + 16;
+    // Q, the K/V ring, (6 + 2 x stages) mbarriers and the TMEM address slot
+    return (size_t)kAM * D * 2 + 2 * (size_t)kKVStages * kCh * D * 2 + (6 + 2 * kKVStages) * 8 + 16;
 }
 
 }  // namespace
+
+int attn_tc_ctas_per_sm() { return kCtasPerSm; }
 
 bool attn_tc_supported(int Hq, int Hkv, int D, int T, medusa_dtype dt) {
     const int G = Hkv > 0 ? Hq / Hkv : 0;

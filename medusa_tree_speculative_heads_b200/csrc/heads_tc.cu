@@ -19,11 +19,16 @@
 //            vocabulary tile it waits at the grid barrier (all of h^(k) must
 //            be written by every CTA)
 //   warps 3-6 epilogue, one TMEM lane (= weight row) per thread: residual
-//            tiles write h^(k) = SiLU(z) + h (bf16); vocabulary tiles update
-//            per-(head, sequence) running softmax statistics and top-8 lists.
+//            tiles write h^(k) = SiLU(z) + h (bf16); vocabulary tiles are
+//            transposed through shared memory so that each thread owns one
+//            sequence (column) and a fixed segment of the tile's rows, and
+//            keeps that column's running softmax statistics and top-8 list
+//            in registers; at a head change the segments of each column are
+//            merged into the CTA's partial for (head, sequence).
 // The residual tiles of every head come first, then the vocabulary tiles;
-// the weight producer keeps prefetching across the grid barrier.  The last
-// CTA to finish merges all CTAs' partials in CTA order and fills the tree.
+// the weight producer keeps prefetching across the grid barrier.  After a
+// second grid barrier the warps of the grid merge the (sequence, head)
+// partials, each in CTA order, and fill the tree.
 // Every wait is bounded (~2 s) and sets MEDUSA_STATUS_TIMEOUT on expiry.
 #include <limits.h>
 
@@ -42,6 +47,11 @@ constexpr int kTK = 64;                  // k-elements per stage (128 bytes, one
 constexpr int kABytes = kTM * kTK * 2;   // 16 KB
 constexpr int kEpiWarp0 = 3;             // first epilogue warp
 constexpr int kSmemBudget = 227 * 1024;
+constexpr int kTS = kTM + 1;             // transposed tile: column stride in floats (odd: no bank conflicts)
+
+// row segments per column in the transposed epilogue (at most 16, so that a
+// column's flush merges few partial states)
+__host__ __device__ constexpr int seg_per_col(int B) { return 128 / B < 16 ? 128 / B : 16; }
 
 struct TcHeadsArgs {
     CUtensorMap mW_res;   // W_res  as (d_in, d_out, K), box (64, 128, 1)
@@ -66,26 +76,7 @@ struct TcHeadsArgs {
     int stages;
 };
 
-__device__ __forceinline__ float warp_max(float x) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(kFull, x, o));
-    return x;
-}
-
 __device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
-
-// sorted insert into a shared-memory top-8 list (one thread)
-__device__ __forceinline__ void smem_list_insert(HeadState* s, float v, int i) {
-    if (!beats(v, i, s->val[kTopK - 1], s->idx[kTopK - 1])) return;
-    int j = kTopK - 1;
-    while (j > 0 && beats(v, i, s->val[j - 1], s->idx[j - 1])) {
-        s->val[j] = s->val[j - 1];
-        s->idx[j] = s->idx[j - 1];
-        --j;
-    }
-    s->val[j] = v;
-    s->idx[j] = i;
-}
 
 template <int N>
 __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid_constant__ TcHeadsArgs a) {
@@ -103,7 +94,8 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
     uint64_t* acc_empty = acc_full + 2;  // [2]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
     int* flag = reinterpret_cast<int*>(tmem_slot + 1);
-    HeadState* st = reinterpret_cast<HeadState*>(tmem_slot + 4);  // [4][N]
+    float* sT = reinterpret_cast<float*>(tmem_slot + 4);  // [B][kTS] transposed tile
+    HeadState* stS = reinterpret_cast<HeadState*>(sT + ((a.B * kTS + 3) & ~3));  // [seg][B] flush states
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int K = a.K, B = a.B;
@@ -134,7 +126,6 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
         tma_prefetch_desc(&a.mh);
         tma_prefetch_desc(&a.mhk);
     }
-    for (int t = threadIdx.x; t < 4 * N; t += blockDim.x) st[t] = empty_state();
     if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
     tc_fence_before();
     __syncthreads();
@@ -227,52 +218,75 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
         }
     } else {
         // ---------------- epilogue ----------------
-        const int ew = warp - kEpiWarp0;     // 0..3
-        const int q = warp & 3;              // TMEM lane quarter this warp may access
-        const int row = q * 32 + lane;       // weight row of the tile held by this thread
-        HeadState* mine = st + ew * N;
+        const int et = threadIdx.x - kEpiWarp0 * 32;  // 0..127
+        const int ew = warp - kEpiWarp0;               // 0..3
+        const int q = warp & 3;                        // TMEM lane quarter this warp may access
+        const int row = q * 32 + lane;                 // weight row of the tile held by this thread
+        // transposed phase: column `col`, rows [r_lo, r_hi) of every tile
+        const int nseg = seg_per_col(B);
+        const int rps = (kTM + nseg - 1) / nseg;
+        const bool col_thread = et < B * nseg;
+        const int col = et % B, seg = et / B;
+        const int r_lo = col_thread ? seg * rps : 0, r_hi = col_thread ? min(kTM, r_lo + rps) : 0;
+        float cm = -INFINITY, cl = 0.f;  // running max and sum of exp(x - cm)
+        float lv[kTopK];
+        int lx[kTopK];
+#pragma unroll
+        for (int j = 0; j < kTopK; ++j) {
+            lv[j] = -INFINITY;
+            lx[j] = INT_MAX;
+        }
         int cur_k = -1;
         bool ok = true;
         auto flush = [&](int kk) {
-            epi_sync();
-            // warp ew merges columns b = ew, ew+4, ... over the 4 epilogue warps
-            for (int b = ew; b < B; b += 4) {
-                float mm = -INFINITY, ll = 0.f;
-                if (lane < 4) {
-                    mm = st[lane * N + b].m;
-                    ll = st[lane * N + b].l;
-                }
-#pragma unroll
-                for (int o = 1; o < 4; o <<= 1) {
-                    const float m2 = __shfl_xor_sync(kFull, mm, o);
-                    const float l2 = __shfl_xor_sync(kFull, ll, o);
-                    merge_ml(mm, ll, m2, l2);
-                }
-                float lv[kTopK];
-                int li2[kTopK];
+            if (col_thread) {
+                HeadState* o = &stS[et];  // = [seg][col]
+                o->m = cm;
+                o->l = cl;
 #pragma unroll
                 for (int j = 0; j < kTopK; ++j) {
-                    lv[j] = -INFINITY;
-                    li2[j] = INT_MAX;
-                }
-                lv[0] = st[(lane >> 3) * N + b].val[lane & 7];
-                li2[0] = st[(lane >> 3) * N + b].idx[lane & 7];
-                float ov;
-                int oi;
-                warp_select(lv, li2, ov, oi);
-                HeadState* dst = &a.part[((long)blockIdx.x * K + kk) * B + b];
-                if (lane < kTopK) {
-                    dst->val[lane] = ov;
-                    dst->idx[lane] = oi;
-                }
-                if (lane == 0) {
-                    dst->m = mm;
-                    dst->l = ll;
+                    o->val[j] = lv[j];
+                    o->idx[j] = lx[j];
                 }
             }
             epi_sync();
-            for (int b = lane; b < B; b += 32) mine[b] = empty_state();
-            __syncwarp();
+            if (et < B) {
+                // merge the column's segments in segment order
+                float mm = -INFINITY, ll = 0.f;
+                float mv[kTopK];
+                int mi[kTopK];
+#pragma unroll
+                for (int j = 0; j < kTopK; ++j) {
+                    mv[j] = -INFINITY;
+                    mi[j] = INT_MAX;
+                }
+                for (int sg = 0; sg < nseg; ++sg) {
+                    const HeadState* o = &stS[sg * B + et];
+                    merge_ml(mm, ll, o->m, o->l);
+                    for (int j = 0; j < kTopK; ++j) {  // each list is sorted: stop at the first that fails
+                        const float v = o->val[j];
+                        const int i = o->idx[j];
+                        if (!beats(v, i, mv[kTopK - 1], mi[kTopK - 1])) break;
+                        list_insert(mv, mi, v, i);
+                    }
+                }
+                HeadState* dst = &a.part[((long)blockIdx.x * K + kk) * B + et];
+                dst->m = mm;
+                dst->l = ll;
+#pragma unroll
+                for (int j = 0; j < kTopK; ++j) {
+                    dst->val[j] = mv[j];
+                    dst->idx[j] = mi[j];
+                }
+            }
+            epi_sync();  // stS is free again
+            cm = -INFINITY;
+            cl = 0.f;
+#pragma unroll
+            for (int j = 0; j < kTopK; ++j) {
+                lv[j] = -INFINITY;
+                lx[j] = INT_MAX;
+            }
         };
         auto arrive_grid = [&]() {
             // this CTA's h^(k) rows are written: publish them (also to the TMA proxy)
@@ -310,12 +324,17 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
                 const int k = (int)(t / tph_r);
                 const int o = (int)(t % tph_r) * kTM + row;
                 if (ok && o < a.d) {
-                    for (int b = 0; b < B; ++b) {
-                        const float z = v[b];
-                        const float y = z / (1.f + expf(-z)) + __bfloat162float(a.h[(long)b * a.d + o]);
-                        const __nv_bfloat16 yb = __float2bfloat16_rn(y);
-                        a.hk[((long)b * K + k) * a.d + o] = yb;
-                        if (a.hk_out) a.hk_out[((long)b * K + k) * a.d + o] = yb;
+                    float hv[N];  // every load before the first store
+#pragma unroll
+                    for (int e = 0; e < N; ++e) hv[e] = e < B ? __bfloat162float(a.h[(long)e * a.d + o]) : 0.f;
+#pragma unroll
+                    for (int e = 0; e < N; ++e) {
+                        if (e < B) {
+                            const float z = v[e];
+                            const __nv_bfloat16 yb = __float2bfloat16_rn(z / (1.f + expf(-z)) + hv[e]);
+                            a.hk[((long)e * K + k) * a.d + o] = yb;
+                            if (a.hk_out) a.hk_out[((long)e * K + k) * a.d + o] = yb;
+                        }
                     }
                 }
                 if (li == n1 - 1) arrive_grid();
@@ -324,33 +343,37 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
             // vocabulary tile
             const long t = t2a + (li - n1);
             const int k = (int)(t / tph_l);
-            const int vrow = (int)(t % tph_l) * kTM + row;
-            const bool valid = ok && vrow < a.V;
+            const int row0 = (int)(t % tph_l) * kTM;
             if (k != cur_k) {
                 if (cur_k >= 0) flush(cur_k);
                 cur_k = k;
             }
-            for (int b = 0; b < B; ++b) {
-                const float x = v[b];
-                if (a.logits && valid) a.logits[((long)b * K + k) * a.V + vrow] = x;
-                // softmax statistics of the tile's 32 rows of this warp
-                const float tm = warp_max(valid ? x : -INFINITY);
+            if (a.logits && ok && row0 + row < a.V) {
+#pragma unroll
+                for (int e = 0; e < N; ++e)
+                    if (e < B) a.logits[((long)e * K + k) * a.V + row0 + row] = v[e];
+            }
+            epi_sync();  // the previous tile's readers are done with sT
+#pragma unroll
+            for (int e = 0; e < N; ++e)
+                if (e < B) sT[e * kTS + row] = v[e];
+            epi_sync();
+            if (ok) {
+                const float* src = sT + col * kTS;
+                const int hi = min(r_hi, a.V - row0);  // rows past V are zero-filled weights
+                float tm = -INFINITY;
+                for (int r = r_lo; r < hi; ++r) tm = fmaxf(tm, src[r]);
                 if (tm > -INFINITY) {
-                    const float tl = warp_sum(valid ? expf(x - tm) : 0.f);
-                    if (lane == 0) merge_ml(mine[b].m, mine[b].l, tm, tl);
+                    const float mn = fmaxf(cm, tm);
+                    float sum = 0.f;
+                    for (int r = r_lo; r < hi; ++r) {
+                        const float x = src[r];
+                        sum += expf(x - mn);
+                        if (beats(x, row0 + r, lv[kTopK - 1], lx[kTopK - 1])) list_insert(lv, lx, x, row0 + r);
+                    }
+                    cl = (cm == -INFINITY ? 0.f : cl * expf(cm - mn)) + sum;
+                    cm = mn;
                 }
-                // top-8: the rows that beat the current 8th entry
-                const float thr_v = mine[b].val[kTopK - 1];
-                const int thr_i = mine[b].idx[kTopK - 1];
-                unsigned mask = __ballot_sync(kFull, valid && beats(x, vrow, thr_v, thr_i));
-                while (mask) {
-                    const int j = __ffs(mask) - 1;
-                    const float xv = __shfl_sync(kFull, x, j);
-                    const int xi = __shfl_sync(kFull, vrow, j);
-                    if (lane == 0) smem_list_insert(&mine[b], xv, xi);
-                    mask &= mask - 1;
-                }
-                __syncwarp();
             }
         }
         if (cur_k >= 0) flush(cur_k);
@@ -363,14 +386,26 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
-    // the last CTA to finish merges every (sequence, head)
+    // grid barrier: every CTA's partials are written; then the (sequence,
+    // head) merges are spread over all warps of the grid
     __threadfence();
     __syncthreads();
-    if (threadIdx.x == 0) *flag = atomicAdd(&a.ctr[1], 1u) == gridDim.x - 1;
+    if (threadIdx.x == 0) {
+        atomicAdd(&a.ctr[1], 1u);
+        const uint64_t t0 = global_ns();
+        while (ld_acquire_u32(&a.ctr[1]) < gridDim.x) {
+            if (global_ns() - t0 > 2000000000ull) {
+                set_status(a.status, MEDUSA_STATUS_TIMEOUT);
+                *flag = 1;
+                break;
+            }
+            __nanosleep(64);
+        }
+    }
     __syncthreads();
-    if (!*flag) return;
+    if (*flag) return;
     __threadfence();
-    for (int p = warp; p < B * K; p += kTcWarps) {
+    for (int p = blockIdx.x * kTcWarps + warp; p < B * K; p += gridDim.x * kTcWarps) {
         const int b = p % B, k = p / B;
         merge_head(a.part, gridDim.x, tph_l, B, b, b, a.V, K, k, a.tree, a.root_token, a.topk_idx, a.topk_prob,
                    a.node_tokens, a.node_q, a.stats, a.status);
@@ -378,23 +413,23 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
 }
 
 template <int N>
-size_t tc_smem_bytes(int stages) {
+size_t tc_smem_bytes(int stages, int B) {
     return 1024 + (size_t)stages * (kABytes + N * kTK * 2) + (2 * (size_t)stages + 4) * 8 + 16 +
-           4 * (size_t)N * sizeof(HeadState);
+           (size_t)((B * kTS + 3) & ~3) * 4 + (size_t)B * seg_per_col(B) * sizeof(HeadState);
 }
 
 template <int N>
-int tc_stages() {
+int tc_stages(int B) {
     int s = 12;
-    while (s > 2 && tc_smem_bytes<N>(s) > (size_t)kSmemBudget) --s;
+    while (s > 2 && tc_smem_bytes<N>(s, B) > (size_t)kSmemBudget) --s;
     return s;
 }
 
 template <int N>
 cudaError_t launch_n(const TcHeadsArgs& args, cudaStream_t st) {
     TcHeadsArgs a = args;
-    a.stages = tc_stages<N>();
-    const size_t smem = tc_smem_bytes<N>(a.stages);
+    a.stages = tc_stages<N>(a.B);
+    const size_t smem = tc_smem_bytes<N>(a.stages, a.B);
     auto kern = heads_tc_kernel<N>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

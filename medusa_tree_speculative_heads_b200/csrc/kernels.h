@@ -59,6 +59,7 @@ size_t attn_workspace_size(int B, int T, int Hq, int Hkv, int D, int max_prefix,
 cudaError_t attn_launch(const AttnArgs& a, cudaStream_t st);
 // tensor-core split kernel (bf16, D in {64,128}, power-of-two group size <= 16)
 bool attn_tc_supported(int Hq, int Hkv, int D, int T, medusa_dtype dt);
+int attn_tc_ctas_per_sm();
 cudaError_t attn_tc_launch(const AttnArgs& a, int m_tiles, int n_splits, int split_len, float scale_log2,
                            float* part_o, float* part_lse, cudaStream_t st);
 

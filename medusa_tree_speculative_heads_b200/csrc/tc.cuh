@@ -75,20 +75,16 @@ __device__ __forceinline__ void tc_commit(uint64_t* bar) {
                  : "memory");
 }
 
-// 32 lanes x 16 consecutive 32-bit columns (one row per thread of the warp)
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
-    uint32_t r[16];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
-}
+// The destination registers of tcgen05.ld hold their values only after
+// tcgen05.wait::ld.  The compiler does not know that, so every wait below also
+// names the loaded registers as read-write operands (and later groups pass
+// through an empty asm ordered after it): no use of them can be scheduled
+// ahead of the wait.
+#define MEDUSA_R16(r) "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), \
+    "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
 
-// same load without waiting: issue several, then tmem_wait_ld() once
+// 32 lanes x 16 consecutive 32-bit columns, no wait: issue several, then
+// tmem_wait_ld() on all of their registers
 __device__ __forceinline__ void tmem_ld16_async(uint32_t taddr, uint32_t (&r)[16]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
@@ -96,7 +92,22 @@ __device__ __forceinline__ void tmem_ld16_async(uint32_t taddr, uint32_t (&r)[16
           "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
         : "r"(taddr));
 }
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+template <int G>
+__device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[G][16]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" : MEDUSA_R16(r[0])::"memory");
+#pragma unroll
+    for (int g = 1; g < G; ++g) asm volatile("" : MEDUSA_R16(r[g]));
+}
+
+// 32 lanes x 16 consecutive 32-bit columns (one row per thread of the warp)
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+    uint32_t r[1][16];
+    tmem_ld16_async(taddr, r[0]);
+    tmem_wait_ld(r);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[0][i]);
+}
+
 // 32 lanes x 16 consecutive 32-bit columns, store (one row per thread)
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
     asm volatile(

@@ -80,7 +80,10 @@ def check(w, parents, inp, ref, out, out2):
     ("tiny", dict(d=1024, V=5003, K=3), (3, 2, 1)),                     # fp32, ragged V
     ("llama8b", dict(d=512, V=3001, K=3), (3, 2, 1)),                   # bf16 register path, ragged V
     ("llama8b", dict(B=3, d=256, V=2000, K=2), (4, 2)),                 # bf16, several sequences
-    ("llama8b", dict(B=10, d=128, V=700, K=2), (2, 2)),                 # two sequence groups (8 + 2)
+    ("llama8b", dict(B=10, d=128, V=700, K=2), (2, 2)),                 # tensor-core path, N = 16
+    ("llama8b", dict(B=17, d=256, V=2003, K=2), (2, 2)),                # N = 32, 7 ragged row segments
+    ("llama8b", dict(B=33, d=320, V=1000, K=2), (2,)),                  # N = 48
+    ("llama8b", dict(B=64, d=512, V=3001, K=3), (3, 2, 1)),             # N = 64, the largest batch
     ("llama8b", dict(d=8192, V=1500, K=1), (4,)),                       # d too wide for registers
     ("llama8b", dict(d=64, V=5, K=2), (3, 2)),                          # V < 8: missing entries are -1
 ])
@@ -97,6 +100,28 @@ def test_heads_parity_llama8b_full_size():
     parents = I.workload_tree(w)
     inp, ref, out, out2 = run_case(w, parents)
     check(w, parents, inp, ref, out, out2)
+
+
+def test_heads_parity_batch64_full_size_sampled():
+    # B=64, d=4096, V=32000, K=3 at full size; the oracle recomputes three
+    # sampled sequences (sequences are independent)
+    w = I.WORKLOADS["stoch_b64"]
+    inp = I.head_inputs(w)
+    dev = {k: v.cuda() for k, v in inp.items()}
+    out = api.heads(dev["h"], dev["W_res"], dev["W_head"], None, dev["root_token"], want_logits=True)
+    torch.cuda.synchronize()
+    assert int(out["status"].item()) == 0
+    tol = float_tol(w.torch_dtype)
+    ti = out["topk_idx"].cpu().numpy()
+    tp = out["topk_prob"].cpu().numpy()
+    for b in (0, 37, 63):
+        ref = oracle.heads(inp["h"][b:b + 1], inp["W_res"], inp["W_head"])
+        assert_float_parity(out["logits"][b:b + 1], ref["logits"], w.torch_dtype, f"logits[{b}]")
+        for k in range(w.K):
+            check_topk(ti[b, k], ref["logits"][0, k], tol)
+            np.testing.assert_allclose(tp[b, k], ref["probs"][0, k, ti[b, k]], rtol=0, atol=tol)
+    order = torch.sort(-out["logits"], dim=-1, stable=True).indices[..., :8].to(torch.int32)
+    assert torch.equal(order, out["topk_idx"])
 
 
 def test_heads_top_list_exact_when_separated():
