@@ -21,7 +21,7 @@
 // exceeds it by more than 8 (log2 units), so P <= 2^8; when it is raised the
 // softmax thread rescales its row of O in TMEM by exp2(m_old - m_new) after
 // the previous PV completed.  The result is the same after the final 1/l.
-// Warps: 0 TMA producer (Q once, K/V chunks in a 2-stage ring), 1 TMEM
+// Warps: 0 TMA producer (Q once, K and V chunks in separate rings), 1 TMEM
 // allocation + MMA issue (QK of chunk j+1 overlaps the softmax of chunk j),
 // 2-5 softmax / output.  Prefix chunks are laid out backwards from the
 // sequence's prefix end, so no cache slot at or past prefix_len is ever read
@@ -43,12 +43,13 @@ namespace {
 constexpr int kAW = 6;       // 0 producer, 1 MMA, 2-5 softmax
 constexpr int kAM = 128;     // query rows per CTA (MMA M)
 constexpr int kCh = 64;      // keys per chunk
-#ifndef MEDUSA_ATTN_CTAS_PER_SM
-#define MEDUSA_ATTN_CTAS_PER_SM 2
-#endif
-constexpr int kCtasPerSm = MEDUSA_ATTN_CTAS_PER_SM;
-// K/V ring depth: two stages keep a CTA within half an SM's shared memory
-constexpr int kKVStages = kCtasPerSm == 2 ? 2 : 6;
+constexpr int kCtasPerSm = 2;
+// K and V rings: a K stage is free once its QK product is done, a V stage
+// once its PV product is; at head_dim 128 three K and two V stages keep a CTA
+// within half of an SM's shared memory
+template <int D> constexpr int k_stages() { return D == 128 ? 3 : 4; }
+template <int D> constexpr int v_stages() { return D == 128 ? 2 : 4; }
+template <int D> constexpr int n_bars() { return 1 + 2 * k_stages<D>() + 2 * v_stages<D>() + 6; }
 
 struct TcAttnArgs {
     CUtensorMap mq;    // q as (D, Hq, B*T), box (64, G, 128/G)
@@ -91,7 +92,8 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
     constexpr int NSUB = D / 64;              // 64-element blocks along D
     constexpr int kQBytes = kAM * D * 2;
     constexpr int kSub = kCh * 128;           // [64 keys x 64 D] block = 8 KB
-    constexpr int kKVBytes = kCh * D * 2;
+    constexpr int kKVBytes = kCh * D * 2;     // one chunk of K (or of V)
+    constexpr int KS = k_stages<D>(), VS = v_stages<D>();
     constexpr uint32_t kIdescQK = idesc_bf16_f32(kAM, kCh);
     constexpr uint32_t kIdescPV = idesc_bf16_f32(kAM, D) | (1u << 16);  // A (P) from TMEM, B (V) MN-major
     constexpr uint32_t kTmemCols = 256;       // S: 2 x 64 columns, O: D columns at 128
@@ -101,15 +103,21 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
     extern __shared__ __align__(1024) uint8_t smem[];
     uint8_t* sQ = smem;
     uint8_t* sK = sQ + kQBytes;
-    uint8_t* sV = sK + kKVStages * kKVBytes;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sV + kKVStages * kKVBytes);
+    uint8_t* sV = sK + KS * kKVBytes;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sV + VS * kKVBytes);
     uint64_t* q_full = bars;
-    uint64_t* kv_full = bars + 1;
-    uint64_t* kv_empty = bars + 1 + kKVStages;
-    uint64_t* s_full = bars + 1 + 2 * kKVStages;
+    uint64_t* k_full = bars + 1;
+    uint64_t* k_empty = k_full + KS;
+    uint64_t* v_full = k_empty + KS;
+    uint64_t* v_empty = v_full + VS;
+    uint64_t* s_full = v_empty + VS;
     uint64_t* p_full = s_full + 2;
-    uint64_t* o_full = p_full + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_full + 1);
+    uint64_t* o_full = p_full + 2;  // one phase per PV product
+    // a single phase, completed with the last PV product: a parity wait on
+    // o_full cannot tell "the last PV done" from "two PVs done" once both of
+    // the last two have completed
+    uint64_t* o_last = o_full + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_last + 1);
 
     const int mt = blockIdx.x, bg = blockIdx.y, split = blockIdx.z;
     const int b = bg / a.Hkv, g = bg % a.Hkv;
@@ -141,15 +149,20 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
-        for (int s = 0; s < kKVStages; ++s) {
-            mbar_init(&kv_full[s], 1);
-            mbar_init(&kv_empty[s], 1);
+        for (int s = 0; s < KS; ++s) {
+            mbar_init(&k_full[s], 1);
+            mbar_init(&k_empty[s], 1);
+        }
+        for (int s = 0; s < VS; ++s) {
+            mbar_init(&v_full[s], 1);
+            mbar_init(&v_empty[s], 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s_full[i], 1);
             mbar_init(&p_full[i], 4);
         }
         mbar_init(o_full, 1);
+        mbar_init(o_last, 1);
         mbar_fence_init();
     }
     if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
@@ -160,38 +173,60 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
 
     if (warp == 0) {
         // ---------------- producer ----------------
+        // K chunks run ahead of V chunks; each is loaded as soon as its ring
+        // stage is free (polled without blocking, so a late V stage never
+        // holds back the next K)
         if (lane == 0 && nc > 0) {
-            int issued = 0;
             mbar_arrive_expect_tx(q_full, kQBytes);
 #pragma unroll
             for (int sub = 0; sub < NSUB; ++sub)
                 tma_load_3d(sQ + sub * (kAM * 128), &a.mq, sub * 64, g * a.G, b * a.T + mt * NB, q_full);
-            for (int j = 0; j < nc; ++j) {
-                const int s = j % kKVStages;
-                if (j >= kKVStages && !mbar_wait(&kv_empty[s], ((j / kKVStages) - 1) & 1)) {
+            int jk = 0, jv = 0;
+            uint64_t t0 = global_ns();
+            uint32_t idle = 0;
+            while (jk < nc || jv < nc) {
+                bool prog = false;
+                if (jk < nc && (jk < KS || mbar_test(&k_empty[jk % KS], ((jk / KS) - 1) & 1))) {
+                    const int s = jk % KS, cs = chunk_start(jk);
+                    mbar_arrive_expect_tx(&k_full[s], kKVBytes);
+#pragma unroll
+                    for (int sub = 0; sub < NSUB; ++sub) {
+                        uint8_t* dk = sK + s * kKVBytes + sub * kSub;
+                        if (tree_split) tma_load_3d(dk, &a.mkt, sub * 64, g, b * a.T + cs, &k_full[s]);
+                        else tma_load_3d(dk, &a.mkc, sub * 64, cs, bg, &k_full[s]);
+                    }
+                    ++jk;
+                    prog = true;
+                }
+                if (jv < jk && (jv < VS || mbar_test(&v_empty[jv % VS], ((jv / VS) - 1) & 1))) {
+                    const int s = jv % VS, cs = chunk_start(jv);
+                    mbar_arrive_expect_tx(&v_full[s], kKVBytes);
+#pragma unroll
+                    for (int sub = 0; sub < NSUB; ++sub) {
+                        uint8_t* dv = sV + s * kKVBytes + sub * kSub;
+                        if (tree_split) tma_load_3d(dv, &a.mvt, sub * 64, g, b * a.T + cs, &v_full[s]);
+                        else tma_load_3d(dv, &a.mvc, sub * 64, cs, bg, &v_full[s]);
+                    }
+                    ++jv;
+                    prog = true;
+                }
+                if (prog) {
+                    idle = 0;
+                    t0 = global_ns();
+                } else if ((++idle & 255u) == 0 && global_ns() - t0 > 2000000000ull) {
                     set_status(a.status, MEDUSA_STATUS_TIMEOUT);
                     break;
                 }
-                const int cs = chunk_start(j);
-                mbar_arrive_expect_tx(&kv_full[s], 2 * kKVBytes);
-#pragma unroll
-                for (int sub = 0; sub < NSUB; ++sub) {
-                    uint8_t* dk = sK + s * kKVBytes + sub * kSub;
-                    uint8_t* dv = sV + s * kKVBytes + sub * kSub;
-                    if (tree_split) {
-                        tma_load_3d(dk, &a.mkt, sub * 64, g, b * a.T + cs, &kv_full[s]);
-                        tma_load_3d(dv, &a.mvt, sub * 64, g, b * a.T + cs, &kv_full[s]);
-                    } else {
-                        tma_load_3d(dk, &a.mkc, sub * 64, cs, bg, &kv_full[s]);
-                        tma_load_3d(dv, &a.mvc, sub * 64, cs, bg, &kv_full[s]);
-                    }
-                }
-                ++issued;
             }
+            // drain: no copy may still be landing when the CTA exits
             mbar_wait(q_full, 0);
-            for (int s = 0; s < kKVStages && s < issued; ++s) {  // drain before exit
-                const int last = s + ((issued - 1 - s) / kKVStages) * kKVStages;
-                mbar_wait(&kv_full[s], (last / kKVStages) & 1);
+            for (int s = 0; s < KS && s < jk; ++s) {
+                const int last = s + ((jk - 1 - s) / KS) * KS;
+                mbar_wait(&k_full[s], (last / KS) & 1);
+            }
+            for (int s = 0; s < VS && s < jv; ++s) {
+                const int last = s + ((jv - 1 - s) / VS) * VS;
+                mbar_wait(&v_full[s], (last / VS) & 1);
             }
         }
     } else if (warp == 1) {
@@ -201,8 +236,8 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
             // S_j goes to TMEM columns (j&1)*64; P_j is written over it, so the
             // buffer is free for S_{j+2} once PV_j has completed (o_full phase j)
             auto issue_qk = [&](int j) -> bool {
-                const int s = j % kKVStages, sb = j & 1;
-                if (!mbar_wait(&kv_full[s], (j / kKVStages) & 1)) return false;
+                const int s = j % KS, sb = j & 1;
+                if (!mbar_wait(&k_full[s], (j / KS) & 1)) return false;
                 if (j >= 2 && !mbar_wait(o_full, (j - 2) & 1)) return false;
                 tc_fence_after();
 #pragma unroll
@@ -214,6 +249,7 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
                         tc_mma_bf16(tmem + sb * kCh, ad + 2 * ks, bd + 2 * ks, kIdescQK, (sub | ks) != 0);
                 }
                 tc_commit(&s_full[sb]);
+                tc_commit(&k_empty[s]);
                 return true;
             };
             if (ok) ok = issue_qk(0);
@@ -223,18 +259,23 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
                     ok = false;
                     break;
                 }
+                const int s = j % VS;
+                if (!mbar_wait(&v_full[s], (j / VS) & 1)) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
-                const int s = j % kKVStages;
                 const uint64_t bd = sw128_mnmajor_desc(smem_addr(sV + s * kKVBytes), kSub);
 #pragma unroll
                 for (int ks = 0; ks < kCh / 16; ++ks)  // 16 keys: 8 P columns, +2 K-groups (2048 B) in V
                     tc_mma_bf16_ts(tmem + 128, tmem + (j & 1) * kCh + ks * 8, bd + (uint64_t)(2048 >> 4) * ks,
                                    kIdescPV, (j | ks) != 0);
                 tc_commit(o_full);
-                tc_commit(&kv_empty[s]);
+                tc_commit(&v_empty[s]);
+                if (j == nc - 1) tc_commit(o_last);
             }
             if (!ok) set_status(a.status, MEDUSA_STATUS_TIMEOUT);
-            else mbar_wait(o_full, (nc - 1) & 1);  // every MMA done before TMEM is released
+            else mbar_wait(o_last, 0);  // every MMA done before TMEM is released
         }
     } else {
         // ---------------- softmax / output ----------------
@@ -350,9 +391,7 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
         }
         // final O (after the last PV) for this row
         float o[D];
-        if (ok && nc > 0) {
-            if (!mbar_wait(o_full, (nc - 1) & 1)) ok = false;
-        }
+        if (ok && nc > 0 && !mbar_wait(o_last, 0)) ok = false;
         if (ok && nc > 0) {
             tc_fence_after();
 #pragma unroll
@@ -393,8 +432,8 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
 
 template <int D>
 size_t tc_attn_smem() {
-    // Q, the K/V ring, (6 + 2 x stages) mbarriers and the TMEM address slot
-    return (size_t)kAM * D * 2 + 2 * (size_t)kKVStages * kCh * D * 2 + (6 + 2 * kKVStages) * 8 + 16;
+    // Q, the K and V rings, the mbarriers and the TMEM address slot
+    return (size_t)kAM * D * 2 + (size_t)(k_stages<D>() + v_stages<D>()) * kCh * D * 2 + n_bars<D>() * 8 + 16;
 }
 
 }  // namespace
@@ -450,10 +489,12 @@ cudaError_t attn_tc_launch(const AttnArgs& x, int m_tiles, int n_splits, int spl
     if (x.D == 128) {
         const size_t smem = tc_attn_smem<128>();
         cudaFuncSetAttribute(tree_attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaFuncSetAttribute(tree_attn_tc_kernel<128>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
         tree_attn_tc_kernel<128><<<grid, kAW * 32, smem, st>>>(a);
     } else {
         const size_t smem = tc_attn_smem<64>();
         cudaFuncSetAttribute(tree_attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaFuncSetAttribute(tree_attn_tc_kernel<64>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
         tree_attn_tc_kernel<64><<<grid, kAW * 32, smem, st>>>(a);
     }
     return cudaGetLastError();
