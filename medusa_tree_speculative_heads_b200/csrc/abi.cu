@@ -308,9 +308,6 @@ extern "C" int tree_verify(medusa_verify_mode mode, const void* target, medusa_d
     if (mode == MEDUSA_VERIFY_GREEDY) {
         if (target_dt != MEDUSA_F32 && target_dt != MEDUSA_BF16)
             return fail(MEDUSA_ERR_UNSUPPORTED, "tree_verify: greedy target dtype");
-        const size_t need = verify_workspace_size(mode, B, V, T);
-        if (!workspace || workspace_bytes < need || !al16(workspace))
-            return fail(MEDUSA_ERR_WORKSPACE, "tree_verify: workspace of %zu bytes, need %zu", workspace_bytes, need);
     } else {
         if (target_dt != MEDUSA_F32)
             return fail(MEDUSA_ERR_UNSUPPORTED, "tree_verify: stochastic target p must be MEDUSA_F32");
@@ -318,6 +315,9 @@ extern "C" int tree_verify(medusa_verify_mode mode, const void* target, medusa_d
         if (q_rows < 1 || (!q_row && q_rows != T))
             return fail(MEDUSA_ERR_INVALID_ARG, "tree_verify: q_rows=%d (must equal T=%d without q_row)", q_rows, T);
     }
+    const size_t need = verify_workspace_size(mode, B, V, T);
+    if (need > 0 && (!workspace || workspace_bytes < need || !al16(workspace)))
+        return fail(MEDUSA_ERR_WORKSPACE, "tree_verify: workspace of %zu bytes, need %zu", workspace_bytes, need);
     VerifyArgs a;
     a.mode = mode;
     a.target = target;

@@ -10,12 +10,18 @@
 //
 // Stochastic ("Speculative Decoding & Medusa Tree Attention", section 2:
 // accept with probability min(1, P_target/P_draft), else resample from
-// normalize(max(0, P_target - P_draft))): one CTA per sequence walks the tree;
-// every vocabulary pass is a block-wide exact integer reduction, and the
-// current distribution after j rejections is recomputed element-wise from the
-// j residual sums, so no V-sized scratch is needed.  All decisions use
-// integer or correctly rounded fp64 operations (explicit _rn intrinsics, no
-// contraction), so results are bit-reproducible.
+// normalize(max(0, P_target - P_draft))): one thread-block cluster per
+// sequence walks the tree, each CTA of the cluster owning a contiguous share
+// of the vocabulary and each warp a contiguous segment of that share (its
+// lanes read consecutive entries).  The
+// current distribution is kept in workspace as the last effective residual's
+// integer weights W and their sum S (P = W / S), so a rejection costs one
+// pass over the vocabulary whatever the number of earlier rejections; sums
+// are exact 64-bit integer reductions over the cluster (shared memory of the
+// peer CTAs).  All decisions use integer or correctly rounded fp64
+// operations (explicit _rn intrinsics, no contraction), so results are
+// bit-reproducible and independent of the cluster size.
+#include <cooperative_groups.h>
 #include <limits.h>
 
 #include "kernels.h"
@@ -186,152 +192,209 @@ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1
     return c;
 }
 
-// P after n rejections at the current node, for one vocabulary entry: each
-// step is W = floor(max(0, P - Q) * 2^32), P = W / S_j (P kept when S_j = 0).
-__device__ __forceinline__ double residual_chain(double P, double Q, const unsigned long long* S_hist, int n) {
-    for (int j = 0; j < n; ++j) {
-        const double diff = __dsub_rn(P, Q);
-        const unsigned long long W = diff > 0.0 ? (unsigned long long)floor(__dmul_rn(diff, 4294967296.0)) : 0ull;
-        const unsigned long long S = S_hist[j];
-        if (S > 0) P = __ddiv_rn((double)W, (double)S);
-    }
-    return P;
+constexpr double kTwo32 = 4294967296.0;
+
+// floor(max(0, x) * 2^32) as an integer weight
+__device__ __forceinline__ unsigned long long weight_2p32(double x) {
+    return x > 0.0 ? (unsigned long long)floor(__dmul_rn(x, kTwo32)) : 0ull;
 }
 
-__device__ __forceinline__ unsigned long long block_sum_u64(unsigned long long x, unsigned long long* red) {
+// Exact sums over the cluster.  Every thread passes its partial; returns the
+// cluster total, and in *before the sum of the partials of lower-ranked CTAs
+// and of lower-indexed warps of this CTA (the exclusive prefix of this warp's
+// segment in vocabulary order: shares and segments are contiguous and
+// rank-ordered).
+struct ClusterSum {
+    unsigned long long warp_tot[kStochThreads / 32];
+    unsigned long long cta_tot;
+};
+__device__ unsigned long long cluster_sum(unsigned long long x, ClusterSum* sh, unsigned long long* before) {
+    namespace cg = cooperative_groups;
+    cg::cluster_group cl = cg::this_cluster();
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    unsigned long long wt = x;  // warp total
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(kFull, x, o);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int o = 16; o > 0; o >>= 1) wt += __shfl_xor_sync(kFull, wt, o);
+    if (lane == 0) sh->warp_tot[warp] = wt;
     __syncthreads();
-    if (lane == 0) red[warp] = x;
-    __syncthreads();
-    unsigned long long t = 0;
-    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += red[w];
-    return t;
+    unsigned long long wbefore = 0, cta = 0;
+    for (int w = 0; w < kStochThreads / 32; ++w) {
+        const unsigned long long t = sh->warp_tot[w];
+        if (w < warp) wbefore += t;
+        cta += t;
+    }
+    if (tid == 0) sh->cta_tot = cta;
+    cl.sync();  // every CTA's total (and its earlier global writes) visible
+    const int rank = (int)cl.block_rank(), C = (int)cl.num_blocks();
+    unsigned long long tot = 0, rbefore = 0;
+    for (int r = 0; r < C; ++r) {
+        const unsigned long long t = cl.map_shared_rank(sh, r)->cta_tot;
+        if (r < rank) rbefore += t;
+        tot += t;
+    }
+    cl.sync();  // nobody reuses sh before every CTA has read it
+    if (before) *before = rbefore + wbefore;
+    return tot;
 }
 
-__global__ void __launch_bounds__(kStochThreads) verify_stochastic_kernel(
+__global__ void __launch_bounds__(kStochThreads, 2) verify_stochastic_kernel(
     const float* __restrict__ p, const float* __restrict__ q, int q_rows, const int32_t* __restrict__ q_row,
     const int32_t* __restrict__ node_tokens, int V, const TreeDev* __restrict__ tree, uint32_t key0, uint32_t key1,
-    uint32_t step, int32_t* accept_path, int max_path, int32_t* accept_len, int32_t* bonus, int32_t* status) {
-    __shared__ unsigned long long S_hist[kMaxTree];
-    __shared__ unsigned long long red[kStochThreads / 32];
-    __shared__ int s_flag, s_found;
-    const int b = blockIdx.x, tid = threadIdx.x;
+    uint32_t step, int32_t* accept_path, int max_path, int32_t* accept_len, int32_t* bonus,
+    unsigned long long* ws_w, int32_t* status) {
+    namespace cg = cooperative_groups;
+    cg::cluster_group cl = cg::this_cluster();
+    __shared__ ClusterSum sh;
+    const int C = (int)cl.num_blocks(), rank = (int)cl.block_rank();
+    const int b = blockIdx.x / C, tid = threadIdx.x;
+    const bool lead = rank == 0 && tid == 0;
     const int T = tree->T;
     const float* Pb = p + (long)b * T * V;
-    int u = 0, L = 1;
-    if (tid == 0) {
+    // Two weight buffers.  `valid` holds the last effective residual (S > 0)
+    // of the current node, -1 while P is still p[b,u,:].  `keep` is the
+    // buffer the latest accept decision may have read (threads of the
+    // cluster may still be reading it, also after the walk moved on); a pass
+    // writes the other one, which becomes valid if its sum is positive (a
+    // residual with S = 0 keeps P).  The cluster-wide sum that ends a pass
+    // orders every later reuse.
+    const long BV = (long)gridDim.x / C * V;
+    // this warp's vocabulary segment [y0, y1); lane l takes y0 + l + 32 i
+    const int warp = tid >> 5, lane = tid & 31;
+    const int share = (V + C - 1) / C;
+    const int v0 = min(V, rank * share), v1 = min(V, v0 + share);
+    const int seg = (v1 - v0 + kStochThreads / 32 - 1) / (kStochThreads / 32);
+    const int y0 = min(v1, v0 + warp * seg), y1 = min(v1, y0 + seg);
+    constexpr int U = 8;  // entries in flight per lane
+
+    int u = 0, L = 1, valid = -1, keep = -1;
+    unsigned long long S_valid = 0;
+    const float* Prow = Pb;
+    auto Wbuf = [&](int i) { return ws_w + (i & 1) * BV + (long)b * V; };
+    // current target distribution at y
+    auto cur = [&](int y) -> double {
+        if (valid < 0) return (double)Prow[y];
+        return __ddiv_rn((double)Wbuf(valid)[y], (double)S_valid);
+    };
+    if (lead) {
         accept_path[(long)b * max_path] = 0;
         for (int t = 1; t < max_path; ++t) accept_path[(long)b * max_path + t] = -1;
     }
-    int nrej = 0;
     const float* Qrow = nullptr;
     for (;;) {
         const int c_begin = tree->child_off[u], c_end = tree->child_off[u + 1];
-        nrej = 0;
+        if (valid >= 0) keep = valid;
+        valid = -1;
+        Prow = Pb + (long)u * V;
         if (c_begin == c_end) break;  // a leaf: no drafted children
         const int qr = q_row ? q_row[u] : u;
         if (qr < 0 || qr >= q_rows) {
-            if (tid == 0) set_status(status, MEDUSA_STATUS_BAD_TOKEN);
+            if (lead) set_status(status, MEDUSA_STATUS_BAD_TOKEN);
             break;
         }
         Qrow = q + ((long)b * q_rows + qr) * V;
-        const float* Prow = Pb + (long)u * V;
         bool moved = false;
         for (int ci = c_begin; ci < c_end; ++ci) {
             const int c = tree->child_idx[ci];
             const int x = node_tokens[(long)b * T + c];
             if (x < 0 || x >= V) {
-                if (tid == 0) set_status(status, MEDUSA_STATUS_BAD_TOKEN);
+                if (lead) set_status(status, MEDUSA_STATUS_BAD_TOKEN);
                 continue;
             }
-            if (tid == 0) {
-                const uint4 r = philox4x32_10(make_uint4((uint32_t)b, (uint32_t)c, step, 0u), key0, key1);
-                const double uc = (double)(r.x >> 8) * (1.0 / 16777216.0);
-                const double Qx = (double)Qrow[x];
-                const double Px = residual_chain((double)Prow[x], Qx, S_hist, nrej);
-                s_flag = __dmul_rn(uc, Qx) < Px;
-            }
-            __syncthreads();
-            const bool acc = s_flag;
-            __syncthreads();
-            if (acc) {
+            // every thread takes the same decision from the same values
+            const uint4 r = philox4x32_10(make_uint4((uint32_t)b, (uint32_t)c, step, 0u), key0, key1);
+            const double uc = (double)(r.x >> 8) * (1.0 / 16777216.0);
+            const double Qx = (double)Qrow[x];
+            if (__dmul_rn(uc, Qx) < cur(x)) {
                 u = c;
-                if (tid == 0) accept_path[(long)b * max_path + L] = c;
+                if (lead) accept_path[(long)b * max_path + L] = c;
                 ++L;
                 moved = true;
                 break;
             }
-            // rejected: residual sum at this node
+            // rejected: W(y) = floor(max(0, P(y) - Q(y)) * 2^32), S = sum W
             unsigned long long part = 0;
-            for (int y = tid; y < V; y += kStochThreads) {
-                const double Qy = (double)Qrow[y];
-                const double P = residual_chain((double)Prow[y], Qy, S_hist, nrej);
-                const double diff = __dsub_rn(P, Qy);
-                part += diff > 0.0 ? (unsigned long long)floor(__dmul_rn(diff, 4294967296.0)) : 0ull;
+            const int nb = keep < 0 ? 0 : keep ^ 1;
+            unsigned long long* Wn = Wbuf(nb);
+            for (int y = y0 + lane; y < y1; y += 32 * U) {
+                double P[U], Q[U];
+#pragma unroll
+                for (int i = 0; i < U; ++i) {
+                    const int yy = y + 32 * i;
+                    P[i] = yy < y1 ? cur(yy) : 0.0;
+                    Q[i] = yy < y1 ? (double)Qrow[yy] : 0.0;
+                }
+#pragma unroll
+                for (int i = 0; i < U; ++i) {
+                    const int yy = y + 32 * i;
+                    if (yy < y1) {
+                        const unsigned long long w = weight_2p32(__dsub_rn(P[i], Q[i]));
+                        Wn[yy] = w;
+                        part += w;
+                    }
+                }
             }
-            const unsigned long long S = block_sum_u64(part, red);
-            if (tid == 0) S_hist[nrej] = S;
-            __syncthreads();
-            ++nrej;
+            const unsigned long long S = cluster_sum(part, &sh, nullptr);
+            if (S > 0) {
+                valid = keep = nb;
+                S_valid = S;
+            }
         }
         if (!moved) break;
     }
-    // bonus from the current distribution P (p[b,u,:] after nrej residual steps)
-    const float* Prow = Pb + (long)u * V;
+    // bonus from the current distribution: weights floor(P(y) * 2^32), kept
+    // in the next buffer for the scan below
+    unsigned long long* Wb = Wbuf(keep < 0 ? 0 : keep ^ 1);
     unsigned long long part = 0;
-    for (int y = tid; y < V; y += kStochThreads) {
-        const double P = nrej ? residual_chain((double)Prow[y], (double)Qrow[y], S_hist, nrej) : (double)Prow[y];
-        part += P > 0.0 ? (unsigned long long)floor(__dmul_rn(P, 4294967296.0)) : 0ull;
+    for (int y = y0 + lane; y < y1; y += 32 * U) {
+        double P[U];
+#pragma unroll
+        for (int i = 0; i < U; ++i) P[i] = y + 32 * i < y1 ? cur(y + 32 * i) : 0.0;
+#pragma unroll
+        for (int i = 0; i < U; ++i)
+            if (y + 32 * i < y1) {
+                const unsigned long long w = weight_2p32(P[i]);
+                Wb[y + 32 * i] = w;
+                part += w;
+            }
     }
-    const unsigned long long S = block_sum_u64(part, red);
+    unsigned long long start;
+    const unsigned long long S = cluster_sum(part, &sh, &start);
+    if (lead) accept_len[b] = L;
+    if (S == 0) {
+        if (lead) {
+            set_status(status, MEDUSA_STATUS_NO_MASS);
+            bonus[b] = 0;
+        }
+        return;
+    }
     const uint4 r = philox4x32_10(make_uint4((uint32_t)b, (uint32_t)u, step, 0u), key0, key1);
     // t = floor(U * S / 2^32) from the exact 128-bit product
     const unsigned long long lo = (unsigned long long)r.y * (S & 0xffffffffull);
     const unsigned long long hi = (unsigned long long)r.y * (S >> 32);
     const unsigned long long t = (lo >> 32) + hi;
-    if (tid == 0) s_found = -1;
-    __syncthreads();
-    int tok = 0;
-    if (S == 0) {
-        if (tid == 0) set_status(status, MEDUSA_STATUS_NO_MASS);
-    } else {
-        // inverse CDF: smallest y with inclusive prefix sum > t, block by block
-        unsigned long long run = 0;
-        const int warp = tid >> 5, lane = tid & 31;
-        __shared__ unsigned long long wsum[kStochThreads / 32];
-        for (int y0 = 0; y0 < V; y0 += kStochThreads) {
-            const int y = y0 + tid;
-            unsigned long long w = 0;
-            if (y < V) {
-                const double P =
-                    nrej ? residual_chain((double)Prow[y], (double)Qrow[y], S_hist, nrej) : (double)Prow[y];
-                w = P > 0.0 ? (unsigned long long)floor(__dmul_rn(P, 4294967296.0)) : 0ull;
-            }
-            unsigned long long inc = w;  // inclusive scan within the warp
+    // the smallest y whose inclusive prefix sum exceeds t lies in the one
+    // warp segment with start <= t < start + (segment total)
+    unsigned long long wtot = part;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) wtot += __shfl_xor_sync(kFull, wtot, o);
+    if (start <= t && t < start + wtot) {
+        unsigned long long run = start;
+        for (int y = y0; y < y1; y += 32) {
+            const unsigned long long w = y + lane < y1 ? Wb[y + lane] : 0ull;
+            unsigned long long inc = w;  // inclusive scan of 32 consecutive entries
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
-                unsigned long long n = __shfl_up_sync(kFull, inc, o);
+                const unsigned long long n = __shfl_up_sync(kFull, inc, o);
                 if (lane >= o) inc += n;
             }
-            if (lane == 31) wsum[warp] = inc;
-            __syncthreads();
-            unsigned long long before = run;
-            for (int w2 = 0; w2 < warp; ++w2) before += wsum[w2];
-            unsigned long long total = run;
-            for (int w2 = 0; w2 < kStochThreads / 32; ++w2) total += wsum[w2];
-            const unsigned long long incl = before + inc;
-            if (y < V && w > 0 && incl > t && incl - w <= t) s_found = y;  // exactly one such y
-            __syncthreads();
-            if (s_found >= 0) break;
-            run = total;
+            const unsigned long long total = __shfl_sync(kFull, inc, 31);
+            if (run + total > t) {
+                const unsigned m = __ballot_sync(kFull, run + inc > t);
+                if (lane == 0) bonus[b] = y + __ffs(m) - 1;
+                break;
+            }
+            run += total;
         }
-        tok = s_found >= 0 ? s_found : 0;
-    }
-    if (tid == 0) {
-        accept_len[b] = L;
-        bonus[b] = tok;
     }
 }
 
@@ -347,8 +410,17 @@ int argmax_splits(int rows, int V) {
 
 }  // namespace
 
+// cluster size of the stochastic kernel: up to 8 CTAs per sequence while the
+// grid fits in one wave
+int stoch_cluster(int B) {
+    int c = 1;
+    while (c < 8 && (long)B * c * 2 <= 2L * num_sms()) c *= 2;  // two 512-thread CTAs per SM
+    return c;
+}
+
 size_t verify_workspace_size(medusa_verify_mode mode, int B, int V, int T) {
-    if (mode != MEDUSA_VERIFY_GREEDY) return 0;
+    if (mode != MEDUSA_VERIFY_GREEDY)  // two buffers of W (u64) per sequence and vocabulary entry
+        return align256(2 * (size_t)B * V * sizeof(unsigned long long));
     int s = argmax_splits(B * T, V);
     return align256((size_t)B * T * s * sizeof(float)) + align256((size_t)B * T * s * sizeof(int));
 }
@@ -374,10 +446,22 @@ cudaError_t verify_launch(const VerifyArgs& a, cudaStream_t st) {
                                                          a.max_path, a.accept_len, a.bonus);
         return cudaGetLastError();
     }
-    verify_stochastic_kernel<<<a.B, kStochThreads, 0, st>>>(
-        (const float*)a.target, a.q, a.q_rows, a.q_row, a.node_tokens, a.V, a.tree, (uint32_t)a.seed,
-        (uint32_t)(a.seed >> 32), a.step, a.accept_path, a.max_path, a.accept_len, a.bonus, a.status);
-    return cudaGetLastError();
+    const int C = stoch_cluster(a.B);
+    unsigned long long* ws_w = (unsigned long long*)a.ws;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.B * C);
+    cfg.blockDim = dim3(kStochThreads);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, verify_stochastic_kernel, (const float*)a.target, a.q, a.q_rows, a.q_row,
+                              a.node_tokens, a.V, a.tree, (uint32_t)a.seed, (uint32_t)(a.seed >> 32), a.step,
+                              a.accept_path, a.max_path, a.accept_len, a.bonus, ws_w, a.status);
 }
 
 }  // namespace medusa

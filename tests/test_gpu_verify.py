@@ -96,7 +96,7 @@ def run_stoch(parents, p, q, tok, seed, step, q_row=None):
     return out
 
 
-@pytest.mark.parametrize("kw", [dict(B=8), dict(B=3, V=777), dict()])
+@pytest.mark.parametrize("kw", [dict(B=8), dict(B=3, V=777), dict(), dict(B=1), dict(B=12, V=3001)])
 def test_stochastic_parity(kw):
     w = I.scaled(I.WORKLOADS["stoch_b64"], **kw)
     parents = I.workload_tree(w)
