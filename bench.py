@@ -34,9 +34,11 @@ import torch  # noqa: E402
 METRIC = "Medusa verify steps/s (8B shape, 117-node tree); tree-attn HBM GB/s vs peak"
 UNIT = "steps/s"
 WORKLOAD = "llama8b"
-# DRAM bytes per launch of the heads stage from an ncu capture (sum over its
-# kernels); None until a capture of the current kernels exists.
-HEADS_DRAM_BYTES = None
+# DRAM bytes (read + write) per launch of the heads kernel, from an ncu capture
+# of the same kernel at V=32000 (1.18303 GB read + 3.86 MB written against
+# 1.18279 GB of weights), scaled to the workload's weight bytes; only for the
+# workload whose launch configuration (B=1, d=4096, K=4) was captured.
+HEADS_DRAM_BYTES = {"llama8b": 4336910336 * (1183026000 + 3864320) / 1182793728}
 
 
 def peaks():
@@ -399,7 +401,7 @@ def run_mine(args, rank, world, local_rank):
         roofline = {"kernel": "medusa_heads (residual GEMV + LM-head GEMV with softmax/top-8 + merge)",
                     "bound": "hbm", "achieved": heads_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                     "frac": heads_gbs / pk["hbm_gbs"], "peak_source": pk["source"],
-                    "algorithmic_bytes": heads_bytes, "traffic": HEADS_DRAM_BYTES}
+                    "algorithmic_bytes": heads_bytes, "traffic": HEADS_DRAM_BYTES.get(w.name) if w == I.WORKLOADS.get(w.name) else None}
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": 1000.0 * t / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,

@@ -244,7 +244,12 @@ int tree_attention(const void* q, const void* k_tree, const void* v_tree, const 
  * node_tokens [B, T] int32; accept_path [B, max_path] int32 out (node ids,
  * root first, -1 padded); accept_len [B] int32 out (>= 1, counts the root);
  * bonus [B] int32 out.  max_path >= the tree's max depth.
- * Workspace: tree_verify_workspace_size(...) bytes.
+ * Workspace: tree_verify_workspace_size(...) bytes, 16-byte aligned, device
+ * memory owned by the caller (greedy: row-argmax partials; stochastic: two
+ * 8-byte integer weights per sequence and vocabulary entry, 16 * B * V bytes
+ * plus alignment).  Its contents need no initialisation; concurrent calls
+ * need separate workspaces.  Too small a workspace fails with
+ * MEDUSA_ERR_WORKSPACE before anything is launched.
  */
 size_t tree_verify_workspace_size(medusa_verify_mode mode, int B, int V, const medusa_tree* tree);
 int tree_verify(medusa_verify_mode mode, const void* target, medusa_dtype target_dt, const float* q, int q_rows,
