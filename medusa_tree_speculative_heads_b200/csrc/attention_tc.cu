@@ -167,7 +167,7 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
     }
     if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
     tc_fence_before();
-    __syncthreads();
+    sync_block();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
@@ -423,7 +423,7 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
         }
     }
     tc_fence_before();
-    __syncthreads();
+    sync_block();
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);

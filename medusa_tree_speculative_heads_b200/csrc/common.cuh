@@ -179,6 +179,17 @@ __device__ __forceinline__ void set_status(int32_t* status, int bits) {
 
 // Total order of (value, index) candidates used by top-s and argmax: a larger
 // value wins; among equal values the lower index wins; NaN never wins.
+// Block-wide barrier after code in which the lanes of a warp took different
+// paths (lane 0 running a producer or MMA loop while the others wait, say).
+// The barrier behind __syncthreads is an aligned one: it must be reached by
+// whole warps, and a warp that arrives with some lanes still elsewhere is
+// counted wrongly (the barrier can release early).  Each warp reconverges
+// first.
+__device__ __forceinline__ void sync_block() {
+    __syncwarp();
+    __syncthreads();
+}
+
 __device__ __forceinline__ bool beats(float v, int i, float w, int j) { return v > w || (v == w && i < j); }
 
 }  // namespace medusa

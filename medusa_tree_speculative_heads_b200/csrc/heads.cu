@@ -373,7 +373,7 @@ __global__ void __launch_bounds__((kFC + 1) * 32, 1) heads_fused_kernel(const __
         s_flag = 0;
     }
     for (int t = threadIdx.x; t < kFC * a.K; t += blockDim.x) sstate[t] = empty_state();
-    __syncthreads();
+    sync_block();
 
     if (warp == kFC) {
         // ---------------- producer ----------------
@@ -551,7 +551,7 @@ __global__ void __launch_bounds__((kFC + 1) * 32, 1) heads_fused_kernel(const __
         }
         if (cur_k >= 0) flush(cur_k);
     }
-    __syncthreads();
+    sync_block();
 
     // this CTA's partial per head it covered
     if (warp < kFC && b1 > b0) {
@@ -599,11 +599,11 @@ __global__ void __launch_bounds__((kFC + 1) * 32, 1) heads_fused_kernel(const __
     __threadfence();
     __syncthreads();
     if (threadIdx.x == 0) s_flag = atomicAdd(&a.ctr[1], 1u) == gridDim.x - 1;
-    __syncthreads();
+    sync_block();
     if (!s_flag) return;
     __threadfence();
     for (int k = warp; k < a.K; k += kFC + 1)
-        merge_head(a.part, gridDim.x, a.V, kBG, 0, 0, a.V, a.K, k, a.tree, a.root_token, a.topk_idx, a.topk_prob,
+        merge_head(a.part, gridDim.x, a.V, 1, kBG, 0, 0, a.V, a.K, k, a.tree, a.root_token, a.topk_idx, a.topk_prob,
                    a.node_tokens, a.node_q, a.stats, a.status);
 }
 
@@ -617,7 +617,7 @@ __global__ void __launch_bounds__(32) heads_merge_kernel(const HeadState* __rest
                                                          float* __restrict__ node_q, float2* __restrict__ stats,
                                                          int32_t* status) {
     const int bb = blockIdx.x % nb, k = blockIdx.x / nb;
-    merge_head(part, nparts, V, kBG, bb, b0 + bb, V, K, k, tree, root_token, topk_idx, topk_prob, node_tokens, node_q,
+    merge_head(part, nparts, V, 1, kBG, bb, b0 + bb, V, K, k, tree, root_token, topk_idx, topk_prob, node_tokens, node_q,
                stats, status);
 }
 
@@ -654,7 +654,7 @@ LmConfig lm_config(int K) {
 int lm_grid_bound() { return num_sms() * (2048 / (kLmWarps * 32)); }
 
 struct HeadsWs {
-    size_t hk, part, stats, ctr, logits, total;
+    size_t hk, part, stats, ctr, slots, logits, total;
 };
 
 HeadsWs heads_ws_layout(int B, int d, int V, int K, medusa_dtype dt) {
@@ -665,7 +665,11 @@ HeadsWs heads_ws_layout(int B, int d, int V, int K, medusa_dtype dt) {
     const int bstride = B > kBG ? (B < 64 ? B : 64) : kBG;  // tensor-core path keeps one partial per sequence
     w.stats = w.part + align256((size_t)lm_grid_bound() * K * bstride * sizeof(HeadState));
     w.ctr = w.stats + align256((size_t)B * K * sizeof(float2));
-    w.logits = w.ctr + 256;
+    // counters, and on the tensor-core path one hand-over flag per CTA and
+    // phase plus the handed-over partial tiles ([2][grid][B][128] fp32)
+    w.slots = w.ctr + align256((size_t)(2 + 2 * num_sms()) * sizeof(unsigned int));
+    const size_t slots = heads_tc_supported(B, d, dt) ? (size_t)2 * num_sms() * B * 128 * sizeof(float) : 0;
+    w.logits = w.slots + align256(slots);
     w.total = w.logits + align256((size_t)B * K * V * sizeof(float));
     return w;
 }
@@ -684,7 +688,7 @@ cudaError_t heads_launch_t(const HeadsArgs& a, cudaStream_t st) {
     cudaError_t e;
     if (heads_tc_supported(a.B, a.d, a.dt)) {
         // bf16: weight streaming on the tensor cores (one cooperative kernel)
-        e = heads_tc_launch(a, hk, part, (unsigned int*)(ws + w.ctr), stats, logits, st);
+        e = heads_tc_launch(a, hk, part, (unsigned int*)(ws + w.ctr), (float*)(ws + w.slots), stats, logits, st);
         if (e != cudaSuccess) return e;
         if (a.probs_out) {
             const long n = (long)a.B * a.K * a.V;

@@ -100,21 +100,36 @@ __device__ __forceinline__ void warp_select(float (&lv)[kTopK], int (&li)[kTopK]
 
 // ---------------------------------------------------------------------------
 // Merge of one (sequence, head): the partials of the CTAs that covered the
-// head, in CTA order (the CTAs split K*uph units evenly, head k owning units
-// [k*uph, (k+1)*uph); partial (c, k, b) sits at part[(c*K + k)*bstride + b]) (so the result does not depend on which CTA runs
-// the merge); writes the top-8 entries with their probabilities, the head's
+// head, in CTA order, so the result does not depend on which CTA runs the
+// merge.  The K*uph tiles (head k owning tiles [k*uph, (k+1)*uph)) are cut
+// into upt units each; the CTAs split the K*uph*upt units evenly and CTA c
+// owns the tiles whose first unit falls in its share; partial (c, k, b) sits
+// at part[(c*K + k)*bstride + b].  Writes the top-8 entries with their probabilities, the head's
 // softmax statistics, and fills the tree nodes this head proposes.  One warp.
 // Partials are read through L2 (they may have been written by other CTAs of
 // the same kernel).
 // ---------------------------------------------------------------------------
-static __device__ __noinline__ void merge_head(const HeadState* __restrict__ part, int nparts, long uph, int bstride, int bb,
+static __device__ __noinline__ void merge_head(const HeadState* __restrict__ part, int nparts, long uph, int upt,
+                                               int bstride, int bb,
                                        int b, int V, int K, int k,
                            const TreeDev* __restrict__ tree, const int32_t* __restrict__ root_token,
                            int32_t* __restrict__ topk_idx, float* __restrict__ topk_prob,
                            int32_t* __restrict__ node_tokens, float* __restrict__ node_q, float2* __restrict__ stats,
                            int32_t* status) {
     const int lane = threadIdx.x & 31;
-    const long R = (long)K * uph;
+    const long R = (long)K * uph * upt;
+    // the tree's shape and the root token are needed at the end: load them
+    // first, so their latency overlaps the partials'
+    constexpr int kTreeChunks = kMaxTree / 32;
+    int rk[kTreeChunks], dp[kTreeChunks];
+    const int T = tree ? tree->T : 0;
+#pragma unroll
+    for (int j = 0; j < kTreeChunks; ++j) {
+        const int i = lane + 32 * j;
+        rk[j] = i < T ? tree->rank[i] : 0;
+        dp[j] = i < T ? tree->depth[i] : 0;
+    }
+    const int rt = (tree && k == 0) ? root_token[b] : 0;
     float mm = -INFINITY, ll = 0.f;
     float lv[kTopK];
     int li[kTopK];
@@ -123,21 +138,45 @@ static __device__ __noinline__ void merge_head(const HeadState* __restrict__ par
         lv[j] = -INFINITY;
         li[j] = INT_MAX;
     }
-    for (int c = lane; c < nparts; c += 32) {
+    // CTA c owns the units [r0, r1), i.e. the tiles whose first unit lies there;
+    // the CTAs covering head k form the range [c_lo, c_hi], the owners of its
+    // first and last tiles (unit u lies in the share of CTA ceil((u+1) N / R) - 1)
+    auto owner = [&](long u) -> int { return (int)(((u + 1) * nparts + R - 1) / R - 1); };
+    const int c_lo = owner((long)k * uph * upt), c_hi = owner(((long)(k + 1) * uph - 1) * upt);
+    // when every share holds a tile start, every CTA of the range covers head k
+    const bool dense = R / nparts >= upt;
+    auto covers = [&](int c) -> bool {
+        if (c > c_hi) return false;
+        if (dense) return true;
         const long r0 = R * c / nparts, r1 = R * (c + 1) / nparts;
-        if (r1 <= r0 || (long)(k + 1) * uph <= r0 || r1 <= (long)k * uph) continue;  // CTA c did not cover head k
-        const HeadState* s = &part[((long)c * K + k) * bstride + bb];
-        float pv[kTopK];
-        int pi[kTopK];
+        return (r1 + upt - 1) / upt > (r0 + upt - 1) / upt;  // owns a tile (in head k, by the range)
+    };
+    // lane l takes CTAs c_lo + l, c_lo + l + 32, ...; two of them per round,
+    // all loads of a round issued before any is used
+    for (int j0 = 0; c_lo + 32 * j0 <= c_hi; j0 += 2) {
+        const int cc[2] = {c_lo + lane + 32 * j0, c_lo + lane + 32 * (j0 + 1)};
+        const bool cv[2] = {covers(cc[0]), covers(cc[1])};
+        float pv[2][kTopK], sm[2], sl[2];
+        int pi[2][kTopK];
 #pragma unroll
-        for (int j = 0; j < kTopK; ++j) {  // issue every load before using any
-            pv[j] = __ldcg(&s->val[j]);
-            pi[j] = __ldcg(&s->idx[j]);
+        for (int u = 0; u < 2; ++u) {
+            if (!cv[u]) continue;
+            const HeadState* s = &part[((long)cc[u] * K + k) * bstride + bb];
+#pragma unroll
+            for (int j = 0; j < kTopK; ++j) {
+                pv[u][j] = __ldcg(&s->val[j]);
+                pi[u][j] = __ldcg(&s->idx[j]);
+            }
+            sm[u] = __ldcg(&s->m);
+            sl[u] = __ldcg(&s->l);
         }
-        const float sm = __ldcg(&s->m), sl = __ldcg(&s->l);
-        merge_ml(mm, ll, sm, sl);
 #pragma unroll
-        for (int j = 0; j < kTopK; ++j) list_insert(lv, li, pv[j], pi[j]);
+        for (int u = 0; u < 2; ++u) {
+            if (!cv[u]) continue;
+            merge_ml(mm, ll, sm[u], sl[u]);
+#pragma unroll
+            for (int j = 0; j < kTopK; ++j) list_insert(lv, li, pv[u][j], pi[u][j]);
+        }
     }
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -156,21 +195,18 @@ static __device__ __noinline__ void merge_head(const HeadState* __restrict__ par
     }
     if (lane == 0 && stats) stats[(long)b * K + k] = make_float2(mm, ll);
     if (tree) {
-        const int T = tree->T;
-        for (int i0 = 0; i0 < T; i0 += 32) {
-            const int i = i0 + lane;
-            const int rk = i < T ? tree->rank[i] : 0;
-            const int dp = i < T ? tree->depth[i] : 0;
-            const int tok = __shfl_sync(kFull, valid ? oi : -1, rk & (kTopK - 1));
-            const float pq = __shfl_sync(kFull, prob, rk & (kTopK - 1));
-            if (i < T && i > 0 && dp == k + 2) {
+#pragma unroll
+        for (int j = 0; j < kTreeChunks; ++j) {
+            const int i = lane + 32 * j;
+            const int tok = __shfl_sync(kFull, valid ? oi : -1, rk[j] & (kTopK - 1));
+            const float pq = __shfl_sync(kFull, prob, rk[j] & (kTopK - 1));
+            if (i < T && i > 0 && dp[j] == k + 2) {
                 node_tokens[(long)b * T + i] = tok;
                 if (node_q) node_q[(long)b * T + i] = pq;
                 if (tok < 0) set_status(status, MEDUSA_STATUS_BAD_TOKEN);
             }
         }
         if (k == 0 && lane == 0) {
-            const int rt = root_token[b];
             node_tokens[(long)b * T] = rt;
             if (node_q) node_q[(long)b * T] = 1.f;
             if (rt < 0 || rt >= V) set_status(status, MEDUSA_STATUS_BAD_TOKEN);

@@ -25,10 +25,15 @@
 //            keeps that column's running softmax statistics and top-8 list
 //            in registers; at a head change the segments of each column are
 //            merged into the CTA's partial for (head, sequence).
-// The residual tiles of every head come first, then the vocabulary tiles;
-// the weight producer keeps prefetching across the grid barrier.  After a
-// second grid barrier the warps of the grid merge the (sequence, head)
-// partials, each in CTA order, and fill the tree.
+// Work split ("stream-K"): in each phase (residual, then vocabulary) the
+// tiles' 64-element k-blocks are laid end to end and every CTA takes an equal
+// contiguous run of them, so all SMs stream the same number of bytes.  A tile
+// cut by a run boundary is summed by the CTA holding its first k-block (its
+// owner, which reaches it last in its run); the CTAs holding the rest reach
+// their part first in theirs, and hand it over as an fp32 partial in global
+// memory with a release flag.  The weight producer keeps prefetching across
+// the grid barrier.  After a second grid barrier the warps of the grid merge
+// the (sequence, head) partials, each in CTA order, and fill the tree.
 // Every wait is bounded (~2 s) and sets MEDUSA_STATUS_TIMEOUT on expiry.
 #include <limits.h>
 
@@ -63,7 +68,8 @@ struct TcHeadsArgs {
     __nv_bfloat16* hk_out;  // nullable copy for the caller
     float* logits;          // [B][K][V], nullable
     HeadState* part;        // [grid][K][B]
-    unsigned int* ctr;      // [2], zero at launch
+    float* slots;           // [2 phases][grid][B][128] handed-over partial tiles
+    unsigned int* ctr;      // [2 + 2 * grid], zero at launch: grid-barrier arrivals, then the slots' flags
     const TreeDev* tree;
     const int32_t* root_token;
     int32_t* topk_idx;
@@ -75,6 +81,38 @@ struct TcHeadsArgs {
     int B, d, V, K;
     int stages;
 };
+
+// A CTA's run of one phase: k-block units [u0, u1) of the phase's tiles laid
+// end to end (tile t holds units [t nkb, (t+1) nkb)), the runs contiguous
+// and in CTA order.  Piece i of the run is the part of one tile it covers.
+struct Run {
+    long u0, u1;
+    int nkb;
+    __device__ Run(long U, int c, int G, int nkb_) : u0(U * c / G), u1(U * (c + 1) / G), nkb(nkb_) {}
+    __device__ int count() const { return u1 > u0 ? (int)((u1 - 1) / nkb - u0 / nkb + 1) : 0; }
+    __device__ void piece(int i, long& t, int& kb0, int& kb1) const {
+        t = u0 / nkb + i;
+        const long lo = u0 > t * nkb ? u0 : t * nkb;
+        const long hi = u1 < (t + 1) * nkb ? u1 : (t + 1) * nkb;
+        kb0 = (int)(lo - t * nkb);
+        kb1 = (int)(hi - t * nkb);
+    }
+};
+
+__device__ __forceinline__ void st_release_u32(unsigned int* p, unsigned int v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// bounded wait for a hand-over flag; false after ~2 s
+__device__ __forceinline__ bool wait_flag(const unsigned int* f) {
+    if (ld_acquire_u32(f)) return true;
+    const uint64_t t0 = global_ns();
+    while (!ld_acquire_u32(f)) {
+        if (global_ns() - t0 > 2000000000ull) return false;
+        __nanosleep(32);
+    }
+    return true;
+}
 
 __device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
 
@@ -99,14 +137,18 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int K = a.K, B = a.B;
+    const int G = gridDim.x, cta = blockIdx.x;
     const int tph_r = (a.d + kTM - 1) / kTM;   // residual tiles per head
     const int tph_l = (a.V + kTM - 1) / kTM;   // vocabulary tiles per head
-    const int nkb = (a.d + kTK - 1) / kTK;
-    const long T1 = (long)K * tph_r, T2 = (long)K * tph_l;
-    const long t1a = T1 * blockIdx.x / gridDim.x, t1b = T1 * (blockIdx.x + 1) / gridDim.x;
-    const long t2a = T2 * blockIdx.x / gridDim.x, t2b = T2 * (blockIdx.x + 1) / gridDim.x;
-    const int n1 = (int)(t1b - t1a), n2 = (int)(t2b - t2a);
-    const int ntiles = n1 + n2;
+    const int nkb = (a.d + kTK - 1) / kTK;     // k-blocks per tile
+    const long U1 = (long)K * tph_r * nkb, U2 = (long)K * tph_l * nkb;
+    const Run run1(U1, cta, G, nkb), run2(U2, cta, G, nkb);
+    const int n1 = run1.count(), n2 = run2.count();
+    const int ntiles = n1 + n2;  // pieces, residual phase first
+    auto piece = [&](int li, long& t, int& kb0, int& kb1) {
+        if (li < n1) run1.piece(li, t, kb0, kb1);
+        else run2.piece(li - n1, t, kb0, kb1);
+    };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
@@ -128,7 +170,7 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
     }
     if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
     tc_fence_before();
-    __syncthreads();
+    sync_block();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
@@ -137,11 +179,13 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
         if (lane == 0) {
             const bool weights = warp == 0;
             const uint32_t bytes = weights ? kABytes : kBBytes;
-            int issued = 0;
+            int it = 0;  // k-blocks issued (ring position)
             bool ok = true;
             for (int li = 0; li < ntiles && ok; ++li) {
                 const bool res = li < n1;
-                const long t = res ? t1a + li : t2a + (li - n1);
+                long t;
+                int kb0, kb1;
+                piece(li, t, kb0, kb1);
                 const int k = (int)(res ? t / tph_r : t / tph_l);
                 const int row0 = (int)(res ? t % tph_r : t % tph_l) * kTM;
                 if (!weights && li == n1) {
@@ -158,8 +202,7 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
                     fence_proxy_async_global();
                     if (!ok) break;
                 }
-                for (int kb = 0; kb < nkb; ++kb) {
-                    const int it = li * nkb + kb;
+                for (int kb = kb0; kb < kb1; ++kb) {
                     const int s = it % S;
                     if (it >= S && !mbar_wait(&empty[s], ((it / S) - 1) & 1)) {
                         set_status(a.status, MEDUSA_STATUS_TIMEOUT);
@@ -174,12 +217,12 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
                         tma_load_2d(sB + (size_t)s * kBBytes, &a.mh, kb * kTK, 0, &full[s]);
                     else
                         tma_load_3d(sB + (size_t)s * kBBytes, &a.mhk, kb * kTK, k, 0, &full[s]);
-                    ++issued;
+                    ++it;
                 }
             }
             // drain: no copy may still be landing when the CTA exits
-            for (int s = 0; s < S && s < issued; ++s) {
-                const int last = s + ((issued - 1 - s) / S) * S;
+            for (int s = 0; s < S && s < it; ++s) {
+                const int last = s + ((it - 1 - s) / S) * S;
                 mbar_wait(&full[s], (last / S) & 1);
             }
         }
@@ -187,6 +230,7 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
             bool ok = true;
+            int it = 0;
             for (int li = 0; li < ntiles && ok; ++li) {
                 const int buf = li & 1;
                 if (li >= 2 && !mbar_wait(&acc_empty[buf], ((li >> 1) - 1) & 1)) {
@@ -195,8 +239,10 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem + buf * N;
-                for (int kb = 0; kb < nkb; ++kb) {
-                    const int it = li * nkb + kb;
+                long t;
+                int kb0, kb1;
+                piece(li, t, kb0, kb1);
+                for (int kb = kb0; kb < kb1; ++kb) {
                     const int s = it % S;
                     if (!mbar_wait(&full[s], (it / S) & 1)) {
                         set_status(a.status, MEDUSA_STATUS_TIMEOUT);
@@ -208,8 +254,9 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
                     const uint64_t bdesc = sw128_kmajor_desc(smem_addr(sB + (size_t)s * kBBytes));
 #pragma unroll
                     for (int ks = 0; ks < kTK / 16; ++ks)  // 16 k-elements = 32 bytes per MMA
-                        tc_mma_bf16(d_tmem, adesc + 2 * ks, bdesc + 2 * ks, kIdesc, (kb | ks) != 0);
+                        tc_mma_bf16(d_tmem, adesc + 2 * ks, bdesc + 2 * ks, kIdesc, (kb != kb0 || ks != 0) ? 1u : 0u);
                     tc_commit(&empty[s]);
+                    ++it;
                 }
                 tc_commit(&acc_full[buf]);
             }
@@ -250,7 +297,49 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
                 }
             }
             epi_sync();
-            if (et < B) {
+            if (nseg >= 8) {
+                // many segments per column: one warp per column, lane s holding
+                // segment s (softmax statistics by a butterfly, top-8 by
+                // repeated warp maxima over the lanes' sorted lists)
+                for (int b = ew; b < B; b += 4) {
+                    float mm = -INFINITY, ll = 0.f;
+                    float mv[kTopK];
+                    int mi[kTopK];
+#pragma unroll
+                    for (int j = 0; j < kTopK; ++j) {
+                        mv[j] = -INFINITY;
+                        mi[j] = INT_MAX;
+                    }
+                    if (lane < nseg) {
+                        const HeadState* o = &stS[lane * B + b];
+                        mm = o->m;
+                        ll = o->l;
+#pragma unroll
+                        for (int j = 0; j < kTopK; ++j) {
+                            mv[j] = o->val[j];
+                            mi[j] = o->idx[j];
+                        }
+                    }
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const float m2 = __shfl_xor_sync(kFull, mm, o);
+                        const float l2 = __shfl_xor_sync(kFull, ll, o);
+                        merge_ml(mm, ll, m2, l2);
+                    }
+                    float ov;
+                    int oi;
+                    warp_select(mv, mi, ov, oi);
+                    HeadState* dst = &a.part[((long)blockIdx.x * K + kk) * B + b];
+                    if (lane < kTopK) {
+                        dst->val[lane] = ov;
+                        dst->idx[lane] = oi;
+                    }
+                    if (lane == 0) {
+                        dst->m = mm;
+                        dst->l = ll;
+                    }
+                }
+            } else if (et < B) {
                 // merge the column's segments in segment order
                 float mm = -INFINITY, ll = 0.f;
                 float mv[kTopK];
@@ -318,9 +407,43 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[buf]);
+            const int ph = li < n1 ? 0 : 1;
+            long t;
+            int kb0, kb1;
+            piece(li, t, kb0, kb1);
+            if (kb0 > 0) {
+                // the later k-blocks of a tile owned by an earlier CTA: hand the
+                // partial sum over (this is the first piece of this CTA's run)
+                float* dst = a.slots + (long)(ph * G + cta) * B * kTM;
+                if (ok) {
+#pragma unroll
+                    for (int e = 0; e < N; ++e)
+                        if (e < B) dst[e * kTM + row] = v[e];
+                }
+                __threadfence();
+                epi_sync();
+                if (et == 0) st_release_u32(&a.ctr[2 + ph * G + cta], 1u);
+                if (li == n1 - 1) arrive_grid();
+                continue;
+            }
+            if (kb1 < nkb && ok) {
+                // the rest of this tile: the first pieces of the next CTAs' runs
+                const long U = ph == 0 ? U1 : U2, tend = (t + 1) * nkb;
+                for (int c2 = cta + 1; c2 < G && U * c2 / G < tend; ++c2) {
+                    if (U * (c2 + 1) / G == U * c2 / G) continue;  // an empty run
+                    if (!wait_flag(&a.ctr[2 + ph * G + c2])) {
+                        if (lane == 0) set_status(a.status, MEDUSA_STATUS_TIMEOUT);
+                        ok = false;
+                        break;
+                    }
+                    const float* src = a.slots + (long)(ph * G + c2) * B * kTM;
+#pragma unroll
+                    for (int e = 0; e < N; ++e)
+                        if (e < B) v[e] += __ldcg(&src[e * kTM + row]);
+                }
+            }
             if (li < n1) {
                 // residual tile: h^(k)[b, o] = SiLU(z) + h[b, o]
-                const long t = t1a + li;
                 const int k = (int)(t / tph_r);
                 const int o = (int)(t % tph_r) * kTM + row;
                 if (ok && o < a.d) {
@@ -341,7 +464,6 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
                 continue;
             }
             // vocabulary tile
-            const long t = t2a + (li - n1);
             const int k = (int)(t / tph_l);
             const int row0 = (int)(t % tph_l) * kTM;
             if (k != cur_k) {
@@ -381,7 +503,7 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
 
     // ---------------- teardown ----------------
     tc_fence_before();
-    __syncthreads();
+    sync_block();
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
@@ -389,7 +511,7 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
     // grid barrier: every CTA's partials are written; then the (sequence,
     // head) merges are spread over all warps of the grid
     __threadfence();
-    __syncthreads();
+    sync_block();
     if (threadIdx.x == 0) {
         atomicAdd(&a.ctr[1], 1u);
         const uint64_t t0 = global_ns();
@@ -402,12 +524,12 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
             __nanosleep(64);
         }
     }
-    __syncthreads();
+    sync_block();
     if (*flag) return;
     __threadfence();
     for (int p = blockIdx.x * kTcWarps + warp; p < B * K; p += gridDim.x * kTcWarps) {
         const int b = p % B, k = p / B;
-        merge_head(a.part, gridDim.x, tph_l, B, b, b, a.V, K, k, a.tree, a.root_token, a.topk_idx, a.topk_prob,
+        merge_head(a.part, gridDim.x, tph_l, nkb, B, b, b, a.V, K, k, a.tree, a.root_token, a.topk_idx, a.topk_prob,
                    a.node_tokens, a.node_q, a.stats, a.status);
     }
 }
@@ -450,8 +572,8 @@ cudaError_t launch_n(const TcHeadsArgs& args, cudaStream_t st) {
 
 bool heads_tc_supported(int B, int d, medusa_dtype dt) { return dt == MEDUSA_BF16 && B >= 1 && B <= 64 && d % 8 == 0; }
 
-cudaError_t heads_tc_launch(const HeadsArgs& x, void* hk, void* part, unsigned int* ctr, float2* stats, float* logits,
-                            cudaStream_t st) {
+cudaError_t heads_tc_launch(const HeadsArgs& x, void* hk, void* part, unsigned int* ctr, float* slots, float2* stats,
+                            float* logits, cudaStream_t st) {
     TcHeadsArgs a;
     const uint64_t d = x.d, V = x.V, K = x.K, B = x.B;
     const int N = (x.B + 15) / 16 * 16;
@@ -481,6 +603,7 @@ cudaError_t heads_tc_launch(const HeadsArgs& x, void* hk, void* part, unsigned i
     a.logits = logits;
     a.part = (HeadState*)part;
     a.ctr = ctr;
+    a.slots = slots;
     a.tree = x.tree;
     a.root_token = x.root_token;
     a.topk_idx = x.topk_idx;
@@ -493,7 +616,7 @@ cudaError_t heads_tc_launch(const HeadsArgs& x, void* hk, void* part, unsigned i
     a.d = x.d;
     a.V = x.V;
     a.K = x.K;
-    cudaError_t e = cudaMemsetAsync(ctr, 0, 2 * sizeof(unsigned int), st);
+    cudaError_t e = cudaMemsetAsync(ctr, 0, (size_t)(2 + 2 * num_sms()) * sizeof(unsigned int), st);
     if (e != cudaSuccess) return e;
     switch (N) {
         case 16: return launch_n<16>(a, st);

@@ -34,8 +34,9 @@ size_t heads_workspace_size(int B, int d, int V, int K, medusa_dtype dt);
 cudaError_t heads_launch(const HeadsArgs& a, cudaStream_t st);
 // tensor-core path (bf16, 1 <= B <= 64, d % 8 == 0)
 bool heads_tc_supported(int B, int d, medusa_dtype dt);
-cudaError_t heads_tc_launch(const HeadsArgs& a, void* hk, void* part, unsigned int* ctr, float2* stats, float* logits,
-                            cudaStream_t st);
+// ctr: 2 + 2 * num_sms() counters (zeroed here); slots: 2 * num_sms() * B * 128 floats
+cudaError_t heads_tc_launch(const HeadsArgs& a, void* hk, void* part, unsigned int* ctr, float* slots, float2* stats,
+                            float* logits, cudaStream_t st);
 
 // ------------------------------ attention ----------------------------------
 struct AttnArgs {

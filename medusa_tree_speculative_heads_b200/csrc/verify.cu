@@ -224,7 +224,8 @@ __device__ unsigned long long cluster_sum(unsigned long long x, ClusterSum* sh, 
         cta += t;
     }
     if (tid == 0) sh->cta_tot = cta;
-    cl.sync();  // every CTA's total (and its earlier global writes) visible
+    __syncwarp();  // the cluster barrier is an aligned one: whole warps
+    cl.sync();     // every CTA's total (and its earlier global writes) visible
     const int rank = (int)cl.block_rank(), C = (int)cl.num_blocks();
     unsigned long long tot = 0, rbefore = 0;
     for (int r = 0; r < C; ++r) {
