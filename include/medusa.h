@@ -18,8 +18,8 @@
  *           sections "The Architectural Blueprint", "1. Combinatorial Tree
  *           Construction", "2. Single-Pass Tree Attention Verification".
  *   [MTP]   "Multi-Token Prediction & Draft-Model-Free Speculative Decoding",
- *           sections "The 2D Tree Attention Mask" and "Production Deployment
- *           Guidelines".
+ *           sections "2. EAGLE & EAGLE-2: Feature-Level Autoregression", "The
+ *           2D Tree Attention Mask" and "Production Deployment Guidelines".
  *
  * Conventions shared by every call
  *   - Every function returns MEDUSA_OK (0) or a negative MEDUSA_ERR_* code;
@@ -107,11 +107,34 @@ int medusa_version(void);
 typedef struct medusa_tree medusa_tree;
 int medusa_tree_create(const int32_t* parent_host, int T, medusa_tree** out);
 
+/*
+ * One tree per sequence ([MTP] "2. EAGLE & EAGLE-2: Feature-Level
+ * Autoregression": dynamic trees shaped per sequence; "Production
+ * Deployment Guidelines": tree depth tuned to the workload).  Tree i's parent
+ * array is parents_host[offsets_host[i] .. offsets_host[i+1]) (HOST arrays;
+ * offsets_host has ntrees + 1 entries, offsets_host[0] = 0), each obeying the
+ * rules above.  A handle with ntrees > 1 is used by calls with B = ntrees:
+ * sequence b uses tree b.  Such calls keep the [B, T, ...] layouts of the
+ * single-tree calls with T = the largest tree's node count (medusa_tree_info);
+ * sequence b uses the first T_b rows of its block.  Rows past T_b are
+ * ignored on input; on output node_tokens holds -1 and node_q 0 there, and
+ * tree_attention writes zeros (lse -inf).  q_row of tree_verify is then
+ * [B, T] (row b * T + u for node u of sequence b).
+ * Errors: as medusa_tree_create, naming the offending tree.
+ */
+int medusa_tree_create_ragged(const int32_t* parents_host, const int32_t* offsets_host, int ntrees,
+                              medusa_tree** out);
+
 /* Frees the handle (synchronises the device first).  NULL is a no-op. */
 int medusa_tree_destroy(medusa_tree* tree);
 
-/* Node count, maximum depth (root = 1) and the largest child count. */
+/* Node count, maximum depth (root = 1) and the largest child count; over all
+ * trees of the handle (T: the largest tree's node count). */
 int medusa_tree_info(const medusa_tree* tree, int* T, int* max_depth, int* max_children);
+
+/* Number of trees in the handle (1 for medusa_tree_create) and, if T_each is
+ * not NULL, each tree's node count (HOST array of ntrees int32). */
+int medusa_tree_ntrees(const medusa_tree* tree, int* ntrees, int32_t* T_each);
 
 /* ------------------------------------------------------------------------ */
 /* Medusa heads                                                              */
@@ -195,7 +218,8 @@ int medusa_heads_noalloc(const void* h, const void* W_res, const void* W_head, i
  * scale: softmax scale; <= 0 means 1/sqrt(D)
  * out      [B, T, Hq, D]       dtype dt
  * lse      [B, T, Hq] f32, nullable: natural-log sum of exp of the scaled scores
- * Limits: D in {64, 128}; Hq % Hkv == 0; T = tree node count (<= 128).
+ * Limits: D in {64, 128}; Hq % Hkv == 0; T = tree node count (<= 128; with
+ * one tree per sequence, the largest tree's).
  * A prefix_len outside [0, max_prefix] sets MEDUSA_STATUS_BAD_PREFIX and the
  * sequence's rows are computed over the clamped prefix.
  * Workspace: tree_attention_workspace_size(...) bytes.
@@ -237,8 +261,8 @@ int tree_attention(const void* q, const void* k_tree, const void* v_tree, const 
  * c's block, U = word1 of the block of the node where the walk ends.  All
  * arithmetic is integer or correctly rounded fp64, so results are exact.
  *   target: p [B, T, V] f32 (target_dt must be MEDUSA_F32);
- *   q [B, q_rows, V] f32; q_row [T] int32 device, nullable (identity, then
- *   q_rows must equal T).  Medusa heads' probs_out [B, K, V] serves as q with
+ *   q [B, q_rows, V] f32; q_row [T] int32 device ([B, T] with one tree per
+ *   sequence), nullable (identity, then q_rows must equal T).  Medusa heads' probs_out [B, K, V] serves as q with
  *   q_row[u] = depth(u) - 1.
  *
  * node_tokens [B, T] int32; accept_path [B, max_path] int32 out (node ids,

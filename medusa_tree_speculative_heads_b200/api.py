@@ -120,7 +120,7 @@ class MedusaStep:
     ``prefix_len`` to advance in place)."""
 
     def __init__(self, *, B: int, d: int, V: int, K: int, Hq: int, Hkv: int, D: int, S_max: int,
-                 parents: Sequence[int], dtype: torch.dtype, mode: int = _b.GREEDY, max_prefix: int = 0,
+                 parents, dtype: torch.dtype, mode: int = _b.GREEDY, max_prefix: int = 0,
                  q_rows: int = 0, device=None):
         dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
         self.B, self.d, self.V, self.K = B, d, V, K

@@ -61,6 +61,8 @@ def lib() -> ctypes.CDLL:
         L.medusa_tree_create.argtypes = [vp, i32, ctypes.POINTER(vp)]
         L.medusa_tree_destroy.argtypes = [vp]
         L.medusa_tree_info.argtypes = [vp, vp, vp, vp]
+        L.medusa_tree_create_ragged.argtypes = [vp, vp, i32, ctypes.POINTER(vp)]
+        L.medusa_tree_ntrees.argtypes = [vp, vp, vp]
         L.medusa_heads_workspace_size.argtypes = [i32, i32, i32, i32, i32]
         L.medusa_heads_workspace_size.restype = sz
         L.medusa_heads.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
@@ -118,17 +120,34 @@ def version() -> int:
 
 
 class Tree:
-    """Owner of a medusa_tree handle (created on the current device)."""
+    """Owner of a medusa_tree handle (created on the current device): one
+    parent list (a tree shared by every sequence) or a list of parent lists
+    (one tree per sequence, medusa_tree_create_ragged)."""
 
-    def __init__(self, parents: Sequence[int]):
-        arr = (ctypes.c_int32 * len(parents))(*[int(x) for x in parents])
+    def __init__(self, parents):
         h = ctypes.c_void_p()
-        _check(lib().medusa_tree_create(arr, len(parents), ctypes.byref(h)))
+        if len(parents) > 0 and hasattr(parents[0], "__len__"):
+            flat = [int(x) for p in parents for x in p]
+            offs = [0]
+            for p in parents:
+                offs.append(offs[-1] + len(p))
+            arr = (ctypes.c_int32 * max(len(flat), 1))(*flat)
+            off = (ctypes.c_int32 * len(offs))(*offs)
+            _check(lib().medusa_tree_create_ragged(arr, off, len(parents), ctypes.byref(h)))
+            self.parents = [[int(x) for x in p] for p in parents]
+        else:
+            arr = (ctypes.c_int32 * len(parents))(*[int(x) for x in parents])
+            _check(lib().medusa_tree_create(arr, len(parents), ctypes.byref(h)))
+            self.parents = [int(x) for x in parents]
         self.handle = h
-        self.parents = [int(x) for x in parents]
         T, dep, mc = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
         _check(lib().medusa_tree_info(h, ctypes.byref(T), ctypes.byref(dep), ctypes.byref(mc)))
         self.T, self.max_depth, self.max_children = T.value, dep.value, mc.value
+        n = ctypes.c_int()
+        _check(lib().medusa_tree_ntrees(h, ctypes.byref(n), None))
+        each = (ctypes.c_int32 * n.value)()
+        _check(lib().medusa_tree_ntrees(h, ctypes.byref(n), each))
+        self.ntrees, self.T_each = n.value, list(each)
 
     def close(self):
         if self.handle:

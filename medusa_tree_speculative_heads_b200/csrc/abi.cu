@@ -6,13 +6,20 @@
 #include <string.h>
 
 #include <string>
+#include <vector>
 
 #include "kernels.h"
 
+// One tree shared by every sequence, or one tree per sequence.  `host` holds
+// the union's extremes (T = the largest tree's node count, the deepest depth,
+// the most children); `trees` every tree as the kernels read it.
 struct medusa_tree {
     medusa::TreeDev host;
+    std::vector<medusa::TreeDev> trees;
     medusa::TreeDev* dev;
     int device;
+    int ntrees() const { return (int)trees.size(); }
+    medusa::TreeRef ref() const { return medusa::TreeRef{dev, ntrees() > 1 ? 1 : 0, host.T}; }
 };
 
 namespace medusa {
@@ -41,12 +48,79 @@ int cuda_fail(cudaError_t e, const char* what) {
     return fail(MEDUSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
 
-int check_tree(const medusa_tree* t) {
+int check_tree(const medusa_tree* t, int B) {
     if (!t) return fail(MEDUSA_ERR_INVALID_ARG, "tree is NULL");
     int dev = -1;
     cudaGetDevice(&dev);
     if (dev != t->device)
         return fail(MEDUSA_ERR_INVALID_ARG, "tree was created on device %d, current device is %d", t->device, dev);
+    if (t->ntrees() > 1 && t->ntrees() != B)
+        return fail(MEDUSA_ERR_INVALID_ARG, "the handle holds %d per-sequence trees, the call has B=%d sequences",
+                    t->ntrees(), B);
+    return MEDUSA_OK;
+}
+
+// Validates one parent array and fills its device description.
+int build_tree(const int32_t* parent, int T, TreeDev& h, const char* who) {
+    if (T < 1) return fail(MEDUSA_ERR_INVALID_ARG, "%s: T = %d < 1", who, T);
+    if (T > kMaxTree) return fail(MEDUSA_ERR_UNSUPPORTED, "%s: T = %d > %d", who, T, kMaxTree);
+    if (parent[0] != -1) return fail(MEDUSA_ERR_INVALID_ARG, "%s: node 0 must be the root (parent -1)", who);
+    for (int i = 1; i < T; ++i)
+        if (parent[i] < 0 || parent[i] >= i)
+            return fail(MEDUSA_ERR_INVALID_ARG,
+                        "%s: parent[%d] = %d; need 0 <= parent[i] < i (one root, topological order)", who, i,
+                        parent[i]);
+    memset(&h, 0, sizeof h);
+    h.T = T;
+    int cnt[kMaxTree] = {0};
+    h.parent[0] = -1;
+    h.depth[0] = 1;
+    h.anc[0][0] = 1u;
+    h.max_depth = 1;
+    for (int i = 1; i < T; ++i) {
+        const int p = parent[i];
+        h.parent[i] = (int16_t)p;
+        h.depth[i] = (uint8_t)(h.depth[p] + 1);
+        h.rank[i] = (uint8_t)cnt[p]++;
+        for (int w = 0; w < 4; ++w) h.anc[i][w] = h.anc[p][w];
+        h.anc[i][i >> 5] |= 1u << (i & 31);
+        if (h.depth[i] > h.max_depth) h.max_depth = h.depth[i];
+    }
+    int off = 0;
+    for (int u = 0; u < T; ++u) {
+        h.child_off[u] = (uint8_t)off;
+        off += cnt[u];
+        if (cnt[u] > h.max_children) h.max_children = cnt[u];
+    }
+    h.child_off[T] = (uint8_t)off;
+    int fill[kMaxTree] = {0};
+    for (int c = 1; c < T; ++c) {
+        const int p = parent[c];
+        h.child_idx[h.child_off[p] + fill[p]++] = (uint8_t)c;
+    }
+    return MEDUSA_OK;
+}
+
+// Uploads the trees of a new handle.
+int finish_tree(medusa_tree* t, medusa_tree** out, const char* who) {
+    TreeDev& x = t->host;
+    memset(&x, 0, sizeof x);
+    for (const TreeDev& h : t->trees) {
+        if (h.T > x.T) x.T = h.T;
+        if (h.max_depth > x.max_depth) x.max_depth = h.max_depth;
+        if (h.max_children > x.max_children) x.max_children = h.max_children;
+    }
+    cudaGetDevice(&t->device);
+    t->dev = nullptr;
+    const size_t bytes = sizeof(TreeDev) * t->trees.size();
+    cudaError_t e = cudaMalloc((void**)&t->dev, bytes);
+    if (e == cudaSuccess) e = cudaMemcpy(t->dev, t->trees.data(), bytes, cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) {
+        if (t->dev) cudaFree(t->dev);
+        delete t;
+        return cuda_fail(e, who);
+    }
+    *out = t;
     return MEDUSA_OK;
 }
 }  // namespace
@@ -83,54 +157,35 @@ extern "C" int medusa_version(void) { return 100; }
 
 extern "C" int medusa_tree_create(const int32_t* parent, int T, medusa_tree** out) {
     if (!parent || !out) return fail(MEDUSA_ERR_INVALID_ARG, "medusa_tree_create: NULL argument");
-    if (T < 1) return fail(MEDUSA_ERR_INVALID_ARG, "medusa_tree_create: T = %d < 1", T);
-    if (T > kMaxTree) return fail(MEDUSA_ERR_UNSUPPORTED, "medusa_tree_create: T = %d > %d", T, kMaxTree);
-    if (parent[0] != -1) return fail(MEDUSA_ERR_INVALID_ARG, "medusa_tree_create: node 0 must be the root (parent -1)");
-    for (int i = 1; i < T; ++i)
-        if (parent[i] < 0 || parent[i] >= i)
-            return fail(MEDUSA_ERR_INVALID_ARG,
-                        "medusa_tree_create: parent[%d] = %d; need 0 <= parent[i] < i (one root, topological order)",
-                        i, parent[i]);
     medusa_tree* t = new medusa_tree();
-    TreeDev& h = t->host;
-    memset(&h, 0, sizeof h);
-    h.T = T;
-    int cnt[kMaxTree] = {0};
-    h.parent[0] = -1;
-    h.depth[0] = 1;
-    h.anc[0][0] = 1u;
-    h.max_depth = 1;
-    for (int i = 1; i < T; ++i) {
-        const int p = parent[i];
-        h.parent[i] = (int16_t)p;
-        h.depth[i] = (uint8_t)(h.depth[p] + 1);
-        h.rank[i] = (uint8_t)cnt[p]++;
-        for (int w = 0; w < 4; ++w) h.anc[i][w] = h.anc[p][w];
-        h.anc[i][i >> 5] |= 1u << (i & 31);
-        if (h.depth[i] > h.max_depth) h.max_depth = h.depth[i];
-    }
-    int off = 0;
-    for (int u = 0; u < T; ++u) {
-        h.child_off[u] = (uint8_t)off;
-        off += cnt[u];
-        if (cnt[u] > h.max_children) h.max_children = cnt[u];
-    }
-    h.child_off[T] = (uint8_t)off;
-    int fill[kMaxTree] = {0};
-    for (int c = 1; c < T; ++c) {
-        const int p = parent[c];
-        h.child_idx[h.child_off[p] + fill[p]++] = (uint8_t)c;
-    }
-    cudaGetDevice(&t->device);
-    cudaError_t e = cudaMalloc((void**)&t->dev, sizeof(TreeDev));
-    if (e == cudaSuccess) e = cudaMemcpy(t->dev, &h, sizeof(TreeDev), cudaMemcpyHostToDevice);
-    if (e != cudaSuccess) {
-        if (t->dev) cudaFree(t->dev);
+    t->trees.resize(1);
+    int rc = build_tree(parent, T, t->trees[0], "medusa_tree_create");
+    if (rc) {
         delete t;
-        return cuda_fail(e, "medusa_tree_create");
+        return rc;
     }
-    *out = t;
-    return ok();
+    rc = finish_tree(t, out, "medusa_tree_create");
+    return rc ? rc : ok();
+}
+
+extern "C" int medusa_tree_create_ragged(const int32_t* parents, const int32_t* offsets, int ntrees,
+                                         medusa_tree** out) {
+    if (!parents || !offsets || !out) return fail(MEDUSA_ERR_INVALID_ARG, "medusa_tree_create_ragged: NULL argument");
+    if (ntrees < 1) return fail(MEDUSA_ERR_INVALID_ARG, "medusa_tree_create_ragged: ntrees = %d < 1", ntrees);
+    if (offsets[0] != 0) return fail(MEDUSA_ERR_INVALID_ARG, "medusa_tree_create_ragged: offsets[0] must be 0");
+    medusa_tree* t = new medusa_tree();
+    t->trees.resize(ntrees);
+    for (int i = 0; i < ntrees; ++i) {
+        char who[64];
+        snprintf(who, sizeof who, "medusa_tree_create_ragged (tree %d)", i);
+        const int rc = build_tree(parents + offsets[i], offsets[i + 1] - offsets[i], t->trees[i], who);
+        if (rc) {
+            delete t;
+            return rc;
+        }
+    }
+    const int rc = finish_tree(t, out, "medusa_tree_create_ragged");
+    return rc ? rc : ok();
 }
 
 extern "C" int medusa_tree_destroy(medusa_tree* t) {
@@ -147,6 +202,14 @@ extern "C" int medusa_tree_info(const medusa_tree* t, int* T, int* max_depth, in
     if (T) *T = t->host.T;
     if (max_depth) *max_depth = t->host.max_depth;
     if (max_children) *max_children = t->host.max_children;
+    return ok();
+}
+
+extern "C" int medusa_tree_ntrees(const medusa_tree* t, int* ntrees, int32_t* T_each) {
+    if (!t || !ntrees) return fail(MEDUSA_ERR_INVALID_ARG, "medusa_tree_ntrees: NULL argument");
+    *ntrees = t->ntrees();
+    if (T_each)
+        for (int i = 0; i < t->ntrees(); ++i) T_each[i] = t->trees[i].T;
     return ok();
 }
 
@@ -178,20 +241,22 @@ extern "C" int medusa_heads(const void* h, const void* W_res, const void* W_head
                     workspace_bytes, heads_workspace_size(B, d, V, K, dt));
     int T = 0;
     if (tree) {
-        int rc = check_tree(tree);
+        int rc = check_tree(tree, B);
         if (rc) return rc;
         if (!node_tokens || !root_token)
             return fail(MEDUSA_ERR_INVALID_ARG, "medusa_heads: a tree needs root_token and node_tokens");
-        const TreeDev& th = tree->host;
-        if (th.max_depth > K + 1)
+        if (tree->host.max_depth > K + 1)
             return fail(MEDUSA_ERR_INVALID_ARG, "medusa_heads: tree depth %d needs more than K=%d heads",
-                        th.max_depth, K);
+                        tree->host.max_depth, K);
         const int smax = V < kTopK ? V : kTopK;
-        for (int i = 1; i < th.T; ++i)
-            if (th.rank[i] >= smax)
-                return fail(MEDUSA_ERR_UNSUPPORTED, "medusa_heads: node %d has sibling rank %d >= %d", i, th.rank[i],
-                            smax);
-        T = th.T;
+        for (int n = 0; n < tree->ntrees(); ++n) {
+            const TreeDev& th = tree->trees[n];
+            for (int i = 1; i < th.T; ++i)
+                if (th.rank[i] >= smax)
+                    return fail(MEDUSA_ERR_UNSUPPORTED, "medusa_heads: node %d of tree %d has sibling rank %d >= %d", i,
+                                n, th.rank[i], smax);
+        }
+        T = tree->host.T;
     }
     HeadsArgs a;
     a.h = h;
@@ -202,7 +267,7 @@ extern "C" int medusa_heads(const void* h, const void* W_res, const void* W_head
     a.V = V;
     a.K = K;
     a.dt = dt;
-    a.tree = tree ? tree->dev : nullptr;
+    a.tree = tree ? tree->ref() : TreeRef{nullptr, 0, 0};
     a.T = T;
     a.root_token = root_token;
     a.topk_idx = topk_idx;
@@ -239,7 +304,7 @@ extern "C" int tree_attention(const void* q, const void* k_tree, const void* v_t
     if (dt != MEDUSA_F32 && dt != MEDUSA_BF16) return fail(MEDUSA_ERR_UNSUPPORTED, "tree_attention: unknown dtype");
     if (!q || !k_tree || !v_tree || !k_cache || !v_cache || !prefix_len || !out)
         return fail(MEDUSA_ERR_INVALID_ARG, "tree_attention: NULL tensor argument");
-    int rc = check_tree(tree);
+    int rc = check_tree(tree, B);
     if (rc) return rc;
     if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || S_max < 0)
         return fail(MEDUSA_ERR_INVALID_ARG, "tree_attention: bad sizes B=%d Hq=%d Hkv=%d S_max=%d", B, Hq, Hkv, S_max);
@@ -269,7 +334,7 @@ extern "C" int tree_attention(const void* q, const void* k_tree, const void* v_t
     a.max_prefix = max_prefix;
     a.scale = scale;
     a.dt = dt;
-    a.tree = tree->dev;
+    a.tree = tree->ref();
     a.out = out;
     a.lse = lse;
     a.ws = workspace;
@@ -298,7 +363,7 @@ extern "C" int tree_verify(medusa_verify_mode mode, const void* target, medusa_d
         return fail(MEDUSA_ERR_INVALID_ARG, "tree_verify: unknown mode");
     if (!target || !node_tokens || !accept_path || !accept_len || !bonus)
         return fail(MEDUSA_ERR_INVALID_ARG, "tree_verify: NULL tensor argument");
-    int rc = check_tree(tree);
+    int rc = check_tree(tree, B);
     if (rc) return rc;
     const int T = tree->host.T;
     if (B < 1 || V < 1) return fail(MEDUSA_ERR_INVALID_ARG, "tree_verify: bad sizes B=%d V=%d", B, V);
@@ -329,7 +394,7 @@ extern "C" int tree_verify(medusa_verify_mode mode, const void* target, medusa_d
     a.B = B;
     a.V = V;
     a.T = T;
-    a.tree = tree->dev;
+    a.tree = tree->ref();
     a.seed = seed;
     a.step = step;
     a.accept_path = accept_path;

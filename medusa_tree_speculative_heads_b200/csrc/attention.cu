@@ -38,10 +38,10 @@ struct AttnParams {
     const int32_t* prefix_len;
     int B, T, Hq, Hkv, G, S_max, max_prefix;
     float scale_log2;
-    int R;          // query rows per (sequence, kv-head) = T * G
+    int R;          // query-row stride per (sequence, kv-head) = T * G (T: the largest tree)
     int n_splits;   // prefix splits + 1 (tree split last)
     int split_len;  // prefix keys per split, a multiple of kBN
-    const TreeDev* tree;
+    TreeRef tree;
     float* part_o;    // [n_splits][B*Hkv][R][D], normalised
     float* part_lse;  // [n_splits][B*Hkv][R], log2 units
     int32_t* status;
@@ -103,6 +103,8 @@ __global__ void __launch_bounds__(kThreads) tree_attn_mma_kernel(const __grid_co
     const int b = bg / p.Hkv, g = bg % p.Hkv;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool tree_split = split == p.n_splits - 1;
+    const TreeDev* tree = p.tree.at(b);
+    const int Rb = tree->T * p.G;  // this sequence's query rows
 
     int S = p.prefix_len[b];
     if (S < 0 || S > p.max_prefix) {
@@ -112,7 +114,7 @@ __global__ void __launch_bounds__(kThreads) tree_attn_mma_kernel(const __grid_co
     int k_begin, k_end;
     if (tree_split) {
         k_begin = 0;
-        k_end = p.T;
+        k_end = tree->T;
     } else {
         k_begin = split * p.split_len;
         k_end = min(S, k_begin + p.split_len);
@@ -124,7 +126,7 @@ __global__ void __launch_bounds__(kThreads) tree_attn_mma_kernel(const __grid_co
     for (int c = tid; c < kBM * CH; c += kThreads) {
         const int row = c / CH, ch = c % CH;
         const int r = mt * kBM + row;
-        const bool valid = r < p.R;
+        const bool valid = r < Rb;
         const int node = valid ? r / p.G : 0, hh = valid ? r % p.G : 0;
         const __nv_bfloat16* src = p.q + (((long)b * p.T + node) * p.Hq + g * p.G + hh) * D + ch * 8;
         cp_async16(smem_u32(sQ) + swz<D>(row, ch), src, valid);
@@ -133,7 +135,7 @@ __global__ void __launch_bounds__(kThreads) tree_attn_mma_kernel(const __grid_co
         for (int t = tid; t < kBM * 4; t += kThreads) {
             const int row = t >> 2, w = t & 3;
             const int r = mt * kBM + row;
-            sAnc[t] = r < p.R ? p.tree->anc[r / p.G][w] : 0u;
+            sAnc[t] = r < Rb ? tree->anc[r / p.G][w] : 0u;
         }
     }
     auto load_chunk = [&](int chunk, int buf) {
@@ -278,7 +280,7 @@ __global__ void __launch_bounds__(kThreads) tree_attn_mma_kernel(const __grid_co
 #pragma unroll
     for (int h2 = 0; h2 < 2; ++h2) {
         const int r = mt * kBM + warp * 16 + (lane >> 2) + h2 * 8;
-        if (r >= p.R) continue;
+        if (r >= Rb) continue;
         const float inv = l_r[h2] > 0.f ? 1.f / l_r[h2] : 0.f;
         float* dst = p.part_o + (((long)split * BH + bg) * p.R + r) * D;
 #pragma unroll
@@ -297,8 +299,8 @@ __global__ void __launch_bounds__(kThreads) tree_attn_mma_kernel(const __grid_co
 template <int D>
 __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restrict__ part_o,
                                                            const float* __restrict__ part_lse, int B, int T, int Hq,
-                                                           int Hkv, int n_splits, __nv_bfloat16* __restrict__ out,
-                                                           float* __restrict__ lse) {
+                                                           int Hkv, int n_splits, TreeRef tree,
+                                                           __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
     const long row = (long)blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= (long)B * T * Hq) return;
@@ -307,6 +309,13 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restri
     const int b = (int)(row / ((long)Hq * T));
     const int G = Hq / Hkv, g = h / G, hh = h % G;
     const int R = T * G, r = i * G + hh;
+    if (i >= tree.at(b)->T) {  // past this sequence's tree: no partials, zero output
+        __nv_bfloat16* dst = out + row * D + lane * (D / 32);
+#pragma unroll
+        for (int e = 0; e < D / 32; ++e) dst[e] = __float2bfloat16_rn(0.f);
+        if (lse && lane == 0) lse[row] = -INFINITY;
+        return;
+    }
     const long BH = (long)B * Hkv, bg = (long)b * Hkv + g;
     constexpr int PL = D / 32;
     float acc[PL];
@@ -363,7 +372,7 @@ __global__ void __launch_bounds__(256) tree_attn_f32_kernel(const float* __restr
                                                             const float* __restrict__ v_cache,
                                                             const int32_t* __restrict__ prefix_len, int B, int T,
                                                             int Hq, int Hkv, int S_max, int max_prefix, float scale,
-                                                            const TreeDev* __restrict__ tree, float* __restrict__ out,
+                                                            TreeRef trees, float* __restrict__ out,
                                                             float* __restrict__ lse, int32_t* status) {
     constexpr int PL = D / 32;
     const long row = (long)blockIdx.x * 8 + (threadIdx.x >> 5);
@@ -373,6 +382,13 @@ __global__ void __launch_bounds__(256) tree_attn_f32_kernel(const float* __restr
     const int i = (int)((row / Hq) % T);
     const int b = (int)(row / ((long)Hq * T));
     const int g = h / (Hq / Hkv);
+    const TreeDev* tree = trees.at(b);
+    if (i >= tree->T) {  // past this sequence's tree: zero output
+#pragma unroll
+        for (int e = 0; e < PL; ++e) out[row * D + lane * PL + e] = 0.f;
+        if (lse && lane == 0) lse[row] = -INFINITY;
+        return;
+    }
     int S = prefix_len[b];
     if (S < 0 || S > max_prefix) {
         if (lane == 0 && i == 0 && h == 0) set_status(status, MEDUSA_STATUS_BAD_PREFIX);
@@ -400,7 +416,7 @@ __global__ void __launch_bounds__(256) tree_attn_f32_kernel(const float* __restr
     };
     const long cbase = ((long)b * Hkv + g) * S_max;
     for (int j = 0; j < S; ++j) visit(k_cache + (cbase + j) * D, v_cache + (cbase + j) * D);
-    for (int j = 0; j < T; ++j)
+    for (int j = 0; j < tree->T; ++j)
         if ((tree->anc[i][j >> 5] >> (j & 31)) & 1u)
             visit(k_tree + (((long)b * T + j) * Hkv + g) * D, v_tree + (((long)b * T + j) * Hkv + g) * D);
 #pragma unroll
@@ -483,7 +499,7 @@ cudaError_t attn_launch_bf16(const AttnArgs& a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     const long rows = (long)a.B * a.T * a.Hq;
     attn_combine_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(p.part_o, p.part_lse, a.B, a.T, a.Hq, a.Hkv,
-                                                                     sp.n_splits, (__nv_bfloat16*)a.out, a.lse);
+                                                                     sp.n_splits, a.tree, (__nv_bfloat16*)a.out, a.lse);
     return cudaGetLastError();
 }
 

@@ -58,7 +58,7 @@ struct TcAttnArgs {
     CUtensorMap mkt;   // k_tree as (D, Hkv, B*T), box (64, 1, 64)
     CUtensorMap mvt;
     const int32_t* prefix_len;
-    const TreeDev* tree;
+    TreeRef tree;
     float* part_o;     // [n_splits][B*Hkv][R][D]
     float* part_lse;   // [n_splits][B*Hkv][R], log2 units
     int32_t* status;
@@ -123,6 +123,8 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
     const int b = bg / a.Hkv, g = bg % a.Hkv;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const bool tree_split = split == a.n_splits - 1;
+    const TreeDev* tree = a.tree.at(b);
+    const int Tb = tree->T;  // this sequence's tree (a.T: the row stride of q and the tree K/V)
     if (smem_addr(smem) & 1023u) {  // never expected; refuse rather than misread swizzled tiles
         if (threadIdx.x == 0) set_status(a.status, MEDUSA_STATUS_TIMEOUT);
         return;
@@ -137,8 +139,8 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
     int k_begin, k_end, nc;
     if (tree_split) {
         k_begin = 0;
-        k_end = a.T;
-        nc = (a.T + kCh - 1) / kCh;
+        k_end = Tb;
+        nc = (Tb + kCh - 1) / kCh;
     } else {
         k_begin = split * a.split_len;
         k_end = min(S, k_begin + a.split_len);
@@ -282,12 +284,12 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
         const int q = warp & 3;
         const int lr = q * 32 + lane;
         const int r = mt * kAM + lr;
-        const bool row_ok = r < a.R;
+        const bool row_ok = r < Tb * a.G;
         const int node = row_ok ? r / a.G : 0;
         uint32_t anc[4] = {0u, 0u, 0u, 0u};
         if (tree_split && row_ok)
 #pragma unroll
-            for (int w = 0; w < 4; ++w) anc[w] = a.tree->anc[node][w];
+            for (int w = 0; w < 4; ++w) anc[w] = tree->anc[node][w];
         float m = -INFINITY, l = 0.f;
         bool ok = true;
         const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
@@ -384,6 +386,25 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
                 tmem_wait_st();
             }
             m = mn;
+            if (tree_split && key0 + kCh > Tb) {
+                // the chunk's rows past this sequence's tree are not its keys
+                // (padding, or another sequence's): P is 0 there, but a NaN in
+                // V would still reach O (0 * NaN), so those V rows are cleared
+                // before the PV product may start
+                const int s = j % VS;
+                if (!mbar_wait(&v_full[s], (j / VS) & 1)) {
+                    ok = false;
+                    break;
+                }
+                const int r0 = Tb - key0, lt = (warp - 2) * 32 + lane;
+                uint8_t* vs = sV + s * kKVBytes;
+                for (int idx = lt; idx < (kCh - r0) * NSUB * 8; idx += 128) {
+                    const int row = r0 + idx / (NSUB * 8), rem = idx % (NSUB * 8);
+                    *reinterpret_cast<uint4*>(vs + (rem >> 3) * kSub + row * 128 + (rem & 7) * 16) =
+                        make_uint4(0u, 0u, 0u, 0u);
+                }
+                fence_proxy_async_shared();
+            }
             tmem_wait_st();  // P (and any rescaled O) in TMEM before the MMA reads it
             tc_fence_before();
             __syncwarp();

@@ -30,6 +30,17 @@ struct TreeDev {
     uint32_t anc[kMaxTree][4];
 };
 
+// The tree(s) of a call: one tree shared by every sequence (stride 0) or one
+// per sequence (stride 1).  T is the node dimension of the [B, T, ...] arrays
+// of the call (the largest tree's node count); sequence b uses its own
+// tree's first at(b)->T rows of them.
+struct TreeRef {
+    const TreeDev* base;
+    int stride;
+    int T;
+    __host__ __device__ const TreeDev* at(int b) const { return base + (long)b * stride; }
+};
+
 // ---------------------------------------------------------------------------
 // small helpers
 // ---------------------------------------------------------------------------

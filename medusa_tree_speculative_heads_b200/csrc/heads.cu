@@ -319,7 +319,7 @@ struct FusedArgs {
     float* logits;
     HeadState* part;     // [grid][K][kBG]
     unsigned int* ctr;   // [2], zero at launch: grid-barrier arrivals, CTAs done
-    const TreeDev* tree;
+    TreeRef tree;
     const int32_t* root_token;
     int32_t* topk_idx;
     float* topk_prob;
@@ -603,13 +603,14 @@ __global__ void __launch_bounds__((kFC + 1) * 32, 1) heads_fused_kernel(const __
     if (!s_flag) return;
     __threadfence();
     for (int k = warp; k < a.K; k += kFC + 1)
-        merge_head(a.part, gridDim.x, a.V, 1, kBG, 0, 0, a.V, a.K, k, a.tree, a.root_token, a.topk_idx, a.topk_prob,
+        merge_head(a.part, gridDim.x, a.V, 1, kBG, 0, 0, a.V, a.K, k, a.tree.base ? a.tree.at(0) : nullptr, a.tree.T,
+                   a.root_token, a.topk_idx, a.topk_prob,
                    a.node_tokens, a.node_q, a.stats, a.status);
 }
 
 // K3 of the general path: one warp per (sequence, head).
 __global__ void __launch_bounds__(32) heads_merge_kernel(const HeadState* __restrict__ part, int nparts, int b0,
-                                                         int nb, int V, int K, const TreeDev* __restrict__ tree,
+                                                         int nb, int V, int K, TreeRef tree,
                                                          const int32_t* __restrict__ root_token,
                                                          int32_t* __restrict__ topk_idx,
                                                          float* __restrict__ topk_prob,
@@ -617,7 +618,8 @@ __global__ void __launch_bounds__(32) heads_merge_kernel(const HeadState* __rest
                                                          float* __restrict__ node_q, float2* __restrict__ stats,
                                                          int32_t* status) {
     const int bb = blockIdx.x % nb, k = blockIdx.x / nb;
-    merge_head(part, nparts, V, 1, kBG, bb, b0 + bb, V, K, k, tree, root_token, topk_idx, topk_prob, node_tokens, node_q,
+    merge_head(part, nparts, V, 1, kBG, bb, b0 + bb, V, K, k, tree.base ? tree.at(b0 + bb) : nullptr, tree.T,
+               root_token, topk_idx, topk_prob, node_tokens, node_q,
                stats, status);
 }
 

@@ -104,15 +104,18 @@ __device__ __forceinline__ void warp_select(float (&lv)[kTopK], int (&li)[kTopK]
 // merge.  The K*uph tiles (head k owning tiles [k*uph, (k+1)*uph)) are cut
 // into upt units each; the CTAs split the K*uph*upt units evenly and CTA c
 // owns the tiles whose first unit falls in its share; partial (c, k, b) sits
-// at part[(c*K + k)*bstride + b].  Writes the top-8 entries with their probabilities, the head's
-// softmax statistics, and fills the tree nodes this head proposes.  One warp.
+// at part[(c*K + k)*bstride + b].  Writes the top-8 entries with their
+// probabilities, the head's softmax statistics, and fills the nodes of
+// sequence b's tree that this head proposes (node_tokens and node_q have Tn
+// nodes per sequence; head 0 also writes the root and sets the rows past
+// that tree to -1 and 0).  One warp.
 // Partials are read through L2 (they may have been written by other CTAs of
 // the same kernel).
 // ---------------------------------------------------------------------------
 static __device__ __noinline__ void merge_head(const HeadState* __restrict__ part, int nparts, long uph, int upt,
                                                int bstride, int bb,
                                        int b, int V, int K, int k,
-                           const TreeDev* __restrict__ tree, const int32_t* __restrict__ root_token,
+                           const TreeDev* __restrict__ tree, int Tn, const int32_t* __restrict__ root_token,
                            int32_t* __restrict__ topk_idx, float* __restrict__ topk_prob,
                            int32_t* __restrict__ node_tokens, float* __restrict__ node_q, float2* __restrict__ stats,
                            int32_t* status) {
@@ -201,14 +204,18 @@ static __device__ __noinline__ void merge_head(const HeadState* __restrict__ par
             const int tok = __shfl_sync(kFull, valid ? oi : -1, rk[j] & (kTopK - 1));
             const float pq = __shfl_sync(kFull, prob, rk[j] & (kTopK - 1));
             if (i < T && i > 0 && dp[j] == k + 2) {
-                node_tokens[(long)b * T + i] = tok;
-                if (node_q) node_q[(long)b * T + i] = pq;
+                node_tokens[(long)b * Tn + i] = tok;
+                if (node_q) node_q[(long)b * Tn + i] = pq;
                 if (tok < 0) set_status(status, MEDUSA_STATUS_BAD_TOKEN);
+            }
+            if (k == 0 && i >= T && i < Tn) {  // rows past this sequence's own tree
+                node_tokens[(long)b * Tn + i] = -1;
+                if (node_q) node_q[(long)b * Tn + i] = 0.f;
             }
         }
         if (k == 0 && lane == 0) {
-            node_tokens[(long)b * T] = rt;
-            if (node_q) node_q[(long)b * T] = 1.f;
+            node_tokens[(long)b * Tn] = rt;
+            if (node_q) node_q[(long)b * Tn] = 1.f;
             if (rt < 0 || rt >= V) set_status(status, MEDUSA_STATUS_BAD_TOKEN);
         }
     }

@@ -70,7 +70,7 @@ struct TcHeadsArgs {
     HeadState* part;        // [grid][K][B]
     float* slots;           // [2 phases][grid][B][128] handed-over partial tiles
     unsigned int* ctr;      // [2 + 2 * grid], zero at launch: grid-barrier arrivals, then the slots' flags
-    const TreeDev* tree;
+    TreeRef tree;
     const int32_t* root_token;
     int32_t* topk_idx;
     float* topk_prob;
@@ -529,7 +529,8 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
     __threadfence();
     for (int p = blockIdx.x * kTcWarps + warp; p < B * K; p += gridDim.x * kTcWarps) {
         const int b = p % B, k = p / B;
-        merge_head(a.part, gridDim.x, tph_l, nkb, B, b, b, a.V, K, k, a.tree, a.root_token, a.topk_idx, a.topk_prob,
+        merge_head(a.part, gridDim.x, tph_l, nkb, B, b, b, a.V, K, k, a.tree.base ? a.tree.at(b) : nullptr, a.tree.T,
+                   a.root_token, a.topk_idx, a.topk_prob,
                    a.node_tokens, a.node_q, a.stats, a.status);
     }
 }

@@ -16,7 +16,7 @@ struct HeadsArgs {
     const void* W_head;
     int B, d, V, K;
     medusa_dtype dt;
-    const TreeDev* tree;  // device, nullable
+    TreeRef tree;  // base NULL: no tree
     int T;
     const int32_t* root_token;
     int32_t* topk_idx;
@@ -49,7 +49,7 @@ struct AttnArgs {
     int B, T, Hq, Hkv, D, S_max, max_prefix;
     float scale;
     medusa_dtype dt;
-    const TreeDev* tree;
+    TreeRef tree;  // T is tree.T
     void* out;
     float* lse;
     void* ws;
@@ -74,7 +74,7 @@ struct VerifyArgs {
     const int32_t* q_row;
     const int32_t* node_tokens;
     int B, V, T;
-    const TreeDev* tree;
+    TreeRef tree;
     uint64_t seed;
     uint32_t step;
     int32_t* accept_path;

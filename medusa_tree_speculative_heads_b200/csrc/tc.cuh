@@ -138,6 +138,12 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)map) : "memory");
 }
 
+// make this thread's generic-proxy shared-memory writes visible to later
+// async-proxy reads (TMA, tcgen05.mma operands)
+__device__ __forceinline__ void fence_proxy_async_shared() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // order this thread's generic-proxy global accesses with later async-proxy
 // (TMA) accesses, and vice versa
 __device__ __forceinline__ void fence_proxy_async_global() {

@@ -118,19 +118,19 @@ constexpr int kMaxSplits = 16;
 __global__ void __launch_bounds__(kWalkThreads) greedy_walk_kernel(const float* __restrict__ pval,
                                                                    const int* __restrict__ pidx, int splits,
                                                                    const int32_t* __restrict__ node_tokens,
-                                                                   const TreeDev* __restrict__ tree,
-                                                                   int32_t* accept_path, int max_path,
+                                                                   TreeRef trees, int32_t* accept_path, int max_path,
                                                                    int32_t* accept_len, int32_t* bonus) {
     __shared__ int pred[kMaxTree];
     __shared__ uint32_t match[kMaxTree / 32];
     __shared__ int best_key[kMaxTree / 32];
     const int b = blockIdx.x, u = threadIdx.x, lane = u & 31, w = u >> 5;
-    const int T = tree->T;
+    const TreeDev* tree = trees.at(b);
+    const int T = tree->T, Tn = trees.T;  // this sequence's nodes; node stride of the arrays
     float bv = -INFINITY;
     int bi = INT_MAX;
     int tok = 0, par = -1, dep = 0;
     if (u < T) {
-        const long base = ((long)b * T + u) * splits;
+        const long base = ((long)b * Tn + u) * splits;
         float lv[kMaxSplits];
         int li[kMaxSplits];
 #pragma unroll
@@ -138,7 +138,7 @@ __global__ void __launch_bounds__(kWalkThreads) greedy_walk_kernel(const float* 
             lv[s] = s < splits ? pval[base + s] : -INFINITY;
             li[s] = s < splits ? pidx[base + s] : INT_MAX;
         }
-        tok = node_tokens[(long)b * T + u];
+        tok = node_tokens[(long)b * Tn + u];
         par = tree->parent[u];
         dep = tree->depth[u];
 #pragma unroll
@@ -240,7 +240,7 @@ __device__ unsigned long long cluster_sum(unsigned long long x, ClusterSum* sh, 
 
 __global__ void __launch_bounds__(kStochThreads, 2) verify_stochastic_kernel(
     const float* __restrict__ p, const float* __restrict__ q, int q_rows, const int32_t* __restrict__ q_row,
-    const int32_t* __restrict__ node_tokens, int V, const TreeDev* __restrict__ tree, uint32_t key0, uint32_t key1,
+    const int32_t* __restrict__ node_tokens, int V, TreeRef trees, uint32_t key0, uint32_t key1,
     uint32_t step, int32_t* accept_path, int max_path, int32_t* accept_len, int32_t* bonus,
     unsigned long long* ws_w, int32_t* status) {
     namespace cg = cooperative_groups;
@@ -249,7 +249,8 @@ __global__ void __launch_bounds__(kStochThreads, 2) verify_stochastic_kernel(
     const int C = (int)cl.num_blocks(), rank = (int)cl.block_rank();
     const int b = blockIdx.x / C, tid = threadIdx.x;
     const bool lead = rank == 0 && tid == 0;
-    const int T = tree->T;
+    const TreeDev* tree = trees.at(b);
+    const int T = trees.T;  // node stride of p, node_tokens (and of q_row with one tree per sequence)
     const float* Pb = p + (long)b * T * V;
     // Two weight buffers.  `valid` holds the last effective residual (S > 0)
     // of the current node, -1 while P is still p[b,u,:].  `keep` is the
@@ -287,7 +288,7 @@ __global__ void __launch_bounds__(kStochThreads, 2) verify_stochastic_kernel(
         valid = -1;
         Prow = Pb + (long)u * V;
         if (c_begin == c_end) break;  // a leaf: no drafted children
-        const int qr = q_row ? q_row[u] : u;
+        const int qr = q_row ? q_row[(trees.stride ? (long)b * T : 0) + u] : u;
         if (qr < 0 || qr >= q_rows) {
             if (lead) set_status(status, MEDUSA_STATUS_BAD_TOKEN);
             break;

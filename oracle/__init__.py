@@ -58,7 +58,7 @@ def lib():
         L.orc_philox4x32_10.argtypes = [vp, vp, vp]
         L.orc_philox4x32_10.restype = None
         L.orc_verify_stochastic.argtypes = [vp, vp, i32, vp, vp, i32, i32, i32, vp, u64, u32, i32, vp, vp, vp,
-                                            vp]
+                                            vp, i32]
         L.orc_kv_commit.argtypes = [vp, vp, vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]
         L.orc_kv_commit.restype = None
         L.orc_residual.argtypes = [vp, vp, i32, vp, vp]
@@ -247,7 +247,9 @@ def residual(P, Q):
     return out, W, int(S)
 
 
-def verify_stochastic(p, q, node_tokens, parents, seed: int, step: int, max_path: int, q_row=None):
+def verify_stochastic(p, q, node_tokens, parents, seed: int, step: int, max_path: int, q_row=None, b0: int = 0):
+    """Rows of p, q, node_tokens are sequences b0, b0+1, ... of the batch (the
+    sequence index selects the Philox counter)."""
     pa = _f32(p)
     qa = _f32(q)
     B, T, V = pa.shape
@@ -261,7 +263,7 @@ def verify_stochastic(p, q, node_tokens, parents, seed: int, step: int, max_path
     status = np.zeros(1, np.int32)
     rc = lib().orc_verify_stochastic(_p(pa), _p(qa), Qrows, _p(qr), _p(nt), B, T, V, _p(par),
                                      ctypes.c_uint64(seed & (2**64 - 1)), ctypes.c_uint32(step & 0xFFFFFFFF),
-                                     max_path, _p(path), _p(ln), _p(bonus), _p(status))
+                                     max_path, _p(path), _p(ln), _p(bonus), _p(status), int(b0))
     if rc != 0:
         raise ValueError("bad verify arguments")
     return path, ln, bonus, int(status[0])

@@ -483,13 +483,15 @@ uint64_t orc_residual(const double* P, const float* Q, int V, double* out, uint6
  * Uniforms: Philox4x32-10 block of (b, node, step); u_c = (word0 >> 8) * 2^-24
  * of child c's block, U = word1 of the block of the node where the walk ends.
  * p, q are fp32 [B,T,V] and [B,Qrows,V]; q_row NULL means q_row[u] = u.
+ * Row b of the arrays is sequence b0 + b of the batch: its uniforms use the
+ * counter of sequence b0 + b (so one sequence can be checked on its own).
  * Outputs as for orc_verify_greedy; status bit 1 is set when a bonus
  * distribution has zero total weight (bonus 0 then).
  */
 int orc_verify_stochastic(const float* p, const float* q, int Qrows, const int32_t* q_row,
                           const int32_t* node_tokens, int B, int T, int V, const int32_t* parent,
                           uint64_t seed, uint32_t step, int max_path, int32_t* path, int32_t* len,
-                          int32_t* bonus, int32_t* status) {
+                          int32_t* bonus, int32_t* status, int b0) {
     int32_t* depth = (int32_t*)malloc(sizeof(int32_t) * T);
     int32_t* rank = (int32_t*)malloc(sizeof(int32_t) * T);
     double* P = (double*)malloc(sizeof(double) * (size_t)V);
@@ -518,7 +520,7 @@ int orc_verify_stochastic(const float* p, const float* q, int Qrows, const int32
                     break;
                 }
                 uint32_t r[4];
-                node_draw(seed, step, b, c, r);
+                node_draw(seed, step, b0 + b, c, r);
                 double uc = (double)(r[0] >> 8) * (1.0 / 16777216.0);
                 if (uc * (double)Q[x] < P[x]) {
                     u = c;
@@ -544,7 +546,7 @@ int orc_verify_stochastic(const float* p, const float* q, int Qrows, const int32
             S += W[y];
         }
         uint32_t r[4];
-        node_draw(seed, step, b, u, r);
+        node_draw(seed, step, b0 + b, u, r);
         int tok = 0;
         if (S == 0) {
             if (status) *status |= 1;

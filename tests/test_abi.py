@@ -46,6 +46,32 @@ def test_tree_create_rejects_bad_parents(lib):
     assert lib.medusa_tree_create(None, 3, ctypes.byref(h)) == B.MEDUSA_ERR_INVALID_ARG
 
 
+def test_ragged_tree_create_rejects_bad_trees(lib):
+    # validation happens on the host, before any device allocation
+    h = ctypes.c_void_p()
+
+    def create(trees):
+        flat = [x for t in trees for x in t]
+        offs = [0]
+        for t in trees:
+            offs.append(offs[-1] + len(t))
+        arr = (ctypes.c_int32 * max(len(flat), 1))(*flat)
+        off = (ctypes.c_int32 * len(offs))(*offs)
+        return lib.medusa_tree_create_ragged(arr, off, len(trees), ctypes.byref(h))
+
+    assert create([[-1, 0], [-1, 1]]) == B.MEDUSA_ERR_INVALID_ARG
+    assert b"tree 1" in lib.medusa_last_error()
+    assert create([[-1, 0, 0], [-1] + list(range(128))]) == B.MEDUSA_ERR_UNSUPPORTED
+    assert b"tree 1" in lib.medusa_last_error()
+    assert create([[-1], []]) == B.MEDUSA_ERR_INVALID_ARG  # an empty tree
+    off = (ctypes.c_int32 * 2)(0, 1)
+    arr = (ctypes.c_int32 * 1)(-1)
+    assert lib.medusa_tree_create_ragged(arr, off, 0, ctypes.byref(h)) == B.MEDUSA_ERR_INVALID_ARG
+    bad = (ctypes.c_int32 * 2)(1, 2)
+    assert lib.medusa_tree_create_ragged(arr, bad, 1, ctypes.byref(h)) == B.MEDUSA_ERR_INVALID_ARG
+    assert lib.medusa_tree_create_ragged(None, off, 1, ctypes.byref(h)) == B.MEDUSA_ERR_INVALID_ARG
+
+
 def test_null_and_size_errors_before_launch(lib):
     # no tensor touches the device: every one of these fails validation first
     assert lib.medusa_heads(None, None, None, 1, 8, 8, 1, 1, None, None, None, None, None, None, None, None, None,

@@ -712,3 +712,24 @@ def test_kv_commit_exact_and_canaries(orc):
             ek[b, :, pl[b] + t] = kt[b, path[b, t]]
             ev[b, :, pl[b] + t] = vt[b, path[b, t]]
     assert torch.equal(k2, ek) and torch.equal(v2, ev)
+
+
+def test_stochastic_rows_checked_one_by_one_match_the_batch(orc):
+    # the sequence index only selects the Philox counter: row b on its own
+    # (b0 = b) gives what it gives inside the whole batch
+    w = I.scaled(I.WORKLOADS["stoch_b64"], B=5, V=300)
+    parents = I.workload_tree(w)
+    d = I.stochastic_inputs(w, parents)
+    maxd = int(max(orc.tree_shape(parents)[0]))
+    path, ln, bonus, _ = orc.verify_stochastic(d["p"], d["q"], d["node_tokens"], parents, 11, 3, maxd)
+    for b in range(w.B):
+        pb, lb, bb, _ = orc.verify_stochastic(d["p"][b:b + 1], d["q"][b:b + 1], d["node_tokens"][b:b + 1],
+                                                 parents, 11, 3, maxd, b0=b)
+        assert np.array_equal(pb[0], path[b]) and lb[0] == ln[b] and bb[0] == bonus[b]
+    # and the counter does matter: row 1 checked as if it were row 0 differs somewhere over a few steps
+    diff = False
+    for step in range(6):
+        p1 = orc.verify_stochastic(d["p"][1:2], d["q"][1:2], d["node_tokens"][1:2], parents, 11, step, maxd, b0=1)
+        p0 = orc.verify_stochastic(d["p"][1:2], d["q"][1:2], d["node_tokens"][1:2], parents, 11, step, maxd, b0=0)
+        diff |= not (np.array_equal(p1[0], p0[0]) and p1[2][0] == p0[2][0])
+    assert diff
