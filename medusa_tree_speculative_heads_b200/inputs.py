@@ -212,6 +212,43 @@ def attention_inputs(w: Workload, T: int, device: str = "cpu", canary: Optional[
             "prefix_len": pl.to(device)}
 
 
+def paged_cache(w: Workload, page_size: int, prefix_len: torch.Tensor, room: int = 64, extra_pages: int = 3,
+                device: str = "cpu", canary: Optional[float] = None) -> Dict[str, torch.Tensor]:
+    """A page pool k_pages, v_pages [num_pages, Hkv, page_size, D] and a block
+    table [B, max_pages] int32: sequence b owns ceil((prefix_len[b] + room) /
+    page_size) pages taken from a seeded random permutation of the pool (its
+    other table entries are -1), and `extra_pages` pages belong to nobody.
+    With ``canary`` every slot no call may read (positions at or past each
+    sequence's prefix, unowned pages) holds that value."""
+    dt = w.torch_dtype
+    g = _gen(w.seed * 7919 + 9, "cpu")
+    pl = [int(x) for x in prefix_len]
+    need = [(n + room + page_size - 1) // page_size for n in pl]
+    max_pages = max(need)
+    num_pages = sum(need) + extra_pages
+    perm = torch.randperm(num_pages, generator=g)
+    table = torch.full((w.B, max_pages), -1, dtype=torch.int32)
+    k = 0
+    for b in range(w.B):
+        table[b, :need[b]] = perm[k:k + need[b]].to(torch.int32)
+        k += need[b]
+    k_pages = _randn((num_pages, w.Hkv, page_size, w.D), g, dtype=dt)
+    v_pages = _randn((num_pages, w.Hkv, page_size, w.D), g, dtype=dt)
+    if canary is not None:
+        owned = torch.zeros(num_pages, dtype=torch.bool)
+        for b in range(w.B):
+            for blk in range(need[b]):
+                page = int(table[b, blk])
+                owned[page] = True
+                lo = max(0, pl[b] - blk * page_size)
+                if lo < page_size:
+                    k_pages[page, :, lo:] = canary
+                    v_pages[page, :, lo:] = canary
+        k_pages[~owned] = canary
+        v_pages[~owned] = canary
+    return {"k_pages": k_pages.to(device), "v_pages": v_pages.to(device), "block_table": table.to(device)}
+
+
 def random_node_tokens(w: Workload, parents: Sequence[int], seed_offset: int = 0) -> torch.Tensor:
     """[B,T] int32 tokens: a random root token and, under every node, distinct
     random tokens for its children (as a top-s list would give)."""

@@ -61,6 +61,11 @@ def lib():
                                             vp, i32]
         L.orc_kv_commit.argtypes = [vp, vp, vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]
         L.orc_kv_commit.restype = None
+        L.orc_gather_pages.argtypes = [vp, vp, i32, i32, i32, vp, i32, i32, i32, i32, i32, vp]
+        L.orc_gather_pages.restype = i32
+        L.orc_kv_commit_paged.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, vp, i32, vp, vp, vp, i32, i32, i32, i32,
+                                          i32, vp]
+        L.orc_kv_commit_paged.restype = None
         L.orc_residual.argtypes = [vp, vp, i32, vp, vp]
         L.orc_residual.restype = u64
         L.orc_round_bf16.argtypes = [dbl]
@@ -293,3 +298,46 @@ def kv_commit(k_cache, v_cache, k_tree, v_tree, path, length, prefix_len):
                         ctypes.c_void_p(kt.data_ptr()), ctypes.c_void_p(vt.data_ptr()), _p(pa), max_path, _p(ln),
                         _p(pl), _p(npl), B, Hkv, D, S_max, T, esize, _p(status))
     return kc, vc, npl, int(status[0])
+
+
+# ----------------------------------------------------------------------------
+# paged KV cache
+# ----------------------------------------------------------------------------
+
+def gather_pages(pages, table, n_pos, S_max: int, fill=None):
+    """Contiguous cache [B, Hkv, S_max, D] (torch, pages' dtype) holding
+    positions s < n_pos[b] of each sequence read through the block table;
+    other entries are `fill` (zeros when None)."""
+    pg = pages.detach().cpu().contiguous()
+    num_pages, Hkv, page_size, D = pg.shape
+    tb = _i32(table)
+    B, max_pages = tb.shape
+    npos = _i32(n_pos)
+    cache = torch.zeros((B, Hkv, S_max, D), dtype=pg.dtype) if fill is None else \
+        torch.full((B, Hkv, S_max, D), fill, dtype=pg.dtype)
+    rc = lib().orc_gather_pages(ctypes.c_void_p(pg.data_ptr()), _p(tb), max_pages, page_size, num_pages, _p(npos),
+                                B, Hkv, D, S_max, pg.element_size(), ctypes.c_void_p(cache.data_ptr()))
+    if rc != 0:
+        raise ValueError("block table does not cover the positions")
+    return cache
+
+
+def kv_commit_paged(k_pages, v_pages, k_tree, v_tree, table, path, length, prefix_len):
+    """Returns (k_pages', v_pages', new_prefix_len, status); inputs untouched."""
+    kp = k_pages.detach().cpu().contiguous().clone()
+    vp_ = v_pages.detach().cpu().contiguous().clone()
+    kt = k_tree.detach().cpu().contiguous()
+    vt = v_tree.detach().cpu().contiguous()
+    num_pages, Hkv, page_size, D = kp.shape
+    B, T = kt.shape[0], kt.shape[1]
+    tb = _i32(table)
+    pa = _i32(path)
+    ln = _i32(length)
+    pl = _i32(prefix_len)
+    npl = np.zeros(B, np.int32)
+    status = np.zeros(1, np.int32)
+    lib().orc_kv_commit_paged(ctypes.c_void_p(kp.data_ptr()), ctypes.c_void_p(vp_.data_ptr()),
+                              ctypes.c_void_p(kt.data_ptr()), ctypes.c_void_p(vt.data_ptr()), _p(tb), tb.shape[1],
+                              page_size, num_pages, _p(pa), pa.shape[1], _p(ln), _p(pl), _p(npl), B, Hkv, D, T,
+                              kp.element_size(), _p(status))
+    return kp, vp_, npl, int(status[0])

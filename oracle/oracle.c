@@ -616,3 +616,86 @@ void orc_kv_commit(void* k_cache, void* v_cache, const void* k_tree, const void*
         new_prefix_len[b] = S + L;
     }
 }
+
+/* ------------------------------------------------------------------------ */
+/* Paged KV cache                                                            */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * [MTP] "Production Deployment Guidelines": tree attention runs inside
+ * PagedAttention, the cache held in non-contiguous physical blocks.  A page
+ * pool pages [num_pages, Hkv, page_size, D] with a block table
+ * table [B, max_pages]: position s of sequence b is slot s % page_size of page
+ * table[b, s / page_size].  Paging is only where a position is stored, so the
+ * attention of a paged cache is the attention of the contiguous cache this
+ * gather builds:
+ *     cache[b, g, s, :] = pages[table[b, s / page_size], g, s % page_size, :]
+ * for s < n_pos[b]; other entries of cache are left as they are.  Returns -1
+ * (nothing written for that sequence) when a needed table entry is outside
+ * [0, num_pages) or s / page_size >= max_pages.
+ */
+int orc_gather_pages(const void* pages, const int32_t* table, int max_pages, int page_size, int num_pages,
+                     const int32_t* n_pos, int B, int Hkv, int D, int S_max, int esize, void* cache) {
+    int rc = 0;
+    for (int b = 0; b < B; ++b) {
+        int n = n_pos[b], ok = n >= 0 && n <= S_max;
+        for (int s = 0; ok && s < n; ++s) {
+            int blk = s / page_size;
+            if (blk >= max_pages) ok = 0;
+            else if (table[(size_t)b * max_pages + blk] < 0 || table[(size_t)b * max_pages + blk] >= num_pages) ok = 0;
+        }
+        if (!ok) {
+            rc = -1;
+            continue;
+        }
+        for (int g = 0; g < Hkv; ++g)
+            for (int s = 0; s < n; ++s) {
+                int page = table[(size_t)b * max_pages + s / page_size];
+                size_t src = ((((size_t)page * Hkv + g) * page_size) + s % page_size) * D * esize;
+                size_t dst = ((((size_t)b * Hkv + g) * S_max) + s) * D * esize;
+                memcpy((char*)cache + dst, (const char*)pages + src, (size_t)D * esize);
+            }
+    }
+    return rc;
+}
+
+/*
+ * Commit into a paged cache: as orc_kv_commit, position prefix_len[b] + t of
+ * sequence b being slot (prefix_len[b] + t) % page_size of page
+ * table[b, (prefix_len[b] + t) / page_size].  A sequence whose new positions
+ * need a block index >= max_pages, or a table entry outside [0, num_pages),
+ * or whose path holds a node id outside [0, T), is left untouched and sets bit
+ * 1 of *status.
+ */
+void orc_kv_commit_paged(void* k_pages, void* v_pages, const void* k_tree, const void* v_tree, const int32_t* table,
+                         int max_pages, int page_size, int num_pages, const int32_t* path, int max_path,
+                         const int32_t* len, const int32_t* prefix_len, int32_t* new_prefix_len, int B, int Hkv, int D,
+                         int T, int esize, int32_t* status) {
+    if (status) *status = 0;
+    for (int b = 0; b < B; ++b) {
+        int S = prefix_len[b], L = len[b];
+        int ok = L >= 0 && L <= max_path && S >= 0;
+        for (int t = 0; ok && t < L; ++t) {
+            int n = path[(size_t)b * max_path + t];
+            int blk = (S + t) / page_size;
+            if (n < 0 || n >= T || blk >= max_pages) ok = 0;
+            else if (table[(size_t)b * max_pages + blk] < 0 || table[(size_t)b * max_pages + blk] >= num_pages) ok = 0;
+        }
+        if (!ok) {
+            if (status) *status |= 1;
+            new_prefix_len[b] = S;
+            continue;
+        }
+        for (int t = 0; t < L; ++t) {
+            int n = path[(size_t)b * max_path + t];
+            int page = table[(size_t)b * max_pages + (S + t) / page_size];
+            for (int g = 0; g < Hkv; ++g) {
+                size_t dst = ((((size_t)page * Hkv + g) * page_size) + (S + t) % page_size) * D * esize;
+                size_t src = ((((size_t)b * T + n) * Hkv) + g) * D * esize;
+                memcpy((char*)k_pages + dst, (const char*)k_tree + src, (size_t)D * esize);
+                memcpy((char*)v_pages + dst, (const char*)v_tree + src, (size_t)D * esize);
+            }
+        }
+        new_prefix_len[b] = S + L;
+    }
+}

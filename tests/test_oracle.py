@@ -733,3 +733,59 @@ def test_stochastic_rows_checked_one_by_one_match_the_batch(orc):
         p0 = orc.verify_stochastic(d["p"][1:2], d["q"][1:2], d["node_tokens"][1:2], parents, 11, step, maxd, b0=0)
         diff |= not (np.array_equal(p1[0], p0[0]) and p1[2][0] == p0[2][0])
     assert diff
+
+
+def test_gather_pages_identity_table_is_a_reshape(orc):
+    # pages laid out in order, one sequence after another: the gather is a reshape
+    B, Hkv, D, ps, npg = 2, 3, 8, 4, 5
+    pages = torch.randn((B * npg, Hkv, ps, D), dtype=torch.float64)
+    table = torch.arange(B * npg, dtype=torch.int32).reshape(B, npg)
+    n_pos = torch.tensor([npg * ps, 7], dtype=torch.int32)
+    cache = orc.gather_pages(pages, table, n_pos, npg * ps)
+    want = pages.reshape(B, npg, Hkv, ps, D).permute(0, 2, 1, 3, 4).reshape(B, Hkv, npg * ps, D)
+    assert torch.equal(cache[0], want[0])
+    assert torch.equal(cache[1, :, :7], want[1, :, :7]) and (cache[1, :, 7:] == 0).all()
+
+
+def test_gather_pages_follows_the_table_and_rejects_holes(orc):
+    g = torch.Generator().manual_seed(0)
+    Hkv, D, ps = 2, 4, 3
+    pages = torch.randn((6, Hkv, ps, D), generator=g)
+    table = torch.tensor([[4, 1, -1], [0, 5, 2]], dtype=torch.int32)
+    cache = orc.gather_pages(pages, table, torch.tensor([5, 9], dtype=torch.int32), 9)
+    for b, n in ((0, 5), (1, 9)):
+        for s in range(n):
+            assert torch.equal(cache[b, :, s], pages[int(table[b, s // ps]), :, s % ps])
+    with pytest.raises(ValueError):  # position 6 needs block 2 of sequence 0, which is -1
+        orc.gather_pages(pages, table, torch.tensor([7, 0], dtype=torch.int32), 9)
+
+
+def test_paged_commit_equals_contiguous_commit_through_the_table(orc):
+    # committing into pages, then gathering, equals committing into the
+    # gathered contiguous cache
+    w = I.scaled(I.WORKLOADS["tiny"], B=3, Hkv=2, D=8, prefix=20)
+    parents = I.product_tree_parents((2, 2))
+    T = len(parents)
+    pl = torch.tensor([3, 20, 9], dtype=torch.int32)
+    pc = I.paged_cache(w, 4, pl, room=T)
+    g = torch.Generator().manual_seed(1)
+    kt = torch.randn((w.B, T, w.Hkv, w.D), generator=g)
+    vt = torch.randn((w.B, T, w.Hkv, w.D), generator=g)
+    path = torch.tensor([[0, 1, 3], [0, 2, -1], [0, -1, -1]], dtype=torch.int32)
+    ln = torch.tensor([3, 2, 1], dtype=torch.int32)
+    S_max = int((pc["block_table"] >= 0).sum(1).max()) * 4
+    kp2, vp2, npl, st = orc.kv_commit_paged(pc["k_pages"], pc["v_pages"], kt, vt, pc["block_table"], path, ln, pl)
+    assert st == 0 and npl.tolist() == [6, 22, 10]
+    kc, vc, npl_c, st_c = orc.kv_commit(orc.gather_pages(pc["k_pages"], pc["block_table"], pl, S_max),
+                                        orc.gather_pages(pc["v_pages"], pc["block_table"], pl, S_max),
+                                        kt, vt, path, ln, pl)
+    assert st_c == 0 and npl_c.tolist() == npl.tolist()
+    assert torch.equal(orc.gather_pages(kp2, pc["block_table"], torch.from_numpy(npl), S_max), kc)
+    assert torch.equal(orc.gather_pages(vp2, pc["block_table"], torch.from_numpy(npl), S_max), vc)
+    # a commit past the owned pages is refused; the other sequences still commit
+    pl4 = torch.tensor([3, 27, 9], dtype=torch.int32)  # sequence 1 owns 7 pages: positions 27, 28 need block 7
+    kp4, _, npl4, st4 = orc.kv_commit_paged(pc["k_pages"], pc["v_pages"], kt, vt, pc["block_table"], path, ln, pl4)
+    assert st4 == 1 and npl4.tolist() == [6, 27, 10]
+    before = orc.gather_pages(pc["k_pages"], pc["block_table"], torch.tensor([0, 28, 0], dtype=torch.int32), 28)
+    after = orc.gather_pages(kp4, pc["block_table"], torch.tensor([0, 28, 0], dtype=torch.int32), 28)
+    assert torch.equal(before[1], after[1])
