@@ -9,6 +9,8 @@
  *   tree_verify     greedy or stochastic verification: longest accepted
  *                   root-to-node path plus one bonus token
  *   kv_commit       append the accepted path's K/V to the cache
+ * tree_attention_paged and kv_commit_paged are the two cache calls over a
+ * paged KV cache (a page pool and a block table).
  *
  * Sources of the operations (public web pages on Medusa):
  *   [SPEC]  "Speculative Decoding & Medusa Tree Attention: Accelerating LLM
@@ -66,7 +68,8 @@ enum {
     MEDUSA_STATUS_CACHE_OVERFLOW = 2, /* kv_commit: prefix_len + len > S_max */
     MEDUSA_STATUS_BAD_PREFIX = 4,     /* prefix_len outside [0, max_prefix] */
     MEDUSA_STATUS_NO_MASS = 8,        /* stochastic bonus drawn from an all-zero distribution */
-    MEDUSA_STATUS_TIMEOUT = 16        /* an internal pipeline wait gave up after ~2 s (a library bug) */
+    MEDUSA_STATUS_TIMEOUT = 16,       /* an internal pipeline wait gave up after ~2 s (a library bug) */
+    MEDUSA_STATUS_BAD_PAGE = 32       /* a needed block-table entry outside [0, num_pages) */
 };
 
 typedef enum { MEDUSA_F32 = 0, MEDUSA_BF16 = 1 } medusa_dtype;
@@ -303,6 +306,58 @@ int tree_verify(medusa_verify_mode mode, const void* target, medusa_dtype target
 int kv_commit(void* k_cache, void* v_cache, const void* k_tree, const void* v_tree, const int32_t* accept_path,
               int max_path, const int32_t* accept_len, const int32_t* prefix_len, int32_t* new_prefix_len, int B,
               int T, int Hkv, int D, int S_max, medusa_dtype dt, int32_t* status, medusa_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Paged KV cache                                                            */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * [MTP] "Production Deployment Guidelines": tree attention runs inside
+ * PagedAttention, the KV cache held in non-contiguous physical blocks.  The
+ * caches of all sequences live in one pool of pages
+ *     k_pages, v_pages [num_pages, Hkv, page_size, D]   dtype dt
+ * and position s of sequence b is slot s % page_size of page
+ *     block_table[b * max_pages + s / page_size]        int32, device
+ * A call reads only the entries it needs: tree_attention_paged those of the
+ * positions below prefix_len[b], kv_commit_paged those of the positions it
+ * writes; the rest of the table may hold anything (-1, say).
+ */
+
+/*
+ * tree_attention with the prefix read through the block table.  Arguments,
+ * layouts, limits, tree handles and the workspace are those of
+ * tree_attention (with tree_attention_paged_workspace_size); max_prefix = 0
+ * means max_pages * page_size, and max_prefix may not exceed it.
+ * page_size >= 1.  bf16 with page_size a multiple of 64 or one of 8, 16, 32
+ * runs on the tensor-core kernel, other page sizes on the fallback kernel.
+ * Slots at or past prefix_len[b] in the sequence's last page may hold
+ * anything, NaN included: they are masked and never reach the output.
+ * A needed table entry outside [0, num_pages) sets MEDUSA_STATUS_BAD_PAGE;
+ * that page's keys are then skipped and the sequence's output is not
+ * meaningful.
+ */
+size_t tree_attention_paged_workspace_size(int B, int Hq, int Hkv, int D, int max_prefix, int max_pages,
+                                           int page_size, const medusa_tree* tree, medusa_dtype dt);
+int tree_attention_paged(const void* q, const void* k_tree, const void* v_tree, const void* k_pages,
+                         const void* v_pages, const int32_t* block_table, int max_pages, int page_size, int num_pages,
+                         const int32_t* prefix_len, int B, int Hq, int Hkv, int D, int max_prefix, float scale,
+                         medusa_dtype dt, const medusa_tree* tree, void* out, float* lse, void* workspace,
+                         size_t workspace_bytes, int32_t* status, medusa_stream_t stream);
+
+/*
+ * kv_commit into the page pool: for t < accept_len[b], position
+ * prefix_len[b] + t of sequence b receives tree[b, accept_path[b,t], g, :]
+ * (K and V, every kv-head g, bit for bit); new_prefix_len[b] =
+ * prefix_len[b] + accept_len[b].  A sequence whose new positions need a
+ * block index >= max_pages or a table entry outside [0, num_pages) is left
+ * untouched (new_prefix_len = prefix_len) and sets
+ * MEDUSA_STATUS_CACHE_OVERFLOW; a path id outside [0, T) sets
+ * MEDUSA_STATUS_BAD_TOKEN.  Other arguments as kv_commit.
+ */
+int kv_commit_paged(void* k_pages, void* v_pages, const void* k_tree, const void* v_tree, const int32_t* block_table,
+                    int max_pages, int page_size, int num_pages, const int32_t* accept_path, int max_path,
+                    const int32_t* accept_len, const int32_t* prefix_len, int32_t* new_prefix_len, int B, int T,
+                    int Hkv, int D, medusa_dtype dt, int32_t* status, medusa_stream_t stream);
 
 #ifdef __cplusplus
 }

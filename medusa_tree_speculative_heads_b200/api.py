@@ -111,6 +111,42 @@ def kv_commit(k_cache, v_cache, k_tree, v_tree, accept_path, accept_len, prefix_
     return {"new_prefix_len": new_prefix_len, "status": st}
 
 
+def tree_attention_paged(q, k_tree, v_tree, k_pages, v_pages, block_table, prefix_len, tree: Tree,
+                         scale: float = 0.0, max_prefix: int = 0, want_lse: bool = False) -> Dict[str, torch.Tensor]:
+    """Tree attention over a paged cache: page pools k/v_pages
+    [num_pages,Hkv,page_size,D], block_table [B,max_pages] int32."""
+    B, T, Hq, D = q.shape
+    Hkv = k_tree.shape[2]
+    num_pages, _, page_size, _ = k_pages.shape
+    max_pages = block_table.shape[1]
+    dev = q.device
+    dt = _b.dtype_code(q.dtype)
+    out = {"out": torch.empty_like(q), "status": _status(dev)}
+    if want_lse:
+        out["lse"] = torch.empty((B, T, Hq), dtype=torch.float32, device=dev)
+    nb = _b.tree_attention_paged_workspace_size(B, Hq, Hkv, D, max_prefix, max_pages, page_size, tree, dt)
+    ws = _ws(nb, dev)
+    _b.tree_attention_paged(q, k_tree, v_tree, k_pages, v_pages, block_table, max_pages, page_size, num_pages,
+                            prefix_len, B, Hq, Hkv, D, max_prefix, scale, dt, tree, out["out"], out.get("lse"), ws,
+                            nb, out["status"])
+    return out
+
+
+def kv_commit_paged(k_pages, v_pages, k_tree, v_tree, block_table, accept_path, accept_len, prefix_len,
+                    new_prefix_len: Optional[torch.Tensor] = None) -> Dict[str, torch.Tensor]:
+    """Append the accepted path's K/V into the page pools through the block table."""
+    num_pages, Hkv, page_size, D = k_pages.shape
+    B, T = k_tree.shape[0], k_tree.shape[1]
+    dev = k_pages.device
+    if new_prefix_len is None:
+        new_prefix_len = torch.empty_like(prefix_len)
+    st = _status(dev)
+    _b.kv_commit_paged(k_pages, v_pages, k_tree, v_tree, block_table, block_table.shape[1], page_size, num_pages,
+                       accept_path, accept_path.shape[1], accept_len, prefix_len, new_prefix_len, B, T, Hkv, D,
+                       _b.dtype_code(k_pages.dtype), st)
+    return {"new_prefix_len": new_prefix_len, "status": st}
+
+
 class MedusaStep:
     """All buffers of one decode step of a fixed shape, allocated once.
 

@@ -31,6 +31,7 @@ STATUS_CACHE_OVERFLOW = 2
 STATUS_BAD_PREFIX = 4
 STATUS_NO_MASS = 8
 STATUS_TIMEOUT = 16
+STATUS_BAD_PAGE = 32
 
 F32, BF16 = 0, 1
 GREEDY, STOCHASTIC = 0, 1
@@ -78,6 +79,12 @@ def lib() -> ctypes.CDLL:
         L.tree_verify.argtypes = [i32, vp, i32, vp, i32, vp, vp, i32, i32, vp, u64, u32, vp, i32, vp, vp, vp, sz, vp,
                                   vp]
         L.kv_commit.argtypes = [vp, vp, vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp]
+        L.tree_attention_paged_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32, i32, vp, i32]
+        L.tree_attention_paged_workspace_size.restype = sz
+        L.tree_attention_paged.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, vp, i32, i32, i32, i32, i32, f32,
+                                           i32, vp, vp, vp, vp, sz, vp, vp]
+        L.kv_commit_paged.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, vp, i32, vp, vp, vp, i32, i32, i32, i32, i32,
+                                      vp, vp]
         _lib = L
     return _lib
 
@@ -211,3 +218,23 @@ def kv_commit(k_cache, v_cache, k_tree, v_tree, accept_path, max_path, accept_le
     _check(lib().kv_commit(_p(k_cache), _p(v_cache), _p(k_tree), _p(v_tree), _p(accept_path), max_path,
                            _p(accept_len), _p(prefix_len), _p(new_prefix_len), B, T, Hkv, D, S_max, dt, _p(status),
                            _stream(stream)))
+
+
+def tree_attention_paged_workspace_size(B, Hq, Hkv, D, max_prefix, max_pages, page_size, tree: Tree, dt) -> int:
+    return lib().tree_attention_paged_workspace_size(B, Hq, Hkv, D, max_prefix, max_pages, page_size, tree.handle, dt)
+
+
+def tree_attention_paged(q, k_tree, v_tree, k_pages, v_pages, block_table, max_pages, page_size, num_pages,
+                         prefix_len, B, Hq, Hkv, D, max_prefix, scale, dt, tree: Tree, out, lse, workspace,
+                         workspace_bytes, status, stream=None):
+    _check(lib().tree_attention_paged(_p(q), _p(k_tree), _p(v_tree), _p(k_pages), _p(v_pages), _p(block_table),
+                                      max_pages, page_size, num_pages, _p(prefix_len), B, Hq, Hkv, D, max_prefix,
+                                      float(scale), dt, tree.handle, _p(out), _p(lse), _p(workspace), workspace_bytes,
+                                      _p(status), _stream(stream)))
+
+
+def kv_commit_paged(k_pages, v_pages, k_tree, v_tree, block_table, max_pages, page_size, num_pages, accept_path,
+                    max_path, accept_len, prefix_len, new_prefix_len, B, T, Hkv, D, dt, status, stream=None):
+    _check(lib().kv_commit_paged(_p(k_pages), _p(v_pages), _p(k_tree), _p(v_tree), _p(block_table), max_pages,
+                                 page_size, num_pages, _p(accept_path), max_path, _p(accept_len), _p(prefix_len),
+                                 _p(new_prefix_len), B, T, Hkv, D, dt, _p(status), _stream(stream)))

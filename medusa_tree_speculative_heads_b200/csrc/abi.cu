@@ -335,6 +335,8 @@ extern "C" int tree_attention(const void* q, const void* k_tree, const void* v_t
     a.scale = scale;
     a.dt = dt;
     a.tree = tree->ref();
+    a.block_table = nullptr;
+    a.max_pages = a.page_size = a.num_pages = 0;
     a.out = out;
     a.lse = lse;
     a.ws = workspace;
@@ -445,8 +447,128 @@ extern "C" int kv_commit(void* k_cache, void* v_cache, const void* k_tree, const
     a.D = D;
     a.S_max = S_max;
     a.esize = esize;
+    a.block_table = nullptr;
+    a.max_pages = a.page_size = a.num_pages = 0;
     a.status = status;
     cudaError_t e = commit_launch(a, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "kv_commit launch");
+    return ok();
+}
+
+// ---------------------------------------------------------------------------
+// paged KV cache
+// ---------------------------------------------------------------------------
+
+extern "C" size_t tree_attention_paged_workspace_size(int B, int Hq, int Hkv, int D, int max_prefix, int max_pages,
+                                                      int page_size, const medusa_tree* tree, medusa_dtype dt) {
+    if (!tree || B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || (D != 64 && D != 128) || max_pages < 1 || page_size < 1)
+        return 0;
+    if (max_prefix <= 0) max_prefix = max_pages * page_size;
+    return attn_workspace_size(B, tree->host.T, Hq, Hkv, D, max_prefix, dt);
+}
+
+extern "C" int tree_attention_paged(const void* q, const void* k_tree, const void* v_tree, const void* k_pages,
+                                    const void* v_pages, const int32_t* block_table, int max_pages, int page_size,
+                                    int num_pages, const int32_t* prefix_len, int B, int Hq, int Hkv, int D,
+                                    int max_prefix, float scale, medusa_dtype dt, const medusa_tree* tree, void* out,
+                                    float* lse, void* workspace, size_t workspace_bytes, int32_t* status,
+                                    medusa_stream_t stream) {
+    if (dt != MEDUSA_F32 && dt != MEDUSA_BF16)
+        return fail(MEDUSA_ERR_UNSUPPORTED, "tree_attention_paged: unknown dtype");
+    if (!q || !k_tree || !v_tree || !k_pages || !v_pages || !block_table || !prefix_len || !out)
+        return fail(MEDUSA_ERR_INVALID_ARG, "tree_attention_paged: NULL tensor argument");
+    int rc = check_tree(tree, B);
+    if (rc) return rc;
+    if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || max_pages < 1 || page_size < 1 || num_pages < 1 ||
+        (long)max_pages * page_size > (1L << 30))
+        return fail(MEDUSA_ERR_INVALID_ARG,
+                    "tree_attention_paged: bad sizes B=%d Hq=%d Hkv=%d max_pages=%d page_size=%d num_pages=%d", B, Hq,
+                    Hkv, max_pages, page_size, num_pages);
+    if (D != 64 && D != 128) return fail(MEDUSA_ERR_UNSUPPORTED, "tree_attention_paged: head_dim %d (64 or 128)", D);
+    const int cap = max_pages * page_size;
+    if (max_prefix <= 0) max_prefix = cap;
+    if (max_prefix > cap)
+        return fail(MEDUSA_ERR_INVALID_ARG, "tree_attention_paged: max_prefix %d > max_pages * page_size = %d",
+                    max_prefix, cap);
+    if (!al16(q) || !al16(k_tree) || !al16(v_tree) || !al16(k_pages) || !al16(v_pages) || !al16(out))
+        return fail(MEDUSA_ERR_INVALID_ARG, "tree_attention_paged: tensors must be 16-byte aligned");
+    const size_t need = attn_workspace_size(B, tree->host.T, Hq, Hkv, D, max_prefix, dt);
+    if (need && (!workspace || workspace_bytes < need || !al16(workspace)))
+        return fail(MEDUSA_ERR_WORKSPACE, "tree_attention_paged: workspace of %zu bytes, need %zu (16-byte aligned)",
+                    workspace_bytes, need);
+    AttnArgs a;
+    a.q = q;
+    a.k_tree = k_tree;
+    a.v_tree = v_tree;
+    a.k_cache = k_pages;
+    a.v_cache = v_pages;
+    a.prefix_len = prefix_len;
+    a.B = B;
+    a.T = tree->host.T;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.D = D;
+    a.S_max = cap;
+    a.max_prefix = max_prefix;
+    a.scale = scale;
+    a.dt = dt;
+    a.tree = tree->ref();
+    a.block_table = block_table;
+    a.max_pages = max_pages;
+    a.page_size = page_size;
+    a.num_pages = num_pages;
+    a.out = out;
+    a.lse = lse;
+    a.ws = workspace;
+    a.ws_bytes = workspace_bytes;
+    a.status = status;
+    cudaError_t e = attn_launch(a, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "tree_attention_paged launch");
+    return ok();
+}
+
+extern "C" int kv_commit_paged(void* k_pages, void* v_pages, const void* k_tree, const void* v_tree,
+                               const int32_t* block_table, int max_pages, int page_size, int num_pages,
+                               const int32_t* accept_path, int max_path, const int32_t* accept_len,
+                               const int32_t* prefix_len, int32_t* new_prefix_len, int B, int T, int Hkv, int D,
+                               medusa_dtype dt, int32_t* status, medusa_stream_t stream) {
+    if (dt != MEDUSA_F32 && dt != MEDUSA_BF16) return fail(MEDUSA_ERR_UNSUPPORTED, "kv_commit_paged: unknown dtype");
+    if (!k_pages || !v_pages || !k_tree || !v_tree || !block_table || !accept_path || !accept_len || !prefix_len ||
+        !new_prefix_len)
+        return fail(MEDUSA_ERR_INVALID_ARG, "kv_commit_paged: NULL tensor argument");
+    const int esize = dt == MEDUSA_BF16 ? 2 : 4;
+    if (B < 1 || T < 1 || T > kMaxTree || Hkv < 1 || D < 1 || max_path < 1 || max_path > kMaxTree ||
+        max_pages < 1 || page_size < 1 || num_pages < 1)
+        return fail(MEDUSA_ERR_INVALID_ARG,
+                    "kv_commit_paged: bad sizes B=%d T=%d Hkv=%d D=%d max_path=%d max_pages=%d page_size=%d "
+                    "num_pages=%d", B, T, Hkv, D, max_path, max_pages, page_size, num_pages);
+    if ((D * esize) % 16)
+        return fail(MEDUSA_ERR_INVALID_ARG, "kv_commit_paged: a K/V row (%d bytes) must be a multiple of 16 bytes",
+                    D * esize);
+    if (!al16(k_pages) || !al16(v_pages) || !al16(k_tree) || !al16(v_tree))
+        return fail(MEDUSA_ERR_INVALID_ARG, "kv_commit_paged: tensors must be 16-byte aligned");
+    CommitArgs a;
+    a.k_cache = k_pages;
+    a.v_cache = v_pages;
+    a.k_tree = k_tree;
+    a.v_tree = v_tree;
+    a.accept_path = accept_path;
+    a.max_path = max_path;
+    a.accept_len = accept_len;
+    a.prefix_len = prefix_len;
+    a.new_prefix_len = new_prefix_len;
+    a.B = B;
+    a.T = T;
+    a.Hkv = Hkv;
+    a.D = D;
+    a.S_max = 0;
+    a.esize = esize;
+    a.block_table = block_table;
+    a.max_pages = max_pages;
+    a.page_size = page_size;
+    a.num_pages = num_pages;
+    a.status = status;
+    cudaError_t e = commit_launch(a, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "kv_commit_paged launch");
     return ok();
 }

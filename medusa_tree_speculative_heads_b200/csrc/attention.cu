@@ -42,6 +42,8 @@ struct AttnParams {
     int n_splits;   // prefix splits + 1 (tree split last)
     int split_len;  // prefix keys per split, a multiple of kBN
     TreeRef tree;
+    const int32_t* block_table;  // NULL: contiguous caches; else page pools [num_pages, Hkv, page_size, D]
+    int max_pages, page_size, num_pages;
     float* part_o;    // [n_splits][B*Hkv][R][D], normalised
     float* part_lse;  // [n_splits][B*Hkv][R], log2 units
     int32_t* status;
@@ -143,13 +145,23 @@ __global__ void __launch_bounds__(kThreads) tree_attn_mma_kernel(const __grid_co
         for (int c = tid; c < kBN * CH; c += kThreads) {
             const int row = c / CH, ch = c % CH;
             const int key = key0 + row;
-            const bool valid = key < k_end;
+            bool valid = key < k_end;
             long off;
             const __nv_bfloat16 *ks, *vs;
             if (tree_split) {
                 off = (((long)b * p.T + (valid ? key : 0)) * p.Hkv + g) * D + ch * 8;
                 ks = p.k_tree + off;
                 vs = p.v_tree + off;
+            } else if (p.block_table) {
+                int page = valid ? __ldg(&p.block_table[(long)b * p.max_pages + key / p.page_size]) : 0;
+                if (valid && (page < 0 || page >= p.num_pages)) {
+                    if (ch == 0) set_status(p.status, MEDUSA_STATUS_BAD_PAGE);
+                    valid = false;
+                    page = 0;
+                }
+                off = (((long)page * p.Hkv + g) * p.page_size + (valid ? key % p.page_size : 0)) * D + ch * 8;
+                ks = p.k_cache + off;
+                vs = p.v_cache + off;
             } else {
                 off = (((long)b * p.Hkv + g) * p.S_max + (valid ? key : 0)) * D + ch * 8;
                 ks = p.k_cache + off;
@@ -372,7 +384,9 @@ __global__ void __launch_bounds__(256) tree_attn_f32_kernel(const float* __restr
                                                             const float* __restrict__ v_cache,
                                                             const int32_t* __restrict__ prefix_len, int B, int T,
                                                             int Hq, int Hkv, int S_max, int max_prefix, float scale,
-                                                            TreeRef trees, float* __restrict__ out,
+                                                            const int32_t* __restrict__ table, int max_pages,
+                                                            int page_size, int num_pages, TreeRef trees,
+                                                            float* __restrict__ out,
                                                             float* __restrict__ lse, int32_t* status) {
     constexpr int PL = D / 32;
     const long row = (long)blockIdx.x * 8 + (threadIdx.x >> 5);
@@ -414,8 +428,20 @@ __global__ void __launch_bounds__(256) tree_attn_f32_kernel(const float* __restr
         for (int e = 0; e < PL; ++e) o[e] = o[e] * a + w * vp[lane * PL + e];
         m = mn;
     };
-    const long cbase = ((long)b * Hkv + g) * S_max;
-    for (int j = 0; j < S; ++j) visit(k_cache + (cbase + j) * D, v_cache + (cbase + j) * D);
+    if (table) {
+        for (int j = 0; j < S; ++j) {
+            const int page = table[(long)b * max_pages + j / page_size];
+            if (page < 0 || page >= num_pages) {
+                if (lane == 0) set_status(status, MEDUSA_STATUS_BAD_PAGE);
+                continue;
+            }
+            const long row = ((long)page * Hkv + g) * page_size + j % page_size;
+            visit(k_cache + row * D, v_cache + row * D);
+        }
+    } else {
+        const long cbase = ((long)b * Hkv + g) * S_max;
+        for (int j = 0; j < S; ++j) visit(k_cache + (cbase + j) * D, v_cache + (cbase + j) * D);
+    }
     for (int j = 0; j < tree->T; ++j)
         if ((tree->anc[i][j >> 5] >> (j & 31)) & 1u)
             visit(k_tree + (((long)b * T + j) * Hkv + g) * D, v_tree + (((long)b * T + j) * Hkv + g) * D);
@@ -452,16 +478,21 @@ SplitPlan plan_splits(int B, int T, int Hq, int Hkv, int max_prefix, int tile_ro
     return sp;
 }
 
-SplitPlan plan_bf16(int B, int T, int Hq, int Hkv, int D, int max_prefix) {
+// the tensor-core kernel runs these shapes (and page sizes, when paged)
+bool use_tc(const AttnArgs& a, int D) {
+    return attn_tc_supported(a.Hq, a.Hkv, D, a.T, a.dt) && (!a.block_table || attn_tc_page_ok(a.page_size));
+}
+
+SplitPlan plan_bf16(int B, int T, int Hq, int Hkv, int D, int max_prefix, bool tc) {
     // tensor-core kernel: 128-row tiles, two CTAs per SM
-    if (attn_tc_supported(Hq, Hkv, D, T, MEDUSA_BF16))
-        return plan_splits(B, T, Hq, Hkv, max_prefix, 128, attn_tc_ctas_per_sm());
+    if (tc) return plan_splits(B, T, Hq, Hkv, max_prefix, 128, attn_tc_ctas_per_sm());
     return plan_splits(B, T, Hq, Hkv, max_prefix);
 }
 
 template <int D>
 cudaError_t attn_launch_bf16(const AttnArgs& a, cudaStream_t st) {
-    SplitPlan sp = plan_bf16(a.B, a.T, a.Hq, a.Hkv, D, a.max_prefix);
+    const bool tc = use_tc(a, D);
+    SplitPlan sp = plan_bf16(a.B, a.T, a.Hq, a.Hkv, D, a.max_prefix, tc);
     AttnParams p;
     p.q = (const __nv_bfloat16*)a.q;
     p.k_tree = (const __nv_bfloat16*)a.k_tree;
@@ -482,12 +513,16 @@ cudaError_t attn_launch_bf16(const AttnArgs& a, cudaStream_t st) {
     p.n_splits = sp.n_splits;
     p.split_len = sp.split_len;
     p.tree = a.tree;
+    p.block_table = a.block_table;
+    p.max_pages = a.max_pages;
+    p.page_size = a.page_size;
+    p.num_pages = a.num_pages;
     const long BH = (long)a.B * a.Hkv;
     p.part_o = (float*)a.ws;
     p.part_lse = (float*)((char*)a.ws + align256((size_t)sp.n_splits * BH * p.R * D * sizeof(float)));
     p.status = a.status;
     cudaError_t e;
-    if (attn_tc_supported(a.Hq, a.Hkv, D, a.T, a.dt)) {
+    if (tc) {
         e = attn_tc_launch(a, sp.m_tiles, sp.n_splits, sp.split_len, p.scale_log2, p.part_o, p.part_lse, st);
     } else {
         const size_t smem = (size_t)kBM * D * 2 + 4 * (size_t)kBN * D * 2 + kBM * 4 * sizeof(uint32_t);
@@ -509,7 +544,8 @@ cudaError_t attn_launch_f32(const AttnArgs& a, cudaStream_t st) {
     const float scale = a.scale > 0.f ? a.scale : 1.f / sqrtf((float)D);
     tree_attn_f32_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(
         (const float*)a.q, (const float*)a.k_tree, (const float*)a.v_tree, (const float*)a.k_cache,
-        (const float*)a.v_cache, a.prefix_len, a.B, a.T, a.Hq, a.Hkv, a.S_max, a.max_prefix, scale, a.tree,
+        (const float*)a.v_cache, a.prefix_len, a.B, a.T, a.Hq, a.Hkv, a.S_max, a.max_prefix, scale, a.block_table,
+        a.max_pages, a.page_size, a.num_pages, a.tree,
         (float*)a.out, a.lse, a.status);
     return cudaGetLastError();
 }
@@ -518,10 +554,12 @@ cudaError_t attn_launch_f32(const AttnArgs& a, cudaStream_t st) {
 
 size_t attn_workspace_size(int B, int T, int Hq, int Hkv, int D, int max_prefix, medusa_dtype dt) {
     if (dt != MEDUSA_BF16) return 0;
-    SplitPlan sp = plan_bf16(B, T, Hq, Hkv, D, max_prefix);
+    // enough for either kernel (a paged call may run either, by page size)
+    const SplitPlan a = plan_bf16(B, T, Hq, Hkv, D, max_prefix, true), b = plan_bf16(B, T, Hq, Hkv, D, max_prefix, false);
+    const size_t splits = a.n_splits > b.n_splits ? a.n_splits : b.n_splits;
     const size_t R = (size_t)T * (Hq / Hkv);
     const size_t BH = (size_t)B * Hkv;
-    return align256(sp.n_splits * BH * R * D * sizeof(float)) + align256(sp.n_splits * BH * R * sizeof(float));
+    return align256(splits * BH * R * D * sizeof(float)) + align256(splits * BH * R * sizeof(float));
 }
 
 cudaError_t attn_launch(const AttnArgs& a, cudaStream_t st) {

@@ -53,12 +53,14 @@ template <int D> constexpr int n_bars() { return 1 + 2 * k_stages<D>() + 2 * v_s
 
 struct TcAttnArgs {
     CUtensorMap mq;    // q as (D, Hq, B*T), box (64, G, 128/G)
-    CUtensorMap mkc;   // k_cache as (D, S_max, B*Hkv), box (64, 64, 1)
-    CUtensorMap mvc;
+    CUtensorMap mkc;   // k_cache as (D, S_max, B*Hkv), box (64, 64, 1); paged: k_pages as
+    CUtensorMap mvc;   //   (D, page_size, num_pages*Hkv), box (64, page_rows, 1)
     CUtensorMap mkt;   // k_tree as (D, Hkv, B*T), box (64, 1, 64)
     CUtensorMap mvt;
     const int32_t* prefix_len;
     TreeRef tree;
+    const int32_t* block_table;  // NULL: contiguous caches
+    int max_pages, page_size, num_pages, page_rows;  // page_rows = min(page_size, 64) rows per TMA box
     float* part_o;     // [n_splits][B*Hkv][R][D]
     float* part_lse;   // [n_splits][B*Hkv][R], log2 units
     int32_t* status;
@@ -146,8 +148,14 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
         k_end = min(S, k_begin + a.split_len);
         nc = k_end > k_begin ? (k_end - k_begin + kCh - 1) / kCh : 0;
     }
-    // first key of chunk j (prefix chunks end exactly at k_end)
-    auto chunk_start = [&](int j) { return tree_split ? j * kCh : k_end - (nc - j) * kCh; };
+    // first key of chunk j: contiguous prefix chunks end exactly at k_end (no
+    // slot past the prefix is read); paged ones start at page-aligned k_begin
+    const bool paged = a.block_table != nullptr;
+    auto chunk_start = [&](int j) {
+        return tree_split ? j * kCh : paged ? k_begin + j * kCh : k_end - (nc - j) * kCh;
+    };
+    // keys past key_end are not the sequence's (their rows are cleared in V)
+    const int key_end = tree_split ? Tb : k_end;
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
@@ -183,32 +191,60 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
 #pragma unroll
             for (int sub = 0; sub < NSUB; ++sub)
                 tma_load_3d(sQ + sub * (kAM * 128), &a.mq, sub * 64, g * a.G, b * a.T + mt * NB, q_full);
+            // one chunk of K or V: 64 keys x D into a ring stage, completing on `bar`
+            auto issue_chunk = [&](uint8_t* base, const CUtensorMap* mc, const CUtensorMap* mt, uint64_t* bar,
+                                   int cs) {
+                if (tree_split || !paged) {
+                    mbar_arrive_expect_tx(bar, kKVBytes);
+#pragma unroll
+                    for (int sub = 0; sub < NSUB; ++sub) {
+                        if (tree_split) tma_load_3d(base + sub * kSub, mt, sub * 64, g, b * a.T + cs, bar);
+                        else tma_load_3d(base + sub * kSub, mc, sub * 64, cs, bg, bar);
+                    }
+                    return;
+                }
+                // paged: boxes of page_rows keys, each from its own page; boxes
+                // at or past k_end are not loaded (their rows are masked, and
+                // cleared in V); an out-of-range page is skipped and reported
+                const int pr = a.page_rows, nbox = kCh / pr;
+                int pages[8];
+                int nload = 0;
+                for (int i = 0; i < nbox; ++i) {
+                    const int pos = cs + i * pr;
+                    pages[i] = -1;
+                    if (pos >= k_end) continue;
+                    const int page = __ldg(&a.block_table[(long)b * a.max_pages + pos / a.page_size]);
+                    if (page < 0 || page >= a.num_pages) {
+                        set_status(a.status, MEDUSA_STATUS_BAD_PAGE);
+                        continue;
+                    }
+                    pages[i] = page;
+                    ++nload;
+                }
+                mbar_arrive_expect_tx(bar, (uint32_t)(nload * pr * 128 * NSUB));
+                for (int i = 0; i < nbox; ++i) {
+                    if (pages[i] < 0) continue;
+                    const int pos = cs + i * pr;
+#pragma unroll
+                    for (int sub = 0; sub < NSUB; ++sub)
+                        tma_load_3d(base + sub * kSub + i * pr * 128, mc, sub * 64, pos % a.page_size,
+                                    pages[i] * a.Hkv + g, bar);
+                }
+            };
             int jk = 0, jv = 0;
             uint64_t t0 = global_ns();
             uint32_t idle = 0;
             while (jk < nc || jv < nc) {
                 bool prog = false;
                 if (jk < nc && (jk < KS || mbar_test(&k_empty[jk % KS], ((jk / KS) - 1) & 1))) {
-                    const int s = jk % KS, cs = chunk_start(jk);
-                    mbar_arrive_expect_tx(&k_full[s], kKVBytes);
-#pragma unroll
-                    for (int sub = 0; sub < NSUB; ++sub) {
-                        uint8_t* dk = sK + s * kKVBytes + sub * kSub;
-                        if (tree_split) tma_load_3d(dk, &a.mkt, sub * 64, g, b * a.T + cs, &k_full[s]);
-                        else tma_load_3d(dk, &a.mkc, sub * 64, cs, bg, &k_full[s]);
-                    }
+                    const int s = jk % KS;
+                    issue_chunk(sK + s * kKVBytes, &a.mkc, &a.mkt, &k_full[s], chunk_start(jk));
                     ++jk;
                     prog = true;
                 }
                 if (jv < jk && (jv < VS || mbar_test(&v_empty[jv % VS], ((jv / VS) - 1) & 1))) {
-                    const int s = jv % VS, cs = chunk_start(jv);
-                    mbar_arrive_expect_tx(&v_full[s], kKVBytes);
-#pragma unroll
-                    for (int sub = 0; sub < NSUB; ++sub) {
-                        uint8_t* dv = sV + s * kKVBytes + sub * kSub;
-                        if (tree_split) tma_load_3d(dv, &a.mvt, sub * 64, g, b * a.T + cs, &v_full[s]);
-                        else tma_load_3d(dv, &a.mvc, sub * 64, cs, bg, &v_full[s]);
-                    }
+                    const int s = jv % VS;
+                    issue_chunk(sV + s * kKVBytes, &a.mvc, &a.mvt, &v_full[s], chunk_start(jv));
                     ++jv;
                     prog = true;
                 }
@@ -317,7 +353,11 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
                 // ancestor bits (keys >= T have none); key0 is 0 or 64
                 vis = key0 == 0 ? ((uint64_t)anc[1] << 32 | anc[0]) : ((uint64_t)anc[3] << 32 | anc[2]);
             } else {
-                vis = key0 >= k_begin ? ~0ull : ~0ull << (k_begin - key0);  // only a first chunk reaches back
+                // keys [k_begin, k_end): a contiguous first chunk may reach back
+                // before k_begin, a paged last chunk past k_end
+                const int lo = key0 >= k_begin ? 0 : k_begin - key0, hi = k_end - key0;
+                vis = lo > 0 ? ~0ull << lo : ~0ull;
+                if (hi < kCh) vis &= (1ull << hi) - 1ull;
             }
             // online softmax in the log2 domain: p = 2^(s * scale * log2 e - mu)
             float mx;
@@ -386,17 +426,17 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
                 tmem_wait_st();
             }
             m = mn;
-            if (tree_split && key0 + kCh > Tb) {
-                // the chunk's rows past this sequence's tree are not its keys
-                // (padding, or another sequence's): P is 0 there, but a NaN in
-                // V would still reach O (0 * NaN), so those V rows are cleared
-                // before the PV product may start
+            if (key0 + kCh > key_end) {
+                // the chunk's rows past this sequence's keys (tree padding,
+                // another sequence's rows, page slots past the prefix, boxes
+                // not loaded) have P = 0, but a NaN in V would still reach O
+                // (0 * NaN), so those V rows are cleared before PV may start
                 const int s = j % VS;
                 if (!mbar_wait(&v_full[s], (j / VS) & 1)) {
                     ok = false;
                     break;
                 }
-                const int r0 = Tb - key0, lt = (warp - 2) * 32 + lane;
+                const int r0 = key_end - key0, lt = (warp - 2) * 32 + lane;
                 uint8_t* vs = sV + s * kKVBytes;
                 for (int idx = lt; idx < (kCh - r0) * NSUB * 8; idx += 128) {
                     const int row = r0 + idx / (NSUB * 8), rem = idx % (NSUB * 8);
@@ -461,6 +501,10 @@ size_t tc_attn_smem() {
 
 int attn_tc_ctas_per_sm() { return kCtasPerSm; }
 
+bool attn_tc_page_ok(int page_size) {
+    return page_size > 0 && (page_size % 64 == 0 || page_size == 8 || page_size == 16 || page_size == 32);
+}
+
 bool attn_tc_supported(int Hq, int Hkv, int D, int T, medusa_dtype dt) {
     const int G = Hkv > 0 ? Hq / Hkv : 0;
     return dt == MEDUSA_BF16 && (D == 64 || D == 128) && G >= 1 && G <= 16 && (G & (G - 1)) == 0 && T <= kMaxTree;
@@ -478,12 +522,23 @@ cudaError_t attn_tc_launch(const AttnArgs& x, int m_tiles, int n_splits, int spl
         const uint32_t box[3] = {64, (uint32_t)G, (uint32_t)(kAM / G)};
         if (!make_tmap_bf16(&a.mq, x.q, 3, dims, strides, box)) return cudaErrorInvalidValue;
     }
-    {
+    if (x.block_table) {
+        const uint64_t ps = x.page_size, NP = (uint64_t)x.num_pages * Hkv;
+        const uint64_t dims[3] = {D, ps, NP}, strides[2] = {D * 2, ps * D * 2};
+        const uint32_t box[3] = {64, (uint32_t)(x.page_size < kCh ? x.page_size : kCh), 1};
+        if (!make_tmap_bf16(&a.mkc, x.k_cache, 3, dims, strides, box)) return cudaErrorInvalidValue;
+        if (!make_tmap_bf16(&a.mvc, x.v_cache, 3, dims, strides, box)) return cudaErrorInvalidValue;
+    } else {
         const uint64_t dims[3] = {D, Smax, BH}, strides[2] = {D * 2, Smax * D * 2};
         const uint32_t box[3] = {64, (uint32_t)kCh, 1};
         if (!make_tmap_bf16(&a.mkc, x.k_cache, 3, dims, strides, box)) return cudaErrorInvalidValue;
         if (!make_tmap_bf16(&a.mvc, x.v_cache, 3, dims, strides, box)) return cudaErrorInvalidValue;
     }
+    a.block_table = x.block_table;
+    a.max_pages = x.max_pages;
+    a.page_size = x.page_size;
+    a.num_pages = x.num_pages;
+    a.page_rows = x.page_size < kCh ? x.page_size : kCh;
     {
         const uint64_t dims[3] = {D, Hkv, BT}, strides[2] = {D * 2, Hkv * D * 2};
         const uint32_t box[3] = {64, 1, (uint32_t)kCh};

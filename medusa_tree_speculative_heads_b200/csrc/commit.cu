@@ -2,7 +2,9 @@
 // Decoding", sections "The 2D Tree Attention Mask" -- the longest accepted
 // path is committed -- and "Production Deployment Guidelines" -- unselected
 // branches are culled): the accepted path's K/V rows are appended to each
-// sequence's cache after its prefix.  One CTA per sequence; 16-byte copies.
+// sequence's cache after its prefix, either a contiguous cache or a page pool
+// read through a block table ("Production Deployment Guidelines": tree
+// attention inside PagedAttention).  One CTA per sequence; 16-byte copies.
 #include "kernels.h"
 
 namespace medusa {
@@ -14,26 +16,35 @@ __global__ void __launch_bounds__(256) kv_commit_kernel(uint8_t* __restrict__ kc
                                                         const int32_t* __restrict__ path, int max_path,
                                                         const int32_t* __restrict__ len, const int32_t* prefix_len,
                                                         int32_t* new_prefix_len, int T, int Hkv, int S_max,
-                                                        int row_bytes, int32_t* status) {
+                                                        int row_bytes, const int32_t* __restrict__ table,
+                                                        int max_pages, int page_size, int num_pages, int32_t* status) {
     __shared__ int s_ok, s_S, s_L;
     __shared__ int s_node[MEDUSA_MAX_TREE];
+    __shared__ int s_page[MEDUSA_MAX_TREE];  // paged: the page of position S + t
     const int b = blockIdx.x, tid = threadIdx.x;
     // read prefix_len before anything is written: new_prefix_len may alias it
     const int S = prefix_len[b], L = len[b];
     const bool len_ok = L >= 0 && L <= max_path && L <= MEDUSA_MAX_TREE && S >= 0;
-    bool node_ok = true;
-    if (len_ok && tid < L) {  // every path entry loaded at once
+    bool node_ok = true, page_ok = true;
+    if (len_ok && tid < L) {  // every path entry (and page) loaded at once
         const int n = path[(long)b * max_path + tid];
         node_ok = n >= 0 && n < T;
         s_node[tid] = n;
+        if (table) {
+            const int blk = (S + tid) / page_size;
+            const int page = blk < max_pages ? table[(long)b * max_pages + blk] : -1;
+            page_ok = page >= 0 && page < num_pages;
+            s_page[tid] = page;
+        }
     }
     const bool all_nodes_ok = __syncthreads_and(node_ok);
+    const bool all_pages_ok = __syncthreads_and(page_ok);
     if (tid == 0) {
         int ok = 1;
         if (!len_ok || !all_nodes_ok) {
             ok = 0;
             set_status(status, MEDUSA_STATUS_BAD_TOKEN);
-        } else if (S + L > S_max) {
+        } else if (table ? !all_pages_ok : S + L > S_max) {
             ok = 0;
             set_status(status, MEDUSA_STATUS_CACHE_OVERFLOW);
         }
@@ -49,7 +60,8 @@ __global__ void __launch_bounds__(256) kv_commit_kernel(uint8_t* __restrict__ kc
             const int t = e / per_t, rem = e % per_t;
             const int g = rem / vecs, c = rem % vecs;
             const long src = (((long)b * T + s_node[t]) * Hkv + g) * row_bytes + c * 16;
-            const long dst = (((long)b * Hkv + g) * S_max + s_S + t) * row_bytes + c * 16;
+            const long dst = table ? (((long)s_page[t] * Hkv + g) * page_size + (s_S + t) % page_size) * row_bytes + c * 16
+                                   : (((long)b * Hkv + g) * S_max + s_S + t) * row_bytes + c * 16;
             *reinterpret_cast<uint4*>(kc + dst) = *reinterpret_cast<const uint4*>(kt + src);
             *reinterpret_cast<uint4*>(vc + dst) = *reinterpret_cast<const uint4*>(vt + src);
         }
@@ -64,7 +76,7 @@ cudaError_t commit_launch(const CommitArgs& a, cudaStream_t st) {
     kv_commit_kernel<<<a.B, 256, 0, st>>>((uint8_t*)a.k_cache, (uint8_t*)a.v_cache, (const uint8_t*)a.k_tree,
                                           (const uint8_t*)a.v_tree, a.accept_path, a.max_path, a.accept_len,
                                           a.prefix_len, a.new_prefix_len, a.T, a.Hkv, a.S_max, a.D * a.esize,
-                                          a.status);
+                                          a.block_table, a.max_pages, a.page_size, a.num_pages, a.status);
     return cudaGetLastError();
 }
 

@@ -50,6 +50,8 @@ struct AttnArgs {
     float scale;
     medusa_dtype dt;
     TreeRef tree;  // T is tree.T
+    const int32_t* block_table;  // NULL: contiguous caches [B, Hkv, S_max, D]; else page pools
+    int max_pages, page_size, num_pages;
     void* out;
     float* lse;
     void* ws;
@@ -61,6 +63,8 @@ cudaError_t attn_launch(const AttnArgs& a, cudaStream_t st);
 // tensor-core split kernel (bf16, D in {64,128}, power-of-two group size <= 16)
 bool attn_tc_supported(int Hq, int Hkv, int D, int T, medusa_dtype dt);
 int attn_tc_ctas_per_sm();
+// page sizes the tensor-core kernel reads (multiples of 64, or 8, 16, 32)
+bool attn_tc_page_ok(int page_size);
 cudaError_t attn_tc_launch(const AttnArgs& a, int m_tiles, int n_splits, int split_len, float scale_log2,
                            float* part_o, float* part_lse, cudaStream_t st);
 
@@ -100,6 +104,8 @@ struct CommitArgs {
     const int32_t* prefix_len;
     int32_t* new_prefix_len;
     int B, T, Hkv, D, S_max, esize;
+    const int32_t* block_table;  // NULL: contiguous cache [B, Hkv, S_max, D]
+    int max_pages, page_size, num_pages;
     int32_t* status;
 };
 cudaError_t commit_launch(const CommitArgs& a, cudaStream_t st);
