@@ -107,7 +107,10 @@ class OracleSample:
     residual block of every head, the LM-head rows of a `fraction` slice of
     the vocabulary, the attention of a `fraction` of the query rows, greedy
     verification over the full tree and the commit.  Inputs are drawn once
-    (not timed); run() returns (seconds, fraction of a full step's work)."""
+    (not timed); run() returns (seconds, fraction of a full step's work).
+    Workloads with a tree per sequence run the tree calls sequence by
+    sequence; a paged cache is read through its block table (the oracle's
+    page gather) and committed through it."""
 
     def __init__(self, w, fraction: float, seed: int = 0):
         import numpy as np
@@ -115,16 +118,21 @@ class OracleSample:
         from medusa_tree_speculative_heads_b200 import inputs as I
         self.w = w
         self.parents = I.workload_tree(w)
-        T = len(self.parents)
+        self.trees = I.sequence_trees(w)
+        T = self.T = max(len(t) for t in self.trees)
         self.Vs = max(8, int(round(w.V * fraction)))
         self.ws = I.scaled(w, V=self.Vs)
         self.hin = I.head_inputs(self.ws)
         self.ain = I.attention_inputs(w, T)
+        self.pc = (I.paged_cache(w, w.page_size, self.ain["prefix_len"], room=T, capacity=w.max_prefix + T)
+                   if w.page_size else None)
         n_rows = w.B * T * w.Hq
         nr = max(1, int(round(n_rows * fraction)))
         g = np.random.default_rng(seed)
         rid = g.choice(n_rows, size=nr, replace=False)
-        self.rows = np.stack([rid // (T * w.Hq), (rid // w.Hq) % T, rid % w.Hq], axis=1)
+        rows = np.stack([rid // (T * w.Hq), (rid // w.Hq) % T, rid % w.Hq], axis=1)
+        # rows of nodes past a sequence's own tree are not part of the step
+        self.rows = rows[[r[1] < len(self.trees[r[0]]) for r in rows]]
         # the residual block and verification/commit run whole; the LM head
         # and attention (all but ~2% of the work) are sampled at `fraction`
         lm = w.K * w.V * w.d
@@ -138,21 +146,55 @@ class OracleSample:
 
         import oracle
         from medusa_tree_speculative_heads_b200 import inputs as I
-        w, parents, hin, ain = self.w, self.parents, self.hin, self.ain
+        w, hin, ain, trees, T = self.w, self.hin, self.ain, self.trees, self.T
+        ragged = w.ragged_trees is not None
         t0 = time.perf_counter()
         ref = oracle.heads(hin["h"], hin["W_res"], hin["W_head"], want_hk=False)
         otop = np.stack([np.stack([oracle.topk(ref["logits"][b, k], 8) for k in range(w.K)]) for b in range(w.B)])
-        otok, _ = oracle.tree_fill(parents, hin["root_token"], otop,
-                                   np.take_along_axis(ref["probs"], otop, axis=-1))
+        otp = np.take_along_axis(ref["probs"], otop, axis=-1)
+        if ragged:
+            otok = np.full((w.B, T), -1, np.int32)
+            for b in range(w.B):
+                tb, _ = oracle.tree_fill(trees[b], hin["root_token"][b:b + 1], otop[b:b + 1], otp[b:b + 1])
+                otok[b, :len(trees[b])] = tb[0]
+        else:
+            otok, _ = oracle.tree_fill(self.parents, hin["root_token"], otop, otp)
         t1 = time.perf_counter()
         if self.logits is None:   # the target model's logits: input generation, not timed
-            self.logits = I.boosted_target_logits(self.ws, parents, torch.from_numpy(otok))
+            self.logits = I.boosted_target_logits(self.ws, self.parents, torch.from_numpy(otok))
         t2 = time.perf_counter()
-        oracle.tree_attention(ain["q"], ain["k_tree"], ain["v_tree"], ain["k_cache"], ain["v_cache"],
-                              ain["prefix_len"], parents, rows=self.rows)
-        maxd = int(max(oracle.tree_shape(parents)[0]))
-        path, ln, _ = oracle.verify_greedy(self.logits, otok, parents, maxd)
-        oracle.kv_commit(ain["k_cache"], ain["v_cache"], ain["k_tree"], ain["v_tree"], path, ln, ain["prefix_len"])
+        kc, vc = ain["k_cache"], ain["v_cache"]
+        if self.pc is not None:   # the prefix read through the block table
+            kc = oracle.gather_pages(self.pc["k_pages"], self.pc["block_table"], ain["prefix_len"], w.S_max)
+            vc = oracle.gather_pages(self.pc["v_pages"], self.pc["block_table"], ain["prefix_len"], w.S_max)
+        if ragged:
+            for b in range(w.B):
+                rb = self.rows[self.rows[:, 0] == b].copy()
+                if len(rb) == 0:
+                    continue
+                rb[:, 0] = 0
+                Tb = len(trees[b])
+                oracle.tree_attention(ain["q"][b:b + 1, :Tb], ain["k_tree"][b:b + 1, :Tb], ain["v_tree"][b:b + 1, :Tb],
+                                      kc[b:b + 1], vc[b:b + 1], ain["prefix_len"][b:b + 1], trees[b], rows=rb)
+        else:
+            oracle.tree_attention(ain["q"], ain["k_tree"], ain["v_tree"], kc, vc, ain["prefix_len"], self.parents,
+                                  rows=self.rows)
+        maxd = max(int(max(oracle.tree_shape(t)[0])) for t in (trees if ragged else [self.parents]))
+        if ragged:
+            path = np.full((w.B, maxd), -1, np.int32)
+            ln = np.zeros(w.B, np.int32)
+            for b in range(w.B):
+                Tb = len(trees[b])
+                pb, lb, _ = oracle.verify_greedy(self.logits[b:b + 1, :Tb], otok[b:b + 1, :Tb], trees[b], maxd)
+                path[b], ln[b] = pb[0], lb[0]
+        else:
+            path, ln, _ = oracle.verify_greedy(self.logits, otok, self.parents, maxd)
+        if self.pc is not None:
+            oracle.kv_commit_paged(self.pc["k_pages"], self.pc["v_pages"], ain["k_tree"], ain["v_tree"],
+                                   self.pc["block_table"], path, ln, ain["prefix_len"])
+        else:
+            oracle.kv_commit(ain["k_cache"], ain["v_cache"], ain["k_tree"], ain["v_tree"], path, ln,
+                             ain["prefix_len"])
         t3 = time.perf_counter()
         return (t1 - t0) + (t3 - t2), self.frac
 
@@ -207,12 +249,19 @@ def whole_job_rate(world: int, steps: int, seconds: float) -> float:
 
 def config_dict(w, world):
     from medusa_tree_speculative_heads_b200 import inputs as I
-    T = len(I.workload_tree(w))
-    tree = f"top-s {w.topk}" if w.topk else f"random tree {w.random_tree}"
+    Ts = [len(t) for t in I.sequence_trees(w)]
+    T = max(Ts)
+    if w.ragged_trees:
+        tree = f"a random tree per sequence {w.ragged_trees} ({min(Ts)}..{max(Ts)} nodes, mean {sum(Ts) / len(Ts):.0f})"
+    else:
+        tree = f"top-s {w.topk}" if w.topk else f"random tree {w.random_tree}"
+    if w.page_size:
+        tree += f", KV in pages of {w.page_size} via a block table"
     prefix = f"prefix U[{w.prefix_range[0]}, {w.prefix_range[1]}]" if w.prefix_range else f"prefix {w.prefix}"
     verify = "stochastic verify" if w.stochastic else f"greedy verify, match prob {w.match_prob}"
     head_gb = w.K * (w.d * w.d + w.V * w.d) * (2 if w.dtype == "bf16" else 4) / 1e9
-    return {"workload": (f"{w.name}: B={w.B} d={w.d} V={w.V} K={w.K} heads, {tree} -> {T}-node tree, "
+    shape = tree if w.ragged_trees else f"{tree} -> {T}-node tree"
+    return {"workload": (f"{w.name}: B={w.B} d={w.d} V={w.V} K={w.K} heads, {shape}, "
                          f"{w.Hq}/{w.Hkv} heads head_dim {w.D}, {prefix}, {verify}, one attention layer"),
             "global_batch": w.B * world, "seq_len": w.max_prefix, "parallelism": f"replicas x{world}",
             "l2": f"inputs larger than L2: each step streams {head_gb:.2f} GB of head weights through the 126 MB L2"}
@@ -250,14 +299,23 @@ def run_mine(args, rank, world, local_rank):
         dist.barrier()
 
     w = I.WORKLOADS[args.workload]
-    parents = I.workload_tree(w)
-    T = len(parents)
+    parents = I.workload_tree(w)       # one parent list, or one per sequence
+    seq_trees = I.sequence_trees(w)
+    T = max(len(t) for t in seq_trees)
     hin = I.head_inputs(w, device="cuda")
     ain = I.attention_inputs(w, T, device="cuda")
+    block_table = None
+    paged = {}
+    if w.page_size:
+        # the cache as a page pool read through a block table
+        pc = I.paged_cache(w, w.page_size, ain["prefix_len"].cpu(), room=T, device="cuda",
+                           capacity=w.max_prefix + T)
+        ain["k_cache"], ain["v_cache"], block_table = pc["k_pages"], pc["v_pages"], pc["block_table"]
+        paged = dict(page_size=w.page_size, max_pages=block_table.shape[1], num_pages=pc["k_pages"].shape[0])
     from medusa_tree_speculative_heads_b200 import binding as Bnd
     mode = Bnd.STOCHASTIC if w.stochastic else Bnd.GREEDY
     step = MedusaStep(B=w.B, d=w.d, V=w.V, K=w.K, Hq=w.Hq, Hkv=w.Hkv, D=w.D, S_max=w.S_max, parents=parents,
-                      dtype=w.torch_dtype, max_prefix=w.max_prefix, device=dev, mode=mode, q_rows=T)
+                      dtype=w.torch_dtype, max_prefix=w.max_prefix, device=dev, mode=mode, q_rows=T, **paged)
     q_draft = vtok = None
     if w.stochastic:
         # the target's and the draft's distributions and the drafted tokens
@@ -276,7 +334,7 @@ def run_mine(args, rank, world, local_rank):
         step.run(h=hin["h"], W_res=hin["W_res"], W_head=hin["W_head"], root_token=hin["root_token"], q=ain["q"],
                  k_tree=ain["k_tree"], v_tree=ain["v_tree"], k_cache=ain["k_cache"], v_cache=ain["v_cache"],
                  prefix_len=ain["prefix_len"], new_prefix_len=new_pl, target=logits, q_draft=q_draft,
-                 node_tokens=vtok)
+                 node_tokens=vtok, block_table=block_table)
 
     def barrier():
         if world > 1:
@@ -300,11 +358,13 @@ def run_mine(args, rank, world, local_rank):
         ev[i][0].record()
         step.heads(hin["h"], hin["W_res"], hin["W_head"], hin["root_token"])
         ev[i][1].record()
-        step.attention(ain["q"], ain["k_tree"], ain["v_tree"], ain["k_cache"], ain["v_cache"], ain["prefix_len"])
+        step.attention(ain["q"], ain["k_tree"], ain["v_tree"], ain["k_cache"], ain["v_cache"], ain["prefix_len"],
+                       block_table)
         ev[i][2].record()
         step.verify(logits, q_draft, None, 0, i, vtok)
         ev[i][3].record()
-        step.commit(ain["k_cache"], ain["v_cache"], ain["k_tree"], ain["v_tree"], ain["prefix_len"], new_pl)
+        step.commit(ain["k_cache"], ain["v_cache"], ain["k_tree"], ain["v_tree"], ain["prefix_len"], new_pl,
+                    block_table)
         ev[i][4].record()
     e1.record()
     torch.cuda.synchronize()
@@ -352,7 +412,7 @@ def run_mine(args, rank, world, local_rank):
         step.run(h=d["h"], W_res=hin["W_res"], W_head=hin["W_head"], root_token=d["root_token"], q=d["q"],
                  k_tree=d["k_tree"], v_tree=d["v_tree"], k_cache=ain["k_cache"], v_cache=ain["v_cache"],
                  prefix_len=ain["prefix_len"], new_prefix_len=new_pl, target=d["target"],
-                 q_draft=d.get("q_draft"), node_tokens=d.get("tokens"))
+                 q_draft=d.get("q_draft"), node_tokens=d.get("tokens"), block_table=block_table)
         used[slot].record(main_stream)
         for o, ho in zip(outs, host_out):
             ho.copy_(o, non_blocking=True)
@@ -376,11 +436,17 @@ def run_mine(args, rank, world, local_rank):
     elt = 2 if w.dtype == "bf16" else 4
     heads_bytes = (w.K * w.d * w.d + w.K * w.V * w.d) * elt + w.B * w.d * elt
     heads_gbs = heads_bytes / stage[0] / 1e9
-    sum_S = int(ain["prefix_len"].sum().item())
-    attn_bytes = (2 * w.Hkv * sum_S * w.D + 2 * w.B * T * w.Hq * w.D + 2 * w.B * T * w.Hkv * w.D) * elt
+    Sb = [int(x) for x in ain["prefix_len"].cpu()]
+    sum_S = sum(Sb)
+    Ts = [len(t) for t in seq_trees]
+    attn_bytes = (2 * w.Hkv * sum_S * w.D + 2 * sum(Ts) * w.Hq * w.D + 2 * sum(Ts) * w.Hkv * w.D) * elt
     attn_gbs = attn_bytes / stage[1] / 1e9
-    anc_pairs = sum(bin(sum(1 << j for j in range(T) if _is_anc(parents, i, j))).count("1") for i in range(T))
-    attn_flops = 4 * w.D * w.Hq * (T * sum_S + anc_pairs * w.B)
+    anc = {}
+    for tr in seq_trees:  # visible (node, tree node) pairs of each distinct tree
+        key = tuple(tr)
+        if key not in anc:
+            anc[key] = sum(1 for i in range(len(tr)) for j in range(len(tr)) if _is_anc(tr, i, j))
+    attn_flops = 4 * w.D * w.Hq * sum(Ts[b] * Sb[b] + anc[tuple(seq_trees[b])] for b in range(w.B))
     attn_tflops = attn_flops / stage[1] / 1e12
 
     # the roofline object describes the step's dominant kernel: the heads

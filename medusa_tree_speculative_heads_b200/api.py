@@ -153,11 +153,14 @@ class MedusaStep:
     ``run`` issues the four library calls on the current stream:
     medusa_heads -> tree_attention -> tree_verify -> kv_commit.  The new
     prefix lengths go to ``new_prefix_len`` (pass the same tensor as
-    ``prefix_len`` to advance in place)."""
+    ``prefix_len`` to advance in place).  ``parents`` is one parent list, or
+    one per sequence.  With ``page_size`` > 0 the cache is a page pool
+    [num_pages, Hkv, page_size, D] read and written through a block table
+    [B, max_pages] (pass it as ``block_table``), and the paged calls run."""
 
     def __init__(self, *, B: int, d: int, V: int, K: int, Hq: int, Hkv: int, D: int, S_max: int,
                  parents, dtype: torch.dtype, mode: int = _b.GREEDY, max_prefix: int = 0,
-                 q_rows: int = 0, device=None):
+                 q_rows: int = 0, device=None, page_size: int = 0, max_pages: int = 0, num_pages: int = 0):
         dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
         self.B, self.d, self.V, self.K = B, d, V, K
         self.Hq, self.Hkv, self.D, self.S_max, self.max_prefix = Hq, Hkv, D, S_max, max_prefix
@@ -178,7 +181,12 @@ class MedusaStep:
         self.bonus = torch.empty((B,), dtype=i32, device=dev)
         self.status = torch.zeros(1, dtype=i32, device=dev)
         self.ws_heads_n = _b.medusa_heads_workspace_size(B, d, V, K, self.dt)
-        self.ws_attn_n = _b.tree_attention_workspace_size(B, Hq, Hkv, D, S_max, max_prefix, self.tree, self.dt)
+        self.page_size, self.max_pages, self.num_pages = page_size, max_pages, num_pages
+        if page_size > 0:
+            self.ws_attn_n = _b.tree_attention_paged_workspace_size(B, Hq, Hkv, D, max_prefix, max_pages, page_size,
+                                                                    self.tree, self.dt)
+        else:
+            self.ws_attn_n = _b.tree_attention_workspace_size(B, Hq, Hkv, D, S_max, max_prefix, self.tree, self.dt)
         self.ws_verify_n = _b.tree_verify_workspace_size(mode, B, V, self.tree)
         self.ws_heads = _ws(self.ws_heads_n, dev)
         self.ws_attn = _ws(self.ws_attn_n, dev)
@@ -189,7 +197,13 @@ class MedusaStep:
                         self.topk_idx, self.topk_prob, self.node_tokens, self.node_q, None, None, probs_out,
                         self.ws_heads, self.ws_heads_n, self.status)
 
-    def attention(self, q, k_tree, v_tree, k_cache, v_cache, prefix_len):
+    def attention(self, q, k_tree, v_tree, k_cache, v_cache, prefix_len, block_table=None):
+        if self.page_size > 0:
+            _b.tree_attention_paged(q, k_tree, v_tree, k_cache, v_cache, block_table, self.max_pages, self.page_size,
+                                    self.num_pages, prefix_len, self.B, self.Hq, self.Hkv, self.D, self.max_prefix,
+                                    0.0, self.dt, self.tree, self.attn_out, None, self.ws_attn, self.ws_attn_n,
+                                    self.status)
+            return
         _b.tree_attention(q, k_tree, v_tree, k_cache, v_cache, prefix_len, self.B, self.Hq, self.Hkv, self.D,
                           self.S_max, self.max_prefix, 0.0, self.dt, self.tree, self.attn_out, None, self.ws_attn,
                           self.ws_attn_n, self.status)
@@ -201,13 +215,18 @@ class MedusaStep:
                        step, self.accept_path, self.max_path, self.accept_len, self.bonus, self.ws_verify,
                        self.ws_verify_n, self.status)
 
-    def commit(self, k_cache, v_cache, k_tree, v_tree, prefix_len, new_prefix_len):
+    def commit(self, k_cache, v_cache, k_tree, v_tree, prefix_len, new_prefix_len, block_table=None):
+        if self.page_size > 0:
+            _b.kv_commit_paged(k_cache, v_cache, k_tree, v_tree, block_table, self.max_pages, self.page_size,
+                               self.num_pages, self.accept_path, self.max_path, self.accept_len, prefix_len,
+                               new_prefix_len, self.B, self.T, self.Hkv, self.D, self.dt, self.status)
+            return
         _b.kv_commit(k_cache, v_cache, k_tree, v_tree, self.accept_path, self.max_path, self.accept_len, prefix_len,
                      new_prefix_len, self.B, self.T, self.Hkv, self.D, self.S_max, self.dt, self.status)
 
     def run(self, *, h, W_res, W_head, root_token, q, k_tree, v_tree, k_cache, v_cache, prefix_len, new_prefix_len,
-            target, q_draft=None, q_row=None, seed: int = 0, step: int = 0, node_tokens=None):
+            target, q_draft=None, q_row=None, seed: int = 0, step: int = 0, node_tokens=None, block_table=None):
         self.heads(h, W_res, W_head, root_token)
-        self.attention(q, k_tree, v_tree, k_cache, v_cache, prefix_len)
+        self.attention(q, k_tree, v_tree, k_cache, v_cache, prefix_len, block_table)
         self.verify(target, q_draft, q_row, seed, step, node_tokens)
-        self.commit(k_cache, v_cache, k_tree, v_tree, prefix_len, new_prefix_len)
+        self.commit(k_cache, v_cache, k_tree, v_tree, prefix_len, new_prefix_len, block_table)

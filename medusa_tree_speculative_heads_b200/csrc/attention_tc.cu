@@ -50,6 +50,7 @@ constexpr int kCtasPerSm = 2;
 template <int D> constexpr int k_stages() { return D == 128 ? 3 : 4; }
 template <int D> constexpr int v_stages() { return D == 128 ? 2 : 4; }
 template <int D> constexpr int n_bars() { return 1 + 2 * k_stages<D>() + 2 * v_stages<D>() + 6; }
+constexpr int kPageRing = 8 * 8 * 4;  // bytes of the page-id ring (8 chunks x 8 boxes)
 
 struct TcAttnArgs {
     CUtensorMap mq;    // q as (D, Hq, B*T), box (64, G, 128/G)
@@ -67,6 +68,13 @@ struct TcAttnArgs {
     int B, T, Hq, Hkv, G, S_max, max_prefix, R, n_splits, split_len;
     float scale_log2;
 };
+
+// 4-byte asynchronous global -> shared copy (cp.async group semantics)
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 // 2^x with the SFU's approximate exponential (relative error ~2^-22, far
 // below the bf16 rounding P goes through; 2^-inf = 0)
@@ -120,6 +128,8 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
     // the last two have completed
     uint64_t* o_last = o_full + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_last + 1);
+    // paged: the page of each box of the last 8 K chunks, for their V loads
+    int* pg_ring = reinterpret_cast<int*>(tmem_slot + 4);  // [8][8]
 
     const int mt = blockIdx.x, bg = blockIdx.y, split = blockIdx.z;
     const int b = bg / a.Hkv, g = bg % a.Hkv;
@@ -191,9 +201,28 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
 #pragma unroll
             for (int sub = 0; sub < NSUB; ++sub)
                 tma_load_3d(sQ + sub * (kAM * 128), &a.mq, sub * 64, g * a.G, b * a.T + mt * NB, q_full);
-            // one chunk of K or V: 64 keys x D into a ring stage, completing on `bar`
+            // Paged: the page of every box (page_rows keys) of a chunk, copied
+            // asynchronously into the chunk's pg_ring slot one chunk ahead (a
+            // K chunk waits only for its own ids; its V chunk reuses them).
+            // Boxes at or past k_end are not loaded (their rows are masked, and
+            // cleared in V); an out-of-range page is skipped and reported.
+            const int pr = paged ? a.page_rows : kCh, nbox = kCh / pr;
+            auto fetch_pages = [&](int j) {
+                if (j >= nc) return;
+                int* ring = pg_ring + (j & 7) * 8;
+                const int cs = chunk_start(j);
+                for (int i = 0; i < nbox; ++i) {
+                    const int pos = cs + i * pr;
+                    if (pos < k_end)
+                        cp_async4(smem_addr(ring + i), &a.block_table[(long)b * a.max_pages + pos / a.page_size]);
+                    else
+                        ring[i] = -1;
+                }
+                cp_async_commit();
+            };
             auto issue_chunk = [&](uint8_t* base, const CUtensorMap* mc, const CUtensorMap* mt, uint64_t* bar,
-                                   int cs) {
+                                   int j, bool is_k) {
+                const int cs = chunk_start(j);
                 if (tree_split || !paged) {
                     mbar_arrive_expect_tx(bar, kKVBytes);
 #pragma unroll
@@ -203,34 +232,32 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
                     }
                     return;
                 }
-                // paged: boxes of page_rows keys, each from its own page; boxes
-                // at or past k_end are not loaded (their rows are masked, and
-                // cleared in V); an out-of-range page is skipped and reported
-                const int pr = a.page_rows, nbox = kCh / pr;
-                int pages[8];
-                int nload = 0;
-                for (int i = 0; i < nbox; ++i) {
-                    const int pos = cs + i * pr;
-                    pages[i] = -1;
-                    if (pos >= k_end) continue;
-                    const int page = __ldg(&a.block_table[(long)b * a.max_pages + pos / a.page_size]);
-                    if (page < 0 || page >= a.num_pages) {
-                        set_status(a.status, MEDUSA_STATUS_BAD_PAGE);
-                        continue;
+                int* ring = pg_ring + (j & 7) * 8;
+                if (is_k) {
+                    cp_async_wait_all();  // this chunk's ids (the only group in flight)
+                    for (int i = 0; i < nbox; ++i) {
+                        const int page = ring[i];
+                        if (page >= a.num_pages || (page < 0 && cs + i * pr < k_end)) {
+                            set_status(a.status, MEDUSA_STATUS_BAD_PAGE);
+                            ring[i] = -1;
+                        }
                     }
-                    pages[i] = page;
-                    ++nload;
+                    fetch_pages(j + 1);  // the next chunk's ids, in flight meanwhile
                 }
+                int nload = 0;
+                for (int i = 0; i < nbox; ++i) nload += ring[i] >= 0;
                 mbar_arrive_expect_tx(bar, (uint32_t)(nload * pr * 128 * NSUB));
                 for (int i = 0; i < nbox; ++i) {
-                    if (pages[i] < 0) continue;
+                    const int page = ring[i];
+                    if (page < 0) continue;
                     const int pos = cs + i * pr;
 #pragma unroll
                     for (int sub = 0; sub < NSUB; ++sub)
                         tma_load_3d(base + sub * kSub + i * pr * 128, mc, sub * 64, pos % a.page_size,
-                                    pages[i] * a.Hkv + g, bar);
+                                    page * a.Hkv + g, bar);
                 }
             };
+            if (paged && !tree_split) fetch_pages(0);
             int jk = 0, jv = 0;
             uint64_t t0 = global_ns();
             uint32_t idle = 0;
@@ -238,13 +265,13 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
                 bool prog = false;
                 if (jk < nc && (jk < KS || mbar_test(&k_empty[jk % KS], ((jk / KS) - 1) & 1))) {
                     const int s = jk % KS;
-                    issue_chunk(sK + s * kKVBytes, &a.mkc, &a.mkt, &k_full[s], chunk_start(jk));
+                    issue_chunk(sK + s * kKVBytes, &a.mkc, &a.mkt, &k_full[s], jk, true);
                     ++jk;
                     prog = true;
                 }
                 if (jv < jk && (jv < VS || mbar_test(&v_empty[jv % VS], ((jv / VS) - 1) & 1))) {
                     const int s = jv % VS;
-                    issue_chunk(sV + s * kKVBytes, &a.mvc, &a.mvt, &v_full[s], chunk_start(jv));
+                    issue_chunk(sV + s * kKVBytes, &a.mvc, &a.mvt, &v_full[s], jv, false);
                     ++jv;
                     prog = true;
                 }
@@ -493,8 +520,9 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
 
 template <int D>
 size_t tc_attn_smem() {
-    // Q, the K and V rings, the mbarriers and the TMEM address slot
-    return (size_t)kAM * D * 2 + (size_t)(k_stages<D>() + v_stages<D>()) * kCh * D * 2 + n_bars<D>() * 8 + 16;
+    // Q, the K and V rings, the mbarriers, the TMEM address slot and the page-id ring
+    return (size_t)kAM * D * 2 + (size_t)(k_stages<D>() + v_stages<D>()) * kCh * D * 2 + n_bars<D>() * 8 + 16 +
+           kPageRing;
 }
 
 }  // namespace

@@ -56,6 +56,8 @@ class Workload:
     random_tree: Optional[tuple] = None    # (T, max_depth, max_children)
     match_prob: float = 0.6          # greedy boost probability
     stochastic: bool = False
+    ragged_trees: Optional[tuple] = None   # (T_min, T_max, max_depth, max_children): a random tree per sequence
+    page_size: int = 0               # > 0: the KV cache is a page pool read through a block table
 
     @property
     def torch_dtype(self):
@@ -83,6 +85,8 @@ WORKLOADS: Dict[str, Workload] = {
                          topk=(4, 4, 2, 2), match_prob=0.6),
     "stoch_b64": Workload("stoch_b64", 4, BF16, 64, 4096, 32000, 3, 32, 8, 128, 1024,
                           random_tree=(32, 4, 6), stochastic=True),
+    "ragged_paged_b8": Workload("ragged_paged_b8", 5, BF16, 8, 4096, 128256, 4, 32, 8, 128, 8192,
+                                prefix_range=(1024, 8192), ragged_trees=(32, 117, 5, 8), page_size=16),
 }
 
 
@@ -143,11 +147,24 @@ def tree_children(parents: Sequence[int]) -> List[List[int]]:
     return ch
 
 
-def workload_tree(w: Workload) -> List[int]:
+def workload_tree(w: Workload):
+    """The workload's tree (a parent list), or with ``ragged_trees`` one
+    parent list per sequence (sizes uniform in [T_min, T_max])."""
+    if w.ragged_trees is not None:
+        g = torch.Generator().manual_seed(1000 + w.seed)
+        lo, hi, md, mc = w.ragged_trees
+        return [random_tree_parents(int(torch.randint(lo, hi + 1, (1,), generator=g)), md, mc, gen=g)
+                for _ in range(w.B)]
     if w.topk is not None:
         return product_tree_parents(w.topk)
     g = torch.Generator().manual_seed(1000 + w.seed)
     return random_tree_parents(*w.random_tree, gen=g)
+
+
+def sequence_trees(w: Workload) -> List[List[int]]:
+    """Parent list of every sequence's tree (the shared tree repeated)."""
+    t = workload_tree(w)
+    return t if w.ragged_trees is not None else [t] * w.B
 
 
 # ----------------------------------------------------------------------------
@@ -213,18 +230,20 @@ def attention_inputs(w: Workload, T: int, device: str = "cpu", canary: Optional[
 
 
 def paged_cache(w: Workload, page_size: int, prefix_len: torch.Tensor, room: int = 64, extra_pages: int = 3,
-                device: str = "cpu", canary: Optional[float] = None) -> Dict[str, torch.Tensor]:
+                device: str = "cpu", canary: Optional[float] = None, capacity: int = 0) -> Dict[str, torch.Tensor]:
     """A page pool k_pages, v_pages [num_pages, Hkv, page_size, D] and a block
     table [B, max_pages] int32: sequence b owns ceil((prefix_len[b] + room) /
     page_size) pages taken from a seeded random permutation of the pool (its
     other table entries are -1), and `extra_pages` pages belong to nobody.
     With ``canary`` every slot no call may read (positions at or past each
-    sequence's prefix, unowned pages) holds that value."""
+    sequence's prefix, unowned pages) holds that value.  The table has room
+    for at least ``capacity`` positions per sequence (entries past the owned
+    pages are -1)."""
     dt = w.torch_dtype
     g = _gen(w.seed * 7919 + 9, "cpu")
     pl = [int(x) for x in prefix_len]
     need = [(n + room + page_size - 1) // page_size for n in pl]
-    max_pages = max(need)
+    max_pages = max(max(need), (capacity + page_size - 1) // page_size)
     num_pages = sum(need) + extra_pages
     perm = torch.randperm(num_pages, generator=g)
     table = torch.full((w.B, max_pages), -1, dtype=torch.int32)
@@ -270,15 +289,18 @@ def boosted_target_logits(w: Workload, parents: Sequence[int], node_tokens: torc
                           device: str = "cpu", boost: float = 10.0, seed_offset: int = 0) -> torch.Tensor:
     """[B,T,V] target logits ~ N(0,1) in the workload dtype; for each node
     with children, with probability ``match_prob`` one uniformly chosen
-    child's token gets ``boost`` added on the parent's row."""
+    child's token gets ``boost`` added on the parent's row.  ``parents`` may
+    be one parent list per sequence (T = the largest tree)."""
     g = _gen(w.seed * 7919 + 5 + seed_offset, device)
-    T = len(parents)
+    per_seq = len(parents) > 0 and hasattr(parents[0], "__len__")
+    trees = list(parents) if per_seq else [parents] * w.B
+    T = max(len(t) for t in trees)
     logits = _randn((w.B, T, w.V), g, dtype=torch.float32, device=device)
     gc = _gen(w.seed * 7919 + 6 + seed_offset, "cpu")
-    ch = tree_children(parents)
     nt = node_tokens.cpu()
     for b in range(w.B):
-        for u in range(T):
+        ch = tree_children(trees[b])
+        for u in range(len(trees[b])):
             if not ch[u]:
                 continue
             if float(torch.rand((1,), generator=gc)) < w.match_prob:

@@ -138,3 +138,52 @@ def test_paged_commit_refuses_a_block_it_does_not_own():
     torch.cuda.synchronize()
     assert int(out["status"].item()) & B.STATUS_CACHE_OVERFLOW
     assert out["new_prefix_len"].cpu().tolist() == [111, 13]
+
+
+def test_step_with_per_sequence_trees_and_paged_cache():
+    # the whole step (heads -> paged attention -> greedy verify -> paged commit)
+    # with a tree per sequence; verify and commit checked against the oracle
+    w = I.scaled(I.WORKLOADS["ragged_paged_b8"], B=3, d=256, V=1000, prefix_range=(100, 700))
+    trees = I.workload_tree(w)
+    T = max(len(t) for t in trees)
+    hin = {k: v.cuda() for k, v in I.head_inputs(w).items()}
+    ain = I.attention_inputs(w, T)
+    pc = I.paged_cache(w, w.page_size, ain["prefix_len"], room=T, capacity=w.max_prefix + T)
+    step = api.MedusaStep(B=w.B, d=w.d, V=w.V, K=w.K, Hq=w.Hq, Hkv=w.Hkv, D=w.D, S_max=w.S_max, parents=trees,
+                          dtype=w.torch_dtype, max_prefix=w.max_prefix, device="cuda", page_size=w.page_size,
+                          max_pages=pc["block_table"].shape[1], num_pages=pc["k_pages"].shape[0])
+    step.heads(hin["h"], hin["W_res"], hin["W_head"], hin["root_token"])
+    torch.cuda.synchronize()
+    node_tokens = step.node_tokens.cpu()
+    logits = I.boosted_target_logits(w, trees, node_tokens)
+    kp, vp, bt = pc["k_pages"].cuda(), pc["v_pages"].cuda(), pc["block_table"].cuda()
+    dev = {k: v.cuda() for k, v in ain.items()}
+    new_pl = torch.empty_like(dev["prefix_len"])
+    step.run(h=hin["h"], W_res=hin["W_res"], W_head=hin["W_head"], root_token=hin["root_token"], q=dev["q"],
+             k_tree=dev["k_tree"], v_tree=dev["v_tree"], k_cache=kp, v_cache=vp, prefix_len=dev["prefix_len"],
+             new_prefix_len=new_pl, target=logits.cuda(), block_table=bt)
+    torch.cuda.synchronize()
+    assert int(step.status.item()) == 0
+    maxd = step.tree.max_depth
+    path = np.full((w.B, maxd), -1, np.int32)
+    ln = np.zeros(w.B, np.int32)
+    for b, par in enumerate(trees):
+        Tb = len(par)
+        pb, lb, _ = oracle.verify_greedy(logits[b:b + 1, :Tb], node_tokens[b:b + 1, :Tb], par, maxd)
+        path[b], ln[b] = pb[0], lb[0]
+    assert np.array_equal(step.accept_path.cpu().numpy(), path)
+    rk, rv, npl, st = oracle.kv_commit_paged(pc["k_pages"], pc["v_pages"], ain["k_tree"], ain["v_tree"],
+                                             pc["block_table"], path, ln, ain["prefix_len"])
+    assert st == 0 and new_pl.cpu().tolist() == npl.tolist()
+    assert torch.equal(kp.cpu(), rk) and torch.equal(vp.cpu(), rv)
+    # the attention output against the oracle on the gathered cache, per sequence
+    S_max = pc["block_table"].shape[1] * w.page_size
+    kc = oracle.gather_pages(pc["k_pages"], pc["block_table"], ain["prefix_len"], S_max)
+    vc = oracle.gather_pages(pc["v_pages"], pc["block_table"], ain["prefix_len"], S_max)
+    o = step.attn_out.float().cpu()
+    for b, par in enumerate(trees):
+        Tb = len(par)
+        ref_o, _ = oracle.tree_attention(ain["q"][b:b + 1, :Tb], ain["k_tree"][b:b + 1, :Tb],
+                                         ain["v_tree"][b:b + 1, :Tb], kc[b:b + 1], vc[b:b + 1],
+                                         ain["prefix_len"][b:b + 1], par)
+        assert_float_parity(o[b, :Tb].reshape(-1, w.D), ref_o, w.torch_dtype, f"out[{b}]")
