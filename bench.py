@@ -35,10 +35,10 @@ METRIC = "Medusa verify steps/s (8B shape, 117-node tree); tree-attn HBM GB/s vs
 UNIT = "steps/s"
 WORKLOAD = "llama8b"
 # DRAM bytes (read + write) per launch of the heads kernel, from an ncu capture
-# of the same kernel at V=32000 (1.18303 GB read + 3.86 MB written against
+# of the same kernel at V=32000 (1.18539 GB read + 4.34 MB written against
 # 1.18279 GB of weights), scaled to the workload's weight bytes; only for the
 # workload whose launch configuration (B=1, d=4096, K=4) was captured.
-HEADS_DRAM_BYTES = {}  # refreshed from the capture of the current kernel
+HEADS_DRAM_BYTES = {"llama8b": 4336910336 * (1185393000 + 4339712) / 1182793728}
 
 
 def peaks():
