@@ -400,6 +400,23 @@ def run_mine(args, rank, world, local_rank):
     for ev in used:
         ev.record(main_stream)
 
+    def run_kwargs(slot):
+        d = dev_in[slot]
+        return dict(h=d["h"], W_res=hin["W_res"], W_head=hin["W_head"], root_token=d["root_token"], q=d["q"],
+                    k_tree=d["k_tree"], v_tree=d["v_tree"], k_cache=ain["k_cache"], v_cache=ain["v_cache"],
+                    prefix_len=ain["prefix_len"], new_prefix_len=new_pl, target=d["target"],
+                    q_draft=d.get("q_draft"), node_tokens=d.get("tokens"), block_table=block_table)
+
+    # one CUDA graph per input slot: a step is one graph launch on the host
+    graphs, e2e_mode = None, "cuda-graph"
+    try:
+        torch.cuda.synchronize()
+        graphs = [step.capture(**run_kwargs(slot)) for slot in range(2)]
+        torch.cuda.synchronize()
+    except Exception as exc:  # capture unsupported here: the four calls are issued eagerly
+        graphs, e2e_mode = None, f"eager ({type(exc).__name__})"
+        torch.cuda.synchronize()
+
     def e2e_step(i):
         slot = i & 1
         with torch.cuda.stream(copy_stream):
@@ -408,11 +425,10 @@ def run_mine(args, rank, world, local_rank):
                 dev_in[slot][n].copy_(host_in[n], non_blocking=True)
             copied[slot].record(copy_stream)
         main_stream.wait_event(copied[slot])
-        d = dev_in[slot]
-        step.run(h=d["h"], W_res=hin["W_res"], W_head=hin["W_head"], root_token=d["root_token"], q=d["q"],
-                 k_tree=d["k_tree"], v_tree=d["v_tree"], k_cache=ain["k_cache"], v_cache=ain["v_cache"],
-                 prefix_len=ain["prefix_len"], new_prefix_len=new_pl, target=d["target"],
-                 q_draft=d.get("q_draft"), node_tokens=d.get("tokens"), block_table=block_table)
+        if graphs is not None:
+            graphs[slot].replay()
+        else:
+            step.run(**run_kwargs(slot))
         used[slot].record(main_stream)
         for o, ho in zip(outs, host_out):
             ho.copy_(o, non_blocking=True)
@@ -484,7 +500,8 @@ def run_mine(args, rank, world, local_rank):
                      "tree_verify": stage[2] * 1e6, "kv_commit": stage[3] * 1e6},
         "mean_accept_len": mean_len,
         "tokens_per_s": value * w.B * (mean_len + 1),
-        "e2e": {"value": value_e2e, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "e2e": {"value": value_e2e, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "mode": e2e_mode},
         "gpu_launches": K * launches_per_step(w),
         "clocks": clk,
     }

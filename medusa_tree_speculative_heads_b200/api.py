@@ -224,6 +224,15 @@ class MedusaStep:
         _b.kv_commit(k_cache, v_cache, k_tree, v_tree, self.accept_path, self.max_path, self.accept_len, prefix_len,
                      new_prefix_len, self.B, self.T, self.Hkv, self.D, self.S_max, self.dt, self.status)
 
+    def capture(self, **run_kwargs) -> "torch.cuda.CUDAGraph":
+        """A CUDA graph of ``run(**run_kwargs)`` (the same buffers every
+        replay): one launch per step instead of the four calls' host work.
+        The buffers must stay allocated while the graph is used."""
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self.run(**run_kwargs)
+        return g
+
     def run(self, *, h, W_res, W_head, root_token, q, k_tree, v_tree, k_cache, v_cache, prefix_len, new_prefix_len,
             target, q_draft=None, q_row=None, seed: int = 0, step: int = 0, node_tokens=None, block_table=None):
         self.heads(h, W_res, W_head, root_token)

@@ -66,3 +66,52 @@ def test_whole_step_matches_oracle(name):
         assert np.array_equal(chain["bonus"], obonus)
         assert np.array_equal(chain["npl"], onpl)
         assert torch.equal(chain["kc"], okc) and torch.equal(chain["vc"], ovc)
+
+
+@pytest.mark.parametrize("name", ["llama8b_small", "stoch_small"])
+def test_graph_replay_equals_eager_step(name):
+    # the step captured in a CUDA graph and replayed gives the eager step's
+    # results bit for bit (the kernels are deterministic)
+    if name == "llama8b_small":
+        w = I.scaled(I.WORKLOADS["llama8b"], B=2, d=512, V=3001, prefix=300)
+    else:
+        w = I.scaled(I.WORKLOADS["stoch_b64"], B=3, V=900)
+    parents = I.workload_tree(w)
+    T = len(parents)
+    from medusa_tree_speculative_heads_b200 import binding as Bnd
+    mode = Bnd.STOCHASTIC if w.stochastic else Bnd.GREEDY
+    step = MedusaStep(B=w.B, d=w.d, V=w.V, K=w.K, Hq=w.Hq, Hkv=w.Hkv, D=w.D, S_max=w.S_max, parents=parents,
+                      dtype=w.torch_dtype, device="cuda", mode=mode, q_rows=T)
+    hin = {k: v.cuda() for k, v in I.head_inputs(w).items()}
+    ain = {k: v.cuda() for k, v in I.attention_inputs(w, T).items()}
+    if w.stochastic:
+        sd = {k: v.cuda() for k, v in I.stochastic_inputs(w, parents).items()}
+        target, q_draft, tok = sd["p"], sd["q"], sd["node_tokens"]
+    else:
+        target = torch.randn((w.B, T, w.V), generator=torch.Generator().manual_seed(2)).to(w.torch_dtype).cuda()
+        q_draft = tok = None
+    new_pl = torch.empty_like(ain["prefix_len"])
+    k0, v0 = ain["k_cache"].clone(), ain["v_cache"].clone()
+    kw = dict(h=hin["h"], W_res=hin["W_res"], W_head=hin["W_head"], root_token=hin["root_token"], q=ain["q"],
+              k_tree=ain["k_tree"], v_tree=ain["v_tree"], k_cache=ain["k_cache"], v_cache=ain["v_cache"],
+              prefix_len=ain["prefix_len"], new_prefix_len=new_pl, target=target, q_draft=q_draft,
+              node_tokens=tok, step=5)
+    step.run(**kw)
+    torch.cuda.synchronize()
+    eager = [x.clone() for x in (step.node_tokens, step.attn_out, step.accept_path, step.accept_len, step.bonus,
+                                 new_pl, ain["k_cache"])]
+    ain["k_cache"].copy_(k0)
+    ain["v_cache"].copy_(v0)
+    for x in (step.node_tokens, step.attn_out, step.accept_path, step.accept_len, step.bonus, new_pl):
+        x.zero_()
+    g = step.capture(**kw)
+    torch.cuda.synchronize()
+    ain["k_cache"].copy_(k0)  # capture does not run the kernels; replay twice from the same state
+    ain["v_cache"].copy_(v0)
+    g.replay()
+    g.replay()
+    torch.cuda.synchronize()
+    assert int(step.status.item()) == 0
+    replay = (step.node_tokens, step.attn_out, step.accept_path, step.accept_len, step.bonus, new_pl, ain["k_cache"])
+    for a, b in zip(eager, replay):
+        assert torch.equal(a, b)
