@@ -97,3 +97,29 @@ def test_workspace_queries_are_pure(lib):
     b = lib.medusa_heads_workspace_size(1, 4096, 128256, 4, 1)
     assert a == b and a > 0
     assert lib.medusa_heads_workspace_size(0, 4096, 128256, 4, 1) == 0
+
+
+def test_paged_calls_validate_before_launch(lib):
+    # every one of these fails on the host, before any device work
+    fake = ctypes.c_void_p(0x1000)
+    nul = None
+    # NULL block table
+    assert lib.tree_attention_paged(fake, fake, fake, fake, fake, nul, 4, 16, 8, fake, 1, 4, 2, 128, 0, ctypes.c_float(0),
+                                    1, nul, fake, nul, fake, 1 << 20, nul, nul) == B.MEDUSA_ERR_INVALID_ARG
+    assert b"NULL" in lib.medusa_last_error()
+    assert lib.kv_commit_paged(fake, fake, fake, fake, nul, 4, 16, 8, fake, 3, fake, fake, fake, 1, 7, 2, 128, 1, nul,
+                               nul) == B.MEDUSA_ERR_INVALID_ARG
+    # bad page geometry
+    assert lib.kv_commit_paged(fake, fake, fake, fake, fake, 4, 0, 8, fake, 3, fake, fake, fake, 1, 7, 2, 128, 1, nul,
+                               nul) == B.MEDUSA_ERR_INVALID_ARG
+    assert lib.kv_commit_paged(fake, fake, fake, fake, fake, 0, 16, 8, fake, 3, fake, fake, fake, 1, 7, 2, 128, 1,
+                               nul, nul) == B.MEDUSA_ERR_INVALID_ARG
+    # a K/V row that is not a multiple of 16 bytes
+    assert lib.kv_commit_paged(fake, fake, fake, fake, fake, 4, 16, 8, fake, 3, fake, fake, fake, 1, 7, 2, 4, 1, nul,
+                               nul) == B.MEDUSA_ERR_INVALID_ARG
+    # unknown dtype
+    assert lib.kv_commit_paged(fake, fake, fake, fake, fake, 4, 16, 8, fake, 3, fake, fake, fake, 1, 7, 2, 128, 9, nul,
+                               nul) == B.MEDUSA_ERR_UNSUPPORTED
+    # the paged workspace query mirrors the contiguous one's domain
+    assert lib.tree_attention_paged_workspace_size(1, 4, 2, 96, 0, 4, 16, nul, 1) == 0
+    assert lib.tree_attention_paged_workspace_size(1, 4, 2, 128, 0, 0, 16, nul, 1) == 0
