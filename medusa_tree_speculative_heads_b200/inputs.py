@@ -17,13 +17,19 @@ Workloads (all synthetic, no dataset or trained weights exist for them):
 * ``stoch_b64`` bf16, B=64, d=4096, V=32000, K=3, a seeded random 32-node tree
   (depth <= 4 counting the root as 1, <= 6 children), 32/8 heads, head_dim
   128, prefix 1024, stochastic verification.
+* ``stoch_logits_b64`` stoch_b64 with verification reading the target's bf16
+  logits at temperature 0.7 instead of fp32 probabilities.
+* ``ragged_paged_b8`` bf16, B=8, the llama8b shapes, a random tree per
+  sequence (32 to 117 nodes, depth <= 5, <= 8 children), prefix uniform in
+  [1024, 8192], the KV cache in 16-row pages read through a block table.
 
 Value distributions: hidden state and all attention tensors N(0,1); head
 weights N(0, 1/d).  Greedy target logits are N(0,1) and, for every node that
 has children, with the workload's match probability one uniformly chosen
 child's token gets +10 on the parent's row.  Stochastic targets: logit of a
 token = -1.1 ln(rank) + N(0, variance 0.5) over a per-row random ranking,
-p = softmax(logit / 0.7) in fp32; the draft is q = 0.7 p + 0.3 Zipf(1.1) on an
+p = softmax(logit / 0.7) in fp32 (the logits themselves for the logits form);
+the draft is q = 0.7 p + 0.3 Zipf(1.1) on an
 independent ranking; every child token is drawn from q at its parent.
 """
 from __future__ import annotations
@@ -58,6 +64,7 @@ class Workload:
     stochastic: bool = False
     ragged_trees: Optional[tuple] = None   # (T_min, T_max, max_depth, max_children): a random tree per sequence
     page_size: int = 0               # > 0: the KV cache is a page pool read through a block table
+    temperature: float = 0.0         # > 0: stochastic verification reads bf16 target logits at this temperature
 
     @property
     def torch_dtype(self):
@@ -85,6 +92,8 @@ WORKLOADS: Dict[str, Workload] = {
                          topk=(4, 4, 2, 2), match_prob=0.6),
     "stoch_b64": Workload("stoch_b64", 4, BF16, 64, 4096, 32000, 3, 32, 8, 128, 1024,
                           random_tree=(32, 4, 6), stochastic=True),
+    "stoch_logits_b64": Workload("stoch_logits_b64", 4, BF16, 64, 4096, 32000, 3, 32, 8, 128, 1024,
+                                 random_tree=(32, 4, 6), stochastic=True, temperature=0.7),
     "ragged_paged_b8": Workload("ragged_paged_b8", 5, BF16, 8, 4096, 128256, 4, 32, 8, 128, 8192,
                                 prefix_range=(1024, 8192), ragged_trees=(32, 117, 5, 8), page_size=16),
 }
@@ -309,15 +318,20 @@ def boosted_target_logits(w: Workload, parents: Sequence[int], node_tokens: torc
     return logits.to(w.torch_dtype)
 
 
+STOCH_TEMPERATURE = 0.7   # the target's sampling temperature in stochastic_inputs
+
+
 def stochastic_inputs(w: Workload, parents: Sequence[int], device: str = "cpu") -> Dict[str, torch.Tensor]:
     """p, q [B,T,V] fp32 and node_tokens [B,T] (children drawn from q at
-    their parent; the root token uniform)."""
+    their parent; the root token uniform); also the target's logits [B,T,V]
+    fp32 with p = softmax(logits / STOCH_TEMPERATURE)."""
     g = _gen(w.seed * 7919 + 7, "cpu")
     T = len(parents)
     V = w.V
     ranks = torch.arange(1, V + 1, dtype=torch.float64)
     p = torch.empty((w.B, T, V), dtype=torch.float32)
     q = torch.empty((w.B, T, V), dtype=torch.float32)
+    logits = torch.empty((w.B, T, V), dtype=torch.float32)
     zipf = ranks.pow(-1.1)
     zipf = (zipf / zipf.sum()).to(torch.float32)
     for b in range(w.B):
@@ -326,7 +340,8 @@ def stochastic_inputs(w: Workload, parents: Sequence[int], device: str = "cpu") 
             logit = torch.empty(V, dtype=torch.float32)
             logit[perm] = (-1.1 * torch.log(ranks)).to(torch.float32)
             logit += torch.randn(V, generator=g) * math.sqrt(0.5)
-            p[b, u] = torch.softmax(logit / 0.7, dim=0)
+            logits[b, u] = logit
+            p[b, u] = torch.softmax(logit / STOCH_TEMPERATURE, dim=0)
             perm2 = torch.randperm(V, generator=g)
             z = torch.empty(V, dtype=torch.float32)
             z[perm2] = zipf
@@ -340,4 +355,4 @@ def stochastic_inputs(w: Workload, parents: Sequence[int], device: str = "cpu") 
                 draws = torch.multinomial(q[b, u].double(), len(ch[u]), replacement=True, generator=g)
                 for c, t in zip(ch[u], draws.tolist()):
                     tok[b, c] = t
-    return {"p": p.to(device), "q": q.to(device), "node_tokens": tok.to(device)}
+    return {"p": p.to(device), "q": q.to(device), "node_tokens": tok.to(device), "logits": logits.to(device)}

@@ -59,6 +59,10 @@ def lib():
         L.orc_philox4x32_10.restype = None
         L.orc_verify_stochastic.argtypes = [vp, vp, i32, vp, vp, i32, i32, i32, vp, u64, u32, i32, vp, vp, vp,
                                             vp, i32]
+        L.orc_verify_stochastic_logits.argtypes = [vp, i32, dbl, vp, i32, vp, vp, i32, i32, i32, vp, u64, u32,
+                                                   i32, vp, vp, vp, vp, i32]
+        L.orc_softmax_temperature.argtypes = [vp, i32, dbl, vp]
+        L.orc_softmax_temperature.restype = None
         L.orc_kv_commit.argtypes = [vp, vp, vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]
         L.orc_kv_commit.restype = None
         L.orc_gather_pages.argtypes = [vp, vp, i32, i32, i32, vp, i32, i32, i32, i32, i32, vp]
@@ -269,6 +273,41 @@ def verify_stochastic(p, q, node_tokens, parents, seed: int, step: int, max_path
     rc = lib().orc_verify_stochastic(_p(pa), _p(qa), Qrows, _p(qr), _p(nt), B, T, V, _p(par),
                                      ctypes.c_uint64(seed & (2**64 - 1)), ctypes.c_uint32(step & 0xFFFFFFFF),
                                      max_path, _p(path), _p(ln), _p(bonus), _p(status), int(b0))
+    if rc != 0:
+        raise ValueError("bad verify arguments")
+    return path, ln, bonus, int(status[0])
+
+
+def softmax_temperature(z, temperature: float):
+    """fp64 P = softmax((z - max z) / tau) of one logits row (numpy f64)."""
+    za = np.ascontiguousarray(np.asarray(z, dtype=np.float64))
+    out = np.empty_like(za)
+    lib().orc_softmax_temperature(_p(za), za.shape[0], ctypes.c_double(1.0 / temperature), _p(out))
+    return out
+
+
+def verify_stochastic_logits(logits, temperature: float, q, node_tokens, parents, seed: int, step: int,
+                             max_path: int, q_row=None, b0: int = 0):
+    """verify_stochastic with every visited node's target distribution taken
+    as softmax(logits row / temperature) in fp64 (logits f32 or bf16 torch)."""
+    lg = logits.detach().cpu().contiguous()
+    dt = BF16 if lg.dtype == torch.bfloat16 else F32
+    if dt == F32:
+        lg = lg.float()
+    qa = _f32(q)
+    B, T, V = lg.shape
+    Qrows = qa.shape[1]
+    nt = _i32(node_tokens)
+    par = _i32(parents)
+    qr = None if q_row is None else _i32(q_row)
+    path = np.zeros((B, max_path), np.int32)
+    ln = np.zeros(B, np.int32)
+    bonus = np.zeros(B, np.int32)
+    status = np.zeros(1, np.int32)
+    rc = lib().orc_verify_stochastic_logits(ctypes.c_void_p(lg.data_ptr()), dt, ctypes.c_double(temperature),
+                                            _p(qa), Qrows, _p(qr), _p(nt), B, T, V, _p(par),
+                                            ctypes.c_uint64(seed & (2**64 - 1)), ctypes.c_uint32(step & 0xFFFFFFFF),
+                                            max_path, _p(path), _p(ln), _p(bonus), _p(status), int(b0))
     if rc != 0:
         raise ValueError("bad verify arguments")
     return path, ln, bonus, int(status[0])

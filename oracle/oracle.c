@@ -488,10 +488,32 @@ uint64_t orc_residual(const double* P, const float* Q, int V, double* out, uint6
  * Outputs as for orc_verify_greedy; status bit 1 is set when a bonus
  * distribution has zero total weight (bonus 0 then).
  */
-int orc_verify_stochastic(const float* p, const float* q, int Qrows, const int32_t* q_row,
-                          const int32_t* node_tokens, int B, int T, int V, const int32_t* parent,
-                          uint64_t seed, uint32_t step, int max_path, int32_t* path, int32_t* len,
-                          int32_t* bonus, int32_t* status, int b0) {
+void orc_softmax_temperature(const double* z, int V, double inv_tau, double* P);
+
+/* where the walk's target rows come from: fp32 probabilities p, or logits
+ * turned into probabilities by orc_softmax_temperature */
+typedef struct {
+    const float* p;      /* [B, T, V] f32, or NULL */
+    const void* logits;  /* [B, T, V] of dtype `dtype` when p is NULL */
+    int dtype;
+    double inv_tau;
+} row_source;
+
+static void load_row(const row_source* src, size_t row, int V, double* P) {
+    if (src->p) {
+        for (int y = 0; y < V; ++y) P[y] = (double)src->p[row * V + y];
+        return;
+    }
+    double* z = (double*)malloc(sizeof(double) * (size_t)V);
+    for (int y = 0; y < V; ++y) z[y] = load(src->logits, src->dtype, row * V + y);
+    orc_softmax_temperature(z, V, src->inv_tau, P);
+    free(z);
+}
+
+static int stochastic_walk(const row_source* src, const float* q, int Qrows, const int32_t* q_row,
+                           const int32_t* node_tokens, int B, int T, int V, const int32_t* parent,
+                           uint64_t seed, uint32_t step, int max_path, int32_t* path, int32_t* len,
+                           int32_t* bonus, int32_t* status, int b0) {
     int32_t* depth = (int32_t*)malloc(sizeof(int32_t) * T);
     int32_t* rank = (int32_t*)malloc(sizeof(int32_t) * T);
     double* P = (double*)malloc(sizeof(double) * (size_t)V);
@@ -503,7 +525,7 @@ int orc_verify_stochastic(const float* p, const float* q, int Qrows, const int32
         int u = 0, L = 1;
         for (int t = 0; t < max_path; ++t) path[(size_t)b * max_path + t] = -1;
         path[(size_t)b * max_path] = 0;
-        for (int y = 0; y < V; ++y) P[y] = (double)p[((size_t)b * T + u) * V + y];
+        load_row(src, (size_t)b * T + u, V, P);
         for (;;) {
             int qr = q_row ? q_row[u] : u;
             if (qr < 0 || qr >= Qrows) {
@@ -530,7 +552,7 @@ int orc_verify_stochastic(const float* p, const float* q, int Qrows, const int32
                     }
                     path[(size_t)b * max_path + L] = c;
                     ++L;
-                    for (int y = 0; y < V; ++y) P[y] = (double)p[((size_t)b * T + u) * V + y];
+                    load_row(src, (size_t)b * T + u, V, P);
                     moved = 1;
                     break;
                 }
@@ -570,6 +592,53 @@ int orc_verify_stochastic(const float* p, const float* q, int Qrows, const int32
     free(P);
     free(W);
     return rc;
+}
+
+int orc_verify_stochastic(const float* p, const float* q, int Qrows, const int32_t* q_row,
+                          const int32_t* node_tokens, int B, int T, int V, const int32_t* parent,
+                          uint64_t seed, uint32_t step, int max_path, int32_t* path, int32_t* len,
+                          int32_t* bonus, int32_t* status, int b0) {
+    row_source src = {p, NULL, 0, 1.0};
+    return stochastic_walk(&src, q, Qrows, q_row, node_tokens, B, T, V, parent, seed, step, max_path, path, len,
+                           bonus, status, b0);
+}
+
+/*
+ * Target distribution from logits at temperature tau (reading: the pages
+ * write P_target without saying how it is obtained from the target model's
+ * logits; the plain softmax, tau = 1, is the pages' case, and tau > 0 is the
+ * usual sampling temperature):
+ *     m = max_y z(y),  e(y) = exp((z(y) - m) * (1/tau)),  Z = sum_y e(y)
+ *     P(y) = e(y) * (1/Z)
+ * in fp64, every product and difference rounded once, Z summed in index
+ * order; inv_tau = 1/tau is passed in.  NaN logits are skipped by the max
+ * and make P NaN (no mass), as does a row without a finite maximum.
+ */
+void orc_softmax_temperature(const double* z, int V, double inv_tau, double* P) {
+    double m = -INFINITY;
+    for (int y = 0; y < V; ++y) m = fmax(m, z[y]);
+    double Z = 0.0;
+    for (int y = 0; y < V; ++y) {
+        P[y] = exp((z[y] - m) * inv_tau);
+        Z += P[y];
+    }
+    const double r = 1.0 / Z;
+    for (int y = 0; y < V; ++y) P[y] = P[y] * r;
+}
+
+/*
+ * Stochastic verification reading the target's logits: the walk of
+ * orc_verify_stochastic with each visited node's P computed from its logits
+ * row by orc_softmax_temperature (logits dtype 0 = f32, 1 = bf16).
+ */
+int orc_verify_stochastic_logits(const void* logits, int dtype, double temperature, const float* q, int Qrows,
+                                 const int32_t* q_row, const int32_t* node_tokens, int B, int T, int V,
+                                 const int32_t* parent, uint64_t seed, uint32_t step, int max_path, int32_t* path,
+                                 int32_t* len, int32_t* bonus, int32_t* status, int b0) {
+    if (!(temperature > 0.0) || !isfinite(temperature)) return -1;
+    row_source src = {NULL, logits, dtype, 1.0 / temperature};
+    return stochastic_walk(&src, q, Qrows, q_row, node_tokens, B, T, V, parent, seed, step, max_path, path, len,
+                           bonus, status, b0);
 }
 
 /* ------------------------------------------------------------------------ */

@@ -789,3 +789,126 @@ def test_paged_commit_equals_contiguous_commit_through_the_table(orc):
     before = orc.gather_pages(pc["k_pages"], pc["block_table"], torch.tensor([0, 28, 0], dtype=torch.int32), 28)
     after = orc.gather_pages(kp4, pc["block_table"], torch.tensor([0, 28, 0], dtype=torch.int32), 28)
     assert torch.equal(before[1], after[1])
+
+
+# ----------------------------------------------------------------------------
+# stochastic verification from logits at a temperature
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("tau", [1.0, 0.7, 2.5])
+def test_softmax_temperature_vs_scipy(orc, tau):
+    # P = softmax(z / tau): the library routine on the same fp64 values
+    from scipy.special import softmax
+    rng = np.random.default_rng(31)
+    z = rng.normal(0.0, 3.0, 5000)
+    z[::97] = -np.inf                                   # masked entries get exactly zero mass
+    P = orc.softmax_temperature(z, tau)
+    want = softmax(z / tau)
+    assert np.abs(P - want).max() <= 1e-15 + 1e-13 * want.max()
+    assert (P[::97] == 0).all()
+    assert abs(P.sum() - 1.0) < 1e-12
+    # one finite entry: a point mass
+    z1 = np.full(9, -np.inf)
+    z1[4] = -12.5
+    assert orc.softmax_temperature(z1, tau).tolist() == [0, 0, 0, 0, 1.0, 0, 0, 0, 0]
+
+
+def _distinct_sibling_tokens(parents, B, V, rng, favour=None, p_favour=0.0):
+    """node tokens [B,T]: siblings distinct; with probability p_favour a
+    child gets favour[b, parent] (when no sibling holds it yet)."""
+    T = len(parents)
+    ch = I.tree_children(parents)
+    tok = np.zeros((B, T), np.int32)
+    for b in range(B):
+        tok[b, 0] = rng.integers(V)
+        for u in range(T):
+            used = set()
+            for c in ch[u]:
+                if favour is not None and favour[b, u] not in used and rng.random() < p_favour:
+                    t = int(favour[b, u])
+                else:
+                    t = int(rng.integers(V))
+                    while t in used:
+                        t = int(rng.integers(V))
+                used.add(t)
+                tok[b, c] = t
+    return tok
+
+
+def test_stochastic_logits_cold_limit_is_greedy(orc):
+    # tau -> 0: gaps of at least 1 between the largest logit and the rest make
+    # exp((z - m) / tau) underflow to 0, so P is the argmax point mass; a child
+    # is then accepted iff its token is the parent's argmax (u * Q(x) < 1),
+    # the residual keeps that point mass, and the bonus is the argmax: the
+    # walk is greedy verification (siblings carry distinct tokens)
+    B, V = 24, 64
+    par = I.product_tree_parents((3, 2, 2))
+    T = len(par)
+    rng = np.random.default_rng(41)
+    z = rng.normal(0.0, 1.0, (B, T, V)).astype(np.float32)
+    top = rng.integers(V, size=(B, T))
+    z[np.arange(B)[:, None], np.arange(T)[None, :], top] = z.max(axis=-1) + 1.5
+    tok = _distinct_sibling_tokens(par, B, V, rng, favour=top, p_favour=0.6)
+    q = rng.random((B, T, V)).astype(np.float32)
+    q /= q.sum(-1, keepdims=True)
+    maxd = int(max(orc.tree_shape(par)[0]))
+    gpath, glen, gbonus = orc.verify_greedy(torch.from_numpy(z), torch.from_numpy(tok), par, maxd)
+    for seed in (3, 2**63 + 11):
+        path, ln, bonus, st = orc.verify_stochastic_logits(torch.from_numpy(z), 1e-3, q, tok, par, seed, 5, maxd)
+        assert st == 0
+        assert np.array_equal(path, gpath) and np.array_equal(ln, glen) and np.array_equal(bonus, gbonus)
+    assert len(set(glen.tolist())) > 2   # the cases reach several depths
+
+
+def test_stochastic_logits_temperature_scaling_and_shift(orc):
+    # P depends on z only through (z - max z) / tau: (2z, 2 tau) and (z + 8, tau)
+    # give the same walk bit for bit (z on a 2^-12 grid, so every shift and
+    # doubling is exact), bf16 logits give what their fp32 widening gives, and
+    # another temperature changes the walk
+    w = I.scaled(I.WORKLOADS["stoch_b64"], B=6, V=400)
+    par = I.workload_tree(w)
+    d = I.stochastic_inputs(w, par)
+    z = torch.round(d["logits"] * 4096) / 4096
+    maxd = int(max(orc.tree_shape(par)[0]))
+
+    def walk(zz, tau):
+        return orc.verify_stochastic_logits(zz, tau, d["q"], d["node_tokens"], par, 17, 2, maxd)[:3]
+
+    base = walk(z, 0.7)
+    for other in (walk(z * 2, 1.4), walk(z + 8.0, 0.7)):
+        assert all(np.array_equal(x, y) for x, y in zip(base, other))
+    zb = z.bfloat16()
+    assert all(np.array_equal(x, y) for x, y in zip(walk(zb, 0.7), walk(zb.float(), 0.7)))
+    assert not all(np.array_equal(x, y) for x, y in zip(base, walk(z, 3.0)))
+
+
+def test_stochastic_logits_first_token_follows_target(orc):
+    # [SPEC] "The Acceptance Sampling Rule (Zero Distributional Drift)" with P
+    # from logits: z = tau * log(P8) makes softmax(z / tau) = P8, so the first
+    # emitted token must follow P8 (3 drafted children from Q8)
+    N, V, tau = 300_000, 8, 0.6
+    par = [-1, 0, 0, 0]
+    rng = np.random.default_rng(7)
+    z = np.broadcast_to((tau * np.log(P8.astype(np.float64))).astype(np.float32), (N, 4, V)).copy()
+    q = np.broadcast_to(Q8, (N, 4, V)).copy()
+    tok = np.zeros((N, 4), np.int32)
+    tok[:, 1:] = rng.choice(V, size=(N, 3), p=Q8.astype(np.float64) / Q8.sum())
+    path, ln, bonus, st = orc.verify_stochastic_logits(torch.from_numpy(z), tau, q, tok, par, 99, 1, 2)
+    assert st == 0
+    first = np.where(ln >= 2, tok[np.arange(N), np.maximum(path[:, 1], 0)], bonus)
+    assert _chi2_pvalue(np.bincount(first, minlength=V), P8.astype(np.float64)) > 1e-3
+
+
+def test_stochastic_logits_rows_without_mass(orc):
+    # a row of -inf logits has no finite maximum: no child is accepted there
+    # and the bonus reports no mass
+    V = 16
+    par = [-1, 0]
+    z = torch.zeros((2, 2, V))
+    z[0, 0] = -float("inf")
+    q = np.full((2, 2, V), 1.0 / V, np.float32)
+    tok = np.array([[0, 3], [0, 3]], np.int32)
+    path, ln, bonus, st = orc.verify_stochastic_logits(z, 1.0, q, tok, par, 1, 0, 2)
+    assert ln[0] == 1 and bonus[0] == 0 and st == 1
+    path, ln, bonus, st = orc.verify_stochastic_logits(z[1:], 1.0, q[1:], tok[1:], par, 1, 0, 2, b0=1)
+    assert st == 0
