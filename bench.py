@@ -140,6 +140,9 @@ class OracleSample:
         res = w.K * w.d * w.d
         self.frac = (res + lm * self.Vs / w.V + att * nr / n_rows) / (res + lm + att)
         self.logits = None
+        # stochastic workloads verify the harness's drafted tokens against its
+        # target (probabilities, or logits at the temperature), whole
+        self.sd = I.stochastic_inputs(w, self.parents) if w.stochastic else None
 
     def run(self):
         import numpy as np
@@ -160,7 +163,7 @@ class OracleSample:
         else:
             otok, _ = oracle.tree_fill(self.parents, hin["root_token"], otop, otp)
         t1 = time.perf_counter()
-        if self.logits is None:   # the target model's logits: input generation, not timed
+        if self.logits is None and self.sd is None:   # the target model's logits: input generation, not timed
             self.logits = I.boosted_target_logits(self.ws, self.parents, torch.from_numpy(otok))
         t2 = time.perf_counter()
         kc, vc = ain["k_cache"], ain["v_cache"]
@@ -187,6 +190,14 @@ class OracleSample:
                 Tb = len(trees[b])
                 pb, lb, _ = oracle.verify_greedy(self.logits[b:b + 1, :Tb], otok[b:b + 1, :Tb], trees[b], maxd)
                 path[b], ln[b] = pb[0], lb[0]
+        elif self.sd is not None:
+            sd = self.sd
+            if w.temperature > 0:
+                path, ln, _, _ = oracle.verify_stochastic_logits(sd["logits"].bfloat16(), w.temperature, sd["q"],
+                                                                 sd["node_tokens"], self.parents, 0, 0, maxd)
+            else:
+                path, ln, _, _ = oracle.verify_stochastic(sd["p"], sd["q"], sd["node_tokens"], self.parents, 0, 0,
+                                                          maxd)
         else:
             path, ln, _ = oracle.verify_greedy(self.logits, otok, self.parents, maxd)
         if self.pc is not None:
@@ -216,7 +227,7 @@ def run_reference(args, rank, world):
         tot_f += f
     value = tot_f / tot_t
     sample = (f"per step: fp64 oracle on the host, residual block of all {w.K} heads, LM-head rows of a 1/64 "
-              f"vocabulary slice, attention of 1/64 of the query rows, full greedy verify and commit; "
+              f"vocabulary slice, attention of 1/64 of the query rows, full verify and commit; "
               f"steps/s scaled by the sampled fraction of the step's work")
     out = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 / value, "higher_is_better": True,
@@ -258,7 +269,11 @@ def config_dict(w, world):
     if w.page_size:
         tree += f", KV in pages of {w.page_size} via a block table"
     prefix = f"prefix U[{w.prefix_range[0]}, {w.prefix_range[1]}]" if w.prefix_range else f"prefix {w.prefix}"
-    verify = "stochastic verify" if w.stochastic else f"greedy verify, match prob {w.match_prob}"
+    if w.stochastic:
+        verify = ("stochastic verify from bf16 logits at temperature " + f"{w.temperature}" if w.temperature > 0
+                  else "stochastic verify from fp32 probabilities")
+    else:
+        verify = f"greedy verify, match prob {w.match_prob}"
     head_gb = w.K * (w.d * w.d + w.V * w.d) * (2 if w.dtype == "bf16" else 4) / 1e9
     shape = tree if w.ragged_trees else f"{tree} -> {T}-node tree"
     return {"workload": (f"{w.name}: B={w.B} d={w.d} V={w.V} K={w.K} heads, {shape}, "
@@ -315,13 +330,16 @@ def run_mine(args, rank, world, local_rank):
     from medusa_tree_speculative_heads_b200 import binding as Bnd
     mode = Bnd.STOCHASTIC if w.stochastic else Bnd.GREEDY
     step = MedusaStep(B=w.B, d=w.d, V=w.V, K=w.K, Hq=w.Hq, Hkv=w.Hkv, D=w.D, S_max=w.S_max, parents=parents,
-                      dtype=w.torch_dtype, max_prefix=w.max_prefix, device=dev, mode=mode, q_rows=T, **paged)
+                      dtype=w.torch_dtype, max_prefix=w.max_prefix, device=dev, mode=mode, q_rows=T,
+                      temperature=w.temperature, **paged)
     q_draft = vtok = None
     if w.stochastic:
         # the target's and the draft's distributions and the drafted tokens
         # (children drawn from q at their parent) come from the harness
         sd = I.stochastic_inputs(w, parents, device="cuda")
         logits, q_draft, vtok = sd["p"], sd["q"], sd["node_tokens"]
+        if w.temperature > 0:   # the target's bf16 logits, read at the temperature
+            logits = sd["logits"].bfloat16()
     else:
         # the target model's logits (outside this path) are synthesised once
         # from the tree the heads propose, with the workload's match probability
@@ -505,18 +523,23 @@ def run_mine(args, rank, world, local_rank):
         "gpu_launches": K * launches_per_step(w),
         "clocks": clk,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and not w.stochastic:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
         oracle.build()
-        sample = OracleSample(w, 1.0)
+        frac = 1.0 / 16 if w.stochastic else 1.0   # B=64: a vocabulary / query-row slice keeps it to seconds
+        sample = OracleSample(w, frac)
         tt, ff = 0.0, 0.0
         while tt < 10.0 and ff < 3.0:
             t1, f1 = sample.run()
             tt += t1
             ff += f1
         out["cpu_baseline"] = {"value": ff / tt, "unit": UNIT, "cores": 1, "kind": "oracle",
-                               "sample": f"{ff:.2f} whole steps of the same workload run by the single-threaded fp64 "
-                                         f"oracle on the host ({tt:.1f} s)"}
+                               "sample": (f"{ff:.2f} whole steps of the same workload run by the single-threaded "
+                                          f"fp64 oracle on the host ({tt:.1f} s)" if frac == 1.0 else
+                                          f"{ff:.2f} steps' worth of work: the fp64 oracle on the host ({tt:.1f} s), "
+                                          f"residual blocks whole, LM-head rows of a 1/16 vocabulary slice, 1/16 of "
+                                          f"the attention rows, verification and commit whole; steps/s scaled by "
+                                          f"the sampled fraction")}
     if rank == 0:
         print(json.dumps(out), flush=True)
     if world > 1:

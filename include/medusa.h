@@ -8,6 +8,8 @@
  *                   its tree ancestors (one attention layer)
  *   tree_verify     greedy or stochastic verification: longest accepted
  *                   root-to-node path plus one bonus token
+ *                   (tree_verify_logits: the stochastic walk reading the
+ *                   target's logits at a temperature)
  *   kv_commit       append the accepted path's K/V to the cache
  * tree_attention_paged and kv_commit_paged are the two cache calls over a
  * paged KV cache (a page pool and a block table).
@@ -284,6 +286,36 @@ int tree_verify(medusa_verify_mode mode, const void* target, medusa_dtype target
                 uint64_t seed, uint32_t step, int32_t* accept_path, int max_path, int32_t* accept_len,
                 int32_t* bonus, void* workspace, size_t workspace_bytes, int32_t* status,
                 medusa_stream_t stream);
+
+/*
+ * STOCHASTIC verification reading the target's logits instead of its
+ * probabilities: the walk of tree_verify (STOCHASTIC) with P, wherever the
+ * walk reads the target's own row of node u, taken as
+ *     m = max_y z(y),   e(y) = exp((z(y) - m) * (1/tau)),   Z = sum_y e(y),
+ *     P(y) = e(y) * (1/Z)
+ * in fp64 (z = logits[b,u,:] widened exactly; each product, difference and
+ * quotient rounded once; 1/tau computed on the host).  The pages write
+ * P_target without saying how it comes from the model's logits; tau = 1 is
+ * the plain softmax, other tau the usual sampling temperature.  No
+ * probability row is materialised: the maximum and Z of each visited row are
+ * reduced over the sequence's thread-block cluster on entry.  The
+ * exponentials and Z's summation order may differ from a sequential fp64
+ * evaluation in the last bits of P; integer decisions differ only when a
+ * value falls within that rounding of a boundary.
+ *   logits [B, T, V], dtype logits_dt (MEDUSA_F32 or MEDUSA_BF16); NaN
+ *   entries are skipped by the maximum and make the row's mass NaN (no
+ *   acceptance; MEDUSA_STATUS_NO_MASS if the walk ends there), as does a row
+ *   without a finite maximum.
+ *   temperature: > 0 and finite, with 1/temperature finite, else
+ *   MEDUSA_ERR_INVALID_ARG.
+ * Every other argument, output and error as tree_verify in STOCHASTIC mode;
+ * workspace: tree_verify_workspace_size(MEDUSA_VERIFY_STOCHASTIC, ...).
+ */
+int tree_verify_logits(const void* logits, medusa_dtype logits_dt, double temperature, const float* q, int q_rows,
+                       const int32_t* q_row, const int32_t* node_tokens, int B, int V, const medusa_tree* tree,
+                       uint64_t seed, uint32_t step, int32_t* accept_path, int max_path, int32_t* accept_len,
+                       int32_t* bonus, void* workspace, size_t workspace_bytes, int32_t* status,
+                       medusa_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* KV commit                                                                 */

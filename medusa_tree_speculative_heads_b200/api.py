@@ -96,6 +96,28 @@ def tree_verify(mode: int, target: torch.Tensor, node_tokens: torch.Tensor, tree
     return out
 
 
+def tree_verify_logits(logits: torch.Tensor, temperature: float, q: torch.Tensor, node_tokens: torch.Tensor,
+                       tree: Tree, q_row: Optional[torch.Tensor] = None, seed: int = 0, step: int = 0,
+                       max_path: Optional[int] = None) -> Dict[str, torch.Tensor]:
+    """Stochastic verification reading the target's logits [B,T,V] (f32 or
+    bf16) at a temperature; q [B,q_rows,V] fp32, optional q_row."""
+    B, T, V = logits.shape
+    dev = logits.device
+    max_path = max_path or tree.max_depth
+    out = {
+        "accept_path": torch.empty((B, max_path), dtype=torch.int32, device=dev),
+        "accept_len": torch.empty((B,), dtype=torch.int32, device=dev),
+        "bonus": torch.empty((B,), dtype=torch.int32, device=dev),
+        "status": _status(dev),
+    }
+    nb = _b.tree_verify_workspace_size(_b.STOCHASTIC, B, V, tree)
+    ws = _ws(nb, dev)
+    _b.tree_verify_logits(logits, _b.dtype_code(logits.dtype), temperature, q, q.shape[1], q_row, node_tokens, B, V,
+                          tree, seed, step, out["accept_path"], max_path, out["accept_len"], out["bonus"], ws, nb,
+                          out["status"])
+    return out
+
+
 def kv_commit(k_cache, v_cache, k_tree, v_tree, accept_path, accept_len, prefix_len,
               new_prefix_len: Optional[torch.Tensor] = None) -> Dict[str, torch.Tensor]:
     """Append the accepted path's K/V in place; returns new_prefix_len (a new
@@ -156,16 +178,22 @@ class MedusaStep:
     ``prefix_len`` to advance in place).  ``parents`` is one parent list, or
     one per sequence.  With ``page_size`` > 0 the cache is a page pool
     [num_pages, Hkv, page_size, D] read and written through a block table
-    [B, max_pages] (pass it as ``block_table``), and the paged calls run."""
+    [B, max_pages] (pass it as ``block_table``), and the paged calls run.
+    With ``temperature`` > 0 (stochastic mode) the target passed to
+    ``verify``/``run`` is the target's logits, read by tree_verify_logits."""
 
     def __init__(self, *, B: int, d: int, V: int, K: int, Hq: int, Hkv: int, D: int, S_max: int,
                  parents, dtype: torch.dtype, mode: int = _b.GREEDY, max_prefix: int = 0,
-                 q_rows: int = 0, device=None, page_size: int = 0, max_pages: int = 0, num_pages: int = 0):
+                 q_rows: int = 0, device=None, page_size: int = 0, max_pages: int = 0, num_pages: int = 0,
+                 temperature: float = 0.0):
         dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
         self.B, self.d, self.V, self.K = B, d, V, K
         self.Hq, self.Hkv, self.D, self.S_max, self.max_prefix = Hq, Hkv, D, S_max, max_prefix
         self.dt = _b.dtype_code(dtype)
         self.mode = mode
+        self.temperature = temperature
+        if temperature > 0 and mode != _b.STOCHASTIC:
+            raise ValueError("a temperature applies to stochastic verification only")
         self.tree = Tree(parents)
         T = self.T = self.tree.T
         self.max_path = self.tree.max_depth
@@ -210,6 +238,12 @@ class MedusaStep:
 
     def verify(self, target, q=None, q_row=None, seed: int = 0, step: int = 0, node_tokens=None):
         tgt_dt = _b.dtype_code(target.dtype)
+        if self.temperature > 0:
+            _b.tree_verify_logits(target, tgt_dt, self.temperature, q, self.q_rows, q_row,
+                                  self.node_tokens if node_tokens is None else node_tokens, self.B, self.V, self.tree,
+                                  seed, step, self.accept_path, self.max_path, self.accept_len, self.bonus,
+                                  self.ws_verify, self.ws_verify_n, self.status)
+            return
         _b.tree_verify(self.mode, target, tgt_dt, q, self.q_rows if q is not None else 0, q_row,
                        self.node_tokens if node_tokens is None else node_tokens, self.B, self.V, self.tree, seed,
                        step, self.accept_path, self.max_path, self.accept_len, self.bonus, self.ws_verify,

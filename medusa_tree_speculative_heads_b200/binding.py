@@ -78,6 +78,8 @@ def lib() -> ctypes.CDLL:
         L.tree_verify_workspace_size.restype = sz
         L.tree_verify.argtypes = [i32, vp, i32, vp, i32, vp, vp, i32, i32, vp, u64, u32, vp, i32, vp, vp, vp, sz, vp,
                                   vp]
+        L.tree_verify_logits.argtypes = [vp, i32, ctypes.c_double, vp, i32, vp, vp, i32, i32, vp, u64, u32, vp, i32,
+                                         vp, vp, vp, sz, vp, vp]
         L.kv_commit.argtypes = [vp, vp, vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp]
         L.tree_attention_paged_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32, i32, vp, i32]
         L.tree_attention_paged_workspace_size.restype = sz
@@ -211,6 +213,14 @@ def tree_verify(mode, target, target_dt, q, q_rows, q_row, node_tokens, B, V, tr
                              tree.handle, ctypes.c_uint64(seed & (2**64 - 1)), ctypes.c_uint32(step & 0xFFFFFFFF),
                              _p(accept_path), max_path, _p(accept_len), _p(bonus), _p(workspace), workspace_bytes,
                              _p(status), _stream(stream)))
+
+
+def tree_verify_logits(logits, logits_dt, temperature, q, q_rows, q_row, node_tokens, B, V, tree: Tree, seed, step,
+                       accept_path, max_path, accept_len, bonus, workspace, workspace_bytes, status, stream=None):
+    _check(lib().tree_verify_logits(_p(logits), logits_dt, float(temperature), _p(q), q_rows, _p(q_row),
+                                    _p(node_tokens), B, V, tree.handle, ctypes.c_uint64(seed & (2**64 - 1)),
+                                    ctypes.c_uint32(step & 0xFFFFFFFF), _p(accept_path), max_path, _p(accept_len),
+                                    _p(bonus), _p(workspace), workspace_bytes, _p(status), _stream(stream)))
 
 
 def kv_commit(k_cache, v_cache, k_tree, v_tree, accept_path, max_path, accept_len, prefix_len, new_prefix_len, B, T,

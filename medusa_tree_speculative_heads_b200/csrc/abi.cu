@@ -1,6 +1,7 @@
 // C ABI of libmedusa: argument validation, the candidate-tree handle,
 // workspace queries and launches.  See include/medusa.h for the contract of
 // every entry point.
+#include <cmath>
 #include <stdarg.h>
 #include <stdio.h>
 #include <string.h>
@@ -356,35 +357,40 @@ extern "C" size_t tree_verify_workspace_size(medusa_verify_mode mode, int B, int
     return verify_workspace_size(mode, B, V, tree->host.T);
 }
 
-extern "C" int tree_verify(medusa_verify_mode mode, const void* target, medusa_dtype target_dt, const float* q,
-                           int q_rows, const int32_t* q_row, const int32_t* node_tokens, int B, int V,
-                           const medusa_tree* tree, uint64_t seed, uint32_t step, int32_t* accept_path, int max_path,
-                           int32_t* accept_len, int32_t* bonus, void* workspace, size_t workspace_bytes,
-                           int32_t* status, medusa_stream_t stream) {
+// shared by tree_verify and tree_verify_logits: `fn` names the call in
+// messages; logits selects the logits form of the stochastic walk
+static int verify_common(const char* fn, medusa_verify_mode mode, const void* target, medusa_dtype target_dt,
+                         bool logits, double temperature, const float* q, int q_rows, const int32_t* q_row,
+                         const int32_t* node_tokens, int B, int V, const medusa_tree* tree, uint64_t seed,
+                         uint32_t step, int32_t* accept_path, int max_path, int32_t* accept_len, int32_t* bonus,
+                         void* workspace, size_t workspace_bytes, int32_t* status, medusa_stream_t stream) {
     if (mode != MEDUSA_VERIFY_GREEDY && mode != MEDUSA_VERIFY_STOCHASTIC)
-        return fail(MEDUSA_ERR_INVALID_ARG, "tree_verify: unknown mode");
+        return fail(MEDUSA_ERR_INVALID_ARG, "%s: unknown mode", fn);
     if (!target || !node_tokens || !accept_path || !accept_len || !bonus)
-        return fail(MEDUSA_ERR_INVALID_ARG, "tree_verify: NULL tensor argument");
+        return fail(MEDUSA_ERR_INVALID_ARG, "%s: NULL tensor argument", fn);
     int rc = check_tree(tree, B);
     if (rc) return rc;
     const int T = tree->host.T;
-    if (B < 1 || V < 1) return fail(MEDUSA_ERR_INVALID_ARG, "tree_verify: bad sizes B=%d V=%d", B, V);
+    if (B < 1 || V < 1) return fail(MEDUSA_ERR_INVALID_ARG, "%s: bad sizes B=%d V=%d", fn, B, V);
     if (max_path < tree->host.max_depth || max_path > kMaxTree)
-        return fail(MEDUSA_ERR_INVALID_ARG, "tree_verify: max_path %d outside [tree depth %d, %d]", max_path,
+        return fail(MEDUSA_ERR_INVALID_ARG, "%s: max_path %d outside [tree depth %d, %d]", fn, max_path,
                     tree->host.max_depth, kMaxTree);
-    if (mode == MEDUSA_VERIFY_GREEDY) {
+    if (mode == MEDUSA_VERIFY_GREEDY || logits) {
         if (target_dt != MEDUSA_F32 && target_dt != MEDUSA_BF16)
-            return fail(MEDUSA_ERR_UNSUPPORTED, "tree_verify: greedy target dtype");
-    } else {
-        if (target_dt != MEDUSA_F32)
-            return fail(MEDUSA_ERR_UNSUPPORTED, "tree_verify: stochastic target p must be MEDUSA_F32");
-        if (!q) return fail(MEDUSA_ERR_INVALID_ARG, "tree_verify: stochastic mode needs q");
+            return fail(MEDUSA_ERR_UNSUPPORTED, "%s: logits dtype must be MEDUSA_F32 or MEDUSA_BF16", fn);
+    } else if (target_dt != MEDUSA_F32) {
+        return fail(MEDUSA_ERR_UNSUPPORTED, "%s: stochastic target p must be MEDUSA_F32", fn);
+    }
+    if (logits && !(temperature > 0.0 && std::isfinite(temperature) && std::isfinite(1.0 / temperature)))
+        return fail(MEDUSA_ERR_INVALID_ARG, "%s: temperature %g must be positive and finite", fn, temperature);
+    if (mode == MEDUSA_VERIFY_STOCHASTIC) {
+        if (!q) return fail(MEDUSA_ERR_INVALID_ARG, "%s: stochastic mode needs q", fn);
         if (q_rows < 1 || (!q_row && q_rows != T))
-            return fail(MEDUSA_ERR_INVALID_ARG, "tree_verify: q_rows=%d (must equal T=%d without q_row)", q_rows, T);
+            return fail(MEDUSA_ERR_INVALID_ARG, "%s: q_rows=%d (must equal T=%d without q_row)", fn, q_rows, T);
     }
     const size_t need = verify_workspace_size(mode, B, V, T);
     if (need > 0 && (!workspace || workspace_bytes < need || !al16(workspace)))
-        return fail(MEDUSA_ERR_WORKSPACE, "tree_verify: workspace of %zu bytes, need %zu", workspace_bytes, need);
+        return fail(MEDUSA_ERR_WORKSPACE, "%s: workspace of %zu bytes, need %zu", fn, workspace_bytes, need);
     VerifyArgs a;
     a.mode = mode;
     a.target = target;
@@ -406,9 +412,31 @@ extern "C" int tree_verify(medusa_verify_mode mode, const void* target, medusa_d
     a.ws = workspace;
     a.ws_bytes = workspace_bytes;
     a.status = status;
+    a.logits = logits;
+    a.inv_tau = logits ? 1.0 / temperature : 1.0;
     cudaError_t e = verify_launch(a, (cudaStream_t)stream);
-    if (e != cudaSuccess) return cuda_fail(e, "tree_verify launch");
+    if (e != cudaSuccess) return cuda_fail(e, fn);
     return ok();
+}
+
+extern "C" int tree_verify(medusa_verify_mode mode, const void* target, medusa_dtype target_dt, const float* q,
+                           int q_rows, const int32_t* q_row, const int32_t* node_tokens, int B, int V,
+                           const medusa_tree* tree, uint64_t seed, uint32_t step, int32_t* accept_path, int max_path,
+                           int32_t* accept_len, int32_t* bonus, void* workspace, size_t workspace_bytes,
+                           int32_t* status, medusa_stream_t stream) {
+    return verify_common("tree_verify", mode, target, target_dt, false, 1.0, q, q_rows, q_row, node_tokens, B, V,
+                         tree, seed, step, accept_path, max_path, accept_len, bonus, workspace, workspace_bytes,
+                         status, stream);
+}
+
+extern "C" int tree_verify_logits(const void* logits, medusa_dtype logits_dt, double temperature, const float* q,
+                                  int q_rows, const int32_t* q_row, const int32_t* node_tokens, int B, int V,
+                                  const medusa_tree* tree, uint64_t seed, uint32_t step, int32_t* accept_path,
+                                  int max_path, int32_t* accept_len, int32_t* bonus, void* workspace,
+                                  size_t workspace_bytes, int32_t* status, medusa_stream_t stream) {
+    return verify_common("tree_verify_logits", MEDUSA_VERIFY_STOCHASTIC, logits, logits_dt, true, temperature, q,
+                         q_rows, q_row, node_tokens, B, V, tree, seed, step, accept_path, max_path, accept_len, bonus,
+                         workspace, workspace_bytes, status, stream);
 }
 
 // ---------------------------------------------------------------------------

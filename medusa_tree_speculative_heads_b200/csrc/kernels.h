@@ -88,6 +88,8 @@ struct VerifyArgs {
     void* ws;
     size_t ws_bytes;
     int32_t* status;
+    bool logits;     // stochastic: target holds logits (target_dt f32/bf16), P = softmax((z - max z) * inv_tau)
+    double inv_tau;  // 1 / temperature
 };
 size_t verify_workspace_size(medusa_verify_mode mode, int B, int V, int T);
 cudaError_t verify_launch(const VerifyArgs& a, cudaStream_t st);

@@ -21,6 +21,14 @@
 // peer CTAs).  All decisions use integer or correctly rounded fp64
 // operations (explicit _rn intrinsics, no contraction), so results are
 // bit-reproducible and independent of the cluster size.
+//
+// The stochastic walk can also read the target's logits z instead of its
+// probabilities: on entering a node the cluster takes the row maximum m and
+// Z = sum exp((z - m) / tau) (fp64, fixed reduction order: lanes, warps,
+// CTAs in rank order), and P(y) = exp((z(y) - m) / tau) / Z is evaluated
+// wherever the walk reads P, so no probability row is ever materialised.
+// The fp64 exponentials and Z's summation order differ from a sequential
+// evaluation only in the last bits of P.
 #include <cooperative_groups.h>
 #include <limits.h>
 
@@ -207,6 +215,8 @@ __device__ __forceinline__ unsigned long long weight_2p32(double x) {
 struct ClusterSum {
     unsigned long long warp_tot[kStochThreads / 32];
     unsigned long long cta_tot;
+    double warp_d[kStochThreads / 32];
+    double cta_d;
 };
 __device__ unsigned long long cluster_sum(unsigned long long x, ClusterSum* sh, unsigned long long* before) {
     namespace cg = cooperative_groups;
@@ -238,8 +248,48 @@ __device__ unsigned long long cluster_sum(unsigned long long x, ClusterSum* sh, 
     return tot;
 }
 
+// fp64 maximum (kMax; NaN skipped) or sum over the cluster, in a fixed
+// order (lane butterfly, warps 0.., CTAs 0..): every thread of the cluster
+// gets the same bits.
+template <bool kMax>
+__device__ double cluster_reduce_f64(double x, ClusterSum* sh) {
+    namespace cg = cooperative_groups;
+    cg::cluster_group cl = cg::this_cluster();
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const double y = __shfl_xor_sync(kFull, x, o);
+        x = kMax ? fmax(x, y) : __dadd_rn(x, y);
+    }
+    if (lane == 0) sh->warp_d[warp] = x;
+    __syncthreads();
+    if (tid == 0) {
+        double c = sh->warp_d[0];
+        for (int w = 1; w < kStochThreads / 32; ++w) c = kMax ? fmax(c, sh->warp_d[w]) : __dadd_rn(c, sh->warp_d[w]);
+        sh->cta_d = c;
+    }
+    __syncwarp();
+    cl.sync();
+    const int C = (int)cl.num_blocks();
+    double t = cl.map_shared_rank(sh, 0)->cta_d;
+    for (int r = 1; r < C; ++r) {
+        const double v = cl.map_shared_rank(sh, r)->cta_d;
+        t = kMax ? fmax(t, v) : __dadd_rn(t, v);
+    }
+    cl.sync();
+    return t;
+}
+
+// target rows: kSrc 0 = probabilities p (f32), 1 = f32 logits, 2 = bf16 logits
+template <int kSrc>
+__device__ __forceinline__ double target_at(const void* row, int y) {
+    if constexpr (kSrc == 2) return (double)__bfloat162float(((const __nv_bfloat16*)row)[y]);
+    else return (double)((const float*)row)[y];
+}
+
+template <int kSrc>
 __global__ void __launch_bounds__(kStochThreads, 2) verify_stochastic_kernel(
-    const float* __restrict__ p, const float* __restrict__ q, int q_rows, const int32_t* __restrict__ q_row,
+    const void* __restrict__ target, double inv_tau, const float* __restrict__ q, int q_rows, const int32_t* __restrict__ q_row,
     const int32_t* __restrict__ node_tokens, int V, TreeRef trees, uint32_t key0, uint32_t key1,
     uint32_t step, int32_t* accept_path, int max_path, int32_t* accept_len, int32_t* bonus,
     unsigned long long* ws_w, int32_t* status) {
@@ -250,8 +300,9 @@ __global__ void __launch_bounds__(kStochThreads, 2) verify_stochastic_kernel(
     const int b = blockIdx.x / C, tid = threadIdx.x;
     const bool lead = rank == 0 && tid == 0;
     const TreeDev* tree = trees.at(b);
-    const int T = trees.T;  // node stride of p, node_tokens (and of q_row with one tree per sequence)
-    const float* Pb = p + (long)b * T * V;
+    const int T = trees.T;  // node stride of target, node_tokens (and of q_row with one tree per sequence)
+    constexpr int kEsz = kSrc == 2 ? 2 : 4;
+    const char* Pb = (const char*)target + (long)b * T * V * kEsz;
     // Two weight buffers.  `valid` holds the last effective residual (S > 0)
     // of the current node, -1 while P is still p[b,u,:].  `keep` is the
     // buffer the latest accept decision may have read (threads of the
@@ -270,12 +321,47 @@ __global__ void __launch_bounds__(kStochThreads, 2) verify_stochastic_kernel(
 
     int u = 0, L = 1, valid = -1, keep = -1;
     unsigned long long S_valid = 0;
-    const float* Prow = Pb;
+    const void* Prow = Pb;
+    double row_m = 0.0, row_r = 1.0;  // logits: the row's maximum and 1 / Z
     auto Wbuf = [&](int i) { return ws_w + (i & 1) * BV + (long)b * V; };
+    // the target's own distribution at y of the current node's row
+    auto target_p = [&](int y) -> double {
+        const double z = target_at<kSrc>(Prow, y);
+        if constexpr (kSrc == 0) return z;
+        else return __dmul_rn(exp(__dmul_rn(__dsub_rn(z, row_m), inv_tau)), row_r);
+    };
     // current target distribution at y
     auto cur = [&](int y) -> double {
-        if (valid < 0) return (double)Prow[y];
+        if (valid < 0) return target_p(y);
         return __ddiv_rn((double)Wbuf(valid)[y], (double)S_valid);
+    };
+    // move to node n's row; with logits, the row's maximum and normaliser
+    // (every thread of the cluster, in step)
+    auto enter_row = [&](int n) {
+        Prow = Pb + (long)n * V * kEsz;
+        if constexpr (kSrc != 0) {
+            double m = -INFINITY;
+            for (int y = y0 + lane; y < y1; y += 32 * U) {
+                double z[U];
+#pragma unroll
+                for (int i = 0; i < U; ++i) z[i] = y + 32 * i < y1 ? target_at<kSrc>(Prow, y + 32 * i) : -INFINITY;
+#pragma unroll
+                for (int i = 0; i < U; ++i) m = fmax(m, z[i]);
+            }
+            m = cluster_reduce_f64<true>(m, &sh);
+            double Z = 0.0;
+            for (int y = y0 + lane; y < y1; y += 32 * U) {
+                double z[U];
+#pragma unroll
+                for (int i = 0; i < U; ++i) z[i] = y + 32 * i < y1 ? target_at<kSrc>(Prow, y + 32 * i) : 0.0;
+#pragma unroll
+                for (int i = 0; i < U; ++i)
+                    if (y + 32 * i < y1) Z = __dadd_rn(Z, exp(__dmul_rn(__dsub_rn(z[i], m), inv_tau)));
+            }
+            Z = cluster_reduce_f64<false>(Z, &sh);
+            row_m = m;
+            row_r = __ddiv_rn(1.0, Z);
+        }
     };
     if (lead) {
         accept_path[(long)b * max_path] = 0;
@@ -286,7 +372,7 @@ __global__ void __launch_bounds__(kStochThreads, 2) verify_stochastic_kernel(
         const int c_begin = tree->child_off[u], c_end = tree->child_off[u + 1];
         if (valid >= 0) keep = valid;
         valid = -1;
-        Prow = Pb + (long)u * V;
+        enter_row(u);
         if (c_begin == c_end) break;  // a leaf: no drafted children
         const int qr = q_row ? q_row[(trees.stride ? (long)b * T : 0) + u] : u;
         if (qr < 0 || qr >= q_rows) {
@@ -461,9 +547,12 @@ cudaError_t verify_launch(const VerifyArgs& a, cudaStream_t st) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, verify_stochastic_kernel, (const float*)a.target, a.q, a.q_rows, a.q_row,
-                              a.node_tokens, a.V, a.tree, (uint32_t)a.seed, (uint32_t)(a.seed >> 32), a.step,
-                              a.accept_path, a.max_path, a.accept_len, a.bonus, ws_w, a.status);
+    auto kernel = !a.logits ? verify_stochastic_kernel<0>
+                  : a.target_dt == MEDUSA_BF16 ? verify_stochastic_kernel<2> : verify_stochastic_kernel<1>;
+    const double inv_tau = a.logits ? a.inv_tau : 1.0;
+    return cudaLaunchKernelEx(&cfg, kernel, a.target, inv_tau, a.q, a.q_rows, a.q_row, a.node_tokens, a.V, a.tree,
+                              (uint32_t)a.seed, (uint32_t)(a.seed >> 32), a.step, a.accept_path, a.max_path,
+                              a.accept_len, a.bonus, ws_w, a.status);
 }
 
 }  // namespace medusa

@@ -208,3 +208,29 @@ def test_step_with_per_sequence_trees():
         for t in range(L):
             assert torch.equal(ain["k_cache"][b, :, S + t], ain["k_tree"][b, int(path[0][t])])
         assert torch.equal(ain["k_cache"][b, :, :S], k0[b, :, :S])
+
+
+def test_stochastic_logits_verify_per_sequence_trees():
+    w = I.scaled(I.WORKLOADS["stoch_b64"], B=5, V=700)
+    trees = ragged_trees(w.B, seed=9)
+    tree = Tree(trees)
+    T = tree.T
+    z = torch.full((w.B, T, w.V), float("nan"))
+    q = torch.full((w.B, T, w.V), float("nan"))
+    tok = torch.full((w.B, T), -1, dtype=torch.int32)
+    for b, par in enumerate(trees):
+        d = I.stochastic_inputs(I.scaled(w, B=1, seed=w.seed + b), par)
+        Tb = len(par)
+        z[b, :Tb], q[b, :Tb], tok[b, :Tb] = d["logits"][0], d["q"][0], d["node_tokens"][0]
+    zb = z.bfloat16()
+    for seed, step in ((7, 0), (2**64 - 3, 11)):
+        out = api.tree_verify_logits(zb.cuda(), 0.7, q.cuda(), tok.cuda(), tree, seed=seed, step=step)
+        torch.cuda.synchronize()
+        assert int(out["status"].item()) == 0
+        for b, par in enumerate(trees):
+            Tb = len(par)
+            path, ln, bonus, _ = oracle.verify_stochastic_logits(zb[b:b + 1, :Tb], 0.7, q[b:b + 1, :Tb],
+                                                                 tok[b:b + 1, :Tb], par, seed, step, tree.max_depth,
+                                                                 b0=b)
+            assert out["accept_path"][b].tolist() == path[0].tolist(), (b, seed)
+            assert int(out["accept_len"][b]) == int(ln[0]) and int(out["bonus"][b]) == int(bonus[0]), (b, seed)

@@ -68,7 +68,7 @@ def test_whole_step_matches_oracle(name):
         assert torch.equal(chain["kc"], okc) and torch.equal(chain["vc"], ovc)
 
 
-@pytest.mark.parametrize("name", ["llama8b_small", "stoch_small"])
+@pytest.mark.parametrize("name", ["llama8b_small", "stoch_small", "stoch_logits_small"])
 def test_graph_replay_equals_eager_step(name):
     # the step captured in a CUDA graph and replayed gives the eager step's
     # results bit for bit (the kernels are deterministic)
@@ -80,13 +80,16 @@ def test_graph_replay_equals_eager_step(name):
     T = len(parents)
     from medusa_tree_speculative_heads_b200 import binding as Bnd
     mode = Bnd.STOCHASTIC if w.stochastic else Bnd.GREEDY
+    tau = I.STOCH_TEMPERATURE if name == "stoch_logits_small" else 0.0
     step = MedusaStep(B=w.B, d=w.d, V=w.V, K=w.K, Hq=w.Hq, Hkv=w.Hkv, D=w.D, S_max=w.S_max, parents=parents,
-                      dtype=w.torch_dtype, device="cuda", mode=mode, q_rows=T)
+                      dtype=w.torch_dtype, device="cuda", mode=mode, q_rows=T, temperature=tau)
     hin = {k: v.cuda() for k, v in I.head_inputs(w).items()}
     ain = {k: v.cuda() for k, v in I.attention_inputs(w, T).items()}
     if w.stochastic:
         sd = {k: v.cuda() for k, v in I.stochastic_inputs(w, parents).items()}
         target, q_draft, tok = sd["p"], sd["q"], sd["node_tokens"]
+        if tau > 0:   # the step reads the target's bf16 logits
+            target = sd["logits"].bfloat16()
     else:
         target = torch.randn((w.B, T, w.V), generator=torch.Generator().manual_seed(2)).to(w.torch_dtype).cuda()
         q_draft = tok = None
@@ -115,3 +118,8 @@ def test_graph_replay_equals_eager_step(name):
     replay = (step.node_tokens, step.attn_out, step.accept_path, step.accept_len, step.bonus, new_pl, ain["k_cache"])
     for a, b in zip(eager, replay):
         assert torch.equal(a, b)
+    if tau > 0:
+        maxd = int(max(oracle.tree_shape(parents)[0]))
+        path, ln, bonus, _ = oracle.verify_stochastic_logits(target, tau, q_draft, tok, parents, 0, 5, maxd)
+        assert np.array_equal(step.accept_path.cpu().numpy(), path)
+        assert np.array_equal(step.accept_len.cpu().numpy(), ln) and np.array_equal(step.bonus.cpu().numpy(), bonus)

@@ -136,3 +136,100 @@ def test_stochastic_draft_equals_target_accepts_first_children():
         chain.append(ch[chain[-1]][0])
     for b in range(w.B):
         assert out["accept_path"][b, : len(chain)].tolist() == chain
+
+
+# ---------------------------------------------------------------------------
+# stochastic verification reading logits at a temperature
+# ---------------------------------------------------------------------------
+
+def run_stoch_logits(parents, z, tau, q, tok, seed, step, q_row=None):
+    tree = Tree(parents)
+    out = api.tree_verify_logits(z.cuda(), tau, q.cuda(), tok.cuda(), tree,
+                                 q_row=None if q_row is None else torch.as_tensor(q_row, dtype=torch.int32).cuda(),
+                                 seed=seed, step=step)
+    torch.cuda.synchronize()
+    return out
+
+
+@pytest.mark.parametrize("kw,dtype,tau", [
+    (dict(B=8), torch.float32, I.STOCH_TEMPERATURE),
+    (dict(B=3, V=777), torch.bfloat16, 1.0),
+    (dict(B=12, V=3001), torch.float32, 2.5),
+    (dict(B=1), torch.bfloat16, I.STOCH_TEMPERATURE),
+    (dict(), torch.bfloat16, I.STOCH_TEMPERATURE),            # the full B=64, V=32000 batch
+])
+def test_stochastic_logits_parity(kw, dtype, tau):
+    # the walk's decisions are integer or fp64; the kernel's exponentials and
+    # its cluster-ordered sum of Z differ from the oracle's only in the last
+    # bits of P, which no decision of these cases falls within
+    w = I.scaled(I.WORKLOADS["stoch_b64"], **kw)
+    parents = I.workload_tree(w)
+    d = I.stochastic_inputs(w, parents)
+    z = d["logits"].to(dtype)
+    maxd = int(max(oracle.tree_shape(parents)[0]))
+    for seed, step in ((0, 0), (0x123456789ABCDEF0, 17), (2**64 - 1, 2**32 - 1)):
+        out = run_stoch_logits(parents, z, tau, d["q"], d["node_tokens"], seed, step)
+        ref = oracle.verify_stochastic_logits(z, tau, d["q"], d["node_tokens"], parents, seed, step, maxd)
+        assert_same(out, ref)
+        assert int(out["status"].item()) == 0
+
+
+def test_stochastic_logits_wide_tree_and_q_row():
+    # many rejections per node (the residual passes re-read P from logits once
+    # per node), Medusa-style shared draft rows
+    w = I.scaled(I.WORKLOADS["stoch_b64"], B=5, V=600)
+    parents = I.product_tree_parents((6, 3, 2))
+    d = I.stochastic_inputs(w, parents)
+    depth, _ = oracle.tree_shape(parents)
+    K = int(depth.max())
+    q_rows = d["q"][:, :K].contiguous()
+    q_row = (depth - 1).astype(np.int32)
+    z = d["logits"].bfloat16()
+    for step in range(4):
+        out = run_stoch_logits(parents, z, 0.7, q_rows, d["node_tokens"], 99, step, q_row=q_row)
+        ref = oracle.verify_stochastic_logits(z, 0.7, q_rows, d["node_tokens"], parents, 99, step, K, q_row=q_row)
+        assert_same(out, ref)
+
+
+def test_stochastic_logits_cold_limit_equals_greedy_kernel():
+    # tau -> 0 with a gap of 1.5 above the rest: P is the argmax point mass and
+    # the stochastic walk reproduces the greedy kernel's result
+    g = np.random.default_rng(5)
+    nb, V = 16, 5000
+    parents = I.product_tree_parents((4, 2, 2))
+    T = len(parents)
+    z = g.normal(0, 1, (nb, T, V)).astype(np.float32)
+    top = g.integers(V, size=(nb, T))
+    z[np.arange(nb)[:, None], np.arange(T)[None, :], top] = z.max(-1) + 1.5
+    ch = I.tree_children(parents)
+    tok = np.zeros((nb, T), np.int32)
+    for b in range(nb):
+        for u in range(T):
+            for i, c in enumerate(ch[u]):   # the first child takes the parent's argmax half the time
+                tok[b, c] = top[b, u] if (i == 0 and g.random() < 0.7) else (top[b, u] + 1 + i) % V
+    q = torch.full((nb, T, V), 1.0 / V)
+    zt, tt = torch.from_numpy(z), torch.from_numpy(tok)
+    out = run_stoch_logits(parents, zt, 1e-3, q, tt, 7, 3)
+    gre = api.tree_verify(B.GREEDY, zt.cuda(), tt.cuda(), Tree(parents))
+    torch.cuda.synchronize()
+    for k in ("accept_path", "accept_len", "bonus"):
+        assert torch.equal(out[k], gre[k]), k
+    assert len(set(out["accept_len"].tolist())) > 1
+
+
+def test_stochastic_logits_no_mass_and_bad_temperature():
+    V = 256
+    parents = [-1, 0]
+    z = torch.zeros((2, 2, V))
+    z[0, 0] = -float("inf")                                     # no finite maximum
+    z[1, 0, 7] = float("nan")                                   # NaN is skipped by the maximum
+    q = torch.full((2, 2, V), 1.0 / V)
+    tok = torch.tensor([[0, 3], [0, 3]], dtype=torch.int32)
+    out = run_stoch_logits(parents, z, 1.0, q, tok, 1, 0)
+    ref = oracle.verify_stochastic_logits(z, 1.0, q, tok, parents, 1, 0, 2)
+    assert_same(out, ref)
+    assert int(out["status"].item()) & B.STATUS_NO_MASS
+    for tau in (0.0, -1.0, float("inf"), float("nan"), 1e-320):
+        with pytest.raises(B.MedusaError) as e:
+            api.tree_verify_logits(z.cuda(), tau, q.cuda(), tok.cuda(), Tree(parents))
+        assert e.value.code == B.MEDUSA_ERR_INVALID_ARG
