@@ -63,6 +63,8 @@ def lib():
                                                    i32, vp, vp, vp, vp, i32]
         L.orc_softmax_temperature.argtypes = [vp, i32, dbl, vp]
         L.orc_softmax_temperature.restype = None
+        L.orc_kv_compact.argtypes = [vp, vp, i32, vp, i32, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]
+        L.orc_kv_compact.restype = None
         L.orc_kv_commit.argtypes = [vp, vp, vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]
         L.orc_kv_commit.restype = None
         L.orc_gather_pages.argtypes = [vp, vp, i32, i32, i32, vp, i32, i32, i32, i32, i32, vp]
@@ -219,6 +221,30 @@ def tree_attention(q, k_tree, v_tree, k_cache, v_cache, prefix_len, parents, sca
     return out, lse
 
 
+def tree_rows_from_cache(cache, prefix_len, T: int):
+    """The tree's K or V [B, T, Hkv, D] when they sit in the cache [B, Hkv,
+    S_max, D] at rows prefix_len[b] .. prefix_len[b] + T - 1 (rows past S_max
+    read as zeros)."""
+    c = cache.detach().cpu()
+    B, Hkv, S_max, D = c.shape
+    out = torch.zeros((B, T, Hkv, D), dtype=c.dtype)
+    for b in range(B):
+        S = int(prefix_len[b])
+        n = max(0, min(T, S_max - S))
+        out[b, :n] = c[b, :, S:S + n].transpose(0, 1)
+    return out
+
+
+def tree_attention_incache(q, k_cache, v_cache, prefix_len, parents, scale: float = 0.0,
+                           rows: Optional[np.ndarray] = None):
+    """tree_attention with the tree's K/V read from the cache rows right after
+    each prefix."""
+    T = q.shape[1]
+    kt = tree_rows_from_cache(k_cache, prefix_len, T)
+    vt = tree_rows_from_cache(v_cache, prefix_len, T)
+    return tree_attention(q, kt, vt, k_cache, v_cache, prefix_len, parents, scale, rows)
+
+
 # ----------------------------------------------------------------------------
 # verification
 # ----------------------------------------------------------------------------
@@ -336,6 +362,24 @@ def kv_commit(k_cache, v_cache, k_tree, v_tree, path, length, prefix_len):
     lib().orc_kv_commit(ctypes.c_void_p(kc.data_ptr()), ctypes.c_void_p(vc.data_ptr()),
                         ctypes.c_void_p(kt.data_ptr()), ctypes.c_void_p(vt.data_ptr()), _p(pa), max_path, _p(ln),
                         _p(pl), _p(npl), B, Hkv, D, S_max, T, esize, _p(status))
+    return kc, vc, npl, int(status[0])
+
+
+def kv_compact(k_layers, v_layers, path, length, prefix_len, T: int):
+    """Returns (k_layers', v_layers', new_prefix_len, status): new torch
+    tensors (the layers stacked [n_layers, B, Hkv, S_max, D]); inputs
+    untouched."""
+    kc = torch.stack([x.detach().cpu() for x in k_layers]).contiguous().clone()
+    vc = torch.stack([x.detach().cpu() for x in v_layers]).contiguous().clone()
+    n_layers, B, Hkv, S_max, D = kc.shape
+    pa = _i32(path)
+    max_path = pa.shape[1]
+    ln = _i32(length)
+    pl = _i32(prefix_len)
+    npl = np.zeros(B, np.int32)
+    status = np.zeros(1, np.int32)
+    lib().orc_kv_compact(ctypes.c_void_p(kc.data_ptr()), ctypes.c_void_p(vc.data_ptr()), n_layers, _p(pa), max_path,
+                         _p(ln), _p(pl), _p(npl), B, Hkv, D, S_max, T, kc.element_size(), _p(status))
     return kc, vc, npl, int(status[0])
 
 

@@ -646,6 +646,57 @@ int orc_verify_stochastic_logits(const void* logits, int dtype, double temperatu
 /* ------------------------------------------------------------------------ */
 
 /*
+ * The commit when the tree's K/V were appended to the cache right after each
+ * prefix before attention ([MTP] "The 2D Tree Attention Mask": the longest
+ * accepted path is kept; "Production Deployment Guidelines": the other
+ * branches are culled): in every layer, the accepted path's rows move down to
+ * just after the prefix,
+ *     new cache_l[b, g, S + t, :] = old cache_l[b, g, S + path[b,t], :],  t < len[b]
+ *     new_prefix_len[b] = S + len[b]          (S = prefix_len[b])
+ * (old rows are copied out first, then written).  caches: n_layers blocks of
+ * [B, Hkv, S_max, D], element size esize, copied bit for bit.  A sequence
+ * whose path is not strictly increasing, holds a node id outside [0, T) or
+ * has len outside [0, max_path] is left untouched (status bit 1), as is one
+ * whose source rows reach S_max (status bit 2); its new_prefix_len is S.
+ */
+void orc_kv_compact(void* k_caches, void* v_caches, int n_layers, const int32_t* path, int max_path,
+                    const int32_t* len, const int32_t* prefix_len, int32_t* new_prefix_len, int B, int Hkv, int D,
+                    int S_max, int T, int esize, int32_t* status) {
+    const size_t row = (size_t)D * esize;
+    const size_t layer_bytes = (size_t)B * Hkv * S_max * row;
+    unsigned char* tmp = (unsigned char*)malloc(row * (size_t)(max_path > 0 ? max_path : 1));
+    if (status) *status = 0;
+    for (int b = 0; b < B; ++b) {
+        const int S = prefix_len[b], L = len[b];
+        int ok = L >= 0 && L <= max_path && S >= 0;
+        for (int t = 0; ok && t < L; ++t) {
+            const int n = path[(size_t)b * max_path + t];
+            const int prev = t > 0 ? path[(size_t)b * max_path + t - 1] : -1;
+            if (n <= prev || n >= T) ok = 0;
+        }
+        if (!ok) {
+            if (status) *status |= 1;
+        } else if (L > 0 && (long)S + path[(size_t)b * max_path + L - 1] >= S_max) {
+            ok = 0;
+            if (status) *status |= 2;
+        }
+        new_prefix_len[b] = ok ? S + L : S;
+        if (!ok) continue;
+        for (int l = 0; l < n_layers; ++l)
+            for (int kv = 0; kv < 2; ++kv) {
+                unsigned char* c = (unsigned char*)(kv ? v_caches : k_caches) + (size_t)l * layer_bytes;
+                for (int g = 0; g < Hkv; ++g) {
+                    unsigned char* blk = c + ((size_t)b * Hkv + g) * S_max * row;
+                    for (int t = 0; t < L; ++t)
+                        memcpy(tmp + (size_t)t * row, blk + (size_t)(S + path[(size_t)b * max_path + t]) * row, row);
+                    for (int t = 0; t < L; ++t) memcpy(blk + (size_t)(S + t) * row, tmp + (size_t)t * row, row);
+                }
+            }
+    }
+    free(tmp);
+}
+
+/*
  * [MTP] "The 2D Tree Attention Mask" (the engine commits the longest accepted
  * path) and "Production Deployment Guidelines" (unselected branches are
  * culled): the K/V rows of the accepted path's nodes are appended, in path

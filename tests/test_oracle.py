@@ -912,3 +912,91 @@ def test_stochastic_logits_rows_without_mass(orc):
     assert ln[0] == 1 and bonus[0] == 0 and st == 1
     path, ln, bonus, st = orc.verify_stochastic_logits(z[1:], 1.0, q[1:], tok[1:], par, 1, 0, 2, b0=1)
     assert st == 0
+
+
+# ----------------------------------------------------------------------------
+# tree K/V in the cache after the prefix; compaction of every layer
+# ----------------------------------------------------------------------------
+
+def test_attention_incache_chain_is_causal_attention_over_the_cache(orc):
+    # with the tree's rows in the cache right after the prefix, a chain tree is
+    # plain causal attention over cache rows [0, S + i] (torch SDPA, a library
+    # routine, with a causal mask offset by S); rows past S + T hold NaN
+    B, T, Hq, Hkv, D, S_max = 2, 5, 4, 2, 8, 16
+    g = torch.Generator().manual_seed(12)
+    q = torch.randn((B, T, Hq, D), generator=g)
+    kc = torch.randn((B, Hkv, S_max, D), generator=g)
+    vc = torch.randn((B, Hkv, S_max, D), generator=g)
+    pl = torch.tensor([9, 0], dtype=torch.int32)
+    for b in range(B):
+        kc[b, :, int(pl[b]) + T:] = float("nan")
+        vc[b, :, int(pl[b]) + T:] = float("nan")
+    par = [-1] + list(range(T - 1))
+    out, _ = orc.tree_attention_incache(q, kc, vc, pl, par)
+    out = out.reshape(B, T, Hq, D)
+    for b in range(B):
+        S = int(pl[b])
+        K_ = kc[b, :, :S + T].double().repeat_interleave(Hq // Hkv, dim=0)
+        V_ = vc[b, :, :S + T].double().repeat_interleave(Hq // Hkv, dim=0)
+        mask = torch.arange(S + T)[None, :] <= (S + torch.arange(T))[:, None]
+        ref = torch.nn.functional.scaled_dot_product_attention(q[b].double().permute(1, 0, 2), K_, V_,
+                                                               attn_mask=mask)
+        np.testing.assert_allclose(out[b], ref.permute(1, 0, 2).numpy(), rtol=1e-12, atol=1e-12)
+
+
+def _row_id_cache(n_layers, B, Hkv, S_max, D, dtype=torch.float32):
+    # every row's values name it: layer * 1e6 + b * 1e4 + g * 1e3 + row + (lane / D)
+    c = torch.empty((n_layers, B, Hkv, S_max, D), dtype=torch.float64)
+    for l in range(n_layers):
+        for b in range(B):
+            for g in range(Hkv):
+                c[l, b, g] = (l * 1e6 + b * 1e4 + g * 1e3 + torch.arange(S_max, dtype=torch.float64)[:, None]
+                              + torch.arange(D, dtype=torch.float64)[None, :] / D)
+    return c.to(dtype)
+
+
+def test_kv_compact_hand_example(orc):
+    # S = 3, path (0, 2, 5): rows 3, 4, 5 <- old rows 3, 5, 8; everything else kept
+    kc = _row_id_cache(1, 1, 2, 12, 4)
+    vc = -kc
+    path = np.array([[0, 2, 5, -1]], np.int32)
+    k2, v2, npl, st = orc.kv_compact([kc[0]], [vc[0]], path, np.array([3], np.int32), np.array([3], np.int32), T=7)
+    assert st == 0 and npl.tolist() == [6]
+    rows = k2[0, 0, 0, :, 0].tolist()
+    assert rows == [0, 1, 2, 3, 5, 8, 6, 7, 8, 9, 10, 11]
+    assert torch.equal(v2, -k2)
+
+
+def test_kv_compact_equals_append_then_commit(orc):
+    # the tree's rows appended after each prefix and compacted = the commit of
+    # the same rows taken as k_tree/v_tree (ragged lengths, every layer alike)
+    B, Hkv, S_max, D, T, n_layers = 3, 2, 24, 8, 7, 3
+    g = torch.Generator().manual_seed(3)
+    kc = torch.randn((n_layers, B, Hkv, S_max, D), generator=g).bfloat16()
+    vc = torch.randn((n_layers, B, Hkv, S_max, D), generator=g).bfloat16()
+    pl = np.array([5, 0, 17], np.int32)
+    path = np.array([[0, 1, 4, 6], [0, 3, -1, -1], [0, 2, 5, -1]], np.int32)
+    ln = np.array([4, 2, 3], np.int32)
+    k2, v2, npl, st = orc.kv_compact(list(kc), list(vc), path, ln, pl, T)
+    assert st == 0 and npl.tolist() == (pl + ln).tolist()
+    for l in range(n_layers):
+        kt = orc.tree_rows_from_cache(kc[l], pl, T)
+        vt = orc.tree_rows_from_cache(vc[l], pl, T)
+        kr, vr, npl_r, st_r = orc.kv_commit(kc[l], vc[l], kt, vt, path, ln, pl)
+        assert st_r == 0 and npl_r.tolist() == npl.tolist()
+        assert torch.equal(k2[l], kr) and torch.equal(v2[l], vr)
+    # and each layer compacted on its own gives the same
+    k1, v1, _, _ = orc.kv_compact([kc[1]], [vc[1]], path, ln, pl, T)
+    assert torch.equal(k1[0], k2[1]) and torch.equal(v1[0], v2[1])
+
+
+def test_kv_compact_refusals(orc):
+    B, Hkv, S_max, D, T = 4, 1, 10, 4, 6
+    kc = _row_id_cache(2, B, Hkv, S_max, D)
+    vc = kc + 0.5
+    pl = np.array([2, 2, 2, 7], np.int32)
+    path = np.array([[0, 3, 3], [0, 6, -1], [0, 1, 2], [0, 1, 3]], np.int32)
+    ln = np.array([3, 2, 4, 3], np.int32)   # repeated node; node >= T; len > max_path; 7 + 3 >= S_max
+    k2, v2, npl, st = orc.kv_compact(list(kc), list(vc), path, ln, pl, T)
+    assert st == 3 and npl.tolist() == pl.tolist()
+    assert torch.equal(k2, kc) and torch.equal(v2, vc)
