@@ -126,6 +126,11 @@ class OracleSample:
         self.ain = I.attention_inputs(w, T)
         self.pc = (I.paged_cache(w, w.page_size, self.ain["prefix_len"], room=T, capacity=w.max_prefix + T)
                    if w.page_size else None)
+        if w.tree_in_cache:   # the tree's K/V after each prefix, as the GPU path holds them
+            for b, tr in enumerate(self.trees):
+                S = int(self.ain["prefix_len"][b])
+                self.ain["k_cache"][b, :, S:S + len(tr)] = self.ain["k_tree"][b, :len(tr)].transpose(0, 1)
+                self.ain["v_cache"][b, :, S:S + len(tr)] = self.ain["v_tree"][b, :len(tr)].transpose(0, 1)
         n_rows = w.B * T * w.Hq
         nr = max(1, int(round(n_rows * fraction)))
         g = np.random.default_rng(seed)
@@ -179,6 +184,8 @@ class OracleSample:
                 Tb = len(trees[b])
                 oracle.tree_attention(ain["q"][b:b + 1, :Tb], ain["k_tree"][b:b + 1, :Tb], ain["v_tree"][b:b + 1, :Tb],
                                       kc[b:b + 1], vc[b:b + 1], ain["prefix_len"][b:b + 1], trees[b], rows=rb)
+        elif w.tree_in_cache:
+            oracle.tree_attention_incache(ain["q"], kc, vc, ain["prefix_len"], self.parents, rows=self.rows)
         else:
             oracle.tree_attention(ain["q"], ain["k_tree"], ain["v_tree"], kc, vc, ain["prefix_len"], self.parents,
                                   rows=self.rows)
@@ -203,6 +210,9 @@ class OracleSample:
         if self.pc is not None:
             oracle.kv_commit_paged(self.pc["k_pages"], self.pc["v_pages"], ain["k_tree"], ain["v_tree"],
                                    self.pc["block_table"], path, ln, ain["prefix_len"])
+        elif w.tree_in_cache:
+            oracle.kv_compact([ain["k_cache"]] * w.layers, [ain["v_cache"]] * w.layers, path, ln, ain["prefix_len"],
+                              T)
         else:
             oracle.kv_commit(ain["k_cache"], ain["v_cache"], ain["k_tree"], ain["v_tree"], path, ln,
                              ain["prefix_len"])
@@ -268,6 +278,9 @@ def config_dict(w, world):
         tree = f"top-s {w.topk}" if w.topk else f"random tree {w.random_tree}"
     if w.page_size:
         tree += f", KV in pages of {w.page_size} via a block table"
+    if w.tree_in_cache:
+        tree += (f", tree K/V appended to the cache after each prefix, commit = in-place compaction of "
+                 f"{w.layers} layers' caches in one launch")
     prefix = f"prefix U[{w.prefix_range[0]}, {w.prefix_range[1]}]" if w.prefix_range else f"prefix {w.prefix}"
     if w.stochastic:
         verify = ("stochastic verify from bf16 logits at temperature " + f"{w.temperature}" if w.temperature > 0
@@ -327,11 +340,23 @@ def run_mine(args, rank, world, local_rank):
                            capacity=w.max_prefix + T)
         ain["k_cache"], ain["v_cache"], block_table = pc["k_pages"], pc["v_pages"], pc["block_table"]
         paged = dict(page_size=w.page_size, max_pages=block_table.shape[1], num_pages=pc["k_pages"].shape[0])
+    k_layers = v_layers = None
+    if w.tree_in_cache:
+        # the tree's K/V appended to each sequence's cache after its prefix (the
+        # target model's layers would write them there); every other layer's
+        # cache is compacted in the same launch
+        for b, tr in enumerate(seq_trees):
+            S = int(ain["prefix_len"][b])
+            ain["k_cache"][b, :, S:S + len(tr)] = ain["k_tree"][b, :len(tr)].transpose(0, 1)
+            ain["v_cache"][b, :, S:S + len(tr)] = ain["v_tree"][b, :len(tr)].transpose(0, 1)
+        k_layers = [ain["k_cache"]] + [ain["k_cache"].clone() for _ in range(w.layers - 1)]
+        v_layers = [ain["v_cache"]] + [ain["v_cache"].clone() for _ in range(w.layers - 1)]
+        ain["k_tree"] = ain["v_tree"] = None
     from medusa_tree_speculative_heads_b200 import binding as Bnd
     mode = Bnd.STOCHASTIC if w.stochastic else Bnd.GREEDY
     step = MedusaStep(B=w.B, d=w.d, V=w.V, K=w.K, Hq=w.Hq, Hkv=w.Hkv, D=w.D, S_max=w.S_max, parents=parents,
                       dtype=w.torch_dtype, max_prefix=w.max_prefix, device=dev, mode=mode, q_rows=T,
-                      temperature=w.temperature, **paged)
+                      temperature=w.temperature, tree_in_cache=w.tree_in_cache, **paged)
     q_draft = vtok = None
     if w.stochastic:
         # the target's and the draft's distributions and the drafted tokens
@@ -352,7 +377,7 @@ def run_mine(args, rank, world, local_rank):
         step.run(h=hin["h"], W_res=hin["W_res"], W_head=hin["W_head"], root_token=hin["root_token"], q=ain["q"],
                  k_tree=ain["k_tree"], v_tree=ain["v_tree"], k_cache=ain["k_cache"], v_cache=ain["v_cache"],
                  prefix_len=ain["prefix_len"], new_prefix_len=new_pl, target=logits, q_draft=q_draft,
-                 node_tokens=vtok, block_table=block_table)
+                 node_tokens=vtok, block_table=block_table, k_layers=k_layers, v_layers=v_layers)
 
     def barrier():
         if world > 1:
@@ -382,7 +407,7 @@ def run_mine(args, rank, world, local_rank):
         step.verify(logits, q_draft, None, 0, i, vtok)
         ev[i][3].record()
         step.commit(ain["k_cache"], ain["v_cache"], ain["k_tree"], ain["v_tree"], ain["prefix_len"], new_pl,
-                    block_table)
+                    block_table, k_layers, v_layers)
         ev[i][4].record()
     e1.record()
     torch.cuda.synchronize()
@@ -400,7 +425,7 @@ def run_mine(args, rank, world, local_rank):
     # the tree's Q/K/V and the target logits) and reads its results back; the
     # copies run on a second stream into two alternating device buffers, so the
     # next step's 31 MB upload overlaps this step's compute, as a serving loop would
-    names_in = ["h", "root_token", "q", "k_tree", "v_tree"]
+    names_in = ["h", "root_token", "q"] + ([] if w.tree_in_cache else ["k_tree", "v_tree"])
     host_in = {n: (hin if n in hin else ain)[n].cpu().pin_memory() for n in names_in}
     host_in["target"] = logits.cpu().pin_memory()
     if w.stochastic:
@@ -421,9 +446,10 @@ def run_mine(args, rank, world, local_rank):
     def run_kwargs(slot):
         d = dev_in[slot]
         return dict(h=d["h"], W_res=hin["W_res"], W_head=hin["W_head"], root_token=d["root_token"], q=d["q"],
-                    k_tree=d["k_tree"], v_tree=d["v_tree"], k_cache=ain["k_cache"], v_cache=ain["v_cache"],
+                    k_tree=d.get("k_tree"), v_tree=d.get("v_tree"), k_cache=ain["k_cache"], v_cache=ain["v_cache"],
                     prefix_len=ain["prefix_len"], new_prefix_len=new_pl, target=d["target"],
-                    q_draft=d.get("q_draft"), node_tokens=d.get("tokens"), block_table=block_table)
+                    q_draft=d.get("q_draft"), node_tokens=d.get("tokens"), block_table=block_table,
+                    k_layers=k_layers, v_layers=v_layers)
 
     # one CUDA graph per input slot: a step is one graph launch on the host
     graphs, e2e_mode = None, "cuda-graph"
@@ -515,8 +541,12 @@ def run_mine(args, rank, world, local_rank):
                            "hbm_gbs": attn_gbs, "hbm_frac": attn_gbs / pk["hbm_gbs"], "tflops": attn_tflops,
                            "tc_frac": attn_tflops / pk["bf16_tflops"], "bound": attn_bound},
         "stage_us": {"medusa_heads": stage[0] * 1e6, "tree_attention": stage[1] * 1e6,
-                     "tree_verify": stage[2] * 1e6, "kv_commit": stage[3] * 1e6},
+                     "tree_verify": stage[2] * 1e6, ("kv_compact" if w.tree_in_cache else "kv_commit"): stage[3] * 1e6},
         "mean_accept_len": mean_len,
+        **({"kv_compact": {"layers": w.layers, "us": stage[3] * 1e6,
+                           "moved_bytes": 2 * 2 * w.layers * w.Hkv * w.D * elt * int(step.accept_len.sum().item()),
+                           "note": "read + write of the accepted rows' K and V in every layer, one launch"}}
+           if w.tree_in_cache else {}),
         "tokens_per_s": value * w.B * (mean_len + 1),
         "e2e": {"value": value_e2e, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "mode": e2e_mode},

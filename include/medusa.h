@@ -11,6 +11,8 @@
  *                   (tree_verify_logits: the stochastic walk reading the
  *                   target's logits at a temperature)
  *   kv_commit       append the accepted path's K/V to the cache
+ * tree_attention_incache and kv_compact are the pair for a cache that already
+ * holds the tree's K/V after each prefix (compaction of every layer at once).
  * tree_attention_paged and kv_commit_paged are the two cache calls over a
  * paged KV cache (a page pool and a block table).
  *
@@ -71,7 +73,8 @@ enum {
     MEDUSA_STATUS_BAD_PREFIX = 4,     /* prefix_len outside [0, max_prefix] */
     MEDUSA_STATUS_NO_MASS = 8,        /* stochastic bonus drawn from an all-zero distribution */
     MEDUSA_STATUS_TIMEOUT = 16,       /* an internal pipeline wait gave up after ~2 s (a library bug) */
-    MEDUSA_STATUS_BAD_PAGE = 32       /* a needed block-table entry outside [0, num_pages) */
+    MEDUSA_STATUS_BAD_PAGE = 32,      /* a needed block-table entry outside [0, num_pages) */
+    MEDUSA_STATUS_BAD_LAYER = 64      /* kv_compact: a layer's cache pointer is NULL or not 16-byte aligned */
 };
 
 typedef enum { MEDUSA_F32 = 0, MEDUSA_BF16 = 1 } medusa_dtype;
@@ -236,6 +239,26 @@ int tree_attention(const void* q, const void* k_tree, const void* v_tree, const 
                    int max_prefix, float scale, medusa_dtype dt, const medusa_tree* tree, void* out, float* lse,
                    void* workspace, size_t workspace_bytes, int32_t* status, medusa_stream_t stream);
 
+/*
+ * tree_attention with this step's tree K/V already written into the cache
+ * right after each prefix (the layout an engine has when the target model's
+ * layers append the tree's K/V to the cache before attention; the commit is
+ * then an in-place compaction, kv_compact):
+ *     k_tree[b, j, g, :] is k_cache[b, g, prefix_len[b] + j, :]  (j < T_b)
+ * and likewise for V.  Every other argument, output and error as
+ * tree_attention; no k_tree / v_tree.  Rows of the cache at or past
+ * prefix_len[b] + T_b are never used (they may hold anything).
+ * Limits: contiguous caches only; max_prefix + T <= S_max (max_prefix 0
+ * means S_max - T), else MEDUSA_ERR_INVALID_ARG.
+ * Workspace: tree_attention_incache_workspace_size(...) bytes.
+ */
+size_t tree_attention_incache_workspace_size(int B, int Hq, int Hkv, int D, int S_max, int max_prefix,
+                                             const medusa_tree* tree, medusa_dtype dt);
+int tree_attention_incache(const void* q, const void* k_cache, const void* v_cache, const int32_t* prefix_len,
+                           int B, int Hq, int Hkv, int D, int S_max, int max_prefix, float scale, medusa_dtype dt,
+                           const medusa_tree* tree, void* out, float* lse, void* workspace, size_t workspace_bytes,
+                           int32_t* status, medusa_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* Verification                                                              */
 /* ------------------------------------------------------------------------ */
@@ -338,6 +361,36 @@ int tree_verify_logits(const void* logits, medusa_dtype logits_dt, double temper
 int kv_commit(void* k_cache, void* v_cache, const void* k_tree, const void* v_tree, const int32_t* accept_path,
               int max_path, const int32_t* accept_len, const int32_t* prefix_len, int32_t* new_prefix_len, int B,
               int T, int Hkv, int D, int S_max, medusa_dtype dt, int32_t* status, medusa_stream_t stream);
+
+/*
+ * The commit when the tree's K/V were appended to the cache before attention
+ * (tree_attention_incache): the accepted path's rows are moved down to just
+ * after the prefix, in place, in every layer's cache in one launch
+ * ([MTP] "The 2D Tree Attention Mask": the longest accepted path is kept;
+ * "Production Deployment Guidelines": the other branches are culled):
+ *     cache_l[b, g, prefix_len[b] + t, :] = old cache_l[b, g, prefix_len[b] + accept_path[b,t], :]
+ * for t < accept_len[b], every layer l < n_layers, K and V, every kv-head g,
+ * bit for bit; then new_prefix_len[b] = prefix_len[b] + accept_len[b].
+ * Rows past the new prefix keep whatever they held.
+ * k_caches, v_caches: DEVICE arrays of n_layers pointers (16-byte aligned
+ *   arrays), each a cache [B, Hkv, S_max, D] of dtype dt, 16-byte aligned,
+ *   updated in place.
+ * accept_path [B, max_path] int32 (strictly increasing node ids < T; the
+ *   output of tree_verify); accept_len [B]; prefix_len [B];
+ *   new_prefix_len [B] out, must not be prefix_len itself (other layers'
+ *   CTAs still read prefix_len), else MEDUSA_ERR_INVALID_ARG.
+ * A sequence whose path is not strictly increasing, holds a node id outside
+ * [0, T) or has accept_len outside [0, max_path] is left untouched
+ * (MEDUSA_STATUS_BAD_TOKEN); one whose rows would reach S_max
+ * (prefix_len + accept_path[L-1] >= S_max) too (MEDUSA_STATUS_CACHE_OVERFLOW);
+ * new_prefix_len = prefix_len for both.  A layer whose pointer is NULL or not
+ * 16-byte aligned is skipped (MEDUSA_STATUS_BAD_LAYER).
+ * Limits: 1 <= n_layers <= 65535; D * element size a multiple of 16 bytes;
+ * T, max_path <= 128.
+ */
+int kv_compact(void* const* k_caches, void* const* v_caches, int n_layers, const int32_t* accept_path, int max_path,
+               const int32_t* accept_len, const int32_t* prefix_len, int32_t* new_prefix_len, int B, int T, int Hkv,
+               int D, int S_max, medusa_dtype dt, int32_t* status, medusa_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* Paged KV cache                                                            */

@@ -118,6 +118,40 @@ def tree_verify_logits(logits: torch.Tensor, temperature: float, q: torch.Tensor
     return out
 
 
+def tree_attention_incache(q, k_cache, v_cache, prefix_len, tree: Tree, scale: float = 0.0, max_prefix: int = 0,
+                           want_lse: bool = False) -> Dict[str, torch.Tensor]:
+    """Tree attention with the tree's K/V in the cache rows right after each
+    prefix: k_cache/v_cache [B,Hkv,S_max,D]."""
+    B, T, Hq, D = q.shape
+    _, Hkv, S_max, _ = k_cache.shape
+    dev = q.device
+    dt = _b.dtype_code(q.dtype)
+    out = {"out": torch.empty_like(q), "status": _status(dev)}
+    if want_lse:
+        out["lse"] = torch.empty((B, T, Hq), dtype=torch.float32, device=dev)
+    nb = _b.tree_attention_incache_workspace_size(B, Hq, Hkv, D, S_max, max_prefix, tree, dt)
+    ws = _ws(nb, dev)
+    _b.tree_attention_incache(q, k_cache, v_cache, prefix_len, B, Hq, Hkv, D, S_max, max_prefix, scale, dt, tree,
+                              out["out"], out.get("lse"), ws, nb, out["status"])
+    return out
+
+
+def kv_compact(k_caches, v_caches, accept_path, accept_len, prefix_len, T: int,
+               new_prefix_len: Optional[torch.Tensor] = None) -> Dict[str, torch.Tensor]:
+    """Compact the accepted path's rows (already in the cache after each
+    prefix) in place, in every layer of the lists k_caches / v_caches
+    ([B,Hkv,S_max,D] each) in one launch; returns new_prefix_len."""
+    B, Hkv, S_max, D = k_caches[0].shape
+    dev = k_caches[0].device
+    if new_prefix_len is None:
+        new_prefix_len = torch.empty_like(prefix_len)
+    kp, vp = _b.layer_pointers(k_caches, dev), _b.layer_pointers(v_caches, dev)
+    st = _status(dev)
+    _b.kv_compact(kp, vp, len(k_caches), accept_path, accept_path.shape[1], accept_len, prefix_len, new_prefix_len, B,
+                  T, Hkv, D, S_max, _b.dtype_code(k_caches[0].dtype), st)
+    return {"new_prefix_len": new_prefix_len, "status": st}
+
+
 def kv_commit(k_cache, v_cache, k_tree, v_tree, accept_path, accept_len, prefix_len,
               new_prefix_len: Optional[torch.Tensor] = None) -> Dict[str, torch.Tensor]:
     """Append the accepted path's K/V in place; returns new_prefix_len (a new
@@ -180,12 +214,16 @@ class MedusaStep:
     [num_pages, Hkv, page_size, D] read and written through a block table
     [B, max_pages] (pass it as ``block_table``), and the paged calls run.
     With ``temperature`` > 0 (stochastic mode) the target passed to
-    ``verify``/``run`` is the target's logits, read by tree_verify_logits."""
+    ``verify``/``run`` is the target's logits, read by tree_verify_logits.
+    With ``tree_in_cache`` the tree's K/V are expected in the (contiguous)
+    cache right after each prefix: attention runs tree_attention_incache and
+    the commit is kv_compact over ``k_layers``/``v_layers`` (every layer's
+    cache; the attended layer's cache among them) in one launch."""
 
     def __init__(self, *, B: int, d: int, V: int, K: int, Hq: int, Hkv: int, D: int, S_max: int,
                  parents, dtype: torch.dtype, mode: int = _b.GREEDY, max_prefix: int = 0,
                  q_rows: int = 0, device=None, page_size: int = 0, max_pages: int = 0, num_pages: int = 0,
-                 temperature: float = 0.0):
+                 temperature: float = 0.0, tree_in_cache: bool = False):
         dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
         self.B, self.d, self.V, self.K = B, d, V, K
         self.Hq, self.Hkv, self.D, self.S_max, self.max_prefix = Hq, Hkv, D, S_max, max_prefix
@@ -210,7 +248,14 @@ class MedusaStep:
         self.status = torch.zeros(1, dtype=i32, device=dev)
         self.ws_heads_n = _b.medusa_heads_workspace_size(B, d, V, K, self.dt)
         self.page_size, self.max_pages, self.num_pages = page_size, max_pages, num_pages
-        if page_size > 0:
+        self.tree_in_cache = tree_in_cache
+        self._layer_ptrs = {}
+        if tree_in_cache and page_size > 0:
+            raise ValueError("the tree-in-cache layout is for contiguous caches")
+        if tree_in_cache:
+            self.ws_attn_n = _b.tree_attention_incache_workspace_size(B, Hq, Hkv, D, S_max, max_prefix, self.tree,
+                                                                      self.dt)
+        elif page_size > 0:
             self.ws_attn_n = _b.tree_attention_paged_workspace_size(B, Hq, Hkv, D, max_prefix, max_pages, page_size,
                                                                     self.tree, self.dt)
         else:
@@ -226,6 +271,11 @@ class MedusaStep:
                         self.ws_heads, self.ws_heads_n, self.status)
 
     def attention(self, q, k_tree, v_tree, k_cache, v_cache, prefix_len, block_table=None):
+        if self.tree_in_cache:
+            _b.tree_attention_incache(q, k_cache, v_cache, prefix_len, self.B, self.Hq, self.Hkv, self.D, self.S_max,
+                                      self.max_prefix, 0.0, self.dt, self.tree, self.attn_out, None, self.ws_attn,
+                                      self.ws_attn_n, self.status)
+            return
         if self.page_size > 0:
             _b.tree_attention_paged(q, k_tree, v_tree, k_cache, v_cache, block_table, self.max_pages, self.page_size,
                                     self.num_pages, prefix_len, self.B, self.Hq, self.Hkv, self.D, self.max_prefix,
@@ -249,7 +299,26 @@ class MedusaStep:
                        step, self.accept_path, self.max_path, self.accept_len, self.bonus, self.ws_verify,
                        self.ws_verify_n, self.status)
 
-    def commit(self, k_cache, v_cache, k_tree, v_tree, prefix_len, new_prefix_len, block_table=None):
+    def layer_pointers(self, k_layers, v_layers):
+        """Device pointer arrays of the layers' caches, built once per list
+        (build them before capturing a graph)."""
+        key = tuple(c.data_ptr() for c in k_layers) + tuple(c.data_ptr() for c in v_layers)
+        if key not in self._layer_ptrs:
+            dev = k_layers[0].device
+            self._layer_ptrs[key] = (_b.layer_pointers(k_layers, dev), _b.layer_pointers(v_layers, dev))
+        return self._layer_ptrs[key]
+
+    def compact(self, k_layers, v_layers, prefix_len, new_prefix_len):
+        kp, vp = self.layer_pointers(k_layers, v_layers)
+        _b.kv_compact(kp, vp, len(k_layers), self.accept_path, self.max_path, self.accept_len, prefix_len,
+                      new_prefix_len, self.B, self.T, self.Hkv, self.D, self.S_max, self.dt, self.status)
+
+    def commit(self, k_cache, v_cache, k_tree, v_tree, prefix_len, new_prefix_len, block_table=None,
+               k_layers=None, v_layers=None):
+        if self.tree_in_cache:
+            self.compact(k_layers if k_layers is not None else [k_cache],
+                         v_layers if v_layers is not None else [v_cache], prefix_len, new_prefix_len)
+            return
         if self.page_size > 0:
             _b.kv_commit_paged(k_cache, v_cache, k_tree, v_tree, block_table, self.max_pages, self.page_size,
                                self.num_pages, self.accept_path, self.max_path, self.accept_len, prefix_len,
@@ -268,8 +337,9 @@ class MedusaStep:
         return g
 
     def run(self, *, h, W_res, W_head, root_token, q, k_tree, v_tree, k_cache, v_cache, prefix_len, new_prefix_len,
-            target, q_draft=None, q_row=None, seed: int = 0, step: int = 0, node_tokens=None, block_table=None):
+            target, q_draft=None, q_row=None, seed: int = 0, step: int = 0, node_tokens=None, block_table=None,
+            k_layers=None, v_layers=None):
         self.heads(h, W_res, W_head, root_token)
         self.attention(q, k_tree, v_tree, k_cache, v_cache, prefix_len, block_table)
         self.verify(target, q_draft, q_row, seed, step, node_tokens)
-        self.commit(k_cache, v_cache, k_tree, v_tree, prefix_len, new_prefix_len, block_table)
+        self.commit(k_cache, v_cache, k_tree, v_tree, prefix_len, new_prefix_len, block_table, k_layers, v_layers)

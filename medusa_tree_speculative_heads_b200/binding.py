@@ -32,6 +32,7 @@ STATUS_BAD_PREFIX = 4
 STATUS_NO_MASS = 8
 STATUS_TIMEOUT = 16
 STATUS_BAD_PAGE = 32
+STATUS_BAD_LAYER = 64
 
 F32, BF16 = 0, 1
 GREEDY, STOCHASTIC = 0, 1
@@ -81,6 +82,11 @@ def lib() -> ctypes.CDLL:
         L.tree_verify_logits.argtypes = [vp, i32, ctypes.c_double, vp, i32, vp, vp, i32, i32, vp, u64, u32, vp, i32,
                                          vp, vp, vp, sz, vp, vp]
         L.kv_commit.argtypes = [vp, vp, vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp]
+        L.tree_attention_incache_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32, vp, i32]
+        L.tree_attention_incache_workspace_size.restype = sz
+        L.tree_attention_incache.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, i32, vp, vp, vp, vp,
+                                             sz, vp, vp]
+        L.kv_compact.argtypes = [vp, vp, i32, vp, i32, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp]
         L.tree_attention_paged_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32, i32, vp, i32]
         L.tree_attention_paged_workspace_size.restype = sz
         L.tree_attention_paged.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, vp, i32, i32, i32, i32, i32, f32,
@@ -221,6 +227,32 @@ def tree_verify_logits(logits, logits_dt, temperature, q, q_rows, q_row, node_to
                                     _p(node_tokens), B, V, tree.handle, ctypes.c_uint64(seed & (2**64 - 1)),
                                     ctypes.c_uint32(step & 0xFFFFFFFF), _p(accept_path), max_path, _p(accept_len),
                                     _p(bonus), _p(workspace), workspace_bytes, _p(status), _stream(stream)))
+
+
+def tree_attention_incache_workspace_size(B, Hq, Hkv, D, S_max, max_prefix, tree: Tree, dt) -> int:
+    return lib().tree_attention_incache_workspace_size(B, Hq, Hkv, D, S_max, max_prefix, tree.handle, dt)
+
+
+def tree_attention_incache(q, k_cache, v_cache, prefix_len, B, Hq, Hkv, D, S_max, max_prefix, scale, dt, tree: Tree,
+                           out, lse, workspace, workspace_bytes, status, stream=None):
+    _check(lib().tree_attention_incache(_p(q), _p(k_cache), _p(v_cache), _p(prefix_len), B, Hq, Hkv, D, S_max,
+                                        max_prefix, float(scale), dt, tree.handle, _p(out), _p(lse), _p(workspace),
+                                        workspace_bytes, _p(status), _stream(stream)))
+
+
+def kv_compact(k_ptrs, v_ptrs, n_layers, accept_path, max_path, accept_len, prefix_len, new_prefix_len, B, T, Hkv, D,
+               S_max, dt, status, stream=None):
+    """k_ptrs, v_ptrs: device int64 tensors [n_layers] holding each layer's
+    cache address (see layer_pointers)."""
+    _check(lib().kv_compact(_p(k_ptrs), _p(v_ptrs), n_layers, _p(accept_path), max_path, _p(accept_len),
+                            _p(prefix_len), _p(new_prefix_len), B, T, Hkv, D, S_max, dt, _p(status),
+                            _stream(stream)))
+
+
+def layer_pointers(caches, device) -> torch.Tensor:
+    """A device int64 tensor of the caches' addresses (the pointer array
+    kv_compact takes)."""
+    return torch.tensor([c.data_ptr() for c in caches], dtype=torch.int64).to(device)
 
 
 def kv_commit(k_cache, v_cache, k_tree, v_tree, accept_path, max_path, accept_len, prefix_len, new_prefix_len, B, T,

@@ -297,27 +297,41 @@ extern "C" size_t tree_attention_workspace_size(int B, int Hq, int Hkv, int D, i
     return attn_workspace_size(B, tree->host.T, Hq, Hkv, D, max_prefix, dt);
 }
 
-extern "C" int tree_attention(const void* q, const void* k_tree, const void* v_tree, const void* k_cache,
-                              const void* v_cache, const int32_t* prefix_len, int B, int Hq, int Hkv, int D,
-                              int S_max, int max_prefix, float scale, medusa_dtype dt, const medusa_tree* tree,
-                              void* out, float* lse, void* workspace, size_t workspace_bytes, int32_t* status,
-                              medusa_stream_t stream) {
-    if (dt != MEDUSA_F32 && dt != MEDUSA_BF16) return fail(MEDUSA_ERR_UNSUPPORTED, "tree_attention: unknown dtype");
-    if (!q || !k_tree || !v_tree || !k_cache || !v_cache || !prefix_len || !out)
-        return fail(MEDUSA_ERR_INVALID_ARG, "tree_attention: NULL tensor argument");
+extern "C" size_t tree_attention_incache_workspace_size(int B, int Hq, int Hkv, int D, int S_max, int max_prefix,
+                                                        const medusa_tree* tree, medusa_dtype dt) {
+    if (!tree || B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || (D != 64 && D != 128)) return 0;
+    if (max_prefix <= 0) max_prefix = S_max - tree->host.T;
+    if (max_prefix < 0) return 0;
+    return attn_workspace_size(B, tree->host.T, Hq, Hkv, D, max_prefix, dt);
+}
+
+// shared by tree_attention and tree_attention_incache (k_tree = v_tree = NULL:
+// the tree's K/V are the cache rows that follow each prefix)
+static int attention_common(const char* fn, const void* q, const void* k_tree, const void* v_tree,
+                            const void* k_cache, const void* v_cache, const int32_t* prefix_len, int B, int Hq,
+                            int Hkv, int D, int S_max, int max_prefix, float scale, medusa_dtype dt,
+                            const medusa_tree* tree, void* out, float* lse, void* workspace, size_t workspace_bytes,
+                            int32_t* status, medusa_stream_t stream) {
+    const bool in_cache = k_tree == nullptr && v_tree == nullptr;
+    if (dt != MEDUSA_F32 && dt != MEDUSA_BF16) return fail(MEDUSA_ERR_UNSUPPORTED, "%s: unknown dtype", fn);
+    if (!q || (!in_cache && (!k_tree || !v_tree)) || !k_cache || !v_cache || !prefix_len || !out)
+        return fail(MEDUSA_ERR_INVALID_ARG, "%s: NULL tensor argument", fn);
     int rc = check_tree(tree, B);
     if (rc) return rc;
     if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || S_max < 0)
-        return fail(MEDUSA_ERR_INVALID_ARG, "tree_attention: bad sizes B=%d Hq=%d Hkv=%d S_max=%d", B, Hq, Hkv, S_max);
-    if (D != 64 && D != 128) return fail(MEDUSA_ERR_UNSUPPORTED, "tree_attention: head_dim %d (64 or 128)", D);
-    if (max_prefix <= 0) max_prefix = S_max;
-    if (max_prefix > S_max)
-        return fail(MEDUSA_ERR_INVALID_ARG, "tree_attention: max_prefix %d > S_max %d", max_prefix, S_max);
+        return fail(MEDUSA_ERR_INVALID_ARG, "%s: bad sizes B=%d Hq=%d Hkv=%d S_max=%d", fn, B, Hq, Hkv, S_max);
+    if (D != 64 && D != 128) return fail(MEDUSA_ERR_UNSUPPORTED, "%s: head_dim %d (64 or 128)", fn, D);
+    const int T = tree->host.T;
+    if (max_prefix <= 0) max_prefix = in_cache ? S_max - T : S_max;
+    if (max_prefix > S_max || (in_cache && max_prefix + T > S_max))
+        return fail(MEDUSA_ERR_INVALID_ARG, "%s: max_prefix %d%s > S_max %d", fn, max_prefix,
+                    in_cache ? " + T" : "", S_max);
+    if (max_prefix < 0) return fail(MEDUSA_ERR_INVALID_ARG, "%s: S_max %d below the tree's T %d", fn, S_max, T);
     if (!al16(q) || !al16(k_tree) || !al16(v_tree) || !al16(k_cache) || !al16(v_cache) || !al16(out))
-        return fail(MEDUSA_ERR_INVALID_ARG, "tree_attention: tensors must be 16-byte aligned");
-    const size_t need = attn_workspace_size(B, tree->host.T, Hq, Hkv, D, max_prefix, dt);
+        return fail(MEDUSA_ERR_INVALID_ARG, "%s: tensors must be 16-byte aligned", fn);
+    const size_t need = attn_workspace_size(B, T, Hq, Hkv, D, max_prefix, dt);
     if (need && (!workspace || workspace_bytes < need || !al16(workspace)))
-        return fail(MEDUSA_ERR_WORKSPACE, "tree_attention: workspace of %zu bytes, need %zu (16-byte aligned)",
+        return fail(MEDUSA_ERR_WORKSPACE, "%s: workspace of %zu bytes, need %zu (16-byte aligned)", fn,
                     workspace_bytes, need);
     AttnArgs a;
     a.q = q;
@@ -327,7 +341,7 @@ extern "C" int tree_attention(const void* q, const void* k_tree, const void* v_t
     a.v_cache = v_cache;
     a.prefix_len = prefix_len;
     a.B = B;
-    a.T = tree->host.T;
+    a.T = T;
     a.Hq = Hq;
     a.Hkv = Hkv;
     a.D = D;
@@ -344,8 +358,28 @@ extern "C" int tree_attention(const void* q, const void* k_tree, const void* v_t
     a.ws_bytes = workspace_bytes;
     a.status = status;
     cudaError_t e = attn_launch(a, (cudaStream_t)stream);
-    if (e != cudaSuccess) return cuda_fail(e, "tree_attention launch");
+    if (e != cudaSuccess) return cuda_fail(e, fn);
     return ok();
+}
+
+extern "C" int tree_attention(const void* q, const void* k_tree, const void* v_tree, const void* k_cache,
+                              const void* v_cache, const int32_t* prefix_len, int B, int Hq, int Hkv, int D,
+                              int S_max, int max_prefix, float scale, medusa_dtype dt, const medusa_tree* tree,
+                              void* out, float* lse, void* workspace, size_t workspace_bytes, int32_t* status,
+                              medusa_stream_t stream) {
+    if (!k_tree || !v_tree) return fail(MEDUSA_ERR_INVALID_ARG, "tree_attention: NULL tensor argument");
+    return attention_common("tree_attention", q, k_tree, v_tree, k_cache, v_cache, prefix_len, B, Hq, Hkv, D, S_max,
+                            max_prefix, scale, dt, tree, out, lse, workspace, workspace_bytes, status, stream);
+}
+
+extern "C" int tree_attention_incache(const void* q, const void* k_cache, const void* v_cache,
+                                      const int32_t* prefix_len, int B, int Hq, int Hkv, int D, int S_max,
+                                      int max_prefix, float scale, medusa_dtype dt, const medusa_tree* tree, void* out,
+                                      float* lse, void* workspace, size_t workspace_bytes, int32_t* status,
+                                      medusa_stream_t stream) {
+    return attention_common("tree_attention_incache", q, nullptr, nullptr, k_cache, v_cache, prefix_len, B, Hq, Hkv,
+                            D, S_max, max_prefix, scale, dt, tree, out, lse, workspace, workspace_bytes, status,
+                            stream);
 }
 
 // ---------------------------------------------------------------------------
@@ -480,6 +514,47 @@ extern "C" int kv_commit(void* k_cache, void* v_cache, const void* k_tree, const
     a.status = status;
     cudaError_t e = commit_launch(a, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "kv_commit launch");
+    return ok();
+}
+
+extern "C" int kv_compact(void* const* k_caches, void* const* v_caches, int n_layers, const int32_t* accept_path,
+                          int max_path, const int32_t* accept_len, const int32_t* prefix_len, int32_t* new_prefix_len,
+                          int B, int T, int Hkv, int D, int S_max, medusa_dtype dt, int32_t* status,
+                          medusa_stream_t stream) {
+    if (dt != MEDUSA_F32 && dt != MEDUSA_BF16) return fail(MEDUSA_ERR_UNSUPPORTED, "kv_compact: unknown dtype");
+    if (!k_caches || !v_caches || !accept_path || !accept_len || !prefix_len || !new_prefix_len)
+        return fail(MEDUSA_ERR_INVALID_ARG, "kv_compact: NULL argument");
+    if (new_prefix_len == prefix_len)
+        return fail(MEDUSA_ERR_INVALID_ARG, "kv_compact: new_prefix_len must not alias prefix_len");
+    const int esize = dt == MEDUSA_BF16 ? 2 : 4;
+    if (n_layers < 1 || n_layers > 65535 || B < 1 || T < 1 || T > kMaxTree || Hkv < 1 || D < 1 || S_max < 0 ||
+        max_path < 1 || max_path > kMaxTree)
+        return fail(MEDUSA_ERR_INVALID_ARG,
+                    "kv_compact: bad sizes n_layers=%d B=%d T=%d Hkv=%d D=%d S_max=%d max_path=%d", n_layers, B, T,
+                    Hkv, D, S_max, max_path);
+    if ((D * esize) % 16)
+        return fail(MEDUSA_ERR_INVALID_ARG, "kv_compact: a K/V row (%d bytes) must be a multiple of 16 bytes",
+                    D * esize);
+    if (!al16(k_caches) || !al16(v_caches))
+        return fail(MEDUSA_ERR_INVALID_ARG, "kv_compact: the pointer arrays must be 16-byte aligned");
+    CompactArgs a;
+    a.k_caches = k_caches;
+    a.v_caches = v_caches;
+    a.n_layers = n_layers;
+    a.accept_path = accept_path;
+    a.max_path = max_path;
+    a.accept_len = accept_len;
+    a.prefix_len = prefix_len;
+    a.new_prefix_len = new_prefix_len;
+    a.B = B;
+    a.T = T;
+    a.Hkv = Hkv;
+    a.D = D;
+    a.S_max = S_max;
+    a.esize = esize;
+    a.status = status;
+    cudaError_t e = compact_launch(a, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "kv_compact launch");
     return ok();
 }
 

@@ -31,7 +31,7 @@ constexpr int kThreads = 128;
 
 struct AttnParams {
     const __nv_bfloat16* q;
-    const __nv_bfloat16* k_tree;
+    const __nv_bfloat16* k_tree;  // NULL: the tree's K/V sit in the cache at rows prefix_len .. prefix_len + T_b
     const __nv_bfloat16* v_tree;
     const __nv_bfloat16* k_cache;
     const __nv_bfloat16* v_cache;
@@ -148,7 +148,11 @@ __global__ void __launch_bounds__(kThreads) tree_attn_mma_kernel(const __grid_co
             bool valid = key < k_end;
             long off;
             const __nv_bfloat16 *ks, *vs;
-            if (tree_split) {
+            if (tree_split && !p.k_tree) {  // the tree's rows follow the prefix in the cache
+                off = (((long)b * p.Hkv + g) * p.S_max + S + (valid ? key : 0)) * D + ch * 8;
+                ks = p.k_cache + off;
+                vs = p.v_cache + off;
+            } else if (tree_split) {
                 off = (((long)b * p.T + (valid ? key : 0)) * p.Hkv + g) * D + ch * 8;
                 ks = p.k_tree + off;
                 vs = p.v_tree + off;
@@ -442,9 +446,15 @@ __global__ void __launch_bounds__(256) tree_attn_f32_kernel(const float* __restr
         const long cbase = ((long)b * Hkv + g) * S_max;
         for (int j = 0; j < S; ++j) visit(k_cache + (cbase + j) * D, v_cache + (cbase + j) * D);
     }
-    for (int j = 0; j < tree->T; ++j)
-        if ((tree->anc[i][j >> 5] >> (j & 31)) & 1u)
+    for (int j = 0; j < tree->T; ++j) {
+        if (!((tree->anc[i][j >> 5] >> (j & 31)) & 1u)) continue;
+        if (k_tree) {
             visit(k_tree + (((long)b * T + j) * Hkv + g) * D, v_tree + (((long)b * T + j) * Hkv + g) * D);
+        } else {  // the tree's rows follow the prefix in the (contiguous) cache
+            const long r = ((long)b * Hkv + g) * S_max + S + j;
+            visit(k_cache + r * D, v_cache + r * D);
+        }
+    }
 #pragma unroll
     for (int e = 0; e < PL; ++e) out[row * D + lane * PL + e] = o[e] / l;
     if (lse && lane == 0) lse[row] = m + logf(l);

@@ -56,7 +56,7 @@ struct TcAttnArgs {
     CUtensorMap mq;    // q as (D, Hq, B*T), box (64, G, 128/G)
     CUtensorMap mkc;   // k_cache as (D, S_max, B*Hkv), box (64, 64, 1); paged: k_pages as
     CUtensorMap mvc;   //   (D, page_size, num_pages*Hkv), box (64, page_rows, 1)
-    CUtensorMap mkt;   // k_tree as (D, Hkv, B*T), box (64, 1, 64)
+    CUtensorMap mkt;   // k_tree as (D, Hkv, B*T), box (64, 1, 64); unused when the tree is in the cache
     CUtensorMap mvt;
     const int32_t* prefix_len;
     TreeRef tree;
@@ -66,6 +66,7 @@ struct TcAttnArgs {
     float* part_lse;   // [n_splits][B*Hkv][R], log2 units
     int32_t* status;
     int B, T, Hq, Hkv, G, S_max, max_prefix, R, n_splits, split_len;
+    int tree_in_cache;  // the tree's K/V are cache rows prefix_len .. prefix_len + T_b (contiguous caches)
     float scale_log2;
 };
 
@@ -227,7 +228,9 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
                     mbar_arrive_expect_tx(bar, kKVBytes);
 #pragma unroll
                     for (int sub = 0; sub < NSUB; ++sub) {
-                        if (tree_split) tma_load_3d(base + sub * kSub, mt, sub * 64, g, b * a.T + cs, bar);
+                        if (tree_split && a.tree_in_cache)  // rows S + cs .. of this (sequence, kv-head)
+                            tma_load_3d(base + sub * kSub, mc, sub * 64, S + cs, bg, bar);
+                        else if (tree_split) tma_load_3d(base + sub * kSub, mt, sub * 64, g, b * a.T + cs, bar);
                         else tma_load_3d(base + sub * kSub, mc, sub * 64, cs, bg, bar);
                     }
                     return;
@@ -567,11 +570,15 @@ cudaError_t attn_tc_launch(const AttnArgs& x, int m_tiles, int n_splits, int spl
     a.page_size = x.page_size;
     a.num_pages = x.num_pages;
     a.page_rows = x.page_size < kCh ? x.page_size : kCh;
-    {
+    a.tree_in_cache = x.k_tree == nullptr;
+    if (!a.tree_in_cache) {
         const uint64_t dims[3] = {D, Hkv, BT}, strides[2] = {D * 2, Hkv * D * 2};
         const uint32_t box[3] = {64, 1, (uint32_t)kCh};
         if (!make_tmap_bf16(&a.mkt, x.k_tree, 3, dims, strides, box)) return cudaErrorInvalidValue;
         if (!make_tmap_bf16(&a.mvt, x.v_tree, 3, dims, strides, box)) return cudaErrorInvalidValue;
+    } else {
+        a.mkt = a.mkc;  // never read
+        a.mvt = a.mvc;
     }
     a.prefix_len = x.prefix_len;
     a.tree = x.tree;

@@ -112,6 +112,21 @@ struct CommitArgs {
 };
 cudaError_t commit_launch(const CommitArgs& a, cudaStream_t st);
 
+// in-place compaction of the tree rows after each prefix, every layer at once
+struct CompactArgs {
+    void* const* k_caches;  // device array [n_layers] of caches [B, Hkv, S_max, D]
+    void* const* v_caches;
+    int n_layers;
+    const int32_t* accept_path;
+    int max_path;
+    const int32_t* accept_len;
+    const int32_t* prefix_len;
+    int32_t* new_prefix_len;
+    int B, T, Hkv, D, S_max, esize;
+    int32_t* status;
+};
+cudaError_t compact_launch(const CompactArgs& a, cudaStream_t st);
+
 // device properties, cached per device
 int num_sms();
 size_t align256(size_t x);

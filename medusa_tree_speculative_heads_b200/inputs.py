@@ -17,6 +17,9 @@ Workloads (all synthetic, no dataset or trained weights exist for them):
 * ``stoch_b64`` bf16, B=64, d=4096, V=32000, K=3, a seeded random 32-node tree
   (depth <= 4 counting the root as 1, <= 6 children), 32/8 heads, head_dim
   128, prefix 1024, stochastic verification.
+* ``llama8b_incache`` llama8b with the tree's K/V appended to the cache after
+  the prefix before attention (S_max = prefix + 128) and the commit as one
+  in-place compaction of 32 layers' caches.
 * ``stoch_logits_b64`` stoch_b64 with verification reading the target's bf16
   logits at temperature 0.7 instead of fp32 probabilities.
 * ``ragged_paged_b8`` bf16, B=8, the llama8b shapes, a random tree per
@@ -65,6 +68,9 @@ class Workload:
     ragged_trees: Optional[tuple] = None   # (T_min, T_max, max_depth, max_children): a random tree per sequence
     page_size: int = 0               # > 0: the KV cache is a page pool read through a block table
     temperature: float = 0.0         # > 0: stochastic verification reads bf16 target logits at this temperature
+    cache_room: int = 64             # cache slots past the longest prefix (S_max = max_prefix + cache_room)
+    tree_in_cache: bool = False      # the tree's K/V are appended to the cache after each prefix before attention
+    layers: int = 1                  # caches compacted per step when the tree is in the cache
 
     @property
     def torch_dtype(self):
@@ -76,8 +82,9 @@ class Workload:
 
     @property
     def S_max(self) -> int:
-        # room for one commit of up to K+1 tokens, rounded to 64 slots
-        return self.max_prefix + 64
+        # room past the longest prefix: one commit of up to K+1 tokens, or the
+        # whole tree when its K/V are appended to the cache
+        return self.max_prefix + self.cache_room
 
 
 WORKLOADS: Dict[str, Workload] = {
@@ -92,6 +99,8 @@ WORKLOADS: Dict[str, Workload] = {
                          topk=(4, 4, 2, 2), match_prob=0.6),
     "stoch_b64": Workload("stoch_b64", 4, BF16, 64, 4096, 32000, 3, 32, 8, 128, 1024,
                           random_tree=(32, 4, 6), stochastic=True),
+    "llama8b_incache": Workload("llama8b_incache", 1, BF16, 1, 4096, 128256, 4, 32, 8, 128, 2048,
+                                topk=(4, 4, 2, 2), match_prob=0.6, cache_room=128, tree_in_cache=True, layers=32),
     "stoch_logits_b64": Workload("stoch_logits_b64", 4, BF16, 64, 4096, 32000, 3, 32, 8, 128, 1024,
                                  random_tree=(32, 4, 6), stochastic=True, temperature=0.7),
     "ragged_paged_b8": Workload("ragged_paged_b8", 5, BF16, 8, 4096, 128256, 4, 32, 8, 128, 8192,
