@@ -4,6 +4,8 @@
  *
  * The step has four calls, run in this order on one CUDA stream:
  *   medusa_heads    Medusa heads, top-s per head, candidate-tree tokens
+ *                   (medusa_heads_shard / medusa_heads_merge: the same over
+ *                   vocabulary shards, one per GPU)
  *   tree_attention  attention of every tree node over the prefix KV cache and
  *                   its tree ancestors (one attention layer)
  *   tree_verify     greedy or stochastic verification: longest accepted
@@ -204,6 +206,55 @@ int medusa_heads_noalloc(const void* h, const void* W_res, const void* W_head, i
                          medusa_dtype dt, const medusa_tree* tree, const int32_t* root_token, int32_t* topk_idx,
                          float* topk_prob, int32_t* node_tokens, float* node_q, void* h_res_out, float* logits_out,
                          float* probs_out, int32_t* status, medusa_stream_t stream);
+
+/*
+ * Vocabulary-sharded heads (one GPU per shard of W_head's rows; the pages
+ * describe no sharding, so this is a library layout, not a step of the
+ * method): the softmax over the full vocabulary and its top-8 are recovered
+ * exactly from each shard's (m, l, top-8), because
+ *     M = max_r m_r,   L = sum_r l_r * exp(m_r - M),   p(x) = exp(z(x) - M) / L
+ * and the global top-8 is the top-8 of the shards' top-8 lists.  Each rank
+ * runs medusa_heads_shard on its rows, the ranks exchange the B*K partials
+ * (72 bytes each; an all-gather in rank order), and every rank (or one) runs
+ * medusa_heads_merge, whose outputs are those of medusa_heads.
+ *
+ * medusa_head_partial: softmax statistics (m = max logit, l = sum of
+ * exp(logit - m)) of one (sequence, head) over a set of vocabulary rows, and
+ * its 8 best (logit, token id) pairs, best first (larger logit, lower id
+ * among equal ones); missing entries are (-inf, INT32_MAX).
+ */
+typedef struct {
+    float m, l;
+    float val[MEDUSA_TOPK];
+    int32_t idx[MEDUSA_TOPK];
+} medusa_head_partial;
+
+/*
+ * medusa_heads over vocabulary rows [v_offset, v_offset + V_shard):
+ * W_head_shard [K, V_shard, d] (those rows of W_head); h, W_res, B, d, K,
+ * dt as medusa_heads (the residual block is computed in full on every
+ * shard).  partial_out [B, K] device: the shard's partial per (sequence,
+ * head), token ids in the full vocabulary.  No tree is filled.
+ * Errors as medusa_heads; v_offset >= 0 and v_offset + V_shard <= INT32_MAX.
+ * Workspace: medusa_heads_shard_workspace_size(B, d, V_shard, K, dt) bytes.
+ */
+size_t medusa_heads_shard_workspace_size(int B, int d, int V_shard, int K, medusa_dtype dt);
+int medusa_heads_shard(const void* h, const void* W_res, const void* W_head_shard, int B, int d, int V_shard,
+                       int v_offset, int K, medusa_dtype dt, medusa_head_partial* partial_out, void* workspace,
+                       size_t workspace_bytes, int32_t* status, medusa_stream_t stream);
+
+/*
+ * Merges n_shards partial sets partials [n_shards, B, K] (device; shard r's
+ * block in rank order, each from medusa_heads_shard) into medusa_heads'
+ * outputs: topk_idx, topk_prob [B, K, 8] and, if tree is given, node_tokens
+ * and node_q [B, T] from root_token [B] (same rules and errors as
+ * medusa_heads).  V is the full vocabulary size (token ids must lie below
+ * it).  The shards' statistics are merged in shard order, so the result does
+ * not depend on which rank merges.  No workspace.
+ */
+int medusa_heads_merge(const medusa_head_partial* partials, int n_shards, int B, int K, int V,
+                       const medusa_tree* tree, const int32_t* root_token, int32_t* topk_idx, float* topk_prob,
+                       int32_t* node_tokens, float* node_q, int32_t* status, medusa_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* Tree attention                                                            */

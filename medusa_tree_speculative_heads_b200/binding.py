@@ -82,6 +82,10 @@ def lib() -> ctypes.CDLL:
         L.tree_verify_logits.argtypes = [vp, i32, ctypes.c_double, vp, i32, vp, vp, i32, i32, vp, u64, u32, vp, i32,
                                          vp, vp, vp, sz, vp, vp]
         L.kv_commit.argtypes = [vp, vp, vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp]
+        L.medusa_heads_shard_workspace_size.argtypes = [i32, i32, i32, i32, i32]
+        L.medusa_heads_shard_workspace_size.restype = sz
+        L.medusa_heads_shard.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp, sz, vp, vp]
+        L.medusa_heads_merge.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp]
         L.tree_attention_incache_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32, vp, i32]
         L.tree_attention_incache_workspace_size.restype = sz
         L.tree_attention_incache.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, i32, vp, vp, vp, vp,
@@ -227,6 +231,26 @@ def tree_verify_logits(logits, logits_dt, temperature, q, q_rows, q_row, node_to
                                     _p(node_tokens), B, V, tree.handle, ctypes.c_uint64(seed & (2**64 - 1)),
                                     ctypes.c_uint32(step & 0xFFFFFFFF), _p(accept_path), max_path, _p(accept_len),
                                     _p(bonus), _p(workspace), workspace_bytes, _p(status), _stream(stream)))
+
+
+PARTIAL_BYTES = 72   # sizeof(medusa_head_partial): m, l, 8 logits, 8 int32 ids
+
+
+def medusa_heads_shard_workspace_size(B, d, V_shard, K, dt) -> int:
+    return lib().medusa_heads_shard_workspace_size(B, d, V_shard, K, dt)
+
+
+def medusa_heads_shard(h, W_res, W_head_shard, B, d, V_shard, v_offset, K, dt, partial_out, workspace,
+                       workspace_bytes, status, stream=None):
+    _check(lib().medusa_heads_shard(_p(h), _p(W_res), _p(W_head_shard), B, d, V_shard, v_offset, K, dt,
+                                    _p(partial_out), _p(workspace), workspace_bytes, _p(status), _stream(stream)))
+
+
+def medusa_heads_merge(partials, n_shards, B, K, V, tree: Optional[Tree], root_token, topk_idx, topk_prob,
+                       node_tokens, node_q, status, stream=None):
+    _check(lib().medusa_heads_merge(_p(partials), n_shards, B, K, V, tree.handle if tree is not None else None,
+                                    _p(root_token), _p(topk_idx), _p(topk_prob), _p(node_tokens), _p(node_q),
+                                    _p(status), _stream(stream)))
 
 
 def tree_attention_incache_workspace_size(B, Hq, Hkv, D, S_max, max_prefix, tree: Tree, dt) -> int:

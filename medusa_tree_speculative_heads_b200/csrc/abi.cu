@@ -2,7 +2,9 @@
 // workspace queries and launches.  See include/medusa.h for the contract of
 // every entry point.
 #include <cmath>
+#include <limits.h>
 #include <stdarg.h>
+#include <stddef.h>
 #include <stdio.h>
 #include <string.h>
 
@@ -223,6 +225,28 @@ extern "C" size_t medusa_heads_workspace_size(int B, int d, int V, int K, medusa
     return heads_workspace_size(B, d, V, K, dt);
 }
 
+// the tree a heads call fills: depth <= K + 1, every sibling rank below
+// min(V, 8), with root tokens and a node-token output
+static int check_heads_tree(const char* fn, const medusa_tree* tree, int B, int V, int K, const int32_t* root_token,
+                            const int32_t* node_tokens) {
+    int rc = check_tree(tree, B);
+    if (rc) return rc;
+    if (!node_tokens || !root_token)
+        return fail(MEDUSA_ERR_INVALID_ARG, "%s: a tree needs root_token and node_tokens", fn);
+    if (tree->host.max_depth > K + 1)
+        return fail(MEDUSA_ERR_INVALID_ARG, "%s: tree depth %d needs more than K=%d heads", fn, tree->host.max_depth,
+                    K);
+    const int smax = V < kTopK ? V : kTopK;
+    for (int n = 0; n < tree->ntrees(); ++n) {
+        const TreeDev& th = tree->trees[n];
+        for (int i = 1; i < th.T; ++i)
+            if (th.rank[i] >= smax)
+                return fail(MEDUSA_ERR_UNSUPPORTED, "%s: node %d of tree %d has sibling rank %d >= %d", fn, i, n,
+                            th.rank[i], smax);
+    }
+    return MEDUSA_OK;
+}
+
 extern "C" int medusa_heads(const void* h, const void* W_res, const void* W_head, int B, int d, int V, int K,
                             medusa_dtype dt, const medusa_tree* tree, const int32_t* root_token, int32_t* topk_idx,
                             float* topk_prob, int32_t* node_tokens, float* node_q, void* h_res_out,
@@ -242,21 +266,8 @@ extern "C" int medusa_heads(const void* h, const void* W_res, const void* W_head
                     workspace_bytes, heads_workspace_size(B, d, V, K, dt));
     int T = 0;
     if (tree) {
-        int rc = check_tree(tree, B);
+        int rc = check_heads_tree("medusa_heads", tree, B, V, K, root_token, node_tokens);
         if (rc) return rc;
-        if (!node_tokens || !root_token)
-            return fail(MEDUSA_ERR_INVALID_ARG, "medusa_heads: a tree needs root_token and node_tokens");
-        if (tree->host.max_depth > K + 1)
-            return fail(MEDUSA_ERR_INVALID_ARG, "medusa_heads: tree depth %d needs more than K=%d heads",
-                        tree->host.max_depth, K);
-        const int smax = V < kTopK ? V : kTopK;
-        for (int n = 0; n < tree->ntrees(); ++n) {
-            const TreeDev& th = tree->trees[n];
-            for (int i = 1; i < th.T; ++i)
-                if (th.rank[i] >= smax)
-                    return fail(MEDUSA_ERR_UNSUPPORTED, "medusa_heads: node %d of tree %d has sibling rank %d >= %d", i,
-                                n, th.rank[i], smax);
-        }
         T = tree->host.T;
     }
     HeadsArgs a;
@@ -283,6 +294,72 @@ extern "C" int medusa_heads(const void* h, const void* W_res, const void* W_head
     a.status = status;
     cudaError_t e = heads_launch(a, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "medusa_heads launch");
+    return ok();
+}
+
+static_assert(sizeof(medusa_head_partial) == 72 && offsetof(medusa_head_partial, val) == 8 &&
+                  offsetof(medusa_head_partial, idx) == 40,
+              "medusa_head_partial must match the kernels' per-(sequence, head) partial");
+
+extern "C" size_t medusa_heads_shard_workspace_size(int B, int d, int V_shard, int K, medusa_dtype dt) {
+    if (B < 1 || d < 1 || V_shard < 1 || K < 1 || K > 16) return 0;
+    return heads_shard_workspace_size(B, d, V_shard, K, dt);
+}
+
+extern "C" int medusa_heads_shard(const void* h, const void* W_res, const void* W_head_shard, int B, int d,
+                                  int V_shard, int v_offset, int K, medusa_dtype dt, medusa_head_partial* partial_out,
+                                  void* workspace, size_t workspace_bytes, int32_t* status, medusa_stream_t stream) {
+    if (dt != MEDUSA_F32 && dt != MEDUSA_BF16) return fail(MEDUSA_ERR_UNSUPPORTED, "medusa_heads_shard: unknown dtype");
+    if (!h || !W_res || !W_head_shard || !partial_out || !workspace)
+        return fail(MEDUSA_ERR_INVALID_ARG, "medusa_heads_shard: NULL argument");
+    if (B < 1 || d < 1 || V_shard < 1 || K < 1 || K > 16 || d > 16384 || v_offset < 0 ||
+        (long long)v_offset + V_shard > INT_MAX)
+        return fail(MEDUSA_ERR_INVALID_ARG, "medusa_heads_shard: bad sizes B=%d d=%d V_shard=%d v_offset=%d K=%d", B,
+                    d, V_shard, v_offset, K);
+    const int vec = dt == MEDUSA_BF16 ? 8 : 4;
+    if (d % vec) return fail(MEDUSA_ERR_INVALID_ARG, "medusa_heads_shard: d=%d must be a multiple of %d", d, vec);
+    if (!al16(h) || !al16(W_res) || !al16(W_head_shard) || !al16(partial_out))
+        return fail(MEDUSA_ERR_INVALID_ARG, "medusa_heads_shard: tensors must be 16-byte aligned");
+    const size_t need = heads_shard_workspace_size(B, d, V_shard, K, dt);
+    if (workspace_bytes < need || !al16(workspace))
+        return fail(MEDUSA_ERR_WORKSPACE, "medusa_heads_shard: workspace of %zu bytes, need %zu (16-byte aligned)",
+                    workspace_bytes, need);
+    HeadsArgs a;
+    memset(&a, 0, sizeof a);
+    a.h = h;
+    a.W_res = W_res;
+    a.W_head = W_head_shard;
+    a.B = B;
+    a.d = d;
+    a.V = V_shard;
+    a.K = K;
+    a.dt = dt;
+    a.tree = TreeRef{nullptr, 0, 0};
+    a.ws = workspace;
+    a.ws_bytes = workspace_bytes;
+    a.status = status;
+    cudaError_t e = heads_shard_launch(a, v_offset, partial_out, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "medusa_heads_shard launch");
+    return ok();
+}
+
+extern "C" int medusa_heads_merge(const medusa_head_partial* partials, int n_shards, int B, int K, int V,
+                                  const medusa_tree* tree, const int32_t* root_token, int32_t* topk_idx,
+                                  float* topk_prob, int32_t* node_tokens, float* node_q, int32_t* status,
+                                  medusa_stream_t stream) {
+    if (!partials || !topk_idx || !topk_prob) return fail(MEDUSA_ERR_INVALID_ARG, "medusa_heads_merge: NULL argument");
+    if (n_shards < 1 || B < 1 || K < 1 || K > 16 || V < 1 || (long long)B * K > 2147483647LL)
+        return fail(MEDUSA_ERR_INVALID_ARG, "medusa_heads_merge: bad sizes n_shards=%d B=%d K=%d V=%d", n_shards, B, K,
+                    V);
+    if (!al16(partials)) return fail(MEDUSA_ERR_INVALID_ARG, "medusa_heads_merge: partials must be 16-byte aligned");
+    if (tree) {
+        int rc = check_heads_tree("medusa_heads_merge", tree, B, V, K, root_token, node_tokens);
+        if (rc) return rc;
+    }
+    cudaError_t e = heads_merge_shards_launch(partials, n_shards, B, K, V, tree ? tree->ref() : TreeRef{nullptr, 0, 0},
+                                              root_token, topk_idx, topk_prob, node_tokens, node_q, status,
+                                              (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "medusa_heads_merge launch");
     return ok();
 }
 

@@ -789,6 +789,112 @@ cudaError_t heads_launch_t(const HeadsArgs& a, cudaStream_t st) {
     return e;
 }
 
+// ---------------------------------------------------------------------------
+// Vocabulary-sharded heads: each shard's (m, l, top-8) per (sequence, head)
+// with global token ids, and the merge of the shards' partials.
+// ---------------------------------------------------------------------------
+
+// one warp per (sequence, head): the shard's statistics and its top-8 logits
+// (read back from the shard's logits at the top-8 ids), ids offset to the
+// full vocabulary
+__global__ void __launch_bounds__(32) heads_pack_shard_kernel(const float2* __restrict__ stats,
+                                                              const int32_t* __restrict__ topk_idx,
+                                                              const float* __restrict__ logits, int BK, int V,
+                                                              int v_offset, HeadState* __restrict__ out) {
+    const int p = blockIdx.x, lane = threadIdx.x;
+    if (p >= BK) return;
+    if (lane < kTopK) {
+        const int i = topk_idx[(long)p * kTopK + lane];
+        out[p].val[lane] = i >= 0 ? logits[(long)p * V + i] : -INFINITY;
+        out[p].idx[lane] = i >= 0 ? i + v_offset : INT_MAX;
+    }
+    if (lane == 0) {
+        const float2 s = stats[p];
+        out[p].m = s.x;
+        out[p].l = s.y;
+    }
+}
+
+// one warp per (sequence, head): the shards' partials merged in shard order
+// (lane r takes shards r, r + 32, ...; the lanes' statistics are then merged
+// by a butterfly and their lists by a warp selection), then the head's
+// top-8 entries, their probabilities exp(logit - M) / L, and the tree nodes
+// this head proposes, as in the unsharded merge
+__global__ void __launch_bounds__(32) heads_merge_shards_kernel(const HeadState* __restrict__ parts, int n_shards,
+                                                                int B, int K, int V_total, TreeRef trees,
+                                                                const int32_t* __restrict__ root_token,
+                                                                int32_t* __restrict__ topk_idx,
+                                                                float* __restrict__ topk_prob,
+                                                                int32_t* __restrict__ node_tokens,
+                                                                float* __restrict__ node_q, int32_t* status) {
+    const int b = blockIdx.x % B, k = blockIdx.x / B, lane = threadIdx.x;
+    float mm = -INFINITY, ll = 0.f;
+    float lv[kTopK];
+    int li[kTopK];
+#pragma unroll
+    for (int j = 0; j < kTopK; ++j) {
+        lv[j] = -INFINITY;
+        li[j] = INT_MAX;
+    }
+    for (int r = lane; r < n_shards; r += 32) {
+        const HeadState* s = &parts[((long)r * B + b) * K + k];
+        merge_ml(mm, ll, s->m, s->l);
+#pragma unroll
+        for (int j = 0; j < kTopK; ++j) list_insert(lv, li, s->val[j], s->idx[j]);
+    }
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float m2 = __shfl_xor_sync(kFull, mm, o);
+        const float l2 = __shfl_xor_sync(kFull, ll, o);
+        merge_ml(mm, ll, m2, l2);
+    }
+    float ov;
+    int oi;
+    warp_select(lv, li, ov, oi);
+    const bool valid = oi != INT_MAX;
+    const float prob = valid ? expf(ov - mm) / ll : 0.f;
+    if (lane < kTopK) {
+        topk_idx[((long)b * K + k) * kTopK + lane] = valid ? oi : -1;
+        topk_prob[((long)b * K + k) * kTopK + lane] = prob;
+    }
+    if (!trees.base) return;
+    const TreeDev* tree = trees.at(b);
+    const int T = tree->T, Tn = trees.T;
+    // every lane takes the (token, prob) of each rank from the lane holding it
+    int tok_r[kTopK];
+    float q_r[kTopK];
+#pragma unroll
+    for (int j = 0; j < kTopK; ++j) {
+        tok_r[j] = __shfl_sync(kFull, valid ? oi : -1, j);
+        q_r[j] = __shfl_sync(kFull, prob, j);
+    }
+    for (int i = lane; i < Tn; i += 32) {
+        if (i > 0 && i < T && tree->depth[i] == k + 2) {
+            int tok = -1;
+            float pq = 0.f;
+#pragma unroll
+            for (int j = 0; j < kTopK; ++j)
+                if (j == tree->rank[i]) {
+                    tok = tok_r[j];
+                    pq = q_r[j];
+                }
+            node_tokens[(long)b * Tn + i] = tok;
+            if (node_q) node_q[(long)b * Tn + i] = pq;
+            if (tok < 0) set_status(status, MEDUSA_STATUS_BAD_TOKEN);
+        }
+        if (k == 0 && i >= T) {  // rows past this sequence's own tree
+            node_tokens[(long)b * Tn + i] = -1;
+            if (node_q) node_q[(long)b * Tn + i] = 0.f;
+        }
+    }
+    if (k == 0 && lane == 0) {
+        const int rt = root_token[b];
+        node_tokens[(long)b * Tn] = rt;
+        if (node_q) node_q[(long)b * Tn] = 1.f;
+        if (rt < 0 || rt >= V_total) set_status(status, MEDUSA_STATUS_BAD_TOKEN);
+    }
+}
+
 }  // namespace
 
 size_t heads_workspace_size(int B, int d, int V, int K, medusa_dtype dt) {
@@ -798,6 +904,40 @@ size_t heads_workspace_size(int B, int d, int V, int K, medusa_dtype dt) {
 cudaError_t heads_launch(const HeadsArgs& a, cudaStream_t st) {
     if (a.dt == MEDUSA_BF16) return heads_launch_t<__nv_bfloat16>(a, st);
     return heads_launch_t<float>(a, st);
+}
+
+size_t heads_shard_workspace_size(int B, int d, int V_shard, int K, medusa_dtype dt) {
+    return heads_ws_layout(B, d, V_shard, K, dt).total + align256((size_t)B * K * kTopK * 8);
+}
+
+cudaError_t heads_shard_launch(const HeadsArgs& x, int v_offset, void* partial_out, cudaStream_t st) {
+    const HeadsWs w = heads_ws_layout(x.B, x.d, x.V, x.K, x.dt);
+    char* ws = (char*)x.ws;
+    HeadsArgs a = x;
+    a.tree = TreeRef{nullptr, 0, 0};
+    a.T = 0;
+    a.root_token = nullptr;
+    a.node_tokens = nullptr;
+    a.node_q = nullptr;
+    a.h_res_out = nullptr;
+    a.probs_out = nullptr;
+    a.logits_out = (float*)(ws + w.logits);  // the shard's logits, for the top-8 values
+    a.topk_idx = (int32_t*)(ws + w.total);
+    a.topk_prob = (float*)(ws + w.total + (size_t)x.B * x.K * kTopK * 4);
+    cudaError_t e = heads_launch(a, st);
+    if (e != cudaSuccess) return e;
+    const int BK = x.B * x.K;
+    heads_pack_shard_kernel<<<BK, 32, 0, st>>>((const float2*)(ws + w.stats), a.topk_idx, a.logits_out, BK, x.V,
+                                               v_offset, (HeadState*)partial_out);
+    return cudaGetLastError();
+}
+
+cudaError_t heads_merge_shards_launch(const void* parts, int n_shards, int B, int K, int V_total, TreeRef tree,
+                                      const int32_t* root_token, int32_t* topk_idx, float* topk_prob,
+                                      int32_t* node_tokens, float* node_q, int32_t* status, cudaStream_t st) {
+    heads_merge_shards_kernel<<<B * K, 32, 0, st>>>((const HeadState*)parts, n_shards, B, K, V_total, tree,
+                                                    root_token, topk_idx, topk_prob, node_tokens, node_q, status);
+    return cudaGetLastError();
 }
 
 }  // namespace medusa

@@ -29,7 +29,9 @@ __device__ __forceinline__ HeadState empty_state() {
     return s;
 }
 
-// merge softmax statistics (m2, l2) into (m, l)
+// merge softmax statistics (m2, l2) into (m, l); every product and the sum
+// rounded once (no fused multiply-add), so merge(a, b) == merge(b, a) bit for
+// bit and the lanes of a butterfly reduction all end with the same (m, l)
 __device__ __forceinline__ void merge_ml(float& m, float& l, float m2, float l2) {
     if (m2 == -INFINITY) return;
     if (m == -INFINITY) {
@@ -38,7 +40,7 @@ __device__ __forceinline__ void merge_ml(float& m, float& l, float m2, float l2)
         return;
     }
     float mn = fmaxf(m, m2);
-    l = l * expf(m - mn) + l2 * expf(m2 - mn);
+    l = __fadd_rn(__fmul_rn(l, expf(m - mn)), __fmul_rn(l2, expf(m2 - mn)));
     m = mn;
 }
 

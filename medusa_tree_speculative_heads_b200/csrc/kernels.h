@@ -32,6 +32,15 @@ struct HeadsArgs {
 };
 size_t heads_workspace_size(int B, int d, int V, int K, medusa_dtype dt);
 cudaError_t heads_launch(const HeadsArgs& a, cudaStream_t st);
+// vocabulary shard: the heads over rows [v_offset, v_offset + V) of the full
+// vocabulary, reduced to one partial (m, l, top-8 logits, global ids) per
+// (sequence, head) in partial_out [B*K] (layout of medusa_head_partial)
+size_t heads_shard_workspace_size(int B, int d, int V_shard, int K, medusa_dtype dt);
+cudaError_t heads_shard_launch(const HeadsArgs& a, int v_offset, void* partial_out, cudaStream_t st);
+// merge of n_shards partial sets [n_shards][B][K] into the heads' outputs
+cudaError_t heads_merge_shards_launch(const void* parts, int n_shards, int B, int K, int V_total, TreeRef tree,
+                                      const int32_t* root_token, int32_t* topk_idx, float* topk_prob,
+                                      int32_t* node_tokens, float* node_q, int32_t* status, cudaStream_t st);
 // tensor-core path (bf16, 1 <= B <= 64, d % 8 == 0)
 bool heads_tc_supported(int B, int d, medusa_dtype dt);
 // ctr: 2 + 2 * num_sms() counters (zeroed here); slots: 2 * num_sms() * B * 128 floats
