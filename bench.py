@@ -388,7 +388,7 @@ def run_mine(args, rank, world, local_rank):
         run_step()
     torch.cuda.synchronize()
 
-    # ---- device-timed steps, with per-stage events ----
+    # ---- per-stage breakdown: the four calls in order on one stream ----
     K = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -397,7 +397,6 @@ def run_mine(args, rank, world, local_rank):
     time.sleep(0.3)
     barrier()
     torch.cuda.synchronize()
-    e0.record()
     for i in range(K):
         ev[i][0].record()
         step.heads(hin["h"], hin["W_res"], hin["W_head"], hin["root_token"])
@@ -410,6 +409,15 @@ def run_mine(args, rank, world, local_rank):
         step.commit(ain["k_cache"], ain["v_cache"], ain["k_tree"], ain["v_tree"], ain["prefix_len"], new_pl,
                     block_table, k_layers, v_layers)
         ev[i][4].record()
+    torch.cuda.synchronize()
+    serial_s = ev[0][0].elapsed_time(ev[K - 1][4]) / 1000.0
+    # ---- device-timed steps (the value): the step as MedusaStep.run issues
+    # it, tree attention on a second stream overlapping the heads' last CTA ----
+    barrier()
+    torch.cuda.synchronize()
+    e0.record()
+    for i in range(K):
+        run_step()
     e1.record()
     torch.cuda.synchronize()
     barrier()
@@ -543,6 +551,7 @@ def run_mine(args, rank, world, local_rank):
                            "tc_frac": attn_tflops / pk["bf16_tflops"], "bound": attn_bound},
         "stage_us": {"medusa_heads": stage[0] * 1e6, "tree_attention": stage[1] * 1e6,
                      "tree_verify": stage[2] * 1e6, ("kv_compact" if w.tree_in_cache else "kv_commit"): stage[3] * 1e6},
+        "serial_ms_per_step": 1000.0 * serial_s / K,
         "mean_accept_len": mean_len,
         **({"kv_compact": {"layers": w.layers, "us": stage[3] * 1e6,
                            "moved_bytes": 2 * 2 * w.layers * w.Hkv * w.D * elt * int(step.accept_len.sum().item()),

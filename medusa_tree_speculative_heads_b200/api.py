@@ -207,7 +207,9 @@ class MedusaStep:
     """All buffers of one decode step of a fixed shape, allocated once.
 
     ``run`` issues the four library calls on the current stream:
-    medusa_heads -> tree_attention -> tree_verify -> kv_commit.  The new
+    medusa_heads -> tree_attention -> tree_verify -> kv_commit, with tree
+    attention on a second stream (joined back before verification) unless
+    ``overlap`` is False.  The new
     prefix lengths go to ``new_prefix_len`` (pass the same tensor as
     ``prefix_len`` to advance in place).  ``parents`` is one parent list, or
     one per sequence.  With ``page_size`` > 0 the cache is a page pool
@@ -223,7 +225,7 @@ class MedusaStep:
     def __init__(self, *, B: int, d: int, V: int, K: int, Hq: int, Hkv: int, D: int, S_max: int,
                  parents, dtype: torch.dtype, mode: int = _b.GREEDY, max_prefix: int = 0,
                  q_rows: int = 0, device=None, page_size: int = 0, max_pages: int = 0, num_pages: int = 0,
-                 temperature: float = 0.0, tree_in_cache: bool = False):
+                 temperature: float = 0.0, tree_in_cache: bool = False, overlap: bool = True):
         dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
         self.B, self.d, self.V, self.K = B, d, V, K
         self.Hq, self.Hkv, self.D, self.S_max, self.max_prefix = Hq, Hkv, D, S_max, max_prefix
@@ -250,6 +252,13 @@ class MedusaStep:
         self.page_size, self.max_pages, self.num_pages = page_size, max_pages, num_pages
         self.tree_in_cache = tree_in_cache
         self._layer_ptrs = {}
+        # run(): tree attention (which reads none of the heads' outputs) on a
+        # second stream, so its CTAs take the SMs the heads kernel frees while
+        # that kernel's last CTA still merges
+        # (the heads on a higher-priority stream: when both calls become ready
+        # at once, the heads kernel, which needs every SM, is dispatched first)
+        self._side = torch.cuda.Stream(device=dev) if overlap else None
+        self._hp = torch.cuda.Stream(device=dev, priority=-1) if overlap else None
         if tree_in_cache and page_size > 0:
             raise ValueError("the tree-in-cache layout is for contiguous caches")
         if tree_in_cache:
@@ -339,7 +348,18 @@ class MedusaStep:
     def run(self, *, h, W_res, W_head, root_token, q, k_tree, v_tree, k_cache, v_cache, prefix_len, new_prefix_len,
             target, q_draft=None, q_row=None, seed: int = 0, step: int = 0, node_tokens=None, block_table=None,
             k_layers=None, v_layers=None):
-        self.heads(h, W_res, W_head, root_token)
-        self.attention(q, k_tree, v_tree, k_cache, v_cache, prefix_len, block_table)
+        if self._side is None:
+            self.heads(h, W_res, W_head, root_token)
+            self.attention(q, k_tree, v_tree, k_cache, v_cache, prefix_len, block_table)
+        else:
+            main = torch.cuda.current_stream(self._side.device)
+            self._hp.wait_stream(main)        # both calls see everything issued before the step
+            self._side.wait_stream(main)
+            with torch.cuda.stream(self._hp):
+                self.heads(h, W_res, W_head, root_token)
+            with torch.cuda.stream(self._side):
+                self.attention(q, k_tree, v_tree, k_cache, v_cache, prefix_len, block_table)
+            main.wait_stream(self._hp)        # verify and commit after both
+            main.wait_stream(self._side)
         self.verify(target, q_draft, q_row, seed, step, node_tokens)
         self.commit(k_cache, v_cache, k_tree, v_tree, prefix_len, new_prefix_len, block_table, k_layers, v_layers)
