@@ -27,8 +27,8 @@
 // Z = sum exp((z - m) / tau) (fp64, fixed reduction order: lanes, warps,
 // CTAs in rank order), and P(y) = exp((z(y) - m) / tau) / Z is evaluated
 // wherever the walk reads P, so no probability row is ever materialised.
-// The fp64 exponentials and Z's summation order differ from a sequential
-// evaluation only in the last bits of P.
+// The fp64 exponentials and Z's summation order (which follows the cluster
+// size) differ from a sequential evaluation only in the last bits of P.
 #include <cooperative_groups.h>
 #include <limits.h>
 
