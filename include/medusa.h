@@ -362,6 +362,23 @@ int tree_verify(medusa_verify_mode mode, const void* target, medusa_dtype target
                 medusa_stream_t stream);
 
 /*
+ * GREEDY verification in its two launches, for callers that run the scan of
+ * the target's rows while other work is still producing the node tokens
+ * (the row scan reads only the target logits; the walk reads the node
+ * tokens).  tree_verify_greedy_rows followed by tree_verify_greedy_walk on
+ * the same workspace gives exactly tree_verify(MEDUSA_VERIFY_GREEDY, ...).
+ * The caller orders the two (same stream, or an event) and must not reuse
+ * the workspace in between.  Arguments as tree_verify; workspace:
+ * tree_verify_workspace_size(MEDUSA_VERIFY_GREEDY, ...).  The walk writes
+ * no status bits (greedy verification has no data-dependent errors).
+ */
+int tree_verify_greedy_rows(const void* target, medusa_dtype target_dt, int B, int V, const medusa_tree* tree,
+                            void* workspace, size_t workspace_bytes, medusa_stream_t stream);
+int tree_verify_greedy_walk(const int32_t* node_tokens, int B, int V, const medusa_tree* tree, int32_t* accept_path,
+                            int max_path, int32_t* accept_len, int32_t* bonus, const void* workspace,
+                            size_t workspace_bytes, medusa_stream_t stream);
+
+/*
  * STOCHASTIC verification reading the target's logits instead of its
  * probabilities: the walk of tree_verify (STOCHASTIC) with P, wherever the
  * walk reads the target's own row of node u, taken as

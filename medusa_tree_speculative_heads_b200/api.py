@@ -259,6 +259,8 @@ class MedusaStep:
         # at once, the heads kernel, which needs every SM, is dispatched first)
         self._side = torch.cuda.Stream(device=dev) if overlap else None
         self._hp = torch.cuda.Stream(device=dev, priority=-1) if overlap else None
+        # greedy verification's scan of the target rows reads neither: a third stream
+        self._side2 = torch.cuda.Stream(device=dev) if overlap else None
         if tree_in_cache and page_size > 0:
             raise ValueError("the tree-in-cache layout is for contiguous caches")
         if tree_in_cache:
@@ -353,13 +355,29 @@ class MedusaStep:
             self.attention(q, k_tree, v_tree, k_cache, v_cache, prefix_len, block_table)
         else:
             main = torch.cuda.current_stream(self._side.device)
-            self._hp.wait_stream(main)        # both calls see everything issued before the step
+            greedy_split = self.mode == _b.GREEDY and self.temperature <= 0
+            self._hp.wait_stream(main)        # every call sees everything issued before the step
             self._side.wait_stream(main)
             with torch.cuda.stream(self._hp):
                 self.heads(h, W_res, W_head, root_token)
             with torch.cuda.stream(self._side):
                 self.attention(q, k_tree, v_tree, k_cache, v_cache, prefix_len, block_table)
-            main.wait_stream(self._hp)        # verify and commit after both
+            if greedy_split:
+                self._side2.wait_stream(main)
+                with torch.cuda.stream(self._side2):
+                    _b.tree_verify_greedy_rows(target, _b.dtype_code(target.dtype), self.B, self.V, self.tree,
+                                               self.ws_verify, self.ws_verify_n)
+                main.wait_stream(self._side2)
+            main.wait_stream(self._hp)        # the walk (or the whole verification) and commit after all
             main.wait_stream(self._side)
+            if greedy_split:
+                _b.tree_verify_greedy_walk(self.node_tokens if node_tokens is None else node_tokens, self.B, self.V,
+                                           self.tree, self.accept_path, self.max_path, self.accept_len, self.bonus,
+                                           self.ws_verify, self.ws_verify_n)
+            else:
+                self.verify(target, q_draft, q_row, seed, step, node_tokens)
+            self.commit(k_cache, v_cache, k_tree, v_tree, prefix_len, new_prefix_len, block_table, k_layers,
+                        v_layers)
+            return
         self.verify(target, q_draft, q_row, seed, step, node_tokens)
         self.commit(k_cache, v_cache, k_tree, v_tree, prefix_len, new_prefix_len, block_table, k_layers, v_layers)

@@ -79,6 +79,8 @@ def lib() -> ctypes.CDLL:
         L.tree_verify_workspace_size.restype = sz
         L.tree_verify.argtypes = [i32, vp, i32, vp, i32, vp, vp, i32, i32, vp, u64, u32, vp, i32, vp, vp, vp, sz, vp,
                                   vp]
+        L.tree_verify_greedy_rows.argtypes = [vp, i32, i32, i32, vp, vp, sz, vp]
+        L.tree_verify_greedy_walk.argtypes = [vp, i32, i32, vp, vp, i32, vp, vp, vp, sz, vp]
         L.tree_verify_logits.argtypes = [vp, i32, ctypes.c_double, vp, i32, vp, vp, i32, i32, vp, u64, u32, vp, i32,
                                          vp, vp, vp, sz, vp, vp]
         L.kv_commit.argtypes = [vp, vp, vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp]
@@ -223,6 +225,17 @@ def tree_verify(mode, target, target_dt, q, q_rows, q_row, node_tokens, B, V, tr
                              tree.handle, ctypes.c_uint64(seed & (2**64 - 1)), ctypes.c_uint32(step & 0xFFFFFFFF),
                              _p(accept_path), max_path, _p(accept_len), _p(bonus), _p(workspace), workspace_bytes,
                              _p(status), _stream(stream)))
+
+
+def tree_verify_greedy_rows(target, target_dt, B, V, tree: Tree, workspace, workspace_bytes, stream=None):
+    _check(lib().tree_verify_greedy_rows(_p(target), target_dt, B, V, tree.handle, _p(workspace), workspace_bytes,
+                                         _stream(stream)))
+
+
+def tree_verify_greedy_walk(node_tokens, B, V, tree: Tree, accept_path, max_path, accept_len, bonus, workspace,
+                            workspace_bytes, stream=None):
+    _check(lib().tree_verify_greedy_walk(_p(node_tokens), B, V, tree.handle, _p(accept_path), max_path,
+                                         _p(accept_len), _p(bonus), _p(workspace), workspace_bytes, _stream(stream)))
 
 
 def tree_verify_logits(logits, logits_dt, temperature, q, q_rows, q_row, node_tokens, B, V, tree: Tree, seed, step,

@@ -540,6 +540,69 @@ extern "C" int tree_verify(medusa_verify_mode mode, const void* target, medusa_d
                          status, stream);
 }
 
+extern "C" int tree_verify_greedy_rows(const void* target, medusa_dtype target_dt, int B, int V,
+                                       const medusa_tree* tree, void* workspace, size_t workspace_bytes,
+                                       medusa_stream_t stream) {
+    if (!target) return fail(MEDUSA_ERR_INVALID_ARG, "tree_verify_greedy_rows: NULL target");
+    if (target_dt != MEDUSA_F32 && target_dt != MEDUSA_BF16)
+        return fail(MEDUSA_ERR_UNSUPPORTED, "tree_verify_greedy_rows: logits dtype must be MEDUSA_F32 or MEDUSA_BF16");
+    int rc = check_tree(tree, B);
+    if (rc) return rc;
+    if (B < 1 || V < 1) return fail(MEDUSA_ERR_INVALID_ARG, "tree_verify_greedy_rows: bad sizes B=%d V=%d", B, V);
+    const size_t need = verify_workspace_size(MEDUSA_VERIFY_GREEDY, B, V, tree->host.T);
+    if (!workspace || workspace_bytes < need || !al16(workspace))
+        return fail(MEDUSA_ERR_WORKSPACE, "tree_verify_greedy_rows: workspace of %zu bytes, need %zu",
+                    workspace_bytes, need);
+    VerifyArgs a;
+    memset(&a, 0, sizeof a);
+    a.mode = MEDUSA_VERIFY_GREEDY;
+    a.target = target;
+    a.target_dt = target_dt;
+    a.B = B;
+    a.V = V;
+    a.T = tree->host.T;
+    a.tree = tree->ref();
+    a.ws = workspace;
+    a.ws_bytes = workspace_bytes;
+    cudaError_t e = verify_greedy_rows_launch(a, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "tree_verify_greedy_rows");
+    return ok();
+}
+
+extern "C" int tree_verify_greedy_walk(const int32_t* node_tokens, int B, int V, const medusa_tree* tree,
+                                       int32_t* accept_path, int max_path, int32_t* accept_len, int32_t* bonus,
+                                       const void* workspace, size_t workspace_bytes, medusa_stream_t stream) {
+    if (!node_tokens || !accept_path || !accept_len || !bonus)
+        return fail(MEDUSA_ERR_INVALID_ARG, "tree_verify_greedy_walk: NULL tensor argument");
+    int rc = check_tree(tree, B);
+    if (rc) return rc;
+    if (B < 1 || V < 1) return fail(MEDUSA_ERR_INVALID_ARG, "tree_verify_greedy_walk: bad sizes B=%d V=%d", B, V);
+    if (max_path < tree->host.max_depth || max_path > kMaxTree)
+        return fail(MEDUSA_ERR_INVALID_ARG, "tree_verify_greedy_walk: max_path %d outside [tree depth %d, %d]",
+                    max_path, tree->host.max_depth, kMaxTree);
+    const size_t need = verify_workspace_size(MEDUSA_VERIFY_GREEDY, B, V, tree->host.T);
+    if (!workspace || workspace_bytes < need || !al16(workspace))
+        return fail(MEDUSA_ERR_WORKSPACE, "tree_verify_greedy_walk: workspace of %zu bytes, need %zu",
+                    workspace_bytes, need);
+    VerifyArgs a;
+    memset(&a, 0, sizeof a);
+    a.mode = MEDUSA_VERIFY_GREEDY;
+    a.node_tokens = node_tokens;
+    a.B = B;
+    a.V = V;
+    a.T = tree->host.T;
+    a.tree = tree->ref();
+    a.accept_path = accept_path;
+    a.max_path = max_path;
+    a.accept_len = accept_len;
+    a.bonus = bonus;
+    a.ws = const_cast<void*>(workspace);
+    a.ws_bytes = workspace_bytes;
+    cudaError_t e = verify_greedy_walk_launch(a, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "tree_verify_greedy_walk");
+    return ok();
+}
+
 extern "C" int tree_verify_logits(const void* logits, medusa_dtype logits_dt, double temperature, const float* q,
                                   int q_rows, const int32_t* q_row, const int32_t* node_tokens, int B, int V,
                                   const medusa_tree* tree, uint64_t seed, uint32_t step, int32_t* accept_path,

@@ -102,6 +102,9 @@ struct VerifyArgs {
 };
 size_t verify_workspace_size(medusa_verify_mode mode, int B, int V, int T);
 cudaError_t verify_launch(const VerifyArgs& a, cudaStream_t st);
+// greedy mode's two launches on their own (verify_launch = rows then walk)
+cudaError_t verify_greedy_rows_launch(const VerifyArgs& a, cudaStream_t st);
+cudaError_t verify_greedy_walk_launch(const VerifyArgs& a, cudaStream_t st);
 
 // ------------------------------- commit ------------------------------------
 struct CommitArgs {

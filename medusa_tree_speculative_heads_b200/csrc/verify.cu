@@ -513,26 +513,40 @@ size_t verify_workspace_size(medusa_verify_mode mode, int B, int V, int T) {
     return align256((size_t)B * T * s * sizeof(float)) + align256((size_t)B * T * s * sizeof(int));
 }
 
+// greedy: the row-argmax partials of every node's target row, in workspace
+cudaError_t verify_greedy_rows_launch(const VerifyArgs& a, cudaStream_t st) {
+    const int rows = a.B * a.T;
+    const int splits = argmax_splits(rows, a.V);
+    int chunk = (a.V + splits - 1) / splits;
+    chunk = (chunk + 7) / 8 * 8;
+    float* pval = (float*)a.ws;
+    int* pidx = (int*)((char*)a.ws + align256((size_t)rows * splits * sizeof(float)));
+    dim3 grid(rows, splits);
+    if (a.target_dt == MEDUSA_BF16)
+        row_argmax_kernel<__nv_bfloat16>
+            <<<grid, kArgmaxThreads, 0, st>>>((const __nv_bfloat16*)a.target, a.V, splits, chunk, pval, pidx);
+    else
+        row_argmax_kernel<float><<<grid, kArgmaxThreads, 0, st>>>((const float*)a.target, a.V, splits, chunk, pval,
+                                                                  pidx);
+    return cudaGetLastError();
+}
+
+// greedy: the tree walk over those partials
+cudaError_t verify_greedy_walk_launch(const VerifyArgs& a, cudaStream_t st) {
+    const int rows = a.B * a.T;
+    const int splits = argmax_splits(rows, a.V);
+    const float* pval = (const float*)a.ws;
+    const int* pidx = (const int*)((const char*)a.ws + align256((size_t)rows * splits * sizeof(float)));
+    greedy_walk_kernel<<<a.B, kWalkThreads, 0, st>>>(pval, pidx, splits, a.node_tokens, a.tree, a.accept_path,
+                                                     a.max_path, a.accept_len, a.bonus);
+    return cudaGetLastError();
+}
+
 cudaError_t verify_launch(const VerifyArgs& a, cudaStream_t st) {
     if (a.mode == MEDUSA_VERIFY_GREEDY) {
-        const int rows = a.B * a.T;
-        const int splits = argmax_splits(rows, a.V);
-        int chunk = (a.V + splits - 1) / splits;
-        chunk = (chunk + 7) / 8 * 8;
-        float* pval = (float*)a.ws;
-        int* pidx = (int*)((char*)a.ws + align256((size_t)rows * splits * sizeof(float)));
-        dim3 grid(rows, splits);
-        if (a.target_dt == MEDUSA_BF16)
-            row_argmax_kernel<__nv_bfloat16>
-                <<<grid, kArgmaxThreads, 0, st>>>((const __nv_bfloat16*)a.target, a.V, splits, chunk, pval, pidx);
-        else
-            row_argmax_kernel<float><<<grid, kArgmaxThreads, 0, st>>>((const float*)a.target, a.V, splits, chunk,
-                                                                      pval, pidx);
-        cudaError_t e = cudaGetLastError();
+        cudaError_t e = verify_greedy_rows_launch(a, st);
         if (e != cudaSuccess) return e;
-        greedy_walk_kernel<<<a.B, kWalkThreads, 0, st>>>(pval, pidx, splits, a.node_tokens, a.tree, a.accept_path,
-                                                         a.max_path, a.accept_len, a.bonus);
-        return cudaGetLastError();
+        return verify_greedy_walk_launch(a, st);
     }
     const int C = stoch_cluster(a.B);
     unsigned long long* ws_w = (unsigned long long*)a.ws;

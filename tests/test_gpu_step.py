@@ -123,3 +123,40 @@ def test_graph_replay_equals_eager_step(name):
         path, ln, bonus, _ = oracle.verify_stochastic_logits(target, tau, q_draft, tok, parents, 0, 5, maxd)
         assert np.array_equal(step.accept_path.cpu().numpy(), path)
         assert np.array_equal(step.accept_len.cpu().numpy(), ln) and np.array_equal(step.bonus.cpu().numpy(), bonus)
+
+
+@pytest.mark.parametrize("name", ["llama8b_small", "stoch_small"])
+def test_overlapped_step_equals_the_calls_in_order(name):
+    # run() with attention (and greedy verification's row scan) on side
+    # streams gives the in-order step's results bit for bit
+    if name == "llama8b_small":
+        w = I.scaled(I.WORKLOADS["llama8b"], B=2, d=512, V=3001, prefix=300)
+    else:
+        w = I.scaled(I.WORKLOADS["stoch_b64"], B=3, V=900)
+    parents = I.workload_tree(w)
+    T = len(parents)
+    from medusa_tree_speculative_heads_b200 import binding as Bnd
+    mode = Bnd.STOCHASTIC if w.stochastic else Bnd.GREEDY
+    hin = {k: v.cuda() for k, v in I.head_inputs(w).items()}
+    ain = {k: v.cuda() for k, v in I.attention_inputs(w, T).items()}
+    if w.stochastic:
+        sd = {k: v.cuda() for k, v in I.stochastic_inputs(w, parents).items()}
+        target, q_draft, tok = sd["p"], sd["q"], sd["node_tokens"]
+    else:
+        target = torch.randn((w.B, T, w.V), generator=torch.Generator().manual_seed(2)).to(w.torch_dtype).cuda()
+        q_draft = tok = None
+    results = []
+    for overlap in (False, True):
+        step = MedusaStep(B=w.B, d=w.d, V=w.V, K=w.K, Hq=w.Hq, Hkv=w.Hkv, D=w.D, S_max=w.S_max, parents=parents,
+                          dtype=w.torch_dtype, device="cuda", mode=mode, q_rows=T, overlap=overlap)
+        kc, vc = ain["k_cache"].clone(), ain["v_cache"].clone()
+        new_pl = torch.empty_like(ain["prefix_len"])
+        step.run(h=hin["h"], W_res=hin["W_res"], W_head=hin["W_head"], root_token=hin["root_token"], q=ain["q"],
+                 k_tree=ain["k_tree"], v_tree=ain["v_tree"], k_cache=kc, v_cache=vc, prefix_len=ain["prefix_len"],
+                 new_prefix_len=new_pl, target=target, q_draft=q_draft, node_tokens=tok, step=3)
+        torch.cuda.synchronize()
+        assert int(step.status.item()) == 0
+        results.append([x.clone() for x in (step.node_tokens, step.attn_out, step.accept_path, step.accept_len,
+                                            step.bonus, new_pl, kc, vc)])
+    for a, b in zip(*results):
+        assert torch.equal(a, b)

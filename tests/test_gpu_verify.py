@@ -233,3 +233,32 @@ def test_stochastic_logits_no_mass_and_bad_temperature():
         with pytest.raises(B.MedusaError) as e:
             api.tree_verify_logits(z.cuda(), tau, q.cuda(), tok.cuda(), Tree(parents))
         assert e.value.code == B.MEDUSA_ERR_INVALID_ARG
+
+
+def test_greedy_rows_then_walk_on_two_streams_is_tree_verify():
+    # the row scan on one stream, the walk on another after an event: the same
+    # result as the one-call greedy verification
+    w = I.scaled(I.WORKLOADS["llama8b"], B=3, V=5000)
+    parents = I.workload_tree(w)
+    tok, logits = greedy_case(w, parents)
+    tree = Tree(parents)
+    lg, tk = logits.cuda(), tok.cuda()
+    ref = api.tree_verify(B.GREEDY, lg, tk, tree)
+    nb = B.tree_verify_workspace_size(B.GREEDY, w.B, w.V, tree)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    path = torch.full_like(ref["accept_path"], -7)
+    ln = torch.full_like(ref["accept_len"], -7)
+    bonus = torch.full_like(ref["bonus"], -7)
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    done = torch.cuda.Event()
+    with torch.cuda.stream(s1):
+        B.tree_verify_greedy_rows(lg, B.dtype_code(lg.dtype), w.B, w.V, tree, ws, nb)
+        done.record(s1)
+    s2.wait_event(done)
+    with torch.cuda.stream(s2):
+        B.tree_verify_greedy_walk(tk, w.B, w.V, tree, path, tree.max_depth, ln, bonus, ws, nb)
+    torch.cuda.synchronize()
+    assert torch.equal(path, ref["accept_path"]) and torch.equal(ln, ref["accept_len"])
+    assert torch.equal(bonus, ref["bonus"])
+    assert_same({"accept_path": path, "accept_len": ln, "bonus": bonus},
+                oracle.verify_greedy(logits, tok, parents, tree.max_depth))
