@@ -123,3 +123,54 @@ def test_paged_calls_validate_before_launch(lib):
     # the paged workspace query mirrors the contiguous one's domain
     assert lib.tree_attention_paged_workspace_size(1, 4, 2, 96, 0, 4, 16, nul, 1) == 0
     assert lib.tree_attention_paged_workspace_size(1, 4, 2, 128, 0, 0, 16, nul, 1) == 0
+
+
+def test_newer_calls_validate_before_launch(lib):
+    # every failure here is found on the host, before any device work
+    fake = ctypes.c_void_p(0x1000)
+    other = ctypes.c_void_p(0x2000)
+    nul = None
+    INV, UNS, WS = B.MEDUSA_ERR_INVALID_ARG, B.MEDUSA_ERR_UNSUPPORTED, B.MEDUSA_ERR_WORKSPACE
+    # kv_compact: NULL arrays, aliased prefix lengths, sizes, row alignment, dtype
+    args = dict(kc=fake, vc=fake, nl=4, path=fake, mp=5, ln=fake, pl=fake, npl=other, B_=2, T=8, Hkv=2, D=128,
+                S=64, dt=1)
+
+    def compact(**kw):
+        a = {**args, **kw}
+        return lib.kv_compact(a["kc"], a["vc"], a["nl"], a["path"], a["mp"], a["ln"], a["pl"], a["npl"], a["B_"],
+                              a["T"], a["Hkv"], a["D"], a["S"], a["dt"], nul, nul)
+    assert compact(kc=nul) == INV
+    assert compact(npl=fake) == INV and b"alias" in lib.medusa_last_error()
+    assert compact(nl=0) == INV and compact(nl=70000) == INV
+    assert compact(mp=129) == INV and compact(T=129) == INV
+    assert compact(D=4) == INV                                  # 8-byte rows
+    assert compact(dt=7) == UNS
+    assert compact(kc=ctypes.c_void_p(0x1008)) == INV           # the pointer array itself misaligned
+    # sharded heads
+    part = fake
+    assert lib.medusa_heads_shard(fake, fake, fake, 1, 64, 100, 0, 2, 1, nul, fake, 1 << 30, nul, nul) == INV
+    assert lib.medusa_heads_shard(fake, fake, fake, 1, 64, 100, -1, 2, 1, part, fake, 1 << 30, nul, nul) == INV
+    assert lib.medusa_heads_shard(fake, fake, fake, 1, 60, 100, 0, 2, 1, part, fake, 1 << 30, nul, nul) == INV
+    assert lib.medusa_heads_shard(fake, fake, fake, 1, 64, 100, 0, 17, 1, part, fake, 1 << 30, nul, nul) == INV
+    assert lib.medusa_heads_shard(fake, fake, fake, 1, 64, 100, 0, 2, 1, part, fake, 16, nul, nul) == WS
+    assert lib.medusa_heads_shard(fake, fake, fake, 1, 64, 100, 0, 2, 5, part, fake, 1 << 30, nul, nul) == UNS
+    assert lib.medusa_heads_shard_workspace_size(1, 64, 0, 2, 1) == 0
+    assert lib.medusa_heads_shard_workspace_size(1, 64, 100, 2, 1) >= lib.medusa_heads_workspace_size(1, 64, 100, 2, 1)
+    assert lib.medusa_heads_merge(nul, 2, 1, 2, 100, nul, nul, fake, fake, nul, nul, nul, nul) == INV
+    assert lib.medusa_heads_merge(fake, 0, 1, 2, 100, nul, nul, fake, fake, nul, nul, nul, nul) == INV
+    assert lib.medusa_heads_merge(ctypes.c_void_p(0x1004), 2, 1, 2, 100, nul, nul, fake, fake, nul, nul, nul,
+                                  nul) == INV
+    # tree K/V in the cache, logits verify, two-launch greedy verify: NULLs and a missing tree
+    assert lib.tree_attention_incache(nul, fake, fake, fake, 1, 4, 2, 128, 256, 0, ctypes.c_float(0), 1, nul, fake,
+                                      nul, fake, 1 << 20, nul, nul) == INV
+    assert lib.tree_attention_incache(fake, fake, fake, fake, 1, 4, 2, 128, 256, 0, ctypes.c_float(0), 1, nul, fake,
+                                      nul, fake, 1 << 20, nul, nul) == INV           # tree NULL
+    assert lib.tree_verify_logits(nul, 1, ctypes.c_double(1.0), fake, 4, nul, fake, 1, 100, nul, 0, 0, fake, 4,
+                                  fake, fake, fake, 1 << 20, nul, nul) == INV
+    assert lib.tree_verify_logits(fake, 5, ctypes.c_double(1.0), fake, 4, nul, fake, 1, 100, nul, 0, 0, fake, 4,
+                                  fake, fake, fake, 1 << 20, nul, nul) == INV        # tree NULL comes first
+    assert lib.tree_verify_greedy_rows(nul, 1, 1, 100, nul, fake, 1 << 20, nul) == INV
+    assert lib.tree_verify_greedy_rows(fake, 5, 1, 100, nul, fake, 1 << 20, nul) == UNS
+    assert lib.tree_verify_greedy_walk(nul, 1, 100, nul, fake, 4, fake, fake, fake, 1 << 20, nul) == INV
+    assert lib.tree_verify_greedy_walk(fake, 1, 100, nul, fake, 4, fake, fake, fake, 1 << 20, nul) == INV
+    assert lib.tree_attention_incache_workspace_size(1, 4, 2, 96, 256, 0, nul, 1) == 0
