@@ -543,6 +543,7 @@ cudaError_t attn_launch_bf16(const AttnArgs& a, cudaStream_t st) {
     }
     if (e != cudaSuccess) return e;
     const long rows = (long)a.B * a.T * a.Hq;
+    prefer_max_smem(attn_combine_kernel<D>);
     attn_combine_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(p.part_o, p.part_lse, a.B, a.T, a.Hq, a.Hkv,
                                                                      sp.n_splits, a.tree, (__nv_bfloat16*)a.out, a.lse);
     return cudaGetLastError();

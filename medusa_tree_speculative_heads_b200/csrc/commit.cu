@@ -147,6 +147,7 @@ __global__ void __launch_bounds__(128) kv_compact_kernel(uint8_t* const* __restr
 
 cudaError_t compact_launch(const CompactArgs& a, cudaStream_t st) {
     const dim3 grid(a.B, a.n_layers);
+    prefer_max_smem(kv_compact_kernel);
     kv_compact_kernel<<<grid, 128, 0, st>>>((uint8_t* const*)a.k_caches, (uint8_t* const*)a.v_caches, a.accept_path,
                                             a.max_path, a.accept_len, a.prefix_len, a.new_prefix_len, a.T, a.Hkv,
                                             a.S_max, a.D * a.esize, a.status);
@@ -154,6 +155,7 @@ cudaError_t compact_launch(const CompactArgs& a, cudaStream_t st) {
 }
 
 cudaError_t commit_launch(const CommitArgs& a, cudaStream_t st) {
+    prefer_max_smem(kv_commit_kernel);
     kv_commit_kernel<<<a.B, 256, 0, st>>>((uint8_t*)a.k_cache, (uint8_t*)a.v_cache, (const uint8_t*)a.k_tree,
                                           (const uint8_t*)a.v_tree, a.accept_path, a.max_path, a.accept_len,
                                           a.prefix_len, a.new_prefix_len, a.T, a.Hkv, a.S_max, a.D * a.esize,

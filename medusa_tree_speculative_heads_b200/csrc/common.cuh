@@ -9,6 +9,19 @@
 
 namespace medusa {
 
+// Prefer the largest shared-memory carveout for a kernel: the heads and
+// tensor-core attention kernels need it, and when every kernel of a step asks
+// for the same split, an SM is never reconfigured between back-to-back
+// launches.
+template <typename Kernel>
+inline void prefer_max_smem(Kernel kernel) {
+    // a hint: if the driver refuses it, drop the error so the launch's own
+    // status check does not report it
+    if (cudaFuncSetAttribute(reinterpret_cast<const void*>(kernel), cudaFuncAttributePreferredSharedMemoryCarveout,
+                             100) != cudaSuccess)
+        (void)cudaGetLastError();
+}
+
 constexpr int kMaxTree = MEDUSA_MAX_TREE;  // nodes per tree
 constexpr int kTopK = MEDUSA_TOPK;         // entries kept per head
 constexpr unsigned kFull = 0xffffffffu;

@@ -556,6 +556,7 @@ cudaError_t launch_n(const TcHeadsArgs& args, cudaStream_t st) {
     auto kern = heads_tc_kernel<N>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
+    prefer_max_smem(kern);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(num_sms());
     cfg.blockDim = dim3(kTcWarps * 32);

@@ -522,6 +522,8 @@ cudaError_t verify_greedy_rows_launch(const VerifyArgs& a, cudaStream_t st) {
     float* pval = (float*)a.ws;
     int* pidx = (int*)((char*)a.ws + align256((size_t)rows * splits * sizeof(float)));
     dim3 grid(rows, splits);
+    if (a.target_dt == MEDUSA_BF16) prefer_max_smem(row_argmax_kernel<__nv_bfloat16>);
+    else prefer_max_smem(row_argmax_kernel<float>);
     if (a.target_dt == MEDUSA_BF16)
         row_argmax_kernel<__nv_bfloat16>
             <<<grid, kArgmaxThreads, 0, st>>>((const __nv_bfloat16*)a.target, a.V, splits, chunk, pval, pidx);
@@ -537,6 +539,7 @@ cudaError_t verify_greedy_walk_launch(const VerifyArgs& a, cudaStream_t st) {
     const int splits = argmax_splits(rows, a.V);
     const float* pval = (const float*)a.ws;
     const int* pidx = (const int*)((const char*)a.ws + align256((size_t)rows * splits * sizeof(float)));
+    prefer_max_smem(greedy_walk_kernel);
     greedy_walk_kernel<<<a.B, kWalkThreads, 0, st>>>(pval, pidx, splits, a.node_tokens, a.tree, a.accept_path,
                                                      a.max_path, a.accept_len, a.bonus);
     return cudaGetLastError();
@@ -564,6 +567,7 @@ cudaError_t verify_launch(const VerifyArgs& a, cudaStream_t st) {
     auto kernel = !a.logits ? verify_stochastic_kernel<0>
                   : a.target_dt == MEDUSA_BF16 ? verify_stochastic_kernel<2> : verify_stochastic_kernel<1>;
     const double inv_tau = a.logits ? a.inv_tau : 1.0;
+    prefer_max_smem(kernel);
     return cudaLaunchKernelEx(&cfg, kernel, a.target, inv_tau, a.q, a.q_rows, a.q_row, a.node_tokens, a.V, a.tree,
                               (uint32_t)a.seed, (uint32_t)(a.seed >> 32), a.step, a.accept_path, a.max_path,
                               a.accept_len, a.bonus, ws_w, a.status);
