@@ -41,43 +41,49 @@ def lib():
     global _lib
     if _lib is None:
         build()
-        L = ctypes.CDLL(_LIB)
-        vp, i32, i64, u32, u64, dbl = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_uint32,
-                                       ctypes.c_uint64, ctypes.c_double)
-        L.orc_tree_mask.argtypes = [vp, i32, vp]
-        L.orc_tree_shape.argtypes = [vp, i32, vp, vp]
-        L.orc_product_tree.argtypes = [vp, i32, vp, i32]
-        L.orc_heads.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, vp, vp]
-        L.orc_heads.restype = None
-        L.orc_topk.argtypes = [vp, i32, i32, vp]
-        L.orc_topk.restype = None
-        L.orc_tree_fill.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp, vp]
-        L.orc_tree_attention.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, dbl, vp,
-                                         i32, vp, vp, vp]
-        L.orc_verify_greedy.argtypes = [vp, i32, vp, i32, i32, i32, vp, i32, vp, vp, vp]
-        L.orc_philox4x32_10.argtypes = [vp, vp, vp]
-        L.orc_philox4x32_10.restype = None
-        L.orc_verify_stochastic.argtypes = [vp, vp, i32, vp, vp, i32, i32, i32, vp, u64, u32, i32, vp, vp, vp,
-                                            vp, i32]
-        L.orc_verify_stochastic_logits.argtypes = [vp, i32, dbl, vp, i32, vp, vp, i32, i32, i32, vp, u64, u32,
-                                                   i32, vp, vp, vp, vp, i32]
-        L.orc_softmax_temperature.argtypes = [vp, i32, dbl, vp]
-        L.orc_softmax_temperature.restype = None
-        L.orc_kv_compact.argtypes = [vp, vp, i32, vp, i32, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]
-        L.orc_kv_compact.restype = None
-        L.orc_kv_commit.argtypes = [vp, vp, vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]
-        L.orc_kv_commit.restype = None
-        L.orc_gather_pages.argtypes = [vp, vp, i32, i32, i32, vp, i32, i32, i32, i32, i32, vp]
-        L.orc_gather_pages.restype = i32
-        L.orc_kv_commit_paged.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, vp, i32, vp, vp, vp, i32, i32, i32, i32,
-                                          i32, vp]
-        L.orc_kv_commit_paged.restype = None
-        L.orc_residual.argtypes = [vp, vp, i32, vp, vp]
-        L.orc_residual.restype = u64
-        L.orc_round_bf16.argtypes = [dbl]
-        L.orc_round_bf16.restype = dbl
-        _lib = L
+        _lib = configure(ctypes.CDLL(_LIB))
     return _lib
+
+
+def configure(L):
+    """Declares the argument and result types of every oracle function on a
+    loaded copy of the library (the tests also load deliberately broken
+    builds of oracle.c through it)."""
+    vp, i32, i64, u32, u64, dbl = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_uint32,
+                                   ctypes.c_uint64, ctypes.c_double)
+    L.orc_tree_mask.argtypes = [vp, i32, vp]
+    L.orc_tree_shape.argtypes = [vp, i32, vp, vp]
+    L.orc_product_tree.argtypes = [vp, i32, vp, i32]
+    L.orc_heads.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, vp, vp]
+    L.orc_heads.restype = None
+    L.orc_topk.argtypes = [vp, i32, i32, vp]
+    L.orc_topk.restype = None
+    L.orc_tree_fill.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp, vp]
+    L.orc_tree_attention.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, dbl, vp,
+                                     i32, vp, vp, vp]
+    L.orc_verify_greedy.argtypes = [vp, i32, vp, i32, i32, i32, vp, i32, vp, vp, vp]
+    L.orc_philox4x32_10.argtypes = [vp, vp, vp]
+    L.orc_philox4x32_10.restype = None
+    L.orc_verify_stochastic.argtypes = [vp, vp, i32, vp, vp, i32, i32, i32, vp, u64, u32, i32, vp, vp, vp,
+                                        vp, i32]
+    L.orc_verify_stochastic_logits.argtypes = [vp, i32, dbl, vp, i32, vp, vp, i32, i32, i32, vp, u64, u32,
+                                               i32, vp, vp, vp, vp, i32]
+    L.orc_softmax_temperature.argtypes = [vp, i32, dbl, vp]
+    L.orc_softmax_temperature.restype = None
+    L.orc_kv_compact.argtypes = [vp, vp, i32, vp, i32, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]
+    L.orc_kv_compact.restype = None
+    L.orc_kv_commit.argtypes = [vp, vp, vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]
+    L.orc_kv_commit.restype = None
+    L.orc_gather_pages.argtypes = [vp, vp, i32, i32, i32, vp, i32, i32, i32, i32, i32, vp]
+    L.orc_gather_pages.restype = i32
+    L.orc_kv_commit_paged.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, vp, i32, vp, vp, vp, i32, i32, i32, i32,
+                                      i32, vp]
+    L.orc_kv_commit_paged.restype = None
+    L.orc_residual.argtypes = [vp, vp, i32, vp, vp]
+    L.orc_residual.restype = u64
+    L.orc_round_bf16.argtypes = [dbl]
+    L.orc_round_bf16.restype = dbl
+    return L
 
 
 # ----------------------------------------------------------------------------
