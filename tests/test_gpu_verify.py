@@ -262,3 +262,22 @@ def test_greedy_rows_then_walk_on_two_streams_is_tree_verify():
     assert torch.equal(bonus, ref["bonus"])
     assert_same({"accept_path": path, "accept_len": ln, "bonus": bonus},
                 oracle.verify_greedy(logits, tok, parents, tree.max_depth))
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_greedy_equally_deep_accepted_nodes(dtype):
+    # sibling tokens drawn from a 4-token vocabulary repeat often, so several
+    # equally deep nodes are accepted: the path must end at the lowest index
+    rng = np.random.default_rng(23)
+    parents = I.product_tree_parents((3, 2, 2))
+    T, V, nb = len(parents), 4, 64
+    ch = I.tree_children(parents)
+    tok = rng.integers(0, V, (nb, T)).astype(np.int32)
+    logits = rng.standard_normal((nb, T, V)).astype(np.float32)
+    for b in range(nb):
+        for u in range(T):
+            if ch[u] and rng.random() < 0.8:
+                logits[b, u, tok[b, ch[u][rng.integers(len(ch[u]))]]] = 10.0
+    lg = torch.from_numpy(logits).to(dtype)
+    out = run_greedy(parents, torch.from_numpy(tok), lg)
+    assert_same(out, oracle.verify_greedy(lg, tok, parents, max_path=4))

@@ -437,6 +437,52 @@ def test_greedy_vs_brute_force(orc):
         assert (path[0, ln[0]:] == -1).all()
 
 
+def test_greedy_equally_deep_nodes_take_the_lowest_index(orc):
+    # two siblings carry the same (matching) token, and so do their children:
+    # nodes 3 and 4 are both accepted at depth 3; the path ends at node 3
+    par = [-1, 0, 0, 1, 2]
+    V = 10
+    logits = torch.zeros((1, 5, V))
+    logits[0, 0, 7] = 5.0          # prediction after the root: 7
+    logits[0, 1, 4] = 5.0          # after node 1: 4
+    logits[0, 2, 4] = 5.0          # after node 2: 4
+    logits[0, 3, 1] = 5.0          # after node 3: 1 (the bonus)
+    logits[0, 4, 2] = 5.0          # after node 4: 2
+    tok = [[0, 7, 7, 4, 4]]
+    path, ln, bonus = orc.verify_greedy(logits, tok, par, max_path=3)
+    assert ln[0] == 3 and path[0].tolist() == [0, 1, 3] and bonus[0] == 1
+    # with duplicated sibling tokens drawn at random, the brute force over
+    # paths (first longest in leaf order = lowest index in breadth-first
+    # order) still agrees
+    rng = np.random.default_rng(17)
+    par = orc.product_tree((3, 2, 2))
+    T, V = len(par), 4
+    children = I.tree_children(par.tolist())
+    ties = 0
+    for trial in range(300):
+        logits = rng.standard_normal((1, T, V)).astype(np.float32)
+        tok = rng.integers(0, V, (1, T)).astype(np.int32)     # few tokens: siblings often repeat
+        for u in range(T):
+            if children[u] and rng.random() < 0.8:
+                logits[0, u, tok[0, children[u][rng.integers(len(children[u]))]]] = 10.0
+        path, ln, bonus = orc.verify_greedy(torch.from_numpy(logits), tok, par, max_path=4)
+        want, wb = _brute_force_greedy(logits[0], tok[0], par.tolist())
+        assert path[0, : ln[0]].tolist() == want and bonus[0] == wb
+        pred = logits[0].argmax(-1)
+        deep = [c for c in range(T) if len(_ancestors(par.tolist(), c)) == ln[0] and
+                all(tok[0, a] == pred[par[a]] for a in _ancestors(par.tolist(), c)[1:])]
+        ties += len(deep) > 1
+    assert ties > 20                  # the tie rule was exercised
+
+
+def _ancestors(par, c):
+    out = []
+    while c != -1:
+        out.append(c)
+        c = par[c]
+    return out[::-1]
+
+
 def test_greedy_draft_equals_target(orc):
     # every node's first child carries the target's prediction at its parent:
     # the whole first-child chain is accepted, bonus = prediction at its end

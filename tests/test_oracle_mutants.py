@@ -42,6 +42,18 @@ MUTANTS = [
      "blk + (size_t)(path[(size_t)b * max_path + t]) * row", [pins.test_kv_compact_hand_example]),
     ("page slot from the page number", "+ s % page_size) * D * esize;", "+ s / page_size) * D * esize;",
      [pins.test_gather_pages_identity_table_is_a_reshape]),
+    ("tree fill ignores the sibling rank", "size_t e = ((size_t)b * K + (depth[i] - 2)) * S + rank[i];",
+     "size_t e = ((size_t)b * K + (depth[i] - 2)) * S + 0;", [pins.test_tree_fill_product_tree]),
+    ("kv-head of a q-head taken modulo", "int g = h / G;", "int g = h % Hkv;",
+     [pins.test_attention_product_tree_vs_sdpa_with_path_mask]),
+    ("deepest accepted node: highest index on ties", "if (acc[c] && depth[c] > depth[best]) best = c;",
+     "if (acc[c] && depth[c] >= depth[best]) best = c;",
+     [pins.test_greedy_equally_deep_nodes_take_the_lowest_index]),
+    ("acceptance without the parent's", "acc[c] = acc[parent[c]] && node_tokens[(size_t)b * T + c] == pred[parent[c]];",
+     "acc[c] = node_tokens[(size_t)b * T + c] == pred[parent[c]];", [pins.test_greedy_vs_brute_force]),
+    ("commit one row late", "size_t dst = ((((size_t)b * Hkv + g) * S_max) + S + t) * D * esize;",
+     "size_t dst = ((((size_t)b * Hkv + g) * S_max) + S + t + 1) * D * esize;",
+     [pins.test_kv_commit_exact_and_canaries]),
 ]
 
 
