@@ -51,6 +51,11 @@ MUTANTS = [
      [pins.test_greedy_equally_deep_nodes_take_the_lowest_index]),
     ("acceptance without the parent's", "acc[c] = acc[parent[c]] && node_tokens[(size_t)b * T + c] == pred[parent[c]];",
      "acc[c] = node_tokens[(size_t)b * T + c] == pred[parent[c]];", [pins.test_greedy_vs_brute_force]),
+    ("children tried in reverse order", "for (int c = u + 1; c < T; ++c) {", "for (int c = T - 1; c > u; --c) {",
+     [pins.test_stochastic_draft_equals_target_accepts_all]),
+    ("the accepted child keeps its parent's target row",
+     "++L;\n                    load_row(src, (size_t)b * T + u, V, P);", "++L;",
+     [lambda o: pins.test_stochastic_first_token_follows_target(o, 1)]),
     ("commit one row late", "size_t dst = ((((size_t)b * Hkv + g) * S_max) + S + t) * D * esize;",
      "size_t dst = ((((size_t)b * Hkv + g) * S_max) + S + t + 1) * D * esize;",
      [pins.test_kv_commit_exact_and_canaries]),
