@@ -56,6 +56,18 @@ MUTANTS = [
     ("the accepted child keeps its parent's target row",
      "++L;\n                    load_row(src, (size_t)b * T + u, V, P);", "++L;",
      [lambda o: pins.test_stochastic_first_token_follows_target(o, 1)]),
+    ("attention's V from the tree row of the wrong kv-head",
+     "size_t voff = (((size_t)b * T + j) * Hkv + g) * D;", "size_t voff = (((size_t)b * T + j) * Hkv + 0) * D;",
+     [pins.test_attention_product_tree_vs_sdpa_with_path_mask]),
+    ("attention reads one prefix key too many",
+     "        int n = 0;\n        for (int j = 0; j < S; ++j) {", "        int n = 0;\n        for (int j = 0; j <= S; ++j) {",
+     [pins.test_attention_chain_tree_is_causal_attention, pins.test_attention_single_node_is_decode_attention]),
+    ("compaction accepts a repeated node", "if (n <= prev || n >= T) ok = 0;", "if (n < prev || n >= T) ok = 0;",
+     [pins.test_kv_compact_refusals]),
+    ("paged commit writes every row into the prefix's last page",
+     "int page = table[(size_t)b * max_pages + (S + t) / page_size];",
+     "int page = table[(size_t)b * max_pages + S / page_size];",
+     [pins.test_paged_commit_equals_contiguous_commit_through_the_table]),
     ("commit one row late", "size_t dst = ((((size_t)b * Hkv + g) * S_max) + S + t) * D * esize;",
      "size_t dst = ((((size_t)b * Hkv + g) * S_max) + S + t + 1) * D * esize;",
      [pins.test_kv_commit_exact_and_canaries]),
