@@ -174,3 +174,16 @@ def test_newer_calls_validate_before_launch(lib):
     assert lib.tree_verify_greedy_walk(nul, 1, 100, nul, fake, 4, fake, fake, fake, 1 << 20, nul) == INV
     assert lib.tree_verify_greedy_walk(fake, 1, 100, nul, fake, 4, fake, fake, fake, 1 << 20, nul) == INV
     assert lib.tree_attention_incache_workspace_size(1, 4, 2, 96, 256, 0, nul, 1) == 0
+
+
+def test_header_is_plain_c(tmp_path):
+    # the boundary is a C ABI: the header compiles as C11 and as C++17 with
+    # every warning on, and needs no CUDA or torch header
+    inc = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+    src = tmp_path / "use.c"
+    src.write_text('#include "medusa.h"\nint f(void) { return MEDUSA_TOPK + (int)sizeof(medusa_head_partial); }\n')
+    import subprocess
+    subprocess.check_call(["gcc", "-std=c11", "-Wall", "-Wextra", "-Werror", "-fsyntax-only", "-I", inc, str(src)])
+    cpp = tmp_path / "use.cpp"
+    cpp.write_text(src.read_text())
+    subprocess.check_call(["g++", "-std=c++17", "-Wall", "-Wextra", "-Werror", "-fsyntax-only", "-I", inc, str(cpp)])
