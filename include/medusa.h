@@ -2,7 +2,9 @@
  * medusa.h -- C ABI of libmedusa.so: one Medusa speculative decode step on an
  * NVIDIA B200 (sm_100a).
  *
- * The step has four calls, run in this order on one CUDA stream:
+ * The step has four calls (tree_attention reads none of medusa_heads'
+ * outputs, so the two may run concurrently on two streams; tree_verify needs
+ * the node tokens and the target's output; kv_commit needs tree_verify's):
  *   medusa_heads    Medusa heads, top-s per head, candidate-tree tokens
  *                   (medusa_heads_shard / medusa_heads_merge: the same over
  *                   vocabulary shards, one per GPU)
@@ -11,7 +13,9 @@
  *   tree_verify     greedy or stochastic verification: longest accepted
  *                   root-to-node path plus one bonus token
  *                   (tree_verify_logits: the stochastic walk reading the
- *                   target's logits at a temperature)
+ *                   target's logits at a temperature; tree_verify_greedy_rows
+ *                   and tree_verify_greedy_walk: greedy verification's two
+ *                   launches on their own)
  *   kv_commit       append the accepted path's K/V to the cache
  * tree_attention_incache and kv_compact are the pair for a cache that already
  * holds the tree's K/V after each prefix (compaction of every layer at once).
