@@ -20,3 +20,34 @@ def test_reference_arm_prints_one_json_line_with_the_contract_keys():
     assert d["config"]["workload"].startswith("tiny:")
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def _bench():
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("bench_module", os.path.join(ROOT, "bench.py"))
+    m = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(m)
+    return m
+
+
+def test_bench_defaults_and_config_keys():
+    b = _bench()
+    from medusa_tree_speculative_heads_b200 import inputs as I
+    assert b.METRIC.startswith("Medusa verify steps/s") and b.UNIT == "steps/s"
+    assert b.WORKLOAD == "llama8b"
+    for name, w in I.WORKLOADS.items():
+        c = b.config_dict(w, 1)
+        assert {"workload", "global_batch", "seq_len", "parallelism", "l2"} <= set(c)
+        assert c["workload"].startswith(name + ":") and c["global_batch"] == w.B
+        assert b.config_dict(w, 4)["global_batch"] == 4 * w.B          # replicas: weak scaling
+
+
+def test_bench_counts_the_library_launches_of_a_step():
+    # the kernels one step launches (the launch list in profiles/ shows six at llama8b)
+    b = _bench()
+    from medusa_tree_speculative_heads_b200 import inputs as I
+    W = I.WORKLOADS
+    assert b.launches_per_step(W["llama8b"]) == 6       # heads, attention + combine, argmax + walk, commit
+    assert b.launches_per_step(W["stoch_b64"]) == 5     # one stochastic verify kernel
+    assert b.launches_per_step(W["tiny"]) == 1 + 1 + 2 + 1   # fp32: fused heads, one attention kernel
+    assert b._is_anc([-1, 0, 1, 0], 2, 0) and b._is_anc([-1, 0, 1, 0], 2, 2) and not b._is_anc([-1, 0, 1, 0], 3, 1)
