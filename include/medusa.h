@@ -197,9 +197,11 @@ int medusa_heads(const void* h, const void* W_res, const void* W_head, int B, in
  *     GPU that loads the library holds it until the process exits.  Sizes
  *     whose medusa_heads_workspace_size exceeds 32 MiB are rejected with
  *     MEDUSA_ERR_UNSUPPORTED and a message; nothing is launched.
- *   - The first call on each device looks up the array's device address (with
- *     that device current) and caches it; make that first call before any
- *     stream capture begins.
+ *   - Every call looks up the array's device address on the current device
+ *     (a host-side lookup, repeated per call so that a reset and re-created
+ *     context never leaves a stale address behind).  The first call on a
+ *     device may also load the library's device code there; make that first
+ *     call before any stream capture begins.
  *   - The call itself allocates nothing (no cudaMalloc/cudaFree).
  *   - Every call on a device shares the one array: calls whose work overlaps
  *     on the GPU (different streams, or different host threads) race and

@@ -342,8 +342,14 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
                 tc_commit(&v_empty[s]);
                 if (j == nc - 1) tc_commit(o_last);
             }
-            if (!ok) set_status(a.status, MEDUSA_STATUS_TIMEOUT);
-            else mbar_wait(o_last, 0);  // every MMA done before TMEM is released
+            if (!ok) {
+                // o_last was not committed (the loop left before the last
+                // chunk): commit it now, so that it completes once every MMA
+                // this thread did issue has finished writing TMEM
+                set_status(a.status, MEDUSA_STATUS_TIMEOUT);
+                tc_commit(o_last);
+            }
+            mbar_wait(o_last, 0);  // every MMA done before TMEM is released (bounded)
         }
     } else {
         // ---------------- softmax / output ----------------

@@ -10,8 +10,6 @@
 // forwards to medusa_heads with that array as the workspace.
 #include <stdio.h>
 
-#include <mutex>
-
 #include "kernels.h"
 
 namespace medusa {
@@ -28,25 +26,21 @@ constexpr size_t kNoAllocScratchBytes = (size_t)32 << 20;
 // cudaGetSymbolAddress below.
 static __device__ __align__(256) uint8_t g_heads_scratch[kNoAllocScratchBytes];
 
-std::mutex g_mu;
-void* g_ptr[64] = {};
-
-// Device address of g_heads_scratch on the current device, looked up once per
-// device (with that device current) and cached.
+// Device address of g_heads_scratch on the current device, with that device
+// current.  Looked up on every call (a host-side table lookup once the
+// library's module is loaded), never cached: a primary context that was reset
+// and re-created reloads the module, and an address kept from before would
+// then point at memory the new context does not own.
 int scratch_address(void** out) {
-    int dev = -1;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return medusa::report_error(MEDUSA_ERR_CUDA, cudaGetErrorString(e));
-    if (dev < 0 || dev >= 64) return medusa::report_error(MEDUSA_ERR_UNSUPPORTED, "medusa_heads_noalloc: device index >= 64");
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_ptr[dev]) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_heads_scratch);
-        if (e != cudaSuccess || !p)
-            return medusa::report_error(MEDUSA_ERR_CUDA, "medusa_heads_noalloc: cudaGetSymbolAddress of the scratch failed");
-        g_ptr[dev] = p;
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_heads_scratch);
+    if (e != cudaSuccess || !p) {
+        char msg[256];
+        snprintf(msg, sizeof msg, "medusa_heads_noalloc: cudaGetSymbolAddress of the scratch failed (%s)",
+                 cudaGetErrorString(e));
+        return medusa::report_error(MEDUSA_ERR_CUDA, msg);
     }
-    *out = g_ptr[dev];
+    *out = p;
     return MEDUSA_OK;
 }
 

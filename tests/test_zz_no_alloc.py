@@ -15,7 +15,6 @@ failure has run every other test before it.
 import pytest
 import torch
 
-from helpers import float_tol
 from medusa_tree_speculative_heads_b200 import binding as B
 from medusa_tree_speculative_heads_b200 import inputs as I
 from medusa_tree_speculative_heads_b200.binding import MedusaError, Tree
@@ -49,13 +48,12 @@ def _call(fn_noalloc, w, inp, tree, o):
         B.medusa_heads(*args, ws, nb, o["status"])
 
 
-def _same(a, b, dtype):
-    tol = float_tol(dtype)
-    for k in ("topk_idx", "node_tokens", "status"):
+def _same(a, b):
+    # the same kernels on the same inputs with the same workspace layout: every
+    # output must be bit-identical (a value perturbed by stale scratch would
+    # still pass a float tolerance)
+    for k in ("topk_idx", "topk_prob", "node_tokens", "node_q", "logits", "probs", "h_res", "status"):
         assert torch.equal(a[k], b[k]), k
-    for k in ("topk_prob", "node_q", "logits", "probs"):
-        assert (a[k] - b[k]).abs().max().item() <= tol, k
-    assert (a["h_res"].float() - b["h_res"].float()).abs().max().item() <= tol
 
 
 @pytest.mark.parametrize("name,kw,tree", [
@@ -74,7 +72,7 @@ def test_noalloc_matches_workspace_entry_point_twice(name, kw, tree):
         _call(True, w, inp, t, mine)
         _call(False, w, inp, t, ref)
         torch.cuda.synchronize()
-        _same(mine, ref, w.torch_dtype)
+        _same(mine, ref)
         assert int(mine["status"].item()) == 0
 
 
