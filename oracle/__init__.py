@@ -23,26 +23,50 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
+_LIB_OMP = os.path.join(_HERE, "liboracle_omp.so")   # the same source built with OpenMP
 _lib = None
+_lib_omp = None
+_use_omp = False
+_CFLAGS = ["-O2", "-std=gnu11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared"]
 
 F32, BF16 = 0, 1
 
 
 def build(force: bool = False) -> str:
-    """Compile oracle.c into liboracle.so with gcc (no FMA contraction)."""
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
-        subprocess.check_call(["gcc", "-O2", "-std=gnu11", "-ffp-contract=off", "-fno-fast-math", "-fPIC",
-                               "-shared", "-o", _LIB + ".tmp", _SRC, "-lm"])
-        os.replace(_LIB + ".tmp", _LIB)
+    """Compile oracle.c with gcc (no FMA contraction) into liboracle.so, and
+    the same source with OpenMP into liboracle_omp.so.  The OpenMP build only
+    shares independent output elements (rows, vocabulary entries) among
+    threads; each element's arithmetic is the serial build's, so the two give
+    bit-identical results."""
+    for out, extra in ((_LIB, []), (_LIB_OMP, ["-fopenmp"])):
+        if force or not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(_SRC):
+            subprocess.check_call(["gcc"] + _CFLAGS + extra + ["-o", out + ".tmp", _SRC, "-lm"])
+            os.replace(out + ".tmp", out)
     return _LIB
 
 
 def lib():
-    global _lib
+    global _lib, _lib_omp
+    if _use_omp:
+        if _lib_omp is None:
+            build()
+            _lib_omp = configure(ctypes.CDLL(_LIB_OMP))
+        return _lib_omp
     if _lib is None:
         build()
         _lib = configure(ctypes.CDLL(_LIB))
     return _lib
+
+
+def use_openmp(on: bool = True) -> None:
+    """Route later calls to the OpenMP build (on) or the serial one (off)."""
+    global _use_omp
+    _use_omp = bool(on)
+
+
+def threads() -> int:
+    """Threads the build currently in use runs its parallel loops on."""
+    return int(lib().orc_threads())
 
 
 def configure(L):
@@ -54,7 +78,9 @@ def configure(L):
     L.orc_tree_mask.argtypes = [vp, i32, vp]
     L.orc_tree_shape.argtypes = [vp, i32, vp, vp]
     L.orc_product_tree.argtypes = [vp, i32, vp, i32]
-    L.orc_heads.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, vp, vp]
+    L.orc_heads.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, vp, vp, vp]
+    L.orc_threads.argtypes = []
+    L.orc_threads.restype = i32
     L.orc_heads.restype = None
     L.orc_topk.argtypes = [vp, i32, i32, vp]
     L.orc_topk.restype = None
@@ -157,9 +183,12 @@ def product_tree(branching: Sequence[int], cap: int = 4096) -> np.ndarray:
 # heads
 # ----------------------------------------------------------------------------
 
-def heads(h, W_res, W_head, b_only: int = -1, k_only: int = -1, want_hk=True, want_probs=True):
+def heads(h, W_res, W_head, b_only: int = -1, k_only: int = -1, want_hk=True, want_probs=True,
+          exact_hk: bool = False):
     """Returns dict of fp64 arrays hk [B,K,d], logits [B,K,V], probs [B,K,V]
-    (rows not selected by b_only/k_only are NaN)."""
+    (rows not selected by b_only/k_only are NaN).  For bf16 inputs h^(k) is
+    rounded to bf16 before the vocabulary projection, unless exact_hk keeps
+    its exact fp64 value."""
     hr, dt = _raw(h)
     wr, dt2 = _raw(W_res)
     wh, dt3 = _raw(W_head)
@@ -169,7 +198,8 @@ def heads(h, W_res, W_head, b_only: int = -1, k_only: int = -1, want_hk=True, wa
     hk = np.full((B, K, d), np.nan) if want_hk else None
     logits = np.full((B, K, V), np.nan)
     probs = np.full((B, K, V), np.nan) if want_probs else None
-    lib().orc_heads(_p(hr), _p(wr), _p(wh), dt, B, d, V, K, b_only, k_only, _p(hk), _p(logits), _p(probs))
+    lib().orc_heads(_p(hr), _p(wr), _p(wh), dt, B, d, V, K, b_only, k_only, 0 if exact_hk else 1, _p(hk), _p(logits),
+                    _p(probs))
     return {"hk": hk, "logits": logits, "probs": probs}
 
 

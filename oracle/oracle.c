@@ -124,6 +124,14 @@ double orc_round_bf16(double x) {
     return r;
 }
 
+/* Threads an OpenMP build uses for its parallel loops (1 in the serial build). */
+#ifdef _OPENMP
+#include <omp.h>
+int orc_threads(void) { return omp_get_max_threads(); }
+#else
+int orc_threads(void) { return 1; }
+#endif
+
 /* ------------------------------------------------------------------------ */
 /* Medusa heads                                                              */
 /* ------------------------------------------------------------------------ */
@@ -136,13 +144,17 @@ double orc_round_bf16(double x) {
  * activation of the model's dtype, so for bf16 inputs it is stored rounded
  * to bf16 (from the exact fp64 value) before the vocabulary projection; the
  * top-s decision is then taken on the same operand precision as a bf16
- * kernel's.  Layouts: h [B,d]; W_res [K,d,d] (output row, input
- * column); W_head [K,V,d].  Outputs (each nullable): hk [B,K,d],
- * logits [B,K,V], probs [B,K,V].  Only sequence b_only / head k_only is
- * computed when those are >= 0 (others untouched).
+ * kernel's.  round_hk = 0 keeps h^(k) at its exact fp64 value instead (the
+ * formula read with no intermediate precision at all), so the distance
+ * between the two readings can be measured.  Layouts: h [B,d]; W_res
+ * [K,d,d] (output row, input column); W_head [K,V,d].  Outputs (each
+ * nullable): hk [B,K,d], logits [B,K,V], probs [B,K,V].  Only sequence
+ * b_only / head k_only is computed when those are >= 0 (others untouched).
+ * The element loops are independent; an OpenMP build shares them among
+ * threads with every element computed exactly as in the serial build.
  */
 void orc_heads(const void* h, const void* W_res, const void* W_head, int dtype,
-               int B, int d, int V, int K, int b_only, int k_only,
+               int B, int d, int V, int K, int b_only, int k_only, int round_hk,
                double* hk_out, double* logits_out, double* probs_out) {
     double* hk = (double*)malloc(sizeof(double) * (size_t)d);
     double* logit = (double*)malloc(sizeof(double) * (size_t)V);
@@ -151,15 +163,17 @@ void orc_heads(const void* h, const void* W_res, const void* W_head, int dtype,
         for (int k = 0; k < K; ++k) {
             if (k_only >= 0 && k != k_only) continue;
             /* residual block */
+#pragma omp parallel for schedule(static)
             for (int o = 0; o < d; ++o) {
                 double z = 0.0;
                 for (int i = 0; i < d; ++i)
                     z += load(W_res, dtype, ((size_t)k * d + o) * d + i) * load(h, dtype, (size_t)b * d + i);
                 double sig = 1.0 / (1.0 + exp(-z));
                 hk[o] = z * sig + load(h, dtype, (size_t)b * d + o);
-                if (dtype == ORC_BF16) hk[o] = orc_round_bf16(hk[o]);
+                if (dtype == ORC_BF16 && round_hk) hk[o] = orc_round_bf16(hk[o]);
             }
             /* projection to the vocabulary */
+#pragma omp parallel for schedule(static)
             for (int v = 0; v < V; ++v) {
                 double acc = 0.0;
                 for (int i = 0; i < d; ++i)
@@ -273,8 +287,23 @@ int orc_tree_attention(const void* q, const void* k_tree, const void* v_tree, co
     int G = Hq / Hkv;
     int total = rows ? nrows : B * T * Hq;
     int maxkeys = S_max + T;
-    double* s = (double*)malloc(sizeof(double) * (size_t)maxkeys);
     int rc = 0;
+    for (int r = 0; rows && r < total; ++r) {
+        int b = rows[3 * r], i = rows[3 * r + 1], h = rows[3 * r + 2];
+        if (b < 0 || b >= B || i < 0 || i >= T || h < 0 || h >= Hq) rc = -1;
+    }
+    for (int b = 0; b < B; ++b)
+        if (prefix_len[b] < 0 || prefix_len[b] > S_max) rc = -1;
+    if (rc != 0) {
+        free(anc);
+        return rc;
+    }
+    /* rows are independent: an OpenMP build shares them among threads, each
+     * with its own score buffer and the same per-row arithmetic */
+#pragma omp parallel
+    {
+    double* s = (double*)malloc(sizeof(double) * (size_t)maxkeys);
+#pragma omp for schedule(dynamic, 8)
     for (int r = 0; r < total; ++r) {
         int b, i, h;
         if (rows) {
@@ -285,11 +314,6 @@ int orc_tree_attention(const void* q, const void* k_tree, const void* v_tree, co
             b = r / (T * Hq);
             i = (r / Hq) % T;
             h = r % Hq;
-        }
-        if (b < 0 || b >= B || i < 0 || i >= T || h < 0 || h >= Hq || prefix_len[b] < 0 ||
-            prefix_len[b] > S_max) {
-            rc = -1;
-            break;
         }
         int g = h / G;
         int S = prefix_len[b];
@@ -331,6 +355,7 @@ int orc_tree_attention(const void* q, const void* k_tree, const void* v_tree, co
         if (lse) lse[r] = m + log(sum);
     }
     free(s);
+    }
     free(anc);
     return rc;
 }
@@ -375,6 +400,7 @@ int orc_verify_greedy(const void* logits, int dtype, const int32_t* node_tokens,
     uint8_t* acc = (uint8_t*)malloc((size_t)T);
     int rc = orc_tree_shape(parent, T, depth, rank);
     for (int b = 0; rc == 0 && b < B; ++b) {
+#pragma omp parallel for schedule(static)
         for (int u = 0; u < T; ++u) pred[u] = row_argmax(logits, dtype, ((size_t)b * T + u) * V, V);
         acc[0] = 1;
         for (int c = 1; c < T; ++c)

@@ -169,6 +169,53 @@ def test_heads_hand_d4_case_b_silu_ln3(orc):
     np.testing.assert_allclose(r["logits"][0, 0], _floats(g["B_logits"]), rtol=0, atol=1e-7)
 
 
+def test_heads_hand_d4_case_c_bf16_activation(orc):
+    # bf16 inputs: h^(k) = SiLU(1) + 1 is stored as the nearest bf16 value
+    # before the vocabulary projection; with exact_hk it stays exact
+    g = read_golden("guide_head_d4.txt")
+    h = torch.tensor([_floats(g["h"])], dtype=torch.float32).bfloat16()
+    W_res = torch.zeros((1, 4, 4), dtype=torch.bfloat16)
+    W_res[0, 0, 0] = 1.0
+    W_head = torch.tensor([_mat(g["W_head"])], dtype=torch.float32).bfloat16()
+    r = orc.heads(h, W_res, W_head)
+    np.testing.assert_array_equal(r["hk"][0, 0], _floats(g["C_hk_bf16"]))
+    np.testing.assert_array_equal(r["logits"][0, 0], _floats(g["C_logits_bf16"]))
+    e = orc.heads(h, W_res, W_head, exact_hk=True)
+    np.testing.assert_allclose(e["hk"][0, 0], _floats(g["C_hk_exact"]), rtol=0, atol=1e-15)
+    np.testing.assert_allclose(e["logits"][0, 0], _floats(g["C_logits_exact"]), rtol=0, atol=1e-15)
+
+
+def test_openmp_build_is_bit_identical_to_serial(orc):
+    # the OpenMP build only spreads independent output elements over threads:
+    # heads, attention and greedy verification give the serial build's bits
+    g = torch.Generator().manual_seed(21)
+    B, d, V, K = 2, 64, 300, 3
+    h = torch.randn((B, d), generator=g).bfloat16()
+    W_res = (torch.randn((K, d, d), generator=g) / 8).bfloat16()
+    W_head = (torch.randn((K, V, d), generator=g) / 8).bfloat16()
+    par = [-1, 0, 0, 1, 1, 2]
+    T, Hq, Hkv, D, S_max = len(par), 4, 2, 64, 40
+    q = torch.randn((B, T, Hq, D), generator=g).bfloat16()
+    kt, vt = (torch.randn((B, T, Hkv, D), generator=g).bfloat16() for _ in range(2))
+    kc, vc = (torch.randn((B, Hkv, S_max, D), generator=g).bfloat16() for _ in range(2))
+    pl = torch.tensor([33, 7], dtype=torch.int32)
+    logits = torch.randn((B, T, V), generator=g)
+    tok = torch.randint(0, V, (B, T), generator=g, dtype=torch.int32)
+    res = []
+    for on in (False, True):
+        orc.use_openmp(on)
+        try:
+            hr = orc.heads(h, W_res, W_head)
+            o, l = orc.tree_attention(q, kt, vt, kc, vc, pl, par)
+            path, ln, bonus = orc.verify_greedy(logits, tok, par, 4)
+            res.append((hr["hk"], hr["logits"], hr["probs"], o, l, path, ln, bonus, orc.threads()))
+        finally:
+            orc.use_openmp(False)
+    for a, b in zip(res[0][:-1], res[1][:-1]):
+        np.testing.assert_array_equal(a, b)
+    assert res[0][-1] == 1 and res[1][-1] >= 1
+
+
 def test_heads_silu_limits(orc):
     # SiLU(z) -> z for z >> 0 and -> 0 for z << 0
     h = torch.tensor([[1.0, 0.0]], dtype=torch.float32)

@@ -29,6 +29,9 @@ MUTANTS = [
      [pins.test_greedy_argmax_ties_lowest_index]),
     ("top-k ties to the highest index", "if (best < 0 || x[i] > x[best]) best = i;",
      "if (best < 0 || x[i] >= x[best]) best = i;", [pins.test_topk_equals_stable_sort]),
+    ("h^(k) not rounded to bf16 for bf16 inputs", "if (dtype == ORC_BF16 && round_hk) hk[o] = orc_round_bf16(hk[o]);",
+     "if (0) hk[o] = orc_round_bf16(hk[o]);",
+     [pins.test_heads_hand_d4_case_c_bf16_activation, pins.test_heads_bf16_stores_hk_as_bf16]),
     ("residual with the sign flipped", "double diff = P[y] - (double)Q[y];", "double diff = (double)Q[y] - P[y];",
      [pins.test_residual_normalises_and_closed_form]),
     ("acceptance test inverted", "if (uc * (double)Q[x] < P[x]) {", "if (uc * (double)Q[x] > P[x]) {",
