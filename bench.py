@@ -221,30 +221,54 @@ class OracleSample:
         return (t1 - t0) + (t3 - t2), self.frac
 
 
+def time_oracle(w, fraction: float, budget_s: float, min_steps: float, omp: bool):
+    """Time the oracle (serial or OpenMP build) on whole steps of workload w
+    (fraction 1) or a sampled slice; returns (steps/s, seconds, steps' worth
+    of work, threads used)."""
+    import oracle
+    oracle.build()
+    oracle.use_openmp(omp)
+    try:
+        sample = OracleSample(w, fraction)
+        tt, ff = 0.0, 0.0
+        while tt < budget_s and ff < min_steps:
+            t1, f1 = sample.run()
+            tt += t1
+            ff += f1
+        return ff / tt, tt, ff, oracle.threads()
+    finally:
+        oracle.use_openmp(False)
+
+
 def run_reference(args, rank, world):
+    """The reference arm: the fp64 oracle (its OpenMP build, every host core)
+    runs whole steps of the same workload -- W untimed, then K timed -- and
+    the line reports what was timed: K whole steps."""
     from medusa_tree_speculative_heads_b200 import inputs as I
     if rank != 0:
         return
     w = I.WORKLOADS[args.workload]
     import oracle
     oracle.build()
-    sample = OracleSample(w, 1.0 / 64, seed=1)
+    oracle.use_openmp(True)
+    sample = OracleSample(w, 1.0, seed=1)
     for _ in range(args.warmup):
         sample.run()
-    tot_t, tot_f = 0.0, 0.0
+    tot_t = 0.0
     for _ in range(args.steps):
         t, f = sample.run()
+        assert f == 1.0
         tot_t += t
-        tot_f += f
-    value = tot_f / tot_t
-    sample = (f"per step: fp64 oracle on the host, residual block of all {w.K} heads, LM-head rows of a 1/64 "
-              f"vocabulary slice, attention of 1/64 of the query rows, full verify and commit; "
-              f"steps/s scaled by the sampled fraction of the step's work")
+    cores = oracle.threads()
+    oracle.use_openmp(False)
+    value = args.steps / tot_t
+    desc = (f"{args.steps} whole steps of the workload (after {args.warmup} untimed), timed one by one: the fp64 "
+            f"oracle's OpenMP build on {cores} host threads; the target logits are inputs, drawn outside the timing")
     out = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
-           "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 / value, "higher_is_better": True,
-           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * tot_t / args.steps,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
            "config": config_dict(w, world),
-           "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+           "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
 
@@ -296,19 +320,198 @@ def config_dict(w, world):
             "l2": f"inputs larger than L2: each step streams {head_gb:.2f} GB of head weights through the 126 MB L2"}
 
 
-def launches_per_step(w, mode_greedy=True):
-    """Library kernels per step: medusa_heads is one cooperative kernel on the
-    bf16 tensor-core path (B <= 64); otherwise residual + per-8-sequence LM
-    and merge kernels."""
+def launches_per_step(w):
+    """Library kernels per step as MedusaStep.run issues it.  medusa_heads is
+    one cooperative kernel on the bf16 tensor-core path (B <= 64), else
+    residual + per-8-sequence LM and merge kernels; tree attention is one
+    kernel (the tensor-core kernel merges its key splits in-cluster; the
+    mma.sync path adds a combine kernel); greedy verification is the row scan
+    plus the walk, which also commits unless the commit is the all-layer
+    compaction; stochastic verification is one kernel, then the commit."""
     if w.dtype == "bf16" and w.B <= 64 and w.d % 8 == 0:
         heads = 1
     elif w.B == 1:
         heads = 1
     else:
         heads = 1 + 2 * ((w.B + 7) // 8)
-    attn = 2 if w.dtype == "bf16" else 1
-    verify = 1 if w.stochastic else 2
-    return heads + attn + verify + 1
+    G = w.Hq // w.Hkv
+    tc = w.dtype == "bf16" and w.D in (64, 128) and G <= 16 and (G & (G - 1)) == 0 and \
+        (w.page_size == 0 or w.page_size % 64 == 0 or w.page_size in (8, 16, 32))
+    attn = 1 if (w.dtype != "bf16" or tc) else 2
+    if w.stochastic:
+        tail = 2
+    else:
+        tail = 3 if w.tree_in_cache else 2
+    return heads + attn + tail
+
+
+class StepCtx:
+    """One workload's decode step on the device: seeded inputs resident in
+    HBM, a MedusaStep, and the step's calls (overlapped as MedusaStep.run
+    issues them, or the four calls in order)."""
+
+    def __init__(self, w, dev):
+        from medusa_tree_speculative_heads_b200 import binding as Bnd
+        from medusa_tree_speculative_heads_b200 import inputs as I
+        from medusa_tree_speculative_heads_b200.api import MedusaStep
+        self.w, self.dev = w, dev
+        self.parents = I.workload_tree(w)       # one parent list, or one per sequence
+        self.seq_trees = I.sequence_trees(w)
+        T = self.T = max(len(t) for t in self.seq_trees)
+        self.hin = hin = I.head_inputs(w, device="cuda")
+        self.ain = ain = I.attention_inputs(w, T, device="cuda")
+        self.block_table = None
+        paged = {}
+        if w.page_size:
+            # the cache as a page pool read through a block table
+            pc = I.paged_cache(w, w.page_size, ain["prefix_len"].cpu(), room=T, device="cuda",
+                               capacity=w.max_prefix + T)
+            ain["k_cache"], ain["v_cache"], self.block_table = pc["k_pages"], pc["v_pages"], pc["block_table"]
+            paged = dict(page_size=w.page_size, max_pages=self.block_table.shape[1], num_pages=pc["k_pages"].shape[0])
+        self.k_layers = self.v_layers = None
+        if w.tree_in_cache:
+            # the tree's K/V appended to each sequence's cache after its prefix
+            # (the target model's layers would write them there); every other
+            # layer's cache is compacted in the same launch
+            for b, tr in enumerate(self.seq_trees):
+                S = int(ain["prefix_len"][b])
+                ain["k_cache"][b, :, S:S + len(tr)] = ain["k_tree"][b, :len(tr)].transpose(0, 1)
+                ain["v_cache"][b, :, S:S + len(tr)] = ain["v_tree"][b, :len(tr)].transpose(0, 1)
+            self.k_layers = [ain["k_cache"]] + [ain["k_cache"].clone() for _ in range(w.layers - 1)]
+            self.v_layers = [ain["v_cache"]] + [ain["v_cache"].clone() for _ in range(w.layers - 1)]
+            ain["k_tree"] = ain["v_tree"] = None
+        mode = Bnd.STOCHASTIC if w.stochastic else Bnd.GREEDY
+        self.step = step = MedusaStep(B=w.B, d=w.d, V=w.V, K=w.K, Hq=w.Hq, Hkv=w.Hkv, D=w.D, S_max=w.S_max,
+                                      parents=self.parents, dtype=w.torch_dtype, max_prefix=w.max_prefix,
+                                      device=dev, mode=mode, q_rows=T, temperature=w.temperature,
+                                      tree_in_cache=w.tree_in_cache, **paged)
+        self.q_draft = self.vtok = None
+        if w.stochastic:
+            # the target's and the draft's distributions and the drafted tokens
+            # (children drawn from q at their parent) come from the harness
+            sd = I.stochastic_inputs(w, self.parents, device="cuda")
+            self.logits, self.q_draft, self.vtok = sd["p"], sd["q"], sd["node_tokens"]
+            if w.temperature > 0:   # the target's bf16 logits, read at the temperature
+                self.logits = sd["logits"].bfloat16()
+        else:
+            # the target model's logits (outside this path) are synthesised once
+            # from the tree the heads propose, with the workload's match probability
+            step.heads(hin["h"], hin["W_res"], hin["W_head"], hin["root_token"])
+            torch.cuda.synchronize()
+            self.logits = I.boosted_target_logits(w, self.parents, step.node_tokens.cpu(), device="cuda")
+        self.new_pl = torch.empty_like(ain["prefix_len"])
+
+    def run_kwargs(self, src=None):
+        """Arguments of MedusaStep.run; `src` replaces the per-step inputs
+        (h, root token, q, tree K/V, target, draft, drafted tokens)."""
+        hin, ain, src = self.hin, self.ain, src or {}
+        return dict(h=src.get("h", hin["h"]), W_res=hin["W_res"], W_head=hin["W_head"],
+                    root_token=src.get("root_token", hin["root_token"]), q=src.get("q", ain["q"]),
+                    k_tree=src.get("k_tree", ain["k_tree"]), v_tree=src.get("v_tree", ain["v_tree"]),
+                    k_cache=ain["k_cache"], v_cache=ain["v_cache"], prefix_len=ain["prefix_len"],
+                    new_prefix_len=self.new_pl, target=src.get("target", self.logits),
+                    q_draft=src.get("q_draft", self.q_draft), node_tokens=src.get("tokens", self.vtok),
+                    block_table=self.block_table, k_layers=self.k_layers, v_layers=self.v_layers)
+
+    def run_step(self):
+        self.step.run(**self.run_kwargs())
+
+    def stages(self, i):
+        """The four calls in order on the current stream."""
+        st, hin, ain = self.step, self.hin, self.ain
+        return [lambda: st.heads(hin["h"], hin["W_res"], hin["W_head"], hin["root_token"]),
+                lambda: st.attention(ain["q"], ain["k_tree"], ain["v_tree"], ain["k_cache"], ain["v_cache"],
+                                     ain["prefix_len"], self.block_table),
+                lambda: st.verify(self.logits, self.q_draft, None, 0, i, self.vtok),
+                lambda: st.commit(ain["k_cache"], ain["v_cache"], ain["k_tree"], ain["v_tree"], ain["prefix_len"],
+                                  self.new_pl, self.block_table, self.k_layers, self.v_layers)]
+
+    def algorithmic(self):
+        """Algorithmic bytes of the heads and of tree attention, and the
+        attention's FLOPs over visible (query, key) pairs only."""
+        w = self.w
+        elt = 2 if w.dtype == "bf16" else 4
+        heads_bytes = (w.K * w.d * w.d + w.K * w.V * w.d) * elt + w.B * w.d * elt
+        Sb = [int(x) for x in self.ain["prefix_len"].cpu()]
+        Ts = [len(t) for t in self.seq_trees]
+        attn_bytes = (2 * w.Hkv * sum(Sb) * w.D + 2 * sum(Ts) * w.Hq * w.D + 2 * sum(Ts) * w.Hkv * w.D) * elt
+        anc = {}
+        for tr in self.seq_trees:  # visible (node, tree node) pairs of each distinct tree
+            key = tuple(tr)
+            if key not in anc:
+                anc[key] = sum(1 for i in range(len(tr)) for j in range(len(tr)) if _is_anc(tr, i, j))
+        attn_flops = 4 * w.D * w.Hq * sum(Ts[b] * Sb[b] + anc[tuple(self.seq_trees[b])] for b in range(w.B))
+        return heads_bytes, attn_bytes, attn_flops
+
+
+L2_FLUSH_BYTES = 256 << 20   # twice the 126 MB L2
+
+
+def measure_stages(ctx, K, flush):
+    """Each of K repetitions: an L2 flush (a 256 MB memset, untimed), then the
+    four calls in order on one stream, each bracketed by CUDA events.
+    Returns the median time of each stage (s) and the mean in-order step (s)."""
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    for i in range(K):
+        flush.zero_()
+        calls = ctx.stages(i)
+        ev[i][0].record()
+        for j, call in enumerate(calls):
+            call()
+            ev[i][j + 1].record()
+    torch.cuda.synchronize()
+    stage = [statistics.median(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K)) / 1000.0 for j in range(4)]
+    serial = statistics.mean(ev[i][0].elapsed_time(ev[i][4]) for i in range(K)) / 1000.0
+    return stage, serial
+
+
+def measure_steps(ctx, K, world, dev, barrier):
+    """K back-to-back steps as MedusaStep.run issues them, CUDA events on the
+    launching stream, barrier and synchronize on both sides; the slowest
+    rank's time (s)."""
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(K):
+        ctx.run_step()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier()
+    return max_over_ranks(e0.elapsed_time(e1) / 1000.0, world, dev)
+
+
+def attention_roofline(attn_bytes, attn_flops, t_attn, pk):
+    gbs = attn_bytes / t_attn / 1e9
+    tflops = attn_flops / t_attn / 1e12
+    bound = "tensor" if attn_flops / (pk["bf16_tflops"] * 1e12) > attn_bytes / (pk["hbm_gbs"] * 1e9) else "hbm"
+    return {"us": t_attn * 1e6, "algorithmic_bytes": attn_bytes, "algorithmic_flops": attn_flops, "hbm_gbs": gbs,
+            "hbm_frac": gbs / pk["hbm_gbs"], "tflops": tflops, "tc_frac": tflops / pk["bf16_tflops"], "bound": bound}
+
+
+def measure_config(name, args, world, dev, barrier, flush, pk):
+    """A compact measurement of another workload (same protocol, fewer steps)."""
+    from medusa_tree_speculative_heads_b200 import inputs as I
+    w = I.WORKLOADS[name]
+    ctx = StepCtx(w, dev)
+    K = max(5, min(args.steps, 30))
+    for _ in range(max(args.warmup, 3)):
+        ctx.run_step()
+    torch.cuda.synchronize()
+    stage, serial = measure_stages(ctx, K, flush)
+    t = measure_steps(ctx, K, world, dev, barrier)
+    hb, ab, af = ctx.algorithmic()
+    out = {"workload": config_dict(w, world)["workload"], "steps": K, "value": whole_job_rate(world, K, t),
+           "unit": UNIT, "ms_per_step": 1000.0 * t / K, "serial_ms_per_step": 1000.0 * serial,
+           "stage_us": {"medusa_heads": stage[0] * 1e6, "tree_attention": stage[1] * 1e6,
+                        "tree_verify": stage[2] * 1e6, "kv_commit": stage[3] * 1e6},
+           "medusa_heads": {"gbs": hb / stage[0] / 1e9, "hbm_frac": hb / stage[0] / 1e9 / pk["hbm_gbs"]},
+           "tree_attention": attention_roofline(ab, af, stage[1], pk),
+           "mean_accept_len": float(ctx.step.accept_len.float().mean().item()),
+           "status": int(ctx.step.status.item())}
+    del ctx
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_mine(args, rank, world, local_rank):
@@ -316,7 +519,6 @@ def run_mine(args, rank, world, local_rank):
 
     from medusa_tree_speculative_heads_b200 import build as build_mod
     from medusa_tree_speculative_heads_b200 import inputs as I
-    from medusa_tree_speculative_heads_b200.api import MedusaStep
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
@@ -327,105 +529,30 @@ def run_mine(args, rank, world, local_rank):
     if world > 1:
         dist.barrier()
 
-    w = I.WORKLOADS[args.workload]
-    parents = I.workload_tree(w)       # one parent list, or one per sequence
-    seq_trees = I.sequence_trees(w)
-    T = max(len(t) for t in seq_trees)
-    hin = I.head_inputs(w, device="cuda")
-    ain = I.attention_inputs(w, T, device="cuda")
-    block_table = None
-    paged = {}
-    if w.page_size:
-        # the cache as a page pool read through a block table
-        pc = I.paged_cache(w, w.page_size, ain["prefix_len"].cpu(), room=T, device="cuda",
-                           capacity=w.max_prefix + T)
-        ain["k_cache"], ain["v_cache"], block_table = pc["k_pages"], pc["v_pages"], pc["block_table"]
-        paged = dict(page_size=w.page_size, max_pages=block_table.shape[1], num_pages=pc["k_pages"].shape[0])
-    k_layers = v_layers = None
-    if w.tree_in_cache:
-        # the tree's K/V appended to each sequence's cache after its prefix (the
-        # target model's layers would write them there); every other layer's
-        # cache is compacted in the same launch
-        for b, tr in enumerate(seq_trees):
-            S = int(ain["prefix_len"][b])
-            ain["k_cache"][b, :, S:S + len(tr)] = ain["k_tree"][b, :len(tr)].transpose(0, 1)
-            ain["v_cache"][b, :, S:S + len(tr)] = ain["v_tree"][b, :len(tr)].transpose(0, 1)
-        k_layers = [ain["k_cache"]] + [ain["k_cache"].clone() for _ in range(w.layers - 1)]
-        v_layers = [ain["v_cache"]] + [ain["v_cache"].clone() for _ in range(w.layers - 1)]
-        ain["k_tree"] = ain["v_tree"] = None
-    from medusa_tree_speculative_heads_b200 import binding as Bnd
-    mode = Bnd.STOCHASTIC if w.stochastic else Bnd.GREEDY
-    step = MedusaStep(B=w.B, d=w.d, V=w.V, K=w.K, Hq=w.Hq, Hkv=w.Hkv, D=w.D, S_max=w.S_max, parents=parents,
-                      dtype=w.torch_dtype, max_prefix=w.max_prefix, device=dev, mode=mode, q_rows=T,
-                      temperature=w.temperature, tree_in_cache=w.tree_in_cache, **paged)
-    q_draft = vtok = None
-    if w.stochastic:
-        # the target's and the draft's distributions and the drafted tokens
-        # (children drawn from q at their parent) come from the harness
-        sd = I.stochastic_inputs(w, parents, device="cuda")
-        logits, q_draft, vtok = sd["p"], sd["q"], sd["node_tokens"]
-        if w.temperature > 0:   # the target's bf16 logits, read at the temperature
-            logits = sd["logits"].bfloat16()
-    else:
-        # the target model's logits (outside this path) are synthesised once
-        # from the tree the heads propose, with the workload's match probability
-        step.heads(hin["h"], hin["W_res"], hin["W_head"], hin["root_token"])
-        torch.cuda.synchronize()
-        logits = I.boosted_target_logits(w, parents, step.node_tokens.cpu(), device="cuda")
-    new_pl = torch.empty_like(ain["prefix_len"])
-
-    def run_step():
-        step.run(h=hin["h"], W_res=hin["W_res"], W_head=hin["W_head"], root_token=hin["root_token"], q=ain["q"],
-                 k_tree=ain["k_tree"], v_tree=ain["v_tree"], k_cache=ain["k_cache"], v_cache=ain["v_cache"],
-                 prefix_len=ain["prefix_len"], new_prefix_len=new_pl, target=logits, q_draft=q_draft,
-                 node_tokens=vtok, block_table=block_table, k_layers=k_layers, v_layers=v_layers)
-
     def barrier():
         if world > 1:
             dist.barrier()
 
+    w = I.WORKLOADS[args.workload]
+    ctx = StepCtx(w, dev)
+    step, hin, ain = ctx.step, ctx.hin, ctx.ain
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     for _ in range(max(args.warmup, 3)):
-        run_step()
+        ctx.run_step()
     torch.cuda.synchronize()
-
-    # ---- per-stage breakdown: the four calls in order on one stream ----
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local_rank)
     clocks.start()
     time.sleep(0.3)
-    barrier()
-    torch.cuda.synchronize()
-    for i in range(K):
-        ev[i][0].record()
-        step.heads(hin["h"], hin["W_res"], hin["W_head"], hin["root_token"])
-        ev[i][1].record()
-        step.attention(ain["q"], ain["k_tree"], ain["v_tree"], ain["k_cache"], ain["v_cache"], ain["prefix_len"],
-                       block_table)
-        ev[i][2].record()
-        step.verify(logits, q_draft, None, 0, i, vtok)
-        ev[i][3].record()
-        step.commit(ain["k_cache"], ain["v_cache"], ain["k_tree"], ain["v_tree"], ain["prefix_len"], new_pl,
-                    block_table, k_layers, v_layers)
-        ev[i][4].record()
-    torch.cuda.synchronize()
-    serial_s = ev[0][0].elapsed_time(ev[K - 1][4]) / 1000.0
+    # ---- per-stage breakdown: the four calls in order, an L2 flush before each
+    # repetition, median of K ----
+    stage, serial_s = measure_stages(ctx, K, flush)
     # ---- device-timed steps (the value): the step as MedusaStep.run issues
-    # it, tree attention on a second stream overlapping the heads' last CTA ----
-    barrier()
-    torch.cuda.synchronize()
-    e0.record()
-    for i in range(K):
-        run_step()
-    e1.record()
-    torch.cuda.synchronize()
-    barrier()
+    # it, tree attention on a second stream overlapping the heads' tail; each
+    # step streams the heads' weights, far more than the 126 MB L2 ----
+    t = measure_steps(ctx, K, world, dev, barrier)
     clk = clocks.stop()
-    t_local = e0.elapsed_time(e1) / 1000.0
-    t = max_over_ranks(t_local, world, dev)
     value = whole_job_rate(world, K, t)
-    stage = [statistics.mean(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K)) / 1000.0 for j in range(4)]
     assert int(step.status.item()) == 0, "device status set during the benchmark"
     mean_len = float(step.accept_len.float().mean().item())
 
@@ -433,13 +560,13 @@ def run_mine(args, rank, world, local_rank):
     # every step copies its own inputs from pinned host memory (h, root token,
     # the tree's Q/K/V and the target logits) and reads its results back; the
     # copies run on a second stream into two alternating device buffers, so the
-    # next step's 31 MB upload overlaps this step's compute, as a serving loop would
+    # next step's upload overlaps this step's compute, as a serving loop would
     names_in = ["h", "root_token", "q"] + ([] if w.tree_in_cache else ["k_tree", "v_tree"])
     host_in = {n: (hin if n in hin else ain)[n].cpu().pin_memory() for n in names_in}
-    host_in["target"] = logits.cpu().pin_memory()
+    host_in["target"] = ctx.logits.cpu().pin_memory()
     if w.stochastic:
-        host_in["q_draft"] = q_draft.cpu().pin_memory()
-        host_in["tokens"] = vtok.cpu().pin_memory()
+        host_in["q_draft"] = ctx.q_draft.cpu().pin_memory()
+        host_in["tokens"] = ctx.vtok.cpu().pin_memory()
     dev_in = [{n: torch.empty_like(host_in[n], device=dev) for n in host_in} for _ in range(2)]
     outs = [step.accept_path, step.accept_len, step.bonus, step.node_tokens]
     host_out = [torch.empty_like(o, device="cpu").pin_memory() for o in outs]
@@ -447,24 +574,28 @@ def run_mine(args, rank, world, local_rank):
     d2h = sum(x.numel() * x.element_size() for x in host_out)
     main_stream = torch.cuda.current_stream()
     copy_stream = torch.cuda.Stream(device=dev)
+    # this machine's host-to-device rate for the step's uploads alone (median of 5)
+    rates = []
+    for _ in range(5):
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(copy_stream):
+            c0.record(copy_stream)
+            for n in host_in:
+                dev_in[0][n].copy_(host_in[n], non_blocking=True)
+            c1.record(copy_stream)
+        c1.synchronize()
+        rates.append(h2d / (c0.elapsed_time(c1) / 1000.0) / 1e9)
+    h2d_gbs = statistics.median(rates)
     copied = [torch.cuda.Event(), torch.cuda.Event()]
     used = [torch.cuda.Event(), torch.cuda.Event()]
-    for ev in used:
-        ev.record(main_stream)
-
-    def run_kwargs(slot):
-        d = dev_in[slot]
-        return dict(h=d["h"], W_res=hin["W_res"], W_head=hin["W_head"], root_token=d["root_token"], q=d["q"],
-                    k_tree=d.get("k_tree"), v_tree=d.get("v_tree"), k_cache=ain["k_cache"], v_cache=ain["v_cache"],
-                    prefix_len=ain["prefix_len"], new_prefix_len=new_pl, target=d["target"],
-                    q_draft=d.get("q_draft"), node_tokens=d.get("tokens"), block_table=block_table,
-                    k_layers=k_layers, v_layers=v_layers)
+    for e in used:
+        e.record(main_stream)
 
     # one CUDA graph per input slot: a step is one graph launch on the host
     graphs, e2e_mode = None, "cuda-graph"
     try:
         torch.cuda.synchronize()
-        graphs = [step.capture(**run_kwargs(slot)) for slot in range(2)]
+        graphs = [step.capture(**ctx.run_kwargs(dev_in[slot])) for slot in range(2)]
         torch.cuda.synchronize()
     except Exception as exc:  # capture unsupported here: the four calls are issued eagerly
         graphs, e2e_mode = None, f"eager ({type(exc).__name__})"
@@ -481,7 +612,7 @@ def run_mine(args, rank, world, local_rank):
         if graphs is not None:
             graphs[slot].replay()
         else:
-            step.run(**run_kwargs(slot))
+            step.run(**ctx.run_kwargs(dev_in[slot]))
         used[slot].record(main_stream)
         for o, ho in zip(outs, host_out):
             ho.copy_(o, non_blocking=True)
@@ -489,6 +620,7 @@ def run_mine(args, rank, world, local_rank):
     for i in range(3):
         e2e_step(i)
     torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
     e0.record()
@@ -499,44 +631,32 @@ def run_mine(args, rank, world, local_rank):
     barrier()
     t_e2e = max_over_ranks(e0.elapsed_time(e1) / 1000.0, world, dev)
     value_e2e = whole_job_rate(world, K, t_e2e)
+    del graphs
 
     # ---- roofline of the dominant stage (the heads) and of tree attention ----
     pk = peaks()
-    elt = 2 if w.dtype == "bf16" else 4
-    heads_bytes = (w.K * w.d * w.d + w.K * w.V * w.d) * elt + w.B * w.d * elt
+    heads_bytes, attn_bytes, attn_flops = ctx.algorithmic()
     heads_gbs = heads_bytes / stage[0] / 1e9
-    Sb = [int(x) for x in ain["prefix_len"].cpu()]
-    sum_S = sum(Sb)
-    Ts = [len(t) for t in seq_trees]
-    attn_bytes = (2 * w.Hkv * sum_S * w.D + 2 * sum(Ts) * w.Hq * w.D + 2 * sum(Ts) * w.Hkv * w.D) * elt
-    attn_gbs = attn_bytes / stage[1] / 1e9
-    anc = {}
-    for tr in seq_trees:  # visible (node, tree node) pairs of each distinct tree
-        key = tuple(tr)
-        if key not in anc:
-            anc[key] = sum(1 for i in range(len(tr)) for j in range(len(tr)) if _is_anc(tr, i, j))
-    attn_flops = 4 * w.D * w.Hq * sum(Ts[b] * Sb[b] + anc[tuple(seq_trees[b])] for b in range(w.B))
-    attn_tflops = attn_flops / stage[1] / 1e12
-
+    att = attention_roofline(attn_bytes, attn_flops, stage[1], pk)
     # the roofline object describes the step's dominant kernel: the heads
     # kernel (HBM-bound weight stream) or, at long contexts, tree attention,
     # bound by whichever of its HBM bytes and tensor-core FLOPs takes longer
-    attn_bound = "tensor" if attn_flops / (pk["bf16_tflops"] * 1e12) > attn_bytes / (pk["hbm_gbs"] * 1e9) else "hbm"
     if stage[1] > stage[0]:
-        if attn_bound == "tensor":
-            roofline = {"kernel": "tree_attention (split-KV tcgen05 kernel + combine)", "bound": "tensor",
-                        "achieved": attn_tflops, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                        "frac": attn_tflops / pk["bf16_tflops"], "peak_source": pk["source"],
-                        "algorithmic_flops": attn_flops, "traffic": None}
+        if att["bound"] == "tensor":
+            roofline = {"kernel": "tree_attention", "bound": "tensor", "achieved": att["tflops"],
+                        "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": att["tc_frac"],
+                        "peak_source": pk["source"], "algorithmic_flops": attn_flops, "traffic": None}
         else:
-            roofline = {"kernel": "tree_attention (split-KV tcgen05 kernel + combine)", "bound": "hbm",
-                        "achieved": attn_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": attn_gbs / pk["hbm_gbs"],
-                        "peak_source": pk["source"], "algorithmic_bytes": attn_bytes, "traffic": None}
+            roofline = {"kernel": "tree_attention", "bound": "hbm", "achieved": att["hbm_gbs"],
+                        "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": att["hbm_frac"], "peak_source": pk["source"],
+                        "algorithmic_bytes": attn_bytes, "traffic": None}
     else:
         roofline = {"kernel": "medusa_heads (residual GEMV + LM-head GEMV with softmax/top-8 + merge)",
                     "bound": "hbm", "achieved": heads_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                     "frac": heads_gbs / pk["hbm_gbs"], "peak_source": pk["source"],
-                    "algorithmic_bytes": heads_bytes, "traffic": HEADS_DRAM_BYTES.get(w.name) if w.name not in OVERRIDDEN else None}
+                    "algorithmic_bytes": heads_bytes,
+                    "traffic": HEADS_DRAM_BYTES.get(w.name) if w.name not in OVERRIDDEN else None}
+    roofline["timing"] = "median of the heads stage over K in-order repetitions, each after a 256 MB L2 flush"
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": 1000.0 * t / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -546,40 +666,45 @@ def run_mine(args, rank, world, local_rank):
                                    f"from the proposed tree with match probability {w.match_prob})"),
         "config": config_dict(w, world),
         "roofline": roofline,
-        "tree_attention": {"us": stage[1] * 1e6, "algorithmic_bytes": attn_bytes, "algorithmic_flops": attn_flops,
-                           "hbm_gbs": attn_gbs, "hbm_frac": attn_gbs / pk["hbm_gbs"], "tflops": attn_tflops,
-                           "tc_frac": attn_tflops / pk["bf16_tflops"], "bound": attn_bound},
+        "tree_attention": att,
         "stage_us": {"medusa_heads": stage[0] * 1e6, "tree_attention": stage[1] * 1e6,
                      "tree_verify": stage[2] * 1e6, ("kv_compact" if w.tree_in_cache else "kv_commit"): stage[3] * 1e6},
-        "serial_ms_per_step": 1000.0 * serial_s / K,
+        "timing": ("value: K back-to-back steps as MedusaStep.run issues them (attention overlapped with the heads' "
+                   "tail), CUDA events on the launching stream; stage_us and serial_ms_per_step: the four calls in "
+                   "order, median (stages) / mean (step) of K repetitions, each after a 256 MB L2 flush"),
+        "serial_ms_per_step": 1000.0 * serial_s,
         "mean_accept_len": mean_len,
         **({"kv_compact": {"layers": w.layers, "us": stage[3] * 1e6,
-                           "moved_bytes": 2 * 2 * w.layers * w.Hkv * w.D * elt * int(step.accept_len.sum().item()),
+                           "moved_bytes": 2 * 2 * w.layers * w.Hkv * w.D * (2 if w.dtype == "bf16" else 4) *
+                           int(step.accept_len.sum().item()),
                            "note": "read + write of the accepted rows' K and V in every layer, one launch"}}
            if w.tree_in_cache else {}),
         "tokens_per_s": value * w.B * (mean_len + 1),
         "e2e": {"value": value_e2e, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "mode": e2e_mode},
+                "mode": e2e_mode, "h2d_gbs_measured": h2d_gbs,
+                "note": "inputs copied from pinned host memory every step; the upload hides behind compute only "
+                        "when h2d_bytes_per_step / h2d_gbs_measured is below the step time"},
         "gpu_launches": K * launches_per_step(w),
         "clocks": clk,
     }
+    del ctx
+    torch.cuda.empty_cache()
+    # ---- the other configurations, each measured the same way (fewer steps) ----
+    names = [n for n in args.configs.split(",") if n and n not in (w.name, "none")]
+    if names:
+        out["configs"] = {n: measure_config(n, args, world, dev, barrier, flush, pk) for n in names}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        import oracle
-        oracle.build()
         frac = 1.0 / 16 if w.stochastic else 1.0   # B=64: a vocabulary / query-row slice keeps it to seconds
-        sample = OracleSample(w, frac)
-        tt, ff = 0.0, 0.0
-        while tt < 10.0 and ff < 3.0:
-            t1, f1 = sample.run()
-            tt += t1
-            ff += f1
-        out["cpu_baseline"] = {"value": ff / tt, "unit": UNIT, "cores": 1, "kind": "oracle",
-                               "sample": (f"{ff:.2f} whole steps of the same workload run by the single-threaded "
-                                          f"fp64 oracle on the host ({tt:.1f} s)" if frac == 1.0 else
-                                          f"{ff:.2f} steps' worth of work: the fp64 oracle on the host ({tt:.1f} s), "
-                                          f"residual blocks whole, LM-head rows of a 1/16 vocabulary slice, 1/16 of "
-                                          f"the attention rows, verification and commit whole; steps/s scaled by "
-                                          f"the sampled fraction")}
+        v_omp, t_omp, f_omp, cores = time_oracle(w, frac, 10.0, 10.0, True)
+        v_one, t_one, f_one, _ = time_oracle(w, frac, 10.0, 3.0, False)
+        what = ("whole steps of the same workload" if frac == 1.0 else
+                "steps' worth of work (residual blocks whole, LM-head rows of a 1/16 vocabulary slice, 1/16 of the "
+                "attention rows, verification and commit whole; steps/s scaled by the sampled fraction)")
+        out["cpu_baseline"] = {"value": v_omp, "unit": UNIT, "cores": cores, "kind": "oracle",
+                               "sample": (f"{f_omp:.2f} {what}: the fp64 oracle's OpenMP build on {cores} host "
+                                          f"threads ({t_omp:.1f} s)"),
+                               "single_thread": {"value": v_one, "unit": UNIT, "cores": 1,
+                                                 "sample": f"{f_one:.2f} {what}, serial build ({t_one:.1f} s)"}}
     if rank == 0:
         print(json.dumps(out), flush=True)
     if world > 1:
@@ -602,6 +727,8 @@ def main():
     ap.add_argument("--impl", default="mine", choices=["mine", "reference"])
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--configs", default="tiny,llama70b_b8,long32k,long128k,stoch_b64",
+                    help="other workloads measured compactly into the line's 'configs' object ('none' for none)")
     ap.add_argument("--override", action="append", default=[],
                     help="replace a workload size, e.g. --override V=32000 (profiling a smaller case)")
     args = ap.parse_args()

@@ -385,6 +385,29 @@ int tree_verify_greedy_walk(const int32_t* node_tokens, int B, int V, const medu
                             size_t workspace_bytes, medusa_stream_t stream);
 
 /*
+ * tree_verify_greedy_walk followed, in the same launch, by the commit of the
+ * path it finds ("Multi-Token Prediction & Draft-Model-Free Speculative
+ * Decoding", section "The 2D Tree Attention Mask": the longest accepted path
+ * is committed; "Medusa Explained", "2. Single-Pass Tree Attention
+ * Verification", step 4).  Gives exactly tree_verify_greedy_walk then
+ * kv_commit (block_table NULL: contiguous cache [B, Hkv, S_max, D]) or
+ * kv_commit_paged (block_table non-NULL: page pools [num_pages, Hkv,
+ * page_size, D]; S_max ignored) with T = the tree's node count, in one
+ * kernel per step instead of two dependent ones.  Walk arguments as
+ * tree_verify_greedy_walk (after tree_verify_greedy_rows on the same
+ * workspace); cache arguments as kv_commit / kv_commit_paged, including
+ * their checks, status bits (CACHE_OVERFLOW, BAD_TOKEN) and in-place
+ * new_prefix_len == prefix_len.  dt is the K/V dtype.
+ */
+int tree_verify_greedy_walk_commit(const int32_t* node_tokens, int B, int V, const medusa_tree* tree,
+                                   int32_t* accept_path, int max_path, int32_t* accept_len, int32_t* bonus,
+                                   const void* workspace, size_t workspace_bytes, void* k_cache, void* v_cache,
+                                   const void* k_tree, const void* v_tree, const int32_t* prefix_len,
+                                   int32_t* new_prefix_len, int Hkv, int D, int S_max, const int32_t* block_table,
+                                   int max_pages, int page_size, int num_pages, medusa_dtype dt, int32_t* status,
+                                   medusa_stream_t stream);
+
+/*
  * STOCHASTIC verification reading the target's logits instead of its
  * probabilities: the walk of tree_verify (STOCHASTIC) with P, wherever the
  * walk reads the target's own row of node u, taken as

@@ -370,10 +370,20 @@ class MedusaStep:
                 main.wait_stream(self._side2)
             main.wait_stream(self._hp)        # the walk (or the whole verification) and commit after all
             main.wait_stream(self._side)
+            tokens = self.node_tokens if node_tokens is None else node_tokens
+            if greedy_split and not self.tree_in_cache:
+                # the walk and the commit of the path it finds: one launch
+                paged = self.page_size > 0
+                _b.tree_verify_greedy_walk_commit(tokens, self.B, self.V, self.tree, self.accept_path, self.max_path,
+                                                  self.accept_len, self.bonus, self.ws_verify, self.ws_verify_n,
+                                                  k_cache, v_cache, k_tree, v_tree, prefix_len, new_prefix_len,
+                                                  self.Hkv, self.D, self.S_max, block_table if paged else None,
+                                                  self.max_pages, self.page_size, self.num_pages, self.dt,
+                                                  self.status)
+                return
             if greedy_split:
-                _b.tree_verify_greedy_walk(self.node_tokens if node_tokens is None else node_tokens, self.B, self.V,
-                                           self.tree, self.accept_path, self.max_path, self.accept_len, self.bonus,
-                                           self.ws_verify, self.ws_verify_n)
+                _b.tree_verify_greedy_walk(tokens, self.B, self.V, self.tree, self.accept_path, self.max_path,
+                                           self.accept_len, self.bonus, self.ws_verify, self.ws_verify_n)
             else:
                 self.verify(target, q_draft, q_row, seed, step, node_tokens)
             self.commit(k_cache, v_cache, k_tree, v_tree, prefix_len, new_prefix_len, block_table, k_layers,

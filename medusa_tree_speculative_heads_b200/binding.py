@@ -81,6 +81,8 @@ def lib() -> ctypes.CDLL:
                                   vp]
         L.tree_verify_greedy_rows.argtypes = [vp, i32, i32, i32, vp, vp, sz, vp]
         L.tree_verify_greedy_walk.argtypes = [vp, i32, i32, vp, vp, i32, vp, vp, vp, sz, vp]
+        L.tree_verify_greedy_walk_commit.argtypes = [vp, i32, i32, vp, vp, i32, vp, vp, vp, sz, vp, vp, vp, vp, vp,
+                                                     vp, i32, i32, i32, vp, i32, i32, i32, i32, vp, vp]
         L.tree_verify_logits.argtypes = [vp, i32, ctypes.c_double, vp, i32, vp, vp, i32, i32, vp, u64, u32, vp, i32,
                                          vp, vp, vp, sz, vp, vp]
         L.kv_commit.argtypes = [vp, vp, vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp]
@@ -236,6 +238,16 @@ def tree_verify_greedy_walk(node_tokens, B, V, tree: Tree, accept_path, max_path
                             workspace_bytes, stream=None):
     _check(lib().tree_verify_greedy_walk(_p(node_tokens), B, V, tree.handle, _p(accept_path), max_path,
                                          _p(accept_len), _p(bonus), _p(workspace), workspace_bytes, _stream(stream)))
+
+
+def tree_verify_greedy_walk_commit(node_tokens, B, V, tree: Tree, accept_path, max_path, accept_len, bonus, workspace,
+                                   workspace_bytes, k_cache, v_cache, k_tree, v_tree, prefix_len, new_prefix_len, Hkv,
+                                   D, S_max, block_table, max_pages, page_size, num_pages, dt, status, stream=None):
+    _check(lib().tree_verify_greedy_walk_commit(_p(node_tokens), B, V, tree.handle, _p(accept_path), max_path,
+                                                _p(accept_len), _p(bonus), _p(workspace), workspace_bytes,
+                                                _p(k_cache), _p(v_cache), _p(k_tree), _p(v_tree), _p(prefix_len),
+                                                _p(new_prefix_len), Hkv, D, S_max, _p(block_table), max_pages,
+                                                page_size, num_pages, dt, _p(status), _stream(stream)))
 
 
 def tree_verify_logits(logits, logits_dt, temperature, q, q_rows, q_row, node_tokens, B, V, tree: Tree, seed, step,

@@ -603,6 +603,80 @@ extern "C" int tree_verify_greedy_walk(const int32_t* node_tokens, int B, int V,
     return ok();
 }
 
+extern "C" int tree_verify_greedy_walk_commit(const int32_t* node_tokens, int B, int V, const medusa_tree* tree,
+                                              int32_t* accept_path, int max_path, int32_t* accept_len,
+                                              int32_t* bonus, const void* workspace, size_t workspace_bytes,
+                                              void* k_cache, void* v_cache, const void* k_tree, const void* v_tree,
+                                              const int32_t* prefix_len, int32_t* new_prefix_len, int Hkv, int D,
+                                              int S_max, const int32_t* block_table, int max_pages, int page_size,
+                                              int num_pages, medusa_dtype dt, int32_t* status,
+                                              medusa_stream_t stream) {
+    const char* fn = "tree_verify_greedy_walk_commit";
+    if (!node_tokens || !accept_path || !accept_len || !bonus)
+        return fail(MEDUSA_ERR_INVALID_ARG, "%s: NULL verification argument", fn);
+    if (!k_cache || !v_cache || !k_tree || !v_tree || !prefix_len || !new_prefix_len)
+        return fail(MEDUSA_ERR_INVALID_ARG, "%s: NULL cache argument", fn);
+    if (dt != MEDUSA_F32 && dt != MEDUSA_BF16) return fail(MEDUSA_ERR_UNSUPPORTED, "%s: unknown dtype", fn);
+    int rc = check_tree(tree, B);
+    if (rc) return rc;
+    const int T = tree->host.T;
+    if (B < 1 || V < 1 || Hkv < 1 || D < 1)
+        return fail(MEDUSA_ERR_INVALID_ARG, "%s: bad sizes B=%d V=%d Hkv=%d D=%d", fn, B, V, Hkv, D);
+    if (max_path < tree->host.max_depth || max_path > kMaxTree)
+        return fail(MEDUSA_ERR_INVALID_ARG, "%s: max_path %d outside [tree depth %d, %d]", fn, max_path,
+                    tree->host.max_depth, kMaxTree);
+    if (block_table ? (max_pages < 1 || page_size < 1 || num_pages < 1) : S_max < 0)
+        return fail(MEDUSA_ERR_INVALID_ARG, "%s: bad cache sizes S_max=%d max_pages=%d page_size=%d num_pages=%d", fn,
+                    S_max, max_pages, page_size, num_pages);
+    const int esize = dt == MEDUSA_BF16 ? 2 : 4;
+    if ((D * esize) % 16)
+        return fail(MEDUSA_ERR_INVALID_ARG, "%s: a K/V row (%d bytes) must be a multiple of 16 bytes", fn, D * esize);
+    if (!al16(k_cache) || !al16(v_cache) || !al16(k_tree) || !al16(v_tree))
+        return fail(MEDUSA_ERR_INVALID_ARG, "%s: tensors must be 16-byte aligned", fn);
+    const size_t need = verify_workspace_size(MEDUSA_VERIFY_GREEDY, B, V, T);
+    if (!workspace || workspace_bytes < need || !al16(workspace))
+        return fail(MEDUSA_ERR_WORKSPACE, "%s: workspace of %zu bytes, need %zu", fn, workspace_bytes, need);
+    VerifyArgs a;
+    memset(&a, 0, sizeof a);
+    a.mode = MEDUSA_VERIFY_GREEDY;
+    a.node_tokens = node_tokens;
+    a.B = B;
+    a.V = V;
+    a.T = T;
+    a.tree = tree->ref();
+    a.accept_path = accept_path;
+    a.max_path = max_path;
+    a.accept_len = accept_len;
+    a.bonus = bonus;
+    a.ws = const_cast<void*>(workspace);
+    a.ws_bytes = workspace_bytes;
+    CommitArgs c;
+    memset(&c, 0, sizeof c);
+    c.k_cache = k_cache;
+    c.v_cache = v_cache;
+    c.k_tree = k_tree;
+    c.v_tree = v_tree;
+    c.accept_path = accept_path;
+    c.max_path = max_path;
+    c.accept_len = accept_len;
+    c.prefix_len = prefix_len;
+    c.new_prefix_len = new_prefix_len;
+    c.B = B;
+    c.T = T;
+    c.Hkv = Hkv;
+    c.D = D;
+    c.S_max = block_table ? 0 : S_max;
+    c.esize = esize;
+    c.block_table = block_table;
+    c.max_pages = block_table ? max_pages : 0;
+    c.page_size = block_table ? page_size : 0;
+    c.num_pages = block_table ? num_pages : 0;
+    c.status = status;
+    cudaError_t e = verify_greedy_walk_commit_launch(a, c, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, fn);
+    return ok();
+}
+
 extern "C" int tree_verify_logits(const void* logits, medusa_dtype logits_dt, double temperature, const float* q,
                                   int q_rows, const int32_t* q_row, const int32_t* node_tokens, int B, int V,
                                   const medusa_tree* tree, uint64_t seed, uint32_t step, int32_t* accept_path,

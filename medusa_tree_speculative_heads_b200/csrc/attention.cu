@@ -493,16 +493,14 @@ bool use_tc(const AttnArgs& a, int D) {
     return attn_tc_supported(a.Hq, a.Hkv, D, a.T, a.dt) && (!a.block_table || attn_tc_page_ok(a.page_size));
 }
 
-SplitPlan plan_bf16(int B, int T, int Hq, int Hkv, int D, int max_prefix, bool tc) {
-    // tensor-core kernel: 128-row tiles, two CTAs per SM
-    if (tc) return plan_splits(B, T, Hq, Hkv, max_prefix, 128, attn_tc_ctas_per_sm());
+SplitPlan plan_bf16(int B, int T, int Hq, int Hkv, int max_prefix) {
     return plan_splits(B, T, Hq, Hkv, max_prefix);
 }
 
 template <int D>
 cudaError_t attn_launch_bf16(const AttnArgs& a, cudaStream_t st) {
     const bool tc = use_tc(a, D);
-    SplitPlan sp = plan_bf16(a.B, a.T, a.Hq, a.Hkv, D, a.max_prefix, tc);
+    SplitPlan sp = plan_bf16(a.B, a.T, a.Hq, a.Hkv, a.max_prefix);
     AttnParams p;
     p.q = (const __nv_bfloat16*)a.q;
     p.k_tree = (const __nv_bfloat16*)a.k_tree;
@@ -531,17 +529,19 @@ cudaError_t attn_launch_bf16(const AttnArgs& a, cudaStream_t st) {
     p.part_o = (float*)a.ws;
     p.part_lse = (float*)((char*)a.ws + align256((size_t)sp.n_splits * BH * p.R * D * sizeof(float)));
     p.status = a.status;
-    cudaError_t e;
     if (tc) {
-        e = attn_tc_launch(a, sp.m_tiles, sp.n_splits, sp.split_len, p.scale_log2, p.part_o, p.part_lse, st);
-    } else {
+        // 128-row tiles; the key splits of a tile merge inside their cluster
+        const int m_tiles = (a.T * p.G + 127) / 128;
+        return attn_tc_launch(a, m_tiles, attn_tc_splits(a.B, a.T, a.Hq, a.Hkv, a.max_prefix), p.scale_log2, st);
+    }
+    {
         const size_t smem = (size_t)kBM * D * 2 + 4 * (size_t)kBN * D * 2 + kBM * 4 * sizeof(uint32_t);
         cudaFuncSetAttribute(tree_attn_mma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         dim3 grid(sp.m_tiles, (unsigned)BH, sp.n_splits);
         tree_attn_mma_kernel<D><<<grid, kThreads, smem, st>>>(p);
-        e = cudaGetLastError();
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
     }
-    if (e != cudaSuccess) return e;
     const long rows = (long)a.B * a.T * a.Hq;
     prefer_max_smem(attn_combine_kernel<D>);
     attn_combine_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(p.part_o, p.part_lse, a.B, a.T, a.Hq, a.Hkv,
@@ -565,9 +565,10 @@ cudaError_t attn_launch_f32(const AttnArgs& a, cudaStream_t st) {
 
 size_t attn_workspace_size(int B, int T, int Hq, int Hkv, int D, int max_prefix, medusa_dtype dt) {
     if (dt != MEDUSA_BF16) return 0;
-    // enough for either kernel (a paged call may run either, by page size)
-    const SplitPlan a = plan_bf16(B, T, Hq, Hkv, D, max_prefix, true), b = plan_bf16(B, T, Hq, Hkv, D, max_prefix, false);
-    const size_t splits = a.n_splits > b.n_splits ? a.n_splits : b.n_splits;
+    // the mma.sync kernel's split partials (the tensor-core kernel needs none,
+    // but a paged call may run either kernel, by page size)
+    const SplitPlan a = plan_bf16(B, T, Hq, Hkv, max_prefix);
+    const size_t splits = a.n_splits;
     const size_t R = (size_t)T * (Hq / Hkv);
     const size_t BH = (size_t)B * Hkv;
     return align256(splits * BH * R * D * sizeof(float)) + align256(splits * BH * R * sizeof(float));

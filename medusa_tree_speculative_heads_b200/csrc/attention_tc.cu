@@ -9,8 +9,10 @@
 //
 // One CTA takes 128 query rows of one (sequence, kv-head) -- rows are
 // node-major, row = node * G + (q-head within the group), so the G q-heads
-// of a node share every K/V element -- and one range of keys (a prefix split
-// or the tree itself).  Per 64-key chunk:
+// of a node share every K/V element -- and a run of 64-key chunks.  A
+// sequence's chunks are its prefix chunks followed by its tree's one or two
+// chunks; the C CTAs of a thread-block cluster (cluster dims (1, 1, C)) take
+// equal runs of that list.  Per chunk:
 //   S   = Q K^T      tcgen05.mma M=128, N=64,  K=D   (both operands K-major)
 //   P   = exp2(S * scale * log2 e - m), masked; bf16, written back into TMEM
 //         over S's own columns
@@ -23,13 +25,20 @@
 // the previous PV completed.  The result is the same after the final 1/l.
 // Warps: 0 TMA producer (Q once, K and V chunks in separate rings), 1 TMEM
 // allocation + MMA issue (QK of chunk j+1 overlaps the softmax of chunk j),
-// 2-5 softmax / output.  Prefix chunks are laid out backwards from the
+// 2-5 softmax / output.  Contiguous prefix chunks are laid backwards from the
 // sequence's prefix end, so no cache slot at or past prefix_len is ever read
-// (the first chunk may reach before the split's start: those keys are
-// finite cache entries or zero-filled, and masked).  Tree keys are masked
-// with each row's ancestor bitmask.  Each CTA writes its normalised partial
-// output and log-sum-exp; a combine kernel merges the splits.  Every wait
-// is bounded (~2 s) and sets MEDUSA_STATUS_TIMEOUT on expiry.
+// (the first chunk may start before position 0: TMA zero-fills those rows,
+// and they are masked); paged prefix chunks are page-aligned from position 0.
+// Tree keys are masked with each row's ancestor bitmask.
+// With C = 1 the softmax threads write the bf16 output rows directly.  With
+// C > 1 every CTA parks its normalised partial rows and their log-sum-exps in
+// its own shared memory (over the drained K/V rings); after a cluster barrier
+// each CTA merges every C-th row of the tile from all C partials, read
+// through distributed shared memory in split order (so the result does not
+// depend on which CTA merges), and a second cluster barrier keeps every CTA's
+// shared memory alive until its peers have read it.  Every pipeline wait is
+// bounded (~2 s) and sets MEDUSA_STATUS_TIMEOUT on expiry.
+#include <cooperative_groups.h>
 #include <limits.h>
 
 #include "kernels.h"
@@ -51,6 +60,10 @@ template <int D> constexpr int k_stages() { return D == 128 ? 3 : 4; }
 template <int D> constexpr int v_stages() { return D == 128 ? 2 : 4; }
 template <int D> constexpr int n_bars() { return 1 + 2 * k_stages<D>() + 2 * v_stages<D>() + 6; }
 constexpr int kPageRing = 8 * 8 * 4;  // bytes of the page-id ring (8 chunks x 8 boxes)
+constexpr int kMaxCluster = 8;        // key splits per tile: a portable cluster size
+// floats per row of a parked partial (D + 4: 16-byte row accesses of
+// consecutive rows fall on distinct banks)
+template <int D> constexpr int o_stride() { return D + 4; }
 
 struct TcAttnArgs {
     CUtensorMap mq;    // q as (D, Hq, B*T), box (64, G, 128/G)
@@ -62,10 +75,10 @@ struct TcAttnArgs {
     TreeRef tree;
     const int32_t* block_table;  // NULL: contiguous caches
     int max_pages, page_size, num_pages, page_rows;  // page_rows = min(page_size, 64) rows per TMA box
-    float* part_o;     // [n_splits][B*Hkv][R][D]
-    float* part_lse;   // [n_splits][B*Hkv][R], log2 units
+    __nv_bfloat16* out;  // [B, T, Hq, D]
+    float* lse;          // [B, T, Hq], natural log; nullable
     int32_t* status;
-    int B, T, Hq, Hkv, G, S_max, max_prefix, R, n_splits, split_len;
+    int B, T, Hq, Hkv, G, S_max, max_prefix;
     int tree_in_cache;  // the tree's K/V are cache rows prefix_len .. prefix_len + T_b (contiguous caches)
     float scale_log2;
 };
@@ -83,6 +96,11 @@ __device__ __forceinline__ float fast_exp2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+__device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
 }
 
 // descriptor of an MN-major operand stored as TMA writes a (64 MN x rows K)
@@ -132,13 +150,14 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
     // paged: the page of each box of the last 8 K chunks, for their V loads
     int* pg_ring = reinterpret_cast<int*>(tmem_slot + 4);  // [8][8]
 
-    const int mt = blockIdx.x, bg = blockIdx.y, split = blockIdx.z;
+    namespace cg = cooperative_groups;
+    const int mt = blockIdx.x, bg = blockIdx.y;
+    const int C = (int)gridDim.z, split = blockIdx.z;  // the key splits of a tile form one cluster
     const int b = bg / a.Hkv, g = bg % a.Hkv;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const bool tree_split = split == a.n_splits - 1;
     const TreeDev* tree = a.tree.at(b);
-    const int Tb = tree->T;  // this sequence's tree (a.T: the row stride of q and the tree K/V)
-    if (smem_addr(smem) & 1023u) {  // never expected; refuse rather than misread swizzled tiles
+    const int Tb = tree->T;  // this sequence's tree (a.T: the row stride of q, out and the tree K/V)
+    if (smem_addr(smem) & 1023u) {  // never expected (uniform over the grid); refuse rather than misread tiles
         if (threadIdx.x == 0) set_status(a.status, MEDUSA_STATUS_TIMEOUT);
         return;
     }
@@ -149,24 +168,20 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
         if (threadIdx.x == 0 && split == 0 && mt == 0 && g == 0) set_status(a.status, MEDUSA_STATUS_BAD_PREFIX);
         S = S < 0 ? 0 : a.max_prefix;
     }
-    int k_begin, k_end, nc;
-    if (tree_split) {
-        k_begin = 0;
-        k_end = Tb;
-        nc = (Tb + kCh - 1) / kCh;
-    } else {
-        k_begin = split * a.split_len;
-        k_end = min(S, k_begin + a.split_len);
-        nc = k_end > k_begin ? (k_end - k_begin + kCh - 1) / kCh : 0;
-    }
-    // first key of chunk j: contiguous prefix chunks end exactly at k_end (no
-    // slot past the prefix is read); paged ones start at page-aligned k_begin
     const bool paged = a.block_table != nullptr;
-    auto chunk_start = [&](int j) {
-        return tree_split ? j * kCh : paged ? k_begin + j * kCh : k_end - (nc - j) * kCh;
+    // the sequence's chunks: nP prefix chunks, then nT tree chunks; this split
+    // takes chunks [c0, c0 + nc) of them
+    const int nP = (S + kCh - 1) / kCh, nT = (Tb + kCh - 1) / kCh, N = nP + nT;
+    const int c0 = (int)((long)N * split / C);
+    const int nc = (int)((long)N * (split + 1) / C) - c0;
+    auto is_tree = [&](int j) { return c0 + j >= nP; };
+    // first key of chunk j: a prefix position (contiguous chunks end exactly at
+    // S, the first one may start below 0; paged ones start at multiples of 64)
+    // or, for a tree chunk, a node index
+    auto chunk_key0 = [&](int j) {
+        const int c = c0 + j;
+        return c >= nP ? (c - nP) * kCh : paged ? c * kCh : S - (nP - c) * kCh;
     };
-    // keys past key_end are not the sequence's (their rows are cleared in V)
-    const int key_end = tree_split ? Tb : k_end;
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
@@ -192,6 +207,13 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
+    // the softmax threads' row: its final (unnormalised) O, max m and sum l
+    const int lr = (warp & 3) * 32 + lane;   // TMEM lane = tile row of a softmax thread
+    const int rrow = mt * kAM + lr;          // row within the (sequence, kv-head)
+    const bool row_ok = warp >= 2 && rrow < Tb * a.G;
+    float o[D];
+    float m = -INFINITY, l = 0.f;
+
     if (warp == 0) {
         // ---------------- producer ----------------
         // K chunks run ahead of V chunks; each is loaded as soon as its ring
@@ -202,35 +224,36 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
 #pragma unroll
             for (int sub = 0; sub < NSUB; ++sub)
                 tma_load_3d(sQ + sub * (kAM * 128), &a.mq, sub * 64, g * a.G, b * a.T + mt * NB, q_full);
-            // Paged: the page of every box (page_rows keys) of a chunk, copied
-            // asynchronously into the chunk's pg_ring slot one chunk ahead (a
-            // K chunk waits only for its own ids; its V chunk reuses them).
-            // Boxes at or past k_end are not loaded (their rows are masked, and
-            // cleared in V); an out-of-range page is skipped and reported.
+            // Paged: the page of every box (page_rows keys) of a prefix chunk,
+            // copied asynchronously into the chunk's pg_ring slot one chunk
+            // ahead (a K chunk waits only for its own ids; its V chunk reuses
+            // them).  Boxes at or past S are not loaded (their rows are masked,
+            // and cleared in V); an out-of-range page is skipped and reported.
             const int pr = paged ? a.page_rows : kCh, nbox = kCh / pr;
             auto fetch_pages = [&](int j) {
-                if (j >= nc) return;
+                if (j >= nc || is_tree(j)) return;
                 int* ring = pg_ring + (j & 7) * 8;
-                const int cs = chunk_start(j);
+                const int cs = chunk_key0(j);
                 for (int i = 0; i < nbox; ++i) {
                     const int pos = cs + i * pr;
-                    if (pos < k_end)
+                    if (pos < S)
                         cp_async4(smem_addr(ring + i), &a.block_table[(long)b * a.max_pages + pos / a.page_size]);
                     else
                         ring[i] = -1;
                 }
                 cp_async_commit();
             };
-            auto issue_chunk = [&](uint8_t* base, const CUtensorMap* mc, const CUtensorMap* mt, uint64_t* bar,
+            auto issue_chunk = [&](uint8_t* base, const CUtensorMap* mc, const CUtensorMap* mtr, uint64_t* bar,
                                    int j, bool is_k) {
-                const int cs = chunk_start(j);
-                if (tree_split || !paged) {
+                const int cs = chunk_key0(j);
+                const bool tr = is_tree(j);
+                if (tr || !paged) {
                     mbar_arrive_expect_tx(bar, kKVBytes);
 #pragma unroll
                     for (int sub = 0; sub < NSUB; ++sub) {
-                        if (tree_split && a.tree_in_cache)  // rows S + cs .. of this (sequence, kv-head)
+                        if (tr && a.tree_in_cache)  // rows S + cs .. of this (sequence, kv-head)
                             tma_load_3d(base + sub * kSub, mc, sub * 64, S + cs, bg, bar);
-                        else if (tree_split) tma_load_3d(base + sub * kSub, mt, sub * 64, g, b * a.T + cs, bar);
+                        else if (tr) tma_load_3d(base + sub * kSub, mtr, sub * 64, g, b * a.T + cs, bar);
                         else tma_load_3d(base + sub * kSub, mc, sub * 64, cs, bg, bar);
                     }
                     return;
@@ -240,7 +263,7 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
                     cp_async_wait_all();  // this chunk's ids (the only group in flight)
                     for (int i = 0; i < nbox; ++i) {
                         const int page = ring[i];
-                        if (page >= a.num_pages || (page < 0 && cs + i * pr < k_end)) {
+                        if (page >= a.num_pages || (page < 0 && cs + i * pr < S)) {
                             set_status(a.status, MEDUSA_STATUS_BAD_PAGE);
                             ring[i] = -1;
                         }
@@ -260,7 +283,7 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
                                     page * a.Hkv + g, bar);
                 }
             };
-            if (paged && !tree_split) fetch_pages(0);
+            if (paged) fetch_pages(0);
             int jk = 0, jv = 0;
             uint64_t t0 = global_ns();
             uint32_t idle = 0;
@@ -287,6 +310,7 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
                 }
             }
             // drain: no copy may still be landing when the CTA exits
+            cp_async_wait_all();
             mbar_wait(q_full, 0);
             for (int s = 0; s < KS && s < jk; ++s) {
                 const int last = s + ((jk - 1 - s) / KS) * KS;
@@ -352,17 +376,13 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
             mbar_wait(o_last, 0);  // every MMA done before TMEM is released (bounded)
         }
     } else {
-        // ---------------- softmax / output ----------------
+        // ---------------- softmax ----------------
         const int q = warp & 3;
-        const int lr = q * 32 + lane;
-        const int r = mt * kAM + lr;
-        const bool row_ok = r < Tb * a.G;
-        const int node = row_ok ? r / a.G : 0;
+        const int node = row_ok ? rrow / a.G : 0;
         uint32_t anc[4] = {0u, 0u, 0u, 0u};
-        if (tree_split && row_ok)
+        if (row_ok && nc > 0 && is_tree(nc - 1))
 #pragma unroll
             for (int w = 0; w < 4; ++w) anc[w] = tree->anc[node][w];
-        float m = -INFINITY, l = 0.f;
         bool ok = true;
         const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
         for (int j = 0; j < nc && ok; ++j) {
@@ -383,15 +403,16 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
                     for (int e = 0; e < 16; ++e) sv[c * 16 + e] = __uint_as_float(raw[c][e]);
             }
             // visible keys of this chunk for this row, bit c = key key0 + c
-            const int key0 = chunk_start(j);
+            const int key0 = chunk_key0(j);
+            const bool tr = is_tree(j);
             uint64_t vis;
-            if (tree_split) {
+            if (tr) {
                 // ancestor bits (keys >= T have none); key0 is 0 or 64
                 vis = key0 == 0 ? ((uint64_t)anc[1] << 32 | anc[0]) : ((uint64_t)anc[3] << 32 | anc[2]);
             } else {
-                // keys [k_begin, k_end): a contiguous first chunk may reach back
-                // before k_begin, a paged last chunk past k_end
-                const int lo = key0 >= k_begin ? 0 : k_begin - key0, hi = k_end - key0;
+                // prefix keys [0, S): a contiguous first chunk may start below
+                // 0, a paged last chunk may reach past S
+                const int lo = key0 >= 0 ? 0 : -key0, hi = S - key0;
                 vis = lo > 0 ? ~0ull << lo : ~0ull;
                 if (hi < kCh) vis &= (1ull << hi) - 1ull;
             }
@@ -462,6 +483,7 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
                 tmem_wait_st();
             }
             m = mn;
+            const int key_end = tr ? Tb : S;
             if (key0 + kCh > key_end) {
                 // the chunk's rows past this sequence's keys (tree padding,
                 // another sequence's rows, page slots past the prefix, boxes
@@ -487,7 +509,6 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
             if (lane == 0) mbar_arrive(&p_full[j & 1]);
         }
         // final O (after the last PV) for this row
-        float o[D];
         if (ok && nc > 0 && !mbar_wait(o_last, 0)) ok = false;
         if (ok && nc > 0) {
             tc_fence_after();
@@ -507,24 +528,113 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
         } else {
 #pragma unroll
             for (int e = 0; e < D; ++e) o[e] = 0.f;
+            l = 0.f;
         }
         if (!ok && lane == 0) set_status(a.status, MEDUSA_STATUS_TIMEOUT);
-        if (row_ok) {
-            const long BH = (long)a.B * a.Hkv;
-            const float inv = l > 0.f ? 1.f / l : 0.f;
-            float* dst = a.part_o + (((long)split * BH + bg) * a.R + r) * D;
+        if (!row_ok) {  // a row past this sequence's tree (or the tile): zero
 #pragma unroll
-            for (int e = 0; e < D; e += 4)
-                *reinterpret_cast<float4*>(dst + e) = make_float4(o[e] * inv, o[e + 1] * inv, o[e + 2] * inv, o[e + 3] * inv);
-            a.part_lse[((long)split * BH + bg) * a.R + r] = l > 0.f ? m + log2f(l) : -INFINITY;
+            for (int e = 0; e < D; ++e) o[e] = 0.f;
+            l = 0.f;
         }
     }
+    // every role is done: no MMA in flight, no copy landing
     tc_fence_before();
     sync_block();
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
+    const int rows_T = a.T * a.G;   // rows of the (sequence, kv-head) in the output (past Tb * G: zeros)
+    // output row r of this (sequence, kv-head): (node, q-head) = (r / G, g * G + r % G)
+    auto out_row = [&](int r) -> long { return ((long)b * a.T + r / a.G) * a.Hq + g * a.G + r % a.G; };
+    if (C == 1) {
+        // a single split: this CTA's rows are final
+        if (warp >= 2 && rrow < rows_T) {
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            const long orow = out_row(rrow);
+            uint4* dst = reinterpret_cast<uint4*>(a.out + orow * D);
+#pragma unroll
+            for (int e = 0; e < D; e += 8) {
+                uint4 v;
+                v.x = pack2_bf16(o[e] * inv, o[e + 1] * inv);
+                v.y = pack2_bf16(o[e + 2] * inv, o[e + 3] * inv);
+                v.z = pack2_bf16(o[e + 4] * inv, o[e + 5] * inv);
+                v.w = pack2_bf16(o[e + 6] * inv, o[e + 7] * inv);
+                dst[e / 8] = v;
+            }
+            if (a.lse) a.lse[orow] = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
+        }
+        return;
+    }
+    // ---- several splits: park the normalised partials, merge over the cluster ----
+    constexpr int OS = o_stride<D>();
+    float* sO = reinterpret_cast<float*>(sK);  // [kAM][OS] over the drained K/V rings
+    float* sL = reinterpret_cast<float*>(sQ);  // [kAM] over Q (no QK is pending)
+    if (warp >= 2) {
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        float* dst = sO + lr * OS;
+#pragma unroll
+        for (int e = 0; e < D; e += 4)
+            *reinterpret_cast<float4*>(dst + e) = make_float4(o[e] * inv, o[e + 1] * inv, o[e + 2] * inv, o[e + 3] * inv);
+        sL[lr] = l > 0.f ? m + log2f(l) : -INFINITY;
+    }
+    cg::cluster_group cl = cg::this_cluster();
+    __syncwarp();  // the cluster barrier is an aligned one: whole warps
+    cl.sync();     // every split's partials are parked
+    constexpr int PL = D / 32;  // elements of a row per lane
+    const int nrows = min(kAM, rows_T - mt * kAM);
+    for (int r = split + C * warp; r < nrows; r += C * kAW) {
+        const long orow = out_row(mt * kAM + r);
+        __nv_bfloat16* dst = a.out + orow * D + lane * PL;
+        if (mt * kAM + r >= Tb * a.G) {  // past this sequence's tree: zero output
+#pragma unroll
+            for (int e = 0; e < PL; ++e) dst[e] = __float2bfloat16_rn(0.f);
+            if (a.lse && lane == 0) a.lse[orow] = -INFINITY;
+            continue;
+        }
+        const float ls = lane < C ? *cl.map_shared_rank(sL + r, lane) : -INFINITY;
+        float M = ls;
+#pragma unroll
+        for (int o2 = 16; o2 > 0; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o2));
+        const float wl = ls == -INFINITY ? 0.f : exp2f(ls - M);
+        float part[kMaxCluster][PL];
+#pragma unroll
+        for (int s = 0; s < kMaxCluster; ++s) {  // every load issued before any is used
+            if (s < C) {
+                const float* src = cl.map_shared_rank(sO, s) + r * OS + lane * PL;
+                if constexpr (PL == 4) {
+                    const float4 v = *reinterpret_cast<const float4*>(src);
+                    part[s][0] = v.x;
+                    part[s][1] = v.y;
+                    part[s][2] = v.z;
+                    part[s][3] = v.w;
+                } else {
+                    const float2 v = *reinterpret_cast<const float2*>(src);
+                    part[s][0] = v.x;
+                    part[s][1] = v.y;
+                }
+            }
+        }
+        float acc[PL], wsum = 0.f;
+#pragma unroll
+        for (int e = 0; e < PL; ++e) acc[e] = 0.f;
+#pragma unroll
+        for (int s = 0; s < kMaxCluster; ++s) {  // in split order
+            const float ws = __shfl_sync(kFull, wl, s);
+            if (s < C && ws > 0.f) {
+                wsum += ws;
+#pragma unroll
+                for (int e = 0; e < PL; ++e) acc[e] = fmaf(ws, part[s][e], acc[e]);
+            }
+        }
+        const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+#pragma unroll
+        for (int e = 0; e < PL; e += 2)
+            *reinterpret_cast<uint32_t*>(dst + e) = pack2_bf16(acc[e] * inv, acc[e + 1] * inv);
+        if (a.lse && lane == 0) a.lse[orow] = wsum > 0.f ? (M + log2f(wsum)) * 0.69314718055994531f : -INFINITY;
+    }
+    __syncwarp();
+    cl.sync();  // the peers are done reading this CTA's shared memory
 }
 
 template <int D>
@@ -533,6 +643,9 @@ size_t tc_attn_smem() {
     return (size_t)kAM * D * 2 + (size_t)(k_stages<D>() + v_stages<D>()) * kCh * D * 2 + n_bars<D>() * 8 + 16 +
            kPageRing;
 }
+// the parked partials fit over the rings, their log-sum-exps over Q
+static_assert(kAM * o_stride<128>() * 4 <= (k_stages<128>() + v_stages<128>()) * kCh * 128 * 2, "partials (D=128)");
+static_assert(kAM * o_stride<64>() * 4 <= (k_stages<64>() + v_stages<64>()) * kCh * 64 * 2, "partials (D=64)");
 
 }  // namespace
 
@@ -547,13 +660,27 @@ bool attn_tc_supported(int Hq, int Hkv, int D, int T, medusa_dtype dt) {
     return dt == MEDUSA_BF16 && (D == 64 || D == 128) && G >= 1 && G <= 16 && (G & (G - 1)) == 0 && T <= kMaxTree;
 }
 
-// launch the tensor-core split kernel; the caller provides the split plan and
-// the partial buffers (same layout as the other bf16 path) and runs the combine
-cudaError_t attn_tc_launch(const AttnArgs& x, int m_tiles, int n_splits, int split_len, float scale_log2,
-                           float* part_o, float* part_lse, cudaStream_t st) {
+// Key splits per 128-row tile: enough CTAs for two per SM, at most a portable
+// cluster and at most the chunks of the longest sequence.
+int attn_tc_splits(int B, int T, int Hq, int Hkv, int max_prefix) {
+    const int G = Hq / Hkv;
+    const long m_tiles = ((long)T * G + kAM - 1) / kAM;
+    const long per_split = m_tiles * B * Hkv;
+    const long target = (long)kCtasPerSm * num_sms();
+    long c = (target + per_split - 1) / per_split;
+    const long chunks = (max_prefix + kCh - 1) / kCh + (T + kCh - 1) / kCh;
+    if (c > kMaxCluster) c = kMaxCluster;
+    if (c > chunks) c = chunks;
+    return c < 1 ? 1 : (int)c;
+}
+
+// launch the tensor-core kernel: m_tiles 128-row tiles per (sequence, kv-head),
+// n_splits key splits per tile (one cluster); writes the output (and lse)
+cudaError_t attn_tc_launch(const AttnArgs& x, int m_tiles, int n_splits, float scale_log2, cudaStream_t st) {
     TcAttnArgs a;
     const uint64_t D = x.D, Hq = x.Hq, Hkv = x.Hkv, BT = (uint64_t)x.B * x.T, Smax = x.S_max, BH = (uint64_t)x.B * x.Hkv;
     const int G = x.Hq / x.Hkv;
+    if (n_splits < 1 || n_splits > kMaxCluster) return cudaErrorInvalidValue;
     {
         const uint64_t dims[3] = {D, Hq, BT}, strides[2] = {D * 2, Hq * D * 2};
         const uint32_t box[3] = {64, (uint32_t)G, (uint32_t)(kAM / G)};
@@ -588,8 +715,8 @@ cudaError_t attn_tc_launch(const AttnArgs& x, int m_tiles, int n_splits, int spl
     }
     a.prefix_len = x.prefix_len;
     a.tree = x.tree;
-    a.part_o = part_o;
-    a.part_lse = part_lse;
+    a.out = (__nv_bfloat16*)x.out;
+    a.lse = x.lse;
     a.status = x.status;
     a.B = x.B;
     a.T = x.T;
@@ -598,23 +725,30 @@ cudaError_t attn_tc_launch(const AttnArgs& x, int m_tiles, int n_splits, int spl
     a.G = G;
     a.S_max = x.S_max;
     a.max_prefix = x.max_prefix;
-    a.R = x.T * G;
-    a.n_splits = n_splits;
-    a.split_len = split_len;
     a.scale_log2 = scale_log2;
-    const dim3 grid(m_tiles, (unsigned)BH, n_splits);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(m_tiles, (unsigned)BH, n_splits);
+    cfg.blockDim = dim3(kAW * 32);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = n_splits;
+    cfg.attrs = attr;
+    cfg.numAttrs = n_splits > 1 ? 1 : 0;
     if (x.D == 128) {
-        const size_t smem = tc_attn_smem<128>();
-        cudaFuncSetAttribute(tree_attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cfg.dynamicSmemBytes = tc_attn_smem<128>();
+        cudaFuncSetAttribute(tree_attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)cfg.dynamicSmemBytes);
         cudaFuncSetAttribute(tree_attn_tc_kernel<128>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-        tree_attn_tc_kernel<128><<<grid, kAW * 32, smem, st>>>(a);
-    } else {
-        const size_t smem = tc_attn_smem<64>();
-        cudaFuncSetAttribute(tree_attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        cudaFuncSetAttribute(tree_attn_tc_kernel<64>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-        tree_attn_tc_kernel<64><<<grid, kAW * 32, smem, st>>>(a);
+        return cudaLaunchKernelEx(&cfg, tree_attn_tc_kernel<128>, a);
     }
-    return cudaGetLastError();
+    cfg.dynamicSmemBytes = tc_attn_smem<64>();
+    cudaFuncSetAttribute(tree_attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)cfg.dynamicSmemBytes);
+    cudaFuncSetAttribute(tree_attn_tc_kernel<64>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    return cudaLaunchKernelEx(&cfg, tree_attn_tc_kernel<64>, a);
 }
 
 }  // namespace medusa

@@ -74,8 +74,10 @@ bool attn_tc_supported(int Hq, int Hkv, int D, int T, medusa_dtype dt);
 int attn_tc_ctas_per_sm();
 // page sizes the tensor-core kernel reads (multiples of 64, or 8, 16, 32)
 bool attn_tc_page_ok(int page_size);
-cudaError_t attn_tc_launch(const AttnArgs& a, int m_tiles, int n_splits, int split_len, float scale_log2,
-                           float* part_o, float* part_lse, cudaStream_t st);
+// key splits per 128-row tile (the CTAs of one cluster, at most 8)
+int attn_tc_splits(int B, int T, int Hq, int Hkv, int max_prefix);
+// writes the output (and lse) itself: the splits merge inside their cluster
+cudaError_t attn_tc_launch(const AttnArgs& a, int m_tiles, int n_splits, float scale_log2, cudaStream_t st);
 
 // ------------------------------- verify ------------------------------------
 struct VerifyArgs {
@@ -123,6 +125,10 @@ struct CommitArgs {
     int32_t* status;
 };
 cudaError_t commit_launch(const CommitArgs& a, cudaStream_t st);
+// greedy verification's walk (VerifyArgs as for verify_greedy_walk_launch)
+// followed, in the same block per sequence, by the commit of the path it found
+// (CommitArgs as for commit_launch; its path, length and T come from the walk)
+cudaError_t verify_greedy_walk_commit_launch(const VerifyArgs& a, const CommitArgs& c, cudaStream_t st);
 
 // in-place compaction of the tree rows after each prefix, every layer at once
 struct CompactArgs {

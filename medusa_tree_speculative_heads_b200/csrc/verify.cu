@@ -31,7 +31,9 @@
 // size) differ from a sequential evaluation only in the last bits of P.
 #include <cooperative_groups.h>
 #include <limits.h>
+#include <string.h>
 
+#include "commit_common.cuh"
 #include "kernels.h"
 
 namespace medusa {
@@ -121,13 +123,28 @@ __global__ void __launch_bounds__(kArgmaxThreads, 4) row_argmax_kernel(const E* 
 // node (lowest index among equally deep ones) ends the path, whose nodes are
 // the set bits of its ancestor mask in increasing index order (a parent's
 // index is below its child's).
+// With a commit (kc != NULL) the same block then appends the accepted path's
+// K/V to the sequence's cache, as kv_commit does.
+struct WalkCommit {
+    uint8_t* kc;  // NULL: no commit
+    uint8_t* vc;
+    const uint8_t* kt;
+    const uint8_t* vt;
+    const int32_t* prefix_len;
+    int32_t* new_prefix_len;
+    int Hkv, S_max, row_bytes;
+    const int32_t* table;  // NULL: contiguous cache
+    int max_pages, page_size, num_pages;
+    int32_t* status;
+};
 constexpr int kWalkThreads = kMaxTree;
 constexpr int kMaxSplits = 16;
 __global__ void __launch_bounds__(kWalkThreads) greedy_walk_kernel(const float* __restrict__ pval,
                                                                    const int* __restrict__ pidx, int splits,
                                                                    const int32_t* __restrict__ node_tokens,
                                                                    TreeRef trees, int32_t* accept_path, int max_path,
-                                                                   int32_t* accept_len, int32_t* bonus) {
+                                                                   int32_t* accept_len, int32_t* bonus,
+                                                                   const WalkCommit cm) {
     __shared__ int pred[kMaxTree];
     __shared__ uint32_t match[kMaxTree / 32];
     __shared__ int best_key[kMaxTree / 32];
@@ -181,6 +198,12 @@ __global__ void __launch_bounds__(kWalkThreads) greedy_walk_kernel(const float* 
         for (int j = L; j < max_path; ++j) accept_path[(long)b * max_path + j] = -1;
         accept_len[b] = L;
         bonus[b] = pred[best];
+    }
+    if (cm.kc) {
+        __syncthreads();  // the path thread 0 wrote is visible to the block
+        commit_sequence(b, cm.kc, cm.vc, cm.kt, cm.vt, accept_path, max_path, accept_len, cm.prefix_len,
+                        cm.new_prefix_len, Tn, cm.Hkv, cm.S_max, cm.row_bytes, cm.table, cm.max_pages, cm.page_size,
+                        cm.num_pages, cm.status);
     }
 }
 
@@ -533,16 +556,41 @@ cudaError_t verify_greedy_rows_launch(const VerifyArgs& a, cudaStream_t st) {
     return cudaGetLastError();
 }
 
-// greedy: the tree walk over those partials
-cudaError_t verify_greedy_walk_launch(const VerifyArgs& a, cudaStream_t st) {
+// greedy: the tree walk over those partials, optionally followed by the commit
+static cudaError_t walk_launch(const VerifyArgs& a, const WalkCommit& cm, cudaStream_t st) {
     const int rows = a.B * a.T;
     const int splits = argmax_splits(rows, a.V);
     const float* pval = (const float*)a.ws;
     const int* pidx = (const int*)((const char*)a.ws + align256((size_t)rows * splits * sizeof(float)));
     prefer_max_smem(greedy_walk_kernel);
     greedy_walk_kernel<<<a.B, kWalkThreads, 0, st>>>(pval, pidx, splits, a.node_tokens, a.tree, a.accept_path,
-                                                     a.max_path, a.accept_len, a.bonus);
+                                                     a.max_path, a.accept_len, a.bonus, cm);
     return cudaGetLastError();
+}
+
+cudaError_t verify_greedy_walk_launch(const VerifyArgs& a, cudaStream_t st) {
+    WalkCommit cm;
+    memset(&cm, 0, sizeof cm);
+    return walk_launch(a, cm, st);
+}
+
+cudaError_t verify_greedy_walk_commit_launch(const VerifyArgs& a, const CommitArgs& c, cudaStream_t st) {
+    WalkCommit cm;
+    cm.kc = (uint8_t*)c.k_cache;
+    cm.vc = (uint8_t*)c.v_cache;
+    cm.kt = (const uint8_t*)c.k_tree;
+    cm.vt = (const uint8_t*)c.v_tree;
+    cm.prefix_len = c.prefix_len;
+    cm.new_prefix_len = c.new_prefix_len;
+    cm.Hkv = c.Hkv;
+    cm.S_max = c.S_max;
+    cm.row_bytes = c.D * c.esize;
+    cm.table = c.block_table;
+    cm.max_pages = c.max_pages;
+    cm.page_size = c.page_size;
+    cm.num_pages = c.num_pages;
+    cm.status = c.status;
+    return walk_launch(a, cm, st);
 }
 
 cudaError_t verify_launch(const VerifyArgs& a, cudaStream_t st) {

@@ -173,6 +173,17 @@ def test_newer_calls_validate_before_launch(lib):
     assert lib.tree_verify_greedy_rows(fake, 5, 1, 100, nul, fake, 1 << 20, nul) == UNS
     assert lib.tree_verify_greedy_walk(nul, 1, 100, nul, fake, 4, fake, fake, fake, 1 << 20, nul) == INV
     assert lib.tree_verify_greedy_walk(fake, 1, 100, nul, fake, 4, fake, fake, fake, 1 << 20, nul) == INV
+    # the walk with its commit: NULL cache arguments, then a missing tree
+    wc = lib.tree_verify_greedy_walk_commit
+    wc.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                   ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
+                   ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                   ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                   ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
+    assert wc(fake, 1, 100, nul, fake, 4, fake, fake, fake, 1 << 20, nul, fake, fake, fake, fake, fake, 8, 128, 256,
+              nul, 0, 0, 0, 1, nul, nul) == INV
+    assert wc(fake, 1, 100, nul, fake, 4, fake, fake, fake, 1 << 20, fake, fake, fake, fake, fake, fake, 8, 128, 256,
+              nul, 0, 0, 0, 1, nul, nul) == INV                                       # tree NULL
     assert lib.tree_attention_incache_workspace_size(1, 4, 2, 96, 256, 0, nul, 1) == 0
 
 

@@ -43,11 +43,13 @@ def test_bench_defaults_and_config_keys():
 
 
 def test_bench_counts_the_library_launches_of_a_step():
-    # the kernels one step launches (the launch list in profiles/ shows six at llama8b)
+    # the kernels one step launches (the launch list in profiles/ shows four at llama8b)
     b = _bench()
     from medusa_tree_speculative_heads_b200 import inputs as I
     W = I.WORKLOADS
-    assert b.launches_per_step(W["llama8b"]) == 6       # heads, attention + combine, argmax + walk, commit
-    assert b.launches_per_step(W["stoch_b64"]) == 5     # one stochastic verify kernel
-    assert b.launches_per_step(W["tiny"]) == 1 + 1 + 2 + 1   # fp32: fused heads, one attention kernel
+    assert b.launches_per_step(W["llama8b"]) == 4       # heads, attention, argmax, walk + commit
+    assert b.launches_per_step(W["stoch_b64"]) == 4     # heads, attention, stochastic verify, commit
+    assert b.launches_per_step(W["tiny"]) == 4          # fp32: fused heads, one attention kernel, argmax, walk + commit
+    assert b.launches_per_step(W["llama8b_incache"]) == 5   # the walk without commit, then the compaction
+    assert b.launches_per_step(I.scaled(W["llama8b"], Hq=24)) == 5   # G = 3: the mma.sync kernel and its combine
     assert b._is_anc([-1, 0, 1, 0], 2, 0) and b._is_anc([-1, 0, 1, 0], 2, 2) and not b._is_anc([-1, 0, 1, 0], 3, 1)

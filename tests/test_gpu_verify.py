@@ -281,3 +281,57 @@ def test_greedy_equally_deep_accepted_nodes(dtype):
     lg = torch.from_numpy(logits).to(dtype)
     out = run_greedy(parents, torch.from_numpy(tok), lg)
     assert_same(out, oracle.verify_greedy(lg, tok, parents, max_path=4))
+
+
+@pytest.mark.parametrize("paged", [False, True])
+def test_greedy_walk_with_commit_equals_walk_then_commit(paged):
+    # the fused walk + commit launch gives exactly the walk followed by
+    # kv_commit (kv_commit_paged), including a sequence whose cache is full
+    from medusa_tree_speculative_heads_b200.api import kv_commit, kv_commit_paged
+    w = I.scaled(I.WORKLOADS["llama8b"], B=4, V=3000, Hkv=2, prefix=40)
+    parents = I.workload_tree(w)
+    tok, logits = greedy_case(w, parents)
+    tree = Tree(parents)
+    T = len(parents)
+    lg, tk = logits.cuda(), tok.cuda()
+    nb = B.tree_verify_workspace_size(B.GREEDY, w.B, w.V, tree)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    B.tree_verify_greedy_rows(lg, B.dtype_code(lg.dtype), w.B, w.V, tree, ws, nb)
+    ain = I.attention_inputs(w, T)
+    pl = torch.tensor([0, 17, 40, w.S_max], dtype=torch.int32)          # the last cache is full
+    pc = I.paged_cache(w, 16, pl, room=4) if paged else None
+    if paged:
+        pc["block_table"][3, int(pl[3]) // 16:] = -1                        # and owns no page past its prefix
+
+    def caches():
+        if paged:
+            return pc["k_pages"].clone().cuda(), pc["v_pages"].clone().cuda()
+        return ain["k_cache"].clone().cuda(), ain["v_cache"].clone().cuda()
+
+    kt, vt, table = ain["k_tree"].cuda(), ain["v_tree"].cuda(), pc["block_table"].cuda() if paged else None
+    # reference: the walk, then the separate commit
+    path = torch.empty((w.B, tree.max_depth), dtype=torch.int32, device="cuda")
+    ln = torch.empty(w.B, dtype=torch.int32, device="cuda")
+    bonus = torch.empty(w.B, dtype=torch.int32, device="cuda")
+    B.tree_verify_greedy_walk(tk, w.B, w.V, tree, path, tree.max_depth, ln, bonus, ws, nb)
+    kc1, vc1 = caches()
+    if paged:
+        r1 = kv_commit_paged(kc1, vc1, kt, vt, table, path, ln, pl.cuda())
+    else:
+        r1 = kv_commit(kc1, vc1, kt, vt, path, ln, pl.cuda())
+    # fused
+    kc2, vc2 = caches()
+    path2, ln2, bonus2 = torch.full_like(path, -7), torch.full_like(ln, -7), torch.full_like(bonus, -7)
+    npl2 = torch.full_like(ln, -7)
+    st2 = torch.zeros(1, dtype=torch.int32, device="cuda")
+    S_max = kc2.shape[2] if not paged else 0
+    B.tree_verify_greedy_walk_commit(tk, w.B, w.V, tree, path2, tree.max_depth, ln2, bonus2, ws, nb, kc2, vc2, kt,
+                                     vt, pl.cuda(), npl2, w.Hkv, w.D, S_max, table,
+                                     table.shape[1] if paged else 0, 16 if paged else 0,
+                                     kc2.shape[0] if paged else 0, B.dtype_code(kc2.dtype), st2)
+    torch.cuda.synchronize()
+    assert torch.equal(path2, path) and torch.equal(ln2, ln) and torch.equal(bonus2, bonus)
+    assert torch.equal(npl2, r1["new_prefix_len"]) and torch.equal(st2, r1["status"])
+    assert int(st2.item()) == B.STATUS_CACHE_OVERFLOW
+    assert torch.equal(kc2, kc1) and torch.equal(vc2, vc1)
+    assert int(npl2[3]) == int(pl[3])          # the overflowing sequence was not committed
