@@ -78,7 +78,8 @@ enum {
     MEDUSA_STATUS_CACHE_OVERFLOW = 2, /* kv_commit: prefix_len + len > S_max */
     MEDUSA_STATUS_BAD_PREFIX = 4,     /* prefix_len outside [0, max_prefix] */
     MEDUSA_STATUS_NO_MASS = 8,        /* stochastic bonus drawn from an all-zero distribution */
-    MEDUSA_STATUS_TIMEOUT = 16,       /* an internal pipeline wait gave up after ~2 s (a library bug) */
+    MEDUSA_STATUS_TIMEOUT = 16,       /* an internal pipeline wait gave up after ~2 s (a library bug), or after
+                                         the limit set by medusa_debug_set_wait_limit */
     MEDUSA_STATUS_BAD_PAGE = 32,      /* a needed block-table entry outside [0, num_pages) */
     MEDUSA_STATUS_BAD_LAYER = 64      /* kv_compact: a layer's cache pointer is NULL or not 16-byte aligned */
 };
@@ -95,6 +96,20 @@ const char* medusa_last_error(void);
 
 /* ABI version (major * 100 + minor). */
 int medusa_version(void);
+
+/*
+ * Error-path testing aid (not part of the method).  Every pipeline wait in
+ * the bf16 heads and tree attention kernels (a stage's copy, an MMA, a
+ * hand-over flag, a grid barrier) gives up after a limit, sets
+ * MEDUSA_STATUS_TIMEOUT in the call's status word and lets the kernel finish
+ * without hanging the GPU.  This sets that limit for calls launched
+ * afterwards, process-wide: ns = 0 restores the default (about two seconds);
+ * ns = 1 makes a wait give up at once unless already satisfied, so those
+ * calls end with MEDUSA_STATUS_TIMEOUT and meaningless outputs.  Waits for
+ * copies and MMAs a kernel has already issued always keep the default limit,
+ * so no kernel exits with work of its own in flight.
+ */
+void medusa_debug_set_wait_limit(uint64_t ns);
 
 /* ------------------------------------------------------------------------ */
 /* Candidate tree                                                            */

@@ -60,6 +60,8 @@ def lib() -> ctypes.CDLL:
         L.medusa_last_error.restype = ctypes.c_char_p
         L.medusa_last_error.argtypes = []
         L.medusa_version.restype = i32
+        L.medusa_debug_set_wait_limit.argtypes = [u64]
+        L.medusa_debug_set_wait_limit.restype = None
         L.medusa_tree_create.argtypes = [vp, i32, ctypes.POINTER(vp)]
         L.medusa_tree_destroy.argtypes = [vp]
         L.medusa_tree_info.argtypes = [vp, vp, vp, vp]
@@ -140,6 +142,12 @@ def dtype_code(t: torch.dtype) -> int:
 
 def version() -> int:
     return lib().medusa_version()
+
+
+def set_wait_limit(ns: int) -> None:
+    """medusa_debug_set_wait_limit: limit of the kernels' pipeline waits for
+    later calls (0: the default of about two seconds; 1: give up at once)."""
+    lib().medusa_debug_set_wait_limit(ctypes.c_uint64(int(ns)))
 
 
 class Tree:

@@ -1,6 +1,7 @@
 // C ABI of libmedusa: argument validation, the candidate-tree handle,
 // workspace queries and launches.  See include/medusa.h for the contract of
 // every entry point.
+#include <atomic>
 #include <cmath>
 #include <limits.h>
 #include <stdarg.h>
@@ -133,6 +134,15 @@ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 // lets other translation units set this thread's last-error message
 int report_error(int code, const char* msg) { return fail(code, "%s", msg); }
 
+namespace {
+std::atomic<uint64_t> g_wait_limit{0};  // 0: kWaitLimitNs
+}  // namespace
+
+uint64_t wait_limit_ns() {
+    const uint64_t v = g_wait_limit.load(std::memory_order_relaxed);
+    return v ? v : kWaitLimitNs;
+}
+
 int num_sms() {
     static int cache[64] = {0};
     int dev = 0;
@@ -153,6 +163,8 @@ using namespace medusa;
 extern "C" const char* medusa_last_error(void) { return g_err.c_str(); }
 
 extern "C" int medusa_version(void) { return 100; }
+
+extern "C" void medusa_debug_set_wait_limit(uint64_t ns) { g_wait_limit.store(ns, std::memory_order_relaxed); }
 
 // ---------------------------------------------------------------------------
 // tree handle

@@ -432,19 +432,52 @@ __global__ void __launch_bounds__(256) tree_attn_f32_kernel(const float* __restr
         for (int e = 0; e < PL; ++e) o[e] = o[e] * a + w * vp[lane * PL + e];
         m = mn;
     };
-    if (table) {
-        for (int j = 0; j < S; ++j) {
-            const int page = table[(long)b * max_pages + j / page_size];
-            if (page < 0 || page >= num_pages) {
-                if (lane == 0) set_status(status, MEDUSA_STATUS_BAD_PAGE);
-                continue;
+    // prefix keys in order, their K/V rows loaded 8 at a time ahead of use
+    // (the same per-key arithmetic as visit(), so the same result)
+    constexpr int kU = 8;
+    const long cbase = ((long)b * Hkv + g) * S_max;
+    for (int j0 = 0; j0 < S; j0 += kU) {
+        float kr[kU][PL], vr[kU][PL];
+        bool have[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const int j = j0 + u;
+            long row = -1;
+            if (j < S) {
+                if (table) {
+                    const int page = table[(long)b * max_pages + j / page_size];
+                    if (page >= 0 && page < num_pages) row = ((long)page * Hkv + g) * page_size + j % page_size;
+                    else if (lane == 0) set_status(status, MEDUSA_STATUS_BAD_PAGE);
+                } else {
+                    row = cbase + j;
+                }
             }
-            const long row = ((long)page * Hkv + g) * page_size + j % page_size;
-            visit(k_cache + row * D, v_cache + row * D);
+            have[u] = row >= 0;
+#pragma unroll
+            for (int e = 0; e < PL; ++e) {
+                kr[u][e] = have[u] ? k_cache[row * D + lane * PL + e] : 0.f;
+                vr[u][e] = have[u] ? v_cache[row * D + lane * PL + e] : 0.f;
+            }
         }
-    } else {
-        const long cbase = ((long)b * Hkv + g) * S_max;
-        for (int j = 0; j < S; ++j) visit(k_cache + (cbase + j) * D, v_cache + (cbase + j) * D);
+        float sc[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            float d = 0.f;
+#pragma unroll
+            for (int e = 0; e < PL; ++e) d = fmaf(qv[e], kr[u][e], d);
+            sc[u] = warp_sum(d) * scale;
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            if (!have[u]) continue;
+            const float mn = fmaxf(m, sc[u]);
+            const float a = m == -INFINITY ? 0.f : expf(m - mn);
+            const float w = expf(sc[u] - mn);
+            l = l * a + w;
+#pragma unroll
+            for (int e = 0; e < PL; ++e) o[e] = o[e] * a + w * vr[u][e];
+            m = mn;
+        }
     }
     for (int j = 0; j < tree->T; ++j) {
         if (!((tree->anc[i][j >> 5] >> (j & 31)) & 1u)) continue;

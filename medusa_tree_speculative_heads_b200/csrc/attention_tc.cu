@@ -81,6 +81,7 @@ struct TcAttnArgs {
     int B, T, Hq, Hkv, G, S_max, max_prefix;
     int tree_in_cache;  // the tree's K/V are cache rows prefix_len .. prefix_len + T_b (contiguous caches)
     float scale_log2;
+    uint64_t wait_ns;   // limit of the pipeline waits (drains of issued work: kWaitLimitNs)
 };
 
 // 4-byte asynchronous global -> shared copy (cp.async group semantics)
@@ -304,7 +305,7 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
                 if (prog) {
                     idle = 0;
                     t0 = global_ns();
-                } else if ((++idle & 255u) == 0 && global_ns() - t0 > 2000000000ull) {
+                } else if ((++idle & 255u) == 0 && global_ns() - t0 > a.wait_ns) {
                     set_status(a.status, MEDUSA_STATUS_TIMEOUT);
                     break;
                 }
@@ -324,13 +325,13 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
         if (lane == 0 && nc > 0) {
-            bool ok = mbar_wait(q_full, 0);
+            bool ok = mbar_wait(q_full, 0, a.wait_ns);
             // S_j goes to TMEM columns (j&1)*64; P_j is written over it, so the
             // buffer is free for S_{j+2} once PV_j has completed (o_full phase j)
             auto issue_qk = [&](int j) -> bool {
                 const int s = j % KS, sb = j & 1;
-                if (!mbar_wait(&k_full[s], (j / KS) & 1)) return false;
-                if (j >= 2 && !mbar_wait(o_full, (j - 2) & 1)) return false;
+                if (!mbar_wait(&k_full[s], (j / KS) & 1, a.wait_ns)) return false;
+                if (j >= 2 && !mbar_wait(o_full, (j - 2) & 1, a.wait_ns)) return false;
                 tc_fence_after();
 #pragma unroll
                 for (int sub = 0; sub < NSUB; ++sub) {
@@ -347,12 +348,12 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
             if (ok) ok = issue_qk(0);
             for (int j = 0; j < nc && ok; ++j) {
                 if (j + 1 < nc && !(ok = issue_qk(j + 1))) break;
-                if (!mbar_wait(&p_full[j & 1], (j >> 1) & 1)) {
+                if (!mbar_wait(&p_full[j & 1], (j >> 1) & 1, a.wait_ns)) {
                     ok = false;
                     break;
                 }
                 const int s = j % VS;
-                if (!mbar_wait(&v_full[s], (j / VS) & 1)) {
+                if (!mbar_wait(&v_full[s], (j / VS) & 1, a.wait_ns)) {
                     ok = false;
                     break;
                 }
@@ -386,7 +387,9 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
         bool ok = true;
         const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
         for (int j = 0; j < nc && ok; ++j) {
-            if (!mbar_wait(&s_full[j & 1], (j >> 1) & 1)) {
+            // every wait before a warp-collective tcgen05 operation is decided
+            // for the whole warp (its lanes test the barrier independently)
+            if (!__all_sync(kFull, mbar_wait(&s_full[j & 1], (j >> 1) & 1, a.wait_ns))) {
                 ok = false;
                 break;
             }
@@ -459,7 +462,7 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
             // rescale this warp's rows of O when some row's reference max rose
             // (after the previous PV has completed)
             if (j >= 1 && __any_sync(kFull, raise)) {
-                if (!mbar_wait(o_full, (j - 1) & 1)) {
+                if (!__all_sync(kFull, mbar_wait(o_full, (j - 1) & 1, a.wait_ns))) {
                     ok = false;
                     break;
                 }
@@ -490,7 +493,7 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
                 // not loaded) have P = 0, but a NaN in V would still reach O
                 // (0 * NaN), so those V rows are cleared before PV may start
                 const int s = j % VS;
-                if (!mbar_wait(&v_full[s], (j / VS) & 1)) {
+                if (!__all_sync(kFull, mbar_wait(&v_full[s], (j / VS) & 1, a.wait_ns))) {
                     ok = false;
                     break;
                 }
@@ -509,7 +512,7 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
             if (lane == 0) mbar_arrive(&p_full[j & 1]);
         }
         // final O (after the last PV) for this row
-        if (ok && nc > 0 && !mbar_wait(o_last, 0)) ok = false;
+        if (ok && nc > 0) ok = __all_sync(kFull, mbar_wait(o_last, 0, a.wait_ns));
         if (ok && nc > 0) {
             tc_fence_after();
 #pragma unroll
@@ -726,6 +729,7 @@ cudaError_t attn_tc_launch(const AttnArgs& x, int m_tiles, int n_splits, float s
     a.S_max = x.S_max;
     a.max_prefix = x.max_prefix;
     a.scale_log2 = scale_log2;
+    a.wait_ns = wait_limit_ns();
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(m_tiles, (unsigned)BH, n_splits);
     cfg.blockDim = dim3(kAW * 32);

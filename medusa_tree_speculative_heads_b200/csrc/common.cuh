@@ -169,15 +169,21 @@ __device__ __forceinline__ uint64_t global_ns() {
     return t;
 }
 
+// Limit of every wait in the kernels: about two seconds.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
 // Wait for the phase of `bar` with the given parity to complete, giving up
-// after about two seconds (returns false then).  Used by every pipeline wait
-// so that a protocol error ends the kernel instead of hanging the GPU.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// after limit_ns (returns false then).  Used by every pipeline wait so that a
+// protocol error ends the kernel instead of hanging the GPU.  limit_ns <= 1
+// gives up at once unless the phase is already complete (a test of the
+// error paths; see medusa_debug_set_wait_limit).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns = kWaitLimitNs) {
+    if (limit_ns <= 1) return mbar_test(bar, parity);
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 255u) == 0 && global_ns() - t0 > 2000000000ull) return false;
+        if ((i & 255u) == 0 && global_ns() - t0 > limit_ns) return false;
     }
 }
 

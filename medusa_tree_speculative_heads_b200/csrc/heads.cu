@@ -669,7 +669,7 @@ HeadsWs heads_ws_layout(int B, int d, int V, int K, medusa_dtype dt) {
     w.ctr = w.stats + align256((size_t)B * K * sizeof(float2));
     // counters, and on the tensor-core path one hand-over flag per CTA and
     // phase plus the handed-over partial tiles ([2][grid][B][128] fp32)
-    w.slots = w.ctr + align256((size_t)(2 + 2 * num_sms()) * sizeof(unsigned int));
+    w.slots = w.ctr + align256((size_t)(2 + 2 * num_sms() + K) * sizeof(unsigned int));
     const size_t slots = heads_tc_supported(B, d, dt) ? (size_t)2 * num_sms() * B * 128 * sizeof(float) : 0;
     w.logits = w.slots + align256(slots);
     w.total = w.logits + align256((size_t)B * K * V * sizeof(float));

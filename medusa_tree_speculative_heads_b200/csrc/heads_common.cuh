@@ -101,6 +101,40 @@ __device__ __forceinline__ void warp_select(float (&lv)[kTopK], int (&li)[kTopK]
 }
 
 // ---------------------------------------------------------------------------
+// Which CTAs hold a partial of head k.  The K*uph tiles (head k owning tiles
+// [k*uph, (k+1)*uph)) are cut into upt units each; nparts CTAs split the
+// K*uph*upt units evenly and CTA c owns the tiles whose first unit falls in
+// its share.  The CTAs owning head k's tiles lie in [c_lo, c_hi], the owners
+// of its first and last tiles (unit u lies in the share of CTA
+// ceil((u+1) nparts / R) - 1); when every share holds a tile start, every
+// CTA of that range owns one of head k's tiles.
+// ---------------------------------------------------------------------------
+struct HeadCover {
+    long R;
+    int nparts, upt, c_lo, c_hi;
+    bool dense;
+    __device__ HeadCover(int nparts_, long uph, int upt_, int K, int k) : nparts(nparts_), upt(upt_) {
+        R = (long)K * uph * upt;
+        c_lo = owner((long)k * uph * upt);
+        c_hi = owner(((long)(k + 1) * uph - 1) * upt);
+        dense = R / nparts >= upt;
+    }
+    __device__ int owner(long u) const { return (int)(((u + 1) * nparts + R - 1) / R - 1); }
+    __device__ bool covers(int c) const {
+        if (c < c_lo || c > c_hi) return false;
+        if (dense) return true;
+        const long r0 = R * c / nparts, r1 = R * (c + 1) / nparts;
+        return (r1 + upt - 1) / upt > (r0 + upt - 1) / upt;  // owns a tile (in head k, by the range)
+    }
+    __device__ int count() const {
+        if (dense) return c_hi - c_lo + 1;
+        int n = 0;
+        for (int c = c_lo; c <= c_hi; ++c) n += covers(c);
+        return n;
+    }
+};
+
+// ---------------------------------------------------------------------------
 // Merge of one (sequence, head): the partials of the CTAs that covered the
 // head, in CTA order, so the result does not depend on which CTA runs the
 // merge.  The K*uph tiles (head k owning tiles [k*uph, (k+1)*uph)) are cut
@@ -122,7 +156,6 @@ static __device__ __noinline__ void merge_head(const HeadState* __restrict__ par
                            int32_t* __restrict__ node_tokens, float* __restrict__ node_q, float2* __restrict__ stats,
                            int32_t* status) {
     const int lane = threadIdx.x & 31;
-    const long R = (long)K * uph * upt;
     // the tree's shape and the root token are needed at the end: load them
     // first, so their latency overlaps the partials'
     constexpr int kTreeChunks = kMaxTree / 32;
@@ -143,19 +176,9 @@ static __device__ __noinline__ void merge_head(const HeadState* __restrict__ par
         lv[j] = -INFINITY;
         li[j] = INT_MAX;
     }
-    // CTA c owns the units [r0, r1), i.e. the tiles whose first unit lies there;
-    // the CTAs covering head k form the range [c_lo, c_hi], the owners of its
-    // first and last tiles (unit u lies in the share of CTA ceil((u+1) N / R) - 1)
-    auto owner = [&](long u) -> int { return (int)(((u + 1) * nparts + R - 1) / R - 1); };
-    const int c_lo = owner((long)k * uph * upt), c_hi = owner(((long)(k + 1) * uph - 1) * upt);
-    // when every share holds a tile start, every CTA of the range covers head k
-    const bool dense = R / nparts >= upt;
-    auto covers = [&](int c) -> bool {
-        if (c > c_hi) return false;
-        if (dense) return true;
-        const long r0 = R * c / nparts, r1 = R * (c + 1) / nparts;
-        return (r1 + upt - 1) / upt > (r0 + upt - 1) / upt;  // owns a tile (in head k, by the range)
-    };
+    const HeadCover hc(nparts, uph, upt, K, k);
+    const int c_lo = hc.c_lo, c_hi = hc.c_hi;
+    auto covers = [&](int c) -> bool { return hc.covers(c); };
     // lane l takes CTAs c_lo + l, c_lo + l + 32, ...; two of them per round,
     // all loads of a round issued before any is used
     for (int j0 = 0; c_lo + 32 * j0 <= c_hi; j0 += 2) {

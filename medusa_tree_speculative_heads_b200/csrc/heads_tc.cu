@@ -32,8 +32,13 @@
 // owner, which reaches it last in its run); the CTAs holding the rest reach
 // their part first in theirs, and hand it over as an fp32 partial in global
 // memory with a release flag.  The weight producer keeps prefetching across
-// the grid barrier.  After a second grid barrier the warps of the grid merge
-// the (sequence, head) partials, each in CTA order, and fill the tree.
+// the grid barrier.  A head's (sequence, head) partials are merged, each in
+// CTA order, and its tree nodes filled, by the last CTA to publish its
+// partial of that head (a per-head arrival counter, no waiting): the first
+// heads are merged while the stream goes on, only the last head's merge ends
+// the kernel.  With more than 16 sequences one CTA would take too long over
+// a head's merges, so there a grid barrier is followed by the merges of all
+// heads spread over every warp of the grid.
 // Every wait is bounded (~2 s) and sets MEDUSA_STATUS_TIMEOUT on expiry.
 #include <limits.h>
 
@@ -80,6 +85,8 @@ struct TcHeadsArgs {
     int32_t* status;
     int B, d, V, K;
     int stages;
+    int merge_per_head;  // B <= 16: each head merged by its last CTA; else all heads after a grid barrier
+    uint64_t wait_ns;    // limit of the pipeline waits (drains of issued work: kWaitLimitNs)
 };
 
 // A CTA's run of one phase: k-block units [u0, u1) of the phase's tiles laid
@@ -103,18 +110,22 @@ __device__ __forceinline__ void st_release_u32(unsigned int* p, unsigned int v) 
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-// bounded wait for a hand-over flag; false after ~2 s
-__device__ __forceinline__ bool wait_flag(const unsigned int* f) {
+// bounded wait for a hand-over flag; false after limit_ns
+__device__ __forceinline__ bool wait_flag(const unsigned int* f, uint64_t limit_ns) {
     if (ld_acquire_u32(f)) return true;
     const uint64_t t0 = global_ns();
     while (!ld_acquire_u32(f)) {
-        if (global_ns() - t0 > 2000000000ull) return false;
+        if (global_ns() - t0 > limit_ns) return false;
         __nanosleep(32);
     }
     return true;
 }
 
-__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
+// the four epilogue warps' barrier (aligned: each warp reconverges first)
+__device__ __forceinline__ void epi_sync() {
+    __syncwarp();
+    asm volatile("bar.sync 2, 128;" ::: "memory");
+}
 
 template <int N>
 __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid_constant__ TcHeadsArgs a) {
@@ -126,12 +137,16 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
     const int S = a.stages;
     uint8_t* sA = smem;
     uint8_t* sB = sA + (size_t)S * kABytes;
-    uint64_t* full = reinterpret_cast<uint64_t*>(sB + (size_t)S * kBBytes);
-    uint64_t* empty = full + S;
+    // a stage is full when both producers' copies landed: each producer has
+    // its own barrier, so each can drain exactly the copies it issued
+    uint64_t* full_w = reinterpret_cast<uint64_t*>(sB + (size_t)S * kBBytes);
+    uint64_t* full_b = full_w + S;
+    uint64_t* empty = full_b + S;
     uint64_t* acc_full = empty + S;    // [2]
     uint64_t* acc_empty = acc_full + 2;  // [2]
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
-    int* flag = reinterpret_cast<int*>(tmem_slot + 1);
+    uint64_t* mma_done = acc_empty + 2;  // every MMA issued has completed
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+    int* last_flag = reinterpret_cast<int*>(tmem_slot + 1);  // this CTA merges the head it just flushed
     float* sT = reinterpret_cast<float*>(tmem_slot + 4);  // [B][kTS] transposed tile
     HeadState* stS = reinterpret_cast<HeadState*>(sT + ((a.B * kTS + 3) & ~3));  // [seg][B] flush states
 
@@ -152,15 +167,16 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            mbar_init(&full[s], 2);  // the weight and the batch producer each arrive with their bytes
+            mbar_init(&full_w[s], 1);
+            mbar_init(&full_b[s], 1);
             mbar_init(&empty[s], 1);
         }
         for (int j = 0; j < 2; ++j) {
             mbar_init(&acc_full[j], 1);
             mbar_init(&acc_empty[j], 4);
         }
+        mbar_init(mma_done, 1);
         mbar_fence_init();
-        *flag = 0;
     }
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&a.mW_res);
@@ -179,6 +195,7 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
         if (lane == 0) {
             const bool weights = warp == 0;
             const uint32_t bytes = weights ? kABytes : kBBytes;
+            uint64_t* full = weights ? full_w : full_b;
             int it = 0;  // k-blocks issued (ring position)
             bool ok = true;
             for (int li = 0; li < ntiles && ok; ++li) {
@@ -192,7 +209,7 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
                     // vocabulary tiles read h^(k): wait until every CTA wrote its rows
                     const uint64_t t0 = global_ns();
                     while (ld_acquire_u32(&a.ctr[0]) < gridDim.x) {
-                        if (global_ns() - t0 > 2000000000ull) {
+                        if (global_ns() - t0 > a.wait_ns) {
                             set_status(a.status, MEDUSA_STATUS_TIMEOUT);
                             ok = false;
                             break;
@@ -204,7 +221,7 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
                 }
                 for (int kb = kb0; kb < kb1; ++kb) {
                     const int s = it % S;
-                    if (it >= S && !mbar_wait(&empty[s], ((it / S) - 1) & 1)) {
+                    if (it >= S && !mbar_wait(&empty[s], ((it / S) - 1) & 1, a.wait_ns)) {
                         set_status(a.status, MEDUSA_STATUS_TIMEOUT);
                         ok = false;
                         break;
@@ -233,7 +250,7 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
             int it = 0;
             for (int li = 0; li < ntiles && ok; ++li) {
                 const int buf = li & 1;
-                if (li >= 2 && !mbar_wait(&acc_empty[buf], ((li >> 1) - 1) & 1)) {
+                if (li >= 2 && !mbar_wait(&acc_empty[buf], ((li >> 1) - 1) & 1, a.wait_ns)) {
                     set_status(a.status, MEDUSA_STATUS_TIMEOUT);
                     break;
                 }
@@ -244,7 +261,8 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
                 piece(li, t, kb0, kb1);
                 for (int kb = kb0; kb < kb1; ++kb) {
                     const int s = it % S;
-                    if (!mbar_wait(&full[s], (it / S) & 1)) {
+                    if (!mbar_wait(&full_w[s], (it / S) & 1, a.wait_ns) ||
+                        !mbar_wait(&full_b[s], (it / S) & 1, a.wait_ns)) {
                         set_status(a.status, MEDUSA_STATUS_TIMEOUT);
                         ok = false;
                         break;
@@ -260,8 +278,9 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
                 }
                 tc_commit(&acc_full[buf]);
             }
-            // let every issued MMA finish before the accumulator is released
-            if (ntiles > 0) mbar_wait(&acc_full[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1);
+            // every MMA this thread issued completes before TMEM is released
+            tc_commit(mma_done);
+            mbar_wait(mma_done, 0);
         }
     } else {
         // ---------------- epilogue ----------------
@@ -368,7 +387,25 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
                     dst->idx[j] = mi[j];
                 }
             }
-            epi_sync();  // stS is free again
+            if (a.merge_per_head) {
+                // the last CTA to publish its partial of head kk merges the
+                // head (every sequence), while its producers and MMA go on
+                // streaming
+                __threadfence();
+                epi_sync();  // stS is free again; every partial of this CTA is written
+                if (et == 0)
+                    *last_flag = atomicAdd(&a.ctr[2 + 2 * G + kk], 1u) + 1u ==
+                                 (unsigned)HeadCover(G, tph_l, nkb, K, kk).count();
+                epi_sync();
+                if (*last_flag) {
+                    __threadfence();
+                    for (int b = ew; b < B; b += 4)
+                        merge_head(a.part, G, tph_l, nkb, B, b, b, a.V, K, kk,
+                                   a.tree.base ? a.tree.at(b) : nullptr, a.tree.T, a.root_token, a.topk_idx,
+                                   a.topk_prob, a.node_tokens, a.node_q, a.stats, a.status);
+                }
+            }
+            epi_sync();  // stS is free again (and last_flag read) before the next flush
             cm = -INFINITY;
             cl = 0.f;
 #pragma unroll
@@ -387,10 +424,13 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
         if (n1 == 0) arrive_grid();
         for (int li = 0; li < ntiles; ++li) {
             const int buf = li & 1;
-            if (ok && !mbar_wait(&acc_full[buf], (li >> 1) & 1)) {
+            if (ok && !mbar_wait(&acc_full[buf], (li >> 1) & 1, a.wait_ns)) {
                 if (lane == 0) set_status(a.status, MEDUSA_STATUS_TIMEOUT);
                 ok = false;
             }
+            // decided for the whole warp before its collective TMEM loads (the
+            // lanes test barriers and flags independently)
+            ok = __all_sync(kFull, ok);
             float v[N];
 #pragma unroll
             for (int e = 0; e < N; ++e) v[e] = 0.f;
@@ -431,7 +471,7 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
                 const long U = ph == 0 ? U1 : U2, tend = (t + 1) * nkb;
                 for (int c2 = cta + 1; c2 < G && U * c2 / G < tend; ++c2) {
                     if (U * (c2 + 1) / G == U * c2 / G) continue;  // an empty run
-                    if (!wait_flag(&a.ctr[2 + ph * G + c2])) {
+                    if (!wait_flag(&a.ctr[2 + ph * G + c2], a.wait_ns)) {
                         if (lane == 0) set_status(a.status, MEDUSA_STATUS_TIMEOUT);
                         ok = false;
                         break;
@@ -508,36 +548,37 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
-    // grid barrier: every CTA's partials are written; then the (sequence,
-    // head) merges are spread over all warps of the grid
+    if (a.merge_per_head) return;
+    // many sequences: a grid barrier (every CTA's partials are written), then
+    // the (sequence, head) merges spread over all warps of the grid
     __threadfence();
     sync_block();
     if (threadIdx.x == 0) {
+        *last_flag = 0;
         atomicAdd(&a.ctr[1], 1u);
         const uint64_t t0 = global_ns();
         while (ld_acquire_u32(&a.ctr[1]) < gridDim.x) {
-            if (global_ns() - t0 > 2000000000ull) {
+            if (global_ns() - t0 > a.wait_ns) {
                 set_status(a.status, MEDUSA_STATUS_TIMEOUT);
-                *flag = 1;
+                *last_flag = 1;
                 break;
             }
             __nanosleep(64);
         }
     }
     sync_block();
-    if (*flag) return;
+    if (*last_flag) return;
     __threadfence();
     for (int p = blockIdx.x * kTcWarps + warp; p < B * K; p += gridDim.x * kTcWarps) {
         const int b = p % B, k = p / B;
         merge_head(a.part, gridDim.x, tph_l, nkb, B, b, b, a.V, K, k, a.tree.base ? a.tree.at(b) : nullptr, a.tree.T,
-                   a.root_token, a.topk_idx, a.topk_prob,
-                   a.node_tokens, a.node_q, a.stats, a.status);
+                   a.root_token, a.topk_idx, a.topk_prob, a.node_tokens, a.node_q, a.stats, a.status);
     }
 }
 
 template <int N>
 size_t tc_smem_bytes(int stages, int B) {
-    return 1024 + (size_t)stages * (kABytes + N * kTK * 2) + (2 * (size_t)stages + 4) * 8 + 16 +
+    return 1024 + (size_t)stages * (kABytes + N * kTK * 2) + (3 * (size_t)stages + 5) * 8 + 16 +
            (size_t)((B * kTS + 3) & ~3) * 4 + (size_t)B * seg_per_col(B) * sizeof(HeadState);
 }
 
@@ -618,7 +659,9 @@ cudaError_t heads_tc_launch(const HeadsArgs& x, void* hk, void* part, unsigned i
     a.d = x.d;
     a.V = x.V;
     a.K = x.K;
-    cudaError_t e = cudaMemsetAsync(ctr, 0, (size_t)(2 + 2 * num_sms()) * sizeof(unsigned int), st);
+    a.merge_per_head = x.B <= 16;
+    a.wait_ns = wait_limit_ns();
+    cudaError_t e = cudaMemsetAsync(ctr, 0, (size_t)(2 + 2 * num_sms() + x.K) * sizeof(unsigned int), st);
     if (e != cudaSuccess) return e;
     switch (N) {
         case 16: return launch_n<16>(a, st);

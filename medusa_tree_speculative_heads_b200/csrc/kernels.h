@@ -43,7 +43,7 @@ cudaError_t heads_merge_shards_launch(const void* parts, int n_shards, int B, in
                                       int32_t* node_tokens, float* node_q, int32_t* status, cudaStream_t st);
 // tensor-core path (bf16, 1 <= B <= 64, d % 8 == 0)
 bool heads_tc_supported(int B, int d, medusa_dtype dt);
-// ctr: 2 + 2 * num_sms() counters (zeroed here); slots: 2 * num_sms() * B * 128 floats
+// ctr: 2 + 2 * num_sms() + K counters (zeroed here); slots: 2 * num_sms() * B * 128 floats
 cudaError_t heads_tc_launch(const HeadsArgs& a, void* hk, void* part, unsigned int* ctr, float* slots, float2* stats,
                             float* logits, cudaStream_t st);
 
@@ -144,6 +144,12 @@ struct CompactArgs {
     int32_t* status;
 };
 cudaError_t compact_launch(const CompactArgs& a, cudaStream_t st);
+
+// limit of the pipeline waits (hand-overs, phases, grid barriers) that the
+// heads and tree attention kernels are given: kWaitLimitNs unless changed by
+// medusa_debug_set_wait_limit; drains of issued copies and MMAs always wait
+// the full kWaitLimitNs
+uint64_t wait_limit_ns();
 
 // device properties, cached per device
 int num_sms();
