@@ -184,6 +184,15 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
         return c >= nP ? (c - nP) * kCh : paged ? c * kCh : S - (nP - c) * kCh;
     };
 
+    if (threadIdx.x == 32) {  // the descriptors' first use is the producer's first copy
+        tma_prefetch_desc(&a.mq);
+        tma_prefetch_desc(&a.mkc);
+        tma_prefetch_desc(&a.mvc);
+        if (!a.tree_in_cache) {
+            tma_prefetch_desc(&a.mkt);
+            tma_prefetch_desc(&a.mvt);
+        }
+    }
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
         for (int s = 0; s < KS; ++s) {

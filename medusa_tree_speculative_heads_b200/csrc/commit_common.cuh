@@ -10,32 +10,29 @@
 
 namespace medusa {
 
-// cache row t of the commit (t < L): K/V of tree node path[t] copied to
-// position prefix_len[b] + t of every kv-head, in a contiguous cache
-// [B, Hkv, S_max, row] or, with a block table, a page pool
+// The commit of a path already in shared memory: cache row t (t < L) gets
+// the K/V of tree node s_node[t] at position S + t of every kv-head, in a
+// contiguous cache [B, Hkv, S_max, row] or, with a block table, a page pool
 // [num_pages, Hkv, page_size, row].  Every check (path length, node ids,
 // cache room or owned pages) is made before anything is written; a failed
-// check sets a status bit and writes nothing but new_prefix_len = prefix_len.
-// prefix_len is read before any write, so new_prefix_len may alias it.
-// Whole block (blockDim.x >= MEDUSA_MAX_TREE threads), 16-byte copies.
-static __device__ __noinline__ void commit_sequence(int b, uint8_t* __restrict__ kc, uint8_t* __restrict__ vc,
-                                                    const uint8_t* __restrict__ kt, const uint8_t* __restrict__ vt,
-                                                    const int32_t* path, int max_path, const int32_t* len,
-                                                    const int32_t* prefix_len, int32_t* new_prefix_len, int T,
-                                                    int Hkv, int S_max, int row_bytes,
-                                                    const int32_t* __restrict__ table, int max_pages, int page_size,
-                                                    int num_pages, int32_t* status) {
-    __shared__ int s_ok, s_S, s_L;
-    __shared__ int s_node[MEDUSA_MAX_TREE];
+// check sets a status bit and writes nothing but new_prefix_len = S.  S is
+// the sequence's prefix length, read before anything is written (so
+// new_prefix_len may alias prefix_len).  Whole block (blockDim.x >=
+// MEDUSA_MAX_TREE threads), 16-byte copies.
+static __device__ __noinline__ void commit_path(int b, const int* s_node, int L, int S, bool len_ok,
+                                                uint8_t* __restrict__ kc, uint8_t* __restrict__ vc,
+                                                const uint8_t* __restrict__ kt, const uint8_t* __restrict__ vt,
+                                                int32_t* new_prefix_len, int T, int Hkv, int S_max, int row_bytes,
+                                                const int32_t* __restrict__ table, int max_pages, int page_size,
+                                                int num_pages, int32_t* status) {
+    __shared__ int s_ok;
     __shared__ int s_page[MEDUSA_MAX_TREE];  // paged: the page of position S + t
     const int tid = threadIdx.x;
-    const int S = prefix_len[b], L = len[b];
-    const bool len_ok = L >= 0 && L <= max_path && L <= MEDUSA_MAX_TREE && S >= 0;
+    len_ok = len_ok && L >= 0 && L <= MEDUSA_MAX_TREE && S >= 0;
     bool node_ok = true, page_ok = true;
-    if (len_ok && tid < L) {  // every path entry (and page) loaded at once
-        const int n = path[(long)b * max_path + tid];
+    if (len_ok && tid < L) {  // every node id (and page) checked at once
+        const int n = s_node[tid];
         node_ok = n >= 0 && n < T;
-        s_node[tid] = n;
         if (table) {
             const int blk = (S + tid) / page_size;
             const int page = blk < max_pages ? table[(long)b * max_pages + blk] : -1;
@@ -55,25 +52,42 @@ static __device__ __noinline__ void commit_sequence(int b, uint8_t* __restrict__
             set_status(status, MEDUSA_STATUS_CACHE_OVERFLOW);
         }
         s_ok = ok;
-        s_S = S;
-        s_L = L;
     }
     __syncthreads();
-    if (s_ok) {
+    const bool ok = s_ok;
+    if (ok) {
         const int vecs = row_bytes / 16;
         const int per_t = Hkv * vecs;
-        for (int e = tid; e < s_L * per_t; e += blockDim.x) {
+        for (int e = tid; e < L * per_t; e += blockDim.x) {
             const int t = e / per_t, rem = e % per_t;
             const int g = rem / vecs, c = rem % vecs;
             const long src = (((long)b * T + s_node[t]) * Hkv + g) * row_bytes + c * 16;
-            const long dst = table ? (((long)s_page[t] * Hkv + g) * page_size + (s_S + t) % page_size) * row_bytes + c * 16
-                                   : (((long)b * Hkv + g) * S_max + s_S + t) * row_bytes + c * 16;
+            const long dst = table ? (((long)s_page[t] * Hkv + g) * page_size + (S + t) % page_size) * row_bytes + c * 16
+                                   : (((long)b * Hkv + g) * S_max + S + t) * row_bytes + c * 16;
             *reinterpret_cast<uint4*>(kc + dst) = *reinterpret_cast<const uint4*>(kt + src);
             *reinterpret_cast<uint4*>(vc + dst) = *reinterpret_cast<const uint4*>(vt + src);
         }
     }
+    if (tid == 0) new_prefix_len[b] = ok ? S + L : S;
+}
+
+// The commit of sequence b's path as kv_commit receives it: path [B,
+// max_path] and len [B] in global memory (see commit_path).
+static __device__ __noinline__ void commit_sequence(int b, uint8_t* __restrict__ kc, uint8_t* __restrict__ vc,
+                                                    const uint8_t* __restrict__ kt, const uint8_t* __restrict__ vt,
+                                                    const int32_t* path, int max_path, const int32_t* len,
+                                                    const int32_t* prefix_len, int32_t* new_prefix_len, int T,
+                                                    int Hkv, int S_max, int row_bytes,
+                                                    const int32_t* __restrict__ table, int max_pages, int page_size,
+                                                    int num_pages, int32_t* status) {
+    __shared__ int s_node[MEDUSA_MAX_TREE];
+    const int tid = threadIdx.x;
+    const int S = prefix_len[b], L = len[b];
+    const bool len_ok = L >= 0 && L <= max_path && L <= MEDUSA_MAX_TREE;
+    if (len_ok && tid < L) s_node[tid] = path[(long)b * max_path + tid];
     __syncthreads();
-    if (tid == 0) new_prefix_len[b] = s_ok ? s_S + s_L : s_S;
+    commit_path(b, s_node, L, S, len_ok, kc, vc, kt, vt, new_prefix_len, T, Hkv, S_max, row_bytes, table, max_pages,
+                page_size, num_pages, status);
 }
 
 }  // namespace medusa

@@ -148,12 +148,17 @@ __global__ void __launch_bounds__(kWalkThreads) greedy_walk_kernel(const float* 
     __shared__ int pred[kMaxTree];
     __shared__ uint32_t match[kMaxTree / 32];
     __shared__ int best_key[kMaxTree / 32];
+    __shared__ uint32_t s_anc_best[kMaxTree / 32];
+    __shared__ int s_path[kMaxTree];
     const int b = blockIdx.x, u = threadIdx.x, lane = u & 31, w = u >> 5;
     const TreeDev* tree = trees.at(b);
     const int T = tree->T, Tn = trees.T;  // this sequence's nodes; node stride of the arrays
+    // every input is loaded up front, the commit's prefix length included
+    const int S_commit = cm.kc ? cm.prefix_len[b] : 0;
     float bv = -INFINITY;
     int bi = INT_MAX;
     int tok = 0, par = -1, dep = 0;
+    uint32_t anc[kMaxTree / 32] = {0u, 0u, 0u, 0u};
     if (u < T) {
         const long base = ((long)b * Tn + u) * splits;
         float lv[kMaxSplits];
@@ -167,6 +172,8 @@ __global__ void __launch_bounds__(kWalkThreads) greedy_walk_kernel(const float* 
         par = tree->parent[u];
         dep = tree->depth[u];
 #pragma unroll
+        for (int k = 0; k < kMaxTree / 32; ++k) anc[k] = tree->anc[u][k];
+#pragma unroll
         for (int s = 0; s < kMaxSplits; ++s) argmax_merge(bv, bi, lv[s], li[s]);
         pred[u] = bi;
     }
@@ -179,7 +186,7 @@ __global__ void __launch_bounds__(kWalkThreads) greedy_walk_kernel(const float* 
     if (u < T) {
         accepted = true;
 #pragma unroll
-        for (int k = 0; k < kMaxTree / 32; ++k) accepted &= (tree->anc[u][k] & ~match[k]) == 0u;
+        for (int k = 0; k < kMaxTree / 32; ++k) accepted &= (anc[k] & ~match[k]) == 0u;
     }
     // deepest accepted node, lowest index among equally deep: maximise depth*256 + (255 - index)
     int key = accepted ? dep * 256 + (255 - u) : -1;
@@ -187,23 +194,37 @@ __global__ void __launch_bounds__(kWalkThreads) greedy_walk_kernel(const float* 
     for (int o = 16; o > 0; o >>= 1) key = max(key, __shfl_xor_sync(kFull, key, o));
     if (lane == 0) best_key[w] = key;
     __syncthreads();
-    if (u == 0) {
-        int k = best_key[0];
-        for (int i = 1; i < kMaxTree / 32; ++i) k = max(k, best_key[i]);
-        const int best = 255 - (k & 255);
-        const int L = k >> 8;
-        int t = 0;
-        for (int j = 0; j <= best; ++j)
-            if ((tree->anc[best][j >> 5] >> (j & 31)) & 1u) accept_path[(long)b * max_path + t++] = j;
-        for (int j = L; j < max_path; ++j) accept_path[(long)b * max_path + j] = -1;
-        accept_len[b] = L;
-        bonus[b] = pred[best];
+    int k = best_key[0];
+#pragma unroll
+    for (int i = 1; i < kMaxTree / 32; ++i) k = max(k, best_key[i]);
+    const int best = 255 - (k & 255);
+    const int L = k >> 8;
+    if (u == best) {
+#pragma unroll
+        for (int i = 0; i < kMaxTree / 32; ++i) s_anc_best[i] = anc[i];
+    }
+    __syncthreads();
+    // the path: the best node's ancestors and itself in increasing index order
+    // (a parent's index is below its child's); node j goes to position
+    // popcount(ancestor bits below j)
+    {
+        const uint32_t word = s_anc_best[u >> 5];
+        if ((word >> (u & 31)) & 1u) {
+            int t = __popc(word & ((1u << (u & 31)) - 1u));
+            for (int i = 0; i < (u >> 5); ++i) t += __popc(s_anc_best[i]);
+            s_path[t] = u;
+            accept_path[(long)b * max_path + t] = u;
+        }
+        if (u >= L && u < max_path) accept_path[(long)b * max_path + u] = -1;
+        if (u == 0) {
+            accept_len[b] = L;
+            bonus[b] = pred[best];
+        }
     }
     if (cm.kc) {
-        __syncthreads();  // the path thread 0 wrote is visible to the block
-        commit_sequence(b, cm.kc, cm.vc, cm.kt, cm.vt, accept_path, max_path, accept_len, cm.prefix_len,
-                        cm.new_prefix_len, Tn, cm.Hkv, cm.S_max, cm.row_bytes, cm.table, cm.max_pages, cm.page_size,
-                        cm.num_pages, cm.status);
+        __syncthreads();  // s_path is complete
+        commit_path(b, s_path, L, S_commit, L <= max_path, cm.kc, cm.vc, cm.kt, cm.vt, cm.new_prefix_len, Tn, cm.Hkv,
+                    cm.S_max, cm.row_bytes, cm.table, cm.max_pages, cm.page_size, cm.num_pages, cm.status);
     }
 }
 
