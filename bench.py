@@ -489,6 +489,32 @@ def attention_roofline(attn_bytes, attn_flops, t_attn, pk):
             "hbm_frac": gbs / pk["hbm_gbs"], "tflops": tflops, "tc_frac": tflops / pk["bf16_tflops"], "bound": bound}
 
 
+def choose_attention_sms(ctx, args):
+    """SMs the heads kernel leaves to tree attention during its weight stream
+    (MedusaStep attention_sms): --attention-sms N, or with "auto" the fastest
+    of 0, 4, 8 and 16 over a few timed steps (the same computation every
+    time; only the launch shape differs)."""
+    if args.attention_sms != "auto":
+        return int(args.attention_sms)
+    best, best_t = 0, None
+    for R in (0, 4, 8, 16):
+        ctx.step.attention_sms = R
+        for _ in range(3):
+            ctx.run_step()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(8):
+            ctx.run_step()
+        e1.record()
+        torch.cuda.synchronize()
+        t = e0.elapsed_time(e1)
+        if best_t is None or t < best_t * 0.995:
+            best, best_t = R, t
+    ctx.step.attention_sms = best
+    return best
+
+
 def measure_config(name, args, world, dev, barrier, flush, pk):
     """A compact measurement of another workload (same protocol, fewer steps)."""
     from medusa_tree_speculative_heads_b200 import inputs as I
@@ -498,6 +524,7 @@ def measure_config(name, args, world, dev, barrier, flush, pk):
     for _ in range(max(args.warmup, 3)):
         ctx.run_step()
     torch.cuda.synchronize()
+    R = choose_attention_sms(ctx, args)
     stage, serial = measure_stages(ctx, K, flush)
     t = measure_steps(ctx, K, world, dev, barrier)
     hb, ab, af = ctx.algorithmic()
@@ -508,7 +535,7 @@ def measure_config(name, args, world, dev, barrier, flush, pk):
            "medusa_heads": {"gbs": hb / stage[0] / 1e9, "hbm_frac": hb / stage[0] / 1e9 / pk["hbm_gbs"]},
            "tree_attention": attention_roofline(ab, af, stage[1], pk),
            "mean_accept_len": float(ctx.step.accept_len.float().mean().item()),
-           "status": int(ctx.step.status.item())}
+           "attention_sms": R, "status": int(ctx.step.status.item())}
     del ctx
     torch.cuda.empty_cache()
     return out
@@ -540,6 +567,7 @@ def run_mine(args, rank, world, local_rank):
     for _ in range(max(args.warmup, 3)):
         ctx.run_step()
     torch.cuda.synchronize()
+    attention_sms = choose_attention_sms(ctx, args)
     K = args.steps
     clocks = ClockSampler(local_rank)
     clocks.start()
@@ -664,7 +692,11 @@ def run_mine(args, rank, world, local_rank):
                                    "ranked target and draft distributions)" if w.stochastic else
                                    "synthetic (seeded random weights and activations; target logits synthesised "
                                    f"from the proposed tree with match probability {w.match_prob})"),
-        "config": config_dict(w, world),
+        "config": {**config_dict(w, world),
+                   "launch": (f"heads kernel on {torch.cuda.get_device_properties(dev).multi_processor_count - attention_sms}"
+                              f" SMs, tree attention (no key splits) on the other {attention_sms} during the weight "
+                              f"stream" if attention_sms else
+                              "heads kernel on every SM, tree attention after it (key splits merged in-cluster)")},
         "roofline": roofline,
         "tree_attention": att,
         "stage_us": {"medusa_heads": stage[0] * 1e6, "tree_attention": stage[1] * 1e6,
@@ -727,6 +759,8 @@ def main():
     ap.add_argument("--impl", default="mine", choices=["mine", "reference"])
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--attention-sms", default="auto",
+                    help="SMs left to tree attention during the heads' weight stream (a number, or auto)")
     ap.add_argument("--configs", default="tiny,llama70b_b8,long32k,long128k,stoch_b64",
                     help="other workloads measured compactly into the line's 'configs' object ('none' for none)")
     ap.add_argument("--override", action="append", default=[],

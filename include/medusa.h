@@ -111,6 +111,21 @@ int medusa_version(void);
  */
 void medusa_debug_set_wait_limit(uint64_t ns);
 
+/*
+ * Launch shape of the calls the calling host thread makes afterwards (a
+ * library convenience for running calls concurrently on separate streams;
+ * not part of the method).  heads_ctas > 0: the bf16 tensor-core heads
+ * kernel (one cooperative CTA per SM by default) uses at most that many
+ * CTAs, leaving the other SMs to kernels on other streams.
+ * attention_splits > 0: the bf16 tensor-core tree attention kernel uses at
+ * most that many key splits per 128-row tile (1: no thread-block cluster,
+ * so its CTAs can run on any free SM).  0 restores the default.  Results
+ * stay within the float tolerances; the launch shape may change the last
+ * bits of floating-point outputs (rounding order of partial sums), never
+ * which work is done.  Returns MEDUSA_ERR_INVALID_ARG for negative values.
+ */
+int medusa_set_launch_shape(int heads_ctas, int attention_splits);
+
 /* ------------------------------------------------------------------------ */
 /* Candidate tree                                                            */
 /* ------------------------------------------------------------------------ */

@@ -225,7 +225,8 @@ class MedusaStep:
     def __init__(self, *, B: int, d: int, V: int, K: int, Hq: int, Hkv: int, D: int, S_max: int,
                  parents, dtype: torch.dtype, mode: int = _b.GREEDY, max_prefix: int = 0,
                  q_rows: int = 0, device=None, page_size: int = 0, max_pages: int = 0, num_pages: int = 0,
-                 temperature: float = 0.0, tree_in_cache: bool = False, overlap: bool = True):
+                 temperature: float = 0.0, tree_in_cache: bool = False, overlap: bool = True,
+                 attention_sms: int = 0):
         dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
         self.B, self.d, self.V, self.K = B, d, V, K
         self.Hq, self.Hkv, self.D, self.S_max, self.max_prefix = Hq, Hkv, D, S_max, max_prefix
@@ -252,6 +253,11 @@ class MedusaStep:
         self.page_size, self.max_pages, self.num_pages = page_size, max_pages, num_pages
         self.tree_in_cache = tree_in_cache
         self._layer_ptrs = {}
+        # run() with attention_sms > 0: the heads kernel leaves that many SMs
+        # free and tree attention runs on them without key splits, during the
+        # heads' weight stream instead of after it
+        self.attention_sms = attention_sms if overlap else 0
+        self._sms = torch.cuda.get_device_properties(dev).multi_processor_count
         # run(): tree attention (which reads none of the heads' outputs) on a
         # second stream, so its CTAs take the SMs the heads kernel frees while
         # that kernel's last CTA still merges
@@ -358,10 +364,17 @@ class MedusaStep:
             greedy_split = self.mode == _b.GREEDY and self.temperature <= 0
             self._hp.wait_stream(main)        # every call sees everything issued before the step
             self._side.wait_stream(main)
-            with torch.cuda.stream(self._hp):
-                self.heads(h, W_res, W_head, root_token)
-            with torch.cuda.stream(self._side):
-                self.attention(q, k_tree, v_tree, k_cache, v_cache, prefix_len, block_table)
+            reserve = 0 < self.attention_sms < self._sms
+            if reserve:
+                _b.set_launch_shape(self._sms - self.attention_sms, 1)
+            try:
+                with torch.cuda.stream(self._hp):
+                    self.heads(h, W_res, W_head, root_token)
+                with torch.cuda.stream(self._side):
+                    self.attention(q, k_tree, v_tree, k_cache, v_cache, prefix_len, block_table)
+            finally:
+                if reserve:
+                    _b.set_launch_shape(0, 0)
             if greedy_split:
                 self._side2.wait_stream(main)
                 with torch.cuda.stream(self._side2):

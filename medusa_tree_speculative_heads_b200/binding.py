@@ -62,6 +62,7 @@ def lib() -> ctypes.CDLL:
         L.medusa_version.restype = i32
         L.medusa_debug_set_wait_limit.argtypes = [u64]
         L.medusa_debug_set_wait_limit.restype = None
+        L.medusa_set_launch_shape.argtypes = [i32, i32]
         L.medusa_tree_create.argtypes = [vp, i32, ctypes.POINTER(vp)]
         L.medusa_tree_destroy.argtypes = [vp]
         L.medusa_tree_info.argtypes = [vp, vp, vp, vp]
@@ -142,6 +143,11 @@ def dtype_code(t: torch.dtype) -> int:
 
 def version() -> int:
     return lib().medusa_version()
+
+
+def set_launch_shape(heads_ctas: int, attention_splits: int) -> None:
+    """medusa_set_launch_shape for later calls from this thread (0, 0: default)."""
+    _check(lib().medusa_set_launch_shape(int(heads_ctas), int(attention_splits)))
 
 
 def set_wait_limit(ns: int) -> None:

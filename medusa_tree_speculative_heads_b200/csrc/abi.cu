@@ -138,6 +138,14 @@ namespace {
 std::atomic<uint64_t> g_wait_limit{0};  // 0: kWaitLimitNs
 }  // namespace
 
+namespace {
+thread_local int g_heads_ctas = 0;        // 0: one CTA per SM
+thread_local int g_attention_splits = 0;  // 0: chosen per call
+}  // namespace
+
+int launch_heads_ctas() { return g_heads_ctas; }
+int launch_attention_splits() { return g_attention_splits; }
+
 uint64_t wait_limit_ns() {
     const uint64_t v = g_wait_limit.load(std::memory_order_relaxed);
     return v ? v : kWaitLimitNs;
@@ -165,6 +173,15 @@ extern "C" const char* medusa_last_error(void) { return g_err.c_str(); }
 extern "C" int medusa_version(void) { return 100; }
 
 extern "C" void medusa_debug_set_wait_limit(uint64_t ns) { g_wait_limit.store(ns, std::memory_order_relaxed); }
+
+extern "C" int medusa_set_launch_shape(int heads_ctas, int attention_splits) {
+    if (heads_ctas < 0 || attention_splits < 0)
+        return fail(MEDUSA_ERR_INVALID_ARG, "medusa_set_launch_shape: negative value (%d, %d)", heads_ctas,
+                    attention_splits);
+    g_heads_ctas = heads_ctas;
+    g_attention_splits = attention_splits;
+    return ok();
+}
 
 // ---------------------------------------------------------------------------
 // tree handle

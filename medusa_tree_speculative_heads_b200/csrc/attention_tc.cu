@@ -683,6 +683,8 @@ int attn_tc_splits(int B, int T, int Hq, int Hkv, int max_prefix) {
     const long chunks = (max_prefix + kCh - 1) / kCh + (T + kCh - 1) / kCh;
     if (c > kMaxCluster) c = kMaxCluster;
     if (c > chunks) c = chunks;
+    const int cap = launch_attention_splits();
+    if (cap > 0 && c > cap) c = cap;
     return c < 1 ? 1 : (int)c;
 }
 

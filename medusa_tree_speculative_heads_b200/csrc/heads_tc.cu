@@ -627,7 +627,9 @@ cudaError_t launch_n(const TcHeadsArgs& args, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     prefer_max_smem(kern);
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(num_sms());
+    // one CTA per SM, or fewer when the caller leaves SMs to other streams
+    const int cap = launch_heads_ctas();
+    cfg.gridDim = dim3(cap > 0 && cap < num_sms() ? cap : num_sms());
     cfg.blockDim = dim3(kTcWarps * 32);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;

@@ -151,6 +151,12 @@ cudaError_t compact_launch(const CompactArgs& a, cudaStream_t st);
 // the full kWaitLimitNs
 uint64_t wait_limit_ns();
 
+// launch shape set by medusa_set_launch_shape on the calling thread: the
+// heads kernel's largest CTA count (0: one per SM) and the attention
+// kernel's largest number of key splits (0: chosen per call)
+int launch_heads_ctas();
+int launch_attention_splits();
+
 // device properties, cached per device
 int num_sms();
 size_t align256(size_t x);

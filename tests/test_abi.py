@@ -173,6 +173,9 @@ def test_newer_calls_validate_before_launch(lib):
     assert lib.tree_verify_greedy_rows(fake, 5, 1, 100, nul, fake, 1 << 20, nul) == UNS
     assert lib.tree_verify_greedy_walk(nul, 1, 100, nul, fake, 4, fake, fake, fake, 1 << 20, nul) == INV
     assert lib.tree_verify_greedy_walk(fake, 1, 100, nul, fake, 4, fake, fake, fake, 1 << 20, nul) == INV
+    # the launch shape refuses negative values and is restored by (0, 0)
+    assert lib.medusa_set_launch_shape(-1, 0) == INV
+    assert lib.medusa_set_launch_shape(100, 1) == 0 and lib.medusa_set_launch_shape(0, 0) == 0
     # the walk with its commit: NULL cache arguments, then a missing tree
     wc = lib.tree_verify_greedy_walk_commit
     wc.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,

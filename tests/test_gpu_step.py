@@ -12,8 +12,10 @@ from medusa_tree_speculative_heads_b200.api import MedusaStep
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("name", ["tiny", "llama8b"])
-def test_whole_step_matches_oracle(name):
+@pytest.mark.parametrize("name,attention_sms", [("tiny", 0), ("llama8b", 0), ("llama8b", 8)])
+def test_whole_step_matches_oracle(name, attention_sms):
+    # attention_sms = 8: the heads kernel on all but 8 SMs, tree attention
+    # (no key splits) on those 8 during the weight stream
     w = I.WORKLOADS[name]
     parents = I.workload_tree(w)
     T = len(parents)
@@ -34,7 +36,7 @@ def test_whole_step_matches_oracle(name):
     # ---- GPU step ----
     d = {k: v.cuda() for k, v in {**hin, **ain}.items()}
     st = MedusaStep(B=w.B, d=w.d, V=w.V, K=w.K, Hq=w.Hq, Hkv=w.Hkv, D=w.D, S_max=w.S_max, parents=parents,
-                    dtype=w.torch_dtype, max_prefix=w.max_prefix)
+                    dtype=w.torch_dtype, max_prefix=w.max_prefix, attention_sms=attention_sms)
     new_pl = torch.empty_like(d["prefix_len"])
     st.run(h=d["h"], W_res=d["W_res"], W_head=d["W_head"], root_token=d["root_token"], q=d["q"], k_tree=d["k_tree"],
            v_tree=d["v_tree"], k_cache=d["k_cache"], v_cache=d["v_cache"], prefix_len=d["prefix_len"],
@@ -68,11 +70,11 @@ def test_whole_step_matches_oracle(name):
         assert torch.equal(chain["kc"], okc) and torch.equal(chain["vc"], ovc)
 
 
-@pytest.mark.parametrize("name", ["llama8b_small", "stoch_small", "stoch_logits_small"])
+@pytest.mark.parametrize("name", ["llama8b_small", "stoch_small", "stoch_logits_small", "llama8b_reserved"])
 def test_graph_replay_equals_eager_step(name):
     # the step captured in a CUDA graph and replayed gives the eager step's
     # results bit for bit (the kernels are deterministic)
-    if name == "llama8b_small":
+    if name.startswith("llama8b"):
         w = I.scaled(I.WORKLOADS["llama8b"], B=2, d=512, V=3001, prefix=300)
     else:
         w = I.scaled(I.WORKLOADS["stoch_b64"], B=3, V=900)
@@ -81,8 +83,11 @@ def test_graph_replay_equals_eager_step(name):
     from medusa_tree_speculative_heads_b200 import binding as Bnd
     mode = Bnd.STOCHASTIC if w.stochastic else Bnd.GREEDY
     tau = I.STOCH_TEMPERATURE if name == "stoch_logits_small" else 0.0
+    # "reserved": the heads kernel leaves 8 SMs to tree attention (the launch
+    # shape is recorded into the graph with the kernels)
     step = MedusaStep(B=w.B, d=w.d, V=w.V, K=w.K, Hq=w.Hq, Hkv=w.Hkv, D=w.D, S_max=w.S_max, parents=parents,
-                      dtype=w.torch_dtype, device="cuda", mode=mode, q_rows=T, temperature=tau)
+                      dtype=w.torch_dtype, device="cuda", mode=mode, q_rows=T, temperature=tau,
+                      attention_sms=8 if name.endswith("reserved") else 0)
     hin = {k: v.cuda() for k, v in I.head_inputs(w).items()}
     ain = {k: v.cuda() for k, v in I.attention_inputs(w, T).items()}
     if w.stochastic:
