@@ -509,6 +509,7 @@ def choose_attention_sms(ctx, args):
         e1.record()
         torch.cuda.synchronize()
         t = e0.elapsed_time(e1)
+        print(f"attention_sms {R}: {1000.0 * t / 8:.1f} us per step", file=sys.stderr, flush=True)
         if best_t is None or t < best_t * 0.995:
             best, best_t = R, t
     ctx.step.attention_sms = best

@@ -11,8 +11,8 @@
 // node-major, row = node * G + (q-head within the group), so the G q-heads
 // of a node share every K/V element -- and a run of 64-key chunks.  A
 // sequence's chunks are its prefix chunks followed by its tree's one or two
-// chunks; the C CTAs of a thread-block cluster (cluster dims (1, 1, C)) take
-// equal runs of that list.  Per chunk:
+// chunks; the C CTAs of a thread-block cluster (cluster dims (1, 1, C), C <=
+// 16, chosen so the grid fills one wave) take equal runs of that list.  Per chunk:
 //   S   = Q K^T      tcgen05.mma M=128, N=64,  K=D   (both operands K-major)
 //   P   = exp2(S * scale * log2 e - m), masked; bf16, written back into TMEM
 //         over S's own columns
@@ -60,7 +60,7 @@ template <int D> constexpr int k_stages() { return D == 128 ? 3 : 4; }
 template <int D> constexpr int v_stages() { return D == 128 ? 2 : 4; }
 template <int D> constexpr int n_bars() { return 1 + 2 * k_stages<D>() + 2 * v_stages<D>() + 6; }
 constexpr int kPageRing = 8 * 8 * 4;  // bytes of the page-id ring (8 chunks x 8 boxes)
-constexpr int kMaxCluster = 8;        // key splits per tile: a portable cluster size
+constexpr int kMaxCluster = 16;       // key splits per tile: at most a (non-portable) cluster of 16
 // floats per row of a parked partial (D + 4: 16-byte row accesses of
 // consecutive rows fall on distinct banks)
 template <int D> constexpr int o_stride() { return D + 4; }
@@ -609,34 +609,39 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
 #pragma unroll
         for (int o2 = 16; o2 > 0; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o2));
         const float wl = ls == -INFINITY ? 0.f : exp2f(ls - M);
-        float part[kMaxCluster][PL];
-#pragma unroll
-        for (int s = 0; s < kMaxCluster; ++s) {  // every load issued before any is used
-            if (s < C) {
-                const float* src = cl.map_shared_rank(sO, s) + r * OS + lane * PL;
-                if constexpr (PL == 4) {
-                    const float4 v = *reinterpret_cast<const float4*>(src);
-                    part[s][0] = v.x;
-                    part[s][1] = v.y;
-                    part[s][2] = v.z;
-                    part[s][3] = v.w;
-                } else {
-                    const float2 v = *reinterpret_cast<const float2*>(src);
-                    part[s][0] = v.x;
-                    part[s][1] = v.y;
-                }
-            }
-        }
         float acc[PL], wsum = 0.f;
 #pragma unroll
         for (int e = 0; e < PL; ++e) acc[e] = 0.f;
+        constexpr int kBatch = 8;  // splits whose rows are loaded at once
 #pragma unroll
-        for (int s = 0; s < kMaxCluster; ++s) {  // in split order
-            const float ws = __shfl_sync(kFull, wl, s);
-            if (s < C && ws > 0.f) {
-                wsum += ws;
+        for (int s0 = 0; s0 < kMaxCluster; s0 += kBatch) {
+            if (s0 >= C) break;
+            float part[kBatch][PL];
 #pragma unroll
-                for (int e = 0; e < PL; ++e) acc[e] = fmaf(ws, part[s][e], acc[e]);
+            for (int u = 0; u < kBatch; ++u) {  // every load of the batch issued before any is used
+                if (s0 + u < C) {
+                    const float* src = cl.map_shared_rank(sO, s0 + u) + r * OS + lane * PL;
+                    if constexpr (PL == 4) {
+                        const float4 v = *reinterpret_cast<const float4*>(src);
+                        part[u][0] = v.x;
+                        part[u][1] = v.y;
+                        part[u][2] = v.z;
+                        part[u][3] = v.w;
+                    } else {
+                        const float2 v = *reinterpret_cast<const float2*>(src);
+                        part[u][0] = v.x;
+                        part[u][1] = v.y;
+                    }
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {  // in split order
+                const float ws = __shfl_sync(kFull, wl, s0 + u);
+                if (s0 + u < C && ws > 0.f) {
+                    wsum += ws;
+#pragma unroll
+                    for (int e = 0; e < PL; ++e) acc[e] = fmaf(ws, part[u][e], acc[e]);
+                }
             }
         }
         const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
@@ -672,14 +677,15 @@ bool attn_tc_supported(int Hq, int Hkv, int D, int T, medusa_dtype dt) {
     return dt == MEDUSA_BF16 && (D == 64 || D == 128) && G >= 1 && G <= 16 && (G & (G - 1)) == 0 && T <= kMaxTree;
 }
 
-// Key splits per 128-row tile: enough CTAs for two per SM, at most a portable
-// cluster and at most the chunks of the longest sequence.
+// Key splits per 128-row tile: as many as fit the grid in one wave of two
+// CTAs per SM (at least 1), at most a cluster of 16 and at most the chunks of
+// the longest sequence.
 int attn_tc_splits(int B, int T, int Hq, int Hkv, int max_prefix) {
     const int G = Hq / Hkv;
     const long m_tiles = ((long)T * G + kAM - 1) / kAM;
     const long per_split = m_tiles * B * Hkv;
     const long target = (long)kCtasPerSm * num_sms();
-    long c = (target + per_split - 1) / per_split;
+    long c = target / per_split;
     const long chunks = (max_prefix + kCh - 1) / kCh + (T + kCh - 1) / kCh;
     if (c > kMaxCluster) c = kMaxCluster;
     if (c > chunks) c = chunks;
@@ -757,12 +763,14 @@ cudaError_t attn_tc_launch(const AttnArgs& x, int m_tiles, int n_splits, float s
         cudaFuncSetAttribute(tree_attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)cfg.dynamicSmemBytes);
         cudaFuncSetAttribute(tree_attn_tc_kernel<128>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+        if (n_splits > 8) cudaFuncSetAttribute(tree_attn_tc_kernel<128>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
         return cudaLaunchKernelEx(&cfg, tree_attn_tc_kernel<128>, a);
     }
     cfg.dynamicSmemBytes = tc_attn_smem<64>();
     cudaFuncSetAttribute(tree_attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)cfg.dynamicSmemBytes);
     cudaFuncSetAttribute(tree_attn_tc_kernel<64>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (n_splits > 8) cudaFuncSetAttribute(tree_attn_tc_kernel<64>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     return cudaLaunchKernelEx(&cfg, tree_attn_tc_kernel<64>, a);
 }
 

@@ -88,7 +88,7 @@ struct TcHeadsArgs {
     float2* stats;
     int32_t* status;
     int B, d, V, K;
-    int sa, sb;  // stages of the weight ring and of the batch-vector ring
+    int stages;
     int merge_per_head;  // B <= 16: each head merged by its last CTA; else all heads after a grid barrier
     uint64_t wait_ns;    // limit of the pipeline waits (drains of issued work: kWaitLimitNs)
 };
@@ -138,19 +138,18 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
     constexpr uint32_t kIdesc = idesc_bf16_f32(kTM, N);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    // Two rings: weight tiles (from HBM, a deep ring: the bytes in flight set
-    // the stream rate) and batch-vector tiles (from L2, a short ring), each
-    // with its own barriers, so each producer can also drain exactly the
-    // copies it issued.  k-block `it` uses weight stage it % SA and batch
-    // stage it % SB.
-    const int SA = a.sa, SB = a.sb;
+    // One ring of stages, each a weight tile (from HBM) and a batch-vector
+    // tile (from L2; issued as early as its weight tile: under a full HBM
+    // stream its latency is as long).  A stage is full when both producers'
+    // copies landed: each producer has its own barrier, so each can drain
+    // exactly the copies it issued.
+    const int S = a.stages;
     uint8_t* sA = smem;
-    uint8_t* sB = sA + (size_t)SA * kABytes;
-    uint64_t* full_w = reinterpret_cast<uint64_t*>(sB + (size_t)SB * kBBytes);
-    uint64_t* empty_w = full_w + SA;
-    uint64_t* full_b = empty_w + SA;
-    uint64_t* empty_b = full_b + SB;
-    uint64_t* acc_full = empty_b + SB;    // [2]
+    uint8_t* sB = sA + (size_t)S * kABytes;
+    uint64_t* full_w = reinterpret_cast<uint64_t*>(sB + (size_t)S * kBBytes);
+    uint64_t* full_b = full_w + S;
+    uint64_t* empty = full_b + S;
+    uint64_t* acc_full = empty + S;    // [2]
     uint64_t* acc_empty = acc_full + 2;  // [2]
     uint64_t* mma_done = acc_empty + 2;  // every MMA issued has completed
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
@@ -175,13 +174,10 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
     };
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < SA; ++s) {
+        for (int s = 0; s < S; ++s) {
             mbar_init(&full_w[s], 1);
-            mbar_init(&empty_w[s], 1);
-        }
-        for (int s = 0; s < SB; ++s) {
             mbar_init(&full_b[s], 1);
-            mbar_init(&empty_b[s], 1);
+            mbar_init(&empty[s], 1);
         }
         for (int j = 0; j < 2; ++j) {
             mbar_init(&acc_full[j], 1);
@@ -207,9 +203,7 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
         if (lane == 0) {
             const bool weights = warp == 0;
             const uint32_t bytes = weights ? kABytes : kBBytes;
-            const int S = weights ? SA : SB;
             uint64_t* full = weights ? full_w : full_b;
-            uint64_t* empty = weights ? empty_w : empty_b;
             int it = 0;  // k-blocks issued (ring position)
             bool ok = true;
             for (int li = 0; li < ntiles && ok; ++li) {
@@ -274,21 +268,20 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
                 int kb0, kb1;
                 piece(li, t, kb0, kb1);
                 for (int kb = kb0; kb < kb1; ++kb) {
-                    const int s = it % SA, sb = it % SB;
-                    if (!mbar_wait(&full_w[s], (it / SA) & 1, a.wait_ns) ||
-                        !mbar_wait(&full_b[sb], (it / SB) & 1, a.wait_ns)) {
+                    const int s = it % S;
+                    if (!mbar_wait(&full_w[s], (it / S) & 1, a.wait_ns) ||
+                        !mbar_wait(&full_b[s], (it / S) & 1, a.wait_ns)) {
                         set_status(a.status, MEDUSA_STATUS_TIMEOUT);
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const uint64_t adesc = sw128_kmajor_desc(smem_addr(sA + (size_t)s * kABytes));
-                    const uint64_t bdesc = sw128_kmajor_desc(smem_addr(sB + (size_t)sb * kBBytes));
+                    const uint64_t bdesc = sw128_kmajor_desc(smem_addr(sB + (size_t)s * kBBytes));
 #pragma unroll
                     for (int ks = 0; ks < kTK / 16; ++ks)  // 16 k-elements = 32 bytes per MMA
                         tc_mma_bf16(d_tmem, adesc + 2 * ks, bdesc + 2 * ks, kIdesc, (kb != kb0 || ks != 0) ? 1u : 0u);
-                    tc_commit(&empty_w[s]);
-                    tc_commit(&empty_b[sb]);
+                    tc_commit(&empty[s]);
                     ++it;
                 }
                 tc_commit(&acc_full[buf]);
@@ -601,27 +594,25 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
 }
 
 template <int N>
-size_t tc_smem_bytes(int sa, int sb, int B) {
-    return 1024 + (size_t)sa * kABytes + (size_t)sb * N * kTK * 2 + (2 * (size_t)(sa + sb) + 5) * 8 + 16 +
+size_t tc_smem_bytes(int stages, int B) {
+    return 1024 + (size_t)stages * (kABytes + N * kTK * 2) + (3 * (size_t)stages + 5) * 8 + 16 +
            (size_t)((B * t_stride<N>() + 3) & ~3) * 4 + (size_t)B * seg_per_col(B) * sizeof(HeadState);
 }
 
-// the batch-vector tiles come from L2: four stages cover its latency; the
-// weight ring takes the rest of shared memory (at most 16 stages)
-constexpr int kBatchStages = 4;
+// as many stages as shared memory holds (at most 16): the weight bytes in
+// flight per SM set the stream rate
 template <int N>
-int tc_weight_stages(int B) {
+int tc_stages(int B) {
     int s = 16;
-    while (s > 2 && tc_smem_bytes<N>(s, kBatchStages, B) > (size_t)kSmemBudget) --s;
+    while (s > 2 && tc_smem_bytes<N>(s, B) > (size_t)kSmemBudget) --s;
     return s;
 }
 
 template <int N>
 cudaError_t launch_n(const TcHeadsArgs& args, cudaStream_t st) {
     TcHeadsArgs a = args;
-    a.sa = tc_weight_stages<N>(a.B);
-    a.sb = kBatchStages;
-    const size_t smem = tc_smem_bytes<N>(a.sa, a.sb, a.B);
+    a.stages = tc_stages<N>(a.B);
+    const size_t smem = tc_smem_bytes<N>(a.stages, a.B);
     auto kern = heads_tc_kernel<N>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
