@@ -31,12 +31,12 @@
 // and they are masked); paged prefix chunks are page-aligned from position 0.
 // Tree keys are masked with each row's ancestor bitmask.
 // With C = 1 the softmax threads write the bf16 output rows directly.  With
-// C > 1 every CTA parks its normalised partial rows and their log-sum-exps in
-// its own shared memory (over the drained K/V rings); after a cluster barrier
-// each CTA merges every C-th row of the tile from all C partials, read
-// through distributed shared memory in split order (so the result does not
-// depend on which CTA merges), and a second cluster barrier keeps every CTA's
-// shared memory alive until its peers have read it.  Every pipeline wait is
+// C > 1, after a cluster barrier (every CTA's K/V rings drained), each softmax
+// thread stores its normalised partial row and log-sum-exp through
+// distributed shared memory into the receive buffer of the CTA that merges
+// that row (row r: CTA r % C); after a second barrier every CTA merges its
+// rows from local shared memory in split order (so the result does not
+// depend on which CTA merges).  Every pipeline wait is
 // bounded (~2 s) and sets MEDUSA_STATUS_TIMEOUT on expiry.
 #include <cooperative_groups.h>
 #include <limits.h>
@@ -578,24 +578,33 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
         }
         return;
     }
-    // ---- several splits: park the normalised partials, merge over the cluster ----
+    // ---- several splits: each row's partial goes to the CTA that merges it ----
+    // Row r of the tile is merged by the cluster's CTA r % C, as its row
+    // r / C.  After a first cluster barrier (every CTA's K/V rings are drained
+    // and free), each softmax thread stores its normalised partial row and its
+    // log-sum-exp (in the row's padding) into that CTA's receive buffer
+    // [C][RPC][OS], at [split][r / C]; after a second barrier each CTA merges
+    // its rows from local shared memory, in split order.
     constexpr int OS = o_stride<D>();
-    float* sO = reinterpret_cast<float*>(sK);  // [kAM][OS] over the drained K/V rings
-    float* sL = reinterpret_cast<float*>(sQ);  // [kAM] over Q (no QK is pending)
-    if (warp >= 2) {
+    const int RPC = (kAM + C - 1) / C;           // rows merged per CTA
+    float* recv = reinterpret_cast<float*>(sK);  // [C][RPC][OS] over the drained K/V rings
+    const int nrows = min(kAM, rows_T - mt * kAM);
+    cg::cluster_group cl = cg::this_cluster();
+    __syncwarp();  // the cluster barrier is an aligned one: whole warps
+    cl.sync();     // every CTA of the cluster is past its main loop
+    if (warp >= 2 && lr < nrows) {
         const float inv = l > 0.f ? 1.f / l : 0.f;
-        float* dst = sO + lr * OS;
+        float* dst = cl.map_shared_rank(recv, lr % C) + ((long)split * RPC + lr / C) * OS;
 #pragma unroll
         for (int e = 0; e < D; e += 4)
             *reinterpret_cast<float4*>(dst + e) = make_float4(o[e] * inv, o[e + 1] * inv, o[e + 2] * inv, o[e + 3] * inv);
-        sL[lr] = l > 0.f ? m + log2f(l) : -INFINITY;
+        *reinterpret_cast<float4*>(dst + D) = make_float4(l > 0.f ? m + log2f(l) : -INFINITY, 0.f, 0.f, 0.f);
     }
-    cg::cluster_group cl = cg::this_cluster();
-    __syncwarp();  // the cluster barrier is an aligned one: whole warps
-    cl.sync();     // every split's partials are parked
+    __syncwarp();
+    cl.sync();  // every partial row has arrived (the stores are released by the barrier)
     constexpr int PL = D / 32;  // elements of a row per lane
-    const int nrows = min(kAM, rows_T - mt * kAM);
-    for (int r = split + C * warp; r < nrows; r += C * kAW) {
+    for (int i = warp; i * C + split < nrows; i += kAW) {
+        const int r = i * C + split;
         const long orow = out_row(mt * kAM + r);
         __nv_bfloat16* dst = a.out + orow * D + lane * PL;
         if (mt * kAM + r >= Tb * a.G) {  // past this sequence's tree: zero output
@@ -604,7 +613,7 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
             if (a.lse && lane == 0) a.lse[orow] = -INFINITY;
             continue;
         }
-        const float ls = lane < C ? *cl.map_shared_rank(sL + r, lane) : -INFINITY;
+        const float ls = lane < C ? recv[((long)lane * RPC + i) * OS + D] : -INFINITY;
         float M = ls;
 #pragma unroll
         for (int o2 = 16; o2 > 0; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o2));
@@ -612,36 +621,15 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
         float acc[PL], wsum = 0.f;
 #pragma unroll
         for (int e = 0; e < PL; ++e) acc[e] = 0.f;
-        constexpr int kBatch = 8;  // splits whose rows are loaded at once
 #pragma unroll
-        for (int s0 = 0; s0 < kMaxCluster; s0 += kBatch) {
-            if (s0 >= C) break;
-            float part[kBatch][PL];
+        for (int s2 = 0; s2 < kMaxCluster; ++s2) {  // in split order
+            if (s2 >= C) break;
+            const float ws = __shfl_sync(kFull, wl, s2);
+            if (ws > 0.f) {
+                const float* src = recv + ((long)s2 * RPC + i) * OS + lane * PL;
+                wsum += ws;
 #pragma unroll
-            for (int u = 0; u < kBatch; ++u) {  // every load of the batch issued before any is used
-                if (s0 + u < C) {
-                    const float* src = cl.map_shared_rank(sO, s0 + u) + r * OS + lane * PL;
-                    if constexpr (PL == 4) {
-                        const float4 v = *reinterpret_cast<const float4*>(src);
-                        part[u][0] = v.x;
-                        part[u][1] = v.y;
-                        part[u][2] = v.z;
-                        part[u][3] = v.w;
-                    } else {
-                        const float2 v = *reinterpret_cast<const float2*>(src);
-                        part[u][0] = v.x;
-                        part[u][1] = v.y;
-                    }
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < kBatch; ++u) {  // in split order
-                const float ws = __shfl_sync(kFull, wl, s0 + u);
-                if (s0 + u < C && ws > 0.f) {
-                    wsum += ws;
-#pragma unroll
-                    for (int e = 0; e < PL; ++e) acc[e] = fmaf(ws, part[u][e], acc[e]);
-                }
+                for (int e = 0; e < PL; ++e) acc[e] = fmaf(ws, src[e], acc[e]);
             }
         }
         const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
@@ -650,8 +638,6 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
             *reinterpret_cast<uint32_t*>(dst + e) = pack2_bf16(acc[e] * inv, acc[e + 1] * inv);
         if (a.lse && lane == 0) a.lse[orow] = wsum > 0.f ? (M + log2f(wsum)) * 0.69314718055994531f : -INFINITY;
     }
-    __syncwarp();
-    cl.sync();  // the peers are done reading this CTA's shared memory
 }
 
 template <int D>
@@ -660,9 +646,12 @@ size_t tc_attn_smem() {
     return (size_t)kAM * D * 2 + (size_t)(k_stages<D>() + v_stages<D>()) * kCh * D * 2 + n_bars<D>() * 8 + 16 +
            kPageRing;
 }
-// the parked partials fit over the rings, their log-sum-exps over Q
-static_assert(kAM * o_stride<128>() * 4 <= (k_stages<128>() + v_stages<128>()) * kCh * 128 * 2, "partials (D=128)");
-static_assert(kAM * o_stride<64>() * 4 <= (k_stages<64>() + v_stages<64>()) * kCh * 64 * 2, "partials (D=64)");
+// the receive buffer ([C][ceil(128 / C)][OS] floats, at most 143 rows for
+// C <= 16) fits over the K/V rings
+static_assert((kAM + kMaxCluster - 1) * o_stride<128>() * 4 <= (k_stages<128>() + v_stages<128>()) * kCh * 128 * 2,
+              "receive buffer (D=128)");
+static_assert((kAM + kMaxCluster - 1) * o_stride<64>() * 4 <= (k_stages<64>() + v_stages<64>()) * kCh * 64 * 2,
+              "receive buffer (D=64)");
 
 }  // namespace
 

@@ -141,14 +141,13 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
     // One ring of stages, each a weight tile (from HBM) and a batch-vector
     // tile (from L2; issued as early as its weight tile: under a full HBM
     // stream its latency is as long).  A stage is full when both producers'
-    // copies landed: each producer has its own barrier, so each can drain
-    // exactly the copies it issued.
+    // copies landed (one barrier, two arrivals with their byte counts: a
+    // single wait per k-block for the MMA thread).
     const int S = a.stages;
     uint8_t* sA = smem;
     uint8_t* sB = sA + (size_t)S * kABytes;
-    uint64_t* full_w = reinterpret_cast<uint64_t*>(sB + (size_t)S * kBBytes);
-    uint64_t* full_b = full_w + S;
-    uint64_t* empty = full_b + S;
+    uint64_t* full = reinterpret_cast<uint64_t*>(sB + (size_t)S * kBBytes);
+    uint64_t* empty = full + S;
     uint64_t* acc_full = empty + S;    // [2]
     uint64_t* acc_empty = acc_full + 2;  // [2]
     uint64_t* mma_done = acc_empty + 2;  // every MMA issued has completed
@@ -175,8 +174,7 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            mbar_init(&full_w[s], 1);
-            mbar_init(&full_b[s], 1);
+            mbar_init(&full[s], 2);  // the weight and the batch producer each arrive with their bytes
             mbar_init(&empty[s], 1);
         }
         for (int j = 0; j < 2; ++j) {
@@ -203,7 +201,6 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
         if (lane == 0) {
             const bool weights = warp == 0;
             const uint32_t bytes = weights ? kABytes : kBBytes;
-            uint64_t* full = weights ? full_w : full_b;
             int it = 0;  // k-blocks issued (ring position)
             bool ok = true;
             for (int li = 0; li < ntiles && ok; ++li) {
@@ -245,10 +242,17 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
                     ++it;
                 }
             }
-            // drain: no copy may still be landing when the CTA exits
+            // drain: no copy may still be landing when the CTA exits.  A stage's
+            // phase also needs the other producer's arrival; if that producer
+            // stopped early (a timed-out wait) the phase never completes, so the
+            // whole drain has one deadline rather than one per stage (the copies
+            // themselves land within microseconds).
+            const uint64_t t_end = global_ns() + kWaitLimitNs;
             for (int s = 0; s < S && s < it; ++s) {
                 const int last = s + ((it - 1 - s) / S) * S;
-                mbar_wait(&full[s], (last / S) & 1);
+                const uint64_t now = global_ns();
+                if (now >= t_end) break;
+                mbar_wait(&full[s], (last / S) & 1, t_end - now);
             }
         }
     } else if (warp == 1) {
@@ -269,8 +273,7 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
                 piece(li, t, kb0, kb1);
                 for (int kb = kb0; kb < kb1; ++kb) {
                     const int s = it % S;
-                    if (!mbar_wait(&full_w[s], (it / S) & 1, a.wait_ns) ||
-                        !mbar_wait(&full_b[s], (it / S) & 1, a.wait_ns)) {
+                    if (!mbar_wait(&full[s], (it / S) & 1, a.wait_ns)) {
                         set_status(a.status, MEDUSA_STATUS_TIMEOUT);
                         ok = false;
                         break;
@@ -595,7 +598,7 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
 
 template <int N>
 size_t tc_smem_bytes(int stages, int B) {
-    return 1024 + (size_t)stages * (kABytes + N * kTK * 2) + (3 * (size_t)stages + 5) * 8 + 16 +
+    return 1024 + (size_t)stages * (kABytes + N * kTK * 2) + (2 * (size_t)stages + 5) * 8 + 16 +
            (size_t)((B * t_stride<N>() + 3) & ~3) * 4 + (size_t)B * seg_per_col(B) * sizeof(HeadState);
 }
 
