@@ -12,7 +12,7 @@
 // of a node share every K/V element -- and a run of 64-key chunks.  A
 // sequence's chunks are its prefix chunks followed by its tree's one or two
 // chunks; the C CTAs of a thread-block cluster (cluster dims (1, 1, C), C <=
-// 16, chosen so the grid fills one wave) take equal runs of that list.  Per chunk:
+// 8) take equal runs of that list.  Per chunk:
 //   S   = Q K^T      tcgen05.mma M=128, N=64,  K=D   (both operands K-major)
 //   P   = exp2(S * scale * log2 e - m), masked; bf16, written back into TMEM
 //         over S's own columns
@@ -60,7 +60,7 @@ template <int D> constexpr int k_stages() { return D == 128 ? 3 : 4; }
 template <int D> constexpr int v_stages() { return D == 128 ? 2 : 4; }
 template <int D> constexpr int n_bars() { return 1 + 2 * k_stages<D>() + 2 * v_stages<D>() + 6; }
 constexpr int kPageRing = 8 * 8 * 4;  // bytes of the page-id ring (8 chunks x 8 boxes)
-constexpr int kMaxCluster = 16;       // key splits per tile: at most a (non-portable) cluster of 16
+constexpr int kMaxCluster = 8;        // key splits per tile: at most a portable cluster of 8
 // floats per row of a parked partial (D + 4: 16-byte row accesses of
 // consecutive rows fall on distinct banks)
 template <int D> constexpr int o_stride() { return D + 4; }
@@ -646,8 +646,8 @@ size_t tc_attn_smem() {
     return (size_t)kAM * D * 2 + (size_t)(k_stages<D>() + v_stages<D>()) * kCh * D * 2 + n_bars<D>() * 8 + 16 +
            kPageRing;
 }
-// the receive buffer ([C][ceil(128 / C)][OS] floats, at most 143 rows for
-// C <= 16) fits over the K/V rings
+// the receive buffer ([C][ceil(128 / C)][OS] floats, at most 135 rows for
+// C <= 8) fits over the K/V rings
 static_assert((kAM + kMaxCluster - 1) * o_stride<128>() * 4 <= (k_stages<128>() + v_stages<128>()) * kCh * 128 * 2,
               "receive buffer (D=128)");
 static_assert((kAM + kMaxCluster - 1) * o_stride<64>() * 4 <= (k_stages<64>() + v_stages<64>()) * kCh * 64 * 2,
@@ -666,15 +666,16 @@ bool attn_tc_supported(int Hq, int Hkv, int D, int T, medusa_dtype dt) {
     return dt == MEDUSA_BF16 && (D == 64 || D == 128) && G >= 1 && G <= 16 && (G & (G - 1)) == 0 && T <= kMaxTree;
 }
 
-// Key splits per 128-row tile: as many as fit the grid in one wave of two
-// CTAs per SM (at least 1), at most a cluster of 16 and at most the chunks of
-// the longest sequence.
+// Key splits per 128-row tile: enough CTAs for two per SM, at most a portable
+// cluster of 8 (a cluster of 9 CTAs at two per SM does not pack into the GPCs:
+// measured, the 288 CTAs of llama8b ran in two waves) and at most the chunks
+// of the longest sequence.
 int attn_tc_splits(int B, int T, int Hq, int Hkv, int max_prefix) {
     const int G = Hq / Hkv;
     const long m_tiles = ((long)T * G + kAM - 1) / kAM;
     const long per_split = m_tiles * B * Hkv;
     const long target = (long)kCtasPerSm * num_sms();
-    long c = target / per_split;
+    long c = (target + per_split - 1) / per_split;
     const long chunks = (max_prefix + kCh - 1) / kCh + (T + kCh - 1) / kCh;
     if (c > kMaxCluster) c = kMaxCluster;
     if (c > chunks) c = chunks;
@@ -752,14 +753,12 @@ cudaError_t attn_tc_launch(const AttnArgs& x, int m_tiles, int n_splits, float s
         cudaFuncSetAttribute(tree_attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)cfg.dynamicSmemBytes);
         cudaFuncSetAttribute(tree_attn_tc_kernel<128>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-        if (n_splits > 8) cudaFuncSetAttribute(tree_attn_tc_kernel<128>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
         return cudaLaunchKernelEx(&cfg, tree_attn_tc_kernel<128>, a);
     }
     cfg.dynamicSmemBytes = tc_attn_smem<64>();
     cudaFuncSetAttribute(tree_attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)cfg.dynamicSmemBytes);
     cudaFuncSetAttribute(tree_attn_tc_kernel<64>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-    if (n_splits > 8) cudaFuncSetAttribute(tree_attn_tc_kernel<64>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     return cudaLaunchKernelEx(&cfg, tree_attn_tc_kernel<64>, a);
 }
 

@@ -36,8 +36,8 @@
 // CTA order, and its tree nodes filled, by the last CTA to publish its
 // partial of that head (a per-head arrival counter, no waiting): the first
 // heads are merged while the stream goes on, only the last head's merge ends
-// the kernel.  With more than 16 sequences one CTA would take too long over
-// a head's merges, so there a grid barrier is followed by the merges of all
+// the kernel.  With more than 4 sequences one CTA would take too long over a
+// head's merges, so there a grid barrier is followed by the merges of all
 // heads spread over every warp of the grid.
 // Every wait is bounded (~2 s) and sets MEDUSA_STATUS_TIMEOUT on expiry.
 #include <limits.h>
@@ -58,10 +58,10 @@ constexpr int kABytes = kTM * kTK * 2;   // 16 KB
 constexpr int kEpiWarp0 = 3;             // first epilogue warp
 constexpr int kSmemBudget = 227 * 1024;
 constexpr int kTS = kTM + 1;             // transposed tile: column stride in floats (odd: no bank conflicts)
-// Above 32 sequences the tile is transposed in two halves of 64 rows, so the
-// buffer holds half of it (the shared memory goes to the weight ring)
-template <int N> constexpr bool half_transpose() { return N > 32; }
-template <int N> constexpr int t_stride() { return half_transpose<N>() ? kTM / 2 + 1 : kTS; }
+// Up to this many sequences a head is merged by its last CTA as soon as the
+// head is done; above it (one CTA would hold up the end with the merges of
+// many sequences) after a grid barrier, spread over every warp of the grid
+constexpr int kMergePerHeadMaxB = 4;
 
 // row segments per column in the transposed epilogue (at most 16, so that a
 // column's flush merges few partial states)
@@ -89,7 +89,7 @@ struct TcHeadsArgs {
     int32_t* status;
     int B, d, V, K;
     int stages;
-    int merge_per_head;  // B <= 16: each head merged by its last CTA; else all heads after a grid barrier
+    int merge_per_head;  // B <= kMergePerHeadMaxB: each head merged by its last CTA; else after a grid barrier
     uint64_t wait_ns;    // limit of the pipeline waits (drains of issued work: kWaitLimitNs)
 };
 
@@ -153,9 +153,8 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
     uint64_t* mma_done = acc_empty + 2;  // every MMA issued has completed
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
     int* last_flag = reinterpret_cast<int*>(tmem_slot + 1);  // this CTA merges the head it just flushed
-    constexpr int TS = t_stride<N>();
-    float* sT = reinterpret_cast<float*>(tmem_slot + 4);  // [B][TS] transposed tile (or half tile)
-    HeadState* stS = reinterpret_cast<HeadState*>(sT + ((a.B * TS + 3) & ~3));  // [seg][B] flush states
+    float* sT = reinterpret_cast<float*>(tmem_slot + 4);  // [B][kTS] transposed tile
+    HeadState* stS = reinterpret_cast<HeadState*>(sT + ((a.B * kTS + 3) & ~3));  // [seg][B] flush states
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int K = a.K, B = a.B;
@@ -526,35 +525,26 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
                 for (int e = 0; e < N; ++e)
                     if (e < B) a.logits[((long)e * K + k) * a.V + row0 + row] = v[e];
             }
-            constexpr int kHalves = half_transpose<N>() ? 2 : 1;
-#pragma unroll 1
-            for (int hh = 0; hh < kHalves; ++hh) {
-                // rows [h0, h0 + kTM / kHalves) of the tile pass through sT
-                const int h0 = hh * (kTM / kHalves), h1 = h0 + kTM / kHalves;
-                epi_sync();  // the previous readers are done with sT
-                if (row >= h0 && row < h1) {
+            epi_sync();  // the previous tile's readers are done with sT
 #pragma unroll
-                    for (int e = 0; e < N; ++e)
-                        if (e < B) sT[e * TS + row - h0] = v[e];
-                }
-                epi_sync();
-                if (ok) {
-                    const float* src = sT + col * TS;  // row r of the tile at src[r - h0]
-                    const int lo = max(r_lo, h0);
-                    const int hi = min(min(r_hi, h1), a.V - row0);  // rows past V are zero-filled weights
-                    float tm = -INFINITY;
-                    for (int r = lo; r < hi; ++r) tm = fmaxf(tm, src[r - h0]);
-                    if (tm > -INFINITY) {
-                        const float mn = fmaxf(cm, tm);
-                        float sum = 0.f;
-                        for (int r = lo; r < hi; ++r) {
-                            const float x = src[r - h0];
-                            sum += expf(x - mn);
-                            if (beats(x, row0 + r, lv[kTopK - 1], lx[kTopK - 1])) list_insert(lv, lx, x, row0 + r);
-                        }
-                        cl = (cm == -INFINITY ? 0.f : cl * expf(cm - mn)) + sum;
-                        cm = mn;
+            for (int e = 0; e < N; ++e)
+                if (e < B) sT[e * kTS + row] = v[e];
+            epi_sync();
+            if (ok) {
+                const float* src = sT + col * kTS;
+                const int hi = min(r_hi, a.V - row0);  // rows past V are zero-filled weights
+                float tm = -INFINITY;
+                for (int r = r_lo; r < hi; ++r) tm = fmaxf(tm, src[r]);
+                if (tm > -INFINITY) {
+                    const float mn = fmaxf(cm, tm);
+                    float sum = 0.f;
+                    for (int r = r_lo; r < hi; ++r) {
+                        const float x = src[r];
+                        sum += expf(x - mn);
+                        if (beats(x, row0 + r, lv[kTopK - 1], lx[kTopK - 1])) list_insert(lv, lx, x, row0 + r);
                     }
+                    cl = (cm == -INFINITY ? 0.f : cl * expf(cm - mn)) + sum;
+                    cm = mn;
                 }
             }
         }
@@ -599,7 +589,7 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
 template <int N>
 size_t tc_smem_bytes(int stages, int B) {
     return 1024 + (size_t)stages * (kABytes + N * kTK * 2) + (2 * (size_t)stages + 5) * 8 + 16 +
-           (size_t)((B * t_stride<N>() + 3) & ~3) * 4 + (size_t)B * seg_per_col(B) * sizeof(HeadState);
+           (size_t)((B * kTS + 3) & ~3) * 4 + (size_t)B * seg_per_col(B) * sizeof(HeadState);
 }
 
 // as many stages as shared memory holds (at most 16): the weight bytes in
@@ -683,7 +673,7 @@ cudaError_t heads_tc_launch(const HeadsArgs& x, void* hk, void* part, unsigned i
     a.d = x.d;
     a.V = x.V;
     a.K = x.K;
-    a.merge_per_head = x.B <= 16;
+    a.merge_per_head = x.B <= kMergePerHeadMaxB;
     a.wait_ns = wait_limit_ns();
     cudaError_t e = cudaMemsetAsync(ctr, 0, (size_t)(2 + 2 * num_sms() + x.K) * sizeof(unsigned int), st);
     if (e != cudaSuccess) return e;
