@@ -416,15 +416,29 @@ class StepCtx:
     def run_step(self):
         self.step.run(**self.run_kwargs())
 
+    @property
+    def fused_commit(self):
+        """Greedy verification commits in the walk's launch (run() does that
+        unless the commit is the all-layer compaction)."""
+        return not self.w.stochastic and not self.w.tree_in_cache
+
     def stages(self, i):
-        """The four calls in order on the current stream."""
+        """The step's calls in order on the current stream, as run() issues
+        them: heads, attention, verification (with the commit fused into the
+        walk in greedy mode), and the commit when it is a separate call."""
         st, hin, ain = self.step, self.hin, self.ain
-        return [lambda: st.heads(hin["h"], hin["W_res"], hin["W_head"], hin["root_token"]),
-                lambda: st.attention(ain["q"], ain["k_tree"], ain["v_tree"], ain["k_cache"], ain["v_cache"],
-                                     ain["prefix_len"], self.block_table),
-                lambda: st.verify(self.logits, self.q_draft, None, 0, i, self.vtok),
-                lambda: st.commit(ain["k_cache"], ain["v_cache"], ain["k_tree"], ain["v_tree"], ain["prefix_len"],
-                                  self.new_pl, self.block_table, self.k_layers, self.v_layers)]
+        calls = [lambda: st.heads(hin["h"], hin["W_res"], hin["W_head"], hin["root_token"]),
+                 lambda: st.attention(ain["q"], ain["k_tree"], ain["v_tree"], ain["k_cache"], ain["v_cache"],
+                                      ain["prefix_len"], self.block_table)]
+        if self.fused_commit:
+            calls.append(lambda: st.verify_commit(self.logits, ain["k_cache"], ain["v_cache"], ain["k_tree"],
+                                                  ain["v_tree"], ain["prefix_len"], self.new_pl, self.block_table))
+        else:
+            calls += [lambda: st.verify(self.logits, self.q_draft, None, 0, i, self.vtok),
+                      lambda: st.commit(ain["k_cache"], ain["v_cache"], ain["k_tree"], ain["v_tree"],
+                                        ain["prefix_len"], self.new_pl, self.block_table, self.k_layers,
+                                        self.v_layers)]
+        return calls
 
     def algorithmic(self):
         """Algorithmic bytes of the heads and of tree attention, and the
@@ -449,9 +463,10 @@ L2_FLUSH_BYTES = 256 << 20   # twice the 126 MB L2
 
 def measure_stages(ctx, K, flush):
     """Each of K repetitions: an L2 flush (a 256 MB memset, untimed), then the
-    four calls in order on one stream, each bracketed by CUDA events.
+    step's calls in order on one stream, each bracketed by CUDA events.
     Returns the median time of each stage (s) and the mean in-order step (s)."""
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    n = len(ctx.stages(0))
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n + 1)] for _ in range(K)]
     for i in range(K):
         flush.zero_()
         calls = ctx.stages(i)
@@ -460,9 +475,21 @@ def measure_stages(ctx, K, flush):
             call()
             ev[i][j + 1].record()
     torch.cuda.synchronize()
-    stage = [statistics.median(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K)) / 1000.0 for j in range(4)]
-    serial = statistics.mean(ev[i][0].elapsed_time(ev[i][4]) for i in range(K)) / 1000.0
+    stage = [statistics.median(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K)) / 1000.0 for j in range(n)]
+    serial = statistics.mean(ev[i][0].elapsed_time(ev[i][n]) for i in range(K)) / 1000.0
     return stage, serial
+
+
+def stage_dict(ctx, stage):
+    """stage_us keys: the commit is reported with verification when the walk
+    does it (one launch)."""
+    d = {"medusa_heads": stage[0] * 1e6, "tree_attention": stage[1] * 1e6}
+    if ctx.fused_commit:
+        d["tree_verify+kv_commit"] = stage[2] * 1e6
+    else:
+        d["tree_verify"] = stage[2] * 1e6
+        d["kv_compact" if ctx.w.tree_in_cache else "kv_commit"] = stage[3] * 1e6
+    return d
 
 
 def measure_steps(ctx, K, world, dev, barrier):
@@ -531,8 +558,7 @@ def measure_config(name, args, world, dev, barrier, flush, pk):
     hb, ab, af = ctx.algorithmic()
     out = {"workload": config_dict(w, world)["workload"], "steps": K, "value": whole_job_rate(world, K, t),
            "unit": UNIT, "ms_per_step": 1000.0 * t / K, "serial_ms_per_step": 1000.0 * serial,
-           "stage_us": {"medusa_heads": stage[0] * 1e6, "tree_attention": stage[1] * 1e6,
-                        "tree_verify": stage[2] * 1e6, "kv_commit": stage[3] * 1e6},
+           "stage_us": stage_dict(ctx, stage),
            "medusa_heads": {"gbs": hb / stage[0] / 1e9, "hbm_frac": hb / stage[0] / 1e9 / pk["hbm_gbs"]},
            "tree_attention": attention_roofline(ab, af, stage[1], pk),
            "mean_accept_len": float(ctx.step.accept_len.float().mean().item()),
@@ -700,14 +726,14 @@ def run_mine(args, rank, world, local_rank):
                               "heads kernel on every SM, tree attention after it (key splits merged in-cluster)")},
         "roofline": roofline,
         "tree_attention": att,
-        "stage_us": {"medusa_heads": stage[0] * 1e6, "tree_attention": stage[1] * 1e6,
-                     "tree_verify": stage[2] * 1e6, ("kv_compact" if w.tree_in_cache else "kv_commit"): stage[3] * 1e6},
+        "stage_us": stage_dict(ctx, stage),
         "timing": ("value: K back-to-back steps as MedusaStep.run issues them (attention overlapped with the heads' "
-                   "tail), CUDA events on the launching stream; stage_us and serial_ms_per_step: the four calls in "
-                   "order, median (stages) / mean (step) of K repetitions, each after a 256 MB L2 flush"),
+                   "tail), CUDA events on the launching stream; stage_us and serial_ms_per_step: the step's calls in "
+                   "order (greedy: the row scan, then the walk that also commits, one launch), median (stages) / "
+                   "mean (step) of K repetitions, each after a 256 MB L2 flush"),
         "serial_ms_per_step": 1000.0 * serial_s,
         "mean_accept_len": mean_len,
-        **({"kv_compact": {"layers": w.layers, "us": stage[3] * 1e6,
+        **({"kv_compact": {"layers": w.layers, "us": stage[-1] * 1e6,
                            "moved_bytes": 2 * 2 * w.layers * w.Hkv * w.D * (2 if w.dtype == "bf16" else 4) *
                            int(step.accept_len.sum().item()),
                            "note": "read + write of the accepted rows' K and V in every layer, one launch"}}

@@ -316,6 +316,21 @@ class MedusaStep:
                        step, self.accept_path, self.max_path, self.accept_len, self.bonus, self.ws_verify,
                        self.ws_verify_n, self.status)
 
+    def verify_commit(self, target, k_cache, v_cache, k_tree, v_tree, prefix_len, new_prefix_len, block_table=None,
+                      node_tokens=None):
+        """Greedy verification and the commit as run() issues them, in order on
+        the current stream: the row scan, then the walk that commits the path
+        it finds (one launch)."""
+        _b.tree_verify_greedy_rows(target, _b.dtype_code(target.dtype), self.B, self.V, self.tree, self.ws_verify,
+                                   self.ws_verify_n)
+        paged = self.page_size > 0
+        _b.tree_verify_greedy_walk_commit(self.node_tokens if node_tokens is None else node_tokens, self.B, self.V,
+                                          self.tree, self.accept_path, self.max_path, self.accept_len, self.bonus,
+                                          self.ws_verify, self.ws_verify_n, k_cache, v_cache, k_tree, v_tree,
+                                          prefix_len, new_prefix_len, self.Hkv, self.D, self.S_max,
+                                          block_table if paged else None, self.max_pages, self.page_size,
+                                          self.num_pages, self.dt, self.status)
+
     def layer_pointers(self, k_layers, v_layers):
         """Device pointer arrays of the layers' caches, built once per list
         (build them before capturing a graph)."""
