@@ -563,10 +563,9 @@ cudaError_t attn_launch_bf16(const AttnArgs& a, cudaStream_t st) {
     p.part_lse = (float*)((char*)a.ws + align256((size_t)sp.n_splits * BH * p.R * D * sizeof(float)));
     p.status = a.status;
     if (tc) {
-        // one or two 128-row tiles per CTA; the key splits of a CTA tile merge
-        // inside their cluster
-        return attn_tc_launch(a, attn_tc_m_tiles(a.T, a.Hq, a.Hkv),
-                              attn_tc_splits(a.B, a.T, a.Hq, a.Hkv, D, a.max_prefix), p.scale_log2, st);
+        // 128-row tiles; the key splits of a tile merge inside their cluster
+        const int m_tiles = (a.T * p.G + 127) / 128;
+        return attn_tc_launch(a, m_tiles, attn_tc_splits(a.B, a.T, a.Hq, a.Hkv, a.max_prefix), p.scale_log2, st);
     }
     {
         const size_t smem = (size_t)kBM * D * 2 + 4 * (size_t)kBN * D * 2 + kBM * 4 * sizeof(uint32_t);

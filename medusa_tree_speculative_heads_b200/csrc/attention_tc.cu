@@ -49,20 +49,18 @@ namespace medusa {
 
 namespace {
 
-constexpr int kAM = 128;     // query rows per tile (MMA M)
+constexpr int kAW = 6;       // 0 producer, 1 MMA, 2-5 softmax
+constexpr int kAM = 128;     // query rows per CTA (MMA M)
 constexpr int kCh = 64;      // keys per chunk
-// NT query tiles per CTA: warps 0 producer, 1 MMA, then four softmax warps
-// per tile.  NT = 1: two CTAs per SM (256 TMEM columns each); NT = 2: one
-// CTA per SM owning all 512 columns, both tiles sharing every K/V chunk.
-template <int NT> constexpr int n_warps() { return 2 + 4 * NT; }
-template <int NT> constexpr int ctas_per_sm() { return NT == 1 ? 2 : 1; }
-// K and V rings: a K stage is free once its QK products are done, a V stage
-// once its PV products are; the stages fill the CTA's share of shared memory
-template <int D, int NT> constexpr int k_stages() { return NT == 1 ? (D == 128 ? 3 : 4) : (D == 128 ? 5 : 6); }
-template <int D, int NT> constexpr int v_stages() { return NT == 1 ? (D == 128 ? 2 : 4) : (D == 128 ? 4 : 6); }
-template <int D, int NT> constexpr int n_bars() { return 1 + 2 * k_stages<D, NT>() + 2 * v_stages<D, NT>() + 6 * NT; }
+constexpr int kCtasPerSm = 2;
+// K and V rings: a K stage is free once its QK product is done, a V stage
+// once its PV product is; at head_dim 128 three K and two V stages keep a CTA
+// within half of an SM's shared memory
+template <int D> constexpr int k_stages() { return D == 128 ? 3 : 4; }
+template <int D> constexpr int v_stages() { return D == 128 ? 2 : 4; }
+template <int D> constexpr int n_bars() { return 1 + 2 * k_stages<D>() + 2 * v_stages<D>() + 6; }
 constexpr int kPageRing = 8 * 8 * 4;  // bytes of the page-id ring (8 chunks x 8 boxes)
-constexpr int kMaxCluster = 16;       // key splits per tile: at most a cluster of 16 (non-portable above 8)
+constexpr int kMaxCluster = 8;        // key splits per tile: at most a portable cluster of 8
 // floats per row of a parked partial (D + 4: 16-byte row accesses of
 // consecutive rows fall on distinct banks)
 template <int D> constexpr int o_stride() { return D + 4; }
@@ -119,26 +117,22 @@ __device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t smem_byte_addr, 
     return d;
 }
 
-template <int D, int NT>
-__global__ void __launch_bounds__(n_warps<NT>() * 32, ctas_per_sm<NT>())
-    tree_attn_tc_kernel(const __grid_constant__ TcAttnArgs a) {
+template <int D>
+__global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(const __grid_constant__ TcAttnArgs a) {
     constexpr int NSUB = D / 64;              // 64-element blocks along D
-    constexpr int kQBytes = kAM * D * 2;      // one tile of Q
+    constexpr int kQBytes = kAM * D * 2;
     constexpr int kSub = kCh * 128;           // [64 keys x 64 D] block = 8 KB
     constexpr int kKVBytes = kCh * D * 2;     // one chunk of K (or of V)
-    constexpr int KS = k_stages<D, NT>(), VS = v_stages<D, NT>();
-    constexpr int kW = n_warps<NT>();
+    constexpr int KS = k_stages<D>(), VS = v_stages<D>();
     constexpr uint32_t kIdescQK = idesc_bf16_f32(kAM, kCh);
     constexpr uint32_t kIdescPV = idesc_bf16_f32(kAM, D) | (1u << 16);  // A (P) from TMEM, B (V) MN-major
-    // TMEM: tile t owns columns [256 t, 256 t + 256): S/P double buffer at +0
-    // and +64, O (D columns) at +128
-    constexpr uint32_t kTmemCols = 256 * NT;
+    constexpr uint32_t kTmemCols = 256;       // S: 2 x 64 columns, O: D columns at 128
     // Dynamic shared memory starts on a 1024-byte boundary when the kernel has
     // no static shared memory; the tiles below rely on it (checked at entry,
-    // so the CTAs fit without alignment padding).
+    // so two CTAs fit per SM without alignment padding).
     extern __shared__ __align__(1024) uint8_t smem[];
-    uint8_t* sQ = smem;                       // [NT] tiles
-    uint8_t* sK = sQ + NT * kQBytes;
+    uint8_t* sQ = smem;
+    uint8_t* sK = sQ + kQBytes;
     uint8_t* sV = sK + KS * kKVBytes;
     uint64_t* bars = reinterpret_cast<uint64_t*>(sV + VS * kKVBytes);
     uint64_t* q_full = bars;
@@ -146,14 +140,14 @@ __global__ void __launch_bounds__(n_warps<NT>() * 32, ctas_per_sm<NT>())
     uint64_t* k_empty = k_full + KS;
     uint64_t* v_full = k_empty + KS;
     uint64_t* v_empty = v_full + VS;
-    uint64_t* s_full = v_empty + VS;          // [NT][2]
-    uint64_t* p_full = s_full + 2 * NT;       // [NT][2]
-    uint64_t* o_full = p_full + 2 * NT;       // [NT]: one phase per PV product of the tile
-    // [NT]: a single phase, completed with the tile's last PV product: a
-    // parity wait on o_full cannot tell "the last PV done" from "two PVs done"
-    // once both of the last two have completed
-    uint64_t* o_last = o_full + NT;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_last + NT);
+    uint64_t* s_full = v_empty + VS;
+    uint64_t* p_full = s_full + 2;
+    uint64_t* o_full = p_full + 2;  // one phase per PV product
+    // a single phase, completed with the last PV product: a parity wait on
+    // o_full cannot tell "the last PV done" from "two PVs done" once both of
+    // the last two have completed
+    uint64_t* o_last = o_full + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_last + 1);
     // paged: the page of each box of the last 8 K chunks, for their V loads
     int* pg_ring = reinterpret_cast<int*>(tmem_slot + 4);  // [8][8]
 
@@ -169,7 +163,6 @@ __global__ void __launch_bounds__(n_warps<NT>() * 32, ctas_per_sm<NT>())
         return;
     }
     const int NB = kAM / a.G;  // nodes per tile
-    const int row0 = mt * NT * kAM;  // first row of this CTA (tile t: rows row0 + 128 t ..)
 
     int S = a.prefix_len[b];
     if (S < 0 || S > a.max_prefix) {
@@ -210,14 +203,12 @@ __global__ void __launch_bounds__(n_warps<NT>() * 32, ctas_per_sm<NT>())
             mbar_init(&v_full[s], 1);
             mbar_init(&v_empty[s], 1);
         }
-        for (int i = 0; i < 2 * NT; ++i) {
+        for (int i = 0; i < 2; ++i) {
             mbar_init(&s_full[i], 1);
             mbar_init(&p_full[i], 4);
         }
-        for (int t = 0; t < NT; ++t) {
-            mbar_init(&o_full[t], 1);
-            mbar_init(&o_last[t], 1);
-        }
+        mbar_init(o_full, 1);
+        mbar_init(o_last, 1);
         mbar_fence_init();
     }
     if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
@@ -226,11 +217,9 @@ __global__ void __launch_bounds__(n_warps<NT>() * 32, ctas_per_sm<NT>())
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    // a softmax thread's tile, TMEM lane (= row of the tile) and row within
-    // the (sequence, kv-head); its final (unnormalised) O, max m and sum l
-    const int tt = warp >= 2 ? (warp - 2) >> 2 : 0;
-    const int lr = (warp & 3) * 32 + lane;
-    const int rrow = row0 + tt * kAM + lr;
+    // the softmax threads' row: its final (unnormalised) O, max m and sum l
+    const int lr = (warp & 3) * 32 + lane;   // TMEM lane = tile row of a softmax thread
+    const int rrow = mt * kAM + lr;          // row within the (sequence, kv-head)
     const bool row_ok = warp >= 2 && rrow < Tb * a.G;
     float o[D];
     float m = -INFINITY, l = 0.f;
@@ -241,13 +230,10 @@ __global__ void __launch_bounds__(n_warps<NT>() * 32, ctas_per_sm<NT>())
         // stage is free (polled without blocking, so a late V stage never
         // holds back the next K)
         if (lane == 0 && nc > 0) {
-            mbar_arrive_expect_tx(q_full, NT * kQBytes);
+            mbar_arrive_expect_tx(q_full, kQBytes);
 #pragma unroll
-            for (int t = 0; t < NT; ++t)
-#pragma unroll
-                for (int sub = 0; sub < NSUB; ++sub)
-                    tma_load_3d(sQ + t * kQBytes + sub * (kAM * 128), &a.mq, sub * 64, g * a.G,
-                                b * a.T + (mt * NT + t) * NB, q_full);
+            for (int sub = 0; sub < NSUB; ++sub)
+                tma_load_3d(sQ + sub * (kAM * 128), &a.mq, sub * 64, g * a.G, b * a.T + mt * NB, q_full);
             // Paged: the page of every box (page_rows keys) of a prefix chunk,
             // copied asynchronously into the chunk's pg_ring slot one chunk
             // ahead (a K chunk waits only for its own ids; its V chunk reuses
@@ -347,72 +333,57 @@ __global__ void __launch_bounds__(n_warps<NT>() * 32, ctas_per_sm<NT>())
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
-        // per chunk: QK of chunk j+1 for every tile (overlapping the softmax of
-        // chunk j), then PV of chunk j tile by tile as each tile's P is ready
         if (lane == 0 && nc > 0) {
             bool ok = mbar_wait(q_full, 0, a.wait_ns);
-            // S_j goes to a tile's TMEM columns (j&1)*64; P_j is written over
-            // it, so the buffer is free for S_{j+2} once PV_j has completed
-            // (the tile's o_full phase j)
+            // S_j goes to TMEM columns (j&1)*64; P_j is written over it, so the
+            // buffer is free for S_{j+2} once PV_j has completed (o_full phase j)
             auto issue_qk = [&](int j) -> bool {
                 const int s = j % KS, sb = j & 1;
                 if (!mbar_wait(&k_full[s], (j / KS) & 1, a.wait_ns)) return false;
-#pragma unroll
-                for (int t = 0; t < NT; ++t)
-                    if (j >= 2 && !mbar_wait(&o_full[t], (j - 2) & 1, a.wait_ns)) return false;
+                if (j >= 2 && !mbar_wait(o_full, (j - 2) & 1, a.wait_ns)) return false;
                 tc_fence_after();
 #pragma unroll
-                for (int t = 0; t < NT; ++t) {
+                for (int sub = 0; sub < NSUB; ++sub) {
+                    const uint64_t ad = sw128_kmajor_desc(smem_addr(sQ + sub * (kAM * 128)));
+                    const uint64_t bd = sw128_kmajor_desc(smem_addr(sK + s * kKVBytes + sub * kSub));
 #pragma unroll
-                    for (int sub = 0; sub < NSUB; ++sub) {
-                        const uint64_t ad = sw128_kmajor_desc(smem_addr(sQ + t * kQBytes + sub * (kAM * 128)));
-                        const uint64_t bd = sw128_kmajor_desc(smem_addr(sK + s * kKVBytes + sub * kSub));
-#pragma unroll
-                        for (int ks = 0; ks < 4; ++ks)
-                            tc_mma_bf16(tmem + t * 256 + sb * kCh, ad + 2 * ks, bd + 2 * ks, kIdescQK,
-                                        (sub | ks) != 0);
-                    }
-                    tc_commit(&s_full[t * 2 + sb]);
+                    for (int ks = 0; ks < 4; ++ks)
+                        tc_mma_bf16(tmem + sb * kCh, ad + 2 * ks, bd + 2 * ks, kIdescQK, (sub | ks) != 0);
                 }
+                tc_commit(&s_full[sb]);
                 tc_commit(&k_empty[s]);
                 return true;
             };
             if (ok) ok = issue_qk(0);
             for (int j = 0; j < nc && ok; ++j) {
                 if (j + 1 < nc && !(ok = issue_qk(j + 1))) break;
+                if (!mbar_wait(&p_full[j & 1], (j >> 1) & 1, a.wait_ns)) {
+                    ok = false;
+                    break;
+                }
                 const int s = j % VS;
                 if (!mbar_wait(&v_full[s], (j / VS) & 1, a.wait_ns)) {
                     ok = false;
                     break;
                 }
+                tc_fence_after();
                 const uint64_t bd = sw128_mnmajor_desc(smem_addr(sV + s * kKVBytes), kSub);
 #pragma unroll
-                for (int t = 0; t < NT && ok; ++t) {
-                    if (!mbar_wait(&p_full[t * 2 + (j & 1)], (j >> 1) & 1, a.wait_ns)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-#pragma unroll
-                    for (int ks = 0; ks < kCh / 16; ++ks)  // 16 keys: 8 P columns, +2 K-groups (2048 B) in V
-                        tc_mma_bf16_ts(tmem + t * 256 + 128, tmem + t * 256 + (j & 1) * kCh + ks * 8,
-                                       bd + (uint64_t)(2048 >> 4) * ks, kIdescPV, (j | ks) != 0);
-                    tc_commit(&o_full[t]);
-                    if (j == nc - 1) tc_commit(&o_last[t]);
-                }
-                if (!ok) break;
+                for (int ks = 0; ks < kCh / 16; ++ks)  // 16 keys: 8 P columns, +2 K-groups (2048 B) in V
+                    tc_mma_bf16_ts(tmem + 128, tmem + (j & 1) * kCh + ks * 8, bd + (uint64_t)(2048 >> 4) * ks,
+                                   kIdescPV, (j | ks) != 0);
+                tc_commit(o_full);
                 tc_commit(&v_empty[s]);
+                if (j == nc - 1) tc_commit(o_last);
             }
             if (!ok) {
-                // the last o_last was not committed (the loop left early):
-                // commit it now, so that it completes once every MMA this
-                // thread did issue has finished writing TMEM
+                // o_last was not committed (the loop left before the last
+                // chunk): commit it now, so that it completes once every MMA
+                // this thread did issue has finished writing TMEM
                 set_status(a.status, MEDUSA_STATUS_TIMEOUT);
-                tc_commit(&o_last[NT - 1]);
+                tc_commit(o_last);
             }
-            // every MMA done before TMEM is released (bounded): the last tile's
-            // o_last is this thread's last commit
-            mbar_wait(&o_last[NT - 1], 0);
+            mbar_wait(o_last, 0);  // every MMA done before TMEM is released (bounded)
         }
     } else {
         // ---------------- softmax ----------------
@@ -423,11 +394,11 @@ __global__ void __launch_bounds__(n_warps<NT>() * 32, ctas_per_sm<NT>())
 #pragma unroll
             for (int w = 0; w < 4; ++w) anc[w] = tree->anc[node][w];
         bool ok = true;
-        const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16) + tt * 256;
+        const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
         for (int j = 0; j < nc && ok; ++j) {
             // every wait before a warp-collective tcgen05 operation is decided
             // for the whole warp (its lanes test the barrier independently)
-            if (!__all_sync(kFull, mbar_wait(&s_full[tt * 2 + (j & 1)], (j >> 1) & 1, a.wait_ns))) {
+            if (!__all_sync(kFull, mbar_wait(&s_full[j & 1], (j >> 1) & 1, a.wait_ns))) {
                 ok = false;
                 break;
             }
@@ -498,9 +469,9 @@ __global__ void __launch_bounds__(n_warps<NT>() * 32, ctas_per_sm<NT>())
             }
             l = l * alpha + rs;
             // rescale this warp's rows of O when some row's reference max rose
-            // (after the tile's previous PV has completed)
+            // (after the previous PV has completed)
             if (j >= 1 && __any_sync(kFull, raise)) {
-                if (!__all_sync(kFull, mbar_wait(&o_full[tt], (j - 1) & 1, a.wait_ns))) {
+                if (!__all_sync(kFull, mbar_wait(o_full, (j - 1) & 1, a.wait_ns))) {
                     ok = false;
                     break;
                 }
@@ -525,12 +496,11 @@ __global__ void __launch_bounds__(n_warps<NT>() * 32, ctas_per_sm<NT>())
             }
             m = mn;
             const int key_end = tr ? Tb : S;
-            if (tt == 0 && key0 + kCh > key_end) {
+            if (key0 + kCh > key_end) {
                 // the chunk's rows past this sequence's keys (tree padding,
                 // another sequence's rows, page slots past the prefix, boxes
                 // not loaded) have P = 0, but a NaN in V would still reach O
-                // (0 * NaN), so tile 0's warps clear those V rows before its PV
-                // may start (the other tiles' PV is issued after tile 0's)
+                // (0 * NaN), so those V rows are cleared before PV may start
                 const int s = j % VS;
                 if (!__all_sync(kFull, mbar_wait(&v_full[s], (j / VS) & 1, a.wait_ns))) {
                     ok = false;
@@ -548,10 +518,10 @@ __global__ void __launch_bounds__(n_warps<NT>() * 32, ctas_per_sm<NT>())
             tmem_wait_st();  // P (and any rescaled O) in TMEM before the MMA reads it
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&p_full[tt * 2 + (j & 1)]);
+            if (lane == 0) mbar_arrive(&p_full[j & 1]);
         }
-        // final O (after the tile's last PV) for this row
-        if (ok && nc > 0) ok = __all_sync(kFull, mbar_wait(&o_last[tt], 0, a.wait_ns));
+        // final O (after the last PV) for this row
+        if (ok && nc > 0) ok = __all_sync(kFull, mbar_wait(o_last, 0, a.wait_ns));
         if (ok && nc > 0) {
             tc_fence_after();
 #pragma unroll
@@ -609,23 +579,22 @@ __global__ void __launch_bounds__(n_warps<NT>() * 32, ctas_per_sm<NT>())
         return;
     }
     // ---- several splits: each row's partial goes to the CTA that merges it ----
-    // Row r of the CTA (r = 128 t + tile row) is merged by the cluster's CTA
-    // r % C, as its row r / C.  After a first cluster barrier (every CTA's
-    // rings drained and free), each softmax thread stores its normalised
-    // partial row and its log-sum-exp (in the row's padding) into that CTA's
-    // receive buffer [C][RPC][OS], at [split][r / C]; after a second barrier
-    // each CTA merges its rows from local shared memory, in split order.
+    // Row r of the tile is merged by the cluster's CTA r % C, as its row
+    // r / C.  After a first cluster barrier (every CTA's K/V rings are drained
+    // and free), each softmax thread stores its normalised partial row and its
+    // log-sum-exp (in the row's padding) into that CTA's receive buffer
+    // [C][RPC][OS], at [split][r / C]; after a second barrier each CTA merges
+    // its rows from local shared memory, in split order.
     constexpr int OS = o_stride<D>();
-    const int RPC = (NT * kAM + C - 1) / C;      // rows merged per CTA
-    float* recv = reinterpret_cast<float*>(sQ);  // [C][RPC][OS] over Q and the drained K/V rings
-    const int nrows = min(NT * kAM, rows_T - row0);
-    const int rl = tt * kAM + lr;                // this thread's row of the CTA
+    const int RPC = (kAM + C - 1) / C;           // rows merged per CTA
+    float* recv = reinterpret_cast<float*>(sK);  // [C][RPC][OS] over the drained K/V rings
+    const int nrows = min(kAM, rows_T - mt * kAM);
     cg::cluster_group cl = cg::this_cluster();
     __syncwarp();  // the cluster barrier is an aligned one: whole warps
     cl.sync();     // every CTA of the cluster is past its main loop
-    if (warp >= 2 && rl < nrows) {
+    if (warp >= 2 && lr < nrows) {
         const float inv = l > 0.f ? 1.f / l : 0.f;
-        float* dst = cl.map_shared_rank(recv, rl % C) + ((long)split * RPC + rl / C) * OS;
+        float* dst = cl.map_shared_rank(recv, lr % C) + ((long)split * RPC + lr / C) * OS;
 #pragma unroll
         for (int e = 0; e < D; e += 4)
             *reinterpret_cast<float4*>(dst + e) = make_float4(o[e] * inv, o[e + 1] * inv, o[e + 2] * inv, o[e + 3] * inv);
@@ -634,11 +603,11 @@ __global__ void __launch_bounds__(n_warps<NT>() * 32, ctas_per_sm<NT>())
     __syncwarp();
     cl.sync();  // every partial row has arrived (the stores are released by the barrier)
     constexpr int PL = D / 32;  // elements of a row per lane
-    for (int i = warp; i * C + split < nrows; i += kW) {
+    for (int i = warp; i * C + split < nrows; i += kAW) {
         const int r = i * C + split;
-        const long orow = out_row(row0 + r);
+        const long orow = out_row(mt * kAM + r);
         __nv_bfloat16* dst = a.out + orow * D + lane * PL;
-        if (row0 + r >= Tb * a.G) {  // past this sequence's tree: zero output
+        if (mt * kAM + r >= Tb * a.G) {  // past this sequence's tree: zero output
 #pragma unroll
             for (int e = 0; e < PL; ++e) dst[e] = __float2bfloat16_rn(0.f);
             if (a.lse && lane == 0) a.lse[orow] = -INFINITY;
@@ -671,64 +640,22 @@ __global__ void __launch_bounds__(n_warps<NT>() * 32, ctas_per_sm<NT>())
     }
 }
 
-template <int D, int NT>
-constexpr size_t tc_attn_smem() {
-    // Q tiles, the K and V rings, the mbarriers, the TMEM address slot and the page-id ring
-    return (size_t)NT * kAM * D * 2 + (size_t)(k_stages<D, NT>() + v_stages<D, NT>()) * kCh * D * 2 +
-           n_bars<D, NT>() * 8 + 16 + kPageRing;
-}
-// the receive buffer ([C][ceil(128 NT / C)][OS] floats, at most 128 NT + 15
-// rows) fits over Q and the K/V rings
-template <int D, int NT>
-constexpr bool recv_fits() {
-    return (NT * kAM + kMaxCluster - 1) * o_stride<D>() * 4 <=
-           NT * kAM * D * 2 + (k_stages<D, NT>() + v_stages<D, NT>()) * kCh * D * 2;
-}
-static_assert(recv_fits<128, 1>() && recv_fits<128, 2>() && recv_fits<64, 1>() && recv_fits<64, 2>(),
-              "receive buffer");
-static_assert(tc_attn_smem<128, 2>() <= 227 * 1024 && 2 * tc_attn_smem<128, 1>() <= 228 * 1024, "shared memory");
-
-// query tiles per CTA: two when a (sequence, kv-head) has more than one tile's rows
-int tiles_per_cta(int T, int Hq, int Hkv) { return (long)T * (Hq / Hkv) > kAM ? 2 : 1; }
-
-template <int D, int NT>
-void set_attrs(int n_splits) {
-    auto k = tree_attn_tc_kernel<D, NT>;
-    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc_attn_smem<D, NT>());
-    cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-    if (n_splits > 8) cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-}
-
-// how many clusters of c CTAs of the two-tile kernel can be resident at once
-// (the hardware packs a cluster into one GPC), cached per device and size
 template <int D>
-int active_clusters(int c) {
-    static int cache[8][kMaxCluster + 1] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 8) dev = 0;
-    if (cache[dev][c]) return cache[dev][c];
-    set_attrs<D, 2>(c);
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(1, 1, c);
-    cfg.blockDim = dim3(n_warps<2>() * 32);
-    cfg.dynamicSmemBytes = tc_attn_smem<D, 2>();
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 1;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = c;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, tree_attn_tc_kernel<D, 2>, &cfg) != cudaSuccess || n < 1) {
-        (void)cudaGetLastError();
-        n = 1;
-    }
-    return cache[dev][c] = n;
+size_t tc_attn_smem() {
+    // Q, the K and V rings, the mbarriers, the TMEM address slot and the page-id ring
+    return (size_t)kAM * D * 2 + (size_t)(k_stages<D>() + v_stages<D>()) * kCh * D * 2 + n_bars<D>() * 8 + 16 +
+           kPageRing;
 }
+// the receive buffer ([C][ceil(128 / C)][OS] floats, at most 135 rows for
+// C <= 8) fits over the K/V rings
+static_assert((kAM + kMaxCluster - 1) * o_stride<128>() * 4 <= (k_stages<128>() + v_stages<128>()) * kCh * 128 * 2,
+              "receive buffer (D=128)");
+static_assert((kAM + kMaxCluster - 1) * o_stride<64>() * 4 <= (k_stages<64>() + v_stages<64>()) * kCh * 64 * 2,
+              "receive buffer (D=64)");
 
 }  // namespace
+
+int attn_tc_ctas_per_sm() { return kCtasPerSm; }
 
 bool attn_tc_page_ok(int page_size) {
     return page_size > 0 && (page_size % 64 == 0 || page_size == 8 || page_size == 16 || page_size == 32);
@@ -739,40 +666,26 @@ bool attn_tc_supported(int Hq, int Hkv, int D, int T, medusa_dtype dt) {
     return dt == MEDUSA_BF16 && (D == 64 || D == 128) && G >= 1 && G <= 16 && (G & (G - 1)) == 0 && T <= kMaxTree;
 }
 
-int attn_tc_m_tiles(int T, int Hq, int Hkv) {
-    const long rows = (long)T * (Hq / Hkv), per = (long)tiles_per_cta(T, Hq, Hkv) * kAM;
-    return (int)((rows + per - 1) / per);
-}
-
-// Key splits per CTA tile (a thread-block cluster).  One-tile CTAs (two per
-// SM): enough splits for two CTAs per SM, at most 8 (a cluster of 9 at two
-// CTAs per SM did not pack into the GPCs: measured, the 288 CTAs of llama8b
-// ran in two waves).  Two-tile CTAs (one per SM): the largest cluster, up to
-// 16, of which every one of the grid's clusters is resident at once (asked
-// of the occupancy calculator).  Never more than the chunks of the longest
-// sequence, nor than medusa_set_launch_shape's cap.
-int attn_tc_splits(int B, int T, int Hq, int Hkv, int D, int max_prefix) {
-    const int NT = tiles_per_cta(T, Hq, Hkv);
-    const long groups = (long)attn_tc_m_tiles(T, Hq, Hkv) * B * Hkv;
+// Key splits per 128-row tile: enough CTAs for two per SM, at most a portable
+// cluster of 8 (a cluster of 9 CTAs at two per SM does not pack into the GPCs:
+// measured, the 288 CTAs of llama8b ran in two waves) and at most the chunks
+// of the longest sequence.
+int attn_tc_splits(int B, int T, int Hq, int Hkv, int max_prefix) {
+    const int G = Hq / Hkv;
+    const long m_tiles = ((long)T * G + kAM - 1) / kAM;
+    const long per_split = m_tiles * B * Hkv;
+    const long target = (long)kCtasPerSm * num_sms();
+    long c = (target + per_split - 1) / per_split;
     const long chunks = (max_prefix + kCh - 1) / kCh + (T + kCh - 1) / kCh;
-    long hi = kMaxCluster;
-    if (hi > chunks) hi = chunks;
+    if (c > kMaxCluster) c = kMaxCluster;
+    if (c > chunks) c = chunks;
     const int cap = launch_attention_splits();
-    if (cap > 0 && hi > cap) hi = cap;
-    if (NT == 1) {
-        long c = (2L * num_sms() + groups - 1) / groups;
-        if (c > 8) c = 8;
-        if (c > hi) c = hi;
-        return c < 1 ? 1 : (int)c;
-    }
-    for (long c = hi; c >= 2; --c)
-        if (groups <= (D == 128 ? active_clusters<128>((int)c) : active_clusters<64>((int)c))) return (int)c;
-    return 1;
+    if (cap > 0 && c > cap) c = cap;
+    return c < 1 ? 1 : (int)c;
 }
 
-// launch the tensor-core kernel: m_tiles CTA tiles per (sequence, kv-head) of
-// tiles_per_cta 128-row tiles each, n_splits key splits per CTA tile (one
-// cluster); writes the output (and lse)
+// launch the tensor-core kernel: m_tiles 128-row tiles per (sequence, kv-head),
+// n_splits key splits per tile (one cluster); writes the output (and lse)
 cudaError_t attn_tc_launch(const AttnArgs& x, int m_tiles, int n_splits, float scale_log2, cudaStream_t st) {
     TcAttnArgs a;
     const uint64_t D = x.D, Hq = x.Hq, Hkv = x.Hkv, BT = (uint64_t)x.B * x.T, Smax = x.S_max, BH = (uint64_t)x.B * x.Hkv;
@@ -824,10 +737,9 @@ cudaError_t attn_tc_launch(const AttnArgs& x, int m_tiles, int n_splits, float s
     a.max_prefix = x.max_prefix;
     a.scale_log2 = scale_log2;
     a.wait_ns = wait_limit_ns();
-    const int NT = tiles_per_cta(x.T, x.Hq, x.Hkv);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(m_tiles, (unsigned)BH, n_splits);
-    cfg.blockDim = dim3((NT == 2 ? n_warps<2>() : n_warps<1>()) * 32);
+    cfg.blockDim = dim3(kAW * 32);
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -837,23 +749,17 @@ cudaError_t attn_tc_launch(const AttnArgs& x, int m_tiles, int n_splits, float s
     cfg.attrs = attr;
     cfg.numAttrs = n_splits > 1 ? 1 : 0;
     if (x.D == 128) {
-        if (NT == 2) {
-            set_attrs<128, 2>(n_splits);
-            cfg.dynamicSmemBytes = tc_attn_smem<128, 2>();
-            return cudaLaunchKernelEx(&cfg, tree_attn_tc_kernel<128, 2>, a);
-        }
-        set_attrs<128, 1>(n_splits);
-        cfg.dynamicSmemBytes = tc_attn_smem<128, 1>();
-        return cudaLaunchKernelEx(&cfg, tree_attn_tc_kernel<128, 1>, a);
+        cfg.dynamicSmemBytes = tc_attn_smem<128>();
+        cudaFuncSetAttribute(tree_attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)cfg.dynamicSmemBytes);
+        cudaFuncSetAttribute(tree_attn_tc_kernel<128>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+        return cudaLaunchKernelEx(&cfg, tree_attn_tc_kernel<128>, a);
     }
-    if (NT == 2) {
-        set_attrs<64, 2>(n_splits);
-        cfg.dynamicSmemBytes = tc_attn_smem<64, 2>();
-        return cudaLaunchKernelEx(&cfg, tree_attn_tc_kernel<64, 2>, a);
-    }
-    set_attrs<64, 1>(n_splits);
-    cfg.dynamicSmemBytes = tc_attn_smem<64, 1>();
-    return cudaLaunchKernelEx(&cfg, tree_attn_tc_kernel<64, 1>, a);
+    cfg.dynamicSmemBytes = tc_attn_smem<64>();
+    cudaFuncSetAttribute(tree_attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)cfg.dynamicSmemBytes);
+    cudaFuncSetAttribute(tree_attn_tc_kernel<64>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    return cudaLaunchKernelEx(&cfg, tree_attn_tc_kernel<64>, a);
 }
 
 }  // namespace medusa

@@ -71,12 +71,11 @@ size_t attn_workspace_size(int B, int T, int Hq, int Hkv, int D, int max_prefix,
 cudaError_t attn_launch(const AttnArgs& a, cudaStream_t st);
 // tensor-core split kernel (bf16, D in {64,128}, power-of-two group size <= 16)
 bool attn_tc_supported(int Hq, int Hkv, int D, int T, medusa_dtype dt);
+int attn_tc_ctas_per_sm();
 // page sizes the tensor-core kernel reads (multiples of 64, or 8, 16, 32)
 bool attn_tc_page_ok(int page_size);
-// CTA tiles per (sequence, kv-head) (one or two 128-row tiles each) and key
-// splits per CTA tile (the CTAs of one cluster, at most 16)
-int attn_tc_m_tiles(int T, int Hq, int Hkv);
-int attn_tc_splits(int B, int T, int Hq, int Hkv, int D, int max_prefix);
+// key splits per 128-row tile (the CTAs of one cluster, at most 8)
+int attn_tc_splits(int B, int T, int Hq, int Hkv, int max_prefix);
 // writes the output (and lse) itself: the splits merge inside their cluster
 cudaError_t attn_tc_launch(const AttnArgs& a, int m_tiles, int n_splits, float scale_log2, cudaStream_t st);
 

@@ -53,6 +53,7 @@ CASES = [
     ("stoch_b64", dict(B=4), "workload", None),                             # 32-node random tree, S=1024
     ("llama8b", dict(prefix=200), (1, 1, 1, 1, 1, 1, 1), None),             # chain tree (causal)
     ("llama8b", dict(prefix=77), (), None),                                 # T=1: plain decode
+    ("llama8b", dict(B=2, Hq=16, Hkv=4, D=64, prefix=700), (4, 4, 2, 2), [700, 65]),  # D=64, two tiles per CTA
 ]
 
 
