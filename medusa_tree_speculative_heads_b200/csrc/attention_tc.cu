@@ -117,8 +117,11 @@ __device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t smem_byte_addr, 
     return d;
 }
 
-template <int D>
+// kTestWaits: the protocol waits take their limit from the arguments (a
+// shortened limit set to test the error paths); otherwise it is the constant
+template <int D, bool kTestWaits>
 __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(const __grid_constant__ TcAttnArgs a) {
+    const uint64_t wait_ns = kTestWaits ? a.wait_ns : kWaitLimitNs;
     constexpr int NSUB = D / 64;              // 64-element blocks along D
     constexpr int kQBytes = kAM * D * 2;
     constexpr int kSub = kCh * 128;           // [64 keys x 64 D] block = 8 KB
@@ -314,7 +317,7 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
                 if (prog) {
                     idle = 0;
                     t0 = global_ns();
-                } else if ((++idle & 255u) == 0 && global_ns() - t0 > a.wait_ns) {
+                } else if ((++idle & 255u) == 0 && global_ns() - t0 > wait_ns) {
                     set_status(a.status, MEDUSA_STATUS_TIMEOUT);
                     break;
                 }
@@ -334,13 +337,13 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
         if (lane == 0 && nc > 0) {
-            bool ok = mbar_wait(q_full, 0, a.wait_ns);
+            bool ok = mbar_wait(q_full, 0, wait_ns);
             // S_j goes to TMEM columns (j&1)*64; P_j is written over it, so the
             // buffer is free for S_{j+2} once PV_j has completed (o_full phase j)
             auto issue_qk = [&](int j) -> bool {
                 const int s = j % KS, sb = j & 1;
-                if (!mbar_wait(&k_full[s], (j / KS) & 1, a.wait_ns)) return false;
-                if (j >= 2 && !mbar_wait(o_full, (j - 2) & 1, a.wait_ns)) return false;
+                if (!mbar_wait(&k_full[s], (j / KS) & 1, wait_ns)) return false;
+                if (j >= 2 && !mbar_wait(o_full, (j - 2) & 1, wait_ns)) return false;
                 tc_fence_after();
 #pragma unroll
                 for (int sub = 0; sub < NSUB; ++sub) {
@@ -357,12 +360,12 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
             if (ok) ok = issue_qk(0);
             for (int j = 0; j < nc && ok; ++j) {
                 if (j + 1 < nc && !(ok = issue_qk(j + 1))) break;
-                if (!mbar_wait(&p_full[j & 1], (j >> 1) & 1, a.wait_ns)) {
+                if (!mbar_wait(&p_full[j & 1], (j >> 1) & 1, wait_ns)) {
                     ok = false;
                     break;
                 }
                 const int s = j % VS;
-                if (!mbar_wait(&v_full[s], (j / VS) & 1, a.wait_ns)) {
+                if (!mbar_wait(&v_full[s], (j / VS) & 1, wait_ns)) {
                     ok = false;
                     break;
                 }
@@ -398,7 +401,7 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
         for (int j = 0; j < nc && ok; ++j) {
             // every wait before a warp-collective tcgen05 operation is decided
             // for the whole warp (its lanes test the barrier independently)
-            if (!__all_sync(kFull, mbar_wait(&s_full[j & 1], (j >> 1) & 1, a.wait_ns))) {
+            if (!__all_sync(kFull, mbar_wait(&s_full[j & 1], (j >> 1) & 1, wait_ns))) {
                 ok = false;
                 break;
             }
@@ -471,7 +474,7 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
             // rescale this warp's rows of O when some row's reference max rose
             // (after the previous PV has completed)
             if (j >= 1 && __any_sync(kFull, raise)) {
-                if (!__all_sync(kFull, mbar_wait(o_full, (j - 1) & 1, a.wait_ns))) {
+                if (!__all_sync(kFull, mbar_wait(o_full, (j - 1) & 1, wait_ns))) {
                     ok = false;
                     break;
                 }
@@ -502,7 +505,7 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
                 // not loaded) have P = 0, but a NaN in V would still reach O
                 // (0 * NaN), so those V rows are cleared before PV may start
                 const int s = j % VS;
-                if (!__all_sync(kFull, mbar_wait(&v_full[s], (j / VS) & 1, a.wait_ns))) {
+                if (!__all_sync(kFull, mbar_wait(&v_full[s], (j / VS) & 1, wait_ns))) {
                     ok = false;
                     break;
                 }
@@ -521,7 +524,7 @@ __global__ void __launch_bounds__(kAW * 32, kCtasPerSm) tree_attn_tc_kernel(cons
             if (lane == 0) mbar_arrive(&p_full[j & 1]);
         }
         // final O (after the last PV) for this row
-        if (ok && nc > 0) ok = __all_sync(kFull, mbar_wait(o_last, 0, a.wait_ns));
+        if (ok && nc > 0) ok = __all_sync(kFull, mbar_wait(o_last, 0, wait_ns));
         if (ok && nc > 0) {
             tc_fence_after();
 #pragma unroll
@@ -653,6 +656,12 @@ static_assert((kAM + kMaxCluster - 1) * o_stride<128>() * 4 <= (k_stages<128>() 
 static_assert((kAM + kMaxCluster - 1) * o_stride<64>() * 4 <= (k_stages<64>() + v_stages<64>()) * kCh * 64 * 2,
               "receive buffer (D=64)");
 
+cudaError_t launch_attn(void (*kern)(TcAttnArgs), cudaLaunchConfig_t& cfg, const TcAttnArgs& a) {
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cfg.dynamicSmemBytes);
+    cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
 }  // namespace
 
 int attn_tc_ctas_per_sm() { return kCtasPerSm; }
@@ -748,18 +757,13 @@ cudaError_t attn_tc_launch(const AttnArgs& x, int m_tiles, int n_splits, float s
     attr[0].val.clusterDim.z = n_splits;
     cfg.attrs = attr;
     cfg.numAttrs = n_splits > 1 ? 1 : 0;
+    const bool test_waits = a.wait_ns != kWaitLimitNs;
     if (x.D == 128) {
         cfg.dynamicSmemBytes = tc_attn_smem<128>();
-        cudaFuncSetAttribute(tree_attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)cfg.dynamicSmemBytes);
-        cudaFuncSetAttribute(tree_attn_tc_kernel<128>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-        return cudaLaunchKernelEx(&cfg, tree_attn_tc_kernel<128>, a);
+        return launch_attn(test_waits ? tree_attn_tc_kernel<128, true> : tree_attn_tc_kernel<128, false>, cfg, a);
     }
     cfg.dynamicSmemBytes = tc_attn_smem<64>();
-    cudaFuncSetAttribute(tree_attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)cfg.dynamicSmemBytes);
-    cudaFuncSetAttribute(tree_attn_tc_kernel<64>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-    return cudaLaunchKernelEx(&cfg, tree_attn_tc_kernel<64>, a);
+    return launch_attn(test_waits ? tree_attn_tc_kernel<64, true> : tree_attn_tc_kernel<64, false>, cfg, a);
 }
 
 }  // namespace medusa

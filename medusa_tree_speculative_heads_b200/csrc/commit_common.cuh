@@ -56,16 +56,34 @@ static __device__ __noinline__ void commit_path(int b, const int* s_node, int L,
     __syncthreads();
     const bool ok = s_ok;
     if (ok) {
+        // four rows' K and V loads in flight per thread before any store
+        constexpr int kBatch = 4;
         const int vecs = row_bytes / 16;
         const int per_t = Hkv * vecs;
-        for (int e = tid; e < L * per_t; e += blockDim.x) {
-            const int t = e / per_t, rem = e % per_t;
-            const int g = rem / vecs, c = rem % vecs;
-            const long src = (((long)b * T + s_node[t]) * Hkv + g) * row_bytes + c * 16;
-            const long dst = table ? (((long)s_page[t] * Hkv + g) * page_size + (S + t) % page_size) * row_bytes + c * 16
+        const int total = L * per_t;
+        for (int e0 = tid; e0 < total; e0 += kBatch * blockDim.x) {
+            uint4 kr[kBatch], vr[kBatch];
+            long dst[kBatch];
+#pragma unroll
+            for (int j = 0; j < kBatch; ++j) {
+                const int e = e0 + j * blockDim.x;
+                if (e < total) {
+                    const int t = e / per_t, rem = e % per_t;
+                    const int g = rem / vecs, c = rem % vecs;
+                    const long src = (((long)b * T + s_node[t]) * Hkv + g) * row_bytes + c * 16;
+                    dst[j] = table ? (((long)s_page[t] * Hkv + g) * page_size + (S + t) % page_size) * row_bytes + c * 16
                                    : (((long)b * Hkv + g) * S_max + S + t) * row_bytes + c * 16;
-            *reinterpret_cast<uint4*>(kc + dst) = *reinterpret_cast<const uint4*>(kt + src);
-            *reinterpret_cast<uint4*>(vc + dst) = *reinterpret_cast<const uint4*>(vt + src);
+                    kr[j] = *reinterpret_cast<const uint4*>(kt + src);
+                    vr[j] = *reinterpret_cast<const uint4*>(vt + src);
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < kBatch; ++j) {
+                if (e0 + j * blockDim.x < total) {
+                    *reinterpret_cast<uint4*>(kc + dst[j]) = kr[j];
+                    *reinterpret_cast<uint4*>(vc + dst[j]) = vr[j];
+                }
+            }
         }
     }
     if (tid == 0) new_prefix_len[b] = ok ? S + L : S;

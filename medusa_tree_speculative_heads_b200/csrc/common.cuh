@@ -98,6 +98,10 @@ struct Elt<float> {
     }
     __device__ __forceinline__ static float to_float(float x) { return x; }
     __device__ __forceinline__ static float from_float(float x) { return x; }
+    // the largest of the vector's elements; NaN only when all are NaN
+    __device__ __forceinline__ static float vmax(const uint4& v) {
+        return fmaxf(fmaxf(__uint_as_float(v.x), __uint_as_float(v.y)), fmaxf(__uint_as_float(v.z), __uint_as_float(v.w)));
+    }
 };
 template <>
 struct Elt<__nv_bfloat16> {
@@ -114,6 +118,18 @@ struct Elt<__nv_bfloat16> {
     }
     __device__ __forceinline__ static float to_float(__nv_bfloat16 x) { return __bfloat162float(x); }
     __device__ __forceinline__ static __nv_bfloat16 from_float(float x) { return __float2bfloat16_rn(x); }
+    // the largest of the vector's elements (exact: a maximum rounds nothing);
+    // the paired maximum returns the other operand when one is NaN, so the
+    // result is NaN only when all eight are
+    __device__ __forceinline__ static float vmax(const uint4& v) {
+        const __nv_bfloat162 m = __hmax2(__hmax2(pair(v.x), pair(v.y)), __hmax2(pair(v.z), pair(v.w)));
+        return fmaxf(__low2float(m), __high2float(m));
+    }
+    __device__ __forceinline__ static __nv_bfloat162 pair(uint32_t u) {
+        __nv_bfloat162 r;
+        memcpy(&r, &u, 4);
+        return r;
+    }
 };
 
 // ---------------------------------------------------------------------------

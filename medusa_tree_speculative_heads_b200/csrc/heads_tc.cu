@@ -62,6 +62,8 @@ constexpr int kTS = kTM + 1;             // transposed tile: column stride in fl
 // head is done; above it (one CTA would hold up the end with the merges of
 // many sequences) after a grid barrier, spread over every warp of the grid
 constexpr int kMergePerHeadMaxB = 4;
+// L2 prefetch distance of the weight stream, in quarters of the ring depth
+constexpr int kPrefetchAheadX4 = 0;
 
 // row segments per column in the transposed epilogue (at most 16, so that a
 // column's flush merges few partial states)
@@ -90,7 +92,7 @@ struct TcHeadsArgs {
     int B, d, V, K;
     int stages;
     int merge_per_head;  // B <= kMergePerHeadMaxB: each head merged by its last CTA; else after a grid barrier
-    uint64_t wait_ns;    // limit of the pipeline waits (drains of issued work: kWaitLimitNs)
+    uint64_t wait_ns;    // limit of the pipeline waits when it differs from kWaitLimitNs (drains: kWaitLimitNs)
 };
 
 // A CTA's run of one phase: k-block units [u0, u1) of the phase's tiles laid
@@ -131,8 +133,13 @@ __device__ __forceinline__ void epi_sync() {
     asm volatile("bar.sync 2, 128;" ::: "memory");
 }
 
-template <int N>
+// kTestWaits: the waits take their limit from the arguments (a shortened limit
+// set to test the error paths); otherwise the limit is the constant one, which
+// keeps the pipeline loops free of the run-time choice (a measurable cost in
+// the weight stream)
+template <int N, bool kTestWaits>
 __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid_constant__ TcHeadsArgs a) {
+    const uint64_t wait_ns = kTestWaits ? a.wait_ns : kWaitLimitNs;
     constexpr int kBBytes = N * kTK * 2;  // batch tile per stage (multiple of 1024)
     constexpr int kTmemCols = N * 2 <= 32 ? 32 : N * 2 <= 64 ? 64 : 128;
     constexpr uint32_t kIdesc = idesc_bf16_f32(kTM, N);
@@ -202,6 +209,30 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
             const uint32_t bytes = weights ? kABytes : kBBytes;
             int it = 0;  // k-blocks issued (ring position)
             bool ok = true;
+            // The weight producer also asks L2 for the weight tile `ahead`
+            // k-blocks past the one it loads: the ring alone keeps S tiles in
+            // flight, which under a full HBM stream is the whole latency-bandwidth
+            // budget of the SM; L2 prefetches extend it without shared memory.
+            int pli = 0, pkb = 0, pkb1 = 0, pu = 0;  // prefetch cursor: piece, k-block, end, unit
+            long pt = 0;
+            if (ntiles > 0) piece(0, pt, pkb, pkb1);
+            auto prefetch_upto = [&](int target, bool issue) {
+                while (pu < target && pli < ntiles) {
+                    if (pkb >= pkb1) {
+                        if (++pli < ntiles) piece(pli, pt, pkb, pkb1);
+                        continue;
+                    }
+                    if (issue) {
+                        const bool r = pli < n1;
+                        tma_prefetch_l2_3d(r ? &a.mW_res : &a.mW_head, pkb * kTK,
+                                           (int)(r ? pt % tph_r : pt % tph_l) * kTM, (int)(r ? pt / tph_r : pt / tph_l));
+                    }
+                    ++pkb;
+                    ++pu;
+                }
+            };
+            const int ahead = kPrefetchAheadX4 * S / 4;
+            if (weights) prefetch_upto(S, false);  // the first S k-blocks are loaded at once
             for (int li = 0; li < ntiles && ok; ++li) {
                 const bool res = li < n1;
                 long t;
@@ -213,7 +244,7 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
                     // vocabulary tiles read h^(k): wait until every CTA wrote its rows
                     const uint64_t t0 = global_ns();
                     while (ld_acquire_u32(&a.ctr[0]) < gridDim.x) {
-                        if (global_ns() - t0 > a.wait_ns) {
+                        if (global_ns() - t0 > wait_ns) {
                             set_status(a.status, MEDUSA_STATUS_TIMEOUT);
                             ok = false;
                             break;
@@ -225,11 +256,12 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
                 }
                 for (int kb = kb0; kb < kb1; ++kb) {
                     const int s = it % S;
-                    if (it >= S && !mbar_wait(&empty[s], ((it / S) - 1) & 1, a.wait_ns)) {
+                    if (it >= S && !mbar_wait(&empty[s], ((it / S) - 1) & 1, wait_ns)) {
                         set_status(a.status, MEDUSA_STATUS_TIMEOUT);
                         ok = false;
                         break;
                     }
+                    if (weights && ahead > 0) prefetch_upto(it + ahead, true);
                     mbar_arrive_expect_tx(&full[s], bytes);
                     if (weights)
                         tma_load_3d(sA + (size_t)s * kABytes, res ? &a.mW_res : &a.mW_head, kb * kTK, row0, k,
@@ -261,7 +293,7 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
             int it = 0;
             for (int li = 0; li < ntiles && ok; ++li) {
                 const int buf = li & 1;
-                if (li >= 2 && !mbar_wait(&acc_empty[buf], ((li >> 1) - 1) & 1, a.wait_ns)) {
+                if (li >= 2 && !mbar_wait(&acc_empty[buf], ((li >> 1) - 1) & 1, wait_ns)) {
                     set_status(a.status, MEDUSA_STATUS_TIMEOUT);
                     break;
                 }
@@ -272,7 +304,7 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
                 piece(li, t, kb0, kb1);
                 for (int kb = kb0; kb < kb1; ++kb) {
                     const int s = it % S;
-                    if (!mbar_wait(&full[s], (it / S) & 1, a.wait_ns)) {
+                    if (!mbar_wait(&full[s], (it / S) & 1, wait_ns)) {
                         set_status(a.status, MEDUSA_STATUS_TIMEOUT);
                         ok = false;
                         break;
@@ -434,7 +466,7 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
         if (n1 == 0) arrive_grid();
         for (int li = 0; li < ntiles; ++li) {
             const int buf = li & 1;
-            if (ok && !mbar_wait(&acc_full[buf], (li >> 1) & 1, a.wait_ns)) {
+            if (ok && !mbar_wait(&acc_full[buf], (li >> 1) & 1, wait_ns)) {
                 if (lane == 0) set_status(a.status, MEDUSA_STATUS_TIMEOUT);
                 ok = false;
             }
@@ -481,7 +513,7 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
                 const long U = ph == 0 ? U1 : U2, tend = (t + 1) * nkb;
                 for (int c2 = cta + 1; c2 < G && U * c2 / G < tend; ++c2) {
                     if (U * (c2 + 1) / G == U * c2 / G) continue;  // an empty run
-                    if (!wait_flag(&a.ctr[2 + ph * G + c2], a.wait_ns)) {
+                    if (!wait_flag(&a.ctr[2 + ph * G + c2], wait_ns)) {
                         if (lane == 0) set_status(a.status, MEDUSA_STATUS_TIMEOUT);
                         ok = false;
                         break;
@@ -568,7 +600,7 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
         atomicAdd(&a.ctr[1], 1u);
         const uint64_t t0 = global_ns();
         while (ld_acquire_u32(&a.ctr[1]) < gridDim.x) {
-            if (global_ns() - t0 > a.wait_ns) {
+            if (global_ns() - t0 > wait_ns) {
                 set_status(a.status, MEDUSA_STATUS_TIMEOUT);
                 *last_flag = 1;
                 break;
@@ -606,7 +638,7 @@ cudaError_t launch_n(const TcHeadsArgs& args, cudaStream_t st) {
     TcHeadsArgs a = args;
     a.stages = tc_stages<N>(a.B);
     const size_t smem = tc_smem_bytes<N>(a.stages, a.B);
-    auto kern = heads_tc_kernel<N>;
+    auto kern = a.wait_ns == kWaitLimitNs ? heads_tc_kernel<N, false> : heads_tc_kernel<N, true>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     prefer_max_smem(kern);

@@ -53,7 +53,12 @@ __device__ __forceinline__ void argmax_merge(float& bv, int& bi, float v, int i)
 }
 
 // Row argmax partials over vocabulary chunks, one block per (row, chunk),
-// 8 independent 16-byte loads in flight per thread.
+// 8 independent 16-byte loads in flight per thread.  A thread visits its
+// vectors in increasing index order and keeps the first vector whose maximum
+// beats everything before it (the vector maximum is a paired max, a few
+// instructions per eight logits instead of a compare-and-select per logit);
+// the winning element is the vector's first one equal to that maximum, so
+// ties go to the lowest index and NaN never wins, as in `beats`.
 template <typename E>
 __global__ void __launch_bounds__(kArgmaxThreads, 4) row_argmax_kernel(const E* __restrict__ x, int V, int splits,
                                                                     int chunk, float* __restrict__ pval,
@@ -73,6 +78,8 @@ __global__ void __launch_bounds__(kArgmaxThreads, 4) row_argmax_kernel(const E* 
         int va = v0;
         if ((((uintptr_t)(rp + v0)) & 15) == 0) {
             const int nvec = (v1 - v0) / VEC;
+            int bc = -1;      // the thread's winning vector
+            uint4 braw = make_uint4(0, 0, 0, 0);
             for (int c0 = threadIdx.x; c0 < nvec; c0 += U * kArgmaxThreads) {
                 uint4 raw[U];
 #pragma unroll
@@ -83,13 +90,22 @@ __global__ void __launch_bounds__(kArgmaxThreads, 4) row_argmax_kernel(const E* 
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
                     const int c = c0 + u * kArgmaxThreads;
-                    if (c < nvec) {
-                        float f[VEC];
-                        Elt<E>::unpack(raw[u], f);
-#pragma unroll
-                        for (int e = 0; e < VEC; ++e) argmax_merge(bv, bi, f[e], v0 + c * VEC + e);
+                    const float mv = Elt<E>::vmax(raw[u]);
+                    if (c < nvec && mv > bv) {
+                        bv = mv;
+                        bc = c;
+                        braw = raw[u];
                     }
                 }
+            }
+            if (bc >= 0) {
+                float f[VEC];
+                Elt<E>::unpack(braw, f);
+                int e = 0;
+#pragma unroll
+                for (int i = VEC - 1; i >= 0; --i)
+                    if (f[i] == bv) e = i;
+                bi = v0 + bc * VEC + e;
             }
             va = v0 + nvec * VEC;
         }

@@ -67,6 +67,49 @@ def test_greedy_ties_nan_and_float32():
         assert out["accept_len"].tolist() == [3, 3]
 
 
+@pytest.mark.parametrize("dt", [torch.bfloat16, torch.float32])
+def test_greedy_argmax_edges_full_vocab(dt):
+    # the row maxima sit next to NaN in the same 16-byte vector, tie across
+    # vocabulary splits and between -0.0 and +0.0, or are -inf; the kernel's
+    # per-vector maximum must pick what a plain scan picks.  The tree is a
+    # chain whose every token is its parent's prediction, so each row's
+    # argmax decides the accepted length (or the bonus token).
+    T, V = 7, 32000
+    parents = [-1] + list(range(T - 1))
+    g = np.random.default_rng(11)
+    z = torch.from_numpy(g.standard_normal((2, T, V)).astype(np.float32))
+    z[0, 0, 100:108] = float("nan")
+    z[0, 0, 103] = 9.0                  # the maximum among NaNs of its vector
+    z[0, 1, 30001] = 8.0                # equal maxima in different splits: the lower index
+    z[0, 1, 5] = 8.0
+    z[0, 2, :] = -float("inf")          # nothing beats -inf: index 0
+    z[0, 3, :] = -1.0
+    z[0, 3, 17] = -0.0                  # -0.0 and +0.0 are equal: the lower index
+    z[0, 3, 21] = 0.0
+    z[0, 4, :] = float("nan")
+    z[0, 4, V - 1] = -5.0               # the last logit of the row, the rest NaN
+    z[0, 5, 8:16] = 7.0                 # a whole vector of equal maxima: its first
+    z[0, 6, 24] = 50.0
+    z[1, 0, 7] = float("inf")
+    z[1, 0, 6] = float("inf")           # two +inf: the lower index
+    z[1, 1, :] = float("nan")           # all NaN: index 0
+    z = z.to(dt)
+    zf = z.float()
+    pred = np.zeros((2, T), np.int64)
+    for b in range(2):
+        for r in range(T):
+            row = zf[b, r]
+            ok = ~torch.isnan(row)
+            pred[b, r] = int(torch.nonzero(row == row[ok].max())[0]) if ok.any() else 0
+    assert pred[0].tolist() == [103, 5, 0, 17, V - 1, 8, 24] and pred[1, :2].tolist() == [6, 0]
+    tok = torch.zeros((2, T), dtype=torch.int32)
+    tok[:, 1:] = torch.from_numpy(pred[:, :-1].astype(np.int32))
+    out = run_greedy(parents, tok, z)
+    ref = oracle.verify_greedy(z, tok, parents, max_path=T)
+    assert_same(out, ref)
+    assert out["accept_len"].tolist() == [T, T] and out["bonus"].tolist() == pred[:, -1].tolist()
+
+
 def test_greedy_draft_equals_target_full_vocab():
     w = I.scaled(I.WORKLOADS["llama8b"], B=2)
     parents = I.workload_tree(w)
