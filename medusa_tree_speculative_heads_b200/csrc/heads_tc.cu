@@ -62,12 +62,50 @@ constexpr int kTS = kTM + 1;             // transposed tile: column stride in fl
 // head is done; above it (one CTA would hold up the end with the merges of
 // many sequences) after a grid barrier, spread over every warp of the grid
 constexpr int kMergePerHeadMaxB = 4;
-// L2 prefetch distance of the weight stream, in quarters of the ring depth
-constexpr int kPrefetchAheadX4 = 0;
 
-// row segments per column in the transposed epilogue (at most 16, so that a
-// column's flush merges few partial states)
+// The vocabulary epilogue splits a tile's B columns (sequences) x 128 rows
+// into units of one column and 128 / R rows, R = row blocks per column (4 for
+// one sequence, 2 for two, else 1), so that B >= 4 gives B units and fewer
+// sequences still give the four epilogue warps one unit each; unit u is
+// column u / R, row block u % R, taken by warp u % 4.
+__host__ __device__ constexpr int row_blocks(int B) { return B >= 4 ? 1 : B == 1 ? 4 : 2; }
+// Above 32 sequences each warp would take 9..16 units, and a unit's top-8
+// list starts empty in every CTA and head (about 30 insertions per column,
+// each a warp-wide step), so there each thread takes one column segment of
+// 128 / seg_per_col(B) rows instead: its running statistics and top-8 list
+// stay in registers; a tile's candidates (rows beating the list's last entry
+// when the tile starts) are queued in shared memory and inserted after the
+// scan, so a warp runs as many insertions as its longest queue, not one per
+// row in which any lane inserts.
+template <int N> constexpr bool units_epilogue() { return N <= 32; }
 __host__ __device__ constexpr int seg_per_col(int B) { return 128 / B < 16 ? 128 / B : 16; }
+__host__ __device__ constexpr int epi_blocks(int B, bool units) { return units ? row_blocks(B) : seg_per_col(B); }
+
+struct TopEntry {
+    float v;
+    int i;
+};
+
+// Insert (v, i) into a top-kTopK list held across a warp, lane j < kTopK
+// holding the j-th best (lanes past kTopK hold -inf and never change).  The
+// entries the new item beats are a suffix of the sorted list; it takes the
+// first of them and the rest move down one lane.
+__device__ __forceinline__ void warp_list_insert(float& lv, int& li, float v, int i) {
+    const int lane = threadIdx.x & 31;
+    const unsigned worse = __ballot_sync(kFull, beats(v, i, lv, li)) & ((1u << kTopK) - 1u);
+    const float uv = __shfl_up_sync(kFull, lv, 1);
+    const int ui = __shfl_up_sync(kFull, li, 1);
+    if (worse) {
+        const int p = __ffs(worse) - 1;
+        if (lane == p) {
+            lv = v;
+            li = i;
+        } else if (lane > p && lane < kTopK) {
+            lv = uv;
+            li = ui;
+        }
+    }
+}
 
 struct TcHeadsArgs {
     CUtensorMap mW_res;   // W_res  as (d_in, d_out, K), box (64, 128, 1)
@@ -161,7 +199,12 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
     int* last_flag = reinterpret_cast<int*>(tmem_slot + 1);  // this CTA merges the head it just flushed
     float* sT = reinterpret_cast<float*>(tmem_slot + 4);  // [B][kTS] transposed tile
-    HeadState* stS = reinterpret_cast<HeadState*>(sT + ((a.B * kTS + 3) & ~3));  // [seg][B] flush states
+    HeadState* stS = reinterpret_cast<HeadState*>(sT + ((a.B * kTS + 3) & ~3));  // [row block][B] flush states
+    constexpr bool kUnits = units_epilogue<N>();
+    const int nunits = a.B * epi_blocks(a.B, kUnits);  // units, or column segments
+    float2* sU = reinterpret_cast<float2*>(stS + nunits);       // [unit][lane] running (max, sum)
+    TopEntry* sL = reinterpret_cast<TopEntry*>(sU + nunits * 32);  // [unit][kTopK] top list, best first
+    uint8_t* sQ = reinterpret_cast<uint8_t*>(stS + nunits);     // segments: [slot][128 threads] candidate rows
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int K = a.K, B = a.B;
@@ -209,30 +252,6 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
             const uint32_t bytes = weights ? kABytes : kBBytes;
             int it = 0;  // k-blocks issued (ring position)
             bool ok = true;
-            // The weight producer also asks L2 for the weight tile `ahead`
-            // k-blocks past the one it loads: the ring alone keeps S tiles in
-            // flight, which under a full HBM stream is the whole latency-bandwidth
-            // budget of the SM; L2 prefetches extend it without shared memory.
-            int pli = 0, pkb = 0, pkb1 = 0, pu = 0;  // prefetch cursor: piece, k-block, end, unit
-            long pt = 0;
-            if (ntiles > 0) piece(0, pt, pkb, pkb1);
-            auto prefetch_upto = [&](int target, bool issue) {
-                while (pu < target && pli < ntiles) {
-                    if (pkb >= pkb1) {
-                        if (++pli < ntiles) piece(pli, pt, pkb, pkb1);
-                        continue;
-                    }
-                    if (issue) {
-                        const bool r = pli < n1;
-                        tma_prefetch_l2_3d(r ? &a.mW_res : &a.mW_head, pkb * kTK,
-                                           (int)(r ? pt % tph_r : pt % tph_l) * kTM, (int)(r ? pt / tph_r : pt / tph_l));
-                    }
-                    ++pkb;
-                    ++pu;
-                }
-            };
-            const int ahead = kPrefetchAheadX4 * S / 4;
-            if (weights) prefetch_upto(S, false);  // the first S k-blocks are loaded at once
             for (int li = 0; li < ntiles && ok; ++li) {
                 const bool res = li < n1;
                 long t;
@@ -261,7 +280,6 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
                         ok = false;
                         break;
                     }
-                    if (weights && ahead > 0) prefetch_upto(it + ahead, true);
                     mbar_arrive_expect_tx(&full[s], bytes);
                     if (weights)
                         tma_load_3d(sA + (size_t)s * kABytes, res ? &a.mW_res : &a.mW_head, kb * kTK, row0, k,
@@ -330,78 +348,78 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
         const int ew = warp - kEpiWarp0;               // 0..3
         const int q = warp & 3;                        // TMEM lane quarter this warp may access
         const int row = q * 32 + lane;                 // weight row of the tile held by this thread
-        // transposed phase: column `col`, rows [r_lo, r_hi) of every tile
-        const int nseg = seg_per_col(B);
-        const int rps = (kTM + nseg - 1) / nseg;
-        const bool col_thread = et < B * nseg;
+        // transposed phase: this warp's units (see row_blocks), state in
+        // shared memory that only the owning warp touches: per unit a lane
+        // keeps the running max and sum of exp(x - max) of its rows (sU), and
+        // the unit's top-8 list (sL) is read into lanes 0..7 when it changes
+        const int R = epi_blocks(B, kUnits);      // row blocks (units) or segments per column
+        const int rpu = (kTM + R - 1) / R;        // rows per unit or segment (units: R divides kTM)
+        // segments: thread et takes column et % B, rows [r_lo, r_hi)
+        const bool col_thread = et < B * R;
         const int col = et % B, seg = et / B;
-        const int r_lo = col_thread ? seg * rps : 0, r_hi = col_thread ? min(kTM, r_lo + rps) : 0;
+        const int r_lo = col_thread ? seg * rpu : 0, r_hi = col_thread ? min(kTM, r_lo + rpu) : 0;
         float cm = -INFINITY, cl = 0.f;  // running max and sum of exp(x - cm)
         float lv[kTopK];
         int lx[kTopK];
+        auto reset_units = [&]() {
+            if constexpr (kUnits) {
+                for (int u = ew; u < nunits; u += 4) {
+                    sU[u * 32 + lane] = make_float2(-INFINITY, 0.f);
+                    if (lane < kTopK) sL[u * kTopK + lane] = TopEntry{-INFINITY, INT_MAX};
+                }
+                __syncwarp();
+            } else {
+                cm = -INFINITY;
+                cl = 0.f;
 #pragma unroll
-        for (int j = 0; j < kTopK; ++j) {
-            lv[j] = -INFINITY;
-            lx[j] = INT_MAX;
-        }
+                for (int j = 0; j < kTopK; ++j) {
+                    lv[j] = -INFINITY;
+                    lx[j] = INT_MAX;
+                }
+            }
+        };
+        reset_units();
         int cur_k = -1;
         bool ok = true;
         auto flush = [&](int kk) {
-            if (col_thread) {
-                HeadState* o = &stS[et];  // = [seg][col]
-                o->m = cm;
-                o->l = cl;
-#pragma unroll
-                for (int j = 0; j < kTopK; ++j) {
-                    o->val[j] = lv[j];
-                    o->idx[j] = lx[j];
-                }
-            }
-            epi_sync();
-            if (nseg >= 8) {
-                // many segments per column: one warp per column, lane s holding
-                // segment s (softmax statistics by a butterfly, top-8 by
-                // repeated warp maxima over the lanes' sorted lists)
-                for (int b = ew; b < B; b += 4) {
-                    float mm = -INFINITY, ll = 0.f;
-                    float mv[kTopK];
-                    int mi[kTopK];
+            // each unit's state, its lanes' statistics merged by a butterfly,
+            // (or each segment's) goes to stS[row block][column]
+            if constexpr (!kUnits) {
+                if (col_thread) {
+                    HeadState* o = &stS[et];  // = [seg][col]
+                    o->m = cm;
+                    o->l = cl;
 #pragma unroll
                     for (int j = 0; j < kTopK; ++j) {
-                        mv[j] = -INFINITY;
-                        mi[j] = INT_MAX;
-                    }
-                    if (lane < nseg) {
-                        const HeadState* o = &stS[lane * B + b];
-                        mm = o->m;
-                        ll = o->l;
-#pragma unroll
-                        for (int j = 0; j < kTopK; ++j) {
-                            mv[j] = o->val[j];
-                            mi[j] = o->idx[j];
-                        }
-                    }
-#pragma unroll
-                    for (int o = 1; o < 32; o <<= 1) {
-                        const float m2 = __shfl_xor_sync(kFull, mm, o);
-                        const float l2 = __shfl_xor_sync(kFull, ll, o);
-                        merge_ml(mm, ll, m2, l2);
-                    }
-                    float ov;
-                    int oi;
-                    warp_select(mv, mi, ov, oi);
-                    HeadState* dst = &a.part[((long)blockIdx.x * K + kk) * B + b];
-                    if (lane < kTopK) {
-                        dst->val[lane] = ov;
-                        dst->idx[lane] = oi;
-                    }
-                    if (lane == 0) {
-                        dst->m = mm;
-                        dst->l = ll;
+                        o->val[j] = lv[j];
+                        o->idx[j] = lx[j];
                     }
                 }
-            } else if (et < B) {
-                // merge the column's segments in segment order
+            }
+            for (int u = ew; kUnits && u < nunits; u += 4) {
+                const float2 ml = sU[u * 32 + lane];
+                float mm = ml.x, ll = ml.y;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float m2 = __shfl_xor_sync(kFull, mm, o);
+                    const float l2 = __shfl_xor_sync(kFull, ll, o);
+                    merge_ml(mm, ll, m2, l2);
+                }
+                HeadState* o = &stS[(u % R) * B + u / R];
+                if (lane == 0) {
+                    o->m = mm;
+                    o->l = ll;
+                }
+                if (lane < kTopK) {
+                    const TopEntry te = sL[u * kTopK + lane];
+                    o->val[lane] = te.v;
+                    o->idx[lane] = te.i;
+                }
+            }
+            const int nseg = R;
+            epi_sync();
+            if (et < B) {
+                // merge the column's row blocks in order
                 float mm = -INFINITY, ll = 0.f;
                 float mv[kTopK];
                 int mi[kTopK];
@@ -448,13 +466,7 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
                 }
             }
             epi_sync();  // stS is free again (and last_flag read) before the next flush
-            cm = -INFINITY;
-            cl = 0.f;
-#pragma unroll
-            for (int j = 0; j < kTopK; ++j) {
-                lv[j] = -INFINITY;
-                lx[j] = INT_MAX;
-            }
+            reset_units();
         };
         auto arrive_grid = [&]() {
             // this CTA's h^(k) rows are written: publish them (also to the TMA proxy)
@@ -466,103 +478,119 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
         if (n1 == 0) arrive_grid();
         for (int li = 0; li < ntiles; ++li) {
             const int buf = li & 1;
+            const int ph = li < n1 ? 0 : 1;
+            const long U = ph == 0 ? U1 : U2;
+            long t;
+            int kb0, kb1;
+            piece(li, t, kb0, kb1);
+            // kb0 > 0: the later k-blocks of a tile owned by an earlier CTA (the
+            // first piece of this CTA's run), handed over as a partial sum
+            const bool handover = kb0 > 0;
+            const bool res = li < n1;
+            const int k = (int)(res ? t / tph_r : t / tph_l);
+            const int row0 = (int)(res ? t % tph_r : t % tph_l) * kTM;
+            if (!handover && !res) {
+                if (k != cur_k) {
+                    if (cur_k >= 0) flush(cur_k);
+                    cur_k = k;
+                }
+                epi_sync();  // the previous tile's readers are done with sT
+            }
             if (ok && !mbar_wait(&acc_full[buf], (li >> 1) & 1, wait_ns)) {
                 if (lane == 0) set_status(a.status, MEDUSA_STATUS_TIMEOUT);
                 ok = false;
             }
-            // decided for the whole warp before its collective TMEM loads (the
-            // lanes test barriers and flags independently)
-            ok = __all_sync(kFull, ok);
-            float v[N];
-#pragma unroll
-            for (int e = 0; e < N; ++e) v[e] = 0.f;
-            if (ok) {
-                tc_fence_after();
-#pragma unroll
-                for (int c = 0; c < N / 16; ++c) {
-                    float t16[16];
-                    tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + buf * N + c * 16, t16);
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) v[c * 16 + e] = t16[e];
-                }
-                tc_fence_before();
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[buf]);
-            const int ph = li < n1 ? 0 : 1;
-            long t;
-            int kb0, kb1;
-            piece(li, t, kb0, kb1);
-            if (kb0 > 0) {
-                // the later k-blocks of a tile owned by an earlier CTA: hand the
-                // partial sum over (this is the first piece of this CTA's run)
-                float* dst = a.slots + (long)(ph * G + cta) * B * kTM;
-                if (ok) {
-#pragma unroll
-                    for (int e = 0; e < N; ++e)
-                        if (e < B) dst[e * kTM + row] = v[e];
-                }
-                __threadfence();
-                epi_sync();
-                if (et == 0) st_release_u32(&a.ctr[2 + ph * G + cta], 1u);
-                if (li == n1 - 1) arrive_grid();
-                continue;
-            }
-            if (kb1 < nkb && ok) {
-                // the rest of this tile: the first pieces of the next CTAs' runs
-                const long U = ph == 0 ? U1 : U2, tend = (t + 1) * nkb;
+            // an owned tile cut by a run boundary: its rest is the first pieces
+            // of the next CTAs' runs, [cta + 1, c2_end), handed over by flags
+            int c2_end = cta + 1;
+            if (!handover && kb1 < nkb && ok) {
+                const long tend = (t + 1) * nkb;
                 for (int c2 = cta + 1; c2 < G && U * c2 / G < tend; ++c2) {
+                    c2_end = c2 + 1;
                     if (U * (c2 + 1) / G == U * c2 / G) continue;  // an empty run
                     if (!wait_flag(&a.ctr[2 + ph * G + c2], wait_ns)) {
                         if (lane == 0) set_status(a.status, MEDUSA_STATUS_TIMEOUT);
                         ok = false;
                         break;
                     }
-                    const float* src = a.slots + (long)(ph * G + c2) * B * kTM;
-#pragma unroll
-                    for (int e = 0; e < N; ++e)
-                        if (e < B) v[e] += __ldcg(&src[e * kTM + row]);
                 }
             }
-            if (li < n1) {
-                // residual tile: h^(k)[b, o] = SiLU(z) + h[b, o]
-                const int k = (int)(t / tph_r);
-                const int o = (int)(t % tph_r) * kTM + row;
-                if (ok && o < a.d) {
-                    float hv[N];  // every load before the first store
+            // decided for the whole warp before its collective TMEM loads (the
+            // lanes test barriers and flags independently)
+            ok = __all_sync(kFull, ok);
+            if (ok) tc_fence_after();
+            const int o = row0 + row;  // residual: output element; vocabulary: token id
+            // 16 columns (sequences) at a time from TMEM: few registers live
 #pragma unroll
-                    for (int e = 0; e < N; ++e) hv[e] = e < B ? __bfloat162float(a.h[(long)e * a.d + o]) : 0.f;
+            for (int c = 0; c < N / 16; ++c) {
+                float v[16];
 #pragma unroll
-                    for (int e = 0; e < N; ++e) {
-                        if (e < B) {
-                            const float z = v[e];
-                            const __nv_bfloat16 yb = __float2bfloat16_rn(z / (1.f + expf(-z)) + hv[e]);
-                            a.hk[((long)e * K + k) * a.d + o] = yb;
-                            if (a.hk_out) a.hk_out[((long)e * K + k) * a.d + o] = yb;
-                        }
+                for (int e = 0; e < 16; ++e) v[e] = 0.f;
+                if (ok) tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + buf * N + c * 16, v);
+                if (handover) {
+                    float* dst = a.slots + (long)(ph * G + cta) * B * kTM;
+                    if (ok) {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e)
+                            if (c * 16 + e < B) dst[(c * 16 + e) * kTM + row] = v[e];
+                    }
+                    continue;
+                }
+                if (ok) {
+                    for (int c2 = cta + 1; c2 < c2_end; ++c2) {
+                        if (U * (c2 + 1) / G == U * c2 / G) continue;
+                        const float* src = a.slots + (long)(ph * G + c2) * B * kTM;
+#pragma unroll
+                        for (int e = 0; e < 16; ++e)
+                            if (c * 16 + e < B) v[e] += __ldcg(&src[(c * 16 + e) * kTM + row]);
                     }
                 }
+                if (res) {
+                    // residual tile: h^(k)[b, o] = SiLU(z) + h[b, o]
+                    if (ok && o < a.d) {
+                        float hv[16];  // every load before the first store
+#pragma unroll
+                        for (int e = 0; e < 16; ++e)
+                            hv[e] = c * 16 + e < B ? __bfloat162float(a.h[(long)(c * 16 + e) * a.d + o]) : 0.f;
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            const int bq = c * 16 + e;
+                            if (bq < B) {
+                                const float z = v[e];
+                                const __nv_bfloat16 yb = __float2bfloat16_rn(z / (1.f + expf(-z)) + hv[e]);
+                                a.hk[((long)bq * K + k) * a.d + o] = yb;
+                                if (a.hk_out) a.hk_out[((long)bq * K + k) * a.d + o] = yb;
+                            }
+                        }
+                    }
+                    continue;
+                }
+                // vocabulary tile
+                if (a.logits && ok && o < a.V) {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        if (c * 16 + e < B) a.logits[((long)(c * 16 + e) * K + k) * a.V + o] = v[e];
+                }
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    if (c * 16 + e < B) sT[(c * 16 + e) * kTS + row] = v[e];
+            }
+            if (ok) tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[buf]);
+            if (handover) {
+                __threadfence();
+                epi_sync();
+                if (et == 0) st_release_u32(&a.ctr[2 + ph * G + cta], 1u);
                 if (li == n1 - 1) arrive_grid();
                 continue;
             }
-            // vocabulary tile
-            const int k = (int)(t / tph_l);
-            const int row0 = (int)(t % tph_l) * kTM;
-            if (k != cur_k) {
-                if (cur_k >= 0) flush(cur_k);
-                cur_k = k;
+            if (res) {
+                if (li == n1 - 1) arrive_grid();
+                continue;
             }
-            if (a.logits && ok && row0 + row < a.V) {
-#pragma unroll
-                for (int e = 0; e < N; ++e)
-                    if (e < B) a.logits[((long)e * K + k) * a.V + row0 + row] = v[e];
-            }
-            epi_sync();  // the previous tile's readers are done with sT
-#pragma unroll
-            for (int e = 0; e < N; ++e)
-                if (e < B) sT[e * kTS + row] = v[e];
             epi_sync();
-            if (ok) {
+            if (!kUnits && ok && col_thread) {
                 const float* src = sT + col * kTS;
                 const int hi = min(r_hi, a.V - row0);  // rows past V are zero-filled weights
                 float tm = -INFINITY;
@@ -570,13 +598,99 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
                 if (tm > -INFINITY) {
                     const float mn = fmaxf(cm, tm);
                     float sum = 0.f;
-                    for (int r = r_lo; r < hi; ++r) {
-                        const float x = src[r];
-                        sum += expf(x - mn);
-                        if (beats(x, row0 + r, lv[kTopK - 1], lx[kTopK - 1])) list_insert(lv, lx, x, row0 + r);
-                    }
+                    for (int r = r_lo; r < hi; ++r) sum += expf(src[r] - mn);
                     cl = (cm == -INFINITY ? 0.f : cl * expf(cm - mn)) + sum;
                     cm = mn;
+                }
+                // top-8: while the list has free places its rows go in
+                // directly; then candidates against the tile's starting
+                // threshold are queued and inserted
+                int r = r_lo;
+                for (; r < hi && lx[kTopK - 1] == INT_MAX; ++r) list_insert(lv, lx, src[r], row0 + r);
+                const float tv = lv[kTopK - 1];
+                const int ti = lx[kTopK - 1];
+                int cnt = 0;
+                for (; r < hi; ++r) {
+                    if (beats(src[r], row0 + r, tv, ti)) {
+                        sQ[cnt * 128 + et] = (uint8_t)r;
+                        ++cnt;
+                    }
+                }
+                for (int i = 0; i < cnt; ++i) {
+                    const int rr = sQ[i * 128 + et];
+                    list_insert(lv, lx, src[rr], row0 + rr);
+                }
+            }
+            if (kUnits && ok) {
+                for (int u = ew; u < nunits; u += 4) {
+                    const int rb = u % R;
+                    const float* src = sT + (u / R) * kTS + rb * rpu;
+                    const int base = row0 + rb * rpu;
+                    // lane-row j of the unit is row base + 32 j + lane (rows
+                    // past V are zero-filled weights and take no part)
+                    float x[4];
+                    bool in[4];
+                    float tm = -INFINITY;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        in[j] = 32 * j < rpu && base + 32 * j + lane < a.V;
+                        x[j] = in[j] ? src[32 * j + lane] : -INFINITY;
+                        tm = fmaxf(tm, x[j]);
+                    }
+                    if (tm > -INFINITY) {
+                        float2 ml = sU[u * 32 + lane];
+                        const float mn = fmaxf(ml.x, tm);
+                        float sum = 0.f;
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            if (in[j]) sum += expf(x[j] - mn);
+                        ml.y = (ml.x == -INFINITY ? 0.f : ml.y * expf(ml.x - mn)) + sum;
+                        ml.x = mn;
+                        sU[u * 32 + lane] = ml;
+                    }
+                    // top-8: the rows beating the list's last entry are the
+                    // candidates; the best remaining one is inserted while it
+                    // still beats the last entry (at most kTopK rounds, fewer
+                    // once the list holds the head's large values)
+                    const TopEntry last = sL[u * kTopK + kTopK - 1];
+                    unsigned mine = 0u;  // bit j: lane-row j is a remaining candidate
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        if (in[j] && beats(x[j], base + 32 * j + lane, last.v, last.i)) mine |= 1u << j;
+                    if (__any_sync(kFull, mine != 0u)) {
+                        TopEntry te = lane < kTopK ? sL[u * kTopK + lane] : TopEntry{-INFINITY, INT_MAX};
+                        for (int round = 0; round < kTopK; ++round) {
+                            float bv = -INFINITY;
+                            int bi = INT_MAX, bj = -1;
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                if (((mine >> j) & 1u) && beats(x[j], base + 32 * j + lane, bv, bi)) {
+                                    bv = x[j];
+                                    bi = base + 32 * j + lane;
+                                    bj = j;
+                                }
+                            }
+                            float wv = bv;
+                            int wi = bi;
+#pragma unroll
+                            for (int o2 = 16; o2 > 0; o2 >>= 1) {
+                                const float ov = __shfl_xor_sync(kFull, wv, o2);
+                                const int oi = __shfl_xor_sync(kFull, wi, o2);
+                                if (beats(ov, oi, wv, wi)) {
+                                    wv = ov;
+                                    wi = oi;
+                                }
+                            }
+                            const float tv = __shfl_sync(kFull, te.v, kTopK - 1);
+                            const int ti = __shfl_sync(kFull, te.i, kTopK - 1);
+                            if (wi == INT_MAX) break;  // no candidate left (wi, wv, tv, ti: the warp's)
+                            if (!beats(wv, wi, tv, ti)) break;
+                            warp_list_insert(te.v, te.i, wv, wi);
+                            if (bi == wi) mine &= ~(1u << bj);  // its lane drops it (row ids are unique)
+                        }
+                        if (lane < kTopK) sL[u * kTopK + lane] = te;
+                        __syncwarp();
+                    }
                 }
             }
         }
@@ -621,7 +735,10 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
 template <int N>
 size_t tc_smem_bytes(int stages, int B) {
     return 1024 + (size_t)stages * (kABytes + N * kTK * 2) + (2 * (size_t)stages + 5) * 8 + 16 +
-           (size_t)((B * kTS + 3) & ~3) * 4 + (size_t)B * seg_per_col(B) * sizeof(HeadState);
+           (size_t)((B * kTS + 3) & ~3) * 4 +
+           (units_epilogue<N>() ? (size_t)B * row_blocks(B) * (sizeof(HeadState) + 32 * sizeof(float2) + kTopK * 8)
+                                : (size_t)B * seg_per_col(B) * sizeof(HeadState) +
+                                      (size_t)((kTM + seg_per_col(B) - 1) / seg_per_col(B)) * 128);
 }
 
 // as many stages as shared memory holds (at most 16): the weight bytes in
