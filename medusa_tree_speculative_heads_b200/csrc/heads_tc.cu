@@ -18,21 +18,23 @@
 //   warp 2   TMA producer of the batch-vector tiles; before the first
 //            vocabulary tile it waits at the grid barrier (all of h^(k) must
 //            be written by every CTA)
-//   warps 3-6 epilogue, one TMEM lane (= weight row) per thread: residual
-//            tiles write h^(k) = SiLU(z) + h (bf16); vocabulary tiles are
-//            transposed through shared memory so that each thread owns one
-//            sequence (column) and a fixed segment of the tile's rows, and
-//            keeps that column's running softmax statistics and top-8 list
-//            in registers; at a head change the segments of each column are
-//            merged into the CTA's partial for (head, sequence).
-// Work split ("stream-K"): in each phase (residual, then vocabulary) the
-// tiles' 64-element k-blocks are laid end to end and every CTA takes an equal
-// contiguous run of them, so all SMs stream the same number of bytes.  A tile
-// cut by a run boundary is summed by the CTA holding its first k-block (its
-// owner, which reaches it last in its run); the CTAs holding the rest reach
-// their part first in theirs, and hand it over as an fp32 partial in global
-// memory with a release flag.  The weight producer keeps prefetching across
-// the grid barrier.  A head's (sequence, head) partials are merged, each in
+//   warps 3-6 epilogue, one TMEM lane (= weight row) per thread, reading
+//            the accumulator 16 columns at a time: residual tiles write
+//            h^(k) = SiLU(z) + h (bf16); vocabulary tiles are transposed
+//            through shared memory, then each column's (sequence's) running
+//            softmax statistics and top-8 list are updated (by warp units up
+//            to 32 sequences, by thread segments above: see row_blocks and
+//            units_epilogue); at a head change they become the CTA's
+//            partial for (head, sequence).
+// Work split ("stream-K"): in the vocabulary phase (and in the residual phase
+// when it has more tiles than there are CTAs; otherwise each CTA takes one
+// whole residual tile) the tiles' 64-element k-blocks are laid end to end and
+// every CTA takes an equal contiguous run of them, so all SMs stream the same
+// number of bytes.  A tile cut by a run boundary is summed by the CTA holding
+// its first k-block (its owner, which reaches it last in its run); the CTAs
+// holding the rest reach their part first in theirs, and hand it over as an
+// fp32 partial in global memory with a release flag.  The weight producer
+// keeps prefetching across the grid barrier.  A head's (sequence, head) partials are merged, each in
 // CTA order, and its tree nodes filled, by the last CTA to publish its
 // partial of that head (a per-head arrival counter, no waiting): the first
 // heads are merged while the stream goes on, only the last head's merge ends
@@ -140,6 +142,13 @@ struct Run {
     long u0, u1;
     int nkb;
     __device__ Run(long U, int c, int G, int nkb_) : u0(U * c / G), u1(U * (c + 1) / G), nkb(nkb_) {}
+    // whole tiles: CTA c takes tile c of T, none when c >= T
+    __device__ static Run whole(long T, int c, int nkb_) {
+        Run r(0, 0, 1, nkb_);
+        r.u0 = (c < T ? c : T) * (long)nkb_;
+        r.u1 = (c < T ? c + 1 : T) * (long)nkb_;
+        return r;
+    }
     __device__ int count() const { return u1 > u0 ? (int)((u1 - 1) / nkb - u0 / nkb + 1) : 0; }
     __device__ void piece(int i, long& t, int& kb0, int& kb1) const {
         t = u0 / nkb + i;
@@ -213,7 +222,13 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
     const int tph_l = (a.V + kTM - 1) / kTM;   // vocabulary tiles per head
     const int nkb = (a.d + kTK - 1) / kTK;     // k-blocks per tile
     const long U1 = (long)K * tph_r * nkb, U2 = (long)K * tph_l * nkb;
-    const Run run1(U1, cta, G, nkb), run2(U2, cta, G, nkb);
+    // The residual phase takes whole tiles when there are no more of them than
+    // CTAs: a tile split over several CTAs has its owner wait for the others'
+    // partial sums before its epilogue, and at these sizes the waits and the
+    // reads of the partials cost more than the streaming time an even split
+    // saves (llama8b: 128 tiles on 148 CTAs, 1 MB each).
+    const long T1 = (long)K * tph_r;
+    const Run run1 = T1 <= G ? Run::whole(T1, cta, nkb) : Run(U1, cta, G, nkb), run2(U2, cta, G, nkb);
     const int n1 = run1.count(), n2 = run2.count();
     const int ntiles = n1 + n2;  // pieces, residual phase first
     auto piece = [&](int li, long& t, int& kb0, int& kb1) {
@@ -476,6 +491,24 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
             if (ew == 0 && lane == 0) atomicAdd(&a.ctr[0], 1u);
         };
         if (n1 == 0) arrive_grid();
+        // A whole residual tile: its h rows are read into sT (free until the
+        // first vocabulary tile) while the MMA streams the tile, so the
+        // epilogue does not wait on them afterwards.
+        const bool h_staged = T1 <= G && n1 == 1;
+        if (h_staged) {
+            const int o = (int)(cta % tph_r) * kTM + row;
+            if (o < a.d) {
+                for (int e0 = 0; e0 < B; e0 += 16) {
+                    float hv[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        hv[e] = e0 + e < B ? __bfloat162float(a.h[(long)(e0 + e) * a.d + o]) : 0.f;
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        if (e0 + e < B) sT[(e0 + e) * kTS + row] = hv[e];
+                }
+            }
+        }
         for (int li = 0; li < ntiles; ++li) {
             const int buf = li & 1;
             const int ph = li < n1 ? 0 : 1;
@@ -551,7 +584,9 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
                         float hv[16];  // every load before the first store
 #pragma unroll
                         for (int e = 0; e < 16; ++e)
-                            hv[e] = c * 16 + e < B ? __bfloat162float(a.h[(long)(c * 16 + e) * a.d + o]) : 0.f;
+                            hv[e] = c * 16 + e >= B ? 0.f
+                                    : h_staged      ? sT[(c * 16 + e) * kTS + row]
+                                                    : __bfloat162float(a.h[(long)(c * 16 + e) * a.d + o]);
 #pragma unroll
                         for (int e = 0; e < 16; ++e) {
                             const int bq = c * 16 + e;
