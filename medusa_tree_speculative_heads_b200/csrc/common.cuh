@@ -154,15 +154,35 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                  : "memory");
 }
 
+// kSuspend: the waiting thread is suspended until the phase completes or
+// kSuspendHintNs pass.  Without the hint try_wait returns after a short
+// hardware-chosen time and the wait loop spins.  In the heads kernel (deep
+// buffering, waits of whole tiles) the spinning producer, MMA and epilogue
+// threads cost 9% of the weight stream at llama8b (752 against 687 us on one
+// box); in tree attention, whose softmax and MMA threads hand each chunk back
+// and forth, the suspended threads woke too late (32k keys: 95 against 100 us),
+// so there the waits spin.
+constexpr uint32_t kSuspendHintNs = 2000;
+
+template <bool kSuspend = false>
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_addr(bar)), "r"(parity)
-        : "memory");
+    if (kSuspend)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(smem_addr(bar)), "r"(parity), "r"(kSuspendHintNs)
+            : "memory");
+    else
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(smem_addr(bar)), "r"(parity)
+            : "memory");
     return ok != 0;
 }
 
@@ -193,13 +213,14 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;
 // protocol error ends the kernel instead of hanging the GPU.  limit_ns <= 1
 // gives up at once unless the phase is already complete (a test of the
 // error paths; see medusa_debug_set_wait_limit).
+template <bool kSuspend = false>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns = kWaitLimitNs) {
     if (limit_ns <= 1) return mbar_test(bar, parity);
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait<kSuspend>(bar, parity)) return true;
     const uint64_t t0 = global_ns();
     for (uint32_t i = 1;; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 255u) == 0 && global_ns() - t0 > limit_ns) return false;
+        if (mbar_try_wait<kSuspend>(bar, parity)) return true;
+        if ((i & (kSuspend ? 15u : 255u)) == 0 && global_ns() - t0 > limit_ns) return false;
     }
 }
 

@@ -290,7 +290,7 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
                 }
                 for (int kb = kb0; kb < kb1; ++kb) {
                     const int s = it % S;
-                    if (it >= S && !mbar_wait(&empty[s], ((it / S) - 1) & 1, wait_ns)) {
+                    if (it >= S && !mbar_wait<true>(&empty[s], ((it / S) - 1) & 1, wait_ns)) {
                         set_status(a.status, MEDUSA_STATUS_TIMEOUT);
                         ok = false;
                         break;
@@ -316,7 +316,7 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
                 const int last = s + ((it - 1 - s) / S) * S;
                 const uint64_t now = global_ns();
                 if (now >= t_end) break;
-                mbar_wait(&full[s], (last / S) & 1, t_end - now);
+                mbar_wait<true>(&full[s], (last / S) & 1, t_end - now);
             }
         }
     } else if (warp == 1) {
@@ -326,7 +326,7 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
             int it = 0;
             for (int li = 0; li < ntiles && ok; ++li) {
                 const int buf = li & 1;
-                if (li >= 2 && !mbar_wait(&acc_empty[buf], ((li >> 1) - 1) & 1, wait_ns)) {
+                if (li >= 2 && !mbar_wait<true>(&acc_empty[buf], ((li >> 1) - 1) & 1, wait_ns)) {
                     set_status(a.status, MEDUSA_STATUS_TIMEOUT);
                     break;
                 }
@@ -337,7 +337,7 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
                 piece(li, t, kb0, kb1);
                 for (int kb = kb0; kb < kb1; ++kb) {
                     const int s = it % S;
-                    if (!mbar_wait(&full[s], (it / S) & 1, wait_ns)) {
+                    if (!mbar_wait<true>(&full[s], (it / S) & 1, wait_ns)) {
                         set_status(a.status, MEDUSA_STATUS_TIMEOUT);
                         ok = false;
                         break;
@@ -355,7 +355,7 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
             }
             // every MMA this thread issued completes before TMEM is released
             tc_commit(mma_done);
-            mbar_wait(mma_done, 0);
+            mbar_wait<true>(mma_done, 0);
         }
     } else {
         // ---------------- epilogue ----------------
@@ -529,7 +529,7 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
                 }
                 epi_sync();  // the previous tile's readers are done with sT
             }
-            if (ok && !mbar_wait(&acc_full[buf], (li >> 1) & 1, wait_ns)) {
+            if (ok && !mbar_wait<true>(&acc_full[buf], (li >> 1) & 1, wait_ns)) {
                 if (lane == 0) set_status(a.status, MEDUSA_STATUS_TIMEOUT);
                 ok = false;
             }
@@ -592,7 +592,11 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
                             const int bq = c * 16 + e;
                             if (bq < B) {
                                 const float z = v[e];
-                                const __nv_bfloat16 yb = __float2bfloat16_rn(z / (1.f + expf(-z)) + hv[e]);
+                                // SiLU with the fast exponential and divide: their
+                                // error is far below the bf16 rounding of h^(k), and
+                                // the accurate divide's slow path (a denominator of
+                                // inf when z < -88) made this loop 1/3 slower
+                                const __nv_bfloat16 yb = __float2bfloat16_rn(__fdividef(z, 1.f + __expf(-z)) + hv[e]);
                                 a.hk[((long)bq * K + k) * a.d + o] = yb;
                                 if (a.hk_out) a.hk_out[((long)bq * K + k) * a.d + o] = yb;
                             }
