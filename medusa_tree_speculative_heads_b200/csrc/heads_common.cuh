@@ -146,7 +146,9 @@ struct HeadCover {
 // nodes per sequence; head 0 also writes the root and sets the rows past
 // that tree to -1 and 0).  One warp.
 // Partials are read through L2 (they may have been written by other CTAs of
-// the same kernel).
+// the same kernel).  dry: everything but the writes (the reads stay inside
+// the workspace and the tree), to bring the code into the instruction cache
+// ahead of a merge on the critical path.
 // ---------------------------------------------------------------------------
 static __device__ __noinline__ void merge_head(const HeadState* __restrict__ part, int nparts, long uph, int upt,
                                                int bstride, int bb,
@@ -154,7 +156,7 @@ static __device__ __noinline__ void merge_head(const HeadState* __restrict__ par
                            const TreeDev* __restrict__ tree, int Tn, const int32_t* __restrict__ root_token,
                            int32_t* __restrict__ topk_idx, float* __restrict__ topk_prob,
                            int32_t* __restrict__ node_tokens, float* __restrict__ node_q, float2* __restrict__ stats,
-                           int32_t* status) {
+                           int32_t* status, bool dry = false) {
     const int lane = threadIdx.x & 31;
     // the tree's shape and the root token are needed at the end: load them
     // first, so their latency overlaps the partials'
@@ -217,6 +219,7 @@ static __device__ __noinline__ void merge_head(const HeadState* __restrict__ par
     warp_select(lv, li, ov, oi);
     const bool valid = oi != INT_MAX;
     const float prob = valid ? expf(ov - mm) / ll : 0.f;
+    if (dry) return;
     if (lane < kTopK) {
         topk_idx[((long)b * K + k) * kTopK + lane] = valid ? oi : -1;
         topk_prob[((long)b * K + k) * kTopK + lane] = prob;

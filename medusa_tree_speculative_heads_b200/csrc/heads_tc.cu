@@ -529,6 +529,15 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
                 }
                 epi_sync();  // the previous tile's readers are done with sT
             }
+            if (li == (ntiles >= 2 ? ntiles - 2 : 0)) {
+                // the merges at the end of the kernel run from a cold
+                // instruction cache: a dry merge while the last tiles stream
+                // brings their code in on each epilogue warp's scheduler (the
+                // last piece can be short, so this goes one piece earlier)
+                merge_head(a.part, G, tph_l, nkb, B, 0, 0, a.V, K, cur_k >= 0 ? cur_k : 0,
+                           a.tree.base ? a.tree.at(0) : nullptr, a.tree.T, a.root_token, a.topk_idx, a.topk_prob,
+                           a.node_tokens, a.node_q, a.stats, a.status, true);
+            }
             if (ok && !mbar_wait<true>(&acc_full[buf], (li >> 1) & 1, wait_ns)) {
                 if (lane == 0) set_status(a.status, MEDUSA_STATUS_TIMEOUT);
                 ok = false;
@@ -553,8 +562,12 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
             ok = __all_sync(kFull, ok);
             if (ok) tc_fence_after();
             const int o = row0 + row;  // residual: output element; vocabulary: token id
-            // 16 columns (sequences) at a time from TMEM: few registers live
-#pragma unroll
+            // 16 columns (sequences) at a time from TMEM: few registers live.
+            // Not unrolled: the residual tile's epilogue runs once per CTA, from
+            // a cold instruction cache, and its four unrolled copies at N = 64
+            // took 6 us each to fetch (22 against 10 us for the residual
+            // epilogue, measured with per-CTA timestamps).
+#pragma unroll 1
             for (int c = 0; c < N / 16; ++c) {
                 float v[16];
 #pragma unroll
