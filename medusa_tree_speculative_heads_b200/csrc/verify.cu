@@ -131,6 +131,96 @@ __global__ void __launch_bounds__(kArgmaxThreads, 4) row_argmax_kernel(const E* 
     }
 }
 
+// The same scan with the chunk staged in shared memory by the bulk-copy
+// engine: one thread issues the chunk's copies (four pieces, each completing
+// on its own mbarrier) as soon as the block starts, so the whole chunk is in
+// flight at once; the threads reduce each piece as it lands.  With four
+// blocks per SM the staged chunks (up to kStageBytes each) hold a whole
+// wave's share of the rows: one DRAM round trip instead of two.
+constexpr int kStageBytes = 52 * 1024;
+constexpr int kStagePieces = 4;
+template <typename E>
+__global__ void __launch_bounds__(kArgmaxThreads, 4) row_argmax_staged_kernel(const E* __restrict__ x, int V, int splits,
+                                                                           int chunk, float* __restrict__ pval,
+                                                                           int* __restrict__ pidx, int32_t* status) {
+    constexpr int VEC = Elt<E>::kVec;
+    constexpr int NW = kArgmaxThreads / 32;
+    extern __shared__ __align__(16) uint8_t sbuf[];
+    __shared__ uint64_t bars[kStagePieces];
+    const long row = blockIdx.x;
+    const int s = blockIdx.y;
+    const int v0 = s * chunk;
+    const int v1 = min(V, v0 + chunk);
+    const E* rp = x + row * (long)V;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nvec = v1 > v0 ? (v1 - v0) / VEC : 0;  // the row starts on a 16-byte boundary (checked by the host)
+    if (threadIdx.x == 0) {
+        for (int p = 0; p < kStagePieces; ++p) mbar_init(&bars[p], 1);
+        mbar_fence_init();
+        for (int p = 0; p < kStagePieces; ++p) {
+            const int vb = nvec * p / kStagePieces, ve = nvec * (p + 1) / kStagePieces;
+            const uint32_t bytes = (uint32_t)(ve - vb) * 16u;
+            mbar_arrive_expect_tx(&bars[p], bytes);
+            if (bytes) bulk_g2s(sbuf + (size_t)vb * 16, rp + v0 + (long)vb * VEC, bytes, &bars[p]);
+        }
+    }
+    __syncthreads();  // the barriers are initialised before anyone waits on them
+    float bv = -INFINITY;
+    int bi = v0;  // lowest index of the chunk: the answer when nothing beats -inf
+    int bc = -1;  // the thread's winning vector
+    uint4 braw = make_uint4(0, 0, 0, 0);
+    bool ok = true;
+    for (int p = 0; p < kStagePieces; ++p) {
+        const int vb = nvec * p / kStagePieces, ve = nvec * (p + 1) / kStagePieces;
+        if (ok && !mbar_wait(&bars[p], 0)) {
+            ok = false;
+            set_status(status, MEDUSA_STATUS_TIMEOUT);
+        }
+        if (!ok) continue;
+        // this thread's vectors of the piece, in increasing index order
+        int c = vb + (int)(((unsigned)(threadIdx.x - vb)) % kArgmaxThreads);
+        for (; c < ve; c += kArgmaxThreads) {
+            const uint4 raw = *reinterpret_cast<const uint4*>(sbuf + (size_t)c * 16);
+            const float mv = Elt<E>::vmax(raw);
+            if (mv > bv) {
+                bv = mv;
+                bc = c;
+                braw = raw;
+            }
+        }
+    }
+    if (!ok)  // the copies still in flight land before the block exits
+        for (int p = 0; p < kStagePieces; ++p) mbar_wait(&bars[p], 0);
+    if (bc >= 0) {
+        float f[VEC];
+        Elt<E>::unpack(braw, f);
+        int e = 0;
+#pragma unroll
+        for (int i = VEC - 1; i >= 0; --i)
+            if (f[i] == bv) e = i;
+        bi = v0 + bc * VEC + e;
+    }
+    for (int v = v0 + nvec * VEC + threadIdx.x; v < v1; v += kArgmaxThreads) argmax_merge(bv, bi, Elt<E>::to_float(rp[v]), v);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(kFull, bv, o);
+        const int oi = __shfl_xor_sync(kFull, bi, o);
+        argmax_merge(bv, bi, ov, oi);
+    }
+    __shared__ float sv[NW];
+    __shared__ int si[NW];
+    if (lane == 0) {
+        sv[warp] = bv;
+        si[warp] = bi;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int w = 1; w < NW; ++w) argmax_merge(bv, bi, sv[w], si[w]);
+        pval[row * splits + s] = bv;
+        pidx[row * splits + s] = bi;
+    }
+}
+
 // One block of 128 threads per sequence, one thread per node: node u's
 // prediction is the merge of its partials (split order); node c "matches"
 // when its token equals its parent's prediction (the root always does).  A
@@ -582,6 +672,25 @@ cudaError_t verify_greedy_rows_launch(const VerifyArgs& a, cudaStream_t st) {
     float* pval = (float*)a.ws;
     int* pidx = (int*)((char*)a.ws + align256((size_t)rows * splits * sizeof(float)));
     dim3 grid(rows, splits);
+    const size_t elt = a.target_dt == MEDUSA_BF16 ? 2 : 4;
+    const size_t stage = (size_t)chunk * elt;
+    // staged when every row starts on a 16-byte boundary and a chunk fits the
+    // stage (contiguous chunks of whole vectors; the row's tail is read directly)
+    if (((uintptr_t)a.target & 15) == 0 && ((size_t)a.V * elt) % 16 == 0 && stage <= (size_t)kStageBytes) {
+        if (a.target_dt == MEDUSA_BF16) {
+            auto k = row_argmax_staged_kernel<__nv_bfloat16>;
+            cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kStageBytes);
+            prefer_max_smem(k);
+            k<<<grid, kArgmaxThreads, stage, st>>>((const __nv_bfloat16*)a.target, a.V, splits, chunk, pval, pidx,
+                                                  a.status);
+        } else {
+            auto k = row_argmax_staged_kernel<float>;
+            cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kStageBytes);
+            prefer_max_smem(k);
+            k<<<grid, kArgmaxThreads, stage, st>>>((const float*)a.target, a.V, splits, chunk, pval, pidx, a.status);
+        }
+        return cudaGetLastError();
+    }
     if (a.target_dt == MEDUSA_BF16) prefer_max_smem(row_argmax_kernel<__nv_bfloat16>);
     else prefer_max_smem(row_argmax_kernel<float>);
     if (a.target_dt == MEDUSA_BF16)
