@@ -75,10 +75,8 @@ __host__ __device__ constexpr int row_blocks(int B) { return B >= 4 ? 1 : B == 1
 // list starts empty in every CTA and head (about 30 insertions per column,
 // each a warp-wide step), so there each thread takes one column segment of
 // 128 / seg_per_col(B) rows instead: its running statistics and top-8 list
-// stay in registers; a tile's candidates (rows beating the list's last entry
-// when the tile starts) are queued in shared memory and inserted after the
-// scan, so a warp runs as many insertions as its longest queue, not one per
-// row in which any lane inserts.
+// stay in registers, and every row goes through a branch-free insertion
+// (no divergence between the lanes' columns).
 template <int N> constexpr bool units_epilogue() { return N <= 32; }
 __host__ __device__ constexpr int seg_per_col(int B) { return 128 / B < 16 ? 128 / B : 16; }
 __host__ __device__ constexpr int epi_blocks(int B, bool units) { return units ? row_blocks(B) : seg_per_col(B); }
@@ -213,7 +211,6 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
     const int nunits = a.B * epi_blocks(a.B, kUnits);  // units, or column segments
     float2* sU = reinterpret_cast<float2*>(stS + nunits);       // [unit][lane] running (max, sum)
     TopEntry* sL = reinterpret_cast<TopEntry*>(sU + nunits * 32);  // [unit][kTopK] top list, best first
-    uint8_t* sQ = reinterpret_cast<uint8_t*>(stS + nunits);     // segments: [slot][128 threads] candidate rows
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int K = a.K, B = a.B;
@@ -654,23 +651,27 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) heads_tc_kernel(const __grid
                     cl = (cm == -INFINITY ? 0.f : cl * expf(cm - mn)) + sum;
                     cm = mn;
                 }
-                // top-8: while the list has free places its rows go in
-                // directly; then candidates against the tile's starting
-                // threshold are queued and inserted
-                int r = r_lo;
-                for (; r < hi && lx[kTopK - 1] == INT_MAX; ++r) list_insert(lv, lx, src[r], row0 + r);
-                const float tv = lv[kTopK - 1];
-                const int ti = lx[kTopK - 1];
-                int cnt = 0;
-                for (; r < hi; ++r) {
-                    if (beats(src[r], row0 + r, tv, ti)) {
-                        sQ[cnt * 128 + et] = (uint8_t)r;
-                        ++cnt;
+                // top-8: every row goes through a branch-free insertion (kept
+                // if it beats the last entry, then bubbled up).  Most rows of a
+                // CTA's first tiles of a head are kept, so filtering first (and
+                // inserting the survivors from a queue) cost more: 30 us on a
+                // first tile against 8-12 us here, measured per CTA at B=64.
+                for (int r = r_lo; r < hi; ++r) {
+                    const float v = src[r];
+                    const int i = row0 + r;
+                    const bool in = beats(v, i, lv[kTopK - 1], lx[kTopK - 1]);
+                    lv[kTopK - 1] = in ? v : lv[kTopK - 1];
+                    lx[kTopK - 1] = in ? i : lx[kTopK - 1];
+#pragma unroll
+                    for (int j = kTopK - 1; j > 0; --j) {
+                        const bool sw = beats(lv[j], lx[j], lv[j - 1], lx[j - 1]);
+                        const float a0 = lv[j], b0 = lv[j - 1];
+                        const int ai = lx[j], bi = lx[j - 1];
+                        lv[j - 1] = sw ? a0 : b0;
+                        lv[j] = sw ? b0 : a0;
+                        lx[j - 1] = sw ? ai : bi;
+                        lx[j] = sw ? bi : ai;
                     }
-                }
-                for (int i = 0; i < cnt; ++i) {
-                    const int rr = sQ[i * 128 + et];
-                    list_insert(lv, lx, src[rr], row0 + rr);
                 }
             }
             if (kUnits && ok) {
@@ -789,8 +790,7 @@ size_t tc_smem_bytes(int stages, int B) {
     return 1024 + (size_t)stages * (kABytes + N * kTK * 2) + (2 * (size_t)stages + 5) * 8 + 16 +
            (size_t)((B * kTS + 3) & ~3) * 4 +
            (units_epilogue<N>() ? (size_t)B * row_blocks(B) * (sizeof(HeadState) + 32 * sizeof(float2) + kTopK * 8)
-                                : (size_t)B * seg_per_col(B) * sizeof(HeadState) +
-                                      (size_t)((kTM + seg_per_col(B) - 1) / seg_per_col(B)) * 128);
+                                : (size_t)B * seg_per_col(B) * sizeof(HeadState));
 }
 
 // as many stages as shared memory holds (at most 16): the weight bytes in
