@@ -125,6 +125,25 @@ def test_greedy_draft_equals_target_full_vocab():
     assert_same(out, oracle.verify_greedy(logits, tok, parents, max_path=5))
 
 
+@pytest.mark.parametrize("dt", [torch.float32, torch.bfloat16])
+def test_greedy_full_vocab_row_scan_paths(dt):
+    # 117 rows of V=128256: bf16 chunks are staged in shared memory by bulk
+    # copies, fp32 chunks (100 KB) are too large for the stage and take the
+    # register-load scan; both must pick exactly the oracle's argmax
+    w = I.scaled(I.WORKLOADS["llama8b"], B=1)
+    parents = I.workload_tree(w)
+    tok, logits = greedy_case(w, parents, 5)
+    logits = logits.to(dt)
+    ch = I.tree_children(parents)
+    am = logits.float().argmax(-1)
+    for u in range(len(parents)):     # the first child of every node is its parent's prediction
+        if ch[u]:
+            tok[0, ch[u][0]] = am[0, u]
+    out = run_greedy(parents, tok, logits)
+    assert_same(out, oracle.verify_greedy(logits, tok, parents, max_path=5))
+    assert out["accept_len"].tolist() == [5]
+
+
 def stoch_case(w, parents):
     d = I.stochastic_inputs(w, parents)
     return d["p"], d["q"], d["node_tokens"]
