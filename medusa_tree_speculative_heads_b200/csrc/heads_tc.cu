@@ -66,11 +66,13 @@ constexpr int kTS = kTM + 1;             // transposed tile: column stride in fl
 constexpr int kMergePerHeadMaxB = 4;
 
 // The vocabulary epilogue splits a tile's B columns (sequences) x 128 rows
-// into units of one column and 128 / R rows, R = row blocks per column (4 for
-// one sequence, 2 for two, else 1), so that B >= 4 gives B units and fewer
-// sequences still give the four epilogue warps one unit each; unit u is
-// column u / R, row block u % R, taken by warp u % 4.
-__host__ __device__ constexpr int row_blocks(int B) { return B >= 4 ? 1 : B == 1 ? 4 : 2; }
+// into units of one column and 128 / R rows (R = row blocks per column); unit
+// u is column u / R, row block u % R, taken by warp u % 4.  R = 1: with fewer
+// than four sequences some epilogue warps idle, but a column's state then
+// needs no merge of row blocks at a head change (splitting one sequence's
+// column over the four warps cost 4 us at llama8b, in the final merge's
+// serial path).
+__host__ __device__ constexpr int row_blocks(int) { return 1; }
 // Above 32 sequences each warp would take 9..16 units, and a unit's top-8
 // list starts empty in every CTA and head (about 30 insertions per column,
 // each a warp-wide step), so there each thread takes one column segment of
