@@ -35,10 +35,10 @@ METRIC = "Medusa verify steps/s (8B shape, 117-node tree); tree-attn HBM GB/s vs
 UNIT = "steps/s"
 WORKLOAD = "llama8b"
 # DRAM bytes (read + write) per launch of the heads kernel, from an ncu capture
-# of the same kernel at V=32000 (1184.602 MB read + 4.289 MB written against
+# of the same kernel at V=32000 (1184.480 MB read + 3.802 MB written against
 # 1182.802 MB algorithmic), scaled to the workload's algorithmic bytes; only for
 # the workload whose launch configuration (B=1, d=4096, K=4) was captured.
-HEADS_DRAM_BYTES = {"llama8b": 4336918528 * (1184602000 + 4288768) / 1182801920}
+HEADS_DRAM_BYTES = {"llama8b": 4336918528 * (1184480000 + 3802112) / 1182801920}
 OVERRIDDEN = set()   # workloads whose sizes --override replaced (no captured traffic applies)
 
 
