@@ -688,6 +688,14 @@ int attn_tc_splits(int B, int T, int Hq, int Hkv, int max_prefix) {
     const long chunks = (max_prefix + kCh - 1) / kCh + (T + kCh - 1) / kCh;
     if (c > kMaxCluster) c = kMaxCluster;
     if (c > chunks) c = chunks;
+    // With few chunks per split (a short prefix) one CTA per SM does better:
+    // a whole SM per CTA and fewer partials to merge (2048 keys at llama8b
+    // shapes: 4 splits of 128 CTAs 25.4 us, 8 splits of 256 CTAs 28.7 us;
+    // at 32k keys 8 splits stay best)
+    if (chunks < 8 * c) {
+        const long c1 = num_sms() / per_split;
+        if (c1 >= 1 && c1 < c) c = c1;
+    }
     const int cap = launch_attention_splits();
     if (cap > 0 && c > cap) c = cap;
     return c < 1 ? 1 : (int)c;
