@@ -34,11 +34,11 @@
 // its first k-block (its owner, which reaches it last in its run); the CTAs
 // holding the rest reach their part first in theirs, and hand it over as an
 // fp32 partial in global memory with a release flag.  The weight producer
-// keeps prefetching across the grid barrier.  A head's (sequence, head) partials are merged, each in
-// CTA order, and its tree nodes filled, by the last CTA to publish its
-// partial of that head (a per-head arrival counter, no waiting): the first
-// heads are merged while the stream goes on, only the last head's merge ends
-// the kernel.  With more than 4 sequences one CTA would take too long over a
+// keeps prefetching across the grid barrier.  A head's (sequence, head)
+// partials are merged, each in CTA order, and its tree nodes filled, by the
+// last CTA to publish its partial of that head (a per-head arrival counter,
+// no waiting); only the merges of the heads whose last tiles end the stream
+// are left at the end of the kernel.  With more than 4 sequences one CTA would take too long over a
 // head's merges, so there a grid barrier is followed by the merges of all
 // heads spread over every warp of the grid.
 // Every wait is bounded (~2 s) and sets MEDUSA_STATUS_TIMEOUT on expiry.
