@@ -204,8 +204,20 @@ static __device__ __noinline__ void merge_head(const HeadState* __restrict__ par
         for (int u = 0; u < 2; ++u) {
             if (!cv[u]) continue;
             merge_ml(mm, ll, sm[u], sl[u]);
+            if (li[0] == INT_MAX) {
+                // the lane's list is empty: a partial's list is sorted, copy it
 #pragma unroll
-            for (int j = 0; j < kTopK; ++j) list_insert(lv, li, pv[u][j], pi[u][j]);
+                for (int j = 0; j < kTopK; ++j) {
+                    lv[j] = pv[u][j];
+                    li[j] = pi[u][j];
+                }
+            } else {
+                // insert in order, up to the first entry that does not make it
+                for (int j = 0; j < kTopK; ++j) {
+                    if (!beats(pv[u][j], pi[u][j], lv[kTopK - 1], li[kTopK - 1])) break;
+                    list_insert(lv, li, pv[u][j], pi[u][j]);
+                }
+            }
         }
     }
 #pragma unroll
